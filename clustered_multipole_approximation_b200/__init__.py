@@ -1,0 +1,239 @@
+"""MuSe (Multipole Semantic Attention) forward operator on B200.
+
+A thin Python binding over the C ABI of ``libmuse.so`` (declared in
+``include/muse.h``): it marshals torch tensors into device pointers and the
+current CUDA stream, and nothing else -- every step of the operator runs in the
+library's sm_100a kernels.  There is no CPU fallback: without the compiled
+library (``python -m clustered_multipole_approximation_b200.build``) every call
+raises.
+
+Entry points (same names as the C ABI):
+    muse_cluster(x, C, iters, seed, role=0, init=None)
+    muse_summarize(k, v, assign, C)
+    muse_attn_fwd(q, k, v, Cq=..., Ck=..., iters=..., seed=..., topk=..., ...)
+    muse_attn_fwd_causal(q, k, v, C=..., block=..., iters=..., seed=..., topk=..., ...)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmuse.so")
+
+MODES = {"monopole": 0, "dipole": 1, "tilted": 2}
+STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED",
+          3: "MUSE_ERR_WORKSPACE", 4: "MUSE_ERR_CUDA", 5: "MUSE_ERR_DEVICE_CHECK"}
+
+
+class MuseError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class muse_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("N", ctypes.c_int), ("D", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class muse_params(ctypes.Structure):
+    _fields_ = [("Cq", ctypes.c_int), ("Ck", ctypes.c_int), ("iters", ctypes.c_int),
+                ("seed", ctypes.c_uint64), ("topk", ctypes.c_int), ("block", ctypes.c_int),
+                ("scale", ctypes.c_float), ("mode", ctypes.c_int)]
+
+
+class muse_debug(ctypes.Structure):
+    _fields_ = [("q_assign", ctypes.c_void_p), ("k_assign", ctypes.c_void_p),
+                ("selected", ctypes.c_void_p), ("k_counts", ctypes.c_void_p),
+                ("q_centroids", ctypes.c_void_p), ("k_centroids", ctypes.c_void_p),
+                ("n_exact", ctypes.c_void_p)]
+
+
+EXPORTS = ["muse_workspace_size", "muse_cluster_workspace_size", "muse_cluster", "muse_summarize",
+           "muse_attn_fwd", "muse_attn_fwd_causal", "muse_status_string", "muse_last_error"]
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libmuse.so and declare its signatures (raises if it is missing)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libmuse.so not built ({path}); run "
+                          "`python -m clustered_multipole_approximation_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, sz, i32, u64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_uint64
+    sp, pp = ctypes.POINTER(muse_shape), ctypes.POINTER(muse_params)
+    dp = ctypes.POINTER(muse_debug)
+    lib.muse_workspace_size.restype = sz
+    lib.muse_workspace_size.argtypes = [sp, pp, i32]
+    lib.muse_cluster_workspace_size.restype = sz
+    lib.muse_cluster_workspace_size.argtypes = [i32] * 5
+    lib.muse_cluster.restype = i32
+    lib.muse_cluster.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, u64, i32, vp, vp, vp, vp,
+                                 vp, sz, vp]
+    lib.muse_summarize.restype = i32
+    lib.muse_summarize.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
+                                   sz, vp]
+    for f in ("muse_attn_fwd", "muse_attn_fwd_causal"):
+        getattr(lib, f).restype = i32
+        getattr(lib, f).argtypes = [vp, vp, vp, vp, sp, pp, dp, vp, sz, vp]
+    lib.muse_status_string.restype = ctypes.c_char_p
+    lib.muse_status_string.argtypes = [i32]
+    lib.muse_last_error.restype = ctypes.c_char_p
+    lib.muse_last_error.argtypes = []
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _check(lib, st: int):
+    if st != 0:
+        raise MuseError(st, lib.muse_last_error().decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return 0
+    if t.dtype == torch.float32:
+        return 1
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def make_params(Cq, Ck, iters, seed, topk, block=0, scale=1.0, mode="dipole") -> muse_params:
+    return muse_params(int(Cq), int(Ck), int(iters), int(seed) & (2 ** 64 - 1), int(topk),
+                       int(block), float(scale), MODES[mode] if isinstance(mode, str) else int(mode))
+
+
+def make_shape(q, k) -> muse_shape:
+    B, Hq, N, D = q.shape
+    return muse_shape(B, Hq, k.shape[1], N, D, _dtype_code(q))
+
+
+def workspace_size(q, k, params: muse_params, causal: bool) -> int:
+    lib = load_library()
+    sh = make_shape(q, k)
+    n = lib.muse_workspace_size(ctypes.byref(sh), ctypes.byref(params), int(causal))
+    if n == 0:
+        raise MuseError(1, lib.muse_last_error().decode())
+    return int(n)
+
+
+def _debug_buffers(q, k, params, causal):
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    if causal:
+        from math import log2
+        lv = int(round(log2(N // params.block))) if N // params.block > 1 else 0
+        out = dict(q_assign=torch.empty(B, Hq, lv, N // 2, **i32),
+                   k_assign=torch.empty(B, Hkv, lv, N // 2, **i32))
+    else:
+        out = dict(q_assign=torch.empty(B, Hq, N, **i32), k_assign=torch.empty(B, Hkv, N, **i32),
+                   k_counts=torch.empty(B, Hkv, params.Ck, **i32),
+                   q_centroids=torch.empty(B, Hq, params.Cq, D, dtype=torch.float32, device=dev),
+                   k_centroids=torch.empty(B, Hkv, params.Ck, D, dtype=torch.float32, device=dev))
+        if params.topk > 0:
+            out["selected"] = torch.empty(B, Hq, params.Cq, params.topk, **i32)
+    out["n_exact"] = torch.empty(B, Hq, N, dtype=torch.int64, device=dev)
+    return out
+
+
+def _attn(causal, q, k, v, params, out=None, workspace=None, debug=False, stream=None):
+    lib = load_library()
+    _need_cuda(q, k, v, out, workspace)
+    if k.shape != v.shape or q.dtype != k.dtype or k.dtype != v.dtype:
+        raise ValueError("k and v must match in shape; q, k, v must share a dtype")
+    sh = make_shape(q, k)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(q, k, params, causal), dtype=torch.uint8,
+                                device=q.device)
+    dbg = None
+    bufs = None
+    if debug:
+        bufs = _debug_buffers(q, k, params, causal)
+        dbg = muse_debug(*[bufs[n].data_ptr() if n in bufs else None for n, _ in muse_debug._fields_])
+    f = lib.muse_attn_fwd_causal if causal else lib.muse_attn_fwd
+    st = f(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(sh), ctypes.byref(params),
+           ctypes.byref(dbg) if dbg is not None else None, _ptr(workspace),
+           workspace.numel(), _stream(stream))
+    _check(lib, st)
+    return (out, bufs) if debug else out
+
+
+def muse_attn_fwd(q, k, v, *, Cq, Ck, iters, seed, topk, scale=1.0, mode="dipole", out=None,
+                  workspace=None, debug=False, stream=None):
+    """Acausal MuSe forward.  q [B,Hq,N,D], k and v [B,Hkv,N,D] (bf16 or fp32,
+    contiguous, CUDA).  Returns O (and a dict of debug tensors if debug)."""
+    p = make_params(Cq, Ck, iters, seed, topk, 0, scale, mode)
+    return _attn(False, q, k, v, p, out, workspace, debug, stream)
+
+
+def muse_attn_fwd_causal(q, k, v, *, C, block, iters, seed, topk, scale=1.0, mode="dipole",
+                         out=None, workspace=None, debug=False, stream=None):
+    """Causal MuSe forward (hierarchical blocks of `block` tokens, C clusters
+    per level and role)."""
+    p = make_params(C, C, iters, seed, topk, block, scale, mode)
+    return _attn(True, q, k, v, p, out, workspace, debug, stream)
+
+
+def muse_cluster(x, C, iters, seed, role=0, init=None, workspace=None, stream=None):
+    """Lloyd k-means of each (b, h) row set of x [B,H,N,D].  Returns
+    (assign [B,H,N] int32, centroids [B,H,C,D] fp32, counts [B,H,C] int32)."""
+    lib = load_library()
+    _need_cuda(x, init, workspace)
+    B, H, N, D = x.shape
+    if init is not None and (init.dtype != torch.float32 or tuple(init.shape) != (B, H, C, D)):
+        raise ValueError("init must be fp32 [B,H,C,D]")
+    if workspace is None:
+        n = lib.muse_cluster_workspace_size(B, H, N, D, C)
+        if n == 0:
+            raise MuseError(1, "invalid sizes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    assign = torch.empty(B, H, N, dtype=torch.int32, device=x.device)
+    cent = torch.empty(B, H, C, D, dtype=torch.float32, device=x.device)
+    counts = torch.empty(B, H, C, dtype=torch.int32, device=x.device)
+    st = lib.muse_cluster(_ptr(x), _dtype_code(x), B, H, N, D, C, iters, int(seed) & (2 ** 64 - 1),
+                          role, _ptr(init), _ptr(assign), _ptr(cent), _ptr(counts),
+                          _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(lib, st)
+    return assign, cent, counts
+
+
+def muse_summarize(k, v, assign, C, with_dipole=True, stream=None):
+    """Key-cluster summaries of a given assignment: (counts, mu, S, M)."""
+    lib = load_library()
+    _need_cuda(k, v, assign)
+    B, H, N, D = k.shape
+    dev = k.device
+    counts = torch.empty(B, H, C, dtype=torch.int32, device=dev)
+    mu = torch.empty(B, H, C, D, dtype=torch.float32, device=dev)
+    S = torch.empty(B, H, C, D, dtype=torch.float32, device=dev)
+    M = torch.empty(B, H, C, D, D, dtype=torch.float32, device=dev) if with_dipole else None
+    st = lib.muse_summarize(_ptr(k), _ptr(v), _dtype_code(k), B, H, N, D, C, _ptr(assign),
+                            _ptr(counts), _ptr(mu), _ptr(S), _ptr(M), None, 0, _stream(stream))
+    _check(lib, st)
+    return counts, mu, S, M

@@ -1,0 +1,347 @@
+// C ABI of libmuse: argument checks, workspace plan, and the launch sequence
+// of each entry point.  Everything runs on the caller's stream; nothing here
+// allocates, frees or synchronises.
+#include <cuda_runtime.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "../../include/muse.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace muse;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+muse_status fail(muse_status s, const char* msg) {
+  g_last_error = msg;
+  return s;
+}
+
+muse_status check_launch() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    g_last_error = std::string("CUDA launch failed: ") + cudaGetErrorString(e);
+    return MUSE_ERR_CUDA;
+  }
+  return MUSE_OK;
+}
+
+int ilog2_exact(int x) {  // -1 unless x is a power of two
+  if (x <= 0 || (x & (x - 1))) return -1;
+  int l = 0;
+  while ((1 << l) < x) ++l;
+  return l;
+}
+
+Levels make_levels(int N, int L, bool causal) {
+  Levels lv{};
+  lv.N = N;
+  lv.causal = causal ? 1 : 0;
+  if (!causal) {
+    lv.nlev = 1;
+    lv.s[0] = N;
+    lv.npairs[0] = 1;
+    lv.tiles_per_pair[0] = cdiv(N, kTile);
+    lv.pairs_per_bh = 1;
+    lv.tiles_per_bh = lv.tiles_per_pair[0];
+    lv.toks_per_bh = N;
+    lv.pmax = 1;
+    return lv;
+  }
+  const int nblk = N / L;
+  lv.nlev = ilog2_exact(nblk);
+  lv.pmax = nblk / 2 > 0 ? nblk / 2 : 1;
+  int pb = 0, tb = 0;
+  for (int l = 0; l < lv.nlev; ++l) {
+    lv.s[l] = L << l;
+    lv.npairs[l] = nblk >> (l + 1);
+    lv.tiles_per_pair[l] = cdiv(lv.s[l], kTile);
+    lv.pair_base[l] = pb;
+    lv.tile_base[l] = tb;
+    lv.tok_base[l] = l * (N / 2);
+    pb += lv.npairs[l];
+    tb += lv.npairs[l] * lv.tiles_per_pair[l];
+  }
+  lv.pairs_per_bh = pb;
+  lv.tiles_per_bh = tb;
+  lv.toks_per_bh = lv.nlev * (N / 2);
+  return lv;
+}
+
+// Bump allocator over the caller's workspace (256-byte aligned pieces).
+struct Carver {
+  char* base;
+  size_t used = 0;
+  template <typename P>
+  P* take(size_t bytes) {
+    size_t at = (used + 255) & ~(size_t)255;
+    used = at + bytes;
+    return base ? reinterpret_cast<P*>(base + at) : nullptr;
+  }
+};
+
+void carve_kstate(Carver& cv, KState& ks, const RoleGeo& g) {
+  const long long BH = g.BH;
+  ks.nprob = (int)(BH * g.lv.pairs_per_bh);
+  ks.ntiles = BH * g.lv.tiles_per_bh;
+  ks.ntok = BH * g.lv.toks_per_bh;
+  const size_t np = ks.nprob, C = g.C, D = g.D;
+  ks.cent64 = cv.take<double>(np * C * D * 8);
+  ks.cent32 = cv.take<float>(np * C * D * 4);
+  ks.cnorm = cv.take<float>(np * C * 4);
+  ks.counts = cv.take<int>(np * C * 4);
+  ks.off = cv.take<int>(np * (C + 1) * 4);
+  ks.assign = cv.take<int>((size_t)ks.ntok * 4);
+  ks.perm = cv.take<int>((size_t)ks.ntok * 4);
+  ks.hist = cv.take<int>((size_t)ks.ntiles * C * 4);
+  ks.arrive = cv.take<int>(np * 4);
+}
+
+RoleGeo make_geo(const void* X, int BH, int D, int C, int role, int dtype, uint64_t seed,
+                 const Levels& lv) {
+  RoleGeo g{};
+  g.lv = lv;
+  g.BH = BH;
+  g.D = D;
+  g.C = C;
+  g.role = role;
+  g.dtype = dtype;
+  g.X = X;
+  g.seed = seed;
+  return g;
+}
+
+constexpr size_t kStage1Budget = (size_t)2 << 30;  // bytes of stage-1 tables per wave
+
+struct AttnPlan {
+  size_t bytes;
+  int wave;  // query problems per stage-1 wave
+};
+
+struct AttnLayout {
+  RoleGeo qg, kg;
+  KState qs, ks;
+  Stage1 s1;
+  float* part;
+  int nq;
+  int wave;
+  size_t bytes;
+};
+
+muse_status validate(const muse_shape* sh, const muse_params* pr, bool causal) {
+  if (!sh || !pr) return fail(MUSE_ERR_INVALID_ARG, "shape and params must not be NULL");
+  if (sh->B < 1 || sh->Hq < 1 || sh->Hkv < 1 || sh->N < 1)
+    return fail(MUSE_ERR_INVALID_ARG, "B, Hq, Hkv and N must be >= 1");
+  if (sh->Hq % sh->Hkv) return fail(MUSE_ERR_INVALID_ARG, "Hq must be a multiple of Hkv");
+  if (sh->D != 64 && sh->D != 128) return fail(MUSE_ERR_UNSUPPORTED, "D must be 64 or 128");
+  if (sh->dtype != MUSE_BF16 && sh->dtype != MUSE_F32)
+    return fail(MUSE_ERR_INVALID_ARG, "dtype must be MUSE_BF16 or MUSE_F32");
+  if (pr->iters < 1) return fail(MUSE_ERR_INVALID_ARG, "iters must be >= 1");
+  if (pr->mode < MUSE_MONOPOLE || pr->mode > MUSE_TILTED)
+    return fail(MUSE_ERR_INVALID_ARG, "unknown mode");
+  if (pr->Cq < 1 || pr->Ck < 1) return fail(MUSE_ERR_INVALID_ARG, "Cq and Ck must be >= 1");
+  if (pr->Cq > kMaxC || pr->Ck > kMaxC)
+    return fail(MUSE_ERR_UNSUPPORTED, "Cq and Ck must be <= 1024");
+  if (pr->topk < 0 || pr->topk > pr->Ck)
+    return fail(MUSE_ERR_INVALID_ARG, "topk must be in [0, Ck]");
+  if (!(pr->scale == pr->scale)) return fail(MUSE_ERR_INVALID_ARG, "scale is NaN");
+  const long long elems = (long long)sh->B * (sh->Hq > sh->Hkv ? sh->Hq : sh->Hkv) * sh->N;
+  if (elems > (1LL << 31) - 1) return fail(MUSE_ERR_UNSUPPORTED, "B*H*N must be < 2^31");
+  if (!causal) {
+    if (pr->Cq > sh->N || pr->Ck > sh->N)
+      return fail(MUSE_ERR_INVALID_ARG, "Cq and Ck must be <= N");
+  } else {
+    if (pr->Cq != pr->Ck) return fail(MUSE_ERR_INVALID_ARG, "causal needs Cq == Ck");
+    if (pr->block < 1 || sh->N % pr->block)
+      return fail(MUSE_ERR_INVALID_ARG, "block must divide N");
+    if (ilog2_exact(sh->N / pr->block) < 0)
+      return fail(MUSE_ERR_INVALID_ARG, "N / block must be a power of two");
+    if (ilog2_exact(sh->N / pr->block) >= kMaxLevels)
+      return fail(MUSE_ERR_UNSUPPORTED, "too many levels");
+  }
+  return MUSE_OK;
+}
+
+AttnLayout layout(const muse_shape* sh, const muse_params* pr, bool causal, const void* Q,
+                  const void* K, void* ws) {
+  AttnLayout L{};
+  const Levels lv = make_levels(sh->N, causal ? pr->block : sh->N, causal);
+  const int dt = sh->dtype == MUSE_BF16 ? 0 : 1;
+  L.kg = make_geo(K, sh->B * sh->Hkv, sh->D, pr->Ck, 0, dt, pr->seed, lv);
+  L.qg = make_geo(Q, sh->B * sh->Hq, sh->D, pr->Cq, 1, dt, pr->seed, lv);
+  Carver cv{static_cast<char*>(ws)};
+  carve_kstate(cv, L.ks, L.kg);
+  carve_kstate(cv, L.qs, L.qg);
+  L.nq = L.qs.nprob;
+  const size_t cc = (size_t)pr->Cq * pr->Ck;
+  const size_t per = cc * 4 * 2 + cc * sh->D * 4 * (pr->mode == MUSE_TILTED ? 2 : 1);
+  size_t wave = L.nq;
+  if (causal && per * wave > kStage1Budget) wave = kStage1Budget / per;
+  if (wave < 1) wave = 1;
+  L.wave = (int)wave;
+  L.s1.logW = cv.take<float>(wave * cc * 4);
+  L.s1.fbias = cv.take<float>(wave * cc * 4);
+  L.s1.U = cv.take<float>(wave * cc * sh->D * 4);
+  L.s1.Kf = pr->mode == MUSE_TILTED ? cv.take<float>(wave * cc * sh->D * 4) : nullptr;
+  const int k1 = pr->topk > 0 ? pr->topk : 1;
+  L.s1.sel = cv.take<int>((size_t)L.nq * pr->Cq * k1 * 4);
+  L.s1.nsel = cv.take<int>((size_t)L.nq * pr->Cq * 4);
+  L.part = causal ? cv.take<float>((size_t)L.qs.ntok * (sh->D + 1) * 4) : nullptr;
+  L.bytes = cv.used + 256;
+  return L;
+}
+
+muse_status attn(const void* Q, const void* K, const void* V, void* O, const muse_shape* sh,
+                 const muse_params* pr, muse_debug* dbg, void* ws, size_t ws_bytes,
+                 cudaStream_t st, bool causal) {
+  muse_status s = validate(sh, pr, causal);
+  if (s != MUSE_OK) return s;
+  if (!Q || !K || !V || !O) return fail(MUSE_ERR_INVALID_ARG, "Q, K, V and O must not be NULL");
+  const AttnLayout need = layout(sh, pr, causal, Q, K, nullptr);
+  if (!ws || ws_bytes < need.bytes) return fail(MUSE_ERR_WORKSPACE, "workspace too small");
+  AttnLayout L = layout(sh, pr, causal, Q, K, ws);
+  AttnArgs a{};
+  a.qg = L.qg;
+  a.kg = L.kg;
+  a.qs = L.qs;
+  a.ks = L.ks;
+  a.V = V;
+  a.O = causal ? nullptr : O;
+  a.part = L.part;
+  a.n_exact = dbg ? reinterpret_cast<long long*>(dbg->n_exact) : nullptr;
+  a.B = sh->B;
+  a.G = sh->Hq / sh->Hkv;
+  a.mode = (int)pr->mode;
+  a.topk = pr->topk;
+  a.scale = pr->scale;
+  a.Cq = pr->Cq;
+  a.Ck = pr->Ck;
+  const size_t elt = sh->dtype == MUSE_BF16 ? 2 : 4;
+  if (a.n_exact && causal)
+    cudaMemsetAsync(a.n_exact, 0, (size_t)sh->B * sh->Hq * sh->N * 8, st);
+  if (L.nq > 0) {
+    cudaMemsetAsync(L.ks.arrive, 0, (size_t)L.ks.nprob * 4, st);
+    cudaMemsetAsync(L.qs.arrive, 0, (size_t)L.qs.nprob * 4, st);
+    run_kmeans(L.kg, L.ks, pr->iters, nullptr, st);
+    run_kmeans(L.qg, L.qs, pr->iters, nullptr, st);
+    for (int q0 = 0; q0 < L.nq; q0 += L.wave) {
+      const int n = L.nq - q0 < L.wave ? L.nq - q0 : L.wave;
+      run_blocks(a, L.s1, q0, n, st);
+    }
+  }
+  if (causal) {
+    a.O = O;
+    run_local_merge(a, pr->block, st);
+  }
+  if (dbg) {
+    const size_t D = sh->D;
+    if (dbg->q_assign) cudaMemcpyAsync(dbg->q_assign, L.qs.assign, (size_t)L.qs.ntok * 4, cudaMemcpyDeviceToDevice, st);
+    if (dbg->k_assign) cudaMemcpyAsync(dbg->k_assign, L.ks.assign, (size_t)L.ks.ntok * 4, cudaMemcpyDeviceToDevice, st);
+    if (!causal) {
+      if (dbg->k_counts) cudaMemcpyAsync(dbg->k_counts, L.ks.counts, (size_t)L.ks.nprob * pr->Ck * 4, cudaMemcpyDeviceToDevice, st);
+      if (dbg->q_centroids) cudaMemcpyAsync(dbg->q_centroids, L.qs.cent32, (size_t)L.qs.nprob * pr->Cq * D * 4, cudaMemcpyDeviceToDevice, st);
+      if (dbg->k_centroids) cudaMemcpyAsync(dbg->k_centroids, L.ks.cent32, (size_t)L.ks.nprob * pr->Ck * D * 4, cudaMemcpyDeviceToDevice, st);
+      if (dbg->selected && pr->topk > 0)
+        cudaMemcpyAsync(dbg->selected, L.s1.sel, (size_t)L.nq * pr->Cq * pr->topk * 4, cudaMemcpyDeviceToDevice, st);
+    }
+  }
+  (void)elt;
+  return check_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t muse_workspace_size(const muse_shape* shape, const muse_params* params, int causal) {
+  if (validate(shape, params, causal != 0) != MUSE_OK) return 0;
+  return layout(shape, params, causal != 0, nullptr, nullptr, nullptr).bytes;
+}
+
+size_t muse_cluster_workspace_size(int B, int H, int N, int D, int C) {
+  if (B < 1 || H < 1 || N < 1 || C < 1 || (D != 64 && D != 128)) return 0;
+  const Levels lv = make_levels(N, N, false);
+  RoleGeo g = make_geo(nullptr, B * H, D, C, 0, 0, 0, lv);
+  Carver cv{nullptr};
+  KState ks{};
+  carve_kstate(cv, ks, g);
+  return cv.used + 256;
+}
+
+muse_status muse_cluster(const void* X, muse_dtype dtype, int B, int H, int N, int D, int C,
+                         int iters, uint64_t seed, int role, const float* init, int32_t* assign,
+                         float* centroids, int32_t* counts, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  if (!X || !assign || !centroids) return fail(MUSE_ERR_INVALID_ARG, "X, assign and centroids must not be NULL");
+  if (B < 1 || H < 1 || N < 1) return fail(MUSE_ERR_INVALID_ARG, "B, H and N must be >= 1");
+  if (D != 64 && D != 128) return fail(MUSE_ERR_UNSUPPORTED, "D must be 64 or 128");
+  if (dtype != MUSE_BF16 && dtype != MUSE_F32) return fail(MUSE_ERR_INVALID_ARG, "bad dtype");
+  if (C < 1 || C > N) return fail(MUSE_ERR_INVALID_ARG, "C must be in [1, N]");
+  if (C > kMaxC) return fail(MUSE_ERR_UNSUPPORTED, "C must be <= 1024");
+  if (iters < 1) return fail(MUSE_ERR_INVALID_ARG, "iters must be >= 1");
+  if (role != 0 && role != 1) return fail(MUSE_ERR_INVALID_ARG, "role must be 0 or 1");
+  if ((long long)B * H * N > (1LL << 31) - 1) return fail(MUSE_ERR_UNSUPPORTED, "B*H*N must be < 2^31");
+  const size_t need = muse_cluster_workspace_size(B, H, N, D, C);
+  if (!ws || ws_bytes < need) return fail(MUSE_ERR_WORKSPACE, "workspace too small");
+  const Levels lv = make_levels(N, N, false);
+  RoleGeo g = make_geo(X, B * H, D, C, role, dtype == MUSE_BF16 ? 0 : 1, seed, lv);
+  Carver cv{static_cast<char*>(ws)};
+  KState ks{};
+  carve_kstate(cv, ks, g);
+  cudaMemsetAsync(ks.arrive, 0, (size_t)ks.nprob * 4, stream);
+  run_kmeans(g, ks, iters, init, stream);
+  cudaMemcpyAsync(assign, ks.assign, (size_t)ks.ntok * 4, cudaMemcpyDeviceToDevice, stream);
+  cudaMemcpyAsync(centroids, ks.cent32, (size_t)ks.nprob * C * D * 4, cudaMemcpyDeviceToDevice, stream);
+  if (counts) cudaMemcpyAsync(counts, ks.counts, (size_t)ks.nprob * C * 4, cudaMemcpyDeviceToDevice, stream);
+  return check_launch();
+}
+
+muse_status muse_summarize(const void* K, const void* V, muse_dtype dtype, int B, int H, int N,
+                           int D, int C, const int32_t* assign, int32_t* counts, float* mu,
+                           float* S, float* M, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!K || !V || !assign || !counts || !mu || !S)
+    return fail(MUSE_ERR_INVALID_ARG, "K, V, assign, counts, mu and S must not be NULL");
+  if (B < 1 || H < 1 || N < 1) return fail(MUSE_ERR_INVALID_ARG, "B, H and N must be >= 1");
+  if (D != 64 && D != 128) return fail(MUSE_ERR_UNSUPPORTED, "D must be 64 or 128");
+  if (dtype != MUSE_BF16 && dtype != MUSE_F32) return fail(MUSE_ERR_INVALID_ARG, "bad dtype");
+  if (C < 1) return fail(MUSE_ERR_INVALID_ARG, "C must be >= 1");
+  if (C > 65535) return fail(MUSE_ERR_UNSUPPORTED, "C must be < 65536");
+  run_summarize(K, V, dtype == MUSE_BF16 ? 0 : 1, B * H, N, D, C, assign, counts, mu, S, M,
+                nullptr, nullptr, stream);
+  return check_launch();
+}
+
+muse_status muse_attn_fwd(const void* Q, const void* K, const void* V, void* O,
+                          const muse_shape* shape, const muse_params* params, muse_debug* debug,
+                          void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return attn(Q, K, V, O, shape, params, debug, ws, ws_bytes, stream, false);
+}
+
+muse_status muse_attn_fwd_causal(const void* Q, const void* K, const void* V, void* O,
+                                 const muse_shape* shape, const muse_params* params,
+                                 muse_debug* debug, void* ws, size_t ws_bytes,
+                                 cudaStream_t stream) {
+  return attn(Q, K, V, O, shape, params, debug, ws, ws_bytes, stream, true);
+}
+
+const char* muse_status_string(muse_status s) {
+  switch (s) {
+    case MUSE_OK: return "ok";
+    case MUSE_ERR_INVALID_ARG: return "invalid argument";
+    case MUSE_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case MUSE_ERR_WORKSPACE: return "workspace too small";
+    case MUSE_ERR_CUDA: return "CUDA error";
+    case MUSE_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+const char* muse_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+// Shared device-side definitions of libmuse: problem geometry, element
+// loads, and the workspace-resident per-problem state.
+//
+// A "problem" is one clustering of one token block: acausal -> the whole
+// sequence of one (b, head); causal -> the key block or the query block of
+// one (level, pair) of the hierarchical decomposition of one (b, head).  Both
+// cases are one level table: acausal has a single level with one pair whose
+// block is the whole sequence.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace muse {
+
+constexpr int kMaxLevels = 24;
+constexpr int kTile = 128;  // tokens per assignment tile
+constexpr int kMaxC = 1024;
+
+struct Levels {
+  int nlev;                 // number of levels (acausal: 1)
+  int causal;
+  int N;                    // sequence length
+  int s[kMaxLevels];        // block size of each level
+  int npairs[kMaxLevels];   // pairs at each level
+  int pair_base[kMaxLevels];   // first pair index of the level (per bh)
+  int tile_base[kMaxLevels];   // first tile index of the level (per bh)
+  int tiles_per_pair[kMaxLevels];
+  int tok_base[kMaxLevels];    // first token slot of the level (per bh)
+  int pairs_per_bh;
+  int tiles_per_bh;
+  int toks_per_bh;
+  int pmax;                 // pairs at level 0 (stream-id stride)
+};
+
+// Geometry of one role (keys or queries) over one tensor.
+struct RoleGeo {
+  Levels lv;
+  int BH;      // B * heads of this tensor
+  int D;
+  int C;       // requested clusters (effective: min(C, s))
+  int role;    // 0 keys, 1 queries
+  int dtype;   // 0 bf16, 1 f32
+  const void* X;
+  uint64_t seed;
+};
+
+struct Prob {
+  int bh, level, pair, s, C;
+  long long row0;   // first row of the block in X (rows of D elements)
+  long long slot0;  // first token slot of the problem (assign / perm arrays)
+  long long tile0;  // first global tile of the problem
+  uint64_t sid;
+};
+
+__host__ __device__ inline int imin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+__device__ inline Prob prob_of(const RoleGeo& g, int pid) {
+  Prob p;
+  const Levels& L = g.lv;
+  p.bh = pid / L.pairs_per_bh;
+  int pi = pid - p.bh * L.pairs_per_bh;
+  int l = 0;
+  while (l + 1 < L.nlev && pi >= L.pair_base[l + 1]) ++l;
+  p.level = l;
+  p.pair = pi - L.pair_base[l];
+  p.s = L.s[l];
+  p.C = imin(g.C, p.s);
+  long long seq0 = (long long)p.bh * L.N;
+  p.row0 = seq0 + (L.causal ? (long long)(2 * p.pair + g.role) * p.s : 0);
+  p.slot0 = (long long)p.bh * L.toks_per_bh + L.tok_base[l] + (long long)p.pair * p.s;
+  p.tile0 = (long long)p.bh * L.tiles_per_bh + L.tile_base[l] +
+            (long long)p.pair * L.tiles_per_pair[l];
+  p.sid = L.causal ? ((uint64_t)p.bh * L.nlev + l) * (uint64_t)L.pmax + p.pair
+                   : (uint64_t)p.bh;
+  return p;
+}
+
+// Global tile -> (problem id, tile within problem).
+__device__ inline void tile_of(const RoleGeo& g, long long t, int* pid, int* tin) {
+  const Levels& L = g.lv;
+  int bh = (int)(t / L.tiles_per_bh);
+  int r = (int)(t - (long long)bh * L.tiles_per_bh);
+  int l = 0;
+  while (l + 1 < L.nlev && r >= L.tile_base[l + 1]) ++l;
+  r -= L.tile_base[l];
+  int pair = r / L.tiles_per_pair[l];
+  *tin = r - pair * L.tiles_per_pair[l];
+  *pid = bh * L.pairs_per_bh + L.pair_base[l] + pair;
+}
+
+template <typename T>
+__device__ inline float ld(const T* p);
+template <>
+__device__ inline float ld<float>(const float* p) { return *p; }
+template <>
+__device__ inline float ld<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+template <typename T>
+__device__ inline void st(T* p, float v);
+template <>
+__device__ inline void st<float>(float* p, float v) { *p = v; }
+template <>
+__device__ inline void st<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+// Per-role k-means state in the workspace.
+struct KState {
+  double* cent64;   // [nprob][C][D] current centroids (fp64 master copy)
+  float* cent32;    // [nprob][C][D] fp32 rounding of cent64
+  float* cnorm;     // [nprob][C]    ||cent32|| (slightly enlarged)
+  int* counts;      // [nprob][C]
+  int* off;         // [nprob][C+1]  segment offsets of the sorted order
+  int* assign;      // [tokens]      cluster of each token (problem-local index)
+  int* perm;        // [tokens]      problem-local token index in cluster-sorted order
+  int* hist;        // [tiles][C]    per-tile histogram, then scatter bases
+  int* arrive;      // [nprob]       tile arrival counters (self-resetting)
+  int nprob;
+  long long ntiles;
+  long long ntok;
+};
+
+}  // namespace muse

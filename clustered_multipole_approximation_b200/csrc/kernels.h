@@ -1,0 +1,48 @@
+// Host-side launchers shared between the translation units of libmuse.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace muse {
+
+// Per-(query problem) stage-1 tables in the workspace.
+struct Stage1 {
+  float* logW;    // [nq][Cq][Ck]  log W_ij, -inf for empty key clusters
+  float* fbias;   // [nq][Cq][Ck]  far-field logit offset (log W, plus the tilt term)
+  float* U;       // [nq][Cq][Ck][D] summary values u_ij
+  float* Kf;      // [nq][Cq][Ck][D] far-field key rows (TILTED only: k_hat_ij)
+  int* sel;       // [nq_total][Cq][topk]
+  int* nsel;      // [nq_total][Cq]
+};
+
+struct AttnArgs {
+  RoleGeo qg, kg;     // query and key geometry
+  KState qs, ks;      // their k-means state
+  const void* V;
+  void* O;            // acausal: final output
+  float* part;        // causal: [nq_total tokens][D + 1] partial (o, lse)
+  long long* n_exact; // optional [B,Hq,N]
+  int B;              // batch
+  int G;              // q-heads per kv-head
+  int mode, topk;
+  float scale;
+  int Cq, Ck;
+};
+
+void run_kmeans(const RoleGeo& g, const KState& ks, int iters, const float* init,
+                cudaStream_t st);
+
+// Stage 1 + selection + stage 2 for query problems [qp0, qp0 + nqp).
+void run_blocks(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
+
+// Causal: exact local block + merge of the level partials into O.
+void run_local_merge(const AttnArgs& a, int L, cudaStream_t st);
+
+// Summaries (n, mu, S, M) of given assignments; used by muse_summarize.
+void run_summarize(const void* K, const void* V, int dtype, int BH, int N, int D, int C,
+                   const int* assign, int* counts, float* mu, float* S, float* M,
+                   int* perm, int* off, cudaStream_t st);
+
+}  // namespace muse

@@ -1,0 +1,388 @@
+// Lloyd k-means over many token blocks at once (the clustering step of
+// MuSe: queries and keys are clustered separately, each in its own space --
+// "Multipole Semantic Attention" gist.science page, Technical Summary, Core
+// Mechanisms, "Bidirectional Semantic Clustering").
+//
+// One round = assign -> scatter -> reduce:
+//   assign   128 tokens per CTA.  An fp32 screen computes every squared
+//            distance together with a certified error bound; a token whose
+//            best and runner-up bounds overlap is re-decided in fp64 with the
+//            same operation order as a plain sequential evaluation, ties to
+//            the lowest index.  The CTA writes its per-cluster histogram; the
+//            last CTA of each problem to finish turns the histograms into
+//            cluster offsets and per-tile scatter bases.
+//   scatter  stable counting-sort scatter: perm lists each problem's tokens
+//            grouped by cluster, ascending token order inside a cluster.
+//   reduce   one warp per (problem, cluster): fp64 sum of the members in
+//            ascending token order, divided by the count; an empty cluster
+//            keeps its centroid.
+// Every reduction has a fixed order, so results are bitwise reproducible and
+// the centroids equal a sequential fp64 evaluation of the same means.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace muse {
+
+// ----------------------------------------------------------------------------
+// seeded start: splitmix64-driven partial Fisher-Yates over the block rows
+// ----------------------------------------------------------------------------
+__device__ inline uint64_t splitmix64_next(uint64_t& state) {
+  uint64_t z = (state += 0x9E3779B97F4A7C15ULL);
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+constexpr int kHashSize = 2 * kMaxC;  // open addressing, load <= 1/2
+
+template <typename T>
+__global__ void __launch_bounds__(128) kmeans_init_kernel(RoleGeo g, KState ks, const float* init) {
+  __shared__ int hkey[kHashSize];
+  __shared__ int hval[kHashSize];
+  __shared__ int pick[kMaxC];
+  const int pid = blockIdx.x;
+  const Prob p = prob_of(g, pid);
+  const int D = g.D, C = p.C;
+  const T* X = static_cast<const T*>(g.X);
+  double* c64 = ks.cent64 + (size_t)pid * g.C * D;
+  float* c32 = ks.cent32 + (size_t)pid * g.C * D;
+  if (init == nullptr) {
+    for (int i = threadIdx.x; i < kHashSize; i += blockDim.x) hkey[i] = -1;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint64_t st = g.seed + 0x9E3779B97F4A7C15ULL * (2ULL * p.sid + (uint64_t)g.role + 1ULL);
+      const int n = p.s;
+      for (int c = 0; c < C; ++c) {
+        uint64_t r = splitmix64_next(st);
+        int j = c + (int)(r % (uint64_t)(n - c));
+        // value currently at position j (identity unless swapped before)
+        int h = j & (kHashSize - 1), vj = j;
+        while (hkey[h] >= 0) {
+          if (hkey[h] == j) { vj = hval[h]; break; }
+          h = (h + 1) & (kHashSize - 1);
+        }
+        int vc = c;
+        int hc = c & (kHashSize - 1);
+        while (hkey[hc] >= 0) {
+          if (hkey[hc] == c) { vc = hval[hc]; break; }
+          hc = (hc + 1) & (kHashSize - 1);
+        }
+        pick[c] = vj;
+        // position j now holds the old value of position c
+        h = j & (kHashSize - 1);
+        while (hkey[h] >= 0 && hkey[h] != j) h = (h + 1) & (kHashSize - 1);
+        hkey[h] = j;
+        hval[h] = vc;
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < C * D; i += blockDim.x) {
+      int c = i / D, d = i - c * D;
+      double v = (double)ld<T>(X + (p.row0 + pick[c]) * D + d);
+      c64[i] = v;
+      c32[i] = (float)v;
+    }
+  } else {
+    const float* src = init + (size_t)p.bh * g.C * D;  // muse_cluster: one problem per bh
+    for (int i = threadIdx.x; i < C * D; i += blockDim.x) {
+      c64[i] = (double)src[i];
+      c32[i] = src[i];
+    }
+  }
+  __syncthreads();
+  // centroid norms for the screen bound
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int c = warp; c < C; c += blockDim.x >> 5) {
+    float s = 0.f;
+    for (int d = lane; d < D; d += 32) {
+      float v = c32[(size_t)c * D + d];
+      s = fmaf(v, v, s);
+    }
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) ks.cnorm[(size_t)pid * g.C + c] = sqrtf(s) * 1.0001f;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// assign: fp32 screen with a certified bound, fp64 re-decision of near ties
+// ----------------------------------------------------------------------------
+constexpr int kChunk = 32;
+
+template <int D>
+constexpr size_t assign_smem() {
+  return ((size_t)kTile * (D + 1) + (size_t)kChunk * D + kMaxC) * sizeof(float) +
+         kMaxC * sizeof(int);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kTile) kmeans_assign_kernel(RoleGeo g, KState ks) {
+  extern __shared__ float as_dyn[];
+  float(*xs)[D + 1] = reinterpret_cast<float(*)[D + 1]>(as_dyn);
+  float(*cs)[D] = reinterpret_cast<float(*)[D]>(as_dyn + kTile * (D + 1));
+  float* cn = as_dyn + kTile * (D + 1) + kChunk * D;
+  int* hist = reinterpret_cast<int*>(cn + kMaxC);
+  __shared__ int flagged[kTile];
+  __shared__ int decision[kTile];
+  __shared__ int nflag;
+  __shared__ int is_last;
+
+  int pid, tin;
+  tile_of(g, blockIdx.x, &pid, &tin);
+  const Prob p = prob_of(g, pid);
+  const int C = p.C;
+  const int t0 = tin * kTile;
+  const int nt = imin(kTile, p.s - t0);
+  const T* X = static_cast<const T*>(g.X);
+  const float* c32 = ks.cent32 + (size_t)pid * g.C * D;
+  const double* c64 = ks.cent64 + (size_t)pid * g.C * D;
+  const int tid = threadIdx.x;
+
+  for (int i = tid; i < C; i += kTile) {
+    cn[i] = ks.cnorm[(size_t)pid * g.C + i];
+    hist[i] = 0;
+  }
+  if (tid == 0) nflag = 0;
+  for (int i = tid; i < nt * D; i += kTile) {
+    int r = i / D, d = i - r * D;
+    xs[r][d] = ld<T>(X + (p.row0 + t0 + r) * D + d);
+  }
+  __syncthreads();
+
+  const bool valid = tid < nt;
+  float xn = 0.f;
+  for (int d = 0; d < D; ++d) xn = fmaf(xs[tid][d], xs[tid][d], xn);
+  xn = sqrtf(xn) * 1.0001f;
+  // |d~ - d| <= u (D+4) d~ + 2.01 u (|x| + |c|) |c|   (u = 2^-24), see the
+  // derivation in the design notes: fp32 rounding of the centroid, of each
+  // difference and of each fused square-accumulate.
+  const float u = 5.9604645e-08f;
+  const float ea = u * (float)(D + 4), eb = 2.01f * u;
+  float bd = INFINITY, be = 0.f, blb = INFINITY, olb = INFINITY;
+  int best = 0;
+  for (int c0 = 0; c0 < C; c0 += kChunk) {
+    const int cc = imin(kChunk, C - c0);
+    __syncthreads();
+    for (int i = tid; i < cc * D; i += kTile) cs[i / D][i % D] = c32[(size_t)c0 * D + i];
+    __syncthreads();
+    if (valid) {
+      for (int k = 0; k < cc; ++k) {
+        float dd = 0.f;
+#pragma unroll 16
+        for (int d = 0; d < D; ++d) {
+          float t = xs[tid][d] - cs[k][d];
+          dd = fmaf(t, t, dd);
+        }
+        const float cnk = cn[c0 + k];
+        const float e = fmaf(ea, dd, eb * (xn + cnk) * cnk);
+        const float lb = dd - e;
+        if (dd < bd) {
+          olb = fminf(olb, blb);
+          bd = dd;
+          be = e;
+          blb = lb;
+          best = c0 + k;
+        } else {
+          olb = fminf(olb, lb);
+        }
+      }
+    }
+  }
+  if (valid && olb <= bd + be) {
+    int slot = atomicAdd(&nflag, 1);
+    flagged[slot] = tid;
+  }
+  __syncthreads();
+  // fp64 re-decision, one warp per flagged token, lanes over clusters; the
+  // distance is accumulated in dimension order without fused operations so
+  // it equals a plain sequential fp64 evaluation bit for bit.
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int f = warp; f < nflag; f += kTile / 32) {
+    const int r = flagged[f];
+    double bdd = 0.0;
+    int bc = -1;
+    for (int c = lane; c < C; c += 32) {
+      const double* cc = c64 + (size_t)c * D;
+      double s = 0.0;
+      for (int d = 0; d < D; ++d) {
+        double t = __dsub_rn((double)xs[r][d], cc[d]);
+        s = __dadd_rn(s, __dmul_rn(t, t));
+      }
+      if (bc < 0 || s < bdd) {
+        bdd = s;
+        bc = c;
+      }
+    }
+    for (int o = 16; o; o >>= 1) {
+      double od = __shfl_xor_sync(0xffffffffu, bdd, o);
+      int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+      if (oc >= 0 && (bc < 0 || od < bdd || (od == bdd && oc < bc))) {
+        bdd = od;
+        bc = oc;
+      }
+    }
+    if (lane == 0) decision[r] = bc;
+  }
+  __syncthreads();
+  if (valid) {
+    if (olb <= bd + be) best = decision[tid];
+    ks.assign[p.slot0 + t0 + tid] = best;
+    atomicAdd(&hist[best], 1);
+  }
+  __syncthreads();
+  int* th = ks.hist + (size_t)blockIdx.x * g.C;
+  for (int i = tid; i < C; i += kTile) th[i] = hist[i];
+  // the last tile of the problem turns histograms into offsets and bases
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int ntp = cdiv(p.s, kTile);
+    is_last = (atomicAdd(&ks.arrive[pid], 1) == ntp - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int ntp = cdiv(p.s, kTile);
+  int* ph = ks.hist + (size_t)p.tile0 * g.C;
+  int* cnt = ks.counts + (size_t)pid * g.C;
+  int* off = ks.off + (size_t)pid * (g.C + 1);
+  for (int c = tid; c < C; c += kTile) {
+    int tot = 0;
+    for (int t = 0; t < ntp; ++t) tot += __ldcg(ph + (size_t)t * g.C + c);
+    hist[c] = tot;
+    cnt[c] = tot;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int c = 0; c < C; ++c) {
+      off[c] = run;
+      int v = hist[c];
+      hist[c] = run;
+      run += v;
+    }
+    off[C] = run;
+    ks.arrive[pid] = 0;
+  }
+  __syncthreads();
+  for (int c = tid; c < C; c += kTile) {
+    int run = hist[c];
+    for (int t = 0; t < ntp; ++t) {
+      int* h = ph + (size_t)t * g.C + c;
+      int v = __ldcg(h);
+      *h = run;
+      run += v;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// scatter: stable counting sort of each problem's tokens by cluster
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(kTile) kmeans_scatter_kernel(RoleGeo g, KState ks) {
+  __shared__ int cnt[kMaxC];
+  int pid, tin;
+  tile_of(g, blockIdx.x, &pid, &tin);
+  const Prob p = prob_of(g, pid);
+  const int t0 = tin * kTile;
+  const int nt = imin(kTile, p.s - t0);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < p.C; i += kTile) cnt[i] = 0;
+  __syncthreads();
+  const int* base = ks.hist + (size_t)blockIdx.x * g.C;
+  const bool valid = tid < nt;
+  const int a = valid ? ks.assign[p.slot0 + t0 + tid] : -1 - tid;
+  const unsigned same = __match_any_sync(0xffffffffu, a);
+  const int rank = __popc(same & ((1u << lane) - 1u));
+  for (int w = 0; w < kTile / 32; ++w) {
+    if (warp == w && valid) {
+      ks.perm[p.slot0 + base[a] + cnt[a] + rank] = t0 + tid;
+    }
+    __syncthreads();
+    if (warp == w && valid && rank == 0) cnt[a] += __popc(same);
+    __syncthreads();
+  }
+}
+
+// ----------------------------------------------------------------------------
+// reduce: centroid = fp64 mean of the members in ascending token order
+// ----------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256) kmeans_reduce_kernel(RoleGeo g, KState ks) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long gw = (long long)blockIdx.x * 8 + warp;
+  const int pid = (int)(gw / g.C), c = (int)(gw - (long long)pid * g.C);
+  if (pid >= ks.nprob) return;
+  const Prob p = prob_of(g, pid);
+  if (c >= p.C) return;
+  const int* off = ks.off + (size_t)pid * (g.C + 1);
+  const int b = off[c], e = off[c + 1];
+  double* c64 = ks.cent64 + ((size_t)pid * g.C + c) * D;
+  float* c32 = ks.cent32 + ((size_t)pid * g.C + c) * D;
+  constexpr int R = D / 32;
+  if (e > b) {
+    const T* X = static_cast<const T*>(g.X);
+    const int* perm = ks.perm + p.slot0;
+    double s[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) s[r] = 0.0;
+    for (int m = b; m < e; ++m) {
+      const T* row = X + (p.row0 + perm[m]) * D;
+#pragma unroll
+      for (int r = 0; r < R; ++r) s[r] = __dadd_rn(s[r], (double)ld<T>(row + lane + 32 * r));
+    }
+    const double n = (double)(e - b);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      double v = __ddiv_rn(s[r], n);
+      c64[lane + 32 * r] = v;
+      c32[lane + 32 * r] = (float)v;
+    }
+  }
+  __syncwarp();
+  float q = 0.f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    float v = c32[lane + 32 * r];
+    q = fmaf(v, v, q);
+  }
+  for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  if (lane == 0) ks.cnorm[(size_t)pid * g.C + c] = sqrtf(q) * 1.0001f;
+}
+
+// ----------------------------------------------------------------------------
+// host-side launchers
+// ----------------------------------------------------------------------------
+template <typename T, int D>
+static void launch_round(const RoleGeo& g, const KState& ks, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)assign_smem<D>());
+    attr = true;
+  }
+  kmeans_assign_kernel<T, D><<<(unsigned)ks.ntiles, kTile, assign_smem<D>(), st>>>(g, ks);
+  kmeans_scatter_kernel<<<(unsigned)ks.ntiles, kTile, 0, st>>>(g, ks);
+  const long long warps = (long long)ks.nprob * g.C;
+  kmeans_reduce_kernel<T, D><<<(unsigned)cdiv((int)warps, 8), 256, 0, st>>>(g, ks);
+}
+
+template <typename T>
+static void run_kmeans_t(const RoleGeo& g, const KState& ks, int iters, const float* init,
+                         cudaStream_t st) {
+  kmeans_init_kernel<T><<<ks.nprob, 128, 0, st>>>(g, ks, init);
+  for (int it = 0; it < iters; ++it) {
+    if (g.D == 64)
+      launch_round<T, 64>(g, ks, st);
+    else
+      launch_round<T, 128>(g, ks, st);
+  }
+}
+
+void run_kmeans(const RoleGeo& g, const KState& ks, int iters, const float* init, cudaStream_t st) {
+  if (g.dtype == 0)
+    run_kmeans_t<__nv_bfloat16>(g, ks, iters, init, st);
+  else
+    run_kmeans_t<float>(g, ks, iters, init, st);
+}
+
+}  // namespace muse

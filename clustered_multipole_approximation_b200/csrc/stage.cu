@@ -1,0 +1,520 @@
+// Stage 1 (query-cluster summaries, selection) and stage 2 (far field +
+// exact retrieval, one softmax) of MuSe, plus the causal local block and the
+// merge of the hierarchical levels.
+//
+// Sources: the gist.science page "Multipole Semantic Attention: A Fast
+// Approximation of Softmax Attention for Pretraining", Technical Summary,
+// Core Mechanisms (residual decomposition; Stage 1 (Coarse); Stage 2
+// (Refinement); Exponential Tilting; Cluster Selection; Exact Attention), and
+// the newx.sg page of the same title, Abstract (monopole + dipole;
+// hierarchical block decomposition).
+//
+// With nu_i the query-cluster centroid, mu_j the key-cluster centroid and
+// k~ = k - mu_j, the kept terms of exp(s (nu_i + q~).(mu_j + k~)) give per key
+// cluster j, as seen from query cluster i:
+//   MONOPOLE  W_ij = n_j,                     u_ij = S_j / n_j
+//   DIPOLE    W_ij = n_j,                     u_ij = sum_t v_t (1 + s nu_i.k~_t) / n_j
+//             (= (S_j + s M_j nu_i) / n_j, the dipole moment contracted with
+//             nu_i, evaluated without forming M_j)
+//   TILTED    w_t = exp(s nu_i.k~_t), W_ij = sum w_t, u_ij = sum w_t v_t / W_ij,
+//             k_hat_ij = sum w_t k_t / W_ij
+// and the far-field logit of a query q of cluster i is
+//   s q.mu_j + log W_ij                                   (MONOPOLE, DIPOLE)
+//   s q.k_hat_ij + s nu_i.(mu_j - k_hat_ij) + log W_ij    (TILTED)
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace muse {
+
+__device__ inline int kv_problem(const AttnArgs& a, int qpid) {
+  const int ppb = a.qg.lv.pairs_per_bh;
+  const int bhq = qpid / ppb, pi = qpid - bhq * ppb;
+  const int Hq = a.qg.BH / a.B, Hkv = a.kg.BH / a.B;
+  const int b = bhq / Hq, hq = bhq - b * Hq;
+  const int bhk = b * Hkv + hq / a.G;
+  return bhk * a.kg.lv.pairs_per_bh + pi;
+}
+
+// ----------------------------------------------------------------------------
+// stage 1: one warp per (query problem, query cluster i) walks every key
+// cluster j of the paired key problem and forms u_ij, log W_ij, the far-field
+// key row and the far-field logit offset
+// ----------------------------------------------------------------------------
+constexpr int kS1W = 8;  // warps (query clusters) per CTA
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kS1W * 32) stage1_kernel(AttnArgs a, Stage1 s1, int qp0) {
+  constexpr int R = D / 32;
+  __shared__ float nu_s[kS1W][D];
+  __shared__ float mu_s[kS1W][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lq = blockIdx.x, qpid = qp0 + lq;
+  const int i = blockIdx.y * kS1W + warp;
+  const Prob pq = prob_of(a.qg, qpid);
+  if (i >= pq.C) return;  // warp-uniform; this kernel has no CTA-wide barrier
+  const int Cq = a.Cq, Ck = a.Ck;
+  if (a.qs.counts[(size_t)qpid * Cq + i] == 0) return;
+  const int kpid = kv_problem(a, qpid);
+  const Prob pk = prob_of(a.kg, kpid);
+  const int* kc = a.ks.counts + (size_t)kpid * Ck;
+  const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
+  const int* perm = a.ks.perm + pk.slot0;
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  float* nu = nu_s[warp];
+  float* mu = mu_s[warp];
+  for (int d = lane; d < D; d += 32) nu[d] = a.qs.cent32[((size_t)qpid * Cq + i) * D + d];
+  const float s = a.scale;
+  const int mode = a.mode;
+  const size_t ij0 = ((size_t)lq * Cq + i) * Ck;
+  for (int j = 0; j < pk.C; ++j) {
+    const int nj = kc[j];
+    const size_t ij = ij0 + j;
+    if (nj == 0) {
+      if (lane == 0) {
+        s1.logW[ij] = -INFINITY;
+        s1.fbias[ij] = -INFINITY;
+      }
+      continue;
+    }
+    __syncwarp();
+    for (int d = lane; d < D; d += 32) mu[d] = a.ks.cent32[((size_t)kpid * Ck + j) * D + d];
+    __syncwarp();
+    float accU[R], accK[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) accU[r] = accK[r] = 0.f;
+    float m = -INFINITY, z = 0.f;
+    const int off = koff[j];
+    for (int t0 = 0; t0 < nj; t0 += 32) {
+      const int cnt = imin(32, nj - t0);
+      const bool on = lane < cnt;
+      const long long row = on ? pk.row0 + perm[off + t0 + lane] : 0;
+      float w = 0.f;
+      if (mode == 0) {
+        w = on ? 1.f : 0.f;
+      } else {
+        float g = 0.f;
+        if (on) {
+          const T* kr = K + row * D;
+#pragma unroll 8
+          for (int d = 0; d < D; ++d) g = fmaf(nu[d], ld<T>(kr + d) - mu[d], g);
+        }
+        const float at = s * g;
+        if (mode == 1) {
+          w = on ? 1.f + at : 0.f;  // first-order term of exp(s nu.k~)
+        } else {
+          float cm = on ? at : -INFINITY;
+          for (int o = 16; o; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+          const float mn = fmaxf(m, cm);
+          const float rs = (m == -INFINITY) ? 0.f : expf(m - mn);
+          w = on ? expf(at - mn) : 0.f;
+          float ws = w;
+          for (int o = 16; o; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
+          z = z * rs + ws;
+          m = mn;
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            accU[r] *= rs;
+            accK[r] *= rs;
+          }
+        }
+      }
+      for (int tt = 0; tt < cnt; ++tt) {
+        const float wt = __shfl_sync(0xffffffffu, w, tt);
+        const long long rt = __shfl_sync(0xffffffffu, row, tt);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int e = lane + 32 * r;
+          accU[r] = fmaf(wt, ld<T>(V + rt * D + e), accU[r]);
+          if (mode == 2) accK[r] = fmaf(wt, ld<T>(K + rt * D + e) - mu[e], accK[r]);
+        }
+      }
+    }
+    if (mode != 2) {
+      const float inv = 1.f / (float)nj;
+#pragma unroll
+      for (int r = 0; r < R; ++r) s1.U[ij * D + lane + 32 * r] = accU[r] * inv;
+      if (lane == 0) {
+        const float lw = logf((float)nj);
+        s1.logW[ij] = lw;
+        s1.fbias[ij] = lw;
+      }
+    } else {
+      // k_hat = mu + sum w k~ / W;  offset = s nu.(mu - k_hat) + log W
+      const float inv = 1.f / z;
+      float part = 0.f;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int e = lane + 32 * r;
+        const float kh = accK[r] * inv;
+        s1.U[ij * D + e] = accU[r] * inv;
+        s1.Kf[ij * D + e] = mu[e] + kh;
+        part = fmaf(nu[e], kh, part);
+      }
+      for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if (lane == 0) {
+        const float lw = m + logf(z);
+        s1.logW[ij] = lw;
+        s1.fbias[ij] = lw - s * part;
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// selection: top-k key clusters per query cluster by s nu_i.mu_j + log W_ij,
+// ties to the lowest j, empty clusters never
+// ----------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) select_kernel(AttnArgs a, Stage1 s1, int qp0) {
+  extern __shared__ double sc_all[];  // [8][Ck]
+  const int lq = blockIdx.x, qpid = qp0 + lq;
+  const Prob pq = prob_of(a.qg, qpid);
+  const int kpid = kv_problem(a, qpid);
+  const Prob pk = prob_of(a.kg, kpid);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Cq = a.Cq, Ck = a.Ck, K1 = a.topk;
+  double* sc = sc_all + (size_t)warp * Ck;
+  const double s = (double)a.scale;
+  const int* kc = a.ks.counts + (size_t)kpid * Ck;
+  for (int i = warp; i < pq.C; i += 8) {
+    const double* nu = a.qs.cent64 + ((size_t)qpid * Cq + i) * D;
+    for (int j = lane; j < pk.C; j += 32) {
+      double v = -INFINITY;
+      if (kc[j] > 0) {
+        const double* mu = a.ks.cent64 + ((size_t)kpid * Ck + j) * D;
+        double dt = 0.0;
+        for (int d = 0; d < D; ++d) dt = __dadd_rn(dt, __dmul_rn(nu[d], mu[d]));
+        const double lw = (a.mode == 2) ? (double)s1.logW[((size_t)lq * Cq + i) * Ck + j]
+                                        : log((double)kc[j]);
+        v = __dadd_rn(__dmul_rn(s, dt), lw);
+      }
+      sc[j] = v;
+    }
+    __syncwarp();
+    int taken = 0;
+    int* out = s1.sel + ((size_t)qpid * Cq + i) * (K1 > 0 ? K1 : 1);
+    for (int r = 0; r < K1; ++r) {
+      double bv = -INFINITY;
+      int bj = -1;
+      for (int j = lane; j < pk.C; j += 32) {
+        const double v = sc[j];
+        if (kc[j] > 0 && v > -INFINITY && (bj < 0 || v > bv)) {
+          bv = v;
+          bj = j;
+        }
+      }
+      for (int o = 16; o; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+        if (oj >= 0 && (bj < 0 || ov > bv || (ov == bv && oj < bj))) {
+          bv = ov;
+          bj = oj;
+        }
+      }
+      if (bj < 0) break;
+      if (lane == 0) out[r] = bj;
+      if (lane == (bj & 31)) sc[bj] = -INFINITY;  // remove from later rounds
+      __syncwarp();
+      ++taken;
+    }
+    if (lane == 0) {
+      for (int r = taken; r < K1; ++r) out[r] = -1;
+      s1.nsel[(size_t)qpid * Cq + i] = taken;
+    }
+    __syncwarp();
+  }
+}
+
+// ----------------------------------------------------------------------------
+// stage 2: far field + exact retrieval in one online softmax
+// ----------------------------------------------------------------------------
+constexpr int kQ = 64;     // queries per pass
+constexpr int kRows = 32;  // key rows staged per step
+
+template <int D>
+struct TPQ {
+  static constexpr int v = D / 64;  // threads per query, 64 dims each
+};
+
+struct Online {
+  float m, l;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kQ * (D / 64)) stage2_kernel(AttnArgs a, Stage1 s1, int qp0) {
+  constexpr int P = D / 64;
+  __shared__ float ks_[kRows][D];
+  __shared__ float vs_[kRows][D];
+  __shared__ float bs_[kRows];
+  __shared__ unsigned char inR[kMaxC];
+  __shared__ int sel[kMaxC];
+
+  const int lq = blockIdx.x, qpid = qp0 + lq, i = blockIdx.y;
+  const Prob pq = prob_of(a.qg, qpid);
+  if (i >= pq.C) return;
+  const int Cq = a.Cq, Ck = a.Ck;
+  const int nqi = a.qs.counts[(size_t)qpid * Cq + i];
+  if (nqi == 0) return;
+  const int kpid = kv_problem(a, qpid);
+  const Prob pk = prob_of(a.kg, kpid);
+  const int tid = threadIdx.x, part = tid % P, qq = tid / P;
+  const int nsel = a.topk > 0 ? s1.nsel[(size_t)qpid * Cq + i] : 0;
+  for (int j = tid; j < pk.C; j += blockDim.x) inR[j] = 0;
+  __syncthreads();
+  for (int r = tid; r < nsel; r += blockDim.x) {
+    const int j = s1.sel[((size_t)qpid * Cq + i) * a.topk + r];
+    sel[r] = j;
+    inR[j] = 1;
+  }
+  __syncthreads();
+  const int* kc = a.ks.counts + (size_t)kpid * Ck;
+  const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
+  long long nexact = 0;
+  for (int r = 0; r < nsel; ++r) nexact += kc[sel[r]];
+
+  const T* Q = static_cast<const T*>(a.qg.X);
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  const int qo = a.qs.off[(size_t)qpid * (Cq + 1) + i];
+  const int* qperm = a.qs.perm + pq.slot0;
+  const int* kperm = a.ks.perm + pk.slot0;
+  const size_t ij0 = ((size_t)lq * Cq + i) * Ck;
+  const bool tilted = a.mode == 2;
+  const float s = a.scale;
+
+  for (int c0 = 0; c0 < nqi; c0 += kQ) {
+    const bool valid = c0 + qq < nqi;
+    const int tq = valid ? qperm[qo + c0 + qq] : 0;
+    float q[64];
+    float acc[64];
+#pragma unroll
+    for (int d = 0; d < 64; ++d) {
+      q[d] = valid ? ld<T>(Q + (pq.row0 + tq) * D + part * 64 + d) : 0.f;
+      acc[d] = 0.f;
+    }
+    float m = -INFINITY, l = 0.f;
+
+    auto consume = [&](int nrows) {
+      for (int r = 0; r < nrows; ++r) {
+        float dt = 0.f;
+#pragma unroll
+        for (int d = 0; d < 64; ++d) dt = fmaf(q[d], ks_[r][part * 64 + d], dt);
+        if (P == 2) dt += __shfl_xor_sync(0xffffffffu, dt, 1);
+        const float lg = fmaf(s, dt, bs_[r]);
+        if (lg == -INFINITY) continue;
+        if (lg > m) {
+          const float sc = (m == -INFINITY) ? 0.f : expf(m - lg);
+          l = l * sc + 1.f;
+#pragma unroll
+          for (int d = 0; d < 64; ++d) acc[d] = fmaf(acc[d], sc, vs_[r][part * 64 + d]);
+          m = lg;
+        } else {
+          const float wt = expf(lg - m);
+          l += wt;
+#pragma unroll
+          for (int d = 0; d < 64; ++d) acc[d] = fmaf(wt, vs_[r][part * 64 + d], acc[d]);
+        }
+      }
+    };
+
+    // far field
+    for (int j0 = 0; j0 < pk.C; j0 += kRows) {
+      const int nr = imin(kRows, pk.C - j0);
+      __syncthreads();
+      for (int e = tid; e < nr * D; e += blockDim.x) {
+        const int r = e / D, d = e - r * D, j = j0 + r;
+        const size_t ij = ij0 + j;
+        ks_[r][d] = tilted ? s1.Kf[ij * D + d] : a.ks.cent32[((size_t)kpid * Ck + j) * D + d];
+        vs_[r][d] = s1.U[ij * D + d];
+      }
+      for (int r = tid; r < nr; r += blockDim.x) {
+        const int j = j0 + r;
+        bs_[r] = (kc[j] == 0 || inR[j]) ? -INFINITY : s1.fbias[ij0 + j];
+      }
+      __syncthreads();
+      consume(nr);
+    }
+    // exact retrieval
+    for (int rr = 0; rr < nsel; ++rr) {
+      const int j = sel[rr], b = koff[j], n = kc[j];
+      for (int t0 = 0; t0 < n; t0 += kRows) {
+        const int nr = imin(kRows, n - t0);
+        __syncthreads();
+        for (int e = tid; e < nr * D; e += blockDim.x) {
+          const int r = e / D, d = e - r * D;
+          const long long row = pk.row0 + kperm[b + t0 + r];
+          ks_[r][d] = ld<T>(K + row * D + d);
+          vs_[r][d] = ld<T>(V + row * D + d);
+        }
+        for (int r = tid; r < nr; r += blockDim.x) bs_[r] = 0.f;
+        __syncthreads();
+        consume(nr);
+      }
+    }
+    if (valid) {
+      const long long row = pq.row0 + tq;
+      const float inv = 1.f / l;
+      if (a.O != nullptr) {
+        T* O = static_cast<T*>(a.O);
+#pragma unroll
+        for (int d = 0; d < 64; ++d) st<T>(O + row * D + part * 64 + d, acc[d] * inv);
+      } else {
+        float* pp = a.part + (size_t)(pq.slot0 + tq) * (D + 1);
+#pragma unroll
+        for (int d = 0; d < 64; ++d) pp[part * 64 + d] = acc[d] * inv;
+        if (part == 0) pp[D] = m + logf(l);
+      }
+      if (a.n_exact != nullptr && part == 0) {
+        if (a.O != nullptr)
+          a.n_exact[row] = nexact;
+        else
+          atomicAdd(reinterpret_cast<unsigned long long*>(a.n_exact + row),
+                    (unsigned long long)nexact);
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// causal: exact local block, then merge the level partials (each partial is
+// the softmax of its terms, entering as one term with logit lse and value o)
+// ----------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kQ * (D / 64)) local_merge_kernel(AttnArgs a, int L) {
+  constexpr int P = D / 64;
+  __shared__ float ks_[kRows][D];
+  __shared__ float vs_[kRows][D];
+  const int bhq = blockIdx.x;
+  const int N = a.qg.lv.N;
+  const int tid = threadIdx.x, part = tid % P, qq = tid / P;
+  const int q0 = blockIdx.y * kQ;
+  const int qpos = q0 + qq;
+  const bool valid = qpos < N;
+  const int Hq = a.qg.BH / a.B, Hkv = a.kg.BH / a.B;
+  const int b = bhq / Hq, hq = bhq - b * Hq;
+  const int bhk = b * Hkv + hq / a.G;
+  const T* Q = static_cast<const T*>(a.qg.X);
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  const long long qrow = (long long)bhq * N + qpos;
+  const long long krow0 = (long long)bhk * N;
+  float q[64], acc[64];
+#pragma unroll
+  for (int d = 0; d < 64; ++d) {
+    q[d] = valid ? ld<T>(Q + qrow * D + part * 64 + d) : 0.f;
+    acc[d] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  const float s = a.scale;
+  const int blk = qpos / L;
+  const int kbeg = (q0 / L) * L;
+  const int kend = imin(q0 + kQ, N);  // exclusive
+  for (int t0 = kbeg; t0 < kend; t0 += kRows) {
+    const int nr = imin(kRows, kend - t0);
+    __syncthreads();
+    for (int e = tid; e < nr * D; e += blockDim.x) {
+      const int r = e / D, d = e - r * D;
+      ks_[r][d] = ld<T>(K + (krow0 + t0 + r) * D + d);
+      vs_[r][d] = ld<T>(V + (krow0 + t0 + r) * D + d);
+    }
+    __syncthreads();
+    for (int r = 0; r < nr; ++r) {
+      const int t = t0 + r;
+      float dt = 0.f;
+#pragma unroll
+      for (int d = 0; d < 64; ++d) dt = fmaf(q[d], ks_[r][part * 64 + d], dt);
+      if (P == 2) dt += __shfl_xor_sync(0xffffffffu, dt, 1);
+      if (!valid || t > qpos || t < blk * L) continue;
+      const float lg = s * dt;
+      if (lg > m) {
+        const float sc = (m == -INFINITY) ? 0.f : expf(m - lg);
+        l = l * sc + 1.f;
+#pragma unroll
+        for (int d = 0; d < 64; ++d) acc[d] = fmaf(acc[d], sc, vs_[r][part * 64 + d]);
+        m = lg;
+      } else {
+        const float wt = expf(lg - m);
+        l += wt;
+#pragma unroll
+        for (int d = 0; d < 64; ++d) acc[d] = fmaf(wt, vs_[r][part * 64 + d], acc[d]);
+      }
+    }
+  }
+  if (!valid) return;
+  const int levels = a.qg.lv.nlev;
+  for (int lv = 0; lv < levels; ++lv) {
+    if (!((blk >> lv) & 1)) continue;
+    const int sz = L << lv, p = blk >> (lv + 1);
+    const long long slot = (long long)bhq * a.qg.lv.toks_per_bh + a.qg.lv.tok_base[lv] +
+                           (long long)p * sz + (qpos - (2 * p + 1) * sz);
+    const float* pp = a.part + slot * (D + 1);
+    const float lg = pp[D];
+    if (lg > m) {
+      const float sc = (m == -INFINITY) ? 0.f : expf(m - lg);
+      l = l * sc + 1.f;
+#pragma unroll
+      for (int d = 0; d < 64; ++d) acc[d] = fmaf(acc[d], sc, pp[part * 64 + d]);
+      m = lg;
+    } else {
+      const float wt = expf(lg - m);
+      l += wt;
+#pragma unroll
+      for (int d = 0; d < 64; ++d) acc[d] = fmaf(wt, pp[part * 64 + d], acc[d]);
+    }
+  }
+  T* O = static_cast<T*>(a.O);
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int d = 0; d < 64; ++d) st<T>(O + qrow * D + part * 64 + d, acc[d] * inv);
+  if (a.n_exact != nullptr && part == 0)
+    atomicAdd(reinterpret_cast<unsigned long long*>(a.n_exact + qrow),
+              (unsigned long long)(qpos - blk * L + 1));
+}
+
+// ----------------------------------------------------------------------------
+// launchers
+// ----------------------------------------------------------------------------
+template <typename T, int D>
+static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         8 * kMaxC * (int)sizeof(double));
+    attr = true;
+  }
+  stage1_kernel<T, D><<<dim3(nqp, cdiv(a.Cq, kS1W)), kS1W * 32, 0, st>>>(a, s1, qp0);
+  if (a.topk > 0) {
+    const size_t smem = (size_t)8 * a.Ck * sizeof(double);
+    select_kernel<D><<<nqp, 256, smem, st>>>(a, s1, qp0);
+  }
+  stage2_kernel<T, D><<<dim3(nqp, a.Cq), kQ * (D / 64), 0, st>>>(a, s1, qp0);
+}
+
+void run_blocks(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st) {
+  const int D = a.qg.D;
+  if (a.qg.dtype == 0) {
+    if (D == 64) blocks_t<__nv_bfloat16, 64>(a, s1, qp0, nqp, st);
+    else blocks_t<__nv_bfloat16, 128>(a, s1, qp0, nqp, st);
+  } else {
+    if (D == 64) blocks_t<float, 64>(a, s1, qp0, nqp, st);
+    else blocks_t<float, 128>(a, s1, qp0, nqp, st);
+  }
+}
+
+void run_local_merge(const AttnArgs& a, int L, cudaStream_t st) {
+  const int D = a.qg.D, N = a.qg.lv.N;
+  dim3 grid(a.qg.BH, cdiv(N, kQ));
+  const int thr = kQ * (D / 64);
+  if (a.qg.dtype == 0) {
+    if (D == 64) local_merge_kernel<__nv_bfloat16, 64><<<grid, thr, 0, st>>>(a, L);
+    else local_merge_kernel<__nv_bfloat16, 128><<<grid, thr, 0, st>>>(a, L);
+  } else {
+    if (D == 64) local_merge_kernel<float, 64><<<grid, thr, 0, st>>>(a, L);
+    else local_merge_kernel<float, 128><<<grid, thr, 0, st>>>(a, L);
+  }
+}
+
+}  // namespace muse

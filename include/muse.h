@@ -1,0 +1,180 @@
+/*
+ * libmuse -- B200 (sm_100a) implementation of the forward operator of
+ * Multipole Semantic Attention (MuSe).
+ *
+ * Sources.  All cited pages carry the title "Multipole Semantic Attention:
+ * A Fast Approximation of Softmax Attention for Pretraining":
+ *   [G]  the gist.science page, section "Technical Summary" -> "Methodology"
+ *        -> "Core Mechanisms" (bidirectional clustering, residual
+ *        decomposition, stage 1 / stage 2, exponential tilting, retrieval);
+ *   [A1] the newx.sg page, section "Abstract" (monopole + dipole
+ *        corrections, hierarchical block decomposition for causal attention,
+ *        O(NCD) acausal and O(NCD log N) causal cost).
+ *
+ * Conventions shared by every entry point.
+ *   - All tensor arguments are DEVICE pointers to contiguous row-major data;
+ *     the caller owns every buffer, including the workspace.  The library
+ *     never allocates, frees or synchronises: all work is enqueued on the
+ *     given stream and the call returns before it finishes.
+ *   - Q is [B,Hq,N,D]; K and V are [B,Hkv,N,D]; O has Q's shape and dtype.
+ *     q-head h reads kv-head h / (Hq/Hkv) (grouped-query attention).
+ *   - Arguments are validated before anything is launched; a failing check
+ *     returns MUSE_ERR_INVALID_ARG (or MUSE_ERR_UNSUPPORTED for shapes the
+ *     kernels do not cover, or MUSE_ERR_WORKSPACE for a short workspace) and
+ *     leaves every output untouched.  A launch error reported by the CUDA
+ *     runtime returns MUSE_ERR_CUDA.  muse_last_error() then gives a message
+ *     (per host thread).
+ *   - Calls with distinct workspaces and outputs may run concurrently.
+ */
+#ifndef MUSE_H_
+#define MUSE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MUSE_OK = 0,
+  MUSE_ERR_INVALID_ARG = 1,
+  MUSE_ERR_UNSUPPORTED = 2,
+  MUSE_ERR_WORKSPACE = 3,
+  MUSE_ERR_CUDA = 4,
+  MUSE_ERR_DEVICE_CHECK = 5
+} muse_status;
+
+typedef enum { MUSE_BF16 = 0, MUSE_F32 = 1 } muse_dtype;
+
+/* Far-field summary of a key cluster j as seen from query cluster i:
+ *   MONOPOLE  count, centroid and summed values ([A1] Abstract; [G] Core
+ *             Mechanisms, retrieval item: "monopole (centroid)");
+ *   DIPOLE    MONOPOLE plus the first-order correction (s/n_j) M_j nu_i with
+ *             M_j = sum_{t in j} v_t (k_t - mu_j)^T ([A1] Abstract);
+ *   TILTED    exponentially tilted summaries weighted by exp(s nu_i . k_t)
+ *             ([G] Core Mechanisms, "Exponential Tilting"). */
+typedef enum { MUSE_MONOPOLE = 0, MUSE_DIPOLE = 1, MUSE_TILTED = 2 } muse_mode;
+
+typedef struct {
+  int B, Hq, Hkv, N, D; /* D in {64, 128}; Hq % Hkv == 0 */
+  muse_dtype dtype;     /* of Q, K, V and O */
+} muse_shape;
+
+typedef struct {
+  int Cq, Ck;      /* query and key clusters (causal: both = C per level) */
+  int iters;       /* Lloyd iterations, >= 1 */
+  uint64_t seed;   /* seeds the k-means start rows */
+  int topk;        /* k1: key clusters retrieved exactly per query cluster */
+  int block;       /* causal local block L (ignored by muse_attn_fwd) */
+  float scale;     /* softmax scale s: logits are s q.k */
+  muse_mode mode;
+} muse_params;
+
+/* Optional device outputs for inspection; any member may be NULL.
+ * Acausal layouts: q_assign [B,Hq,N], k_assign [B,Hkv,N],
+ *   q_centroids [B,Hq,Cq,D], k_centroids [B,Hkv,Ck,D], k_counts [B,Hkv,Ck],
+ *   selected [B,Hq,Cq,topk] (rank order, -1 padded), n_exact [B,Hq,N].
+ * Causal layouts: q_assign [B,Hq,levels,N/2], k_assign [B,Hkv,levels,N/2]
+ *   (entry (l, p*s + r) is token r of pair p's block at level l, s = L 2^l),
+ *   n_exact [B,Hq,N]; the centroid, count and selection members are not
+ *   written by the causal entry point. */
+typedef struct {
+  int32_t *q_assign, *k_assign, *selected, *k_counts;
+  float *q_centroids, *k_centroids;
+  int64_t *n_exact;
+} muse_debug;
+
+/* Workspace bytes muse_attn_fwd (causal == 0) or muse_attn_fwd_causal
+ * (causal != 0) needs for this shape and these parameters; 0 if the
+ * arguments are invalid. */
+size_t muse_workspace_size(const muse_shape *shape, const muse_params *params,
+                           int causal);
+
+/* Workspace bytes of muse_cluster / muse_summarize for these sizes. */
+size_t muse_cluster_workspace_size(int B, int H, int N, int D, int C);
+
+/*
+ * Lloyd k-means of every (b, h) row set of X [B,H,N,D] into C clusters
+ * ([G] Core Mechanisms, "Bidirectional Semantic Clustering"; the algorithm
+ * is not named on the pages -- Lloyd with squared Euclidean distance is the
+ * reading taken here).
+ *   iters        >= 1 rounds of (assign, update).  Ties in the assignment
+ *                go to the lowest cluster index; an empty cluster keeps its
+ *                previous centroid.
+ *   init         NULL: start from C distinct rows chosen by a partial
+ *                Fisher-Yates shuffle driven by splitmix64 seeded with
+ *                seed + 0x9E3779B97F4A7C15 * (2 (b H + h) + role + 1);
+ *                else fp32 start centroids [B,H,C,D].
+ *   role         0 = key stream, 1 = query stream (selects the seed stream;
+ *                muse_attn_fwd clusters keys with role 0 and queries with
+ *                role 1).
+ *   assign       out [B,H,N] int32: cluster of each row after the last round.
+ *   centroids    out [B,H,C,D] fp32: centroids after the last update.
+ *   counts       out [B,H,C] int32 (may be NULL).
+ * 1 <= C <= min(N, 1024); D in {64, 128}.
+ */
+muse_status muse_cluster(const void *X, muse_dtype dtype, int B, int H, int N,
+                         int D, int C, int iters, uint64_t seed, int role,
+                         const float *init, int32_t *assign, float *centroids,
+                         int32_t *counts, void *ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/*
+ * Key-cluster summaries for a given assignment ([A1] Abstract: monopole and
+ * dipole): counts n_j, centroid mu_j (mean of members; zero when empty),
+ * S_j = sum_{t in j} v_t and M_j[e][d] = sum_{t in j} v_t[e] (k_t[d] - mu_j[d]).
+ *   assign  [B,H,N] int32 in [0, C).
+ *   counts [B,H,C] int32, mu [B,H,C,D] f32, S [B,H,C,D] f32,
+ *   M [B,H,C,D,D] f32 (M may be NULL).
+ */
+muse_status muse_summarize(const void *K, const void *V, muse_dtype dtype,
+                           int B, int H, int N, int D, int C,
+                           const int32_t *assign, int32_t *counts, float *mu,
+                           float *S, float *M, void *ws, size_t ws_bytes,
+                           cudaStream_t stream);
+
+/*
+ * Acausal MuSe forward ([G] Core Mechanisms; [A1] Abstract, O(NCD) form).
+ * Per (b, kv-head) the keys are clustered (Ck) and summarised; per q-head the
+ * queries are clustered (Cq).  Stage 1 scores every key cluster j from every
+ * query cluster i, s_ij = s nu_i.mu_j + log W_ij, and retrieves the top
+ * `topk` (ties to the lowest j, empty clusters never).  Stage 2 gives each
+ * query one far-field term per other non-empty cluster (logit
+ * s q.mu_j + log W_ij, or for TILTED s (q - nu_i).k_hat_ij + s nu_i.mu_j +
+ * log W_ij; value u_ij) plus one exact term per key of the retrieved
+ * clusters, all in one softmax.  O is written in the input dtype.
+ * Requires 1 <= Cq, Ck <= min(N, 1024), 0 <= topk <= Ck, iters >= 1.
+ */
+muse_status muse_attn_fwd(const void *Q, const void *K, const void *V, void *O,
+                          const muse_shape *shape, const muse_params *params,
+                          muse_debug *debug, void *ws, size_t ws_bytes,
+                          cudaStream_t stream);
+
+/*
+ * Causal MuSe forward by the hierarchical block decomposition ([A1]
+ * Abstract).  With L = params->block (N % L == 0, N/L a power of two), the
+ * query at position q in block b = q / L attends exactly to the keys
+ * [bL, q] of its own block, and for every level l whose bit is set in b to
+ * the key block [2p s, (2p+1) s) (s = L 2^l, p = b >> (l+1)) through one MuSe
+ * block problem clustered inside that key block and the query block
+ * [(2p+1) s, (2p+2) s) with C_eff = min(Ck, s) clusters; topk is a per-block
+ * problem budget.  All terms meet in one softmax.  Requires Cq == Ck.
+ */
+muse_status muse_attn_fwd_causal(const void *Q, const void *K, const void *V,
+                                 void *O, const muse_shape *shape,
+                                 const muse_params *params, muse_debug *debug,
+                                 void *ws, size_t ws_bytes, cudaStream_t stream);
+
+const char *muse_status_string(muse_status status);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char *muse_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUSE_H_ */

@@ -1,0 +1,94 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/muse.h declares, sizes workspaces, and rejects bad
+arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import clustered_multipole_approximation_b200 as muse
+from clustered_multipole_approximation_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return muse.load_library()
+
+
+def declared_symbols():
+    syms = set()
+    for name in os.listdir(os.path.join(ROOT, "include")):
+        if name.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", name)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            syms |= set(re.findall(r"\b(muse_[a-z0-9_]+)\s*\(", txt))
+    return syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    syms = declared_symbols()
+    assert {"muse_cluster", "muse_summarize", "muse_attn_fwd", "muse_attn_fwd_causal"} <= syms
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(muse.EXPORTS) <= syms
+
+
+def shape(B=1, Hq=2, Hkv=1, N=1024, D=64, dt=0):
+    return muse.muse_shape(B, Hq, Hkv, N, D, dt)
+
+
+def params(Cq=16, Ck=16, iters=3, topk=2, block=0, mode=1):
+    return muse.muse_params(Cq, Ck, iters, 1, topk, block, 1.0, mode)
+
+
+def test_workspace_size_valid_and_invalid(lib):
+    ws = lib.muse_workspace_size(ctypes.byref(shape()), ctypes.byref(params()), 0)
+    assert ws > 0
+    wsc = lib.muse_workspace_size(ctypes.byref(shape()), ctypes.byref(params(block=128)), 1)
+    assert wsc > 0
+    bad = [(shape(D=96), params(), 0), (shape(Hq=3, Hkv=2), params(), 0),
+           (shape(), params(Cq=0), 0), (shape(), params(Ck=2000), 0),
+           (shape(N=100), params(Cq=101, Ck=5), 0), (shape(), params(topk=17), 0),
+           (shape(), params(iters=0), 0), (shape(), params(mode=7), 0),
+           (shape(), params(block=100), 1), (shape(N=768), params(block=128), 1),
+           (shape(), params(Cq=8, Ck=16, block=128), 1)]
+    for sh, pr, c in bad:
+        assert lib.muse_workspace_size(ctypes.byref(sh), ctypes.byref(pr), c) == 0
+    assert lib.muse_cluster_workspace_size(1, 2, 1000, 64, 10) > 0
+    assert lib.muse_cluster_workspace_size(1, 2, 1000, 80, 10) == 0
+
+
+def test_invalid_arguments_return_errors_without_launch(lib):
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+    sh, pr = shape(), params()
+    st = lib.muse_attn_fwd(None, fake, fake, fake, ctypes.byref(sh), ctypes.byref(pr), None,
+                           fake, 1 << 30, None)
+    assert st == 1 and b"NULL" in lib.muse_last_error()
+    st = lib.muse_attn_fwd(fake, fake, fake, fake, ctypes.byref(shape(D=80)), ctypes.byref(pr),
+                           None, fake, 1 << 30, None)
+    assert st == 2
+    st = lib.muse_attn_fwd(fake, fake, fake, fake, ctypes.byref(sh), ctypes.byref(pr), None,
+                           fake, 16, None)
+    assert st == 3 and b"workspace" in lib.muse_last_error()
+    st = lib.muse_attn_fwd_causal(fake, fake, fake, fake, ctypes.byref(sh),
+                                  ctypes.byref(params(block=100)), None, fake, 1 << 30, None)
+    assert st == 1
+    st = lib.muse_cluster(fake, 0, 1, 1, 100, 64, 200, 3, 0, 0, None, fake, fake, None, fake,
+                          1 << 30, None)
+    assert st == 1
+    st = lib.muse_cluster(fake, 0, 1, 1, 100, 64, 10, 3, 0, 2, None, fake, fake, None, fake,
+                          1 << 30, None)
+    assert st == 1
+    st = lib.muse_summarize(fake, fake, 0, 1, 1, 100, 48, 10, fake, fake, fake, fake, None, None,
+                            0, None)
+    assert st == 2
+    assert lib.muse_status_string(3) == b"workspace too small"
+
+
+def test_product_path_fails_loudly_without_library(tmp_path):
+    with pytest.raises(ImportError):
+        muse.load_library(str(tmp_path / "missing.so"))

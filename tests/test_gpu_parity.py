@@ -1,0 +1,278 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Assignments, cluster counts, retrieval sets and exact-key counts must match
+bit for bit (a k-means mismatch is tolerated only as a documented near tie);
+outputs must match within 1e-5 (fp32 inputs) or 2e-3 (bf16 inputs) max-abs,
+and the relative squared error against exact attention within 1e-3 of the
+oracle's.
+"""
+import numpy as np
+import pytest
+import torch
+
+import clustered_multipole_approximation_b200 as muse
+import oracle
+from clustered_multipole_approximation_b200 import build
+from clustered_multipole_approximation_b200.inputs import WORKLOADS, clustered_qkv, make_inputs
+from helpers import TOL, assert_assign_match, assert_close, rse, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+    muse.load_library()
+
+
+def gpu_acausal(Q, K, V, dtype, C, iters, seed, topk, scale=1.0, mode="dipole", Cq=None):
+    q, k, v = to_dev(Q, dtype), to_dev(K, dtype), to_dev(V, dtype)
+    O, dbg = muse.muse_attn_fwd(q, k, v, Cq=Cq or C, Ck=C, iters=iters, seed=seed, topk=topk,
+                                scale=scale, mode=mode, debug=True)
+    torch.cuda.synchronize()
+    return O.float().cpu().numpy(), {n: t.cpu().numpy() for n, t in dbg.items()}
+
+
+def check_acausal(Q, K, V, dtype, C, iters, seed, topk, scale=1.0, mode="dipole", heads=None,
+                  Cq=None, check_rse=True):
+    B, Hq = Q.shape[:2]
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    O, g = gpu_acausal(Q, K, V, dtype, C, iters, seed, topk, scale, mode, Cq)
+    mask = None
+    if heads is not None:
+        mask = np.zeros((B, Hq), np.uint8)
+        for b, h in heads:
+            mask[b, h] = 1
+    r = oracle.muse_acausal(Q, K, V, Cq or C, C, iters, seed, topk, scale, mode, hq_mask=mask)
+    sel_heads = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else heads
+    for b, h in sel_heads:
+        hk = h // G
+        assert_assign_match(g["k_assign"][b, hk], r["k_assign"][b, hk], what=f"k_assign b{b}h{hk}")
+        assert_assign_match(g["q_assign"][b, h], r["q_assign"][b, h], what=f"q_assign b{b}h{h}")
+        assert (g["k_counts"][b, hk] == r["k_count"][b, hk]).all()
+        np.testing.assert_allclose(g["k_centroids"][b, hk], r["k_cent"][b, hk], rtol=2e-7, atol=1e-7)
+        np.testing.assert_allclose(g["q_centroids"][b, h], r["q_cent"][b, h], rtol=2e-7, atol=1e-7)
+        if topk > 0:
+            qc = np.bincount(r["q_assign"][b, h], minlength=Cq or C)
+            live = qc > 0  # rows of empty query clusters are never used
+            assert (g["selected"][b, h][live] == r["selected"][b, h][live]).all(), f"R b{b}h{h}"
+        assert (g["n_exact"][b, h] == r["n_exact"][b, h]).all()
+        assert_close(O[b, h], r["O"][b, h], TOL[dtype], f"O b{b}h{h}")
+    if check_rse:
+        E = oracle.exact_attention(Q, K, V, scale, hq_mask=mask)
+        idx = tuple(np.array(sel_heads).T)
+        r_gpu = rse(O[idx], E[idx])
+        r_orc = rse(r["O"][idx], E[idx])
+        assert abs(r_gpu - r_orc) < 1e-3, (r_gpu, r_orc)
+    return O, g, r
+
+
+# ---------------------------------------------------------------------------
+# acausal
+# ---------------------------------------------------------------------------
+def test_workload_acausal_f32_n1k():
+    w = WORKLOADS["acausal-f32-n1k"]
+    Q, K, V = make_inputs(w)
+    check_acausal(Q, K, V, w.dtype, w.C, w.iters, w.cluster_seed, w.topk, w.scale, w.mode)
+
+
+@pytest.mark.parametrize("mode", ["dipole", "monopole"])
+def test_workload_acausal_bf16_h8_n8k(mode):
+    w = WORKLOADS["acausal-bf16-h8-n8k"]
+    Q, K, V = make_inputs(w)
+    check_acausal(Q, K, V, w.dtype, w.C, w.iters, w.cluster_seed, w.topk, w.scale, mode,
+                  heads=[(0, 0), (0, 5)])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+def test_small_acausal_gqa_ragged(dtype, D, mode):
+    Q, K, V = clustered_qkv(2, 4, 2, 1000, D, 12, 0.3, 0.0, dtype, 31 + D)
+    check_acausal(Q, K, V, dtype, 13, 5, 77, 3, 1.0, mode, Cq=11)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_singleton_key_clusters_match_exact_attention(dtype):
+    Q, K, V = clustered_qkv(1, 2, 1, 256, 64, 8, 0.3, 0.0, dtype, 5)
+    O, _, _ = check_acausal(Q, K, V, dtype, 256, 2, 3, 0, 1.0, "dipole", Cq=16)
+    E = oracle.exact_attention(Q, K, V)
+    assert_close(O, E, TOL[dtype], "O vs exact")
+
+
+def test_retrieving_all_clusters_is_exact():
+    Q, K, V = clustered_qkv(1, 1, 1, 512, 64, 8, 0.3, 0.0, "f32", 6)
+    O, _, _ = check_acausal(Q, K, V, "f32", 8, 4, 9, 8)
+    assert_close(O, oracle.exact_attention(Q, K, V), 1e-5, "O vs exact")
+
+
+def test_duplicate_tokens_and_empty_clusters():
+    rng = np.random.default_rng(0)
+    base = rng.standard_normal((5, 64)).astype(np.float32) * 0.4
+    Q = base[rng.integers(0, 5, (1, 1, 300))].astype(np.float32)
+    K = base[rng.integers(0, 5, (1, 1, 300))].astype(np.float32)
+    V = rng.standard_normal((1, 1, 300, 64)).astype(np.float32)
+    # 9 clusters over 5 distinct points: several clusters end up empty
+    _, g, r = check_acausal(Q, K, V, "f32", 9, 3, 4, 2, check_rse=False)
+    assert (r["k_count"] == 0).any()
+
+
+def test_single_cluster_and_topk_zero():
+    Q, K, V = clustered_qkv(1, 1, 1, 300, 64, 4, 0.3, 0.0, "bf16", 8)
+    check_acausal(Q, K, V, "bf16", 1, 2, 1, 0, 1.0, "dipole", Cq=1)
+
+
+def test_repeatable_bit_for_bit():
+    Q, K, V = clustered_qkv(1, 2, 2, 2048, 64, 16, 0.3, 0.0, "bf16", 12)
+    a, _ = gpu_acausal(Q, K, V, "bf16", 32, 5, 3, 4)
+    b, _ = gpu_acausal(Q, K, V, "bf16", 32, 5, 3, 4)
+    assert (a == b).all()
+
+
+# ---------------------------------------------------------------------------
+# clustering and summaries on their own
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_muse_cluster_seeded(dtype):
+    X, _, _ = clustered_qkv(2, 3, 3, 777, 64, 10, 0.3, 0.0, dtype, 40)
+    x = to_dev(X, dtype)
+    for role in (0, 1):
+        a, c, n = muse.muse_cluster(x, 12, 6, 1234, role=role)
+        a, c, n = a.cpu().numpy(), c.cpu().numpy(), n.cpu().numpy()
+        for b in range(2):
+            for h in range(3):
+                ra, rc, rn, _ = oracle.kmeans(X[b, h], 12, 6, 1234, b * 3 + h, role)
+                assert_assign_match(a[b, h], ra, what=f"assign b{b}h{h}")
+                assert (n[b, h] == rn).all()
+                np.testing.assert_allclose(c[b, h], rc, rtol=2e-7, atol=1e-7)
+
+
+def test_muse_cluster_one_round_from_given_centroids():
+    X, _, _ = clustered_qkv(1, 2, 2, 1500, 128, 20, 0.3, 0.0, "bf16", 41)
+    rng = np.random.default_rng(1)
+    init = rng.standard_normal((1, 2, 24, 128)).astype(np.float32) * 0.3
+    a, c, n = muse.muse_cluster(to_dev(X, "bf16"), 24, 1, 0, init=torch.from_numpy(init).cuda())
+    for h in range(2):
+        ra, _ = oracle.kmeans_assign(X[0, h], init[0, h])
+        rc, rn = oracle.kmeans_update(X[0, h], ra, init[0, h])
+        assert_assign_match(a[0, h].cpu().numpy(), ra, X[0, h].astype(np.float64),
+                            init[0, h].astype(np.float64))
+        np.testing.assert_allclose(c[0, h].cpu().numpy(), rc, rtol=2e-7, atol=1e-7)
+
+
+def test_muse_summarize():
+    K, _, V = clustered_qkv(1, 2, 2, 600, 64, 6, 0.3, 0.0, "f32", 42)
+    rng = np.random.default_rng(3)
+    assign = rng.integers(0, 7, (1, 2, 600)).astype(np.int32)
+    assign[0, 1][assign[0, 1] == 3] = 4  # cluster 3 empty in head 1
+    cnt, mu, S, M = muse.muse_summarize(to_dev(K, "f32"), to_dev(V, "f32"),
+                                        torch.from_numpy(assign).cuda(), 7)
+    for h in range(2):
+        rmu, rn = oracle.kmeans_update(K[0, h], assign[0, h], np.zeros((7, 64)))
+        rS, rM = oracle.summaries(K[0, h], V[0, h], 7, assign[0, h], rmu)
+        assert (cnt[0, h].cpu().numpy() == rn).all()
+        np.testing.assert_allclose(mu[0, h].cpu().numpy(), rmu, rtol=1e-6, atol=1e-6)
+        np.testing.assert_allclose(S[0, h].cpu().numpy(), rS, rtol=1e-5, atol=1e-4)
+        np.testing.assert_allclose(M[0, h].cpu().numpy(), rM, rtol=1e-4, atol=1e-4)
+
+
+# ---------------------------------------------------------------------------
+# causal
+# ---------------------------------------------------------------------------
+def gpu_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale=1.0, mode="dipole"):
+    q, k, v = to_dev(Q, dtype), to_dev(K, dtype), to_dev(V, dtype)
+    O, dbg = muse.muse_attn_fwd_causal(q, k, v, C=C, block=L, iters=iters, seed=seed, topk=topk,
+                                       scale=scale, mode=mode, debug=True)
+    torch.cuda.synchronize()
+    return O.float().cpu().numpy(), {n: t.cpu().numpy() for n, t in dbg.items()}
+
+
+def check_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale=1.0, mode="dipole", heads=None):
+    B, Hq = Q.shape[:2]
+    G = Hq // K.shape[1]
+    O, g = gpu_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale, mode)
+    mask = None
+    if heads is not None:
+        mask = np.zeros((B, Hq), np.uint8)
+        for b, h in heads:
+            mask[b, h] = 1
+    r = oracle.muse_causal(Q, K, V, L, C, iters, seed, topk, scale, mode, hq_mask=mask)
+    sel = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else heads
+    for b, h in sel:
+        assert_assign_match(g["k_assign"][b, h // G], r["k_assign"][b, h // G], what="k_assign")
+        assert_assign_match(g["q_assign"][b, h], r["q_assign"][b, h], what="q_assign")
+        assert (g["n_exact"][b, h] == r["n_exact"][b, h]).all()
+        assert_close(O[b, h], r["O"][b, h], TOL[dtype], f"O b{b}h{h}")
+    E = oracle.exact_attention(Q, K, V, scale, causal=True, hq_mask=mask)
+    idx = tuple(np.array(sel).T)
+    assert abs(rse(O[idx], E[idx]) - rse(r["O"][idx], E[idx])) < 1e-3
+    return O, g, r
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+def test_small_causal_gqa(dtype, mode):
+    Q, K, V = clustered_qkv(1, 4, 2, 1024, 64, 8, 0.3, 0.0, dtype, 50)
+    check_causal(Q, K, V, dtype, 64, 12, 4, 21, 2, 1.0, mode)
+
+
+def test_causal_d128_clusters_above_block_size():
+    # C = 96 > L = 64: level 0 uses singleton clusters (C_eff = 64)
+    Q, K, V = clustered_qkv(2, 2, 2, 512, 128, 8, 0.3, 0.0, "bf16", 51)
+    check_causal(Q, K, V, "bf16", 64, 96, 3, 2, 4)
+
+
+def test_causal_single_block_is_exact():
+    Q, K, V = clustered_qkv(1, 2, 1, 256, 64, 8, 0.3, 0.0, "f32", 52)
+    O, _ = gpu_causal(Q, K, V, "f32", 256, 8, 3, 1, 2)
+    assert_close(O, oracle.exact_attention(Q, K, V, causal=True), 1e-5, "O vs exact causal")
+
+
+def test_causal_never_reads_the_future_on_gpu():
+    Q, K, V = clustered_qkv(1, 2, 1, 1024, 64, 8, 0.3, 0.0, "bf16", 53)
+    base, _ = gpu_causal(Q, K, V, "bf16", 128, 16, 4, 7, 2)
+    for t0 in (0, 127, 128, 500, 1000):
+        K2, V2 = K.copy(), V.copy()
+        K2[:, :, t0 + 1:] *= -1.5
+        V2[:, :, t0 + 1:] += 1.0
+        o, _ = gpu_causal(Q, K2, V2, "bf16", 128, 16, 4, 7, 2)
+        assert (o[:, :, : t0 + 1] == base[:, :, : t0 + 1]).all(), t0
+
+
+def test_workload_causal_b2h8_n16k():
+    w = WORKLOADS["causal-bf16-b2h8-n16k"]
+    Q, K, V = make_inputs(w)
+    check_causal(Q, K, V, w.dtype, w.block, w.C, w.iters, w.cluster_seed, w.topk, w.scale,
+                 w.mode, heads=[(0, 0), (1, 7)])
+
+
+@pytest.mark.parametrize("name", ["causal-gqa32x8-n64k-d64", "causal-gqa32x8-n32k-d128"])
+def test_workload_causal_gqa_full_size_sampled(name):
+    """Full-size GQA causal workloads: sampled k-means problems against the
+    oracle's k-means, then the oracle fed the GPU's clusterings
+    (teacher-forced) on one q-head, compared output by output."""
+    w = WORKLOADS[name]
+    Q, K, V = make_inputs(w)
+    O, g = gpu_causal(Q, K, V, w.dtype, w.block, w.C, w.iters, w.cluster_seed, w.topk, w.scale,
+                      w.mode)
+    assert np.isfinite(O).all()
+    N, L = w.N, w.block
+    levels = oracle.causal_levels(N, L)
+    pmax = (N // L) // 2
+    for lv, p in [(0, 3), (2, 1), (levels - 1, 0)]:
+        s = L << lv
+        Ce = min(w.C, s)
+        slot = slice(lv * (N // 2) + p * s, lv * (N // 2) + (p + 1) * s)
+        ka, _, _, _ = oracle.kmeans(K[0, 0, 2 * p * s:(2 * p + 1) * s], Ce, w.iters,
+                                    w.cluster_seed, (0 * levels + lv) * pmax + p, 0)
+        assert_assign_match(g["k_assign"][0, 0].reshape(-1)[slot], ka, what=f"k lv{lv} p{p}")
+        qa, _, _, _ = oracle.kmeans(Q[0, 0, (2 * p + 1) * s:(2 * p + 2) * s], Ce, w.iters,
+                                    w.cluster_seed, (0 * levels + lv) * pmax + p, 1)
+        assert_assign_match(g["q_assign"][0, 0].reshape(-1)[slot], qa, what=f"q lv{lv} p{p}")
+    mask = np.zeros((1, w.Hq), np.uint8)
+    mask[0, 0] = 1
+    r = oracle.muse_causal(Q, K, V, L, w.C, w.iters, w.cluster_seed, w.topk, w.scale, w.mode,
+                           hq_mask=mask, q_assign_in=g["q_assign"], k_assign_in=g["k_assign"])
+    assert (g["n_exact"][0, 0] == r["n_exact"][0, 0]).all()
+    assert_close(O[0, 0], r["O"][0, 0], TOL[w.dtype], "O head 0")
