@@ -36,7 +36,8 @@ class MuseError(RuntimeError):
 
 class muse_shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
-                ("N", ctypes.c_int), ("D", ctypes.c_int), ("dtype", ctypes.c_int)]
+                ("N", ctypes.c_int), ("D", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("out_f32", ctypes.c_int)]
 
 
 class muse_params(ctypes.Structure):
@@ -49,11 +50,12 @@ class muse_debug(ctypes.Structure):
     _fields_ = [("q_assign", ctypes.c_void_p), ("k_assign", ctypes.c_void_p),
                 ("selected", ctypes.c_void_p), ("k_counts", ctypes.c_void_p),
                 ("q_centroids", ctypes.c_void_p), ("k_centroids", ctypes.c_void_p),
-                ("n_exact", ctypes.c_void_p)]
+                ("n_exact", ctypes.c_void_p), ("device_error", ctypes.c_void_p)]
 
 
 EXPORTS = ["muse_workspace_size", "muse_cluster_workspace_size", "muse_cluster", "muse_summarize",
-           "muse_attn_fwd", "muse_attn_fwd_causal", "muse_status_string", "muse_last_error"]
+           "muse_attn_fwd", "muse_attn_fwd_causal", "muse_status_string", "muse_last_error",
+           "muse_profile_enable", "muse_profile_read"]
 
 _lib = None
 
@@ -87,6 +89,11 @@ def load_library(path: str = LIB_PATH):
     lib.muse_status_string.argtypes = [i32]
     lib.muse_last_error.restype = ctypes.c_char_p
     lib.muse_last_error.argtypes = []
+    lib.muse_profile_enable.restype = None
+    lib.muse_profile_enable.argtypes = [i32]
+    lib.muse_profile_read.restype = i32
+    lib.muse_profile_read.argtypes = [ctypes.c_char_p, i32, ctypes.POINTER(ctypes.c_int),
+                                      ctypes.POINTER(ctypes.c_double), i32]
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -125,9 +132,9 @@ def make_params(Cq, Ck, iters, seed, topk, block=0, scale=1.0, mode="dipole") ->
                        int(block), float(scale), MODES[mode] if isinstance(mode, str) else int(mode))
 
 
-def make_shape(q, k) -> muse_shape:
+def make_shape(q, k, out_f32: bool = False) -> muse_shape:
     B, Hq, N, D = q.shape
-    return muse_shape(B, Hq, k.shape[1], N, D, _dtype_code(q))
+    return muse_shape(B, Hq, k.shape[1], N, D, _dtype_code(q), int(bool(out_f32)))
 
 
 def workspace_size(q, k, params: muse_params, causal: bool) -> int:
@@ -157,17 +164,24 @@ def _debug_buffers(q, k, params, causal):
         if params.topk > 0:
             out["selected"] = torch.empty(B, Hq, params.Cq, params.topk, **i32)
     out["n_exact"] = torch.empty(B, Hq, N, dtype=torch.int64, device=dev)
+    out["device_error"] = torch.full((1,), -1, dtype=torch.int32, device=dev)
     return out
 
 
-def _attn(causal, q, k, v, params, out=None, workspace=None, debug=False, stream=None):
+def _attn(causal, q, k, v, params, out=None, workspace=None, debug=False, stream=None,
+          out_dtype=None):
     lib = load_library()
     _need_cuda(q, k, v, out, workspace)
     if k.shape != v.shape or q.dtype != k.dtype or k.dtype != v.dtype:
         raise ValueError("k and v must match in shape; q, k, v must share a dtype")
-    sh = make_shape(q, k)
+    if out is not None:
+        out_dtype = out.dtype
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out_dtype not in (q.dtype, torch.float32):
+        raise ValueError("the output dtype must be the input dtype or float32")
+    sh = make_shape(q, k, out_dtype == torch.float32 and q.dtype != torch.float32)
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
     if workspace is None:
         workspace = torch.empty(workspace_size(q, k, params, causal), dtype=torch.uint8,
                                 device=q.device)
@@ -185,19 +199,20 @@ def _attn(causal, q, k, v, params, out=None, workspace=None, debug=False, stream
 
 
 def muse_attn_fwd(q, k, v, *, Cq, Ck, iters, seed, topk, scale=1.0, mode="dipole", out=None,
-                  workspace=None, debug=False, stream=None):
+                  workspace=None, debug=False, stream=None, out_dtype=None):
     """Acausal MuSe forward.  q [B,Hq,N,D], k and v [B,Hkv,N,D] (bf16 or fp32,
-    contiguous, CUDA).  Returns O (and a dict of debug tensors if debug)."""
+    contiguous, CUDA).  Returns O (input dtype, or fp32 with out_dtype=float32)
+    and, with debug, a dict of inspection tensors."""
     p = make_params(Cq, Ck, iters, seed, topk, 0, scale, mode)
-    return _attn(False, q, k, v, p, out, workspace, debug, stream)
+    return _attn(False, q, k, v, p, out, workspace, debug, stream, out_dtype)
 
 
 def muse_attn_fwd_causal(q, k, v, *, C, block, iters, seed, topk, scale=1.0, mode="dipole",
-                         out=None, workspace=None, debug=False, stream=None):
+                         out=None, workspace=None, debug=False, stream=None, out_dtype=None):
     """Causal MuSe forward (hierarchical blocks of `block` tokens, C clusters
     per level and role)."""
     p = make_params(C, C, iters, seed, topk, block, scale, mode)
-    return _attn(True, q, k, v, p, out, workspace, debug, stream)
+    return _attn(True, q, k, v, p, out, workspace, debug, stream, out_dtype)
 
 
 def muse_cluster(x, C, iters, seed, role=0, init=None, workspace=None, stream=None):
@@ -237,3 +252,23 @@ def muse_summarize(k, v, assign, C, with_dipole=True, stream=None):
                             _ptr(counts), _ptr(mu), _ptr(S), _ptr(M), None, 0, _stream(stream))
     _check(lib, st)
     return counts, mu, S, M
+
+
+def profile_enable(on: bool = True) -> None:
+    """Bracket every library kernel launch with CUDA events (benchmarks)."""
+    load_library().muse_profile_enable(int(bool(on)))
+
+
+def profile_read() -> dict:
+    """{kernel name: (launches, total ms)} since the last read; clears it."""
+    lib = load_library()
+    cap, stride = 64, 64
+    names = ctypes.create_string_buffer(cap * stride)
+    launches = (ctypes.c_int * cap)()
+    ms = (ctypes.c_double * cap)()
+    n = lib.muse_profile_read(names, stride, launches, ms, cap)
+    out = {}
+    for i in range(min(n, cap)):
+        nm = names.raw[i * stride:(i + 1) * stride].split(b"\0", 1)[0].decode()
+        out[nm] = (int(launches[i]), float(ms[i]))
+    return out

@@ -99,6 +99,9 @@ void carve_kstate(Carver& cv, KState& ks, const RoleGeo& g) {
   ks.perm = cv.take<int>((size_t)ks.ntok * 4);
   ks.hist = cv.take<int>((size_t)ks.ntiles * C * 4);
   ks.arrive = cv.take<int>(np * 4);
+  ks.cbf_hi = cv.take<__nv_bfloat16>(np * C * D * 2);
+  ks.cbf_lo = cv.take<__nv_bfloat16>(np * C * D * 2);
+  ks.cn2 = cv.take<float>(np * C * 4);
 }
 
 RoleGeo make_geo(const void* X, int BH, int D, int C, int role, int dtype, uint64_t seed,
@@ -123,6 +126,7 @@ struct AttnPlan {
 };
 
 struct AttnLayout {
+  int* err;
   RoleGeo qg, kg;
   KState qs, ks;
   Stage1 s1;
@@ -140,6 +144,7 @@ muse_status validate(const muse_shape* sh, const muse_params* pr, bool causal) {
   if (sh->D != 64 && sh->D != 128) return fail(MUSE_ERR_UNSUPPORTED, "D must be 64 or 128");
   if (sh->dtype != MUSE_BF16 && sh->dtype != MUSE_F32)
     return fail(MUSE_ERR_INVALID_ARG, "dtype must be MUSE_BF16 or MUSE_F32");
+  if (sh->out_f32 != 0 && sh->out_f32 != 1) return fail(MUSE_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
   if (pr->iters < 1) return fail(MUSE_ERR_INVALID_ARG, "iters must be >= 1");
   if (pr->mode < MUSE_MONOPOLE || pr->mode > MUSE_TILTED)
     return fail(MUSE_ERR_INVALID_ARG, "unknown mode");
@@ -174,8 +179,10 @@ AttnLayout layout(const muse_shape* sh, const muse_params* pr, bool causal, cons
   L.kg = make_geo(K, sh->B * sh->Hkv, sh->D, pr->Ck, 0, dt, pr->seed, lv);
   L.qg = make_geo(Q, sh->B * sh->Hq, sh->D, pr->Cq, 1, dt, pr->seed, lv);
   Carver cv{static_cast<char*>(ws)};
+  L.err = cv.take<int>(4);
   carve_kstate(cv, L.ks, L.kg);
   carve_kstate(cv, L.qs, L.qg);
+  L.ks.err = L.qs.err = L.err;
   L.nq = L.qs.nprob;
   const size_t cc = (size_t)pr->Cq * pr->Ck;
   const size_t per = cc * 4 * 2 + cc * sh->D * 4 * (pr->mode == MUSE_TILTED ? 2 : 1);
@@ -211,6 +218,7 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   a.ks = L.ks;
   a.V = V;
   a.O = causal ? nullptr : O;
+  a.out_f32 = sh->out_f32 ? 1 : 0;
   a.part = L.part;
   a.n_exact = dbg ? reinterpret_cast<long long*>(dbg->n_exact) : nullptr;
   a.B = sh->B;
@@ -223,6 +231,7 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   const size_t elt = sh->dtype == MUSE_BF16 ? 2 : 4;
   if (a.n_exact && causal)
     cudaMemsetAsync(a.n_exact, 0, (size_t)sh->B * sh->Hq * sh->N * 8, st);
+  cudaMemsetAsync(L.err, 0, 4, st);
   if (L.nq > 0) {
     cudaMemsetAsync(L.ks.arrive, 0, (size_t)L.ks.nprob * 4, st);
     cudaMemsetAsync(L.qs.arrive, 0, (size_t)L.qs.nprob * 4, st);
@@ -239,6 +248,7 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   }
   if (dbg) {
     const size_t D = sh->D;
+    if (dbg->device_error) cudaMemcpyAsync(dbg->device_error, L.err, 4, cudaMemcpyDeviceToDevice, st);
     if (dbg->q_assign) cudaMemcpyAsync(dbg->q_assign, L.qs.assign, (size_t)L.qs.ntok * 4, cudaMemcpyDeviceToDevice, st);
     if (dbg->k_assign) cudaMemcpyAsync(dbg->k_assign, L.ks.assign, (size_t)L.ks.ntok * 4, cudaMemcpyDeviceToDevice, st);
     if (!causal) {
@@ -268,6 +278,7 @@ size_t muse_cluster_workspace_size(int B, int H, int N, int D, int C) {
   RoleGeo g = make_geo(nullptr, B * H, D, C, 0, 0, 0, lv);
   Carver cv{nullptr};
   KState ks{};
+  cv.take<int>(4);
   carve_kstate(cv, ks, g);
   return cv.used + 256;
 }
@@ -291,7 +302,10 @@ muse_status muse_cluster(const void* X, muse_dtype dtype, int B, int H, int N, i
   RoleGeo g = make_geo(X, B * H, D, C, role, dtype == MUSE_BF16 ? 0 : 1, seed, lv);
   Carver cv{static_cast<char*>(ws)};
   KState ks{};
+  int* err = cv.take<int>(4);
   carve_kstate(cv, ks, g);
+  ks.err = err;
+  cudaMemsetAsync(err, 0, 4, stream);
   cudaMemsetAsync(ks.arrive, 0, (size_t)ks.nprob * 4, stream);
   run_kmeans(g, ks, iters, init, stream);
   cudaMemcpyAsync(assign, ks.assign, (size_t)ks.ntok * 4, cudaMemcpyDeviceToDevice, stream);

@@ -116,6 +116,10 @@ struct KState {
   int* perm;        // [tokens]      problem-local token index in cluster-sorted order
   int* hist;        // [tiles][C]    per-tile histogram, then scatter bases
   int* arrive;      // [nprob]       tile arrival counters (self-resetting)
+  __nv_bfloat16* cbf_hi;  // [nprob][C][D] bf16 rounding of cent32
+  __nv_bfloat16* cbf_lo;  // [nprob][C][D] bf16 rounding of cent32 - cbf_hi
+  float* cn2;       // [nprob][C]    ||c||^2 (fp64 sum rounded to fp32)
+  int* err;         // device error word (0 = ok)
   int nprob;
   long long ntiles;
   long long ntok;

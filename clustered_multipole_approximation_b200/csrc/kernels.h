@@ -7,6 +7,14 @@
 
 namespace muse {
 
+// Brackets one kernel launch with profiling events when profiling is on.
+struct ProfScope {
+  ProfScope(cudaStream_t st, const char* name);
+  ~ProfScope();
+  cudaStream_t st;
+  int slot;
+};
+
 // Per-(query problem) stage-1 tables in the workspace.
 struct Stage1 {
   float* logW;    // [nq][Cq][Ck]  log W_ij, -inf for empty key clusters
@@ -22,6 +30,7 @@ struct AttnArgs {
   KState qs, ks;      // their k-means state
   const void* V;
   void* O;            // acausal: final output
+  int out_f32;        // O is fp32 (else the input dtype)
   float* part;        // causal: [nq_total tokens][D + 1] partial (o, lse)
   long long* n_exact; // optional [B,Hq,N]
   int B;              // batch
@@ -34,8 +43,14 @@ struct AttnArgs {
 void run_kmeans(const RoleGeo& g, const KState& ks, int iters, const float* init,
                 cudaStream_t st);
 
+// Tensor-core (tcgen05) assignment screen for bf16 inputs.
+void launch_assign_tc(const RoleGeo& g, const KState& ks, cudaStream_t st);
+
 // Stage 1 + selection + stage 2 for query problems [qp0, qp0 + nqp).
 void run_blocks(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
+
+// Stage 2 on tensor cores (bf16 inputs).
+void run_stage2_mma(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 
 // Causal: exact local block + merge of the level partials into O.
 void run_local_merge(const AttnArgs& a, int L, cudaStream_t st);

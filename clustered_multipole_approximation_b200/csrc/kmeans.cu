@@ -20,6 +20,7 @@
 // the centroids equal a sequential fp64 evaluation of the same means.
 #include "common.cuh"
 #include "kernels.h"
+#include "kmeans_tail.cuh"
 
 namespace muse {
 
@@ -90,16 +91,28 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(RoleGeo g, KState ks, 
     }
   }
   __syncthreads();
-  // centroid norms for the screen bound
+  // centroid norms for the screen bounds, and the bf16 split for the tensor cores
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int c = warp; c < C; c += blockDim.x >> 5) {
     float s = 0.f;
+    double s2 = 0.0;
     for (int d = lane; d < D; d += 32) {
-      float v = c32[(size_t)c * D + d];
+      const size_t i = (size_t)c * D + d;
+      float v = c32[i];
       s = fmaf(v, v, s);
+      s2 += c64[i] * c64[i];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      ks.cbf_hi[(size_t)pid * g.C * D + i] = hi;
+      ks.cbf_lo[(size_t)pid * g.C * D + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
     }
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) ks.cnorm[(size_t)pid * g.C + c] = sqrtf(s) * 1.0001f;
+    for (int o = 16; o; o >>= 1) {
+      s += __shfl_xor_sync(0xffffffffu, s, o);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    if (lane == 0) {
+      ks.cnorm[(size_t)pid * g.C + c] = sqrtf(s) * 1.0001f;
+      ks.cn2[(size_t)pid * g.C + c] = (float)s2;
+    }
   }
 }
 
@@ -134,7 +147,6 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(RoleGeo g, KState 
   const int nt = imin(kTile, p.s - t0);
   const T* X = static_cast<const T*>(g.X);
   const float* c32 = ks.cent32 + (size_t)pid * g.C * D;
-  const double* c64 = ks.cent64 + (size_t)pid * g.C * D;
   const int tid = threadIdx.x;
 
   for (int i = tid; i < C; i += kTile) {
@@ -187,92 +199,9 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_kernel(RoleGeo g, KState 
       }
     }
   }
-  if (valid && olb <= bd + be) {
-    int slot = atomicAdd(&nflag, 1);
-    flagged[slot] = tid;
-  }
-  __syncthreads();
-  // fp64 re-decision, one warp per flagged token, lanes over clusters; the
-  // distance is accumulated in dimension order without fused operations so
-  // it equals a plain sequential fp64 evaluation bit for bit.
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int f = warp; f < nflag; f += kTile / 32) {
-    const int r = flagged[f];
-    double bdd = 0.0;
-    int bc = -1;
-    for (int c = lane; c < C; c += 32) {
-      const double* cc = c64 + (size_t)c * D;
-      double s = 0.0;
-      for (int d = 0; d < D; ++d) {
-        double t = __dsub_rn((double)xs[r][d], cc[d]);
-        s = __dadd_rn(s, __dmul_rn(t, t));
-      }
-      if (bc < 0 || s < bdd) {
-        bdd = s;
-        bc = c;
-      }
-    }
-    for (int o = 16; o; o >>= 1) {
-      double od = __shfl_xor_sync(0xffffffffu, bdd, o);
-      int oc = __shfl_xor_sync(0xffffffffu, bc, o);
-      if (oc >= 0 && (bc < 0 || od < bdd || (od == bdd && oc < bc))) {
-        bdd = od;
-        bc = oc;
-      }
-    }
-    if (lane == 0) decision[r] = bc;
-  }
-  __syncthreads();
-  if (valid) {
-    if (olb <= bd + be) best = decision[tid];
-    ks.assign[p.slot0 + t0 + tid] = best;
-    atomicAdd(&hist[best], 1);
-  }
-  __syncthreads();
-  int* th = ks.hist + (size_t)blockIdx.x * g.C;
-  for (int i = tid; i < C; i += kTile) th[i] = hist[i];
-  // the last tile of the problem turns histograms into offsets and bases
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int ntp = cdiv(p.s, kTile);
-    is_last = (atomicAdd(&ks.arrive[pid], 1) == ntp - 1);
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  const int ntp = cdiv(p.s, kTile);
-  int* ph = ks.hist + (size_t)p.tile0 * g.C;
-  int* cnt = ks.counts + (size_t)pid * g.C;
-  int* off = ks.off + (size_t)pid * (g.C + 1);
-  for (int c = tid; c < C; c += kTile) {
-    int tot = 0;
-    for (int t = 0; t < ntp; ++t) tot += __ldcg(ph + (size_t)t * g.C + c);
-    hist[c] = tot;
-    cnt[c] = tot;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int c = 0; c < C; ++c) {
-      off[c] = run;
-      int v = hist[c];
-      hist[c] = run;
-      run += v;
-    }
-    off[C] = run;
-    ks.arrive[pid] = 0;
-  }
-  __syncthreads();
-  for (int c = tid; c < C; c += kTile) {
-    int run = hist[c];
-    for (int t = 0; t < ntp; ++t) {
-      int* h = ph + (size_t)t * g.C + c;
-      int v = __ldcg(h);
-      *h = run;
-      run += v;
-    }
-  }
+  auto xrow = [&](int r, int d) { return xs[r][d]; };
+  assign_tail<D>(g, ks, p, pid, t0, nt, best, valid && olb <= bd + be, xrow, hist, flagged,
+                 decision, &nflag, &is_last);
 }
 
 // ----------------------------------------------------------------------------
@@ -331,22 +260,30 @@ __global__ void __launch_bounds__(256) kmeans_reduce_kernel(RoleGeo g, KState ks
       for (int r = 0; r < R; ++r) s[r] = __dadd_rn(s[r], (double)ld<T>(row + lane + 32 * r));
     }
     const double n = (double)(e - b);
+    double q2 = 0.0;
+    float q = 0.f;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      double v = __ddiv_rn(s[r], n);
+      const double v = __ddiv_rn(s[r], n);
+      const float v32 = (float)v;
+      const size_t i = ((size_t)pid * g.C + c) * D + lane + 32 * r;
       c64[lane + 32 * r] = v;
-      c32[lane + 32 * r] = (float)v;
+      c32[lane + 32 * r] = v32;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v32);
+      ks.cbf_hi[i] = hi;
+      ks.cbf_lo[i] = __float2bfloat16_rn(v32 - __bfloat162float(hi));
+      q2 += v * v;
+      q = fmaf(v32, v32, q);
+    }
+    for (int o = 16; o; o >>= 1) {
+      q += __shfl_xor_sync(0xffffffffu, q, o);
+      q2 += __shfl_xor_sync(0xffffffffu, q2, o);
+    }
+    if (lane == 0) {
+      ks.cnorm[(size_t)pid * g.C + c] = sqrtf(q) * 1.0001f;
+      ks.cn2[(size_t)pid * g.C + c] = (float)q2;
     }
   }
-  __syncwarp();
-  float q = 0.f;
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    float v = c32[lane + 32 * r];
-    q = fmaf(v, v, q);
-  }
-  for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-  if (lane == 0) ks.cnorm[(size_t)pid * g.C + c] = sqrtf(q) * 1.0001f;
 }
 
 // ----------------------------------------------------------------------------
@@ -360,16 +297,31 @@ static void launch_round(const RoleGeo& g, const KState& ks, cudaStream_t st) {
                          (int)assign_smem<D>());
     attr = true;
   }
-  kmeans_assign_kernel<T, D><<<(unsigned)ks.ntiles, kTile, assign_smem<D>(), st>>>(g, ks);
-  kmeans_scatter_kernel<<<(unsigned)ks.ntiles, kTile, 0, st>>>(g, ks);
+  {
+    ProfScope ps(st, "kmeans_assign");
+    if (sizeof(T) == 2)
+      launch_assign_tc(g, ks, st);
+    else
+      kmeans_assign_kernel<T, D><<<(unsigned)ks.ntiles, kTile, assign_smem<D>(), st>>>(g, ks);
+  }
+  {
+    ProfScope ps(st, "kmeans_scatter");
+    kmeans_scatter_kernel<<<(unsigned)ks.ntiles, kTile, 0, st>>>(g, ks);
+  }
   const long long warps = (long long)ks.nprob * g.C;
-  kmeans_reduce_kernel<T, D><<<(unsigned)cdiv((int)warps, 8), 256, 0, st>>>(g, ks);
+  {
+    ProfScope ps(st, "kmeans_reduce");
+    kmeans_reduce_kernel<T, D><<<(unsigned)cdiv((int)warps, 8), 256, 0, st>>>(g, ks);
+  }
 }
 
 template <typename T>
 static void run_kmeans_t(const RoleGeo& g, const KState& ks, int iters, const float* init,
                          cudaStream_t st) {
-  kmeans_init_kernel<T><<<ks.nprob, 128, 0, st>>>(g, ks, init);
+  {
+    ProfScope ps(st, "kmeans_init");
+    kmeans_init_kernel<T><<<ks.nprob, 128, 0, st>>>(g, ks, init);
+  }
   for (int it = 0; it < iters; ++it) {
     if (g.D == 64)
       launch_round<T, 64>(g, ks, st);

@@ -38,126 +38,214 @@ __device__ inline int kv_problem(const AttnArgs& a, int qpid) {
 }
 
 // ----------------------------------------------------------------------------
-// stage 1: one warp per (query problem, query cluster i) walks every key
-// cluster j of the paired key problem and forms u_ij, log W_ij, the far-field
-// key row and the far-field logit offset
+// stage 1: one CTA per (query problem, key cluster j).  The cluster's members
+// (k - mu_j and v) are staged in shared memory once; query centroids come in
+// chunks of 32.  For each chunk the CTA forms a_ti = s nu_i.k~_t, the weights
+// (1 + a for DIPOLE, exp(a - max) for TILTED) and the weighted sums over the
+// members, giving u_ij, log W_ij, the far-field key row and logit offset.
 // ----------------------------------------------------------------------------
-constexpr int kS1W = 8;  // warps (query clusters) per CTA
+constexpr int kS1T = 256;  // threads
+constexpr int kS1M = 128;  // members per staged chunk
+constexpr int kS1I = 32;   // query clusters per pass
+
+template <int D>
+constexpr size_t stage1_smem() {
+  return sizeof(float) * ((size_t)2 * kS1M * (D + 1) + (size_t)kS1I * (D + 1) +
+                          (size_t)kS1M * (kS1I + 1) + (size_t)kS1I * D + D + 3 * kS1I);
+}
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kS1W * 32) stage1_kernel(AttnArgs a, Stage1 s1, int qp0) {
-  constexpr int R = D / 32;
-  __shared__ float nu_s[kS1W][D];
-  __shared__ float mu_s[kS1W][D];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int lq = blockIdx.x, qpid = qp0 + lq;
-  const int i = blockIdx.y * kS1W + warp;
+__global__ void __launch_bounds__(kS1T) stage1_kernel(AttnArgs a, Stage1 s1, int qp0) {
+  constexpr int GROUPS = kS1T / D;      // query-cluster lanes per pass
+  constexpr int R = kS1I / GROUPS;      // outputs (i, e) per thread
+  extern __shared__ float sm1[];
+  float(*kt)[D + 1] = reinterpret_cast<float(*)[D + 1]>(sm1);
+  float(*vt)[D + 1] = reinterpret_cast<float(*)[D + 1]>(sm1 + kS1M * (D + 1));
+  float(*nu)[D + 1] = reinterpret_cast<float(*)[D + 1]>(sm1 + 2 * kS1M * (D + 1));
+  float(*ws)[kS1I + 1] = reinterpret_cast<float(*)[kS1I + 1]>(sm1 + 2 * kS1M * (D + 1) + kS1I * (D + 1));
+  float(*red)[D] = reinterpret_cast<float(*)[D]>(sm1 + 2 * kS1M * (D + 1) + kS1I * (D + 1) +
+                                                 kS1M * (kS1I + 1));
+  float* mu = reinterpret_cast<float*>(red) + kS1I * D;
+  float* mrun = mu + D;
+  float* zrun = mrun + kS1I;
+  float* rsc = zrun + kS1I;
+
+  const int lq = blockIdx.x, qpid = qp0 + lq, j = blockIdx.y;
   const Prob pq = prob_of(a.qg, qpid);
-  if (i >= pq.C) return;  // warp-uniform; this kernel has no CTA-wide barrier
-  const int Cq = a.Cq, Ck = a.Ck;
-  if (a.qs.counts[(size_t)qpid * Cq + i] == 0) return;
   const int kpid = kv_problem(a, qpid);
   const Prob pk = prob_of(a.kg, kpid);
-  const int* kc = a.ks.counts + (size_t)kpid * Ck;
-  const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
+  if (j >= pk.C) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Cq = a.Cq, Ck = a.Ck;
+  const int nj = a.ks.counts[(size_t)kpid * Ck + j];
+  const size_t ij0 = ((size_t)lq * Cq) * Ck + j;  // + i * Ck
+  if (nj == 0) {
+    for (int i = tid; i < pq.C; i += kS1T) {
+      s1.logW[ij0 + (size_t)i * Ck] = -INFINITY;
+      s1.fbias[ij0 + (size_t)i * Ck] = -INFINITY;
+    }
+    return;
+  }
+  const int off = a.ks.off[(size_t)kpid * (Ck + 1) + j];
   const int* perm = a.ks.perm + pk.slot0;
   const T* K = static_cast<const T*>(a.kg.X);
   const T* V = static_cast<const T*>(a.V);
-  float* nu = nu_s[warp];
-  float* mu = mu_s[warp];
-  for (int d = lane; d < D; d += 32) nu[d] = a.qs.cent32[((size_t)qpid * Cq + i) * D + d];
+  for (int d = tid; d < D; d += kS1T) mu[d] = a.ks.cent32[((size_t)kpid * Ck + j) * D + d];
+  __syncthreads();
   const float s = a.scale;
   const int mode = a.mode;
-  const size_t ij0 = ((size_t)lq * Cq + i) * Ck;
-  for (int j = 0; j < pk.C; ++j) {
-    const int nj = kc[j];
-    const size_t ij = ij0 + j;
-    if (nj == 0) {
-      if (lane == 0) {
-        s1.logW[ij] = -INFINITY;
-        s1.fbias[ij] = -INFINITY;
-      }
-      continue;
+  const float lognj = logf((float)nj);
+
+  auto load_chunk = [&](int c0, int cnt) {
+    for (int e = tid; e < cnt * D; e += kS1T) {
+      const int r = e / D, d = e - r * D;
+      const long long row = pk.row0 + perm[off + c0 + r];
+      kt[r][d] = ld<T>(K + row * D + d) - mu[d];
+      vt[r][d] = ld<T>(V + row * D + d);
     }
-    __syncwarp();
-    for (int d = lane; d < D; d += 32) mu[d] = a.ks.cent32[((size_t)kpid * Ck + j) * D + d];
-    __syncwarp();
+  };
+
+  const int e = tid % D, g0 = tid / D;
+  if (mode == 0) {  // MONOPOLE: u_ij = S_j / n_j for every i
+    float acc = 0.f;
+    for (int c0 = 0; c0 < nj; c0 += kS1M) {
+      const int cnt = imin(kS1M, nj - c0);
+      __syncthreads();
+      load_chunk(c0, cnt);
+      __syncthreads();
+      if (tid < D)
+        for (int t = 0; t < cnt; ++t) acc += vt[t][tid];
+    }
+    if (tid < D) red[0][tid] = acc / (float)nj;
+    __syncthreads();
+    for (int idx = tid; idx < pq.C * D; idx += kS1T) {
+      const int i = idx / D, d = idx - i * D;
+      s1.U[(ij0 + (size_t)i * Ck) * D + d] = red[0][d];
+    }
+    for (int i = tid; i < pq.C; i += kS1T) {
+      s1.logW[ij0 + (size_t)i * Ck] = lognj;
+      s1.fbias[ij0 + (size_t)i * Ck] = lognj;
+    }
+    return;
+  }
+
+  const bool one_chunk = nj <= kS1M;
+  if (one_chunk) load_chunk(0, nj);
+  for (int i0 = 0; i0 < pq.C; i0 += kS1I) {
+    const int ic = imin(kS1I, pq.C - i0);
+    __syncthreads();
+    for (int idx = tid; idx < ic * D; idx += kS1T) {
+      const int ii = idx / D, d = idx - ii * D;
+      nu[ii][d] = a.qs.cent32[((size_t)qpid * Cq + i0 + ii) * D + d];
+    }
+    if (tid < kS1I) {
+      mrun[tid] = -INFINITY;
+      zrun[tid] = 0.f;
+    }
     float accU[R], accK[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) accU[r] = accK[r] = 0.f;
-    float m = -INFINITY, z = 0.f;
-    const int off = koff[j];
-    for (int t0 = 0; t0 < nj; t0 += 32) {
-      const int cnt = imin(32, nj - t0);
-      const bool on = lane < cnt;
-      const long long row = on ? pk.row0 + perm[off + t0 + lane] : 0;
-      float w = 0.f;
-      if (mode == 0) {
-        w = on ? 1.f : 0.f;
-      } else {
-        float g = 0.f;
-        if (on) {
-          const T* kr = K + row * D;
-#pragma unroll 8
-          for (int d = 0; d < D; ++d) g = fmaf(nu[d], ld<T>(kr + d) - mu[d], g);
+    for (int c0 = 0; c0 < nj; c0 += kS1M) {
+      const int cnt = imin(kS1M, nj - c0);
+      if (!one_chunk) {
+        __syncthreads();
+        load_chunk(c0, cnt);
+      }
+      __syncthreads();
+      // a_ti = s nu_i . k~_t
+      for (int idx = tid; idx < kS1M * kS1I; idx += kS1T) {
+        const int tt = idx >> 5, ii = idx & 31;
+        if (tt < cnt && ii < ic) {
+          float g = 0.f;
+#pragma unroll 16
+          for (int d = 0; d < D; ++d) g = fmaf(nu[ii][d], kt[tt][d], g);
+          ws[tt][ii] = s * g;
         }
-        const float at = s * g;
-        if (mode == 1) {
-          w = on ? 1.f + at : 0.f;  // first-order term of exp(s nu.k~)
-        } else {
-          float cm = on ? at : -INFINITY;
-          for (int o = 16; o; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
-          const float mn = fmaxf(m, cm);
-          const float rs = (m == -INFINITY) ? 0.f : expf(m - mn);
-          w = on ? expf(at - mn) : 0.f;
-          float ws = w;
-          for (int o = 16; o; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
-          z = z * rs + ws;
-          m = mn;
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            accU[r] *= rs;
-            accK[r] *= rs;
+      }
+      __syncthreads();
+      if (mode == 1) {
+        for (int idx = tid; idx < cnt * kS1I; idx += kS1T) {
+          const int tt = idx >> 5, ii = idx & 31;
+          ws[tt][ii] = 1.f + ws[tt][ii];  // first-order term of exp(s nu.k~)
+        }
+      } else {
+        // per query cluster: running max-shifted exponential weights
+        for (int ii = warp; ii < ic; ii += kS1T / 32) {
+          float mx = -INFINITY;
+          for (int tt = lane; tt < cnt; tt += 32) mx = fmaxf(mx, ws[tt][ii]);
+          for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float mo = mrun[ii], mn = fmaxf(mo, mx);
+          float zs = 0.f;
+          for (int tt = lane; tt < cnt; tt += 32) {
+            const float wv = expf(ws[tt][ii] - mn);
+            ws[tt][ii] = wv;
+            zs += wv;
+          }
+          for (int o = 16; o; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+          if (lane == 0) {
+            const float rs = (mo == -INFINITY) ? 0.f : expf(mo - mn);
+            rsc[ii] = rs;
+            zrun[ii] = zrun[ii] * rs + zs;
+            mrun[ii] = mn;
           }
         }
       }
-      for (int tt = 0; tt < cnt; ++tt) {
-        const float wt = __shfl_sync(0xffffffffu, w, tt);
-        const long long rt = __shfl_sync(0xffffffffu, row, tt);
+      __syncthreads();
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const int e = lane + 32 * r;
-          accU[r] = fmaf(wt, ld<T>(V + rt * D + e), accU[r]);
-          if (mode == 2) accK[r] = fmaf(wt, ld<T>(K + rt * D + e) - mu[e], accK[r]);
+      for (int r = 0; r < R; ++r) {
+        const int ii = g0 + GROUPS * r;
+        if (ii >= ic) continue;
+        float su = 0.f, sk = 0.f;
+        for (int tt = 0; tt < cnt; ++tt) {
+          const float wv = ws[tt][ii];
+          su = fmaf(wv, vt[tt][e], su);
+          if (mode == 2) sk = fmaf(wv, kt[tt][e], sk);
+        }
+        if (mode == 2) {
+          const float rs = rsc[ii];
+          accU[r] = fmaf(accU[r], rs, su);
+          accK[r] = fmaf(accK[r], rs, sk);
+        } else {
+          accU[r] += su;
         }
       }
     }
-    if (mode != 2) {
+    // outputs of this chunk of query clusters
+    if (mode == 1) {
       const float inv = 1.f / (float)nj;
 #pragma unroll
-      for (int r = 0; r < R; ++r) s1.U[ij * D + lane + 32 * r] = accU[r] * inv;
-      if (lane == 0) {
-        const float lw = logf((float)nj);
-        s1.logW[ij] = lw;
-        s1.fbias[ij] = lw;
+      for (int r = 0; r < R; ++r) {
+        const int ii = g0 + GROUPS * r;
+        if (ii < ic) s1.U[(ij0 + (size_t)(i0 + ii) * Ck) * D + e] = accU[r] * inv;
+      }
+      for (int ii = tid; ii < ic; ii += kS1T) {
+        s1.logW[ij0 + (size_t)(i0 + ii) * Ck] = lognj;
+        s1.fbias[ij0 + (size_t)(i0 + ii) * Ck] = lognj;
       }
     } else {
-      // k_hat = mu + sum w k~ / W;  offset = s nu.(mu - k_hat) + log W
-      const float inv = 1.f / z;
-      float part = 0.f;
+      // k_hat = mu + sum w k~ / W;  offset = log W - s nu.(k_hat - mu)
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        const int e = lane + 32 * r;
+        const int ii = g0 + GROUPS * r;
+        if (ii >= ic) continue;
+        const float inv = 1.f / zrun[ii];
         const float kh = accK[r] * inv;
+        const size_t ij = ij0 + (size_t)(i0 + ii) * Ck;
         s1.U[ij * D + e] = accU[r] * inv;
         s1.Kf[ij * D + e] = mu[e] + kh;
-        part = fmaf(nu[e], kh, part);
+        red[ii][e] = nu[ii][e] * kh;
       }
-      for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-      if (lane == 0) {
-        const float lw = m + logf(z);
-        s1.logW[ij] = lw;
-        s1.fbias[ij] = lw - s * part;
+      __syncthreads();
+      for (int ii = warp; ii < ic; ii += kS1T / 32) {
+        float part = 0.f;
+        for (int d = lane; d < D; d += 32) part += red[ii][d];
+        for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) {
+          const float lw = mrun[ii] + logf(zrun[ii]);
+          const size_t ij = ij0 + (size_t)(i0 + ii) * Ck;
+          s1.logW[ij] = lw;
+          s1.fbias[ij] = lw - s * part;
+        }
       }
     }
   }
@@ -179,7 +267,9 @@ __global__ void __launch_bounds__(256) select_kernel(AttnArgs a, Stage1 s1, int 
   double* sc = sc_all + (size_t)warp * Ck;
   const double s = (double)a.scale;
   const int* kc = a.ks.counts + (size_t)kpid * Ck;
-  for (int i = warp; i < pq.C; i += 8) {
+  {
+    const int i = blockIdx.y * 8 + warp;
+    if (i >= pq.C) return;  // warp-uniform; no CTA-wide barrier below
     const double* nu = a.qs.cent64 + ((size_t)qpid * Cq + i) * D;
     for (int j = lane; j < pk.C; j += 32) {
       double v = -INFINITY;
@@ -243,7 +333,7 @@ struct Online {
   float m, l;
 };
 
-template <typename T, int D>
+template <typename T, typename TO, int D>
 __global__ void __launch_bounds__(kQ * (D / 64)) stage2_kernel(AttnArgs a, Stage1 s1, int qp0) {
   constexpr int P = D / 64;
   __shared__ float ks_[kRows][D];
@@ -358,9 +448,9 @@ __global__ void __launch_bounds__(kQ * (D / 64)) stage2_kernel(AttnArgs a, Stage
       const long long row = pq.row0 + tq;
       const float inv = 1.f / l;
       if (a.O != nullptr) {
-        T* O = static_cast<T*>(a.O);
+        TO* O = static_cast<TO*>(a.O);
 #pragma unroll
-        for (int d = 0; d < 64; ++d) st<T>(O + row * D + part * 64 + d, acc[d] * inv);
+        for (int d = 0; d < 64; ++d) st<TO>(O + row * D + part * 64 + d, acc[d] * inv);
       } else {
         float* pp = a.part + (size_t)(pq.slot0 + tq) * (D + 1);
 #pragma unroll
@@ -382,7 +472,7 @@ __global__ void __launch_bounds__(kQ * (D / 64)) stage2_kernel(AttnArgs a, Stage
 // causal: exact local block, then merge the level partials (each partial is
 // the softmax of its terms, entering as one term with logit lse and value o)
 // ----------------------------------------------------------------------------
-template <typename T, int D>
+template <typename T, typename TO, int D>
 __global__ void __launch_bounds__(kQ * (D / 64)) local_merge_kernel(AttnArgs a, int L) {
   constexpr int P = D / 64;
   __shared__ float ks_[kRows][D];
@@ -465,10 +555,10 @@ __global__ void __launch_bounds__(kQ * (D / 64)) local_merge_kernel(AttnArgs a, 
       for (int d = 0; d < 64; ++d) acc[d] = fmaf(wt, pp[part * 64 + d], acc[d]);
     }
   }
-  T* O = static_cast<T*>(a.O);
+  TO* O = static_cast<TO*>(a.O);
   const float inv = 1.f / l;
 #pragma unroll
-  for (int d = 0; d < 64; ++d) st<T>(O + qrow * D + part * 64 + d, acc[d] * inv);
+  for (int d = 0; d < 64; ++d) st<TO>(O + qrow * D + part * 64 + d, acc[d] * inv);
   if (a.n_exact != nullptr && part == 0)
     atomicAdd(reinterpret_cast<unsigned long long*>(a.n_exact + qrow),
               (unsigned long long)(qpos - blk * L + 1));
@@ -481,16 +571,31 @@ template <typename T, int D>
 static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
+    cudaFuncSetAttribute(stage1_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)stage1_smem<D>());
     cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          8 * kMaxC * (int)sizeof(double));
     attr = true;
   }
-  stage1_kernel<T, D><<<dim3(nqp, cdiv(a.Cq, kS1W)), kS1W * 32, 0, st>>>(a, s1, qp0);
-  if (a.topk > 0) {
-    const size_t smem = (size_t)8 * a.Ck * sizeof(double);
-    select_kernel<D><<<nqp, 256, smem, st>>>(a, s1, qp0);
+  {
+    ProfScope ps(st, "stage1_summaries");
+    stage1_kernel<T, D><<<dim3(nqp, a.Ck), kS1T, stage1_smem<D>(), st>>>(a, s1, qp0);
   }
-  stage2_kernel<T, D><<<dim3(nqp, a.Cq), kQ * (D / 64), 0, st>>>(a, s1, qp0);
+  if (a.topk > 0) {
+    ProfScope ps(st, "stage1_select");
+    const size_t smem = (size_t)8 * a.Ck * sizeof(double);
+    select_kernel<D><<<dim3(nqp, cdiv(a.Cq, 8)), 256, smem, st>>>(a, s1, qp0);
+  }
+  if (sizeof(T) == 2) {
+    ProfScope ps(st, "stage2_attn");
+    run_stage2_mma(a, s1, qp0, nqp, st);
+  } else {
+    ProfScope ps(st, "stage2_attn");
+    if (a.out_f32)
+      stage2_kernel<T, float, D><<<dim3(nqp, a.Cq), kQ * (D / 64), 0, st>>>(a, s1, qp0);
+    else
+      stage2_kernel<T, T, D><<<dim3(nqp, a.Cq), kQ * (D / 64), 0, st>>>(a, s1, qp0);
+  }
 }
 
 void run_blocks(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st) {
@@ -508,12 +613,19 @@ void run_local_merge(const AttnArgs& a, int L, cudaStream_t st) {
   const int D = a.qg.D, N = a.qg.lv.N;
   dim3 grid(a.qg.BH, cdiv(N, kQ));
   const int thr = kQ * (D / 64);
+  ProfScope ps(st, "causal_local_merge");
+  using bf = __nv_bfloat16;
   if (a.qg.dtype == 0) {
-    if (D == 64) local_merge_kernel<__nv_bfloat16, 64><<<grid, thr, 0, st>>>(a, L);
-    else local_merge_kernel<__nv_bfloat16, 128><<<grid, thr, 0, st>>>(a, L);
+    if (a.out_f32) {
+      if (D == 64) local_merge_kernel<bf, float, 64><<<grid, thr, 0, st>>>(a, L);
+      else local_merge_kernel<bf, float, 128><<<grid, thr, 0, st>>>(a, L);
+    } else {
+      if (D == 64) local_merge_kernel<bf, bf, 64><<<grid, thr, 0, st>>>(a, L);
+      else local_merge_kernel<bf, bf, 128><<<grid, thr, 0, st>>>(a, L);
+    }
   } else {
-    if (D == 64) local_merge_kernel<float, 64><<<grid, thr, 0, st>>>(a, L);
-    else local_merge_kernel<float, 128><<<grid, thr, 0, st>>>(a, L);
+    if (D == 64) local_merge_kernel<float, float, 64><<<grid, thr, 0, st>>>(a, L);
+    else local_merge_kernel<float, float, 128><<<grid, thr, 0, st>>>(a, L);
   }
 }
 

@@ -112,6 +112,7 @@ void run_summarize(const void* K, const void* V, int dtype, int BH, int N, int D
                    const int* assign, int* counts, float* mu, float* S, float* M, int*, int*,
                    cudaStream_t st) {
   dim3 grid(BH, C);
+  ProfScope ps(st, "summarize");
   if (dtype == 0) {
     auto k = static_cast<const __nv_bfloat16*>(K);
     auto v = static_cast<const __nv_bfloat16*>(V);

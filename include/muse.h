@@ -16,7 +16,8 @@
  *     the caller owns every buffer, including the workspace.  The library
  *     never allocates, frees or synchronises: all work is enqueued on the
  *     given stream and the call returns before it finishes.
- *   - Q is [B,Hq,N,D]; K and V are [B,Hkv,N,D]; O has Q's shape and dtype.
+ *   - Q is [B,Hq,N,D]; K and V are [B,Hkv,N,D]; O has Q's shape, and Q's
+ *     dtype unless muse_shape.out_f32 asks for fp32.
  *     q-head h reads kv-head h / (Hq/Hkv) (grouped-query attention).
  *   - Arguments are validated before anything is launched; a failing check
  *     returns MUSE_ERR_INVALID_ARG (or MUSE_ERR_UNSUPPORTED for shapes the
@@ -51,7 +52,7 @@ typedef enum { MUSE_BF16 = 0, MUSE_F32 = 1 } muse_dtype;
 
 /* Far-field summary of a key cluster j as seen from query cluster i:
  *   MONOPOLE  count, centroid and summed values ([A1] Abstract; [G] Core
- *             Mechanisms, retrieval item: "monopole (centroid)");
+ *             Mechanisms, "Retrieval-Augmented Approximation");
  *   DIPOLE    MONOPOLE plus the first-order correction (s/n_j) M_j nu_i with
  *             M_j = sum_{t in j} v_t (k_t - mu_j)^T ([A1] Abstract);
  *   TILTED    exponentially tilted summaries weighted by exp(s nu_i . k_t)
@@ -60,7 +61,8 @@ typedef enum { MUSE_MONOPOLE = 0, MUSE_DIPOLE = 1, MUSE_TILTED = 2 } muse_mode;
 
 typedef struct {
   int B, Hq, Hkv, N, D; /* D in {64, 128}; Hq % Hkv == 0 */
-  muse_dtype dtype;     /* of Q, K, V and O */
+  muse_dtype dtype;     /* of Q, K and V (and of O unless out_f32) */
+  int out_f32;          /* 0: O in dtype; 1: O in fp32 */
 } muse_shape;
 
 typedef struct {
@@ -85,6 +87,9 @@ typedef struct {
   int32_t *q_assign, *k_assign, *selected, *k_counts;
   float *q_centroids, *k_centroids;
   int64_t *n_exact;
+  int32_t *device_error; /* 0, or non-zero if a kernel's bounded wait on the
+                            tensor cores gave up (its tokens were then
+                            re-decided on the fp64 path) */
 } muse_debug;
 
 /* Workspace bytes muse_attn_fwd (causal == 0) or muse_attn_fwd_causal
@@ -145,7 +150,8 @@ muse_status muse_summarize(const void *K, const void *V, muse_dtype dtype,
  * query one far-field term per other non-empty cluster (logit
  * s q.mu_j + log W_ij, or for TILTED s (q - nu_i).k_hat_ij + s nu_i.mu_j +
  * log W_ij; value u_ij) plus one exact term per key of the retrieved
- * clusters, all in one softmax.  O is written in the input dtype.
+ * clusters, all in one softmax.  O is written in the input dtype (fp32 with
+ * out_f32); all arithmetic before that store is fp32 or wider.
  * Requires 1 <= Cq, Ck <= min(N, 1024), 0 <= topk <= Ck, iters >= 1.
  */
 muse_status muse_attn_fwd(const void *Q, const void *K, const void *V, void *O,
@@ -169,6 +175,17 @@ muse_status muse_attn_fwd_causal(const void *Q, const void *K, const void *V,
                                  void *ws, size_t ws_bytes, cudaStream_t stream);
 
 const char *muse_status_string(muse_status status);
+
+/* Per-kernel timing, for benchmarks (instrumentation only; no paper
+ * counterpart).  While enabled, every kernel launched by the library is
+ * bracketed by two CUDA events recorded on its launch stream.
+ * muse_profile_read() waits for the recorded events, writes up to `cap`
+ * entries -- kernel name (NUL-terminated, at most name_stride bytes, into
+ * names + i * name_stride), launch count and summed milliseconds -- returns
+ * the number of distinct kernels, and clears the record.  Not thread-safe. */
+void muse_profile_enable(int on);
+int muse_profile_read(char *names, int name_stride, int *launches, double *ms,
+                      int cap);
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char *muse_last_error(void);

@@ -28,9 +28,14 @@ def _built():
 def gpu_acausal(Q, K, V, dtype, C, iters, seed, topk, scale=1.0, mode="dipole", Cq=None):
     q, k, v = to_dev(Q, dtype), to_dev(K, dtype), to_dev(V, dtype)
     O, dbg = muse.muse_attn_fwd(q, k, v, Cq=Cq or C, Ck=C, iters=iters, seed=seed, topk=topk,
-                                scale=scale, mode=mode, debug=True)
+                                scale=scale, mode=mode, debug=True, out_dtype=torch.float32)
+    Ob = muse.muse_attn_fwd(q, k, v, Cq=Cq or C, Ck=C, iters=iters, seed=seed, topk=topk,
+                            scale=scale, mode=mode)
     torch.cuda.synchronize()
-    return O.float().cpu().numpy(), {n: t.cpu().numpy() for n, t in dbg.items()}
+    # the input-dtype output is the fp32 result rounded once
+    assert torch.equal(Ob, O.to(Ob.dtype))
+    assert int(dbg["device_error"].item()) == 0
+    return O.cpu().numpy(), {n: t.cpu().numpy() for n, t in dbg.items()}
 
 
 def check_acausal(Q, K, V, dtype, C, iters, seed, topk, scale=1.0, mode="dipole", heads=None,
@@ -183,9 +188,14 @@ def test_muse_summarize():
 def gpu_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale=1.0, mode="dipole"):
     q, k, v = to_dev(Q, dtype), to_dev(K, dtype), to_dev(V, dtype)
     O, dbg = muse.muse_attn_fwd_causal(q, k, v, C=C, block=L, iters=iters, seed=seed, topk=topk,
-                                       scale=scale, mode=mode, debug=True)
+                                       scale=scale, mode=mode, debug=True,
+                                       out_dtype=torch.float32)
+    Ob = muse.muse_attn_fwd_causal(q, k, v, C=C, block=L, iters=iters, seed=seed, topk=topk,
+                                   scale=scale, mode=mode)
     torch.cuda.synchronize()
-    return O.float().cpu().numpy(), {n: t.cpu().numpy() for n, t in dbg.items()}
+    assert torch.equal(Ob, O.to(Ob.dtype))
+    assert int(dbg["device_error"].item()) == 0
+    return O.cpu().numpy(), {n: t.cpu().numpy() for n, t in dbg.items()}
 
 
 def check_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale=1.0, mode="dipole", heads=None):
