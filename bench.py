@@ -158,13 +158,35 @@ def total_algorithmic_flops(work, iters):
 
 
 # ---------------------------------------------------------------------------
+# multi-rank plumbing (one independent layer per rank, no data-path collective)
+# ---------------------------------------------------------------------------
+def rank_data_seed(w, rank: int) -> int:
+    """Each rank draws its own layer of the workload."""
+    return w.data_seed + rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The slowest rank's value (every rank gets it)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(tokens_per_rank: int, world: int, steps: int, max_ms: float) -> float:
+    """Tokens processed by all ranks per second of the slowest rank."""
+    return tokens_per_rank * world * steps / (max_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
 def run_muse(args, w, rank, world, device):
     import clustered_multipole_approximation_b200 as muse
 
     mode = args.mode or w.mode
-    Q, K, V = make_inputs(w, seed=w.data_seed + rank)
+    Q, K, V = make_inputs(w, seed=rank_data_seed(w, rank))
     cast = (lambda x: torch.from_numpy(x).to(torch.bfloat16)) if w.dtype == "bf16" else torch.from_numpy
     hq, hk, hv = cast(Q).pin_memory(), cast(K).pin_memory(), cast(V).pin_memory()
     q, k, v = hq.to(device), hk.to(device), hv.to(device)
@@ -221,15 +243,12 @@ def run_muse(args, w, rank, world, device):
     muse.profile_enable(False)
     prof = muse.profile_read()
     clocks = clk.stop()
-    total_ms = sum(a.elapsed_time(b) for a, b in evs)
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, device)
     if world > 1:
-        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
         torch.distributed.barrier()
     torch.cuda.synchronize()
     tokens = w.B * w.N
-    value = tokens * world * args.steps / (total_ms / 1e3)
+    value = whole_job_throughput(tokens, world, args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
     # end to end through the public API: host inputs in, host output back
@@ -249,11 +268,8 @@ def run_muse(args, w, rank, world, device):
         torch.cuda.synchronize()
         if i >= args.warmup:
             e2e_ms += e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": tokens * world * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
+    e2e = {"value": whole_job_throughput(tokens, world, args.steps, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": int(hq.numel() * hq.element_size() * 1 + hk.numel() * hk.element_size()
                                      + hv.numel() * hv.element_size()),
            "d2h_bytes_per_step": int(ho.numel() * ho.element_size())}

@@ -36,6 +36,19 @@ __device__ inline uint64_t splitmix64_next(uint64_t& state) {
 
 constexpr int kHashSize = 2 * kMaxC;  // open addressing, load <= 1/2
 
+// r mod m for a 32-bit m, exactly: reduce the high word first, then the
+// remaining < m * 2^32 by a double-precision quotient estimate and an exact
+// integer correction (the generic 64-bit remainder is a long software loop).
+__device__ inline uint32_t mod_u64_u32(uint64_t r, uint32_t m) {
+  if (m < (1u << 16)) return (uint32_t)(r % m);
+  const uint64_t t = ((uint64_t)((uint32_t)(r >> 32) % m) << 32) | (uint32_t)r;
+  uint64_t q = (uint64_t)((double)t / (double)m);
+  long long rem = (long long)(t - q * (uint64_t)m);
+  while (rem < 0) rem += m;
+  while (rem >= (long long)m) rem -= m;
+  return (uint32_t)rem;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(128) kmeans_init_kernel(RoleGeo g, KState ks, const float* init) {
   __shared__ int hkey[kHashSize];
@@ -55,7 +68,7 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(RoleGeo g, KState ks, 
       const int n = p.s;
       for (int c = 0; c < C; ++c) {
         uint64_t r = splitmix64_next(st);
-        int j = c + (int)(r % (uint64_t)(n - c));
+        int j = c + (int)mod_u64_u32(r, (uint32_t)(n - c));
         // value currently at position j (identity unless swapped before)
         int h = j & (kHashSize - 1), vj = j;
         while (hkey[h] >= 0) {
@@ -254,7 +267,22 @@ __global__ void __launch_bounds__(256) kmeans_reduce_kernel(RoleGeo g, KState ks
     double s[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) s[r] = 0.0;
-    for (int m = b; m < e; ++m) {
+    constexpr int U = 8;  // members loaded ahead; the adds stay in token order
+    int m = b;
+    for (; m + U <= e; m += U) {
+      float v[U][R];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const T* row = X + (p.row0 + perm[m + u]) * D;
+#pragma unroll
+        for (int r = 0; r < R; ++r) v[u][r] = ld<T>(row + lane + 32 * r);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int r = 0; r < R; ++r) s[r] = __dadd_rn(s[r], (double)v[u][r]);
+    }
+    for (; m < e; ++m) {
       const T* row = X + (p.row0 + perm[m]) * D;
 #pragma unroll
       for (int r = 0; r < R; ++r) s[r] = __dadd_rn(s[r], (double)ld<T>(row + lane + 32 * r));

@@ -153,6 +153,19 @@ def test_muse_cluster_seeded(dtype):
                 np.testing.assert_allclose(c[b, h], rc, rtol=2e-7, atol=1e-7)
 
 
+@pytest.mark.parametrize("C,D,N", [(1, 64, 300), (16, 64, 500), (100, 128, 1000), (256, 64, 2000),
+                                   (300, 128, 1500), (1024, 64, 3000)])
+def test_muse_cluster_bf16_cluster_counts(C, D, N):
+    # C > 256 exercises several tensor-core passes per tile
+    X, _, _ = clustered_qkv(1, 2, 2, N, D, 24, 0.3, 0.0, "bf16", 43 + C)
+    a, c, n = muse.muse_cluster(to_dev(X, "bf16"), C, 3, 99, role=1)
+    for h in range(2):
+        ra, rc, rn, _ = oracle.kmeans(X[0, h], C, 3, 99, h, 1)
+        assert_assign_match(a[0, h].cpu().numpy(), ra, what=f"assign h{h}")
+        assert (n[0, h].cpu().numpy() == rn).all()
+        np.testing.assert_allclose(c[0, h].cpu().numpy(), rc, rtol=2e-7, atol=1e-7)
+
+
 def test_muse_cluster_one_round_from_given_centroids():
     X, _, _ = clustered_qkv(1, 2, 2, 1500, 128, 20, 0.3, 0.0, "bf16", 41)
     rng = np.random.default_rng(1)
