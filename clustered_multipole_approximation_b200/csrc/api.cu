@@ -1,6 +1,7 @@
 // C ABI of libmuse: argument checks, workspace plan, and the launch sequence
 // of each entry point.  Everything runs on the caller's stream; nothing here
 // allocates, frees or synchronises.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdio.h>
 
@@ -127,6 +128,7 @@ struct AttnPlan {
 
 struct AttnLayout {
   int* err;
+  __half* V16;
   RoleGeo qg, kg;
   KState qs, ks;
   Stage1 s1;
@@ -185,15 +187,23 @@ AttnLayout layout(const muse_shape* sh, const muse_params* pr, bool causal, cons
   L.ks.err = L.qs.err = L.err;
   L.nq = L.qs.nprob;
   const size_t cc = (size_t)pr->Cq * pr->Ck;
-  const size_t per = cc * 4 * 2 + cc * sh->D * 4 * (pr->mode == MUSE_TILTED ? 2 : 1);
+  const size_t per = cc * 4 * 2 + cc * sh->D * 4 * (pr->mode == MUSE_TILTED ? 2 : 1);  // upper bound
   size_t wave = L.nq;
   if (causal && per * wave > kStage1Budget) wave = kStage1Budget / per;
   if (wave < 1) wave = 1;
   L.wave = (int)wave;
   L.s1.logW = cv.take<float>(wave * cc * 4);
   L.s1.fbias = cv.take<float>(wave * cc * 4);
-  L.s1.U = cv.take<float>(wave * cc * sh->D * 4);
-  L.s1.Kf = pr->mode == MUSE_TILTED ? cv.take<float>(wave * cc * sh->D * 4) : nullptr;
+  const bool tilted = pr->mode == MUSE_TILTED;
+  if (dt == 0) {
+    L.s1.Uh = cv.take<__half>(wave * cc * sh->D * 2);
+    L.s1.Kfh = tilted ? cv.take<__nv_bfloat16>(wave * cc * sh->D * 2) : nullptr;
+    L.s1.Kfl = tilted ? cv.take<__nv_bfloat16>(wave * cc * sh->D * 2) : nullptr;
+    L.V16 = cv.take<__half>((size_t)sh->B * sh->Hkv * sh->N * sh->D * 2);
+  } else {
+    L.s1.U = cv.take<float>(wave * cc * sh->D * 4);
+    L.s1.Kf = tilted ? cv.take<float>(wave * cc * sh->D * 4) : nullptr;
+  }
   const int k1 = pr->topk > 0 ? pr->topk : 1;
   L.s1.sel = cv.take<int>((size_t)L.nq * pr->Cq * k1 * 4);
   L.s1.nsel = cv.take<int>((size_t)L.nq * pr->Cq * 4);
@@ -217,6 +227,7 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   a.qs = L.qs;
   a.ks = L.ks;
   a.V = V;
+  a.V16 = L.V16;
   a.O = causal ? nullptr : O;
   a.out_f32 = sh->out_f32 ? 1 : 0;
   a.part = L.part;
@@ -232,11 +243,23 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   if (a.n_exact && causal)
     cudaMemsetAsync(a.n_exact, 0, (size_t)sh->B * sh->Hq * sh->N * 8, st);
   cudaMemsetAsync(L.err, 0, 4, st);
+  if (L.nq > 0 && L.V16) run_bf16_to_half(V, L.V16, (size_t)sh->B * sh->Hkv * sh->N * sh->D, st);
   if (L.nq > 0) {
     cudaMemsetAsync(L.ks.arrive, 0, (size_t)L.ks.nprob * 4, st);
     cudaMemsetAsync(L.qs.arrive, 0, (size_t)L.qs.nprob * 4, st);
-    run_kmeans(L.kg, L.ks, pr->iters, nullptr, st);
-    run_kmeans(L.qg, L.qs, pr->iters, nullptr, st);
+    run_kmeans_init(L.kg, L.ks, nullptr, st);
+    run_kmeans_init(L.qg, L.qs, nullptr, st);
+    const RoleGeo gs[2] = {L.kg, L.qg};
+    const KState kss[2] = {L.ks, L.qs};
+    bool fused;
+    {
+      ProfScope ps(st, "kmeans_fused");
+      fused = launch_kmeans_fused(gs, kss, 2, pr->iters, st);
+    }
+    if (!fused) {
+      run_kmeans_rounds(L.kg, L.ks, pr->iters, st);
+      run_kmeans_rounds(L.qg, L.qs, pr->iters, st);
+    }
     for (int q0 = 0; q0 < L.nq; q0 += L.wave) {
       const int n = L.nq - q0 < L.wave ? L.nq - q0 : L.wave;
       run_blocks(a, L.s1, q0, n, st);
@@ -307,7 +330,13 @@ muse_status muse_cluster(const void* X, muse_dtype dtype, int B, int H, int N, i
   ks.err = err;
   cudaMemsetAsync(err, 0, 4, stream);
   cudaMemsetAsync(ks.arrive, 0, (size_t)ks.nprob * 4, stream);
-  run_kmeans(g, ks, iters, init, stream);
+  run_kmeans_init(g, ks, init, stream);
+  bool fused;
+  {
+    ProfScope ps(stream, "kmeans_fused");
+    fused = launch_kmeans_fused(&g, &ks, 1, iters, stream);
+  }
+  if (!fused) run_kmeans_rounds(g, ks, iters, stream);
   cudaMemcpyAsync(assign, ks.assign, (size_t)ks.ntok * 4, cudaMemcpyDeviceToDevice, stream);
   cudaMemcpyAsync(centroids, ks.cent32, (size_t)ks.nprob * C * D * 4, cudaMemcpyDeviceToDevice, stream);
   if (counts) cudaMemcpyAsync(counts, ks.counts, (size_t)ks.nprob * C * 4, cudaMemcpyDeviceToDevice, stream);

@@ -1,6 +1,7 @@
 // Host-side launchers shared between the translation units of libmuse.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -19,8 +20,12 @@ struct ProfScope {
 struct Stage1 {
   float* logW;    // [nq][Cq][Ck]  log W_ij, -inf for empty key clusters
   float* fbias;   // [nq][Cq][Ck]  far-field logit offset (log W, plus the tilt term)
-  float* U;       // [nq][Cq][Ck][D] summary values u_ij
-  float* Kf;      // [nq][Cq][Ck][D] far-field key rows (TILTED only: k_hat_ij)
+  // fp32 inputs: fp32 tables; bf16 inputs: the tensor-core operand forms
+  float* U;       // [nq][Cq][Ck][D] summary values u_ij (fp32 path)
+  float* Kf;      // [nq][Cq][Ck][D] far-field key rows, TILTED only: k_hat_ij (fp32 path)
+  __half* Uh;     // [nq][Cq][Ck][D] u_ij in fp16 (bf16 path)
+  __nv_bfloat16* Kfh;  // [nq][Cq][Ck][D] bf16 hi / lo split of k_hat_ij (bf16 path, TILTED)
+  __nv_bfloat16* Kfl;
   int* sel;       // [nq_total][Cq][topk]
   int* nsel;      // [nq_total][Cq]
 };
@@ -29,6 +34,7 @@ struct AttnArgs {
   RoleGeo qg, kg;     // query and key geometry
   KState qs, ks;      // their k-means state
   const void* V;
+  const __half* V16;  // fp16 copy of V (bf16 inputs; the PV operand)
   void* O;            // acausal: final output
   int out_f32;        // O is fp32 (else the input dtype)
   float* part;        // causal: [nq_total tokens][D + 1] partial (o, lse)
@@ -43,11 +49,25 @@ struct AttnArgs {
 void run_kmeans(const RoleGeo& g, const KState& ks, int iters, const float* init,
                 cudaStream_t st);
 
+// Seeded (or given) start centroids for a problem set.
+void run_kmeans_init(const RoleGeo& g, const KState& ks, const float* init, cudaStream_t st);
+
+// All Lloyd rounds of up to two problem sets in one persistent launch
+// (thread-block clusters, bf16 inputs); false if these sets are not covered.
+bool launch_kmeans_fused(const RoleGeo* gs, const KState* kss, int nsets, int iters,
+                         cudaStream_t st);
+
+// Lloyd rounds one launch sequence at a time (any dtype / size).
+void run_kmeans_rounds(const RoleGeo& g, const KState& ks, int iters, cudaStream_t st);
+
 // Tensor-core (tcgen05) assignment screen for bf16 inputs.
 void launch_assign_tc(const RoleGeo& g, const KState& ks, cudaStream_t st);
 
 // Stage 1 + selection + stage 2 for query problems [qp0, qp0 + nqp).
 void run_blocks(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
+
+// fp16 copy of a bf16 tensor (n elements, n % 8 == 0).
+void run_bf16_to_half(const void* src, __half* dst, size_t n, cudaStream_t st);
 
 // Stage 2 on tensor cores (bf16 inputs).
 void run_stage2_mma(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);

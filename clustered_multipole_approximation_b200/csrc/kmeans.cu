@@ -50,7 +50,7 @@ __device__ inline uint32_t mod_u64_u32(uint64_t r, uint32_t m) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(128) kmeans_init_kernel(RoleGeo g, KState ks, const float* init) {
+__global__ void __launch_bounds__(256) kmeans_init_kernel(RoleGeo g, KState ks, const float* init) {
   __shared__ int hkey[kHashSize];
   __shared__ int hval[kHashSize];
   __shared__ int pick[kMaxC];
@@ -63,12 +63,20 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(RoleGeo g, KState ks, 
   if (init == nullptr) {
     for (int i = threadIdx.x; i < kHashSize; i += blockDim.x) hkey[i] = -1;
     __syncthreads();
+    // splitmix64 is counter based: draw c uses state0 + (c + 1) * gamma, so
+    // every swap target j_c is computed in parallel; only the swaps themselves
+    // are applied in order below.
+    const uint64_t st0 = g.seed + 0x9E3779B97F4A7C15ULL * (2ULL * p.sid + (uint64_t)g.role + 1ULL);
+    const int n = p.s;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      uint64_t st = st0 + 0x9E3779B97F4A7C15ULL * (uint64_t)c;
+      const uint64_t r = splitmix64_next(st);
+      pick[c] = c + (int)mod_u64_u32(r, (uint32_t)(n - c));
+    }
+    __syncthreads();
     if (threadIdx.x == 0) {
-      uint64_t st = g.seed + 0x9E3779B97F4A7C15ULL * (2ULL * p.sid + (uint64_t)g.role + 1ULL);
-      const int n = p.s;
       for (int c = 0; c < C; ++c) {
-        uint64_t r = splitmix64_next(st);
-        int j = c + (int)mod_u64_u32(r, (uint32_t)(n - c));
+        const int j = pick[c];
         // value currently at position j (identity unless swapped before)
         int h = j & (kHashSize - 1), vj = j;
         while (hkey[h] >= 0) {
@@ -90,41 +98,51 @@ __global__ void __launch_bounds__(128) kmeans_init_kernel(RoleGeo g, KState ks, 
       }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < C * D; i += blockDim.x) {
-      int c = i / D, d = i - c * D;
-      double v = (double)ld<T>(X + (p.row0 + pick[c]) * D + d);
-      c64[i] = v;
-      c32[i] = (float)v;
-    }
-  } else {
-    const float* src = init + (size_t)p.bh * g.C * D;  // muse_cluster: one problem per bh
-    for (int i = threadIdx.x; i < C * D; i += blockDim.x) {
-      c64[i] = (double)src[i];
-      c32[i] = src[i];
-    }
   }
-  __syncthreads();
-  // centroid norms for the screen bounds, and the bf16 split for the tensor cores
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int c = warp; c < C; c += blockDim.x >> 5) {
-    float s = 0.f;
-    double s2 = 0.0;
-    for (int d = lane; d < D; d += 32) {
-      const size_t i = (size_t)c * D + d;
-      float v = c32[i];
-      s = fmaf(v, v, s);
-      s2 += c64[i] * c64[i];
-      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-      ks.cbf_hi[(size_t)pid * g.C * D + i] = hi;
-      ks.cbf_lo[(size_t)pid * g.C * D + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
-    }
-    for (int o = 16; o; o >>= 1) {
-      s += __shfl_xor_sync(0xffffffffu, s, o);
-      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-    }
-    if (lane == 0) {
-      ks.cnorm[(size_t)pid * g.C + c] = sqrtf(s) * 1.0001f;
-      ks.cn2[(size_t)pid * g.C + c] = (float)s2;
+  // one warp per centroid row, four rows per step (loads issued together):
+  // fp64/fp32 copies, the bf16 split for the tensor cores, and the norms
+  const float* src = init ? init + (size_t)p.bh * g.C * D : nullptr;  // muse_cluster: one problem per bh
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  constexpr int RR = 4;
+  for (int c0 = warp * RR; c0 < C; c0 += nw * RR) {
+    float v[RR][4];
+#pragma unroll
+    for (int u = 0; u < RR; ++u)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int c = c0 + u, d = lane + 32 * r;
+        v[u][r] = 0.f;
+        if (c < C && d < D)
+          v[u][r] = src ? src[(size_t)c * D + d] : ld<T>(X + (p.row0 + pick[c]) * D + d);
+      }
+#pragma unroll
+    for (int u = 0; u < RR; ++u) {
+      const int c = c0 + u;
+      if (c >= C) break;
+      float s = 0.f;
+      double s2 = 0.0;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int d = lane + 32 * r;
+        if (d >= D) break;
+        const size_t i = (size_t)c * D + d;
+        const float x = v[u][r];
+        c64[i] = (double)x;
+        c32[i] = x;
+        s = fmaf(x, x, s);
+        s2 += (double)x * (double)x;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+        ks.cbf_hi[(size_t)pid * g.C * D + i] = hi;
+        ks.cbf_lo[(size_t)pid * g.C * D + i] = __float2bfloat16_rn(x - __bfloat162float(hi));
+      }
+      for (int o = 16; o; o >>= 1) {
+        s += __shfl_xor_sync(0xffffffffu, s, o);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+      }
+      if (lane == 0) {
+        ks.cnorm[(size_t)pid * g.C + c] = sqrtf(s) * 1.0001f;
+        ks.cn2[(size_t)pid * g.C + c] = (float)s2;
+      }
     }
   }
 }
@@ -344,12 +362,20 @@ static void launch_round(const RoleGeo& g, const KState& ks, cudaStream_t st) {
 }
 
 template <typename T>
-static void run_kmeans_t(const RoleGeo& g, const KState& ks, int iters, const float* init,
-                         cudaStream_t st) {
-  {
-    ProfScope ps(st, "kmeans_init");
-    kmeans_init_kernel<T><<<ks.nprob, 128, 0, st>>>(g, ks, init);
-  }
+static void init_t(const RoleGeo& g, const KState& ks, const float* init, cudaStream_t st) {
+  ProfScope ps(st, "kmeans_init");
+  kmeans_init_kernel<T><<<ks.nprob, 256, 0, st>>>(g, ks, init);
+}
+
+void run_kmeans_init(const RoleGeo& g, const KState& ks, const float* init, cudaStream_t st) {
+  if (g.dtype == 0)
+    init_t<__nv_bfloat16>(g, ks, init, st);
+  else
+    init_t<float>(g, ks, init, st);
+}
+
+template <typename T>
+static void rounds_t(const RoleGeo& g, const KState& ks, int iters, cudaStream_t st) {
   for (int it = 0; it < iters; ++it) {
     if (g.D == 64)
       launch_round<T, 64>(g, ks, st);
@@ -358,11 +384,16 @@ static void run_kmeans_t(const RoleGeo& g, const KState& ks, int iters, const fl
   }
 }
 
-void run_kmeans(const RoleGeo& g, const KState& ks, int iters, const float* init, cudaStream_t st) {
+void run_kmeans_rounds(const RoleGeo& g, const KState& ks, int iters, cudaStream_t st) {
   if (g.dtype == 0)
-    run_kmeans_t<__nv_bfloat16>(g, ks, iters, init, st);
+    rounds_t<__nv_bfloat16>(g, ks, iters, st);
   else
-    run_kmeans_t<float>(g, ks, iters, init, st);
+    rounds_t<float>(g, ks, iters, st);
+}
+
+void run_kmeans(const RoleGeo& g, const KState& ks, int iters, const float* init, cudaStream_t st) {
+  run_kmeans_init(g, ks, init, st);
+  run_kmeans_rounds(g, ks, iters, st);
 }
 
 }  // namespace muse

@@ -73,9 +73,16 @@ __device__ inline void assign_tail(const RoleGeo& g, const KState& ks, const Pro
   int* ph = ks.hist + (size_t)p.tile0 * g.C;
   int* cnt = ks.counts + (size_t)pid * g.C;
   int* off = ks.off + (size_t)pid * (g.C + 1);
+  constexpr int U = 16;  // tile counts fetched per round trip
   for (int c = tid; c < C; c += blockDim.x) {
     int tot = 0;
-    for (int t = 0; t < ntp; ++t) tot += __ldcg(ph + (size_t)t * g.C + c);
+    for (int t0 = 0; t0 < ntp; t0 += U) {
+      int v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) v[u] = (t0 + u < ntp) ? __ldcg(ph + (size_t)(t0 + u) * g.C + c) : 0;
+#pragma unroll
+      for (int u = 0; u < U; ++u) tot += v[u];
+    }
     hist[c] = tot;
     cnt[c] = tot;
   }
@@ -94,11 +101,15 @@ __device__ inline void assign_tail(const RoleGeo& g, const KState& ks, const Pro
   __syncthreads();
   for (int c = tid; c < C; c += blockDim.x) {
     int run = hist[c];
-    for (int t = 0; t < ntp; ++t) {
-      int* h = ph + (size_t)t * g.C + c;
-      int v = __ldcg(h);
-      *h = run;
-      run += v;
+    for (int t0 = 0; t0 < ntp; t0 += U) {
+      int v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) v[u] = (t0 + u < ntp) ? __ldcg(ph + (size_t)(t0 + u) * g.C + c) : 0;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (t0 + u < ntp) ph[(size_t)(t0 + u) * g.C + c] = run;
+        run += v[u];
+      }
     }
   }
 }

@@ -21,6 +21,7 @@
 // and the far-field logit of a query q of cluster i is
 //   s q.mu_j + log W_ij                                   (MONOPOLE, DIPOLE)
 //   s q.k_hat_ij + s nu_i.(mu_j - k_hat_ij) + log W_ij    (TILTED)
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "common.cuh"
@@ -44,6 +45,21 @@ __device__ inline int kv_problem(const AttnArgs& a, int qpid) {
 // (1 + a for DIPOLE, exp(a - max) for TILTED) and the weighted sums over the
 // members, giving u_ij, log W_ij, the far-field key row and logit offset.
 // ----------------------------------------------------------------------------
+// Stage-1 table stores in the form the stage-2 kernel of the input dtype reads.
+__device__ inline void put_u(const Stage1& s1, size_t i, float v) {
+  if (s1.Uh) s1.Uh[i] = __float2half_rn(v);
+  else s1.U[i] = v;
+}
+__device__ inline void put_kf(const Stage1& s1, size_t i, float v) {
+  if (s1.Kfh) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    s1.Kfh[i] = hi;
+    s1.Kfl[i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+  } else {
+    s1.Kf[i] = v;
+  }
+}
+
 constexpr int kS1T = 256;  // threads
 constexpr int kS1M = 128;  // members per staged chunk
 constexpr int kS1I = 32;   // query clusters per pass
@@ -120,7 +136,7 @@ __global__ void __launch_bounds__(kS1T) stage1_kernel(AttnArgs a, Stage1 s1, int
     __syncthreads();
     for (int idx = tid; idx < pq.C * D; idx += kS1T) {
       const int i = idx / D, d = idx - i * D;
-      s1.U[(ij0 + (size_t)i * Ck) * D + d] = red[0][d];
+      put_u(s1, (ij0 + (size_t)i * Ck) * D + d, red[0][d]);
     }
     for (int i = tid; i < pq.C; i += kS1T) {
       s1.logW[ij0 + (size_t)i * Ck] = lognj;
@@ -216,7 +232,7 @@ __global__ void __launch_bounds__(kS1T) stage1_kernel(AttnArgs a, Stage1 s1, int
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const int ii = g0 + GROUPS * r;
-        if (ii < ic) s1.U[(ij0 + (size_t)(i0 + ii) * Ck) * D + e] = accU[r] * inv;
+        if (ii < ic) put_u(s1, (ij0 + (size_t)(i0 + ii) * Ck) * D + e, accU[r] * inv);
       }
       for (int ii = tid; ii < ic; ii += kS1T) {
         s1.logW[ij0 + (size_t)(i0 + ii) * Ck] = lognj;
@@ -231,8 +247,8 @@ __global__ void __launch_bounds__(kS1T) stage1_kernel(AttnArgs a, Stage1 s1, int
         const float inv = 1.f / zrun[ii];
         const float kh = accK[r] * inv;
         const size_t ij = ij0 + (size_t)(i0 + ii) * Ck;
-        s1.U[ij * D + e] = accU[r] * inv;
-        s1.Kf[ij * D + e] = mu[e] + kh;
+        put_u(s1, ij * D + e, accU[r] * inv);
+        put_kf(s1, ij * D + e, mu[e] + kh);
         red[ii][e] = nu[ii][e] * kh;
       }
       __syncthreads();

@@ -7,11 +7,13 @@
 //     Core Mechanisms: Stage 2 (Refinement));
 //   - exact attention over every key of the retrieved clusters (same page,
 //     Exact Attention).
-// Each warp owns 16 query rows; S = Q K^T runs as bf16 m16n8k16 MMAs with fp32
-// accumulation.  bf16 query and key rows are exact; a far-field key row (fp32)
-// is split into hi + lo bf16 parts and contracted twice, leaving a residual of
-// 2^-18 relative.  P and V enter the PV product as fp16 (V bf16 -> fp16 is
-// exact in fp16's normal range; u_ij rounds to 11 bits), accumulating in fp32.
+// Eight warps own 16 query rows each (128 queries per pass).  S = Q K^T runs
+// as bf16 m16n8k16 MMAs with fp32 accumulation: bf16 query and key rows are
+// exact, a far-field key row (fp32) enters as its bf16 hi + lo split (two
+// MMAs, residual 2^-18 relative).  P and V enter the PV product as fp16 (the
+// fp16 copy of V is exact in fp16's normal range; u_ij is rounded to 11 bits),
+// accumulating in fp32.  Key blocks of 64 rows stream through shared memory
+// with cp.async, two blocks in flight.
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -22,9 +24,9 @@ namespace muse {
 
 namespace {
 
-constexpr int kMQ = 64;      // queries per pass (4 warps x 16 rows)
+constexpr int kMQ = 128;     // queries per pass (8 warps x 16 rows)
 constexpr int kMK = 64;      // key rows per block
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 
 __device__ inline int kvp(const AttnArgs& a, int qpid) {
   const int ppb = a.qg.lv.pairs_per_bh;
@@ -37,6 +39,15 @@ __device__ inline int kvp(const AttnArgs& a, int qpid) {
 __device__ inline uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+// 16-byte async copy; src_bytes = 0 fills the destination with zeros.
+__device__ inline void cp16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes));
+}
+__device__ inline void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ inline void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
 __device__ inline void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -66,18 +77,35 @@ __device__ inline void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// 2^x on the special-function unit (PTX ex2.approx, relative error ~2^-22;
+// ex2(-inf) = 0).
+__device__ inline float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Running maxima start at a finite floor so that fully masked blocks need no
+// special case: exp2(-inf - floor) = 0 and exp2(floor - floor) = 1.
+constexpr float kMaxFloor = -1.0e30f;
+
 __device__ inline uint32_t pack_h2(float x, float y) {
   __half2 h = __floats2half2_rn(x, y);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
 template <int D>
-struct Smem2 {
-  __nv_bfloat16 q[kMQ][D + 8];
+struct KBuf {
   __nv_bfloat16 k[kMK][D + 8];    // exact keys, or the hi part of far keys
   __nv_bfloat16 k2[kMK][D + 8];   // lo part of far keys
   __half v[kMK][D + 8];
   float bias[kMK];
+};
+
+template <int D>
+struct Smem2 {
+  __nv_bfloat16 q[kMQ][D + 8];
+  KBuf<D> buf[2];
   unsigned char inR[kMaxC];
   int sel[kMaxC];
 };
@@ -89,12 +117,35 @@ size_t stage2_mma_smem() {
   return sizeof(Smem2<D>);
 }
 
+__global__ void bf16_to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
+                                    size_t n8) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+    uint4 o;
+    __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) h[u] = __float22half2_rn(__bfloat1622float2(b[u]));
+    reinterpret_cast<uint4*>(dst)[i] = o;
+  }
+}
+
+void run_bf16_to_half(const void* src, __half* dst, size_t n, cudaStream_t st) {
+  ProfScope ps(st, "v_to_half");
+  const size_t n8 = n / 8;
+  const int blocks = (int)((n8 + 255) / 256 < 148 * 8 ? (n8 + 255) / 256 : 148 * 8);
+  bf16_to_half_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), dst, n8);
+}
+
 template <typename TO, int D>
-__global__ void __launch_bounds__(kThreads) stage2_mma_kernel(AttnArgs a, Stage1 s1, int qp0) {
+__global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(AttnArgs a, Stage1 s1,
+                                                                               int qp0) {
   extern __shared__ __align__(16) unsigned char sm2_raw[];
   Smem2<D>& sm = *reinterpret_cast<Smem2<D>*>(sm2_raw);
   constexpr int KD = D / 16;   // k-steps over the head dimension
   constexpr int ND = D / 8;    // n-tiles over the head dimension
+  constexpr int CH = D / 8;    // 16-byte chunks per row
   const int lq = blockIdx.x, qpid = qp0 + lq, i = blockIdx.y;
   const Prob pq = prob_of(a.qg, qpid);
   if (i >= pq.C) return;
@@ -117,186 +168,186 @@ __global__ void __launch_bounds__(kThreads) stage2_mma_kernel(AttnArgs a, Stage1
   const int* kc = a.ks.counts + (size_t)kpid * Ck;
   const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
   long long nexact = 0;
-  for (int r = 0; r < nsel; ++r) nexact += kc[sm.sel[r]];
+  int nblk_exact = 0;
+  for (int r = 0; r < nsel; ++r) {
+    nexact += kc[sm.sel[r]];
+    nblk_exact += cdiv(kc[sm.sel[r]], kMK);
+  }
+  const int nblk_far = cdiv(pk.C, kMK);
+  const int nblk = nblk_far + nblk_exact;
 
   const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.qg.X);
   const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.kg.X);
-  const __nv_bfloat16* V = static_cast<const __nv_bfloat16*>(a.V);
+  const __half* V16 = a.V16;
   const int qo = a.qs.off[(size_t)qpid * (Cq + 1) + i];
   const int* qperm = a.qs.perm + pq.slot0;
   const int* kperm = a.ks.perm + pk.slot0;
   const size_t ij0 = ((size_t)lq * Cq + i) * Ck;
   const bool tilted = a.mode == 2;
   const float sl2 = a.scale * 1.4426950408889634f;  // logits in base-2 units
+  const __nv_bfloat16* khi = tilted ? s1.Kfh + ij0 * D : a.ks.cbf_hi + (size_t)kpid * Ck * D;
+  const __nv_bfloat16* klo = tilted ? s1.Kfl + ij0 * D : a.ks.cbf_lo + (size_t)kpid * Ck * D;
+  const __half* uh = s1.Uh + ij0 * D;
 
-  for (int c0 = 0; c0 < nqi; c0 += kMQ) {
-    const int nq = imin(kMQ, nqi - c0);
-    __syncthreads();
-    // gather the chunk's query rows (16-byte pieces), zero rows past the end
-    for (int e = tid; e < kMQ * (D / 8); e += kThreads) {
-      const int r = e / (D / 8), c = (e % (D / 8)) * 8;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (r < nq) {
-        const long long row = pq.row0 + qperm[qo + c0 + r];
-        val = *reinterpret_cast<const uint4*>(Q + row * D + c);
-      }
-      *reinterpret_cast<uint4*>(&sm.q[r][c]) = val;
-    }
-    __syncthreads();
-    uint32_t qa[KD][4];
-#pragma unroll
-    for (int kk = 0; kk < KD; ++kk) {
-      const int row = warp * 16 + (lane & 15), col = kk * 16 + (lane >> 4) * 8;
-      ldsm_x4(smem_u32(&sm.q[row][col]), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-    }
-    float o[ND][4];
-#pragma unroll
-    for (int n = 0; n < ND; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-
-    // one block of up to 64 staged key rows
-    auto consume = [&](bool two_part) {
-      float sc[kMK / 8][4];
-#pragma unroll
-      for (int n = 0; n < kMK / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < KD; ++kk) {
-#pragma unroll
-        for (int np = 0; np < kMK / 16; ++np) {
-          const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-          const int col = kk * 16 + ((lane >> 3) & 1) * 8;
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(smem_u32(&sm.k[key][col]), b0, b1, b2, b3);
-          mma_bf16(sc[2 * np], qa[kk], b0, b1);
-          mma_bf16(sc[2 * np + 1], qa[kk], b2, b3);
-          if (two_part) {
-            ldsm_x4(smem_u32(&sm.k2[key][col]), b0, b1, b2, b3);
-            mma_bf16(sc[2 * np], qa[kk], b0, b1);
-            mma_bf16(sc[2 * np + 1], qa[kk], b2, b3);
-          }
-        }
-      }
-      // logits (base 2), row maxima over this block
-      float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-      for (int n = 0; n < kMK / 8; ++n) {
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int col = n * 8 + 2 * t4 + (h & 1);
-          const float lg = fmaf(sl2, sc[n][h], sm.bias[col]);
-          sc[n][h] = lg;
-          mx[h >> 1] = fmaxf(mx[h >> 1], lg);
-        }
-      }
-      float scale[2];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-        const float mn = fmaxf(mrow[r], mx[r]);
-        scale[r] = (mrow[r] == -INFINITY) ? 0.f : exp2f(mrow[r] - mn);
-        mrow[r] = mn;
-      }
-      float rs[2] = {0.f, 0.f};
-#pragma unroll
-      for (int n = 0; n < kMK / 8; ++n) {
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float m = mrow[h >> 1];
-          const float p = (m == -INFINITY) ? 0.f : exp2f(sc[n][h] - m);
-          sc[n][h] = p;
-          rs[h >> 1] += p;
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
-        rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
-        lrow[r] = lrow[r] * scale[r] + rs[r];
-      }
-#pragma unroll
-      for (int n = 0; n < ND; ++n) {
-        o[n][0] *= scale[0];
-        o[n][1] *= scale[0];
-        o[n][2] *= scale[1];
-        o[n][3] *= scale[1];
-      }
-      // O += P V  (P as fp16 A fragments straight from the S accumulators)
-#pragma unroll
-      for (int kk = 0; kk < kMK / 16; ++kk) {
-        uint32_t pa[4];
-        pa[0] = pack_h2(sc[2 * kk][0], sc[2 * kk][1]);
-        pa[1] = pack_h2(sc[2 * kk][2], sc[2 * kk][3]);
-        pa[2] = pack_h2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-        pa[3] = pack_h2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
-#pragma unroll
-        for (int np = 0; np < ND / 2; ++np) {
-          const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const int col = np * 16 + (lane >> 4) * 8;
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(smem_u32(&sm.v[key][col]), b0, b1, b2, b3);
-          mma_f16(o[2 * np], pa, b0, b1);
-          mma_f16(o[2 * np + 1], pa, b2, b3);
-        }
-      }
-    };
-
-    // far field
-    for (int j0 = 0; j0 < pk.C; j0 += kMK) {
-      __syncthreads();
-      for (int e = tid; e < kMK * (D / 4); e += kThreads) {
-        const int r = e / (D / 4), c = (e % (D / 4)) * 4, j = j0 + r;
+  // block b (far blocks first, then the retrieved clusters' keys) into buf
+  auto issue = [&](int b, KBuf<D>& B) {
+    if (b < nblk_far) {
+      const int j0 = b * kMK;
+      for (int e = tid; e < kMK * CH; e += kThreads) {
+        const int r = e / CH, c = (e % CH) * 8, j = j0 + r;
         const bool live = j < pk.C && kc[j] > 0 && !sm.inR[j];
-        float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), uv = kv;
-        if (live) {
-          const size_t ij = ij0 + j;
-          kv = tilted ? *reinterpret_cast<const float4*>(s1.Kf + ij * D + c)
-                      : *reinterpret_cast<const float4*>(a.ks.cent32 + ((size_t)kpid * Ck + j) * D + c);
-          uv = *reinterpret_cast<const float4*>(s1.U + ij * D + c);
-        }
-        const float kx[4] = {kv.x, kv.y, kv.z, kv.w};
-        const float ux[4] = {uv.x, uv.y, uv.z, uv.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const __nv_bfloat16 hi = __float2bfloat16_rn(kx[u]);
-          sm.k[r][c + u] = hi;
-          sm.k2[r][c + u] = __float2bfloat16_rn(kx[u] - __bfloat162float(hi));
-          sm.v[r][c + u] = __float2half_rn(ux[u]);
-        }
+        const size_t o = (size_t)(live ? j : 0) * D + c;
+        cp16(&B.k[r][c], khi + o, live ? 16 : 0);
+        cp16(&B.k2[r][c], klo + o, live ? 16 : 0);
+        cp16(&B.v[r][c], uh + o, live ? 16 : 0);
       }
       for (int r = tid; r < kMK; r += kThreads) {
         const int j = j0 + r;
         const bool live = j < pk.C && kc[j] > 0 && !sm.inR[j];
-        sm.bias[r] = live ? s1.fbias[ij0 + j] * 1.4426950408889634f : -INFINITY;
+        B.bias[r] = live ? s1.fbias[ij0 + j] * 1.4426950408889634f : -INFINITY;
+      }
+    } else {
+      // locate the exact block: cluster rr of the selection, rows t0..t0+63
+      int rem = b - nblk_far, rr = 0;
+      while (true) {
+        const int nbj = cdiv(kc[sm.sel[rr]], kMK);
+        if (rem < nbj) break;
+        rem -= nbj;
+        ++rr;
+      }
+      const int j = sm.sel[rr], n = kc[j], t0 = rem * kMK, nr = imin(kMK, n - t0);
+      const int base = koff[j] + t0;
+      for (int e = tid; e < kMK * CH; e += kThreads) {
+        const int r = e / CH, c = (e % CH) * 8;
+        const bool live = r < nr;
+        const long long row = pk.row0 + (live ? kperm[base + r] : 0);
+        cp16(&B.k[r][c], K + row * D + c, live ? 16 : 0);
+        cp16(&B.v[r][c], V16 + row * D + c, live ? 16 : 0);
+      }
+      for (int r = tid; r < kMK; r += kThreads) B.bias[r] = r < nr ? 0.f : -INFINITY;
+    }
+    cp_commit();
+  };
+
+  for (int c0 = 0; c0 < nqi; c0 += kMQ) {
+    const int nq = imin(kMQ, nqi - c0);
+    const bool wact = warp * 16 < nq;  // warps with no query rows skip the math
+    __syncthreads();
+    for (int e = tid; e < kMQ * CH; e += kThreads) {
+      const int r = e / CH, c = (e % CH) * 8;
+      const bool live = r < nq;
+      const long long row = pq.row0 + (live ? qperm[qo + c0 + r] : 0);
+      cp16(&sm.q[r][c], Q + row * D + c, live ? 16 : 0);
+    }
+    issue(0, sm.buf[0]);  // commits the query rows with block 0
+    uint32_t qa[KD][4];
+    float o[ND][4];
+#pragma unroll
+    for (int n = 0; n < ND; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float mrow[2] = {kMaxFloor, kMaxFloor}, lrow[2] = {0.f, 0.f};
+
+    for (int b = 0; b < nblk; ++b) {
+      if (b + 1 < nblk) {
+        issue(b + 1, sm.buf[(b + 1) & 1]);
+        cp_wait<1>();
+      } else {
+        cp_wait<0>();
       }
       __syncthreads();
-      consume(true);
-    }
-    // exact retrieval
-    for (int rr = 0; rr < nsel; ++rr) {
-      const int j = sm.sel[rr], b = koff[j], n = kc[j];
-      for (int t0 = 0; t0 < n; t0 += kMK) {
-        const int nr = imin(kMK, n - t0);
-        __syncthreads();
-        for (int e = tid; e < kMK * (D / 8); e += kThreads) {
-          const int r = e / (D / 8), c = (e % (D / 8)) * 8;
-          uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
-          if (r < nr) {
-            const long long row = pk.row0 + kperm[b + t0 + r];
-            kv = *reinterpret_cast<const uint4*>(K + row * D + c);
-            vv = *reinterpret_cast<const uint4*>(V + row * D + c);
-          }
-          *reinterpret_cast<uint4*>(&sm.k[r][c]) = kv;
-          const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(&vv);
+      if (b == 0 && wact) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) sm.v[r][c + u] = __float2half_rn(__bfloat162float(vb[u]));
+        for (int kk = 0; kk < KD; ++kk) {
+          const int row = warp * 16 + (lane & 15), col = kk * 16 + (lane >> 4) * 8;
+          ldsm_x4(smem_u32(&sm.q[row][col]), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
         }
-        for (int r = tid; r < kMK; r += kThreads) sm.bias[r] = r < nr ? 0.f : -INFINITY;
-        __syncthreads();
-        consume(false);
       }
+      const KBuf<D>& B = sm.buf[b & 1];
+      const bool two = b < nblk_far;
+      if (wact) {
+        float sc[kMK / 8][4];
+#pragma unroll
+        for (int n = 0; n < kMK / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KD; ++kk) {
+#pragma unroll
+          for (int np = 0; np < kMK / 16; ++np) {
+            const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+            const int col = kk * 16 + ((lane >> 3) & 1) * 8;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(smem_u32(&B.k[key][col]), b0, b1, b2, b3);
+            mma_bf16(sc[2 * np], qa[kk], b0, b1);
+            mma_bf16(sc[2 * np + 1], qa[kk], b2, b3);
+            if (two) {
+              ldsm_x4(smem_u32(&B.k2[key][col]), b0, b1, b2, b3);
+              mma_bf16(sc[2 * np], qa[kk], b0, b1);
+              mma_bf16(sc[2 * np + 1], qa[kk], b2, b3);
+            }
+          }
+        }
+        float mx[2] = {kMaxFloor, kMaxFloor};
+#pragma unroll
+        for (int n = 0; n < kMK / 8; ++n) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int col = n * 8 + 2 * t4 + (h & 1);
+            const float lg = fmaf(sl2, sc[n][h], B.bias[col]);
+            sc[n][h] = lg;
+            mx[h >> 1] = fmaxf(mx[h >> 1], lg);
+          }
+        }
+        float scale[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+          const float mn = fmaxf(mrow[r], mx[r]);
+          scale[r] = fast_exp2(mrow[r] - mn);
+          mrow[r] = mn;
+        }
+        float rs[2] = {0.f, 0.f};
+#pragma unroll
+        for (int n = 0; n < kMK / 8; ++n) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float p = fast_exp2(sc[n][h] - mrow[h >> 1]);
+            sc[n][h] = p;
+            rs[h >> 1] += p;
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
+          rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
+          lrow[r] = lrow[r] * scale[r] + rs[r];
+        }
+#pragma unroll
+        for (int n = 0; n < ND; ++n) {
+          o[n][0] *= scale[0];
+          o[n][1] *= scale[0];
+          o[n][2] *= scale[1];
+          o[n][3] *= scale[1];
+        }
+#pragma unroll
+        for (int kk = 0; kk < kMK / 16; ++kk) {
+          uint32_t pa[4];
+          pa[0] = pack_h2(sc[2 * kk][0], sc[2 * kk][1]);
+          pa[1] = pack_h2(sc[2 * kk][2], sc[2 * kk][3]);
+          pa[2] = pack_h2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+          pa[3] = pack_h2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+#pragma unroll
+          for (int np = 0; np < ND / 2; ++np) {
+            const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int col = np * 16 + (lane >> 4) * 8;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(smem_u32(&B.v[key][col]), b0, b1, b2, b3);
+            mma_f16(o[2 * np], pa, b0, b1);
+            mma_f16(o[2 * np + 1], pa, b2, b3);
+          }
+        }
+      }
+      __syncthreads();
     }
-    // write the chunk's rows
+    // write the pass's rows
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const int qr = warp * 16 + g + 8 * r;
