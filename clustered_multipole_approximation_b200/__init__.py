@@ -55,7 +55,8 @@ class muse_debug(ctypes.Structure):
 
 EXPORTS = ["muse_workspace_size", "muse_cluster_workspace_size", "muse_cluster", "muse_summarize",
            "muse_attn_fwd", "muse_attn_fwd_causal", "muse_status_string", "muse_last_error",
-           "muse_profile_enable", "muse_profile_read"]
+           "muse_profile_enable", "muse_profile_read", "muse_cluster_static",
+           "muse_cluster_static_capacity"]
 
 _lib = None
 
@@ -89,6 +90,11 @@ def load_library(path: str = LIB_PATH):
     lib.muse_status_string.argtypes = [i32]
     lib.muse_last_error.restype = ctypes.c_char_p
     lib.muse_last_error.argtypes = []
+    lib.muse_cluster_static.restype = i32
+    lib.muse_cluster_static.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, u64, i32, vp, vp,
+                                        vp, vp, vp]
+    lib.muse_cluster_static_capacity.restype = sz
+    lib.muse_cluster_static_capacity.argtypes = []
     lib.muse_profile_enable.restype = None
     lib.muse_profile_enable.argtypes = [i32]
     lib.muse_profile_read.restype = i32
@@ -234,6 +240,23 @@ def muse_cluster(x, C, iters, seed, role=0, init=None, workspace=None, stream=No
     st = lib.muse_cluster(_ptr(x), _dtype_code(x), B, H, N, D, C, iters, int(seed) & (2 ** 64 - 1),
                           role, _ptr(init), _ptr(assign), _ptr(cent), _ptr(counts),
                           _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(lib, st)
+    return assign, cent, counts
+
+
+def muse_cluster_static(x, C, iters, seed, role=0, init=None, stream=None):
+    """muse_cluster for callers that cannot allocate a workspace: the scratch
+    is the fixed array built into the library (see include/muse.h for its
+    limit and its sharing rules).  Returns (assign, centroids, counts)."""
+    lib = load_library()
+    _need_cuda(x, init)
+    B, H, N, D = x.shape
+    assign = torch.empty(B, H, N, dtype=torch.int32, device=x.device)
+    cent = torch.empty(B, H, C, D, dtype=torch.float32, device=x.device)
+    counts = torch.empty(B, H, C, dtype=torch.int32, device=x.device)
+    st = lib.muse_cluster_static(_ptr(x), _dtype_code(x), B, H, N, D, C, iters,
+                                 int(seed) & (2 ** 64 - 1), role, _ptr(init), _ptr(assign),
+                                 _ptr(cent), _ptr(counts), _stream(stream))
     _check(lib, st)
     return assign, cent, counts
 

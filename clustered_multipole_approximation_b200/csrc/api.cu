@@ -288,6 +288,10 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
 
 }  // namespace
 
+namespace muse {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace muse
+
 extern "C" {
 
 size_t muse_workspace_size(const muse_shape* shape, const muse_params* params, int causal) {

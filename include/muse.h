@@ -174,6 +174,30 @@ muse_status muse_attn_fwd_causal(const void *Q, const void *K, const void *V,
                                  const muse_params *params, muse_debug *debug,
                                  void *ws, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * muse_cluster without a workspace argument, for callers that cannot
+ * allocate device memory (no counterpart on the pages: this is a packaging
+ * choice of this library).  The scratch comes from a fixed array compiled
+ * into the library (muse_cluster_static_capacity() bytes, 16 MiB, held on
+ * every GPU that loads the library until the process exits); sizes whose
+ * muse_cluster_workspace_size() exceeds it return MUSE_ERR_WORKSPACE with a
+ * message and launch nothing.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current):
+ * make that first call before any stream capture.  All calls share the one
+ * array and it keeps the last call's contents -- the parts that must start at
+ * zero are cleared by each call -- so calls whose work overlaps on the GPU
+ * (other streams, other host threads) race.  Arguments and outputs are those
+ * of muse_cluster.
+ */
+muse_status muse_cluster_static(const void *X, muse_dtype dtype, int B, int H,
+                                int N, int D, int C, int iters, uint64_t seed,
+                                int role, const float *init, int32_t *assign,
+                                float *centroids, int32_t *counts,
+                                cudaStream_t stream);
+
+/* Bytes of the scratch array built into the library for muse_cluster_static. */
+size_t muse_cluster_static_capacity(void);
+
 const char *muse_status_string(muse_status status);
 
 /* Per-kernel timing, for benchmarks (instrumentation only; no paper
