@@ -64,18 +64,22 @@ __device__ inline bool mbar_wait(uint32_t mbar, uint32_t parity) {
   }
   return false;
 }
-__device__ inline void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+// 16 columns without waiting; pair with tmem_wait() before using the values
+__device__ inline void tmem_ld16_nw(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-#pragma unroll
-  for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(r[u]);
 }
+__device__ inline void tmem_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ inline void cp16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr(dst)), "l"(src),
+               "r"(src_bytes));
+}
+__device__ inline void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+__device__ inline void cp_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 __device__ inline void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ inline void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 __device__ inline void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
@@ -91,7 +95,7 @@ __host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc) {
   L.NC = NC;
   L.tpc = tpc;
   size_t o = 0;
-  L.a = o;    o += (size_t)2 * L.KB * kTile * 128;   // two tiles in flight
+  L.a = o;    o += (size_t)3 * L.KB * kTile * 128;   // in use, under MMA, loading
   L.bh = o;   o += (size_t)L.KB * NC * 128;
   L.bl = o;   o += (size_t)L.KB * NC * 128;
   L.cn2 = o;  o += (size_t)NC * 4;
@@ -142,7 +146,32 @@ __device__ inline int block_scan_excl(int* a, int n, int* tmp) {
 
 constexpr int kFT = 256;  // threads of the fused kernel (8 warps)
 
-template <int D>
+// acc[k][.] += x for the warp-uniform k (registers stay registers).
+template <int KA, int R>
+__device__ inline void acc_add(double (&acc)[KA > 0 ? KA : 1][R], int k, const double (&x)[R]) {
+#define MUSE_ACC_CASE(K)                                                     \
+  case K:                                                                    \
+    if (K < (KA > 0 ? KA : 1)) {                                             \
+      _Pragma("unroll") for (int q = 0; q < R; ++q)                          \
+          acc[K < (KA > 0 ? KA : 1) ? K : 0][q] =                            \
+              __dadd_rn(acc[K < (KA > 0 ? KA : 1) ? K : 0][q], x[q]);        \
+    }                                                                        \
+    break;
+  switch (k) {
+    MUSE_ACC_CASE(0) MUSE_ACC_CASE(1) MUSE_ACC_CASE(2) MUSE_ACC_CASE(3)
+    MUSE_ACC_CASE(4) MUSE_ACC_CASE(5) MUSE_ACC_CASE(6) MUSE_ACC_CASE(7)
+    MUSE_ACC_CASE(8) MUSE_ACC_CASE(9) MUSE_ACC_CASE(10) MUSE_ACC_CASE(11)
+    MUSE_ACC_CASE(12) MUSE_ACC_CASE(13) MUSE_ACC_CASE(14) MUSE_ACC_CASE(15)
+    default: break;
+  }
+#undef MUSE_ACC_CASE
+}
+
+// KA > 0: each warp keeps the fp64 sums of its clusters (c = w mod 8, at most
+// 8 KA of them) in registers and the fp64 centroids are staged in shared
+// memory for the re-decision; KA == 0: sums in shared memory, centroids read
+// from L2.
+template <int D, int KA>
 __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int iters, int NCT,
                                                              int NC, int tpc_max, int tcols) {
   cg::cluster_group cluster = cg::this_cluster();
@@ -154,12 +183,13 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   const KState& ks = fs.ks[set];
   const int blk = (int)blockIdx.x - (set ? fs.nblk0 : 0);
   constexpr int KB = D / 64;
+  constexpr int R = D / 32;
   constexpr int ATILE = KB * kTile * 128;  // bytes of one swizzled token tile
   unsigned char* A0 = base + Lo.a;
   unsigned char* BH = base + Lo.bh;
   unsigned char* BL = base + Lo.bl;
   float* cn2s = reinterpret_cast<float*>(base + Lo.cn2);
-  double* sacc = reinterpret_cast<double*>(base + Lo.acc);
+  double* sacc = reinterpret_cast<double*>(base + Lo.acc);  // KA > 0: staged centroids first
   int* lcnt = reinterpret_cast<int*>(base + Lo.lcnt);
   int* loff = reinterpret_cast<int*>(base + Lo.loff);
   unsigned short* asg = reinterpret_cast<unsigned short*>(base + Lo.asg);
@@ -210,20 +240,20 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   const int hw = ncp / 2;                  // columns per half
   const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(ncp >> 3) << 17) |
                          ((uint32_t)(128 >> 4) << 24);
-  const double* c64 = ks.cent64 + cbase * D;
+  const double* c64g = ks.cent64 + cbase * D;
 
   auto xrow = [&](const unsigned char* A, int r, int d) -> float {
     const int kb = d >> 6, k = d & 63;
     const unsigned char* pz = A + kb * kTile * 128 + sw128_chunk(r, k >> 3) + ((k & 7) << 1);
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(pz));
   };
-  auto load_tile = [&](int tl, unsigned char* A) {
+  auto load_tile = [&](int tl, unsigned char* A) {  // cp.async; caller commits
     const int t0 = tl * kTile, nt = imin(kTile, p.s - t0);
     for (int e = tid; e < kTile * KB * 8; e += kFT) {
       const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, cq = q & 7;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < nt) v = *reinterpret_cast<const uint4*>(X + (p.row0 + t0 + r) * D + kb * 64 + cq * 8);
-      *reinterpret_cast<uint4*>(A + kb * kTile * 128 + sw128_chunk(r, cq)) = v;
+      const bool live = r < nt;
+      cp16(A + kb * kTile * 128 + sw128_chunk(r, cq),
+           X + (p.row0 + t0 + (live ? r : 0)) * D + kb * 64 + cq * 8, live ? 16 : 0);
     }
   };
   auto issue_mma = [&](const unsigned char* A, int buf) {
@@ -240,25 +270,28 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     }
     mma_commit(saddr(&mbar[buf]));
   };
+  auto tile_buf = [&](int k) { return A0 + (k % 3) * ATILE; };
 
   for (int it = 0; it < iters; ++it) {
     const bool last = it + 1 == iters;
-    // ---- centroids of this round; clear the partial sums -----------------------
+    // ---- centroids of this round (bf16 split; KA > 0: fp64 copy too) ----------
     for (int e = tid; e < ncp * KB * 8; e += kFT) {
       const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, cq = q & 7;
-      uint4 vh = make_uint4(0, 0, 0, 0), vl = vh;
-      if (r < C) {
-        const size_t off = (cbase + r) * D + kb * 64 + cq * 8;
-        vh = __ldcg(reinterpret_cast<const uint4*>(ks.cbf_hi + off));
-        vl = __ldcg(reinterpret_cast<const uint4*>(ks.cbf_lo + off));
-      }
-      *reinterpret_cast<uint4*>(BH + kb * NC * 128 + sw128_chunk(r, cq)) = vh;
-      *reinterpret_cast<uint4*>(BL + kb * NC * 128 + sw128_chunk(r, cq)) = vl;
+      const bool live = r < C;
+      const size_t off = (cbase + (live ? r : 0)) * D + kb * 64 + cq * 8;
+      cp16(BH + kb * NC * 128 + sw128_chunk(r, cq), ks.cbf_hi + off, live ? 16 : 0);
+      cp16(BL + kb * NC * 128 + sw128_chunk(r, cq), ks.cbf_lo + off, live ? 16 : 0);
     }
-    for (int e = tid; e < C * D; e += kFT) sacc[e] = 0.0;
+    if (KA > 0)
+      for (int e = tid; e < C * D / 2; e += kFT) cp16(sacc + 2 * e, c64g + 2 * e, 16);
+    if (KA == 0)
+      for (int e = tid; e < C * D; e += kFT) sacc[e] = 0.0;
     for (int c = tid; c < C; c += kFT) lcnt[c] = 0;
     if (tid == 0) cmax_s = 0.f;
-    __syncthreads();
+    if (ntl > 0) load_tile(tile0, tile_buf(0));
+    cp_commit();
+    if (ntl > 1) load_tile(tile0 + 1, tile_buf(1));
+    cp_commit();
     {
       float m = 0.f;
       for (int c = tid; c < C; c += kFT) {
@@ -267,47 +300,53 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         m = fmaxf(m, v);
       }
       for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      __syncthreads();
       if (lane == 0) atomicMax(reinterpret_cast<int*>(&cmax_s), __float_as_int(m));
     }
-    if (ntl > 0) load_tile(tile0, A0);
+    asm volatile("cp.async.wait_group 1;\n" ::: "memory");  // centroids and tile 0
     fence_async_smem();
     fence_before();
     __syncthreads();
     fence_after();
     const float cm = sqrtf(cmax_s) * 1.0001f;
-    if (ntl > 0 && tid == 0) issue_mma(A0, 0);
+    if (ntl > 0 && tid == 0) issue_mma(tile_buf(0), 0);
+    double racc[KA > 0 ? KA : 1][R];
+#pragma unroll
+    for (int kk = 0; kk < (KA > 0 ? KA : 1); ++kk)
+#pragma unroll
+      for (int q = 0; q < R; ++q) racc[kk][q] = 0.0;
 
     for (int k = 0; k < ntl; ++k) {
       const int tl = tile0 + k, buf = k & 1;
       const int t0 = tl * kTile, nt = imin(kTile, p.s - t0);
-      unsigned char* A = A0 + buf * ATILE;
-      // ---- next tile's load and MMA overlap this tile's epilogue --------------
+      const unsigned char* A = tile_buf(k);
+      // ---- tile k+1 goes to the tensor cores, tile k+2 starts loading ---------
       if (k + 1 < ntl) {
-        load_tile(tl + 1, A0 + (buf ^ 1) * ATILE);
+        cp_wait_all();
         fence_async_smem();
         fence_before();
         __syncthreads();
         fence_after();
-        if (tid == 0) issue_mma(A0 + (buf ^ 1) * ATILE, buf ^ 1);
+        if (tid == 0) issue_mma(tile_buf(k + 1), buf ^ 1);
+        if (k + 2 < ntl) load_tile(tl + 2, tile_buf(k + 2));
+        cp_commit();
       }
       // token norm for the screen bound (own row, 16-byte loads)
       float xn = 0.f;
-      if (tid < kTile) {
-        if (tid < nt) {
-          const uint4* xr = reinterpret_cast<const uint4*>(X + (p.row0 + t0 + tid) * D);
-          float q2 = 0.f;
+      if (tid < nt) {
+        const uint4* xr = reinterpret_cast<const uint4*>(X + (p.row0 + t0 + tid) * D);
+        float q2 = 0.f;
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) {
-            const uint4 v = xr[c];
-            const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 v = xr[c];
+          const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 f = __bfloat1622float2(b[u]);
-              q2 = fmaf(f.x, f.x, fmaf(f.y, f.y, q2));
-            }
+          for (int u = 0; u < 4; ++u) {
+            const float2 f = __bfloat1622float2(b[u]);
+            q2 = fmaf(f.x, f.x, fmaf(f.y, f.y, q2));
           }
-          xn = sqrtf(q2) * 1.0001f;
         }
+        xn = sqrtf(q2) * 1.0001f;
       }
       __syncwarp();
       const bool done = mbar_wait(saddr(&mbar[buf]), phase[buf]);
@@ -317,25 +356,53 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       fence_after();
       const uint32_t tm = tbase + (uint32_t)(buf * ncp) + ((uint32_t)((warp & 3) * 32) << 16);
       // ---- epilogue: each half of the warps scans half of the columns ---------
+      // four independent best / runner-up trackers (columns c = 4m + u) keep
+      // the compare chain short; merged by (value, index) so ties keep the
+      // lowest index
       float b1 = INFINITY, b2 = INFINITY;
       int bi = 0;
       if (ok) {
-        for (int cc = half * hw; cc < (half + 1) * hw; cc += 16) {
-          float acc[16];
-          tmem_ld16(tm + (uint32_t)cc, acc);
+        float t1[4], t2[4];
+        int ti[4];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int c = cc + u;
-            if (c < C) {
-              const float dd = fmaf(-2.f, acc[u], cn2s[c]);
-              if (dd < b1) {
-                b2 = b1;
-                b1 = dd;
-                bi = c;
-              } else if (dd < b2) {
-                b2 = dd;
+        for (int u = 0; u < 4; ++u) {
+          t1[u] = INFINITY;
+          t2[u] = INFINITY;
+          ti[u] = 0;
+        }
+        for (int c0 = half * hw; c0 < (half + 1) * hw; c0 += 64) {
+          uint32_t rv[4][16];
+          const int nb = imin(4, ((half + 1) * hw - c0) / 16);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (u < nb) tmem_ld16_nw(tm + (uint32_t)(c0 + 16 * u), rv[u]);
+          tmem_wait();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (u >= nb) break;
+#pragma unroll
+            for (int v = 0; v < 16; ++v) {
+              const int c = c0 + 16 * u + v;
+              const int tk = v & 3;
+              const float dd = c < C ? fmaf(-2.f, __uint_as_float(rv[u][v]), cn2s[c]) : INFINITY;
+              if (dd < t1[tk]) {
+                t2[tk] = t1[tk];
+                t1[tk] = dd;
+                ti[tk] = c;
+              } else if (dd < t2[tk]) {
+                t2[tk] = dd;
               }
             }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (t1[u] < b1 || (t1[u] == b1 && ti[u] < bi)) {
+            b2 = fminf(b1, t2[u]);
+            b1 = t1[u];
+            bi = ti[u];
+          } else {
+            b2 = fminf(b2, t1[u]);
           }
         }
       }
@@ -355,7 +422,9 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         } else {
           b2 = fminf(b2, u1);
         }
-        const float E = 2.f * 6.1035156e-05f * xn * cm + 2.3841858e-07f * (cm * cm + 2.f * xn * cm);
+        // |screen - exact| <= 2 eta |x| |c| + 2^-22 (|c|^2 + 2 |x| |c|), eta = 2^-15:
+        // bf16 split residual (2^-18) plus fp32 accumulation of 2D exact products
+        const float E = 2.f * 3.0517578e-05f * xn * cm + 2.3841858e-07f * (cm * cm + 2.f * xn * cm);
         const bool flag = tid < nt && (!ok || (b2 - b1) <= 2.f * E);
         // exact re-decision: only clusters inside the certified band can win
         int bx = bi;
@@ -364,19 +433,23 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
           int bc = -1;
           const float lim = b1 + 2.f * E;
           for (int cc = 0; cc < ncp; cc += 16) {
-            float accv[16];
-            if (ok) tmem_ld16(tm + (uint32_t)cc, accv);
+            uint32_t rv[16];
+            if (ok) {
+              tmem_ld16_nw(tm + (uint32_t)cc, rv);
+              tmem_wait();
+            }
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
               const int c = cc + u;
-              const bool cand = flag && c < C && (!ok || fmaf(-2.f, accv[u], cn2s[c]) <= lim);
+              const bool cand =
+                  flag && c < C && (!ok || fmaf(-2.f, __uint_as_float(rv[u]), cn2s[c]) <= lim);
               if (cand) {
-                const double* ccen = c64 + (size_t)c * D;
+                const double* ccen = (KA > 0 ? (const double*)sacc : c64g) + (size_t)c * D;
                 double sd = 0.0;
                 for (int d0 = 0; d0 < D; d0 += 16) {
                   double cv[16];
 #pragma unroll
-                  for (int kk = 0; kk < 16; ++kk) cv[kk] = __ldcg(ccen + d0 + kk);
+                  for (int kk = 0; kk < 16; ++kk) cv[kk] = KA > 0 ? ccen[d0 + kk] : __ldcg(ccen + d0 + kk);
 #pragma unroll
                   for (int kk = 0; kk < 16; ++kk) {
                     const double t = __dsub_rn((double)xrow(A, row, d0 + kk), cv[kk]);
@@ -402,36 +475,46 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       }
       fence_before();
       __syncthreads();
-      // ---- fp64 partial sums: warp w owns the clusters c = w (mod 8); it walks
-      // their tokens in tile order (lanes over dimensions), so each
-      // accumulator sees its members in ascending token order ----------------
-      {
-        constexpr int R2 = D / 32;
-        for (int r0 = 0; r0 < nt; r0 += 32) {
-          const int ra = r0 + lane < nt ? tasg[r0 + lane] : -1;
-          unsigned mine = __ballot_sync(0xffffffffu, ra >= 0 && (ra & 7) == warp);
-          while (mine) {
-            const int bit = __ffs(mine) - 1;
-            mine &= mine - 1;
-            const int r = r0 + bit;
-            const int a = __shfl_sync(0xffffffffu, ra, bit);
+      // ---- fp64 partial sums: warp w owns the clusters c = w (mod 8) and walks
+      // their tokens in tile order (lanes over dimensions), so every sum sees
+      // its members in ascending token order --------------------------------------
+      for (int r0 = 0; r0 < nt; r0 += 32) {
+        const int ra = r0 + lane < nt ? tasg[r0 + lane] : -1;
+        unsigned mine = __ballot_sync(0xffffffffu, ra >= 0 && (ra & 7) == warp);
+        while (mine) {
+          const int bit = __ffs(mine) - 1;
+          mine &= mine - 1;
+          const int r = r0 + bit;
+          const int a = __shfl_sync(0xffffffffu, ra, bit);
+          double x[R];
+#pragma unroll
+          for (int q = 0; q < R; ++q) x[q] = (double)xrow(A, r, lane + 32 * q);
+          if (KA > 0) {
+            acc_add<KA, R>(racc, a >> 3, x);
+          } else {
             double* sp = sacc + (size_t)a * D;
 #pragma unroll
-            for (int q = 0; q < R2; ++q) {
-              const int d = lane + 32 * q;
-              sp[d] = __dadd_rn(sp[d], (double)xrow(A, r, d));
-            }
+            for (int q = 0; q < R; ++q) sp[lane + 32 * q] = __dadd_rn(sp[lane + 32 * q], x[q]);
           }
         }
       }
       __syncthreads();
+    }
+    if (KA > 0) {
+      // the staged centroids are no longer read: publish the sums there
+#pragma unroll
+      for (int kk = 0; kk < (KA > 0 ? KA : 1); ++kk) {
+        const int c = kk * 8 + warp;
+        if (c < C)
+#pragma unroll
+          for (int q = 0; q < R; ++q) sacc[(size_t)c * D + lane + 32 * q] = racc[kk][q];
+      }
     }
     // ---- last round: this CTA's tokens grouped by cluster (stable) ----------
     if (last) {
       for (int c = tid; c < C; c += kFT) loff[c] = lcnt[c];
       __syncthreads();
       block_scan_excl(loff, C, scan_tmp);
-      __syncthreads();
       if (warp == 0) {
         for (int b0 = 0; b0 < ntok; b0 += 32) {
           const int t = b0 + lane;
@@ -465,7 +548,6 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       if (tid == 0) goff[C] = tot;
       __syncthreads();
     }
-    constexpr int R = D / 32;
     for (int c = rank + NCT * warp; c < C; c += NCT * (kFT / 32)) {
       const int n = gcnt[c];
       if (last && lane == 0) {
@@ -474,13 +556,13 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         if (c == C - 1) ks.off[(size_t)pid * (g.C + 1) + C] = goff[C];
       }
       if (n == 0) continue;  // an empty cluster keeps its centroid
-      double s[R];
+      double sm[R];
 #pragma unroll
-      for (int r = 0; r < R; ++r) s[r] = 0.0;
+      for (int q = 0; q < R; ++q) sm[q] = 0.0;
       for (int rr = 0; rr < NCT; ++rr) {
         const double* ra = cluster.map_shared_rank(sacc, rr) + (size_t)c * D;
 #pragma unroll
-        for (int r = 0; r < R; ++r) s[r] = __dadd_rn(s[r], ra[lane + 32 * r]);
+        for (int q = 0; q < R; ++q) sm[q] = __dadd_rn(sm[q], ra[lane + 32 * q]);
       }
       if (last) {
         int pos = goff[c];
@@ -495,26 +577,26 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       }
       const double nn = (double)n;
       double q2 = 0.0;
-      float q = 0.f;
+      float qf = 0.f;
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const double v = __ddiv_rn(s[r], nn);
+      for (int q = 0; q < R; ++q) {
+        const double v = __ddiv_rn(sm[q], nn);
         const float v32 = (float)v;
-        const size_t i = (cbase + c) * D + lane + 32 * r;
+        const size_t i = (cbase + c) * D + lane + 32 * q;
         ks.cent64[i] = v;
         ks.cent32[i] = v32;
         const __nv_bfloat16 hi = __float2bfloat16_rn(v32);
         ks.cbf_hi[i] = hi;
         ks.cbf_lo[i] = __float2bfloat16_rn(v32 - __bfloat162float(hi));
         q2 += v * v;
-        q = fmaf(v32, v32, q);
+        qf = fmaf(v32, v32, qf);
       }
       for (int o = 16; o; o >>= 1) {
-        q += __shfl_xor_sync(0xffffffffu, q, o);
+        qf += __shfl_xor_sync(0xffffffffu, qf, o);
         q2 += __shfl_xor_sync(0xffffffffu, q2, o);
       }
       if (lane == 0) {
-        ks.cnorm[cbase + c] = sqrtf(q) * 1.0001f;
+        ks.cnorm[cbase + c] = sqrtf(qf) * 1.0001f;
         ks.cn2[cbase + c] = (float)q2;
       }
     }
@@ -529,7 +611,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
 
 // Returns false (nothing launched) when the fused path does not cover these
 // problem sets: more than 256 clusters, or more than 65535 tokens per CTA.
-template <int D>
+template <int D, int KA>
 static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int iters,
                            cudaStream_t st) {
   int cmax = 0;
@@ -541,10 +623,15 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
   int tcols = 32;
   while (tcols < 2 * NC) tcols <<= 1;  // two accumulators (tiles in flight)
   const int nprob = kss[0].nprob + (nsets > 1 ? kss[1].nprob : 0);
-  // largest portable cluster size whose clusters are all resident at once
+  // largest cluster size (up to 16, beyond the portable 8 where the GPU
+  // allows it) whose clusters are all resident at once
   int NCT = 0;
   FusedLayout L{};
-  for (int nct = 8; nct >= 1; --nct) {
+  const bool big_ok =
+      cudaFuncSetAttribute(kmeans_fused_kernel<D, KA>,
+                           cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  if (!big_ok) cudaGetLastError();
+  for (int nct = big_ok ? 16 : 8; nct >= 1; --nct) {
     int tpc_max = 1;
     for (int k = 0; k < nsets; ++k)
       for (int l = 0; l < gs[k].lv.nlev; ++l) {
@@ -554,7 +641,7 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
     if (tpc_max * kTile > 65535) break;
     const FusedLayout Lc = fused_layout(D, NC, tpc_max);
     if (Lc.total > 218 * 1024) continue;  // leaves room for the static shared arrays
-    cudaFuncSetAttribute(kmeans_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(kmeans_fused_kernel<D, KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)Lc.total);
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3((unsigned)(nprob * nct));
@@ -568,11 +655,11 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
     q.attrs = qa;
     q.numAttrs = 1;
     int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, kmeans_fused_kernel<D>, &q) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&active, kmeans_fused_kernel<D, KA>, &q) != cudaSuccess) {
       cudaGetLastError();
       active = 0;
     }
-    if (NCT == 0) {  // fallback: the largest size that fits at all
+    if (nct <= 8 && NCT == 0) {  // fallback: the largest portable size that fits at all
       NCT = nct;
       L = Lc;
     }
@@ -590,7 +677,7 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
   }
   fs.nblk0 = kss[0].nprob * NCT;
   const int nblk = fs.nblk0 + (nsets > 1 ? kss[1].nprob * NCT : 0);
-  cudaFuncSetAttribute(kmeans_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaFuncSetAttribute(kmeans_fused_kernel<D, KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)L.total);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)nblk);
@@ -604,14 +691,20 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D>, fs, iters, NCT, NC, L.tpc, tcols);
+  cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, KA>, fs, iters, NCT, NC, L.tpc, tcols);
   return true;
 }
 
 bool launch_kmeans_fused(const RoleGeo* gs, const KState* kss, int nsets, int iters,
                          cudaStream_t st) {
-  return gs[0].D == 64 ? launch_fused_t<64>(gs, kss, nsets, iters, st)
-                       : launch_fused_t<128>(gs, kss, nsets, iters, st);
+  int cmax = 0;
+  for (int k = 0; k < nsets; ++k) cmax = cmax > gs[k].C ? cmax : gs[k].C;
+  // register sums when a warp's clusters (C / 8) x its dimensions (D / 32) fit in 32 doubles
+  if (gs[0].D == 64)
+    return cmax <= 128 ? launch_fused_t<64, 16>(gs, kss, nsets, iters, st)
+                       : launch_fused_t<64, 0>(gs, kss, nsets, iters, st);
+  return cmax <= 64 ? launch_fused_t<128, 8>(gs, kss, nsets, iters, st)
+                    : launch_fused_t<128, 0>(gs, kss, nsets, iters, st);
 }
 
 }  // namespace muse

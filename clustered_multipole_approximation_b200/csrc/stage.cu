@@ -595,7 +595,10 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
   }
   {
     ProfScope ps(st, "stage1_summaries");
-    stage1_kernel<T, D><<<dim3(nqp, a.Ck), kS1T, stage1_smem<D>(), st>>>(a, s1, qp0);
+    if (sizeof(T) == 2 && a.mode == 1)
+      run_stage1_dipole_mma(a, s1, qp0, nqp, st);
+    else
+      stage1_kernel<T, D><<<dim3(nqp, a.Ck), kS1T, stage1_smem<D>(), st>>>(a, s1, qp0);
   }
   if (a.topk > 0) {
     ProfScope ps(st, "stage1_select");
