@@ -108,6 +108,7 @@ struct Smem2 {
   KBuf<D> buf[2];
   unsigned char inR[kMaxC];
   int sel[kMaxC];
+  int selstart[kMaxC];  // start of each retrieved cluster in the concatenated list
 };
 
 }  // namespace
@@ -167,12 +168,14 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
   __syncthreads();
   const int* kc = a.ks.counts + (size_t)kpid * Ck;
   const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
+  // the retrieved clusters' members, concatenated in selection order, are one
+  // list of exact keys cut into blocks of 64 (a block may span two clusters)
   long long nexact = 0;
-  int nblk_exact = 0;
   for (int r = 0; r < nsel; ++r) {
+    sm.selstart[r] = (int)nexact;
     nexact += kc[sm.sel[r]];
-    nblk_exact += cdiv(kc[sm.sel[r]], kMK);
   }
+  const int nblk_exact = cdiv((int)nexact, kMK);
   const int nblk_far = cdiv(pk.C, kMK);
   const int nblk = nblk_far + nblk_exact;
 
@@ -207,20 +210,19 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
         B.bias[r] = live ? s1.fbias[ij0 + j] * 1.4426950408889634f : -INFINITY;
       }
     } else {
-      // locate the exact block: cluster rr of the selection, rows t0..t0+63
-      int rem = b - nblk_far, rr = 0;
-      while (true) {
-        const int nbj = cdiv(kc[sm.sel[rr]], kMK);
-        if (rem < nbj) break;
-        rem -= nbj;
-        ++rr;
-      }
-      const int j = sm.sel[rr], n = kc[j], t0 = rem * kMK, nr = imin(kMK, n - t0);
-      const int base = koff[j] + t0;
+      // rows p0 .. p0+63 of the concatenated member list
+      const int p0 = (b - nblk_far) * kMK;
+      const int nr = imin(kMK, (int)nexact - p0);
       for (int e = tid; e < kMK * CH; e += kThreads) {
         const int r = e / CH, c = (e % CH) * 8;
         const bool live = r < nr;
-        const long long row = pk.row0 + (live ? kperm[base + r] : 0);
+        long long row = pk.row0;
+        if (live) {
+          const int pos = p0 + r;
+          int rr = 0;
+          while (rr + 1 < nsel && sm.selstart[rr + 1] <= pos) ++rr;
+          row += kperm[koff[sm.sel[rr]] + pos - sm.selstart[rr]];
+        }
         cp16(&B.k[r][c], K + row * D + c, live ? 16 : 0);
         cp16(&B.v[r][c], V16 + row * D + c, live ? 16 : 0);
       }
