@@ -98,7 +98,8 @@ void carve_kstate(Carver& cv, KState& ks, const RoleGeo& g) {
   ks.off = cv.take<int>(np * (C + 1) * 4);
   ks.assign = cv.take<int>((size_t)ks.ntok * 4);
   ks.perm = cv.take<int>((size_t)ks.ntok * 4);
-  ks.hist = cv.take<int>((size_t)ks.ntiles * C * 4);
+  ks.hist = cv.take<int>((size_t)ks.ntiles * (C + 1) * 4);
+  ks.tlist = cv.take<unsigned short>((size_t)ks.ntok * 2);
   ks.arrive = cv.take<int>(np * 4);
   ks.cbf_hi = cv.take<__nv_bfloat16>(np * C * D * 2);
   ks.cbf_lo = cv.take<__nv_bfloat16>(np * C * D * 2);
@@ -247,10 +248,9 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   if (L.nq > 0) {
     cudaMemsetAsync(L.ks.arrive, 0, (size_t)L.ks.nprob * 4, st);
     cudaMemsetAsync(L.qs.arrive, 0, (size_t)L.qs.nprob * 4, st);
-    run_kmeans_init(L.kg, L.ks, nullptr, st);
-    run_kmeans_init(L.qg, L.qs, nullptr, st);
     const RoleGeo gs[2] = {L.kg, L.qg};
     const KState kss[2] = {L.ks, L.qs};
+    run_kmeans_init(gs, kss, 2, nullptr, st);
     bool fused;
     {
       ProfScope ps(st, "kmeans_fused");
@@ -334,7 +334,7 @@ muse_status muse_cluster(const void* X, muse_dtype dtype, int B, int H, int N, i
   ks.err = err;
   cudaMemsetAsync(err, 0, 4, stream);
   cudaMemsetAsync(ks.arrive, 0, (size_t)ks.nprob * 4, stream);
-  run_kmeans_init(g, ks, init, stream);
+  run_kmeans_init(&g, &ks, 1, init, stream);
   bool fused;
   {
     ProfScope ps(stream, "kmeans_fused");

@@ -114,7 +114,10 @@ struct KState {
   int* off;         // [nprob][C+1]  segment offsets of the sorted order
   int* assign;      // [tokens]      cluster of each token (problem-local index)
   int* perm;        // [tokens]      problem-local token index in cluster-sorted order
-  int* hist;        // [tiles][C]    per-tile histogram, then scatter bases
+  int* hist;        // [tiles][C+1]  per-tile histogram, then scatter bases; the
+                    //               persistent k-means: per-CTA list offsets
+  unsigned short* tlist;  // [tokens]  persistent k-means: each CTA's tokens grouped
+                          //           by cluster (CTA-local token index)
   int* arrive;      // [nprob]       tile arrival counters (self-resetting)
   __nv_bfloat16* cbf_hi;  // [nprob][C][D] bf16 rounding of cent32
   __nv_bfloat16* cbf_lo;  // [nprob][C][D] bf16 rounding of cent32 - cbf_hi

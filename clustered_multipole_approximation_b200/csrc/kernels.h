@@ -49,8 +49,9 @@ struct AttnArgs {
 void run_kmeans(const RoleGeo& g, const KState& ks, int iters, const float* init,
                 cudaStream_t st);
 
-// Seeded (or given) start centroids for a problem set.
-void run_kmeans_init(const RoleGeo& g, const KState& ks, const float* init, cudaStream_t st);
+// Seeded (or given) start centroids for up to two problem sets, one launch.
+void run_kmeans_init(const RoleGeo* gs, const KState* kss, int nsets, const float* init,
+                     cudaStream_t st);
 
 // All Lloyd rounds of up to two problem sets in one persistent launch
 // (thread-block clusters, bf16 inputs); false if these sets are not covered.

@@ -34,8 +34,6 @@ __device__ inline uint64_t splitmix64_next(uint64_t& state) {
   return z ^ (z >> 31);
 }
 
-constexpr int kHashSize = 2 * kMaxC;  // open addressing, load <= 1/2
-
 // r mod m for a 32-bit m, exactly: reduce the high word first, then the
 // remaining < m * 2^32 by a double-precision quotient estimate and an exact
 // integer correction (the generic 64-bit remainder is a long software loop).
@@ -49,53 +47,52 @@ __device__ inline uint32_t mod_u64_u32(uint64_t r, uint32_t m) {
   return (uint32_t)rem;
 }
 
+// Both roles' problems in one launch: CTAs [0, nblk0) serve set 0.
+struct InitSets {
+  RoleGeo g[2];
+  KState ks[2];
+  int nblk0;
+};
+
 template <typename T>
-__global__ void __launch_bounds__(256) kmeans_init_kernel(RoleGeo g, KState ks, const float* init) {
-  __shared__ int hkey[kHashSize];
-  __shared__ int hval[kHashSize];
+__global__ void __launch_bounds__(256) kmeans_init_kernel(InitSets is, const float* init) {
+  __shared__ int jd[kMaxC];
   __shared__ int pick[kMaxC];
-  const int pid = blockIdx.x;
+  const int set = (int)blockIdx.x < is.nblk0 ? 0 : 1;
+  const RoleGeo& g = is.g[set];
+  const KState& ks = is.ks[set];
+  const int pid = (int)blockIdx.x - (set ? is.nblk0 : 0);
   const Prob p = prob_of(g, pid);
   const int D = g.D, C = p.C;
   const T* X = static_cast<const T*>(g.X);
   double* c64 = ks.cent64 + (size_t)pid * g.C * D;
   float* c32 = ks.cent32 + (size_t)pid * g.C * D;
   if (init == nullptr) {
-    for (int i = threadIdx.x; i < kHashSize; i += blockDim.x) hkey[i] = -1;
-    __syncthreads();
-    // splitmix64 is counter based: draw c uses state0 + (c + 1) * gamma, so
-    // every swap target j_c is computed in parallel; only the swaps themselves
-    // are applied in order below.
+    // Partial Fisher-Yates: step c swaps positions c and j_c = c + (r_c mod
+    // (n - c)) of the identity and picks the new value at c.  splitmix64 is
+    // counter based (draw c uses state0 + (c + 1) * gamma), so every j_c is
+    // drawn in parallel.  The swaps are resolved without replaying them: the
+    // value at a position pos >= s before step s is the value that stood at
+    // position c' before step c', for the latest c' < s with j_c' = pos (step
+    // c' moved it there), else pos itself; the recursion ends because c' < pos.
     const uint64_t st0 = g.seed + 0x9E3779B97F4A7C15ULL * (2ULL * p.sid + (uint64_t)g.role + 1ULL);
     const int n = p.s;
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
       uint64_t st = st0 + 0x9E3779B97F4A7C15ULL * (uint64_t)c;
       const uint64_t r = splitmix64_next(st);
-      pick[c] = c + (int)mod_u64_u32(r, (uint32_t)(n - c));
+      jd[c] = c + (int)mod_u64_u32(r, (uint32_t)(n - c));
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      for (int c = 0; c < C; ++c) {
-        const int j = pick[c];
-        // value currently at position j (identity unless swapped before)
-        int h = j & (kHashSize - 1), vj = j;
-        while (hkey[h] >= 0) {
-          if (hkey[h] == j) { vj = hval[h]; break; }
-          h = (h + 1) & (kHashSize - 1);
-        }
-        int vc = c;
-        int hc = c & (kHashSize - 1);
-        while (hkey[hc] >= 0) {
-          if (hkey[hc] == c) { vc = hval[hc]; break; }
-          hc = (hc + 1) & (kHashSize - 1);
-        }
-        pick[c] = vj;
-        // position j now holds the old value of position c
-        h = j & (kHashSize - 1);
-        while (hkey[h] >= 0 && hkey[h] != j) h = (h + 1) & (kHashSize - 1);
-        hkey[h] = j;
-        hval[h] = vc;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      int pos = jd[c], s = c;
+      for (;;) {
+        int f = s - 1;
+        while (f >= 0 && jd[f] != pos) --f;
+        if (f < 0) break;
+        pos = f;
+        s = f;
       }
+      pick[c] = pos;
     }
     __syncthreads();
   }
@@ -362,16 +359,25 @@ static void launch_round(const RoleGeo& g, const KState& ks, cudaStream_t st) {
 }
 
 template <typename T>
-static void init_t(const RoleGeo& g, const KState& ks, const float* init, cudaStream_t st) {
+static void init_t(const RoleGeo* gs, const KState* kss, int nsets, const float* init,
+                   cudaStream_t st) {
   ProfScope ps(st, "kmeans_init");
-  kmeans_init_kernel<T><<<ks.nprob, 256, 0, st>>>(g, ks, init);
+  InitSets is{};
+  for (int k = 0; k < nsets; ++k) {
+    is.g[k] = gs[k];
+    is.ks[k] = kss[k];
+  }
+  is.nblk0 = kss[0].nprob;
+  const int nblk = kss[0].nprob + (nsets > 1 ? kss[1].nprob : 0);
+  kmeans_init_kernel<T><<<(unsigned)nblk, 256, 0, st>>>(is, init);
 }
 
-void run_kmeans_init(const RoleGeo& g, const KState& ks, const float* init, cudaStream_t st) {
-  if (g.dtype == 0)
-    init_t<__nv_bfloat16>(g, ks, init, st);
+void run_kmeans_init(const RoleGeo* gs, const KState* kss, int nsets, const float* init,
+                     cudaStream_t st) {
+  if (gs[0].dtype == 0)
+    init_t<__nv_bfloat16>(gs, kss, nsets, init, st);
   else
-    init_t<float>(g, ks, init, st);
+    init_t<float>(gs, kss, nsets, init, st);
 }
 
 template <typename T>
@@ -392,7 +398,7 @@ void run_kmeans_rounds(const RoleGeo& g, const KState& ks, int iters, cudaStream
 }
 
 void run_kmeans(const RoleGeo& g, const KState& ks, int iters, const float* init, cudaStream_t st) {
-  run_kmeans_init(g, ks, init, st);
+  run_kmeans_init(&g, &ks, 1, init, st);
   run_kmeans_rounds(g, ks, iters, st);
 }
 

@@ -5,19 +5,27 @@
 // Attention: A Fast Approximation of Softmax Attention for Pretraining",
 // Technical Summary, Core Mechanisms, "Bidirectional Semantic Clustering").
 // Round structure inside the kernel:
-//   1. every CTA screens its 128-token tiles against the centroids with
-//      tcgen05.mma (bf16 hi/lo split of the centroids, fp32 TMEM accumulator),
-//      keeps best/runner-up per token and re-decides uncertain tokens in fp64;
-//   2. every CTA sorts its tokens by cluster (stable counting sort in shared
-//      memory) and publishes its per-cluster counts and member lists;
-//   3. cluster barrier; cluster c is owned by CTA rank c % NCT, which reads all
-//      CTAs' counts and member lists through distributed shared memory and sums
-//      the member rows in ascending token order in fp64 (the same order as a
-//      plain sequential evaluation), then writes the new centroid (fp64, fp32,
-//      bf16 hi/lo, norms) to global memory;
-//   4. cluster barrier, next round.
-// After the last round the owners also write the counts, segment offsets and
-// the cluster-sorted permutation that the summaries and stage 2 read.
+//   1. every CTA streams its 128-token tiles through shared memory (a cp.async
+//      ring of three) and screens them against the centroids with
+//      tcgen05.mma (bf16 hi/lo split of the centroids, fp32 TMEM accumulator;
+//      two accumulators, so the tensor cores run one tile ahead of the
+//      epilogue).  The epilogue keeps the best and runner-up screened distance
+//      of every token; a token whose gap lies inside the certified error of
+//      the screen goes to a queue;
+//   2. the CTA's warps drain the queue: a queued token gets the exact fp64
+//      argmin over all clusters, each distance summed in dimension order with
+//      no fused operations (a plain sequential fp64 evaluation, bit for bit);
+//   3. the CTA groups its tokens by cluster (stable counting sort) and
+//      publishes the grouped list and its per-cluster offsets in global memory;
+//   4. cluster barrier; cluster c is owned by CTA rank c % NCT, where a group
+//      of D/8 lanes walks the members of c over all CTAs in ascending token
+//      order and sums their rows in fp64 -- the order of a plain sequential
+//      evaluation -- with 16 rows in flight, then writes the new centroid
+//      (fp64, fp32, bf16 hi/lo, norms) to global memory;
+//   5. cluster barrier, next round.
+// After the last round every CTA writes its tokens' assignments and the
+// owners write the counts, segment offsets and the cluster-sorted permutation
+// that the summaries and stage 2 read.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
@@ -30,7 +38,12 @@ namespace muse {
 
 namespace {
 
-constexpr int kNCF = 256;  // centroids handled by the fused path (one MMA pass)
+constexpr int kNCF = 256;          // centroids handled by the fused path (one MMA pass)
+constexpr int kFT = 256;           // threads of the fused kernel
+constexpr int kWarps = kFT / 32;
+constexpr int kMaxNCT = 16;        // CTAs per problem
+constexpr int kRowsInFlight = 16;  // member rows an owner group loads per batch
+constexpr size_t kSmemLimit = 218 * 1024;  // dynamic shared memory (static arrays come on top)
 
 __device__ inline uint32_t saddr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -85,28 +98,79 @@ __device__ inline void fence_after() { asm volatile("tcgen05.fence::after_thread
 __device__ inline void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
 struct FusedLayout {
-  int KB, NC, tpc;  // K-blocks, centroid columns (multiple of 32), tiles per CTA
-  size_t a, bh, bl, cn2, acc, asg, list, lcnt, loff, total;
+  int KB, NC, tpc, stage;  // K-blocks, centroid columns (multiple of 32), tiles per CTA
+  size_t a, bh, bl, cn2, xs, whist, loff, gtab, xn, asg, queue, cst, total;
 };
 
-__host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc) {
+// Owner groups per CTA: D/8 lanes per cluster.
+__host__ __device__ constexpr int owner_groups(int D) { return kWarps * (32 / (D / 8)); }
+
+__host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc, bool stage) {
   FusedLayout L;
   L.KB = D / 64;
   L.NC = NC;
   L.tpc = tpc;
+  L.stage = stage ? 1 : 0;
   size_t o = 0;
-  L.a = o;    o += (size_t)3 * L.KB * kTile * 128;   // in use, under MMA, loading
-  L.bh = o;   o += (size_t)L.KB * NC * 128;
-  L.bl = o;   o += (size_t)L.KB * NC * 128;
-  L.cn2 = o;  o += (size_t)NC * 4;
+  L.a = o;     o += (size_t)3 * L.KB * kTile * 128;  // in use, under MMA, loading
+  L.bh = o;    o += (size_t)L.KB * NC * 128;
+  L.bl = o;    o += (size_t)L.KB * NC * 128;
+  L.cn2 = o;   o += (size_t)NC * 4;
   o = (o + 15) & ~(size_t)15;
-  L.acc = o;  o += (size_t)NC * D * 8;   // per-cluster fp64 partial sums of this CTA
-  L.lcnt = o; o += (size_t)kNCF * 4;
-  L.loff = o; o += (size_t)(kNCF + 1) * 4;
-  L.asg = o;  o += (size_t)tpc * kTile * 2;
-  L.list = o; o += (size_t)tpc * kTile * 2;
+  L.xs = o;    o += (size_t)kWarps * D * 8;           // queued token rows in fp64
+  L.whist = o; o += (size_t)kWarps * NC * 4;          // per-warp counts, then bases
+  L.loff = o;  o += (size_t)(NC + 1) * 4;
+  L.gtab = o;  o += (size_t)owner_groups(D) * (2 * kMaxNCT + 1) * 4;
+  L.xn = o;    o += (size_t)tpc * kTile * 4;          // token norms (screen bound)
+  L.asg = o;   o += (size_t)tpc * kTile * 2;
+  L.queue = o; o += (size_t)tpc * kTile * 2;
+  o = (o + 15) & ~(size_t)15;
+  L.cst = o;                                          // fp64 centroids, row stride D + 1
+  if (stage) o += (size_t)NC * (D + 1) * 8;
   L.total = o + 1024;
   return L;
+}
+
+// Exact fp64 argmin over the C centroids for one token (x in fp64, shared
+// memory, broadcast), lanes over clusters; ties go to the lowest index.
+template <int D, bool STAGED>
+__device__ inline int exact_argmin(const double* x, const double* cst, const double* c64, int C,
+                                   int lane) {
+  constexpr int MM = kNCF / 32;
+  double sd[MM];
+#pragma unroll
+  for (int m = 0; m < MM; ++m) sd[m] = 0.0;
+  for (int d = 0; d < D; ++d) {
+    const double xd = x[d];
+#pragma unroll
+    for (int m = 0; m < MM; ++m) {
+      const int c = lane + 32 * m;
+      if (c < C) {
+        const double cv = STAGED ? cst[c * (D + 1) + d] : __ldcg(c64 + (size_t)c * D + d);
+        const double t = __dsub_rn(xd, cv);
+        sd[m] = __dadd_rn(sd[m], __dmul_rn(t, t));
+      }
+    }
+  }
+  double bd = 0.0;
+  int bc = -1;
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    const int c = lane + 32 * m;
+    if (c < C && (bc < 0 || sd[m] < bd)) {
+      bd = sd[m];
+      bc = c;
+    }
+  }
+  for (int o = 16; o; o >>= 1) {
+    const double od = __shfl_xor_sync(0xffffffffu, bd, o);
+    const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+    if (oc >= 0 && (bc < 0 || od < bd || (od == bd && oc < bc))) {
+      bd = od;
+      bc = oc;
+    }
+  }
+  return bc;
 }
 
 }  // namespace
@@ -144,64 +208,42 @@ __device__ inline int block_scan_excl(int* a, int n, int* tmp) {
   return total;
 }
 
-constexpr int kFT = 256;  // threads of the fused kernel (8 warps)
-
-// acc[k][.] += x for the warp-uniform k (registers stay registers).
-template <int KA, int R>
-__device__ inline void acc_add(double (&acc)[KA > 0 ? KA : 1][R], int k, const double (&x)[R]) {
-#define MUSE_ACC_CASE(K)                                                     \
-  case K:                                                                    \
-    if (K < (KA > 0 ? KA : 1)) {                                             \
-      _Pragma("unroll") for (int q = 0; q < R; ++q)                          \
-          acc[K < (KA > 0 ? KA : 1) ? K : 0][q] =                            \
-              __dadd_rn(acc[K < (KA > 0 ? KA : 1) ? K : 0][q], x[q]);        \
-    }                                                                        \
-    break;
-  switch (k) {
-    MUSE_ACC_CASE(0) MUSE_ACC_CASE(1) MUSE_ACC_CASE(2) MUSE_ACC_CASE(3)
-    MUSE_ACC_CASE(4) MUSE_ACC_CASE(5) MUSE_ACC_CASE(6) MUSE_ACC_CASE(7)
-    MUSE_ACC_CASE(8) MUSE_ACC_CASE(9) MUSE_ACC_CASE(10) MUSE_ACC_CASE(11)
-    MUSE_ACC_CASE(12) MUSE_ACC_CASE(13) MUSE_ACC_CASE(14) MUSE_ACC_CASE(15)
-    default: break;
-  }
-#undef MUSE_ACC_CASE
-}
-
-// KA > 0: each warp keeps the fp64 sums of its clusters (c = w mod 8, at most
-// 8 KA of them) in registers and the fp64 centroids are staged in shared
-// memory for the re-decision; KA == 0: sums in shared memory, centroids read
-// from L2.
-template <int D, int KA>
+template <int D>
 __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int iters, int NCT,
-                                                             int NC, int tpc_max, int tcols) {
+                                                             int NC, int tpc_max, int tcols,
+                                                             int stage) {
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(1024) unsigned char fz_dyn[];
   unsigned char* base = fz_dyn + ((1024 - (saddr(fz_dyn) & 1023)) & 1023);
-  const FusedLayout Lo = fused_layout(D, NC, tpc_max);
+  const FusedLayout Lo = fused_layout(D, NC, tpc_max, stage != 0);
   const int set = (int)blockIdx.x < fs.nblk0 ? 0 : 1;
   const RoleGeo& g = fs.g[set];
   const KState& ks = fs.ks[set];
   const int blk = (int)blockIdx.x - (set ? fs.nblk0 : 0);
   constexpr int KB = D / 64;
-  constexpr int R = D / 32;
-  constexpr int ATILE = KB * kTile * 128;  // bytes of one swizzled token tile
+  constexpr int LPC = D / 8;                 // owner lanes per cluster, 8 dimensions each
+  constexpr int G = owner_groups(D);         // owner groups per CTA
+  constexpr int EPL = kRowsInFlight / LPC;   // list entries a lane fetches per batch
+  constexpr int ATILE = KB * kTile * 128;    // bytes of one swizzled token tile
   unsigned char* A0 = base + Lo.a;
   unsigned char* BH = base + Lo.bh;
   unsigned char* BL = base + Lo.bl;
   float* cn2s = reinterpret_cast<float*>(base + Lo.cn2);
-  double* sacc = reinterpret_cast<double*>(base + Lo.acc);  // KA > 0: staged centroids first
-  int* lcnt = reinterpret_cast<int*>(base + Lo.lcnt);
+  double* xs = reinterpret_cast<double*>(base + Lo.xs);
+  int* whist = reinterpret_cast<int*>(base + Lo.whist);
   int* loff = reinterpret_cast<int*>(base + Lo.loff);
+  int* gtab = reinterpret_cast<int*>(base + Lo.gtab);
+  float* xns = reinterpret_cast<float*>(base + Lo.xn);
   unsigned short* asg = reinterpret_cast<unsigned short*>(base + Lo.asg);
-  unsigned short* list = reinterpret_cast<unsigned short*>(base + Lo.list);
+  unsigned short* queue = reinterpret_cast<unsigned short*>(base + Lo.queue);
+  double* cst = reinterpret_cast<double*>(base + Lo.cst);
   __shared__ __align__(8) uint64_t mbar[2];
   __shared__ uint32_t tmem_slot;
   __shared__ float hb1[kTile], hb2[kTile];   // upper column half: best, runner-up
   __shared__ int hbi[kTile];
-  __shared__ int tasg[kTile];                // assignment of the tile's tokens
   __shared__ int scan_tmp[32];
   __shared__ float cmax_s;
-  __shared__ int gcnt[kNCF];
+  __shared__ int qcount;
   __shared__ int goff[kNCF + 1];
 
   const int rank = (int)cluster.block_rank();
@@ -210,6 +252,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   const int C = p.C;
   const int ntp = cdiv(p.s, kTile);
   const int tpc = cdiv(ntp, NCT);
+  const int nra = cdiv(ntp, tpc);          // ranks that hold tokens
   const int tile0 = rank * tpc, tile1 = imin(ntp, tile0 + tpc);
   const int ntl = tile1 > tile0 ? tile1 - tile0 : 0;
   const int tok0 = tile0 * kTile, tok1 = imin(p.s, tile1 * kTile);
@@ -219,6 +262,8 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   const int row = tid & (kTile - 1);      // TMEM lane / token row of this thread
   const int half = warp >> 2;             // column half of this thread's epilogue
   const size_t cbase = (size_t)pid * g.C;
+  int* xoff = ks.hist + (size_t)p.tile0 * (g.C + 1);  // row r: rank r's list offsets
+  unsigned short* tl = ks.tlist + p.slot0;           // rank r's list at r * tpc * kTile
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
@@ -242,13 +287,8 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
                          ((uint32_t)(128 >> 4) << 24);
   const double* c64g = ks.cent64 + cbase * D;
 
-  auto xrow = [&](const unsigned char* A, int r, int d) -> float {
-    const int kb = d >> 6, k = d & 63;
-    const unsigned char* pz = A + kb * kTile * 128 + sw128_chunk(r, k >> 3) + ((k & 7) << 1);
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(pz));
-  };
-  auto load_tile = [&](int tl, unsigned char* A) {  // cp.async; caller commits
-    const int t0 = tl * kTile, nt = imin(kTile, p.s - t0);
+  auto load_tile = [&](int tl_, unsigned char* A) {  // cp.async; caller commits
+    const int t0 = tl_ * kTile, nt = imin(kTile, p.s - t0);
     for (int e = tid; e < kTile * KB * 8; e += kFT) {
       const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, cq = q & 7;
       const bool live = r < nt;
@@ -274,7 +314,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
 
   for (int it = 0; it < iters; ++it) {
     const bool last = it + 1 == iters;
-    // ---- centroids of this round (bf16 split; KA > 0: fp64 copy too) ----------
+    // ---- centroids of this round (bf16 split, tensor-core operand) ----------
     for (int e = tid; e < ncp * KB * 8; e += kFT) {
       const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, cq = q & 7;
       const bool live = r < C;
@@ -282,22 +322,21 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       cp16(BH + kb * NC * 128 + sw128_chunk(r, cq), ks.cbf_hi + off, live ? 16 : 0);
       cp16(BL + kb * NC * 128 + sw128_chunk(r, cq), ks.cbf_lo + off, live ? 16 : 0);
     }
-    if (KA > 0)
-      for (int e = tid; e < C * D / 2; e += kFT) cp16(sacc + 2 * e, c64g + 2 * e, 16);
-    if (KA == 0)
-      for (int e = tid; e < C * D; e += kFT) sacc[e] = 0.0;
-    for (int c = tid; c < C; c += kFT) lcnt[c] = 0;
-    if (tid == 0) cmax_s = 0.f;
+    if (tid == 0) {
+      cmax_s = 0.f;
+      qcount = 0;
+    }
     if (ntl > 0) load_tile(tile0, tile_buf(0));
     cp_commit();
     if (ntl > 1) load_tile(tile0 + 1, tile_buf(1));
     cp_commit();
     {
+      // padding columns get +inf so they never win
       float m = 0.f;
-      for (int c = tid; c < C; c += kFT) {
-        const float v = __ldcg(ks.cn2 + cbase + c);
+      for (int c = tid; c < ncp; c += kFT) {
+        const float v = c < C ? __ldcg(ks.cn2 + cbase + c) : INFINITY;
         cn2s[c] = v;
-        m = fmaxf(m, v);
+        if (c < C) m = fmaxf(m, v);
       }
       for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       __syncthreads();
@@ -310,15 +349,11 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     fence_after();
     const float cm = sqrtf(cmax_s) * 1.0001f;
     if (ntl > 0 && tid == 0) issue_mma(tile_buf(0), 0);
-    double racc[KA > 0 ? KA : 1][R];
-#pragma unroll
-    for (int kk = 0; kk < (KA > 0 ? KA : 1); ++kk)
-#pragma unroll
-      for (int q = 0; q < R; ++q) racc[kk][q] = 0.0;
 
     for (int k = 0; k < ntl; ++k) {
-      const int tl = tile0 + k, buf = k & 1;
-      const int t0 = tl * kTile, nt = imin(kTile, p.s - t0);
+      const int tl_ = tile0 + k, buf = k & 1;
+      const int t0 = tl_ * kTile, nt = imin(kTile, p.s - t0);
+      const int u = t0 - tok0 + row;         // CTA-local token index of this row
       const unsigned char* A = tile_buf(k);
       // ---- tile k+1 goes to the tensor cores, tile k+2 starts loading ---------
       if (k + 1 < ntl) {
@@ -328,27 +363,26 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         __syncthreads();
         fence_after();
         if (tid == 0) issue_mma(tile_buf(k + 1), buf ^ 1);
-        if (k + 2 < ntl) load_tile(tl + 2, tile_buf(k + 2));
+        if (k + 2 < ntl) load_tile(tl_ + 2, tile_buf(k + 2));
         cp_commit();
       }
-      // token norm for the screen bound (own row, 16-byte loads)
-      float xn = 0.f;
-      if (tid < nt) {
-        const uint4* xr = reinterpret_cast<const uint4*>(X + (p.row0 + t0 + tid) * D);
+      // token norms for the screen bound, from the staged tile, first round only
+      if (it == 0 && half == 0 && row < nt) {
         float q2 = 0.f;
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 v = xr[c];
-          const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+        for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 f = __bfloat1622float2(b[u]);
-            q2 = fmaf(f.x, f.x, fmaf(f.y, f.y, q2));
+          for (int q = 0; q < 8; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4*>(A + kb * kTile * 128 + sw128_chunk(row, q));
+            const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(b[e]);
+              q2 = fmaf(f.x, f.x, fmaf(f.y, f.y, q2));
+            }
           }
-        }
-        xn = sqrtf(q2) * 1.0001f;
+        xns[u] = sqrtf(q2) * 1.0001f;
       }
-      __syncwarp();
       const bool done = mbar_wait(saddr(&mbar[buf]), phase[buf]);
       phase[buf] ^= 1u;
       const bool ok = __syncthreads_and(done);
@@ -356,53 +390,54 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       fence_after();
       const uint32_t tm = tbase + (uint32_t)(buf * ncp) + ((uint32_t)((warp & 3) * 32) << 16);
       // ---- epilogue: each half of the warps scans half of the columns ---------
-      // four independent best / runner-up trackers (columns c = 4m + u) keep
-      // the compare chain short; merged by (value, index) so ties keep the
-      // lowest index
+      // four independent best / runner-up trackers (columns c = 4m + e) keep
+      // the compare chains short; merged by (value, index)
       float b1 = INFINITY, b2 = INFINITY;
       int bi = 0;
       if (ok) {
         float t1[4], t2[4];
         int ti[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          t1[u] = INFINITY;
-          t2[u] = INFINITY;
-          ti[u] = 0;
+        for (int e = 0; e < 4; ++e) {
+          t1[e] = INFINITY;
+          t2[e] = INFINITY;
+          ti[e] = 0;
         }
         for (int c0 = half * hw; c0 < (half + 1) * hw; c0 += 64) {
           uint32_t rv[4][16];
           const int nb = imin(4, ((half + 1) * hw - c0) / 16);
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (u < nb) tmem_ld16_nw(tm + (uint32_t)(c0 + 16 * u), rv[u]);
+          for (int q = 0; q < 4; ++q)
+            if (q < nb) tmem_ld16_nw(tm + (uint32_t)(c0 + 16 * q), rv[q]);
           tmem_wait();
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (u >= nb) break;
+          for (int q = 0; q < 4; ++q) {
+            if (q >= nb) break;
+            const float4* cq4 = reinterpret_cast<const float4*>(cn2s + c0 + 16 * q);
 #pragma unroll
-            for (int v = 0; v < 16; ++v) {
-              const int c = c0 + 16 * u + v;
-              const int tk = v & 3;
-              const float dd = c < C ? fmaf(-2.f, __uint_as_float(rv[u][v]), cn2s[c]) : INFINITY;
-              if (dd < t1[tk]) {
-                t2[tk] = t1[tk];
-                t1[tk] = dd;
-                ti[tk] = c;
-              } else if (dd < t2[tk]) {
-                t2[tk] = dd;
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const float4 cc = cq4[v4];
+              const float cn[4] = {cc.x, cc.y, cc.z, cc.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = c0 + 16 * q + 4 * v4 + e;
+                const float dd = fmaf(-2.f, __uint_as_float(rv[q][4 * v4 + e]), cn[e]);
+                const bool lt = dd < t1[e];
+                t2[e] = lt ? t1[e] : fminf(t2[e], dd);
+                ti[e] = lt ? c : ti[e];
+                t1[e] = lt ? dd : t1[e];
               }
             }
           }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (t1[u] < b1 || (t1[u] == b1 && ti[u] < bi)) {
-            b2 = fminf(b1, t2[u]);
-            b1 = t1[u];
-            bi = ti[u];
+        for (int e = 0; e < 4; ++e) {
+          if (t1[e] < b1 || (t1[e] == b1 && ti[e] < bi)) {
+            b2 = fminf(b1, t2[e]);
+            b1 = t1[e];
+            bi = ti[e];
           } else {
-            b2 = fminf(b2, t1[u]);
+            b2 = fminf(b2, t1[e]);
           }
         }
       }
@@ -412,7 +447,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         hbi[row] = bi;
       }
       __syncthreads();
-      if (half == 0) {
+      if (half == 0 && row < nt) {
         // merge the upper half (higher indices lose ties)
         const float u1 = hb1[row], u2 = hb2[row];
         if (u1 < b1) {
@@ -424,180 +459,225 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         }
         // |screen - exact| <= 2 eta |x| |c| + 2^-22 (|c|^2 + 2 |x| |c|), eta = 2^-15:
         // bf16 split residual (2^-18) plus fp32 accumulation of 2D exact products
+        const float xn = xns[u];
         const float E = 2.f * 3.0517578e-05f * xn * cm + 2.3841858e-07f * (cm * cm + 2.f * xn * cm);
-        const bool flag = tid < nt && (!ok || (b2 - b1) <= 2.f * E);
-        // exact re-decision: only clusters inside the certified band can win
-        int bx = bi;
-        if (__any_sync(0xffffffffu, flag)) {
-          double best = 0.0;
-          int bc = -1;
-          const float lim = b1 + 2.f * E;
-          for (int cc = 0; cc < ncp; cc += 16) {
-            uint32_t rv[16];
-            if (ok) {
-              tmem_ld16_nw(tm + (uint32_t)cc, rv);
-              tmem_wait();
-            }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const int c = cc + u;
-              const bool cand =
-                  flag && c < C && (!ok || fmaf(-2.f, __uint_as_float(rv[u]), cn2s[c]) <= lim);
-              if (cand) {
-                const double* ccen = (KA > 0 ? (const double*)sacc : c64g) + (size_t)c * D;
-                double sd = 0.0;
-                for (int d0 = 0; d0 < D; d0 += 16) {
-                  double cv[16];
-#pragma unroll
-                  for (int kk = 0; kk < 16; ++kk) cv[kk] = KA > 0 ? ccen[d0 + kk] : __ldcg(ccen + d0 + kk);
-#pragma unroll
-                  for (int kk = 0; kk < 16; ++kk) {
-                    const double t = __dsub_rn((double)xrow(A, row, d0 + kk), cv[kk]);
-                    sd = __dadd_rn(sd, __dmul_rn(t, t));
-                  }
-                }
-                if (bc < 0 || sd < best) {
-                  best = sd;
-                  bc = c;
-                }
-              }
-            }
-          }
-          if (flag) bx = bc;
-        }
-        const int a = tid < nt ? bx : -1;
-        tasg[row] = a;
-        if (a >= 0) {
-          asg[t0 - tok0 + row] = (unsigned short)a;
-          atomicAdd(&lcnt[a], 1);
-          if (last) ks.assign[p.slot0 + t0 + row] = a;
-        }
+        asg[u] = (unsigned short)bi;
+        if (!ok || (b2 - b1) <= 2.f * E) queue[atomicAdd(&qcount, 1)] = (unsigned short)u;
       }
-      fence_before();
-      __syncthreads();
-      // ---- fp64 partial sums: warp w owns the clusters c = w (mod 8) and walks
-      // their tokens in tile order (lanes over dimensions), so every sum sees
-      // its members in ascending token order --------------------------------------
-      for (int r0 = 0; r0 < nt; r0 += 32) {
-        const int ra = r0 + lane < nt ? tasg[r0 + lane] : -1;
-        unsigned mine = __ballot_sync(0xffffffffu, ra >= 0 && (ra & 7) == warp);
-        while (mine) {
-          const int bit = __ffs(mine) - 1;
-          mine &= mine - 1;
-          const int r = r0 + bit;
-          const int a = __shfl_sync(0xffffffffu, ra, bit);
-          double x[R];
-#pragma unroll
-          for (int q = 0; q < R; ++q) x[q] = (double)xrow(A, r, lane + 32 * q);
-          if (KA > 0) {
-            acc_add<KA, R>(racc, a >> 3, x);
-          } else {
-            double* sp = sacc + (size_t)a * D;
-#pragma unroll
-            for (int q = 0; q < R; ++q) sp[lane + 32 * q] = __dadd_rn(sp[lane + 32 * q], x[q]);
-          }
+    }
+    __syncthreads();
+    // ---- exact fp64 decision of the queued tokens, one warp per token --------
+    const int qn = qcount;
+    if (qn > 0) {
+      if (stage) {
+        for (int e = tid; e < C * D; e += kFT) {
+          const int c = e / D, d = e - c * D;
+          cst[c * (D + 1) + d] = __ldcg(c64g + e);
         }
+        __syncthreads();
+      }
+      double* xw = xs + warp * D;
+      for (int e = warp; e < qn; e += kWarps) {
+        const int uq = queue[e];
+        const __nv_bfloat16* xr = X + (p.row0 + tok0 + uq) * D;
+        for (int d = lane; d < D; d += 32) xw[d] = (double)__bfloat162float(xr[d]);
+        __syncwarp();
+        const int bc = stage ? exact_argmin<D, true>(xw, cst, c64g, C, lane)
+                             : exact_argmin<D, false>(xw, cst, c64g, C, lane);
+        if (lane == 0) asg[uq] = (unsigned short)bc;
+        __syncwarp();
       }
       __syncthreads();
     }
-    if (KA > 0) {
-      // the staged centroids are no longer read: publish the sums there
-#pragma unroll
-      for (int kk = 0; kk < (KA > 0 ? KA : 1); ++kk) {
-        const int c = kk * 8 + warp;
-        if (c < C)
-#pragma unroll
-          for (int q = 0; q < R; ++q) sacc[(size_t)c * D + lane + 32 * q] = racc[kk][q];
+    // ---- group this CTA's tokens by cluster (stable) and publish the list ----
+    {
+      const int per = cdiv(cdiv(ntok, kWarps), 32) * 32;
+      const int lo = imin(ntok, warp * per), hi = imin(ntok, lo + per);
+      int* wh = whist + warp * NC;
+      for (int c = lane; c < C; c += 32) wh[c] = 0;
+      __syncwarp();
+      for (int b0 = lo; b0 < hi; b0 += 32) {
+        const int t = b0 + lane;
+        const int a = t < hi ? (int)asg[t] : -1 - lane;
+        const unsigned same = __match_any_sync(0xffffffffu, a);
+        if (a >= 0 && __ffs(same) - 1 == lane) wh[a] += __popc(same);
+        __syncwarp();
       }
-    }
-    // ---- last round: this CTA's tokens grouped by cluster (stable) ----------
-    if (last) {
-      for (int c = tid; c < C; c += kFT) loff[c] = lcnt[c];
+      __syncthreads();
+      for (int c = tid; c < C; c += kFT) {
+        int run = 0;
+        for (int w = 0; w < kWarps; ++w) {
+          const int h = whist[w * NC + c];
+          whist[w * NC + c] = run;
+          run += h;
+        }
+        loff[c] = run;
+      }
       __syncthreads();
       block_scan_excl(loff, C, scan_tmp);
-      if (warp == 0) {
-        for (int b0 = 0; b0 < ntok; b0 += 32) {
-          const int t = b0 + lane;
-          const int aa = t < ntok ? (int)asg[t] : -1 - lane;
-          const unsigned same = __match_any_sync(0xffffffffu, aa);
-          const int rnk = __popc(same & ((1u << lane) - 1u));
-          int pos = 0;
-          if (t < ntok) pos = loff[aa] + rnk;
-          __syncwarp();
-          if (t < ntok) list[pos] = (unsigned short)t;
-          if (t < ntok && rnk == 0) loff[aa] += __popc(same);
-          __syncwarp();
-        }
+      int* xr = xoff + (size_t)rank * (g.C + 1);
+      for (int c = tid; c < C; c += kFT) {
+        const int s0 = loff[c];
+        for (int w = 0; w < kWarps; ++w) whist[w * NC + c] += s0;
+        if (ntok > 0) xr[c] = s0;
       }
+      if (tid == 0 && ntok > 0) xr[C] = ntok;
       __syncthreads();
-      for (int c = tid; c < C; c += kFT) loff[c] -= lcnt[c];  // back to segment starts
+      unsigned short* myl = tl + (size_t)rank * tpc * kTile;
+      for (int b0 = lo; b0 < hi; b0 += 32) {
+        const int t = b0 + lane;
+        const int a = t < hi ? (int)asg[t] : -1 - lane;
+        const unsigned same = __match_any_sync(0xffffffffu, a);
+        if (a >= 0) myl[wh[a] + __popc(same & ((1u << lane) - 1u))] = (unsigned short)t;
+        __syncwarp();
+        if (a >= 0 && __ffs(same) - 1 == lane) wh[a] += __popc(same);
+        __syncwarp();
+      }
+      if (last)
+        for (int t = tid; t < ntok; t += kFT) ks.assign[p.slot0 + tok0 + t] = asg[t];
     }
     __threadfence();
     cluster.sync();
-    // ---- owners: counts, offsets, means from the CTAs' partial sums ----------
-    for (int c = tid; c < C; c += kFT) {
-      int tot = 0;
-      for (int r = 0; r < NCT; ++r) tot += *cluster.map_shared_rank(lcnt + c, r);
-      gcnt[c] = tot;
-    }
-    __syncthreads();
+    // ---- owners: counts, offsets, means over all CTAs' members ----------------
     if (last) {
-      for (int c = tid; c < C; c += kFT) goff[c] = gcnt[c];
+      for (int c = tid; c < C; c += kFT) {
+        int tot = 0;
+        for (int r = 0; r < nra; ++r) {
+          const int* xr = xoff + (size_t)r * (g.C + 1);
+          tot += __ldcg(xr + c + 1) - __ldcg(xr + c);
+        }
+        goff[c] = tot;
+      }
       __syncthreads();
       const int tot = block_scan_excl(goff, C, scan_tmp);
       if (tid == 0) goff[C] = tot;
       __syncthreads();
     }
-    for (int c = rank + NCT * warp; c < C; c += NCT * (kFT / 32)) {
-      const int n = gcnt[c];
-      if (last && lane == 0) {
-        ks.counts[cbase + c] = n;
-        ks.off[(size_t)pid * (g.C + 1) + c] = goff[c];
-        if (c == C - 1) ks.off[(size_t)pid * (g.C + 1) + C] = goff[C];
-      }
-      if (n == 0) continue;  // an empty cluster keeps its centroid
-      double sm[R];
-#pragma unroll
-      for (int q = 0; q < R; ++q) sm[q] = 0.0;
-      for (int rr = 0; rr < NCT; ++rr) {
-        const double* ra = cluster.map_shared_rank(sacc, rr) + (size_t)c * D;
-#pragma unroll
-        for (int q = 0; q < R; ++q) sm[q] = __dadd_rn(sm[q], ra[lane + 32 * q]);
-      }
-      if (last) {
-        int pos = goff[c];
-        for (int rr = 0; rr < NCT; ++rr) {
-          const int m0 = *cluster.map_shared_rank(loff + c, rr);
-          const int mc = *cluster.map_shared_rank(lcnt + c, rr);
-          const unsigned short* rl = cluster.map_shared_rank(list, rr);
-          const int rtok0 = rr * tpc * kTile;
-          for (int m = lane; m < mc; m += 32) ks.perm[p.slot0 + pos + m] = rtok0 + rl[m0 + m];
-          pos += mc;
+    {
+      const int gi = warp * (32 / LPC) + lane / LPC;  // owner group of this lane
+      const int sub = lane % LPC;                     // its 8 dimensions: 8 sub .. 8 sub + 7
+      const int gl0 = lane / LPC * LPC;               // first lane of the group
+      const unsigned gmask = LPC == 32 ? 0xffffffffu : (((1u << LPC) - 1u) << gl0);
+      int* gP = gtab + gi * (2 * kMaxNCT + 1);  // [0, nra]: members before rank r
+      int* gB = gP + kMaxNCT + 1;               // [r]: list index of rank r's first member
+      for (int i = gi;; i += G) {
+        const int c = rank + NCT * i;
+        if (c >= C) break;
+        for (int r = sub; r < nra; r += LPC) {
+          const int* xr = xoff + (size_t)r * (g.C + 1);
+          const int m0 = __ldcg(xr + c), m1 = __ldcg(xr + c + 1);
+          gP[r + 1] = m1 - m0;
+          gB[r] = r * tpc * kTile + m0;
         }
-      }
-      const double nn = (double)n;
-      double q2 = 0.0;
-      float qf = 0.f;
+        __syncwarp(gmask);
+        if (sub == 0) {
+          gP[0] = 0;
+          for (int r = 0; r < nra; ++r) gP[r + 1] += gP[r];
+        }
+        __syncwarp(gmask);
+        const int n = gP[nra];
+        int cur[EPL];
 #pragma unroll
-      for (int q = 0; q < R; ++q) {
-        const double v = __ddiv_rn(sm[q], nn);
-        const float v32 = (float)v;
-        const size_t i = (cbase + c) * D + lane + 32 * q;
-        ks.cent64[i] = v;
-        ks.cent32[i] = v32;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v32);
-        ks.cbf_hi[i] = hi;
-        ks.cbf_lo[i] = __float2bfloat16_rn(v32 - __bfloat162float(hi));
-        q2 += v * v;
-        qf = fmaf(v32, v32, qf);
-      }
-      for (int o = 16; o; o >>= 1) {
-        qf += __shfl_xor_sync(0xffffffffu, qf, o);
-        q2 += __shfl_xor_sync(0xffffffffu, q2, o);
-      }
-      if (lane == 0) {
-        ks.cnorm[cbase + c] = sqrtf(qf) * 1.0001f;
-        ks.cn2[cbase + c] = (float)q2;
+        for (int q = 0; q < EPL; ++q) cur[q] = 0;
+        // problem-local token of member j (concatenated over ranks, ascending)
+        auto fetch = [&](int j0, int (&e)[EPL]) {
+#pragma unroll
+          for (int q = 0; q < EPL; ++q) {
+            const int j = j0 + sub + q * LPC;
+            e[q] = 0;
+            if (j < n) {
+              int r = cur[q];
+              while (gP[r + 1] <= j) ++r;
+              cur[q] = r;
+              e[q] = r * tpc * kTile + (int)__ldcg(tl + gB[r] + (j - gP[r]));
+            }
+          }
+        };
+        double acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.0;
+        int en[EPL];
+        fetch(0, en);
+        for (int j0 = 0; j0 < n; j0 += kRowsInFlight) {
+          int ec[EPL];
+#pragma unroll
+          for (int q = 0; q < EPL; ++q) ec[q] = en[q];
+          uint4 v[kRowsInFlight];
+#pragma unroll
+          for (int k = 0; k < kRowsInFlight; ++k) {
+            const int t = __shfl_sync(gmask, ec[k / LPC], gl0 + k % LPC);
+            v[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (j0 + k < n)
+              v[k] = __ldg(reinterpret_cast<const uint4*>(X + (p.row0 + t) * D + sub * 8));
+          }
+          if (last)
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+              const int j = j0 + sub + q * LPC;
+              if (j < n) ks.perm[p.slot0 + goff[c] + j] = ec[q];
+            }
+          if (j0 + kRowsInFlight < n) fetch(j0 + kRowsInFlight, en);
+#pragma unroll
+          for (int k = 0; k < kRowsInFlight; ++k) {
+            if (j0 + k < n) {
+              const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(b[e]);
+                acc[2 * e] = __dadd_rn(acc[2 * e], (double)f.x);
+                acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], (double)f.y);
+              }
+            }
+          }
+        }
+        if (last && sub == 0) {
+          ks.counts[cbase + c] = n;
+          ks.off[(size_t)pid * (g.C + 1) + c] = goff[c];
+          if (c == C - 1) ks.off[(size_t)pid * (g.C + 1) + C] = goff[C];
+        }
+        if (n > 0) {  // an empty cluster keeps its centroid
+          const double nn = (double)n;
+          double q2 = 0.0;
+          float qf = 0.f;
+          double v64[8];
+          float v32[8];
+          __nv_bfloat16 hi[8], lo[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            v64[q] = __ddiv_rn(acc[q], nn);
+            v32[q] = (float)v64[q];
+            hi[q] = __float2bfloat16_rn(v32[q]);
+            lo[q] = __float2bfloat16_rn(v32[q] - __bfloat162float(hi[q]));
+            q2 += v64[q] * v64[q];
+            qf = fmaf(v32[q], v32[q], qf);
+          }
+          const size_t i0 = (cbase + c) * D + sub * 8;
+          double2* d64 = reinterpret_cast<double2*>(ks.cent64 + i0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) d64[q] = make_double2(v64[2 * q], v64[2 * q + 1]);
+          float4* d32 = reinterpret_cast<float4*>(ks.cent32 + i0);
+          d32[0] = make_float4(v32[0], v32[1], v32[2], v32[3]);
+          d32[1] = make_float4(v32[4], v32[5], v32[6], v32[7]);
+          uint32_t wh[4], wl[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            wh[q] = (uint32_t)__bfloat16_as_ushort(hi[2 * q]) |
+                    ((uint32_t)__bfloat16_as_ushort(hi[2 * q + 1]) << 16);
+            wl[q] = (uint32_t)__bfloat16_as_ushort(lo[2 * q]) |
+                    ((uint32_t)__bfloat16_as_ushort(lo[2 * q + 1]) << 16);
+          }
+          *reinterpret_cast<uint4*>(ks.cbf_hi + i0) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          *reinterpret_cast<uint4*>(ks.cbf_lo + i0) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          for (int o = LPC / 2; o; o >>= 1) {
+            qf += __shfl_xor_sync(gmask, qf, o);
+            q2 += __shfl_xor_sync(gmask, q2, o);
+          }
+          if (sub == 0) {
+            ks.cnorm[cbase + c] = sqrtf(qf) * 1.0001f;
+            ks.cn2[cbase + c] = (float)q2;
+          }
+        }
+        __syncwarp(gmask);  // the group's tables are rewritten for its next cluster
       }
     }
     __threadfence();
@@ -611,7 +691,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
 
 // Returns false (nothing launched) when the fused path does not cover these
 // problem sets: more than 256 clusters, or more than 65535 tokens per CTA.
-template <int D, int KA>
+template <int D>
 static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int iters,
                            cudaStream_t st) {
   int cmax = 0;
@@ -628,10 +708,10 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
   int NCT = 0;
   FusedLayout L{};
   const bool big_ok =
-      cudaFuncSetAttribute(kmeans_fused_kernel<D, KA>,
+      cudaFuncSetAttribute(kmeans_fused_kernel<D>,
                            cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
   if (!big_ok) cudaGetLastError();
-  for (int nct = big_ok ? 16 : 8; nct >= 1; --nct) {
+  for (int nct = big_ok ? kMaxNCT : 8; nct >= 1; --nct) {
     int tpc_max = 1;
     for (int k = 0; k < nsets; ++k)
       for (int l = 0; l < gs[k].lv.nlev; ++l) {
@@ -639,9 +719,10 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
         tpc_max = tpc_max > tpc ? tpc_max : tpc;
       }
     if (tpc_max * kTile > 65535) break;
-    const FusedLayout Lc = fused_layout(D, NC, tpc_max);
-    if (Lc.total > 218 * 1024) continue;  // leaves room for the static shared arrays
-    cudaFuncSetAttribute(kmeans_fused_kernel<D, KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    FusedLayout Lc = fused_layout(D, NC, tpc_max, true);
+    if (Lc.total > kSmemLimit) Lc = fused_layout(D, NC, tpc_max, false);
+    if (Lc.total > kSmemLimit) continue;
+    cudaFuncSetAttribute(kmeans_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)Lc.total);
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3((unsigned)(nprob * nct));
@@ -655,7 +736,7 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
     q.attrs = qa;
     q.numAttrs = 1;
     int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, kmeans_fused_kernel<D, KA>, &q) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&active, kmeans_fused_kernel<D>, &q) != cudaSuccess) {
       cudaGetLastError();
       active = 0;
     }
@@ -677,7 +758,7 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
   }
   fs.nblk0 = kss[0].nprob * NCT;
   const int nblk = fs.nblk0 + (nsets > 1 ? kss[1].nprob * NCT : 0);
-  cudaFuncSetAttribute(kmeans_fused_kernel<D, KA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaFuncSetAttribute(kmeans_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)L.total);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)nblk);
@@ -691,20 +772,14 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, KA>, fs, iters, NCT, NC, L.tpc, tcols);
+  cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D>, fs, iters, NCT, NC, L.tpc, tcols, L.stage);
   return true;
 }
 
 bool launch_kmeans_fused(const RoleGeo* gs, const KState* kss, int nsets, int iters,
                          cudaStream_t st) {
-  int cmax = 0;
-  for (int k = 0; k < nsets; ++k) cmax = cmax > gs[k].C ? cmax : gs[k].C;
-  // register sums when a warp's clusters (C / 8) x its dimensions (D / 32) fit in 32 doubles
-  if (gs[0].D == 64)
-    return cmax <= 128 ? launch_fused_t<64, 16>(gs, kss, nsets, iters, st)
-                       : launch_fused_t<64, 0>(gs, kss, nsets, iters, st);
-  return cmax <= 64 ? launch_fused_t<128, 8>(gs, kss, nsets, iters, st)
-                    : launch_fused_t<128, 0>(gs, kss, nsets, iters, st);
+  return gs[0].D == 64 ? launch_fused_t<64>(gs, kss, nsets, iters, st)
+                       : launch_fused_t<128>(gs, kss, nsets, iters, st);
 }
 
 }  // namespace muse
