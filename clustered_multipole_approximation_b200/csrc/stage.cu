@@ -271,33 +271,72 @@ __global__ void __launch_bounds__(kS1T) stage1_kernel(AttnArgs a, Stage1 s1, int
 // selection: top-k key clusters per query cluster by s nu_i.mu_j + log W_ij,
 // ties to the lowest j, empty clusters never
 // ----------------------------------------------------------------------------
+// Query clusters handled by one CTA of the selection kernel (two per warp).
+constexpr int kSelQ = 16;
+
+// Key centroids per CTA staged in shared memory when they fit (row stride
+// D + 1 doubles keeps the lanes' rows on distinct banks).
 template <int D>
+constexpr size_t select_stage_bytes(int Ck) {
+  return (size_t)Ck * (D + 1) * sizeof(double);
+}
+constexpr size_t kSelectSmemMax = 200 * 1024;
+
+// One warp per query cluster: lanes over key clusters, four key clusters per
+// lane at a time (independent fp64 chains, each in dimension order with no
+// fused operations, as a plain sequential evaluation), then top-k1 by k1
+// rounds of warp argmax, ties to the lowest index.
+template <int D, bool STAGED>
 __global__ void __launch_bounds__(256) select_kernel(AttnArgs a, Stage1 s1, int qp0) {
-  extern __shared__ double sc_all[];  // [8][Ck]
+  extern __shared__ double sel_smem[];
   const int lq = blockIdx.x, qpid = qp0 + lq;
   const Prob pq = prob_of(a.qg, qpid);
   const int kpid = kv_problem(a, qpid);
   const Prob pk = prob_of(a.kg, kpid);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Cq = a.Cq, Ck = a.Ck, K1 = a.topk;
-  double* sc = sc_all + (size_t)warp * Ck;
+  const int ck = pk.C;
+  const double* mug = a.ks.cent64 + (size_t)kpid * Ck * D;
+  double* mus = sel_smem;                                            // [ck][D + 1]
+  double* sc = sel_smem + (STAGED ? (size_t)Ck * (D + 1) : 0) + (size_t)warp * Ck;
+  if (STAGED) {
+    for (int e = threadIdx.x; e < ck * D; e += blockDim.x) {
+      const int j = e / D, d = e - j * D;
+      mus[j * (D + 1) + d] = mug[e];
+    }
+    __syncthreads();
+  }
   const double s = (double)a.scale;
   const int* kc = a.ks.counts + (size_t)kpid * Ck;
-  {
-    const int i = blockIdx.y * 8 + warp;
-    if (i >= pq.C) return;  // warp-uniform; no CTA-wide barrier below
+  const int i1 = imin(pq.C, (blockIdx.y + 1) * kSelQ);
+  for (int i = blockIdx.y * kSelQ + warp; i < i1; i += 8) {  // warp-uniform
     const double* nu = a.qs.cent64 + ((size_t)qpid * Cq + i) * D;
-    for (int j = lane; j < pk.C; j += 32) {
-      double v = -INFINITY;
-      if (kc[j] > 0) {
-        const double* mu = a.ks.cent64 + ((size_t)kpid * Ck + j) * D;
-        double dt = 0.0;
-        for (int d = 0; d < D; ++d) dt = __dadd_rn(dt, __dmul_rn(nu[d], mu[d]));
-        const double lw = (a.mode == 2) ? (double)s1.logW[((size_t)lq * Cq + i) * Ck + j]
-                                        : log((double)kc[j]);
-        v = __dadd_rn(__dmul_rn(s, dt), lw);
+    for (int jb = 0; jb < ck; jb += 128) {
+      double dt[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int d = 0; d < D; ++d) {
+        const double nv = nu[d];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = jb + lane + 32 * u;
+          if (j < ck) {
+            const double mv = STAGED ? mus[j * (D + 1) + d] : mug[(size_t)j * D + d];
+            dt[u] = __dadd_rn(dt[u], __dmul_rn(nv, mv));
+          }
+        }
       }
-      sc[j] = v;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = jb + lane + 32 * u;
+        if (j < ck) {
+          double v = -INFINITY;
+          if (kc[j] > 0) {
+            const double lw = (a.mode == 2) ? (double)s1.logW[((size_t)lq * Cq + i) * Ck + j]
+                                            : log((double)kc[j]);
+            v = __dadd_rn(__dmul_rn(s, dt[u]), lw);
+          }
+          sc[j] = v;
+        }
+      }
     }
     __syncwarp();
     int taken = 0;
@@ -305,9 +344,9 @@ __global__ void __launch_bounds__(256) select_kernel(AttnArgs a, Stage1 s1, int 
     for (int r = 0; r < K1; ++r) {
       double bv = -INFINITY;
       int bj = -1;
-      for (int j = lane; j < pk.C; j += 32) {
+      for (int j = lane; j < ck; j += 32) {
         const double v = sc[j];
-        if (kc[j] > 0 && v > -INFINITY && (bj < 0 || v > bv)) {
+        if (v > -INFINITY && (bj < 0 || v > bv)) {
           bv = v;
           bj = j;
         }
@@ -589,7 +628,9 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
   if (!attr) {
     cudaFuncSetAttribute(stage1_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)stage1_smem<D>());
-    cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(select_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kSelectSmemMax);
+    cudaFuncSetAttribute(select_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          8 * kMaxC * (int)sizeof(double));
     attr = true;
   }
@@ -603,7 +644,11 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
   if (a.topk > 0) {
     ProfScope ps(st, "stage1_select");
     const size_t smem = (size_t)8 * a.Ck * sizeof(double);
-    select_kernel<D><<<dim3(nqp, cdiv(a.Cq, 8)), 256, smem, st>>>(a, s1, qp0);
+    const dim3 grid(nqp, cdiv(a.Cq, kSelQ));
+    if (smem + select_stage_bytes<D>(a.Ck) <= kSelectSmemMax)
+      select_kernel<D, true><<<grid, 256, smem + select_stage_bytes<D>(a.Ck), st>>>(a, s1, qp0);
+    else
+      select_kernel<D, false><<<grid, 256, smem, st>>>(a, s1, qp0);
   }
   if (sizeof(T) == 2) {
     ProfScope ps(st, "stage2_attn");
