@@ -17,11 +17,12 @@
 //      no fused operations (a plain sequential fp64 evaluation, bit for bit);
 //   3. the CTA groups its tokens by cluster (stable counting sort) and
 //      publishes the grouped list and its per-cluster offsets in global memory;
-//   4. cluster barrier; cluster c is owned by CTA rank c % NCT, where a group
-//      of D/8 lanes walks the members of c over all CTAs in ascending token
-//      order and sums their rows in fp64 -- the order of a plain sequential
-//      evaluation -- with 16 rows in flight, then writes the new centroid
-//      (fp64, fp32, bf16 hi/lo, norms) to global memory;
+//   4. cluster barrier; cluster c is owned by CTA rank c % NCT, where one warp
+//      (clusters taken largest first) walks the members of c over all CTAs in
+//      ascending token order and sums their rows in fp64 -- the order of a
+//      plain sequential evaluation -- lanes over dimensions, with the next
+//      batch of rows in flight, then writes the new centroid (fp64, fp32,
+//      bf16 hi/lo, norms) to global memory;
 //   5. cluster barrier, next round.
 // After the last round every CTA writes its tokens' assignments and the
 // owners write the counts, segment offsets and the cluster-sorted permutation
@@ -42,7 +43,6 @@ constexpr int kNCF = 256;          // centroids handled by the fused path (one M
 constexpr int kFT = 256;           // threads of the fused kernel
 constexpr int kWarps = kFT / 32;
 constexpr int kMaxNCT = 16;        // CTAs per problem
-constexpr int kRowsInFlight = 16;  // member rows an owner group loads per batch
 constexpr size_t kSmemLimit = 218 * 1024;  // dynamic shared memory (static arrays come on top)
 
 __device__ inline uint32_t saddr(const void* p) {
@@ -102,9 +102,6 @@ struct FusedLayout {
   size_t a, bh, bl, cn2, xs, whist, loff, gtab, xn, asg, queue, cst, total;
 };
 
-// Owner groups per CTA: D/8 lanes per cluster.
-__host__ __device__ constexpr int owner_groups(int D) { return kWarps * (32 / (D / 8)); }
-
 __host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc, bool stage) {
   FusedLayout L;
   L.KB = D / 64;
@@ -120,7 +117,7 @@ __host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc, bool
   L.xs = o;    o += (size_t)kWarps * D * 8;           // queued token rows in fp64
   L.whist = o; o += (size_t)kWarps * NC * 4;          // per-warp counts, then bases
   L.loff = o;  o += (size_t)(NC + 1) * 4;
-  L.gtab = o;  o += (size_t)owner_groups(D) * (2 * kMaxNCT + 1) * 4;
+  L.gtab = o;  o += (size_t)kWarps * (2 * kMaxNCT + 1) * 4;   // owner warps' rank tables
   L.xn = o;    o += (size_t)tpc * kTile * 4;          // token norms (screen bound)
   L.asg = o;   o += (size_t)tpc * kTile * 2;
   L.queue = o; o += (size_t)tpc * kTile * 2;
@@ -129,6 +126,31 @@ __host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc, bool
   if (stage) o += (size_t)NC * (D + 1) * 8;
   L.total = o + 1024;
   return L;
+}
+
+// A lane's share of one bf16 row in the owner sums: D / 32 consecutive values.
+template <int D>
+struct LaneRow;
+template <>
+struct LaneRow<64> {
+  using T = uint32_t;
+};
+template <>
+struct LaneRow<128> {
+  using T = uint2;
+};
+__device__ inline void add_row(double (&acc)[2], uint32_t w) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  acc[0] = __dadd_rn(acc[0], (double)f.x);
+  acc[1] = __dadd_rn(acc[1], (double)f.y);
+}
+__device__ inline void add_row(double (&acc)[4], uint2 w) {
+  const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+  const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+  acc[0] = __dadd_rn(acc[0], (double)f0.x);
+  acc[1] = __dadd_rn(acc[1], (double)f0.y);
+  acc[2] = __dadd_rn(acc[2], (double)f1.x);
+  acc[3] = __dadd_rn(acc[3], (double)f1.y);
 }
 
 // Exact fp64 argmin over the C centroids for one token (x in fp64, shared
@@ -221,9 +243,9 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   const KState& ks = fs.ks[set];
   const int blk = (int)blockIdx.x - (set ? fs.nblk0 : 0);
   constexpr int KB = D / 64;
-  constexpr int LPC = D / 8;                 // owner lanes per cluster, 8 dimensions each
-  constexpr int G = owner_groups(D);         // owner groups per CTA
-  constexpr int EPL = kRowsInFlight / LPC;   // list entries a lane fetches per batch
+  constexpr int VPL = D / 32;                // owner sums: dimensions per lane
+  constexpr int kOB = D == 64 ? 32 : 16;     // owner sums: member rows per batch
+  using RowT = typename LaneRow<D>::T;
   constexpr int ATILE = KB * kTile * 128;    // bytes of one swizzled token tile
   unsigned char* A0 = base + Lo.a;
   unsigned char* BH = base + Lo.bh;
@@ -245,6 +267,8 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   __shared__ float cmax_s;
   __shared__ int qcount;
   __shared__ int goff[kNCF + 1];
+  __shared__ int own_n[kNCF], own_ord[kNCF];  // owned clusters: sizes, largest-first order
+  __shared__ int own_ctr;
 
   const int rank = (int)cluster.block_rank();
   const int pid = blk / NCT;
@@ -470,9 +494,19 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     const int qn = qcount;
     if (qn > 0) {
       if (stage) {
-        for (int e = tid; e < C * D; e += kFT) {
-          const int c = e / D, d = e - c * D;
-          cst[c * (D + 1) + d] = __ldcg(c64g + e);
+        const int tot = C * D;
+        for (int e0 = tid; e0 < tot; e0 += 16 * kFT) {  // 16 loads in flight per thread
+          double v[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) v[u] = e0 + u * kFT < tot ? __ldcg(c64g + e0 + u * kFT) : 0.0;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int e = e0 + u * kFT;
+            if (e < tot) {
+              const int c = e / D, d = e - c * D;
+              cst[c * (D + 1) + d] = v[u];
+            }
+          }
         }
         __syncthreads();
       }
@@ -553,84 +587,99 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       if (tid == 0) goff[C] = tot;
       __syncthreads();
     }
+    // ---- owners: this CTA's clusters, largest first, one warp per cluster ----
     {
-      const int gi = warp * (32 / LPC) + lane / LPC;  // owner group of this lane
-      const int sub = lane % LPC;                     // its 8 dimensions: 8 sub .. 8 sub + 7
-      const int gl0 = lane / LPC * LPC;               // first lane of the group
-      const unsigned gmask = LPC == 32 ? 0xffffffffu : (((1u << LPC) - 1u) << gl0);
-      int* gP = gtab + gi * (2 * kMaxNCT + 1);  // [0, nra]: members before rank r
-      int* gB = gP + kMaxNCT + 1;               // [r]: list index of rank r's first member
-      for (int i = gi;; i += G) {
+      const int nown = C > rank ? cdiv(C - rank, NCT) : 0;  // clusters rank + NCT i
+      for (int i = tid; i < nown; i += kFT) {
         const int c = rank + NCT * i;
-        if (c >= C) break;
-        for (int r = sub; r < nra; r += LPC) {
+        int n = 0;
+        for (int r = 0; r < nra; ++r) {
           const int* xr = xoff + (size_t)r * (g.C + 1);
-          const int m0 = __ldcg(xr + c), m1 = __ldcg(xr + c + 1);
-          gP[r + 1] = m1 - m0;
-          gB[r] = r * tpc * kTile + m0;
+          n += __ldcg(xr + c + 1) - __ldcg(xr + c);
         }
-        __syncwarp(gmask);
-        if (sub == 0) {
-          gP[0] = 0;
-          for (int r = 0; r < nra; ++r) gP[r + 1] += gP[r];
-        }
-        __syncwarp(gmask);
-        const int n = gP[nra];
-        int cur[EPL];
-#pragma unroll
-        for (int q = 0; q < EPL; ++q) cur[q] = 0;
-        // problem-local token of member j (concatenated over ranks, ascending)
-        auto fetch = [&](int j0, int (&e)[EPL]) {
-#pragma unroll
-          for (int q = 0; q < EPL; ++q) {
-            const int j = j0 + sub + q * LPC;
-            e[q] = 0;
-            if (j < n) {
-              int r = cur[q];
-              while (gP[r + 1] <= j) ++r;
-              cur[q] = r;
-              e[q] = r * tpc * kTile + (int)__ldcg(tl + gB[r] + (j - gP[r]));
-            }
+        own_n[i] = n;
+      }
+      __syncthreads();
+      if (tid == 0) {  // sizes descending, so the largest clusters start first
+        own_ctr = 0;
+        for (int i = 0; i < nown; ++i) {
+          const int nv = own_n[i];
+          int j = i - 1;
+          while (j >= 0 && own_n[own_ord[j]] < nv) {
+            own_ord[j + 1] = own_ord[j];
+            --j;
           }
+          own_ord[j + 1] = i;
+        }
+      }
+      __syncthreads();
+      int* gP = gtab + warp * (2 * kMaxNCT + 1);  // [0, nra]: members before rank r
+      int* gB = gP + kMaxNCT + 1;                 // [r]: list index of rank r's first member
+      const RowT* Xl = reinterpret_cast<const RowT*>(X + p.row0 * D) + lane;
+      for (;;) {
+        int k = 0;
+        if (lane == 0) k = atomicAdd(&own_ctr, 1);
+        k = __shfl_sync(0xffffffffu, k, 0);
+        if (k >= nown) break;
+        const int c = rank + NCT * own_ord[k];
+        const int n = own_n[own_ord[k]];
+        int cnt = 0, m0 = 0;
+        if (lane < nra) {
+          const int* xr = xoff + (size_t)lane * (g.C + 1);
+          m0 = __ldcg(xr + c);
+          cnt = __ldcg(xr + c + 1) - m0;
+        }
+        int incl = cnt;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (lane < nra) {
+          gP[lane] = incl - cnt;
+          gB[lane] = lane * tpc * kTile + m0;
+        }
+        if (lane == 0) gP[nra] = n;
+        __syncwarp();
+        // member j (concatenated over ranks, ascending token order) -> its
+        // problem-local token; lanes fetch the entries of a batch in parallel
+        int cur = 0;
+        auto entry = [&](int j) -> int {
+          if (j >= n || lane >= kOB) return 0;
+          while (gP[cur + 1] <= j) ++cur;
+          return cur * tpc * kTile + (int)__ldcg(tl + gB[cur] + (j - gP[cur]));
         };
-        double acc[8];
+        const size_t pbase = (size_t)p.slot0 + (last ? goff[c] : 0);
+        double acc[VPL];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] = 0.0;
-        int en[EPL];
-        fetch(0, en);
-        for (int j0 = 0; j0 < n; j0 += kRowsInFlight) {
-          int ec[EPL];
+        for (int e = 0; e < VPL; ++e) acc[e] = 0.0;
+        // two batches in flight: rows of batch b+1 load while batch b is summed
+        int ec = entry(lane);
+        RowT vc[kOB];
 #pragma unroll
-          for (int q = 0; q < EPL; ++q) ec[q] = en[q];
-          uint4 v[kRowsInFlight];
-#pragma unroll
-          for (int k = 0; k < kRowsInFlight; ++k) {
-            const int t = __shfl_sync(gmask, ec[k / LPC], gl0 + k % LPC);
-            v[k] = make_uint4(0u, 0u, 0u, 0u);
-            if (j0 + k < n)
-              v[k] = __ldg(reinterpret_cast<const uint4*>(X + (p.row0 + t) * D + sub * 8));
-          }
-          if (last)
-#pragma unroll
-            for (int q = 0; q < EPL; ++q) {
-              const int j = j0 + sub + q * LPC;
-              if (j < n) ks.perm[p.slot0 + goff[c] + j] = ec[q];
-            }
-          if (j0 + kRowsInFlight < n) fetch(j0 + kRowsInFlight, en);
-#pragma unroll
-          for (int k = 0; k < kRowsInFlight; ++k) {
-            if (j0 + k < n) {
-              const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(b[e]);
-                acc[2 * e] = __dadd_rn(acc[2 * e], (double)f.x);
-                acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], (double)f.y);
-              }
-            }
-          }
+        for (int q = 0; q < kOB; ++q) {
+          const int t = __shfl_sync(0xffffffffu, ec, q);
+          vc[q] = q < n ? __ldg(Xl + (size_t)t * (D / VPL)) : RowT{};
         }
-        if (last && sub == 0) {
+        if (last && lane < kOB && lane < n) ks.perm[pbase + lane] = ec;
+        int en = entry(kOB + lane);
+        for (int j0 = 0; j0 < n; j0 += kOB) {
+          const bool more = j0 + kOB < n;
+          RowT vn[kOB];
+#pragma unroll
+          for (int q = 0; q < kOB; ++q) {
+            const int t = __shfl_sync(0xffffffffu, en, q);
+            vn[q] = more && j0 + kOB + q < n ? __ldg(Xl + (size_t)t * (D / VPL)) : RowT{};
+          }
+          if (last && more && lane < kOB && j0 + kOB + lane < n) ks.perm[pbase + j0 + kOB + lane] = en;
+          const int en2 = more ? entry(j0 + 2 * kOB + lane) : 0;
+#pragma unroll
+          for (int q = 0; q < kOB; ++q)
+            if (j0 + q < n) add_row(acc, vc[q]);
+#pragma unroll
+          for (int q = 0; q < kOB; ++q) vc[q] = vn[q];
+          en = en2;
+        }
+        if (last && lane == 0) {
           ks.counts[cbase + c] = n;
           ks.off[(size_t)pid * (g.C + 1) + c] = goff[c];
           if (c == C - 1) ks.off[(size_t)pid * (g.C + 1) + C] = goff[C];
@@ -639,45 +688,43 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
           const double nn = (double)n;
           double q2 = 0.0;
           float qf = 0.f;
-          double v64[8];
-          float v32[8];
-          __nv_bfloat16 hi[8], lo[8];
+          double v64[VPL];
+          float v32[VPL];
+          uint32_t wh[VPL / 2], wl[VPL / 2];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            v64[q] = __ddiv_rn(acc[q], nn);
-            v32[q] = (float)v64[q];
-            hi[q] = __float2bfloat16_rn(v32[q]);
-            lo[q] = __float2bfloat16_rn(v32[q] - __bfloat162float(hi[q]));
-            q2 += v64[q] * v64[q];
-            qf = fmaf(v32[q], v32[q], qf);
+          for (int e = 0; e < VPL; ++e) {
+            v64[e] = __ddiv_rn(acc[e], nn);
+            v32[e] = (float)v64[e];
+            q2 += v64[e] * v64[e];
+            qf = fmaf(v32[e], v32[e], qf);
           }
-          const size_t i0 = (cbase + c) * D + sub * 8;
-          double2* d64 = reinterpret_cast<double2*>(ks.cent64 + i0);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) d64[q] = make_double2(v64[2 * q], v64[2 * q + 1]);
-          float4* d32 = reinterpret_cast<float4*>(ks.cent32 + i0);
-          d32[0] = make_float4(v32[0], v32[1], v32[2], v32[3]);
-          d32[1] = make_float4(v32[4], v32[5], v32[6], v32[7]);
-          uint32_t wh[4], wl[4];
+          for (int e = 0; e < VPL / 2; ++e) {
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(v32[2 * e]);
+            const __nv_bfloat16 h1 = __float2bfloat16_rn(v32[2 * e + 1]);
+            const __nv_bfloat16 l0 = __float2bfloat16_rn(v32[2 * e] - __bfloat162float(h0));
+            const __nv_bfloat16 l1 = __float2bfloat16_rn(v32[2 * e + 1] - __bfloat162float(h1));
+            wh[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+            wl[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+          }
+          const size_t i0 = (cbase + c) * D + (size_t)lane * VPL;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            wh[q] = (uint32_t)__bfloat16_as_ushort(hi[2 * q]) |
-                    ((uint32_t)__bfloat16_as_ushort(hi[2 * q + 1]) << 16);
-            wl[q] = (uint32_t)__bfloat16_as_ushort(lo[2 * q]) |
-                    ((uint32_t)__bfloat16_as_ushort(lo[2 * q + 1]) << 16);
+          for (int e = 0; e < VPL / 2; ++e) {
+            reinterpret_cast<double2*>(ks.cent64 + i0)[e] = make_double2(v64[2 * e], v64[2 * e + 1]);
+            reinterpret_cast<float2*>(ks.cent32 + i0)[e] = make_float2(v32[2 * e], v32[2 * e + 1]);
+            reinterpret_cast<uint32_t*>(ks.cbf_hi + i0)[e] = wh[e];
+            reinterpret_cast<uint32_t*>(ks.cbf_lo + i0)[e] = wl[e];
           }
-          *reinterpret_cast<uint4*>(ks.cbf_hi + i0) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-          *reinterpret_cast<uint4*>(ks.cbf_lo + i0) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-          for (int o = LPC / 2; o; o >>= 1) {
-            qf += __shfl_xor_sync(gmask, qf, o);
-            q2 += __shfl_xor_sync(gmask, q2, o);
+          for (int o = 16; o; o >>= 1) {
+            qf += __shfl_xor_sync(0xffffffffu, qf, o);
+            q2 += __shfl_xor_sync(0xffffffffu, q2, o);
           }
-          if (sub == 0) {
+          if (lane == 0) {
             ks.cnorm[cbase + c] = sqrtf(qf) * 1.0001f;
             ks.cn2[cbase + c] = (float)q2;
           }
         }
-        __syncwarp(gmask);  // the group's tables are rewritten for its next cluster
+        __syncwarp();  // the warp's tables are rewritten for its next cluster
       }
     }
     __threadfence();
