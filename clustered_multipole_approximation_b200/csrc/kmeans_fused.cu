@@ -1,5 +1,7 @@
-// Persistent Lloyd k-means for bf16 inputs: one thread-block cluster of NCT
-// CTAs per problem runs every round in a single launch.
+// Persistent Lloyd k-means for bf16 inputs: NCT CTAs per problem run every
+// round in a single launch -- a cooperative launch when all problems fit on
+// the GPU at once with more CTAs each than a thread-block cluster allows,
+// else one thread-block cluster per problem.
 //
 // The clustering step of MuSe (gist.science page "Multipole Semantic
 // Attention: A Fast Approximation of Softmax Attention for Pretraining",
@@ -17,13 +19,13 @@
 //      no fused operations (a plain sequential fp64 evaluation, bit for bit);
 //   3. the CTA groups its tokens by cluster (stable counting sort) and
 //      publishes the grouped list and its per-cluster offsets in global memory;
-//   4. cluster barrier; cluster c is owned by CTA rank c % NCT, where one warp
+//   4. barrier; cluster c is owned by CTA rank c % NCT, where one warp
 //      (clusters taken largest first) walks the members of c over all CTAs in
 //      ascending token order and sums their rows in fp64 -- the order of a
 //      plain sequential evaluation -- lanes over dimensions, with the next
 //      batch of rows in flight, then writes the new centroid (fp64, fp32,
 //      bf16 hi/lo, norms) to global memory;
-//   5. cluster barrier, next round.
+//   5. barrier, next round.
 // After the last round every CTA writes its tokens' assignments and the
 // owners write the counts, segment offsets and the cluster-sorted permutation
 // that the summaries and stage 2 read.
@@ -42,7 +44,8 @@ namespace {
 constexpr int kNCF = 256;          // centroids handled by the fused path (one MMA pass)
 constexpr int kFT = 256;           // threads of the fused kernel
 constexpr int kWarps = kFT / 32;
-constexpr int kMaxNCT = 16;        // CTAs per problem
+constexpr int kMaxNCT = 32;        // CTAs per problem
+constexpr int kSpinLimit = 1 << 24;  // team barrier polls (64 ns apart) before giving up
 constexpr size_t kSmemLimit = 218 * 1024;  // dynamic shared memory (static arrays come on top)
 
 __device__ inline uint32_t saddr(const void* p) {
@@ -230,7 +233,10 @@ __device__ inline int block_scan_excl(int* a, int n, int* tmp) {
   return total;
 }
 
-template <int D>
+// COOP: a cooperative launch of NCT CTAs per problem (all resident at once;
+// a problem's CTAs meet at a barrier on a workspace counter); otherwise one
+// thread-block cluster of NCT CTAs per problem (hardware cluster barrier).
+template <int D, bool COOP>
 __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int iters, int NCT,
                                                              int NC, int tpc_max, int tcols,
                                                              int stage) {
@@ -269,8 +275,9 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   __shared__ int goff[kNCF + 1];
   __shared__ int own_n[kNCF], own_ord[kNCF];  // owned clusters: sizes, largest-first order
   __shared__ int own_ctr;
+  __shared__ int bar_fail;
 
-  const int rank = (int)cluster.block_rank();
+  const int rank = COOP ? (int)blockIdx.x % NCT : (int)cluster.block_rank();
   const int pid = blk / NCT;
   const Prob p = prob_of(g, pid);
   const int C = p.C;
@@ -287,6 +294,37 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   const int half = warp >> 2;             // column half of this thread's epilogue
   const size_t cbase = (size_t)pid * g.C;
   int* xoff = ks.hist + (size_t)p.tile0 * (g.C + 1);  // row r: rank r's list offsets
+  // team barrier (COOP): arrival counter of this problem, monotonic over the launch
+  int* bar_ctr = ks.arrive + pid;
+  int nbar = 0;
+  auto team_sync = [&]() {
+    if (COOP) {
+      __syncthreads();
+      if (tid == 0) {
+        ++nbar;
+        __threadfence();
+        atomicAdd(bar_ctr, 1);
+        if (!bar_fail) {
+          for (int it = 0;; ++it) {
+            int v;
+            asm volatile("ld.acquire.gpu.global.s32 %0, [%1];\n" : "=r"(v) : "l"(bar_ctr) : "memory");
+            if (v >= nbar * NCT) break;
+            if (it >= kSpinLimit) {  // a CTA of the problem never arrived: give up, flag
+              bar_fail = 1;
+              atomicExch(ks.err, 1);
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
+        __threadfence();
+      }
+      __syncthreads();
+    } else {
+      __threadfence();
+      cluster.sync();
+    }
+  };
   unsigned short* tl = ks.tlist + p.slot0;           // rank r's list at r * tpc * kTile
 
   if (warp == 0) {
@@ -296,6 +334,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
   }
   if (tid == 0) {
+    bar_fail = 0;
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(saddr(&mbar[0])));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(saddr(&mbar[1])));
     asm volatile("fence.mbarrier_init.release.cluster;\n");
@@ -570,8 +609,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       if (last)
         for (int t = tid; t < ntok; t += kFT) ks.assign[p.slot0 + tok0 + t] = asg[t];
     }
-    __threadfence();
-    cluster.sync();
+    team_sync();
     // ---- owners: counts, offsets, means over all CTAs' members ----------------
     if (last) {
       for (int c = tid; c < C; c += kFT) {
@@ -727,8 +765,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         __syncwarp();  // the warp's tables are rewritten for its next cluster
       }
     }
-    __threadfence();
-    cluster.sync();
+    team_sync();
   }
   fence_before();
   __syncthreads();
@@ -741,36 +778,42 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
 template <int D>
 static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int iters,
                            cudaStream_t st) {
-  int cmax = 0;
+  int cmax = 0, ntp_max = 1;
   for (int k = 0; k < nsets; ++k) {
     if (gs[k].dtype != 0 || gs[k].C > kNCF || gs[k].D != D) return false;
     cmax = cmax > gs[k].C ? cmax : gs[k].C;
+    for (int l = 0; l < gs[k].lv.nlev; ++l) {
+      const int ntp = cdiv(gs[k].lv.s[l], kTile);
+      ntp_max = ntp_max > ntp ? ntp_max : ntp;
+    }
   }
   const int NC = (cmax + 31) & ~31;
   int tcols = 32;
   while (tcols < 2 * NC) tcols <<= 1;  // two accumulators (tiles in flight)
   const int nprob = kss[0].nprob + (nsets > 1 ? kss[1].nprob : 0);
-  // largest cluster size (up to 16, beyond the portable 8 where the GPU
-  // allows it) whose clusters are all resident at once
+  auto layout_for = [&](int nct, FusedLayout& Lc) {
+    const int tpc_max = cdiv(ntp_max, nct);
+    if (tpc_max * kTile > 65535) return false;
+    Lc = fused_layout(D, NC, tpc_max, true);
+    if (Lc.total > kSmemLimit) Lc = fused_layout(D, NC, tpc_max, false);
+    return Lc.total <= kSmemLimit;
+  };
+  // thread-block clusters: the largest size (up to 16, beyond the portable 8
+  // where the GPU allows it) whose clusters are all resident at once
   int NCT = 0;
   FusedLayout L{};
   const bool big_ok =
-      cudaFuncSetAttribute(kmeans_fused_kernel<D>,
+      cudaFuncSetAttribute(kmeans_fused_kernel<D, false>,
                            cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
   if (!big_ok) cudaGetLastError();
-  for (int nct = big_ok ? kMaxNCT : 8; nct >= 1; --nct) {
-    int tpc_max = 1;
-    for (int k = 0; k < nsets; ++k)
-      for (int l = 0; l < gs[k].lv.nlev; ++l) {
-        const int tpc = cdiv(cdiv(gs[k].lv.s[l], kTile), nct);
-        tpc_max = tpc_max > tpc ? tpc_max : tpc;
-      }
-    if (tpc_max * kTile > 65535) break;
-    FusedLayout Lc = fused_layout(D, NC, tpc_max, true);
-    if (Lc.total > kSmemLimit) Lc = fused_layout(D, NC, tpc_max, false);
-    if (Lc.total > kSmemLimit) continue;
-    cudaFuncSetAttribute(kmeans_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)Lc.total);
+  for (int nct = big_ok ? 16 : 8; nct >= 1; --nct) {
+    FusedLayout Lc;
+    if (!layout_for(nct, Lc)) {
+      if (cdiv(ntp_max, nct) * kTile > 65535) break;
+      continue;
+    }
+    cudaFuncSetAttribute(kmeans_fused_kernel<D, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lc.total);
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3((unsigned)(nprob * nct));
     q.blockDim = dim3(kFT);
@@ -783,7 +826,7 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
     q.attrs = qa;
     q.numAttrs = 1;
     int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, kmeans_fused_kernel<D>, &q) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&active, kmeans_fused_kernel<D, false>, &q) != cudaSuccess) {
       cudaGetLastError();
       active = 0;
     }
@@ -797,6 +840,32 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
       break;
     }
   }
+  // cooperative launch: when every problem can have more CTAs than a cluster
+  // gives it and all CTAs are resident at once
+  int dev = 0, nsm = 0, coop_ok = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&coop_ok, cudaDevAttrCooperativeLaunch, dev);
+  int nctc = nsm / nprob;
+  nctc = nctc < kMaxNCT ? nctc : kMaxNCT;
+  nctc = nctc < ntp_max ? nctc : ntp_max;
+  bool coop = false;
+  FusedLayout Lq;
+  if (coop_ok && nctc > NCT && layout_for(nctc, Lq)) {
+    cudaFuncSetAttribute(kmeans_fused_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)Lq.total);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kmeans_fused_kernel<D, true>, kFT,
+                                                      Lq.total) == cudaSuccess) {
+      coop = (long long)per_sm * nsm >= (long long)nprob * nctc;
+    } else {
+      cudaGetLastError();
+    }
+  }
+  if (coop) {
+    NCT = nctc;
+    L = Lq;
+  }
   if (NCT == 0) return false;
   FusedSets fs{};
   for (int k = 0; k < nsets; ++k) {
@@ -805,21 +874,32 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
   }
   fs.nblk0 = kss[0].nprob * NCT;
   const int nblk = fs.nblk0 + (nsets > 1 ? kss[1].nprob * NCT : 0);
-  cudaFuncSetAttribute(kmeans_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)L.total);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)nblk);
   cfg.blockDim = dim3(kFT);
   cfg.dynamicSmemBytes = L.total;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = NCT;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  if (coop) {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = NCT;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D>, fs, iters, NCT, NC, L.tpc, tcols, L.stage);
+  if (coop) {
+    cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, true>, fs, iters, NCT, NC, L.tpc, tcols,
+                       L.stage);
+  } else {
+    cudaFuncSetAttribute(kmeans_fused_kernel<D, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, false>, fs, iters, NCT, NC, L.tpc, tcols,
+                       L.stage);
+  }
   return true;
 }
 

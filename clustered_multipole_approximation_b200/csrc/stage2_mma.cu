@@ -27,6 +27,7 @@ namespace {
 constexpr int kMQ = 128;     // queries per pass (8 warps x 16 rows)
 constexpr int kMK = 64;      // key rows per block
 constexpr int kThreads = 256;
+constexpr int kXRows = 2048;  // exact rows resolved once per CTA
 
 __device__ inline int kvp(const AttnArgs& a, int qpid) {
   const int ppb = a.qg.lv.pairs_per_bh;
@@ -107,8 +108,11 @@ struct Smem2 {
   __nv_bfloat16 q[kMQ][D + 8];
   KBuf<D> buf[2];
   unsigned char inR[kMaxC];
+  float fb[kMaxC];      // far-field logit offset (base 2) per key cluster, -inf if not far
   int sel[kMaxC];
   int selstart[kMaxC];  // start of each retrieved cluster in the concatenated list
+  int selbase[kMaxC];   // its first position in the key problem's sorted order
+  int xrow[kXRows];     // the concatenated list's rows, when it has at most kXRows
 };
 
 }  // namespace
@@ -168,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
   __syncthreads();
   const int* kc = a.ks.counts + (size_t)kpid * Ck;
   const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
+  const int* kperm = a.ks.perm + pk.slot0;
   // the retrieved clusters' members, concatenated in selection order, are one
   // list of exact keys cut into blocks of 64 (a block may span two clusters)
   long long nexact = 0;
@@ -175,6 +180,34 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
     sm.selstart[r] = (int)nexact;
     nexact += kc[sm.sel[r]];
   }
+  // per-CTA tables: far-field offsets, the retrieved clusters' first sorted
+  // positions and, when it fits, the row of every exact key
+  for (int j = tid; j < pk.C; j += kThreads)
+    sm.fb[j] = (kc[j] > 0 && !sm.inR[j]) ? s1.fbias[((size_t)lq * Cq + i) * Ck + j] * 1.4426950408889634f
+                                       : -INFINITY;
+  for (int r = tid; r < nsel; r += kThreads) sm.selbase[r] = koff[sm.sel[r]];
+  __syncthreads();
+  const bool prerow = nexact <= kXRows;
+  if (prerow) {
+    constexpr int U = 2;
+    for (int q0 = tid; q0 < (int)nexact; q0 += U * kThreads) {
+      int v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int pos = q0 + u * kThreads;
+        v[u] = 0;
+        if (pos < (int)nexact) {
+          int rr = 0;
+          while (rr + 1 < nsel && sm.selstart[rr + 1] <= pos) ++rr;
+          v[u] = kperm[sm.selbase[rr] + pos - sm.selstart[rr]];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (q0 + u * kThreads < (int)nexact) sm.xrow[q0 + u * kThreads] = v[u];
+    }
+  }
+  __syncthreads();
   const int nblk_exact = cdiv((int)nexact, kMK);
   const int nblk_far = cdiv(pk.C, kMK);
   const int nblk = nblk_far + nblk_exact;
@@ -184,7 +217,6 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
   const __half* V16 = a.V16;
   const int qo = a.qs.off[(size_t)qpid * (Cq + 1) + i];
   const int* qperm = a.qs.perm + pq.slot0;
-  const int* kperm = a.ks.perm + pk.slot0;
   const size_t ij0 = ((size_t)lq * Cq + i) * Ck;
   const bool tilted = a.mode == 2;
   const float sl2 = a.scale * 1.4426950408889634f;  // logits in base-2 units
@@ -198,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
       const int j0 = b * kMK;
       for (int e = tid; e < kMK * CH; e += kThreads) {
         const int r = e / CH, c = (e % CH) * 8, j = j0 + r;
-        const bool live = j < pk.C && kc[j] > 0 && !sm.inR[j];
+        const bool live = j < pk.C && sm.fb[j] > -INFINITY;
         const size_t o = (size_t)(live ? j : 0) * D + c;
         cp16(&B.k[r][c], khi + o, live ? 16 : 0);
         cp16(&B.k2[r][c], klo + o, live ? 16 : 0);
@@ -206,8 +238,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
       }
       for (int r = tid; r < kMK; r += kThreads) {
         const int j = j0 + r;
-        const bool live = j < pk.C && kc[j] > 0 && !sm.inR[j];
-        B.bias[r] = live ? s1.fbias[ij0 + j] * 1.4426950408889634f : -INFINITY;
+        B.bias[r] = j < pk.C ? sm.fb[j] : -INFINITY;
       }
     } else {
       // rows p0 .. p0+63 of the concatenated member list
@@ -219,9 +250,13 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
         long long row = pk.row0;
         if (live) {
           const int pos = p0 + r;
-          int rr = 0;
-          while (rr + 1 < nsel && sm.selstart[rr + 1] <= pos) ++rr;
-          row += kperm[koff[sm.sel[rr]] + pos - sm.selstart[rr]];
+          if (prerow) {
+            row += sm.xrow[pos];
+          } else {
+            int rr = 0;
+            while (rr + 1 < nsel && sm.selstart[rr + 1] <= pos) ++rr;
+            row += kperm[sm.selbase[rr] + pos - sm.selstart[rr]];
+          }
         }
         cp16(&B.k[r][c], K + row * D + c, live ? 16 : 0);
         cp16(&B.v[r][c], V16 + row * D + c, live ? 16 : 0);
