@@ -47,11 +47,13 @@ __device__ inline uint32_t mod_u64_u32(uint64_t r, uint32_t m) {
   return (uint32_t)rem;
 }
 
-// Both roles' problems in one launch: CTAs [0, nblk0) serve set 0.
+// Both roles' problems in one launch: CTAs [0, nblk0) serve set 0.  Each
+// problem is split over `nsplit` CTAs, each writing a slice of the rows.
 struct InitSets {
   RoleGeo g[2];
   KState ks[2];
   int nblk0;
+  int nsplit;
 };
 
 template <typename T>
@@ -61,9 +63,12 @@ __global__ void __launch_bounds__(256) kmeans_init_kernel(InitSets is, const flo
   const int set = (int)blockIdx.x < is.nblk0 ? 0 : 1;
   const RoleGeo& g = is.g[set];
   const KState& ks = is.ks[set];
-  const int pid = (int)blockIdx.x - (set ? is.nblk0 : 0);
+  const int blk = (int)blockIdx.x - (set ? is.nblk0 : 0);
+  const int pid = blk / is.nsplit, part = blk - pid * is.nsplit;
   const Prob p = prob_of(g, pid);
   const int D = g.D, C = p.C;
+  const int rows = cdiv(C, is.nsplit);
+  const int cb = part * rows, ce = imin(C, cb + rows);  // this CTA's rows
   const T* X = static_cast<const T*>(g.X);
   double* c64 = ks.cent64 + (size_t)pid * g.C * D;
   float* c32 = ks.cent32 + (size_t)pid * g.C * D;
@@ -83,7 +88,7 @@ __global__ void __launch_bounds__(256) kmeans_init_kernel(InitSets is, const flo
       jd[c] = c + (int)mod_u64_u32(r, (uint32_t)(n - c));
     }
     __syncthreads();
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    for (int c = cb + (int)threadIdx.x; c < ce; c += blockDim.x) {
       int pos = jd[c], s = c;
       for (;;) {
         int f = s - 1;
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(256) kmeans_init_kernel(InitSets is, const flo
   const float* src = init ? init + (size_t)p.bh * g.C * D : nullptr;  // muse_cluster: one problem per bh
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   constexpr int RR = 4;
-  for (int c0 = warp * RR; c0 < C; c0 += nw * RR) {
+  for (int c0 = cb + warp * RR; c0 < ce; c0 += nw * RR) {
     float v[RR][4];
 #pragma unroll
     for (int u = 0; u < RR; ++u)
@@ -109,13 +114,13 @@ __global__ void __launch_bounds__(256) kmeans_init_kernel(InitSets is, const flo
       for (int r = 0; r < 4; ++r) {
         const int c = c0 + u, d = lane + 32 * r;
         v[u][r] = 0.f;
-        if (c < C && d < D)
+        if (c < ce && d < D)
           v[u][r] = src ? src[(size_t)c * D + d] : ld<T>(X + (p.row0 + pick[c]) * D + d);
       }
 #pragma unroll
     for (int u = 0; u < RR; ++u) {
       const int c = c0 + u;
-      if (c >= C) break;
+      if (c >= ce) break;
       float s = 0.f;
       double s2 = 0.0;
 #pragma unroll
@@ -367,8 +372,10 @@ static void init_t(const RoleGeo* gs, const KState* kss, int nsets, const float*
     is.g[k] = gs[k];
     is.ks[k] = kss[k];
   }
-  is.nblk0 = kss[0].nprob;
-  const int nblk = kss[0].nprob + (nsets > 1 ? kss[1].nprob : 0);
+  const int nprob = kss[0].nprob + (nsets > 1 ? kss[1].nprob : 0);
+  is.nsplit = nprob >= 148 ? 1 : 8;  // spread few problems over more SMs
+  is.nblk0 = kss[0].nprob * is.nsplit;
+  const int nblk = nprob * is.nsplit;
   kmeans_init_kernel<T><<<(unsigned)nblk, 256, 0, st>>>(is, init);
 }
 

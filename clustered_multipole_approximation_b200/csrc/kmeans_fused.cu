@@ -46,6 +46,7 @@ constexpr int kFT = 256;           // threads of the fused kernel
 constexpr int kWarps = kFT / 32;
 constexpr int kMaxNCT = 32;        // CTAs per problem
 constexpr int kSpinLimit = 1 << 24;  // team barrier polls (64 ns apart) before giving up
+constexpr int kOT = kNCF + kMaxNCT;  // (owned cluster, rank) pairs per CTA, at most
 constexpr size_t kSmemLimit = 218 * 1024;  // dynamic shared memory (static arrays come on top)
 
 __device__ inline uint32_t saddr(const void* p) {
@@ -274,6 +275,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   __shared__ int qcount;
   __shared__ int goff[kNCF + 1];
   __shared__ int own_n[kNCF], own_ord[kNCF];  // owned clusters: sizes, largest-first order
+  __shared__ int otab[2 * kOT];               // owned clusters x ranks: list start, count
   __shared__ int own_ctr;
   __shared__ int bar_fail;
 
@@ -612,13 +614,12 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     team_sync();
     // ---- owners: counts, offsets, means over all CTAs' members ----------------
     if (last) {
-      for (int c = tid; c < C; c += kFT) {
-        int tot = 0;
-        for (int r = 0; r < nra; ++r) {
-          const int* xr = xoff + (size_t)r * (g.C + 1);
-          tot += __ldcg(xr + c + 1) - __ldcg(xr + c);
-        }
-        goff[c] = tot;
+      for (int c = tid; c < C; c += kFT) goff[c] = 0;
+      __syncthreads();
+      for (int k = tid; k < C * nra; k += kFT) {  // (cluster, rank) pairs
+        const int c = k / nra, r = k - c * nra;
+        const int* xr = xoff + (size_t)r * (g.C + 1) + c;
+        atomicAdd(&goff[c], __ldcg(xr + 1) - __ldcg(xr));
       }
       __syncthreads();
       const int tot = block_scan_excl(goff, C, scan_tmp);
@@ -628,27 +629,31 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     // ---- owners: this CTA's clusters, largest first, one warp per cluster ----
     {
       const int nown = C > rank ? cdiv(C - rank, NCT) : 0;  // clusters rank + NCT i
+      // (owned cluster, rank) pairs, one thread each: list start and count
+      // (nown * nra < C + NCT <= kOT pairs)
+      for (int k = tid; k < nown * nra; k += kFT) {
+        const int i = k / nra, r = k - i * nra;
+        const int* xr = xoff + (size_t)r * (g.C + 1) + rank + NCT * i;
+        const int m0 = __ldcg(xr), m1 = __ldcg(xr + 1);
+        otab[2 * k] = m0;
+        otab[2 * k + 1] = m1 - m0;
+      }
+      if (tid == 0) own_ctr = 0;
+      __syncthreads();
       for (int i = tid; i < nown; i += kFT) {
-        const int c = rank + NCT * i;
         int n = 0;
-        for (int r = 0; r < nra; ++r) {
-          const int* xr = xoff + (size_t)r * (g.C + 1);
-          n += __ldcg(xr + c + 1) - __ldcg(xr + c);
-        }
+        for (int r = 0; r < nra; ++r) n += otab[2 * (i * nra + r) + 1];
         own_n[i] = n;
       }
       __syncthreads();
-      if (tid == 0) {  // sizes descending, so the largest clusters start first
-        own_ctr = 0;
-        for (int i = 0; i < nown; ++i) {
-          const int nv = own_n[i];
-          int j = i - 1;
-          while (j >= 0 && own_n[own_ord[j]] < nv) {
-            own_ord[j + 1] = own_ord[j];
-            --j;
-          }
-          own_ord[j + 1] = i;
+      for (int i = tid; i < nown; i += kFT) {  // sizes descending: largest clusters first
+        const int ni = own_n[i];
+        int rk = 0;
+        for (int k = 0; k < nown; ++k) {
+          const int nk = own_n[k];
+          rk += (nk > ni || (nk == ni && k < i)) ? 1 : 0;
         }
+        own_ord[rk] = i;
       }
       __syncthreads();
       int* gP = gtab + warp * (2 * kMaxNCT + 1);  // [0, nra]: members before rank r
@@ -659,13 +664,13 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         if (lane == 0) k = atomicAdd(&own_ctr, 1);
         k = __shfl_sync(0xffffffffu, k, 0);
         if (k >= nown) break;
-        const int c = rank + NCT * own_ord[k];
-        const int n = own_n[own_ord[k]];
+        const int io = own_ord[k];
+        const int c = rank + NCT * io;
+        const int n = own_n[io];
         int cnt = 0, m0 = 0;
         if (lane < nra) {
-          const int* xr = xoff + (size_t)lane * (g.C + 1);
-          m0 = __ldcg(xr + c);
-          cnt = __ldcg(xr + c + 1) - m0;
+          m0 = otab[2 * (io * nra + lane)];
+          cnt = otab[2 * (io * nra + lane) + 1];
         }
         int incl = cnt;
         for (int o = 1; o < 32; o <<= 1) {
@@ -690,32 +695,36 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         double acc[VPL];
 #pragma unroll
         for (int e = 0; e < VPL; ++e) acc[e] = 0.0;
-        // two batches in flight: rows of batch b+1 load while batch b is summed
-        int ec = entry(lane);
-        RowT vc[kOB];
-#pragma unroll
-        for (int q = 0; q < kOB; ++q) {
-          const int t = __shfl_sync(0xffffffffu, ec, q);
-          vc[q] = q < n ? __ldg(Xl + (size_t)t * (D / VPL)) : RowT{};
-        }
-        if (last && lane < kOB && lane < n) ks.perm[pbase + lane] = ec;
-        int en = entry(kOB + lane);
-        for (int j0 = 0; j0 < n; j0 += kOB) {
-          const bool more = j0 + kOB < n;
-          RowT vn[kOB];
+        // three batches in flight: rows of batches b+1 and b+2 load while
+        // batch b is summed
+        auto rows = [&](int e, int jb, RowT (&v)[kOB]) {
 #pragma unroll
           for (int q = 0; q < kOB; ++q) {
-            const int t = __shfl_sync(0xffffffffu, en, q);
-            vn[q] = more && j0 + kOB + q < n ? __ldg(Xl + (size_t)t * (D / VPL)) : RowT{};
+            const int t = __shfl_sync(0xffffffffu, e, q);
+            v[q] = jb + q < n ? __ldg(Xl + (size_t)t * (D / VPL)) : RowT{};
           }
-          if (last && more && lane < kOB && j0 + kOB + lane < n) ks.perm[pbase + j0 + kOB + lane] = en;
-          const int en2 = more ? entry(j0 + 2 * kOB + lane) : 0;
+        };
+        RowT va[kOB], vb[kOB], vc[kOB];
+        int ea = entry(lane);
+        rows(ea, 0, va);
+        int eb = entry(kOB + lane);
+        rows(eb, kOB, vb);
+        int ec = entry(2 * kOB + lane);
+        for (int j0 = 0; j0 < n; j0 += kOB) {
+          rows(ec, j0 + 2 * kOB, vc);
+          const int ed = j0 + 3 * kOB < n ? entry(j0 + 3 * kOB + lane) : 0;
+          if (last && lane < kOB && j0 + lane < n) ks.perm[pbase + j0 + lane] = ea;
 #pragma unroll
           for (int q = 0; q < kOB; ++q)
-            if (j0 + q < n) add_row(acc, vc[q]);
+            if (j0 + q < n) add_row(acc, va[q]);
 #pragma unroll
-          for (int q = 0; q < kOB; ++q) vc[q] = vn[q];
-          en = en2;
+          for (int q = 0; q < kOB; ++q) {
+            va[q] = vb[q];
+            vb[q] = vc[q];
+          }
+          ea = eb;
+          eb = ec;
+          ec = ed;
         }
         if (last && lane == 0) {
           ks.counts[cbase + c] = n;

@@ -300,9 +300,22 @@ __global__ void __launch_bounds__(256) select_kernel(AttnArgs a, Stage1 s1, int 
   double* mus = sel_smem;                                            // [ck][D + 1]
   double* sc = sel_smem + (STAGED ? (size_t)Ck * (D + 1) : 0) + (size_t)warp * Ck;
   if (STAGED) {
-    for (int e = threadIdx.x; e < ck * D; e += blockDim.x) {
-      const int j = e / D, d = e - j * D;
-      mus[j * (D + 1) + d] = mug[e];
+    const int tot = ck * D;
+    for (int e0 = threadIdx.x; e0 < tot; e0 += 8 * blockDim.x) {  // 8 loads in flight
+      double v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = e0 + u * blockDim.x;
+        v[u] = e < tot ? mug[e] : 0.0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = e0 + u * blockDim.x;
+        if (e < tot) {
+          const int j = e / D, d = e - j * D;
+          mus[j * (D + 1) + d] = v[u];
+        }
+      }
     }
     __syncthreads();
   }
@@ -637,7 +650,7 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
   {
     ProfScope ps(st, "stage1_summaries");
     if (sizeof(T) == 2 && a.mode == 1)
-      run_stage1_dipole_mma(a, s1, qp0, nqp, st);
+      run_stage1_dipole_tc(a, s1, qp0, nqp, st);
     else
       stage1_kernel<T, D><<<dim3(nqp, a.Ck), kS1T, stage1_smem<D>(), st>>>(a, s1, qp0);
   }
