@@ -74,8 +74,6 @@ void run_bf16_to_half(const void* src, __half* dst, size_t n, cudaStream_t st);
 void run_stage2_mma(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 // Stage 1 (DIPOLE) on tcgen05 tensor cores (bf16 inputs).
 void run_stage1_dipole_tc(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
-// Stage 2 on tcgen05 tensor cores (bf16 inputs).
-void run_stage2_tc(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 
 // Causal: exact local block + merge of the level partials into O.
 void run_local_merge(const AttnArgs& a, int L, cudaStream_t st);

@@ -271,8 +271,8 @@ __global__ void __launch_bounds__(kS1T) stage1_kernel(AttnArgs a, Stage1 s1, int
 // selection: top-k key clusters per query cluster by s nu_i.mu_j + log W_ij,
 // ties to the lowest j, empty clusters never
 // ----------------------------------------------------------------------------
-// Query clusters handled by one CTA of the selection kernel (two per warp).
-constexpr int kSelQ = 16;
+// Query clusters handled by one CTA of the selection kernel (one per warp).
+constexpr int kSelQ = 8;
 
 // Key centroids per CTA staged in shared memory when they fit (row stride
 // D + 1 doubles keeps the lanes' rows on distinct banks).
