@@ -118,6 +118,14 @@ class Clocks:
 # ---------------------------------------------------------------------------
 # algorithmic work per kernel launch (what the method must compute)
 # ---------------------------------------------------------------------------
+# DRAM bytes (read + write) of one launch of a kernel on a workload, from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum, caches flushed as in the
+# timed region).  An entry is removed whenever its kernel changes.
+NCU_TRAFFIC = {
+    ("acausal-bf16-h8-n8k", "kmeans_fused"): 18_463_488 + 3_584,
+}
+
+
 def algorithmic_work(w, mode, dbg):
     """Per-launch algorithmic FLOPs and bytes of the acausal kernels, from the
     shapes and the actual retrieval counts.  A multiply-add counts 2 FLOPs."""
@@ -284,7 +292,8 @@ def run_muse(args, w, rank, world, device):
     dom_launches, dom_ms = prof[dom]
     avg_ms = dom_ms / dom_launches
     roofline = {"kernel": dom, "bound": "tensor", "achieved": None,
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": None, "traffic": None,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": None,
+                "traffic": NCU_TRAFFIC.get((w.name, dom)),
                 "peak_source": f"{how} bf16 dense (burst)", "avg_launch_ms": avg_ms}
     if not w.causal:
         work = algorithmic_work(w, mode, {n: t.cpu().numpy() for n, t in dbg.items()})
