@@ -202,11 +202,14 @@ __device__ inline int exact_argmin(const double* x, const double* cst, const dou
 }  // namespace
 
 // Up to two independent problem sets (the key and the query clusterings)
-// share one launch: CTAs [0, nblk0) serve set 0, the rest set 1.
+// share one launch: CTAs [0, nblk0) serve set 0, the rest set 1.  lvl >= 0
+// restricts a launch to the problems of one causal level (all (b, head) pairs
+// of that level), so each level gets its own CTAs per problem.
 struct FusedSets {
   RoleGeo g[2];
   KState ks[2];
   int nblk0;
+  int lvl;
 };
 
 // Exclusive scan of n <= 2 * blockDim.x ints in shared memory, called by
@@ -280,7 +283,11 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   __shared__ int bar_fail;
 
   const int rank = COOP ? (int)blockIdx.x % NCT : (int)cluster.block_rank();
-  const int pid = blk / NCT;
+  int pid = blk / NCT;
+  if (fs.lvl >= 0) {  // j-th problem of the level -> problem id
+    const int np = g.lv.npairs[fs.lvl];
+    pid = (pid / np) * g.lv.pairs_per_bh + g.lv.pair_base[fs.lvl] + pid % np;
+  }
   const Prob p = prob_of(g, pid);
   const int C = p.C;
   const int ntp = cdiv(p.s, kTile);
@@ -782,24 +789,26 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tbase), "r"(tcols));
 }
 
-// Returns false (nothing launched) when the fused path does not cover these
-// problem sets: more than 256 clusters, or more than 65535 tokens per CTA.
+// CTAs per problem and launch form for the problems of one level (lvl >= 0)
+// or of all levels (lvl < 0, the acausal single level).
+struct FusedPlan {
+  bool coop;
+  int NCT;
+  FusedLayout L;
+};
+
 template <int D>
-static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int iters,
-                           cudaStream_t st) {
-  int cmax = 0, ntp_max = 1;
+static bool plan_fused(const RoleGeo* gs, const KState* kss, int nsets, int lvl, int NC,
+                       FusedPlan& plan) {
+  int ntp_max = 1, nprob = 0;
   for (int k = 0; k < nsets; ++k) {
-    if (gs[k].dtype != 0 || gs[k].C > kNCF || gs[k].D != D) return false;
-    cmax = cmax > gs[k].C ? cmax : gs[k].C;
-    for (int l = 0; l < gs[k].lv.nlev; ++l) {
+    const int l0 = lvl < 0 ? 0 : lvl, l1 = lvl < 0 ? gs[k].lv.nlev : lvl + 1;
+    for (int l = l0; l < l1; ++l) {
       const int ntp = cdiv(gs[k].lv.s[l], kTile);
       ntp_max = ntp_max > ntp ? ntp_max : ntp;
     }
+    nprob += lvl < 0 ? kss[k].nprob : gs[k].BH * gs[k].lv.npairs[lvl];
   }
-  const int NC = (cmax + 31) & ~31;
-  int tcols = 32;
-  while (tcols < 2 * NC) tcols <<= 1;  // two accumulators (tiles in flight)
-  const int nprob = kss[0].nprob + (nsets > 1 ? kss[1].nprob : 0);
   auto layout_for = [&](int nct, FusedLayout& Lc) {
     const int tpc_max = cdiv(ntp_max, nct);
     if (tpc_max * kTile > 65535) return false;
@@ -807,18 +816,46 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
     if (Lc.total > kSmemLimit) Lc = fused_layout(D, NC, tpc_max, false);
     return Lc.total <= kSmemLimit;
   };
-  // thread-block clusters: the largest size (up to 16, beyond the portable 8
-  // where the GPU allows it) whose clusters are all resident at once
-  int NCT = 0;
-  FusedLayout L{};
+  int dev = 0, nsm = 0, coop_ok = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&coop_ok, cudaDevAttrCooperativeLaunch, dev);
+  // cooperative launch: every problem's CTAs resident at once, as many per
+  // problem as the GPU allows (at most one per tile)
+  int nctc = nsm / (nprob > 0 ? nprob : 1);
+  nctc = nctc < kMaxNCT ? nctc : kMaxNCT;
+  nctc = nctc < ntp_max ? nctc : ntp_max;
+  if (coop_ok && nctc >= 2 && layout_for(nctc, plan.L)) {
+    cudaFuncSetAttribute(kmeans_fused_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)plan.L.total);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kmeans_fused_kernel<D, true>, kFT,
+                                                      plan.L.total) == cudaSuccess &&
+        (long long)per_sm * nsm >= (long long)nprob * nctc) {
+      plan.coop = true;
+      plan.NCT = nctc;
+      return true;
+    }
+    cudaGetLastError();
+  }
+  // thread-block clusters, in waves when the problems do not all fit: about
+  // eight tiles per CTA (the per-round fixed costs stay small against the
+  // tiles), at least enough CTAs to fill the GPU, at most one per tile
   const bool big_ok =
       cudaFuncSetAttribute(kmeans_fused_kernel<D, false>,
                            cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
   if (!big_ok) cudaGetLastError();
-  for (int nct = big_ok ? 16 : 8; nct >= 1; --nct) {
+  const int cmax = big_ok ? 16 : 8;
+  int nct = cdiv(ntp_max, 8);
+  const int fill = nsm / (nprob > 0 ? nprob : 1);
+  nct = nct > fill ? nct : fill;
+  nct = nct < ntp_max ? nct : ntp_max;
+  nct = nct < cmax ? nct : cmax;
+  nct = nct > 1 ? nct : 1;
+  for (; nct >= 1; --nct) {
     FusedLayout Lc;
     if (!layout_for(nct, Lc)) {
-      if (cdiv(ntp_max, nct) * kTile > 65535) break;
+      if (cdiv(ntp_max, nct) * kTile > 65535) return false;
       continue;
     }
     cudaFuncSetAttribute(kmeans_fused_kernel<D, false>,
@@ -839,76 +876,85 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
       cudaGetLastError();
       active = 0;
     }
-    if (nct <= 8 && NCT == 0) {  // fallback: the largest portable size that fits at all
-      NCT = nct;
-      L = Lc;
-    }
-    if (active >= nprob) {
-      NCT = nct;
-      L = Lc;
-      break;
+    if (active >= 1) {
+      plan.coop = false;
+      plan.NCT = nct;
+      plan.L = Lc;
+      return true;
     }
   }
-  // cooperative launch: when every problem can have more CTAs than a cluster
-  // gives it and all CTAs are resident at once
-  int dev = 0, nsm = 0, coop_ok = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  cudaDeviceGetAttribute(&coop_ok, cudaDevAttrCooperativeLaunch, dev);
-  int nctc = nsm / nprob;
-  nctc = nctc < kMaxNCT ? nctc : kMaxNCT;
-  nctc = nctc < ntp_max ? nctc : ntp_max;
-  bool coop = false;
-  FusedLayout Lq;
-  if (coop_ok && nctc > NCT && layout_for(nctc, Lq)) {
-    cudaFuncSetAttribute(kmeans_fused_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)Lq.total);
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kmeans_fused_kernel<D, true>, kFT,
-                                                      Lq.total) == cudaSuccess) {
-      coop = (long long)per_sm * nsm >= (long long)nprob * nctc;
-    } else {
-      cudaGetLastError();
-    }
-  }
-  if (coop) {
-    NCT = nctc;
-    L = Lq;
-  }
-  if (NCT == 0) return false;
+  return false;
+}
+
+template <int D>
+static void launch_plan(const RoleGeo* gs, const KState* kss, int nsets, int lvl, int iters,
+                        int NC, int tcols, const FusedPlan& plan, cudaStream_t st) {
   FusedSets fs{};
+  int np[2] = {0, 0};
   for (int k = 0; k < nsets; ++k) {
     fs.g[k] = gs[k];
     fs.ks[k] = kss[k];
+    np[k] = lvl < 0 ? kss[k].nprob : gs[k].BH * gs[k].lv.npairs[lvl];
   }
-  fs.nblk0 = kss[0].nprob * NCT;
-  const int nblk = fs.nblk0 + (nsets > 1 ? kss[1].nprob * NCT : 0);
+  fs.lvl = lvl;
+  fs.nblk0 = np[0] * plan.NCT;
+  const int nblk = (np[0] + np[1]) * plan.NCT;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)nblk);
   cfg.blockDim = dim3(kFT);
-  cfg.dynamicSmemBytes = L.total;
+  cfg.dynamicSmemBytes = plan.L.total;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  if (coop) {
+  if (plan.coop) {
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
   } else {
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = NCT;
+    attr[0].val.clusterDim.x = plan.NCT;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
   }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (coop) {
-    cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, true>, fs, iters, NCT, NC, L.tpc, tcols,
-                       L.stage);
+  if (plan.coop) {
+    cudaFuncSetAttribute(kmeans_fused_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)plan.L.total);
+    cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, true>, fs, iters, plan.NCT, NC, plan.L.tpc,
+                       tcols, plan.L.stage);
   } else {
     cudaFuncSetAttribute(kmeans_fused_kernel<D, false>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
-    cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, false>, fs, iters, NCT, NC, L.tpc, tcols,
-                       L.stage);
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.L.total);
+    cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, false>, fs, iters, plan.NCT, NC, plan.L.tpc,
+                       tcols, plan.L.stage);
   }
+}
+
+// Returns false (nothing launched) when the fused path does not cover these
+// problem sets: more than 256 clusters, or no layout fits in shared memory.
+// A causal problem set (several levels) gets one launch per level, each with
+// its own CTAs per problem.
+template <int D>
+static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int iters,
+                           cudaStream_t st) {
+  int cmax = 0;
+  for (int k = 0; k < nsets; ++k) {
+    if (gs[k].dtype != 0 || gs[k].C > kNCF || gs[k].D != D) return false;
+    if (k > 0 && gs[k].lv.nlev != gs[0].lv.nlev) return false;
+    cmax = cmax > gs[k].C ? cmax : gs[k].C;
+  }
+  const int NC = (cmax + 31) & ~31;
+  int tcols = 32;
+  while (tcols < 2 * NC) tcols <<= 1;  // two accumulators (tiles in flight)
+  const int nlev = gs[0].lv.nlev;
+  FusedPlan plans[kMaxLevels];
+  if (nlev == 1) {
+    if (!plan_fused<D>(gs, kss, nsets, -1, NC, plans[0])) return false;
+    launch_plan<D>(gs, kss, nsets, -1, iters, NC, tcols, plans[0], st);
+    return true;
+  }
+  for (int l = 0; l < nlev; ++l)
+    if (!plan_fused<D>(gs, kss, nsets, l, NC, plans[l])) return false;
+  for (int l = 0; l < nlev; ++l) launch_plan<D>(gs, kss, nsets, l, iters, NC, tcols, plans[l], st);
   return true;
 }
 
