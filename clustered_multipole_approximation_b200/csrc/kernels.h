@@ -77,6 +77,8 @@ void run_stage1_dipole_tc(const AttnArgs& a, const Stage1& s1, int qp0, int nqp,
 
 // Causal: exact local block + merge of the level partials into O.
 void run_local_merge(const AttnArgs& a, int L, cudaStream_t st);
+// The same on mma.sync tiles (bf16, L a multiple of 128); false if not covered.
+bool run_local_mma(const AttnArgs& a, int L, cudaStream_t st);
 
 // Summaries (n, mu, S, M) of given assignments; used by muse_summarize.
 void run_summarize(const void* K, const void* V, int dtype, int BH, int N, int D, int C,

@@ -687,10 +687,11 @@ void run_blocks(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStrea
 }
 
 void run_local_merge(const AttnArgs& a, int L, cudaStream_t st) {
+  ProfScope ps(st, "causal_local_merge");
+  if (run_local_mma(a, L, st)) return;  // bf16, L a multiple of 128: tensor-core tiles
   const int D = a.qg.D, N = a.qg.lv.N;
   dim3 grid(a.qg.BH, cdiv(N, kQ));
   const int thr = kQ * (D / 64);
-  ProfScope ps(st, "causal_local_merge");
   using bf = __nv_bfloat16;
   if (a.qg.dtype == 0) {
     if (a.out_f32) {

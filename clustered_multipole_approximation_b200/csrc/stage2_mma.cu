@@ -419,6 +419,229 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
   }
 }
 
+// Causal exact local block + merge of the level partials, on mma.sync tiles
+// (bf16 inputs; gist.science page "Multipole Semantic Attention: A Fast
+// Approximation of Softmax Attention for Pretraining", Technical Summary,
+// hierarchical causal decomposition: exact attention inside each local
+// block, approximated levels beyond it).  One CTA of 8 warps per 128
+// consecutive queries of one (b, q-head); the local block length L is a
+// multiple of 128, so the tile lies inside one block and its keys are the
+// contiguous run [block start, last query], streamed in 64-row blocks with
+// cp.async, two in flight.  S = Q K^T in bf16 with fp32 accumulation, the
+// causal mask on the diagonal blocks, one online softmax in base 2, P and V in
+// fp16; then every level partial of the row (normalised output, log-sum-exp)
+// enters the same softmax as one term.
+template <int D>
+struct LocSmem {
+  __nv_bfloat16 q[kMQ][D + 8];
+  __nv_bfloat16 k[2][kMK][D + 8];
+  __half v[2][kMK][D + 8];
+};
+
+template <typename TO, int D>
+__global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) local_mma_kernel(AttnArgs a, int L) {
+  extern __shared__ __align__(16) unsigned char loc_raw[];
+  LocSmem<D>& sm = *reinterpret_cast<LocSmem<D>*>(loc_raw);
+  constexpr int KD = D / 16, ND = D / 8, CH = D / 8;
+  const int bhq = blockIdx.x, N = a.qg.lv.N;
+  const int q0 = blockIdx.y * kMQ;
+  const int nq = imin(kMQ, N - q0);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+  const bool wact = warp * 16 < nq;
+  const int Hq = a.qg.BH / a.B, Hkv = a.kg.BH / a.B;
+  const int bhk = (bhq / Hq) * Hkv + (bhq % Hq) / a.G;
+  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.qg.X) + (size_t)bhq * N * D;
+  const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.kg.X) + (size_t)bhk * N * D;
+  const __half* V16 = a.V16 + (size_t)bhk * N * D;
+  const int blk = q0 / L, kbeg = blk * L, kend = q0 + nq;  // keys [kbeg, kend)
+  const int nkb = cdiv(kend - kbeg, kMK);
+  const float sl2 = a.scale * 1.4426950408889634f;
+  auto issue = [&](int b) {
+    const int t0 = kbeg + b * kMK, nr = imin(kMK, kend - t0), st = b & 1;
+    for (int e = tid; e < kMK * CH; e += kThreads) {
+      const int r = e / CH, c = (e % CH) * 8;
+      const bool live = r < nr;
+      const size_t o = (size_t)(live ? t0 + r : 0) * D + c;
+      cp16(&sm.k[st][r][c], K + o, live ? 16 : 0);
+      cp16(&sm.v[st][r][c], V16 + o, live ? 16 : 0);
+    }
+    cp_commit();
+  };
+  for (int e = tid; e < kMQ * CH; e += kThreads) {
+    const int r = e / CH, c = (e % CH) * 8;
+    const bool live = r < nq;
+    cp16(&sm.q[r][c], Q + (size_t)(live ? q0 + r : 0) * D + c, live ? 16 : 0);
+  }
+  issue(0);  // commits the query rows with block 0
+  uint32_t qa[KD][4];
+  float o[ND][4];
+#pragma unroll
+  for (int n = 0; n < ND; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float mrow[2] = {kMaxFloor, kMaxFloor}, lrow[2] = {0.f, 0.f};
+  const int qpos[2] = {q0 + warp * 16 + g, q0 + warp * 16 + g + 8};
+
+  for (int b = 0; b < nkb; ++b) {
+    if (b + 1 < nkb) {
+      issue(b + 1);
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
+    }
+    __syncthreads();
+    if (b == 0 && wact) {
+#pragma unroll
+      for (int kk = 0; kk < KD; ++kk) {
+        const int row = warp * 16 + (lane & 15), col = kk * 16 + (lane >> 4) * 8;
+        ldsm_x4(smem_u32(&sm.q[row][col]), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+      }
+    }
+    const int st = b & 1, t0 = kbeg + b * kMK;
+    // blocks wholly after this warp's last row contribute nothing
+    if (wact && t0 <= q0 + warp * 16 + 15) {
+      float sc[kMK / 8][4];
+#pragma unroll
+      for (int n = 0; n < kMK / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KD; ++kk) {
+#pragma unroll
+        for (int np = 0; np < kMK / 16; ++np) {
+          const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int col = kk * 16 + ((lane >> 3) & 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(smem_u32(&sm.k[st][key][col]), b0, b1, b2, b3);
+          mma_bf16(sc[2 * np], qa[kk], b0, b1);
+          mma_bf16(sc[2 * np + 1], qa[kk], b2, b3);
+        }
+      }
+      float mx[2] = {kMaxFloor, kMaxFloor};
+#pragma unroll
+      for (int n = 0; n < kMK / 8; ++n) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const int t = t0 + n * 8 + 2 * t4 + (h & 1);
+          const float lg = (t < kend && t <= qpos[h >> 1]) ? sl2 * sc[n][h] : -INFINITY;
+          sc[n][h] = lg;
+          mx[h >> 1] = fmaxf(mx[h >> 1], lg);
+        }
+      }
+      float scale[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+        const float mn = fmaxf(mrow[r], mx[r]);
+        scale[r] = fast_exp2(mrow[r] - mn);
+        mrow[r] = mn;
+      }
+      float rs[2] = {0.f, 0.f};
+#pragma unroll
+      for (int n = 0; n < kMK / 8; ++n) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float pv = fast_exp2(sc[n][h] - mrow[h >> 1]);
+          sc[n][h] = pv;
+          rs[h >> 1] += pv;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
+        rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
+        lrow[r] = lrow[r] * scale[r] + rs[r];
+      }
+#pragma unroll
+      for (int n = 0; n < ND; ++n) {
+        o[n][0] *= scale[0];
+        o[n][1] *= scale[0];
+        o[n][2] *= scale[1];
+        o[n][3] *= scale[1];
+      }
+#pragma unroll
+      for (int kk = 0; kk < kMK / 16; ++kk) {
+        uint32_t pa[4];
+        pa[0] = pack_h2(sc[2 * kk][0], sc[2 * kk][1]);
+        pa[1] = pack_h2(sc[2 * kk][2], sc[2 * kk][3]);
+        pa[2] = pack_h2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+        pa[3] = pack_h2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+#pragma unroll
+        for (int np = 0; np < ND / 2; ++np) {
+          const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int col = np * 16 + (lane >> 4) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(smem_u32(&sm.v[st][key][col]), b0, b1, b2, b3);
+          mma_f16(o[2 * np], pa, b0, b1);
+          mma_f16(o[2 * np + 1], pa, b2, b3);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (!wact) return;
+  // ---- the level partials of each row, one softmax term each -----------------
+  const int levels = a.qg.lv.nlev;
+  const float* part = a.part;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int qp = qpos[r];
+    if (qp >= kend) continue;
+    for (int lv = 0; lv < levels; ++lv) {
+      if (!((blk >> lv) & 1)) continue;
+      const int sz = L << lv, pp_ = blk >> (lv + 1);
+      const long long slot = (long long)bhq * a.qg.lv.toks_per_bh + a.qg.lv.tok_base[lv] +
+                             (long long)pp_ * sz + (qp - (2 * pp_ + 1) * sz);
+      const float* pp = part + slot * (D + 1);
+      const float lg = pp[D] * 1.4426950408889634f;  // natural log -> base 2
+      const float mn = fmaxf(mrow[r], lg);
+      const float sc = fast_exp2(mrow[r] - mn), wt = fast_exp2(lg - mn);
+      lrow[r] = lrow[r] * sc + wt;
+#pragma unroll
+      for (int n = 0; n < ND; ++n) {
+        const int c = n * 8 + 2 * t4;
+        o[n][2 * r] = fmaf(o[n][2 * r], sc, wt * pp[c]);
+        o[n][2 * r + 1] = fmaf(o[n][2 * r + 1], sc, wt * pp[c + 1]);
+      }
+      mrow[r] = mn;
+    }
+    TO* O = static_cast<TO*>(a.O) + ((size_t)bhq * N + qp) * D;
+    const float inv = 1.f / lrow[r];
+#pragma unroll
+    for (int n = 0; n < ND; ++n) {
+      st<TO>(O + n * 8 + 2 * t4, o[n][2 * r] * inv);
+      st<TO>(O + n * 8 + 2 * t4 + 1, o[n][2 * r + 1] * inv);
+    }
+    if (a.n_exact != nullptr && t4 == 0)
+      atomicAdd(reinterpret_cast<unsigned long long*>(a.n_exact + (size_t)bhq * N + qp),
+                (unsigned long long)(qp - kbeg + 1));
+  }
+}
+
+template <int D>
+static void launch_local(const AttnArgs& a, int L, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(local_mma_kernel<float, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)sizeof(LocSmem<D>));
+    cudaFuncSetAttribute(local_mma_kernel<__nv_bfloat16, D>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(LocSmem<D>));
+    attr = true;
+  }
+  dim3 grid(a.qg.BH, cdiv(a.qg.lv.N, kMQ));
+  if (a.out_f32)
+    local_mma_kernel<float, D><<<grid, kThreads, sizeof(LocSmem<D>), st>>>(a, L);
+  else
+    local_mma_kernel<__nv_bfloat16, D><<<grid, kThreads, sizeof(LocSmem<D>), st>>>(a, L);
+}
+
+bool run_local_mma(const AttnArgs& a, int L, cudaStream_t st) {
+  if (a.qg.dtype != 0 || L % kMQ != 0 || a.V16 == nullptr) return false;
+  if (a.qg.D == 64)
+    launch_local<64>(a, L, st);
+  else
+    launch_local<128>(a, L, st);
+  return true;
+}
+
 template <int D>
 static void launch_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st) {
   static bool attr = false;
