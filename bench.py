@@ -122,7 +122,7 @@ class Clocks:
 # capture (dram__bytes_read.sum + dram__bytes_write.sum, caches flushed as in the
 # timed region).  An entry is removed whenever its kernel changes.
 NCU_TRAFFIC = {
-    ("acausal-bf16-h8-n8k", "kmeans_fused"): 18_463_488 + 3_584,
+    ("acausal-bf16-h8-n8k", "kmeans_fused"): 18_488_064 + 3_584,
 }
 
 
