@@ -300,11 +300,14 @@ def run_muse(args, w, rank, world, device):
         if dom in work:
             ach = work[dom]["flops"] / (avg_ms / 1e3) / 1e12
             roofline.update(achieved=ach, frac=ach / pk["bf16_tflops"],
+                            frac_of_sustained_peak=ach / pk["bf16_tflops_sustained"],
                             flops_per_launch=work[dom]["flops"])
         f_alg = total_algorithmic_flops(work, w.iters)
         whole = {"algorithmic_tflop": f_alg / 1e12,
                  "achieved_tflops": f_alg / (ms_per_step / 1e3) / 1e12,
-                 "frac_of_bf16_peak": f_alg / (ms_per_step / 1e3) / 1e12 / pk["bf16_tflops"]}
+                 "frac_of_bf16_peak": f_alg / (ms_per_step / 1e3) / 1e12 / pk["bf16_tflops"],
+                 "frac_of_bf16_sustained_peak":
+                     f_alg / (ms_per_step / 1e3) / 1e12 / pk["bf16_tflops_sustained"]}
     else:
         whole = None
     kernels = {n: {"launches": c, "ms_total": round(t, 4), "share": round(t / sum(x[1] for x in prof.values()), 4)}
