@@ -47,6 +47,7 @@ constexpr int kWarps = kFT / 32;
 constexpr int kMaxNCT = 32;        // CTAs per problem
 constexpr int kSpinLimit = 1 << 24;  // team barrier polls (64 ns apart) before giving up
 constexpr int kOT = kNCF + kMaxNCT;  // (owned cluster, rank) pairs per CTA, at most
+constexpr int kTilesPerCta = 16;     // cluster launches: target tiles per CTA
 constexpr size_t kSmemLimit = 218 * 1024;  // dynamic shared memory (static arrays come on top)
 
 __device__ inline uint32_t saddr(const void* p) {
@@ -839,25 +840,24 @@ static bool plan_fused(const RoleGeo* gs, const KState* kss, int nsets, int lvl,
     cudaGetLastError();
   }
   // thread-block clusters, in waves when the problems do not all fit: about
-  // eight tiles per CTA (the per-round fixed costs stay small against the
-  // tiles), at least enough CTAs to fill the GPU, at most one per tile
+  // sixteen tiles per CTA (the per-round fixed costs -- set-up, drain, sort,
+  // owner sums, barriers -- stay small against the tiles), at least enough
+  // CTAs to fill the GPU, at most one per tile; when that layout does not fit
+  // in shared memory, more CTAs (fewer tiles each), else fewer
   const bool big_ok =
       cudaFuncSetAttribute(kmeans_fused_kernel<D, false>,
                            cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
   if (!big_ok) cudaGetLastError();
   const int cmax = big_ok ? 16 : 8;
-  int nct = cdiv(ntp_max, 8);
+  int nct0 = cdiv(ntp_max, kTilesPerCta);
   const int fill = nsm / (nprob > 0 ? nprob : 1);
-  nct = nct > fill ? nct : fill;
-  nct = nct < ntp_max ? nct : ntp_max;
-  nct = nct < cmax ? nct : cmax;
-  nct = nct > 1 ? nct : 1;
-  for (; nct >= 1; --nct) {
+  nct0 = nct0 > fill ? nct0 : fill;
+  nct0 = nct0 < ntp_max ? nct0 : ntp_max;
+  nct0 = nct0 < cmax ? nct0 : cmax;
+  nct0 = nct0 > 1 ? nct0 : 1;
+  auto try_nct = [&](int nct) {
     FusedLayout Lc;
-    if (!layout_for(nct, Lc)) {
-      if (cdiv(ntp_max, nct) * kTile > 65535) return false;
-      continue;
-    }
+    if (!layout_for(nct, Lc)) return false;
     cudaFuncSetAttribute(kmeans_fused_kernel<D, false>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lc.total);
     cudaLaunchConfig_t q = {};
@@ -876,13 +876,16 @@ static bool plan_fused(const RoleGeo* gs, const KState* kss, int nsets, int lvl,
       cudaGetLastError();
       active = 0;
     }
-    if (active >= 1) {
-      plan.coop = false;
-      plan.NCT = nct;
-      plan.L = Lc;
-      return true;
-    }
-  }
+    if (active < 1) return false;
+    plan.coop = false;
+    plan.NCT = nct;
+    plan.L = Lc;
+    return true;
+  };
+  for (int nct = nct0; nct <= cmax && nct <= ntp_max; ++nct)
+    if (try_nct(nct)) return true;
+  for (int nct = nct0 - 1; nct >= 1; --nct)
+    if (try_nct(nct)) return true;
   return false;
 }
 
