@@ -102,25 +102,30 @@ __device__ inline void fence_before() { asm volatile("tcgen05.fence::before_thre
 __device__ inline void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 __device__ inline void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
+// flags: bit 0 stages the fp64 centroids for the exact re-decisions; bit 1
+// keeps two token tiles in shared memory instead of three (large C and D).
 struct FusedLayout {
-  int KB, NC, tpc, stage;  // K-blocks, centroid columns (multiple of 32), tiles per CTA
+  int KB, NC, tpc, flags;  // K-blocks, centroid columns (multiple of 32), tiles per CTA
   size_t a, bh, bl, cn2, xs, whist, loff, gtab, xn, asg, queue, cst, total;
 };
 
-__host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc, bool stage) {
+__host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc, int flags) {
   FusedLayout L;
   L.KB = D / 64;
   L.NC = NC;
   L.tpc = tpc;
-  L.stage = stage ? 1 : 0;
+  L.flags = flags;
+  const int ring = (flags & 2) ? 2 : 3;
   size_t o = 0;
-  L.a = o;     o += (size_t)3 * L.KB * kTile * 128;  // in use, under MMA, loading
+  L.a = o;     o += (size_t)ring * L.KB * kTile * 128;  // in use, under MMA, loading
+  // the queued rows and the per-warp counts are used only after a round's
+  // tiles are done: they share the tile slots
+  L.xs = L.a;                                          // queued token rows in fp64
+  L.whist = L.a + (size_t)kWarps * D * 8;              // per-warp counts, then bases
   L.bh = o;    o += (size_t)L.KB * NC * 128;
   L.bl = o;    o += (size_t)L.KB * NC * 128;
   L.cn2 = o;   o += (size_t)NC * 4;
   o = (o + 15) & ~(size_t)15;
-  L.xs = o;    o += (size_t)kWarps * D * 8;           // queued token rows in fp64
-  L.whist = o; o += (size_t)kWarps * NC * 4;          // per-warp counts, then bases
   L.loff = o;  o += (size_t)(NC + 1) * 4;
   L.gtab = o;  o += (size_t)kWarps * (2 * kMaxNCT + 1) * 4;   // owner warps' rank tables
   L.xn = o;    o += (size_t)tpc * kTile * 4;          // token norms (screen bound)
@@ -128,7 +133,7 @@ __host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc, bool
   L.queue = o; o += (size_t)tpc * kTile * 2;
   o = (o + 15) & ~(size_t)15;
   L.cst = o;                                          // fp64 centroids, row stride D + 1
-  if (stage) o += (size_t)NC * (D + 1) * 8;
+  if (flags & 1) o += (size_t)NC * (D + 1) * 8;
   L.total = o + 1024;
   return L;
 }
@@ -248,7 +253,8 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(1024) unsigned char fz_dyn[];
   unsigned char* base = fz_dyn + ((1024 - (saddr(fz_dyn) & 1023)) & 1023);
-  const FusedLayout Lo = fused_layout(D, NC, tpc_max, stage != 0);
+  const FusedLayout Lo = fused_layout(D, NC, tpc_max, stage);
+  const int ring = (stage & 2) ? 2 : 3;  // token tile slots
   const int set = (int)blockIdx.x < fs.nblk0 ? 0 : 1;
   const RoleGeo& g = fs.g[set];
   const KState& ks = fs.ks[set];
@@ -383,7 +389,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     }
     mma_commit(saddr(&mbar[buf]));
   };
-  auto tile_buf = [&](int k) { return A0 + (k % 3) * ATILE; };
+  auto tile_buf = [&](int k) { return A0 + (k % ring) * ATILE; };
 
   for (int it = 0; it < iters; ++it) {
     const bool last = it + 1 == iters;
@@ -436,7 +442,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         __syncthreads();
         fence_after();
         if (tid == 0) issue_mma(tile_buf(k + 1), buf ^ 1);
-        if (k + 2 < ntl) load_tile(tl_ + 2, tile_buf(k + 2));
+        if (ring == 3 && k + 2 < ntl) load_tile(tl_ + 2, tile_buf(k + 2));
         cp_commit();
       }
       // token norms for the screen bound, from the staged tile, first round only
@@ -460,6 +466,10 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       phase[buf] ^= 1u;
       const bool ok = __syncthreads_and(done);
       if (!ok && tid == 0) atomicExch(ks.err, 1);
+      if (ring == 2 && k + 2 < ntl) {  // tile k's slot is free once its MMA is done
+        load_tile(tl_ + 2, tile_buf(k + 2));
+        cp_commit();
+      }
       fence_after();
       const uint32_t tm = tbase + (uint32_t)(buf * ncp) + ((uint32_t)((warp & 3) * 32) << 16);
       // ---- epilogue: each half of the warps scans half of the columns ---------
@@ -542,7 +552,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     // ---- exact fp64 decision of the queued tokens, one warp per token --------
     const int qn = qcount;
     if (qn > 0) {
-      if (stage) {
+      if (stage & 1) {
         const int tot = C * D;
         for (int e0 = tid; e0 < tot; e0 += 16 * kFT) {  // 16 loads in flight per thread
           double v[16];
@@ -565,7 +575,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         const __nv_bfloat16* xr = X + (p.row0 + tok0 + uq) * D;
         for (int d = lane; d < D; d += 32) xw[d] = (double)__bfloat162float(xr[d]);
         __syncwarp();
-        const int bc = stage ? exact_argmin<D, true>(xw, cst, c64g, C, lane)
+        const int bc = (stage & 1) ? exact_argmin<D, true>(xw, cst, c64g, C, lane)
                              : exact_argmin<D, false>(xw, cst, c64g, C, lane);
         if (lane == 0) asg[uq] = (unsigned short)bc;
         __syncwarp();
@@ -813,9 +823,11 @@ static bool plan_fused(const RoleGeo* gs, const KState* kss, int nsets, int lvl,
   auto layout_for = [&](int nct, FusedLayout& Lc) {
     const int tpc_max = cdiv(ntp_max, nct);
     if (tpc_max * kTile > 65535) return false;
-    Lc = fused_layout(D, NC, tpc_max, true);
-    if (Lc.total > kSmemLimit) Lc = fused_layout(D, NC, tpc_max, false);
-    return Lc.total <= kSmemLimit;
+    for (int flags : {1, 0, 3, 2}) {  // three tile slots first, staging first
+      Lc = fused_layout(D, NC, tpc_max, flags);
+      if (Lc.total <= kSmemLimit) return true;
+    }
+    return false;
   };
   int dev = 0, nsm = 0, coop_ok = 0;
   cudaGetDevice(&dev);
@@ -923,12 +935,12 @@ static void launch_plan(const RoleGeo* gs, const KState* kss, int nsets, int lvl
     cudaFuncSetAttribute(kmeans_fused_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)plan.L.total);
     cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, true>, fs, iters, plan.NCT, NC, plan.L.tpc,
-                       tcols, plan.L.stage);
+                       tcols, plan.L.flags);
   } else {
     cudaFuncSetAttribute(kmeans_fused_kernel<D, false>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.L.total);
     cudaLaunchKernelEx(&cfg, kmeans_fused_kernel<D, false>, fs, iters, plan.NCT, NC, plan.L.tpc,
-                       tcols, plan.L.stage);
+                       tcols, plan.L.flags);
   }
 }
 
