@@ -198,6 +198,7 @@ AttnLayout layout(const muse_shape* sh, const muse_params* pr, bool causal, cons
   const bool tilted = pr->mode == MUSE_TILTED;
   if (dt == 0) {
     L.s1.Uh = cv.take<__half>(wave * cc * sh->D * 2);
+    L.s1.Ul = cv.take<__half>(wave * cc * sh->D * 2);
     L.s1.Kfh = tilted ? cv.take<__nv_bfloat16>(wave * cc * sh->D * 2) : nullptr;
     L.s1.Kfl = tilted ? cv.take<__nv_bfloat16>(wave * cc * sh->D * 2) : nullptr;
     L.V16 = cv.take<__half>((size_t)sh->B * sh->Hkv * sh->N * sh->D * 2);
@@ -240,6 +241,10 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   a.scale = pr->scale;
   a.Cq = pr->Cq;
   a.Ck = pr->Ck;
+  // bf16 DIPOLE causal levels with few tokens per cluster: per key token
+  a.dense_lv = (causal && sh->dtype == MUSE_BF16 && pr->mode == MUSE_DIPOLE && L.V16)
+                   ? dense_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck)
+                   : 0;
   const size_t elt = sh->dtype == MUSE_BF16 ? 2 : 4;
   if (a.n_exact && causal)
     cudaMemsetAsync(a.n_exact, 0, (size_t)sh->B * sh->Hq * sh->N * 8, st);

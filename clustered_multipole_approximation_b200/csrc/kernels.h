@@ -24,6 +24,7 @@ struct Stage1 {
   float* U;       // [nq][Cq][Ck][D] summary values u_ij (fp32 path)
   float* Kf;      // [nq][Cq][Ck][D] far-field key rows, TILTED only: k_hat_ij (fp32 path)
   __half* Uh;     // [nq][Cq][Ck][D] u_ij in fp16 (bf16 path)
+  __half* Ul;     // [nq][Cq][Ck][D] u_ij - Uh in fp16 (bf16 path)
   __nv_bfloat16* Kfh;  // [nq][Cq][Ck][D] bf16 hi / lo split of k_hat_ij (bf16 path, TILTED)
   __nv_bfloat16* Kfl;
   int* sel;       // [nq_total][Cq][topk]
@@ -44,7 +45,19 @@ struct AttnArgs {
   int mode, topk;
   float scale;
   int Cq, Ck;
+  int dense_lv;       // causal levels (bit l) whose far field runs per key token
 };
+
+// Key problem that a query problem attends: the same (b, level, pair) of the
+// kv-head its q-head shares.
+__device__ inline int kv_problem(const AttnArgs& a, int qpid) {
+  const int ppb = a.qg.lv.pairs_per_bh;
+  const int bhq = qpid / ppb, pi = qpid - bhq * ppb;
+  const int Hq = a.qg.BH / a.B, Hkv = a.kg.BH / a.B;
+  const int b = bhq / Hq, hq = bhq - b * Hq;
+  const int bhk = b * Hkv + hq / a.G;
+  return bhk * a.kg.lv.pairs_per_bh + pi;
+}
 
 void run_kmeans(const RoleGeo& g, const KState& ks, int iters, const float* init,
                 cudaStream_t st);
@@ -74,6 +87,12 @@ void run_bf16_to_half(const void* src, __half* dst, size_t n, cudaStream_t st);
 void run_stage2_mma(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 // Stage 1 (DIPOLE) on tcgen05 tensor cores (bf16 inputs).
 void run_stage1_dipole_tc(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
+
+// The levels in a.dense_lv (bf16 DIPOLE, causal): far field and retrieved
+// keys per key token on mma.sync tiles, no stage-1 tables.
+void run_stage2_dense(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
+// Levels the dense form covers for these sizes (bit l set), 0 if none.
+int dense_levels(const Levels& lv, int D, int Cq, int Ck);
 
 // Causal: exact local block + merge of the level partials into O.
 void run_local_merge(const AttnArgs& a, int L, cudaStream_t st);

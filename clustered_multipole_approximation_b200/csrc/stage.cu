@@ -29,15 +29,6 @@
 
 namespace muse {
 
-__device__ inline int kv_problem(const AttnArgs& a, int qpid) {
-  const int ppb = a.qg.lv.pairs_per_bh;
-  const int bhq = qpid / ppb, pi = qpid - bhq * ppb;
-  const int Hq = a.qg.BH / a.B, Hkv = a.kg.BH / a.B;
-  const int b = bhq / Hq, hq = bhq - b * Hq;
-  const int bhk = b * Hkv + hq / a.G;
-  return bhk * a.kg.lv.pairs_per_bh + pi;
-}
-
 // ----------------------------------------------------------------------------
 // stage 1: one CTA per (query problem, key cluster j).  The cluster's members
 // (k - mu_j and v) are staged in shared memory once; query centroids come in
@@ -47,8 +38,13 @@ __device__ inline int kv_problem(const AttnArgs& a, int qpid) {
 // ----------------------------------------------------------------------------
 // Stage-1 table stores in the form the stage-2 kernel of the input dtype reads.
 __device__ inline void put_u(const Stage1& s1, size_t i, float v) {
-  if (s1.Uh) s1.Uh[i] = __float2half_rn(v);
-  else s1.U[i] = v;
+  if (s1.Uh) {
+    const __half hi = __float2half_rn(v);
+    s1.Uh[i] = hi;
+    s1.Ul[i] = __float2half_rn(v - __half2float(hi));
+  } else {
+    s1.U[i] = v;
+  }
 }
 __device__ inline void put_kf(const Stage1& s1, size_t i, float v) {
   if (s1.Kfh) {
@@ -664,8 +660,11 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
       select_kernel<D, false><<<grid, 256, smem, st>>>(a, s1, qp0);
   }
   if (sizeof(T) == 2) {
-    ProfScope ps(st, "stage2_attn");
-    run_stage2_mma(a, s1, qp0, nqp, st);
+    {
+      ProfScope ps(st, "stage2_attn");
+      run_stage2_mma(a, s1, qp0, nqp, st);
+    }
+    if (a.dense_lv) run_stage2_dense(a, s1, qp0, nqp, st);
   } else {
     ProfScope ps(st, "stage2_attn");
     if (a.out_f32)

@@ -12,13 +12,16 @@
 //   G = K nu^T      tcgen05.mma kind::f16, M=128 members, N=128 query
 //                   clusters, bf16 keys x bf16 hi + lo split of nu (two MMAs
 //                   into one fp32 TMEM accumulator);
-//   W = 1 + s (G - nu . mu_j)   thread t forms member t's row in fp16 and
-//                   stores it as the MN-major A operand of the next MMA;
-//   U += W^T V      tcgen05.mma, M=128 query clusters, N=D, K=128 members,
-//                   fp16 operands (both MN-major: rows as they are formed or
-//                   stored), fp32 accumulator resident in TMEM over the chunks.
-// Thread i then writes u_ij = U[i] / n_j in fp16 (128 contiguous bytes per
-// 64 dimensions), the operand form of stage 2.
+//   W = 1 + s (G - nu . mu_j)   thread t forms member t's row as an fp16
+//                   hi + lo pair and stores both as MN-major A operands;
+//   U += W_hi^T V + W_lo^T V   tcgen05.mma, M=128 query clusters, N=D,
+//                   K=128 members, fp16 operands (both MN-major: rows as they
+//                   are formed or stored), fp32 accumulator resident in TMEM
+//                   over the chunks.  The split keeps u_ij accurate when the
+//                   dipole factors are large (heavy-tailed keys): one fp16
+//                   rounding of W costs 2^-11 |W| per member.
+// Thread i then writes u_ij = U[i] / n_j as an fp16 hi + lo pair (128
+// contiguous bytes per 64 dimensions each), the operand form of stage 2.
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -90,6 +93,13 @@ __device__ inline uint32_t h2bits(float x, float y) {
   const __half2 h = __floats2half2_rn(x, y);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
+// fp16 pair (x, y) = hi + lo (residual 2^-22 relative).
+__device__ inline void split_h2bits(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x, y);
+  const float2 f = __half22float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = h2bits(x - f.x, y - f.y);
+}
 
 template <int D>
 struct S1Layout {
@@ -100,6 +110,10 @@ struct S1Layout {
   static constexpr int KM = NL + OP;        // member keys, K-major
   static constexpr int VM = KM + OP;        // member values (fp16), MN-major B
   static constexpr int W = VM + OP;         // [2 cluster chunks][128 members][128 B], MN-major A
+  // fp16 residual of W, same layout: it takes the nu operands' place (2 x
+  // 128 x 128 bytes fit in NH, or in NH and NL for D = 64), which the G MMA
+  // of the member chunk has finished with; every chunk reloads nu
+  static constexpr int WL = NH;
   static constexpr int NM = W + 2 * kR * 128;  // nu_i . mu_j
   static constexpr int MU = NM + kR * 4;
   static constexpr int TOTAL = MU + D * 4 + 1024;
@@ -120,10 +134,8 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
 
   const int lq = blockIdx.x, qpid = qp0 + lq, j = blockIdx.y;
   const Prob pq = prob_of(a.qg, qpid);
-  const int ppb = a.qg.lv.pairs_per_bh;
-  const int bhq = qpid / ppb, pi = qpid - bhq * ppb;
-  const int Hq = a.qg.BH / a.B, Hkv = a.kg.BH / a.B;
-  const int kpid = ((bhq / Hq) * Hkv + (bhq % Hq) / a.G) * a.kg.lv.pairs_per_bh + pi;
+  if ((a.dense_lv >> pq.level) & 1) return;  // that level's far field runs per key token
+  const int kpid = kv_problem(a, qpid);
   const Prob pk = prob_of(a.kg, kpid);
   if (j >= pk.C) return;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -178,15 +190,6 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
 
   for (int i0 = 0; i0 < pq.C; i0 += kR) {
     const int ic = imin(kR, pq.C - i0);
-    // query centroids (bf16 split) of this pass; rows past ic are zero
-    for (int e = tid; e < kR * KB * 8; e += kS1T) {
-      const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, c = q & 7;
-      const bool live = r < ic;
-      const size_t o = ((size_t)qpid * Cq + i0 + (live ? r : 0)) * D + kb * 64 + c * 8;
-      const uint32_t so = kb * kR * 128 + swz(r, c);
-      cp16(sb + Lt::NH + so, a.qs.cbf_hi + o, live ? 16 : 0);
-      cp16(sb + Lt::NL + so, a.qs.cbf_lo + o, live ? 16 : 0);
-    }
     {
       float dt = 0.f;
       if (tid < ic) {
@@ -204,6 +207,15 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
     }
     for (int t0 = 0; t0 < nj; t0 += kR) {
       const int nt = imin(kR, nj - t0);
+      // query centroids (bf16 split) of this pass; rows past ic are zero
+      for (int e = tid; e < kR * KB * 8; e += kS1T) {
+        const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, c = q & 7;
+        const bool live = r < ic;
+        const size_t o = ((size_t)qpid * Cq + i0 + (live ? r : 0)) * D + kb * 64 + c * 8;
+        const uint32_t so = kb * kR * 128 + swz(r, c);
+        cp16(sb + Lt::NH + so, a.qs.cbf_hi + o, live ? 16 : 0);
+        cp16(sb + Lt::NL + so, a.qs.cbf_lo + o, live ? 16 : 0);
+      }
       for (int e = tid; e < kR * KB * 8; e += kS1T) {
         const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, c = q & 7;
         const bool live = r < nt;
@@ -251,8 +263,12 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
             const float gv = __uint_as_float(g4[ii >> 4][ii & 15]);
             w[u] = tid < nt ? fmaf(s, gv - nm[64 * h + ii], 1.f) : 0.f;
           }
-          *reinterpret_cast<uint4*>(wrow + swz(tid, c)) =
-              make_uint4(h2bits(w[0], w[1]), h2bits(w[2], w[3]), h2bits(w[4], w[5]), h2bits(w[6], w[7]));
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) split_h2bits(w[2 * u], w[2 * u + 1], hi[u], lo[u]);
+          *reinterpret_cast<uint4*>(wrow + swz(tid, c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(wrow + (Lt::WL - Lt::W) + swz(tid, c)) =
+              make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       }
       fence_async();
@@ -261,33 +277,34 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
       fence_after();
       if (tid == 0) {
 #pragma unroll
-        for (int k = 0; k < kR / 16; ++k)  // 16 members per step: two 8-row groups
-          umma(tU, desc_mn(sb + Lt::W + 2048 * k, kR * 128), desc_mn(sb + Lt::VM + 2048 * k, kR * 128),
-               id_u, (t0 > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < kR / 16; ++k) {  // 16 members per step: two 8-row groups
+          const uint64_t vd = desc_mn(sb + Lt::VM + 2048 * k, kR * 128);
+          umma(tU, desc_mn(sb + Lt::W + 2048 * k, kR * 128), vd, id_u, (t0 > 0 || k > 0) ? 1u : 0u);
+          umma(tU, desc_mn(sb + Lt::WL + 2048 * k, kR * 128), vd, id_u, 1u);
+        }
         umma_commit(s32(&mbar[1]));
       }
       ok = wait_mbar(s32(&mbar[1]), ph[1]) && ok;  // the operands are reloaded next chunk
       ph[1] ^= 1u;
       fence_after();
     }
-    // ---- u_ij = U[i] / n_j in fp16, thread i = query cluster i0 + i -----------
+    // ---- u_ij = U[i] / n_j as fp16 hi + lo, thread i = query cluster i0 + i ---
 #pragma unroll
     for (int d0 = 0; d0 < D; d0 += 16) {
       uint32_t r1[16];
       tld16(tl + kR + d0, r1);
       tld_wait();
       if (tid < ic) {
-        __half* dst = s1.Uh + (ij0 + (size_t)(i0 + tid) * Ck) * D + d0;
-        uint4 w0 = make_uint4(h2bits(__uint_as_float(r1[0]) * inv_n, __uint_as_float(r1[1]) * inv_n),
-                              h2bits(__uint_as_float(r1[2]) * inv_n, __uint_as_float(r1[3]) * inv_n),
-                              h2bits(__uint_as_float(r1[4]) * inv_n, __uint_as_float(r1[5]) * inv_n),
-                              h2bits(__uint_as_float(r1[6]) * inv_n, __uint_as_float(r1[7]) * inv_n));
-        uint4 w1 = make_uint4(h2bits(__uint_as_float(r1[8]) * inv_n, __uint_as_float(r1[9]) * inv_n),
-                              h2bits(__uint_as_float(r1[10]) * inv_n, __uint_as_float(r1[11]) * inv_n),
-                              h2bits(__uint_as_float(r1[12]) * inv_n, __uint_as_float(r1[13]) * inv_n),
-                              h2bits(__uint_as_float(r1[14]) * inv_n, __uint_as_float(r1[15]) * inv_n));
-        reinterpret_cast<uint4*>(dst)[0] = w0;
-        reinterpret_cast<uint4*>(dst)[1] = w1;
+        const size_t o = (ij0 + (size_t)(i0 + tid) * Ck) * D + d0;
+        uint32_t hi[8], lo[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          split_h2bits(__uint_as_float(r1[2 * u]) * inv_n, __uint_as_float(r1[2 * u + 1]) * inv_n,
+                       hi[u], lo[u]);
+        reinterpret_cast<uint4*>(s1.Uh + o)[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        reinterpret_cast<uint4*>(s1.Uh + o)[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+        reinterpret_cast<uint4*>(s1.Ul + o)[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        reinterpret_cast<uint4*>(s1.Ul + o)[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
       }
     }
     fence_before();

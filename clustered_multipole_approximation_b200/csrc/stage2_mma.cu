@@ -11,14 +11,15 @@
 // as bf16 m16n8k16 MMAs with fp32 accumulation: bf16 query and key rows are
 // exact, a far-field key row (fp32) enters as its bf16 hi + lo split (two
 // MMAs, residual 2^-18 relative).  P and V enter the PV product as fp16 (the
-// fp16 copy of V is exact in fp16's normal range; u_ij is rounded to 11 bits),
-// accumulating in fp32.  Key blocks of 64 rows stream through shared memory
+// fp16 copy of V is exact in fp16's normal range); for far rows P and u_ij
+// each enter as an fp16 hi + lo pair, accumulating in fp32.  Key blocks of 64 rows stream through shared memory
 // with cp.async, two blocks in flight.
 #include <cuda_fp16.h>
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "mma_sync.cuh"
 
 namespace muse {
 
@@ -29,77 +30,12 @@ constexpr int kMK = 64;      // key rows per block
 constexpr int kThreads = 256;
 constexpr int kXRows = 2048;  // exact rows resolved once per CTA
 
-__device__ inline int kvp(const AttnArgs& a, int qpid) {
-  const int ppb = a.qg.lv.pairs_per_bh;
-  const int bhq = qpid / ppb, pi = qpid - bhq * ppb;
-  const int Hq = a.qg.BH / a.B, Hkv = a.kg.BH / a.B;
-  const int b = bhq / Hq, hq = bhq - b * Hq;
-  return (b * Hkv + hq / a.G) * a.kg.lv.pairs_per_bh + pi;
-}
-
-__device__ inline uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// 16-byte async copy; src_bytes = 0 fills the destination with zeros.
-__device__ inline void cp16(void* dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(src_bytes));
-}
-__device__ inline void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ inline void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
-
-__device__ inline void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ inline void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ inline void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ inline void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// 2^x on the special-function unit (PTX ex2.approx, relative error ~2^-22;
-// ex2(-inf) = 0).
-__device__ inline float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Running maxima start at a finite floor so that fully masked blocks need no
-// special case: exp2(-inf - floor) = 0 and exp2(floor - floor) = 1.
-constexpr float kMaxFloor = -1.0e30f;
-
-__device__ inline uint32_t pack_h2(float x, float y) {
-  __half2 h = __floats2half2_rn(x, y);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 template <int D>
 struct KBuf {
   __nv_bfloat16 k[kMK][D + 8];    // exact keys, or the hi part of far keys
   __nv_bfloat16 k2[kMK][D + 8];   // lo part of far keys
-  __half v[kMK][D + 8];
+  __half v[kMK][D + 8];           // exact values, or the hi part of u_ij
+  __half v2[kMK][D + 8];          // lo part of u_ij (far blocks)
   float bias[kMK];
 };
 
@@ -107,13 +43,14 @@ template <int D>
 struct Smem2 {
   __nv_bfloat16 q[kMQ][D + 8];
   KBuf<D> buf[2];
-  unsigned char inR[kMaxC];
   float fb[kMaxC];      // far-field logit offset (base 2) per key cluster, -inf if not far
-  int sel[kMaxC];
+  unsigned short sel[kMaxC];
   int selstart[kMaxC];  // start of each retrieved cluster in the concatenated list
   int selbase[kMaxC];   // its first position in the key problem's sorted order
   int xrow[kXRows];     // the concatenated list's rows, when it has at most kXRows
 };
+// two CTAs per SM at D = 64 (228 KB per SM, 1 KB reserved per CTA)
+static_assert(2 * (sizeof(Smem2<64>) + 1024) <= 228 * 1024, "stage-2 tables too large");
 
 }  // namespace
 
@@ -153,24 +90,24 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
   constexpr int CH = D / 8;    // 16-byte chunks per row
   const int lq = blockIdx.x, qpid = qp0 + lq, i = blockIdx.y;
   const Prob pq = prob_of(a.qg, qpid);
-  if (i >= pq.C) return;
+  if (i >= pq.C || ((a.dense_lv >> pq.level) & 1)) return;
   const int Cq = a.Cq, Ck = a.Ck;
   const int nqi = a.qs.counts[(size_t)qpid * Cq + i];
   if (nqi == 0) return;
-  const int kpid = kvp(a, qpid);
+  const int kpid = kv_problem(a, qpid);
   const Prob pk = prob_of(a.kg, kpid);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;
   const int nsel = a.topk > 0 ? s1.nsel[(size_t)qpid * Cq + i] : 0;
-  for (int j = tid; j < pk.C; j += kThreads) sm.inR[j] = 0;
-  __syncthreads();
-  for (int r = tid; r < nsel; r += kThreads) {
-    const int j = s1.sel[((size_t)qpid * Cq + i) * a.topk + r];
-    sm.sel[r] = j;
-    sm.inR[j] = 1;
-  }
-  __syncthreads();
   const int* kc = a.ks.counts + (size_t)kpid * Ck;
+  // far-field offsets of the non-empty clusters; the retrieved ones are then
+  // taken out of the far field (their keys enter exactly)
+  for (int r = tid; r < nsel; r += kThreads)
+    sm.sel[r] = (unsigned short)s1.sel[((size_t)qpid * Cq + i) * a.topk + r];
+  for (int j = tid; j < pk.C; j += kThreads)
+    sm.fb[j] = kc[j] > 0 ? s1.fbias[((size_t)lq * Cq + i) * Ck + j] * 1.4426950408889634f : -INFINITY;
+  __syncthreads();
+  for (int r = tid; r < nsel; r += kThreads) sm.fb[sm.sel[r]] = -INFINITY;
   const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
   const int* kperm = a.ks.perm + pk.slot0;
   // the retrieved clusters' members, concatenated in selection order, are one
@@ -180,11 +117,8 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
     sm.selstart[r] = (int)nexact;
     nexact += kc[sm.sel[r]];
   }
-  // per-CTA tables: far-field offsets, the retrieved clusters' first sorted
-  // positions and, when it fits, the row of every exact key
-  for (int j = tid; j < pk.C; j += kThreads)
-    sm.fb[j] = (kc[j] > 0 && !sm.inR[j]) ? s1.fbias[((size_t)lq * Cq + i) * Ck + j] * 1.4426950408889634f
-                                       : -INFINITY;
+  // per-CTA tables: the retrieved clusters' first sorted positions and, when
+  // it fits, the row of every exact key
   for (int r = tid; r < nsel; r += kThreads) sm.selbase[r] = koff[sm.sel[r]];
   __syncthreads();
   const bool prerow = nexact <= kXRows;
@@ -223,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
   const __nv_bfloat16* khi = tilted ? s1.Kfh + ij0 * D : a.ks.cbf_hi + (size_t)kpid * Ck * D;
   const __nv_bfloat16* klo = tilted ? s1.Kfl + ij0 * D : a.ks.cbf_lo + (size_t)kpid * Ck * D;
   const __half* uh = s1.Uh + ij0 * D;
+  const __half* ul = s1.Ul + ij0 * D;
 
   // block b (far blocks first, then the retrieved clusters' keys) into buf
   auto issue = [&](int b, KBuf<D>& B) {
@@ -235,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
         cp16(&B.k[r][c], khi + o, live ? 16 : 0);
         cp16(&B.k2[r][c], klo + o, live ? 16 : 0);
         cp16(&B.v[r][c], uh + o, live ? 16 : 0);
+        cp16(&B.v2[r][c], ul + o, live ? 16 : 0);
       }
       for (int r = tid; r < kMK; r += kThreads) {
         const int j = j0 + r;
@@ -364,6 +300,9 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
           o[n][2] *= scale[1];
           o[n][3] *= scale[1];
         }
+        // far rows: P and u_ij each as an fp16 hi + lo pair (P_hi u_hi +
+        // P_lo u_hi + P_hi u_lo), since a dipole summary can be far larger
+        // than the values it averages; exact rows: P and v in fp16
 #pragma unroll
         for (int kk = 0; kk < kMK / 16; ++kk) {
           uint32_t pa[4];
@@ -379,6 +318,28 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
             ldsm_x4_t(smem_u32(&B.v[key][col]), b0, b1, b2, b3);
             mma_f16(o[2 * np], pa, b0, b1);
             mma_f16(o[2 * np + 1], pa, b2, b3);
+          }
+        }
+        if (two) {
+#pragma unroll
+          for (int kk = 0; kk < kMK / 16; ++kk) {
+            uint32_t pa[4], pl[4];
+            split_h2(sc[2 * kk][0], sc[2 * kk][1], pa[0], pl[0]);
+            split_h2(sc[2 * kk][2], sc[2 * kk][3], pa[1], pl[1]);
+            split_h2(sc[2 * kk + 1][0], sc[2 * kk + 1][1], pa[2], pl[2]);
+            split_h2(sc[2 * kk + 1][2], sc[2 * kk + 1][3], pa[3], pl[3]);
+#pragma unroll
+            for (int np = 0; np < ND / 2; ++np) {
+              const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+              const int col = np * 16 + (lane >> 4) * 8;
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4_t(smem_u32(&B.v[key][col]), b0, b1, b2, b3);
+              mma_f16(o[2 * np], pl, b0, b1);
+              mma_f16(o[2 * np + 1], pl, b2, b3);
+              ldsm_x4_t(smem_u32(&B.v2[key][col]), b0, b1, b2, b3);
+              mma_f16(o[2 * np], pa, b0, b1);
+              mma_f16(o[2 * np + 1], pa, b2, b3);
+            }
           }
         }
       }

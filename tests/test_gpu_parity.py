@@ -246,6 +246,24 @@ def test_causal_d128_clusters_above_block_size():
     check_causal(Q, K, V, "bf16", 64, 96, 3, 2, 4)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("topk", [0, 3])
+def test_causal_low_levels_per_key_token(D, topk):
+    """Levels with at most 8 keys per cluster (s = 128 and 256 with C = 32)
+    take the far field one key token at a time; the levels above (s = 512,
+    1024) keep the per-cluster tables.  Every head against the oracle, with a
+    heavy-tailed norm factor on q and k."""
+    Q, K, V = clustered_qkv(1, 4, 2, 2048, D, 24, 0.3, 0.5, "bf16", 60 + D + topk)
+    muse.profile_read()
+    muse.profile_enable(True)
+    try:
+        check_causal(Q, K, V, "bf16", 128, 32, 4, 61, topk)
+    finally:
+        muse.profile_enable(False)
+        launched = muse.profile_read()
+    assert "stage2_dense" in launched and "stage2_attn" in launched, launched
+
+
 def test_causal_single_block_is_exact():
     Q, K, V = clustered_qkv(1, 2, 1, 256, 64, 8, 0.3, 0.0, "f32", 52)
     O, _ = gpu_causal(Q, K, V, "f32", 256, 8, 3, 1, 2)
