@@ -151,7 +151,10 @@ muse_status muse_summarize(const void *K, const void *V, muse_dtype dtype,
  * s q.mu_j + log W_ij, or for TILTED s (q - nu_i).k_hat_ij + s nu_i.mu_j +
  * log W_ij; value u_ij) plus one exact term per key of the retrieved
  * clusters, all in one softmax.  O is written in the input dtype (fp32 with
- * out_f32); all arithmetic before that store is fp32 or wider.
+ * out_f32).  Accumulation is fp32 or wider.  For bf16 inputs the tensor-core
+ * operands are 16-bit: q, k and v exactly; centroids, summary values u_ij
+ * and far-field weights as bf16/fp16 hi + lo pairs; the softmax weights of
+ * exact keys rounded once to fp16.
  * Requires 1 <= Cq, Ck <= min(N, 1024), 0 <= topk <= Ck, iters >= 1.
  */
 muse_status muse_attn_fwd(const void *Q, const void *K, const void *V, void *O,
@@ -168,6 +171,9 @@ muse_status muse_attn_fwd(const void *Q, const void *K, const void *V, void *O,
  * block problem clustered inside that key block and the query block
  * [(2p+1) s, (2p+2) s) with C_eff = min(Ck, s) clusters; topk is a per-block
  * problem budget.  All terms meet in one softmax.  Requires Cq == Ck.
+ * For bf16 DIPOLE, levels with s <= 8 C_eff (s a multiple of 128, Ck <= 256)
+ * evaluate the far field one key token at a time (the same sums, expanded
+ * over each cluster's tokens) instead of through per-cluster summaries.
  */
 muse_status muse_attn_fwd_causal(const void *Q, const void *K, const void *V,
                                  void *O, const muse_shape *shape,
