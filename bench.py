@@ -12,6 +12,11 @@ timed (CUDA events on the launching stream).  With N > 1 (torchrun) every rank
 runs its own layer (weak scaling, no collective on the data path) and the time
 is the max over ranks.
 
+The headline line is the 8-head 8k acausal layer (DIPOLE).  The default run
+also times every other configuration with N >= 8k (the MONOPOLE variant of
+the 8k layer and the three causal layers) and reports each under
+"workloads", with its own roofline figures.
+
 --impl reference times the fp64 CPU oracle (the plain statement of the
 method) on the host cores, each step a bounded sample of the same workload.
 """
@@ -49,6 +54,8 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
     p.add_argument("--mode", default=None, choices=[None, "dipole", "monopole", "tilted"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-side", action="store_true",
+                   help="skip the other N >= 8k configurations of the default run")
     return p.parse_args()
 
 
@@ -116,57 +123,104 @@ class Clocks:
 
 
 # ---------------------------------------------------------------------------
-# algorithmic work per kernel launch (what the method must compute)
+# algorithmic work of one call (what the method must compute)
 # ---------------------------------------------------------------------------
 # DRAM bytes (read + write) of one launch of a kernel on a workload, from one ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum, caches flushed as in the
 # timed region).  An entry is removed whenever its kernel changes.
-NCU_TRAFFIC = {
-    ("acausal-bf16-h8-n8k", "kmeans_fused"): 18_488_064 + 3_584,
-}
+NCU_TRAFFIC: dict = {}
+
+# The library's per-kernel profiling names -> what they compute.
+TENSOR_KERNELS = ("kmeans_fused", "stage1_summaries", "stage2_attn", "stage2_dense",
+                  "causal_local_merge")
+
+
+def level_table(w):
+    """(block size s, pairs per head, effective clusters, per-key-token far field)
+    of every level; the acausal operator is one level with one block problem.
+    The per-key-token form runs where the library's dense-level rule admits it:
+    bf16 DIPOLE, C <= 256, s a multiple of 128, s <= 2048 and s <= 8 C_eff."""
+    if not w.causal:
+        return [(w.N, 1, w.C, False)]
+    out, s = [], w.block
+    while s < w.N:
+        ce = min(w.C, s)
+        dense = (w.dtype == "bf16" and w.mode == "dipole" and w.C <= 256 and s % 128 == 0
+                 and s <= 2048 and s <= 8 * ce)
+        out.append((s, w.N // (2 * s), ce, dense))
+        s *= 2
+    return out
+
+
+def retrieval_rows(w, mode, dbg):
+    """Far-field rows and exact retrieved keys summed over every query, per
+    level, counted from the actual clusterings and retrieval sets: a query of
+    cluster i in block problem p has one far row per non-empty key cluster
+    outside R_i and one exact key per member of R_i's clusters."""
+    G = w.Hq // w.Hkv
+    qa, ka = dbg["q_assign"], dbg["k_assign"]
+    sel = dbg.get("selected")
+    far = []
+    exact = []
+    pbase = 0
+    for lv, (s, npairs, ce, _dense) in enumerate(level_table(w)):
+        f_lv = e_lv = 0.0
+        for b in range(w.B):
+            for h in range(w.Hq):
+                if w.causal:
+                    qb = qa[b, h, lv].reshape(npairs, s)
+                    kb = ka[b, h // G, lv].reshape(npairs, s)
+                    sl = sel[b, h, pbase:pbase + npairs, :ce] if sel is not None else None
+                else:
+                    qb, kb = qa[b, h][None], ka[b, h // G][None]
+                    sl = sel[b, h][None] if sel is not None else None
+                off = (np.arange(npairs) * ce)[:, None]
+                nq = np.bincount((qb + off).ravel(), minlength=npairs * ce).reshape(npairs, ce)
+                nk = np.bincount((kb + off).ravel(), minlength=npairs * ce).reshape(npairs, ce)
+                nonempty = (nk > 0).sum(1, keepdims=True)
+                if sl is None or sl.shape[-1] == 0:
+                    nsel = np.zeros((npairs, ce))
+                    ex = np.zeros((npairs, ce))
+                else:
+                    ok = sl >= 0
+                    nsel = ok.sum(-1)
+                    got = np.take_along_axis(nk[:, None, :].repeat(ce, 1),
+                                             np.where(ok, sl, 0), axis=2)
+                    ex = (got * ok).sum(-1)
+                f_lv += float((nq * (nonempty - nsel)).sum())
+                e_lv += float((nq * ex).sum())
+        far.append(f_lv)
+        exact.append(e_lv)
+        pbase += npairs
+    return far, exact
 
 
 def algorithmic_work(w, mode, dbg):
-    """Per-launch algorithmic FLOPs and bytes of the acausal kernels, from the
-    shapes and the actual retrieval counts.  A multiply-add counts 2 FLOPs."""
-    B, Hq, Hkv, N, D, C = w.B, w.Hq, w.Hkv, w.N, w.D, w.C
-    G = Hq // Hkv
+    """Per-call algorithmic FLOPs of each kernel and of the whole operator
+    (a multiply-add counts 2 FLOPs), and the operator's algorithmic bytes:
+      k-means       T * 2 * tokens * C_eff * D per role (every level);
+      stage 1       min(2 C_eff^2 D^2 + 2 s D^2, 4 s C_eff D) per query problem
+                    (the dipole contraction; 0 for MONOPOLE);
+      stage 2       4 D per far row and per exact retrieved key;
+      local block   4 D per (query, key) pair of the causal local block;
+      bytes         Q, K and V read once, O written once."""
+    B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
+    far, exact = retrieval_rows(w, mode, dbg)
+    work = dict.fromkeys(TENSOR_KERNELS, 0.0)
+    for lv, (s, npairs, ce, dense) in enumerate(level_table(w)):
+        toks = npairs * s
+        work["kmeans_fused"] += w.iters * 2.0 * toks * ce * D * B * (Hq + Hkv)
+        if not dense and mode != "monopole":
+            work["stage1_summaries"] += npairs * B * Hq * min(2.0 * ce * ce * D * D + 2.0 * s * D * D,
+                                                              4.0 * s * ce * D)
+        work["stage2_dense" if dense else "stage2_attn"] += 4.0 * D * (far[lv] + exact[lv])
+    if w.causal:
+        L = w.block
+        work["causal_local_merge"] = 4.0 * D * B * Hq * (w.N // L) * L * (L + 1) / 2
     elt = 2 if w.dtype == "bf16" else 4
-    roles = [B * Hkv, B * Hq]
-    work = {}
-    # one assign launch per role and round: distances of every token to C centroids
-    work["kmeans_assign"] = dict(
-        flops=sum(2.0 * N * C * D * r for r in roles) / 2,
-        bytes=sum(N * D * elt * r + N * 4 * r for r in roles) / 2)
-    work["kmeans_reduce"] = dict(flops=sum(N * D * r for r in roles) / 2,
-                                 bytes=sum(N * D * elt * r for r in roles) / 2)
-    # the persistent k-means: every round of both clusterings in one launch
-    work["kmeans_fused"] = dict(flops=w.iters * sum(2.0 * N * C * D * r for r in roles),
-                                bytes=w.iters * sum(N * D * elt * r for r in roles))
-    # stage 1: the dipole contraction sum_t v_t (1 + s nu_i.k~_t) for every (i, t)
-    s1 = 0.0 if mode == "monopole" else 4.0 * N * D * C * B * Hq
-    work["stage1_summaries"] = dict(flops=s1, bytes=B * Hq * C * C * D * 4.0)
-    # stage 2: QK^T and PV for every far-field cluster and every retrieved key
-    k_counts = dbg["k_counts"]
-    q_assign = dbg["q_assign"]
-    sel = dbg.get("selected")
-    far_rows = 0.0
-    for b in range(B):
-        for h in range(Hq):
-            nonempty = int((k_counts[b, h // G] > 0).sum())
-            nq = np.bincount(q_assign[b, h], minlength=C)
-            nsel = (sel[b, h] >= 0).sum(-1) if sel is not None else np.zeros(C)
-            far_rows += float((nq * (nonempty - nsel)).sum())
-    exact = float(np.asarray(dbg["n_exact"], dtype=np.float64).sum())
-    work["stage2_attn"] = dict(flops=4.0 * D * (far_rows + exact),
-                               bytes=2.0 * B * Hq * N * D * elt + B * Hq * C * C * D * 4.0)
-    return work
-
-
-def total_algorithmic_flops(work, iters):
-    return (work["kmeans_fused"]["flops"] + work["stage1_summaries"]["flops"]
-            + work["stage2_attn"]["flops"])
-
+    nbytes = (B * Hq * w.N * D * 2 + 2 * B * Hkv * w.N * D) * elt
+    retrieved = sum(exact)
+    return work, sum(work.values()), nbytes, retrieved
 
 # ---------------------------------------------------------------------------
 # multi-rank plumbing (one independent layer per rank, no data-path collective)
@@ -193,13 +247,16 @@ def whole_job_throughput(tokens_per_rank: int, world: int, steps: int, max_ms: f
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
-def run_muse(args, w, rank, world, device):
+def run_muse(w, mode, steps, warmup, rank, world, device, e2e_leg=True):
+    """Times `steps` calls of the operator on workload `w` (inputs resident in
+    HBM, L2 flushed between calls) and, with e2e_leg, the same through host
+    buffers; returns the measurements and the roofline figures."""
     import clustered_multipole_approximation_b200 as muse
 
-    mode = args.mode or w.mode
     Q, K, V = make_inputs(w, seed=rank_data_seed(w, rank))
     cast = (lambda x: torch.from_numpy(x).to(torch.bfloat16)) if w.dtype == "bf16" else torch.from_numpy
     hq, hk, hv = cast(Q).pin_memory(), cast(K).pin_memory(), cast(V).pin_memory()
+    del Q, K, V
     q, k, v = hq.to(device), hk.to(device), hv.to(device)
     out = torch.empty_like(q)
     kw = dict(iters=w.iters, seed=w.cluster_seed, topk=w.topk, scale=w.scale, mode=mode)
@@ -219,19 +276,27 @@ def run_muse(args, w, rank, world, device):
         fn(q, k, v, out=out, workspace=ws, **kw)
 
     # one untimed call with inspection outputs: retrieval counts and accuracy
-    _, dbg = fn(q, k, v, debug=True, **kw)
-    o_chk = fn(q, k, v, **kw)
-    qq = q.float()
+    o_chk, dbg = fn(q, k, v, debug=True, workspace=ws, **kw)
+    muse.device_status(dbg["device_error"])
+    dbg = {n: t.cpu().numpy() for n, t in dbg.items()}
     G = w.Hq // w.Hkv
-    kk = k.float().repeat_interleave(G, dim=1)
-    vv = v.float().repeat_interleave(G, dim=1)
-    E = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, is_causal=w.causal,
-                                                         scale=w.scale)
-    rse_val = float(((o_chk.float() - E) ** 2).sum() / (E ** 2).sum())
-    del E, kk, vv, qq
+    num = den = 0.0
+    for h0 in range(0, w.Hq, G):  # exact attention one kv-group at a time (memory)
+        qq = q[:, h0:h0 + G].float()
+        kk = k[:, h0 // G:h0 // G + 1].float().expand(-1, G, -1, -1)
+        vv = v[:, h0 // G:h0 // G + 1].float().expand(-1, G, -1, -1)
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        with sdpa_kernel([SDPBackend.EFFICIENT_ATTENTION]):  # never the N^2-memory path
+            E = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, is_causal=w.causal,
+                                                                 scale=w.scale)
+        num += float(((o_chk[:, h0:h0 + G].float() - E) ** 2).sum())
+        den += float((E ** 2).sum())
+        del E, qq, kk, vv
+    rse_val = num / den
+    del o_chk
     torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
@@ -240,9 +305,10 @@ def run_muse(args, w, rank, world, device):
     torch.cuda.synchronize()
     clk = Clocks(device.index if device.index is not None else 0)
     clk.start()
+    muse.profile_read()
     muse.profile_enable(True)
     evs = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush.zero_()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -259,59 +325,74 @@ def run_muse(args, w, rank, world, device):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     tokens = w.B * w.N
-    value = whole_job_throughput(tokens, world, args.steps, total_ms)
-    ms_per_step = total_ms / args.steps
+    value = whole_job_throughput(tokens, world, steps, total_ms)
+    ms_per_step = total_ms / steps
 
-    # end to end through the public API: host inputs in, host output back
-    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    e2e_ms = 0.0
-    for i in range(args.warmup + args.steps):
-        flush.zero_()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        step()
-        ho.copy_(out, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            e2e_ms += e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, world, device)
-    e2e = {"value": whole_job_throughput(tokens, world, args.steps, e2e_ms), "unit": UNIT,
-           "h2d_bytes_per_step": int(hq.numel() * hq.element_size() * 1 + hk.numel() * hk.element_size()
-                                     + hv.numel() * hv.element_size()),
-           "d2h_bytes_per_step": int(ho.numel() * ho.element_size())}
+    e2e = None
+    if e2e_leg:
+        # end to end through the public API: host inputs in, host output back
+        ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        e2e_ms = 0.0
+        for i in range(warmup + steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(out, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= warmup:
+                e2e_ms += e0.elapsed_time(e1)
+        e2e_ms = max_over_ranks(e2e_ms, world, device)
+        e2e = {"value": whole_job_throughput(tokens, world, steps, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": int(hq.numel() * hq.element_size()
+                                         + hk.numel() * hk.element_size()
+                                         + hv.numel() * hv.element_size()),
+               "d2h_bytes_per_step": int(ho.numel() * ho.element_size())}
 
-    # roofline of the dominant kernel
+    # roofline: the dominant kernel, and the whole operator
     pk, how = peaks()
+    work, f_alg, b_alg, retrieved = algorithmic_work(w, mode, dbg)
+    exact_total = float(np.asarray(dbg["n_exact"], dtype=np.float64).sum())
+    local = work["causal_local_merge"] / (4.0 * w.D) if w.causal else 0.0
+    # the counted retrieval equals the library's own exact-key count
+    assert abs(exact_total - local - retrieved) < 0.5, (exact_total, local, retrieved)
     launches = sum(n for n, _ in prof.values())
     dom = max(prof, key=lambda n: prof[n][1])
     dom_launches, dom_ms = prof[dom]
-    avg_ms = dom_ms / dom_launches
-    roofline = {"kernel": dom, "bound": "tensor", "achieved": None,
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": None,
-                "traffic": NCU_TRAFFIC.get((w.name, dom)),
-                "peak_source": f"{how} bf16 dense (burst)", "avg_launch_ms": avg_ms}
-    if not w.causal:
-        work = algorithmic_work(w, mode, {n: t.cpu().numpy() for n, t in dbg.items()})
-        if dom in work:
-            ach = work[dom]["flops"] / (avg_ms / 1e3) / 1e12
-            roofline.update(achieved=ach, frac=ach / pk["bf16_tflops"],
-                            frac_of_sustained_peak=ach / pk["bf16_tflops_sustained"],
-                            flops_per_launch=work[dom]["flops"])
-        f_alg = total_algorithmic_flops(work, w.iters)
-        whole = {"algorithmic_tflop": f_alg / 1e12,
-                 "achieved_tflops": f_alg / (ms_per_step / 1e3) / 1e12,
-                 "frac_of_bf16_peak": f_alg / (ms_per_step / 1e3) / 1e12 / pk["bf16_tflops"],
-                 "frac_of_bf16_sustained_peak":
-                     f_alg / (ms_per_step / 1e3) / 1e12 / pk["bf16_tflops_sustained"]}
-    else:
-        whole = None
-    kernels = {n: {"launches": c, "ms_total": round(t, 4), "share": round(t / sum(x[1] for x in prof.values()), 4)}
-               for n, (c, t) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    peak = pk["bf16_tflops"]
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": None, "peak": peak,
+                "unit": "TFLOP/s", "frac": None, "traffic": NCU_TRAFFIC.get((w.name, dom)),
+                "peak_source": f"{how} bf16 dense (burst)",
+                "launches_per_call": dom_launches / steps,
+                "avg_launch_ms": dom_ms / dom_launches}
+    if work.get(dom):
+        per_call_ms = dom_ms / steps
+        ach = work[dom] / (per_call_ms / 1e3) / 1e12
+        roofline.update(achieved=ach, frac=ach / peak,
+                        frac_of_sustained_peak=ach / pk["bf16_tflops_sustained"],
+                        flops_per_launch=work[dom] / (dom_launches / steps))
+    t_roof = max(f_alg / (peak * 1e12), b_alg / (pk["hbm_gbs"] * 1e9))
+    whole = {"algorithmic_tflop": f_alg / 1e12, "algorithmic_gb": b_alg / 1e9,
+             "roofline_ms": t_roof * 1e3,
+             "achieved_tflops": f_alg / (ms_per_step / 1e3) / 1e12,
+             "frac": t_roof / (ms_per_step / 1e3),
+             "frac_of_bf16_sustained_peak":
+                 f_alg / (ms_per_step / 1e3) / 1e12 / pk["bf16_tflops_sustained"],
+             "flops_by_kernel": {n: f for n, f in work.items() if f}}
+    tot = sum(x[1] for x in prof.values())
+    kernels = {}
+    for n, (c, t) in sorted(prof.items(), key=lambda kv: -kv[1][1]):
+        e = {"launches": c, "ms_per_call": round(t / steps, 4), "share": round(t / tot, 4)}
+        if work.get(n):
+            e["tflops"] = round(work[n] / (t / steps / 1e3) / 1e12, 2)
+        kernels[n] = e
+    del q, k, v, out, ws, flush
+    torch.cuda.empty_cache()
     return dict(value=value, ms_per_step=ms_per_step, e2e=e2e, roofline=roofline, clocks=clocks,
                 gpu_launches=launches, kernels=kernels, rse=rse_val, mode=mode, whole_op=whole)
 
@@ -370,6 +451,20 @@ def config_of(w, mode):
     return c
 
 
+# Configurations timed next to the headline one in the default run (one line
+# each under "workloads"): every configuration with N >= 8k.
+SIDE_WORKLOADS = [("acausal-bf16-h8-n8k", "monopole"), ("causal-bf16-b2h8-n16k", None),
+                  ("causal-gqa32x8-n64k-d64", None), ("causal-gqa32x8-n32k-d128", None)]
+
+
+def side_entry(r, w, steps, warmup):
+    return {"config": config_of(w, r["mode"]), "value": r["value"], "unit": UNIT,
+            "ms_per_step": r["ms_per_step"], "steps": steps, "warmup": warmup,
+            "roofline": r["roofline"], "whole_operator": r["whole_op"],
+            "rse_vs_exact": r["rse"], "kernels": r["kernels"], "clocks": r["clocks"],
+            "gpu_launches": r["gpu_launches"]}
+
+
 def main():
     args = parse()
     w = WORKLOADS[args.workload]
@@ -386,7 +481,8 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
-    r = run_muse(args, w, rank, world, device)
+    mode = args.mode or w.mode
+    r = run_muse(w, mode, args.steps, args.warmup, rank, world, device)
     line = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -396,6 +492,16 @@ def main():
             "e2e": r["e2e"], "roofline": r["roofline"], "clocks": r["clocks"],
             "gpu_launches": r["gpu_launches"], "rse_vs_exact": r["rse"], "kernels": r["kernels"],
             "whole_operator": r["whole_op"]}
+    if world == 1 and not args.no_side and args.workload == DEFAULT_WORKLOAD and args.mode is None:
+        side = {}
+        for name, m in SIDE_WORKLOADS:
+            sw = WORKLOADS[name]
+            sm = m or sw.mode
+            big = sw.B * sw.Hq * sw.N >= 1 << 20
+            st, wu = (6, 3) if big else (args.steps, args.warmup)
+            rr = run_muse(sw, sm, st, wu, rank, world, device, e2e_leg=False)
+            side[f"{name}/{sm}"] = side_entry(rr, sw, st, wu)
+        line["workloads"] = side
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads = min(w.B * w.Hq, 8)
         dt, tps, thr = oracle_sample(w, r["mode"], heads)

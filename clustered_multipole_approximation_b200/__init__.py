@@ -56,7 +56,10 @@ class muse_debug(ctypes.Structure):
 EXPORTS = ["muse_workspace_size", "muse_cluster_workspace_size", "muse_cluster", "muse_summarize",
            "muse_attn_fwd", "muse_attn_fwd_causal", "muse_status_string", "muse_last_error",
            "muse_profile_enable", "muse_profile_read", "muse_cluster_static",
-           "muse_cluster_static_capacity"]
+           "muse_cluster_static_capacity", "muse_device_status", "muse_debug_inject_barrier_fault"]
+
+# Bits of the device error word (include/muse.h MUSE_DEVERR_*).
+DEVERR = {1: "MUSE_DEVERR_MMA_WAIT", 2: "MUSE_DEVERR_TEAM_BARRIER", 4: "MUSE_DEVERR_V_RANGE"}
 
 _lib = None
 
@@ -79,7 +82,7 @@ def load_library(path: str = LIB_PATH):
     lib.muse_cluster_workspace_size.argtypes = [i32] * 5
     lib.muse_cluster.restype = i32
     lib.muse_cluster.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, u64, i32, vp, vp, vp, vp,
-                                 vp, sz, vp]
+                                 vp, vp, sz, vp]
     lib.muse_summarize.restype = i32
     lib.muse_summarize.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
                                    sz, vp]
@@ -92,7 +95,11 @@ def load_library(path: str = LIB_PATH):
     lib.muse_last_error.argtypes = []
     lib.muse_cluster_static.restype = i32
     lib.muse_cluster_static.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, u64, i32, vp, vp,
-                                        vp, vp, vp]
+                                        vp, vp, vp, vp]
+    lib.muse_device_status.restype = i32
+    lib.muse_device_status.argtypes = [vp, vp]
+    lib.muse_debug_inject_barrier_fault.restype = None
+    lib.muse_debug_inject_barrier_fault.argtypes = [i32, i32]
     lib.muse_cluster_static_capacity.restype = sz
     lib.muse_cluster_static_capacity.argtypes = []
     lib.muse_profile_enable.restype = None
@@ -159,9 +166,13 @@ def _debug_buffers(q, k, params, causal):
     i32 = dict(dtype=torch.int32, device=dev)
     if causal:
         from math import log2
-        lv = int(round(log2(N // params.block))) if N // params.block > 1 else 0
+        nblk = N // params.block
+        lv = int(round(log2(nblk))) if nblk > 1 else 0
         out = dict(q_assign=torch.empty(B, Hq, lv, N // 2, **i32),
                    k_assign=torch.empty(B, Hkv, lv, N // 2, **i32))
+        if params.topk > 0 and nblk > 1:
+            # one row block per block problem, problems numbered level by level
+            out["selected"] = torch.empty(B, Hq, nblk - 1, params.Cq, params.topk, **i32)
     else:
         out = dict(q_assign=torch.empty(B, Hq, N, **i32), k_assign=torch.empty(B, Hkv, N, **i32),
                    k_counts=torch.empty(B, Hkv, params.Ck, **i32),
@@ -221,11 +232,23 @@ def muse_attn_fwd_causal(q, k, v, *, C, block, iters, seed, topk, scale=1.0, mod
     return _attn(True, q, k, v, p, out, workspace, debug, stream, out_dtype)
 
 
-def muse_cluster(x, C, iters, seed, role=0, init=None, workspace=None, stream=None):
-    """Lloyd k-means of each (b, h) row set of x [B,H,N,D].  Returns
-    (assign [B,H,N] int32, centroids [B,H,C,D] fp32, counts [B,H,C] int32)."""
+def device_status(device_error, stream=None) -> None:
+    """Wait for the stream, read a device error word (an int32 CUDA tensor
+    written by an entry point) and raise MuseError(MUSE_ERR_DEVICE_CHECK)
+    naming its MUSE_DEVERR_* bits if it is not 0."""
     lib = load_library()
-    _need_cuda(x, init, workspace)
+    _need_cuda(device_error)
+    _check(lib, lib.muse_device_status(_ptr(device_error), _stream(stream)))
+
+
+def muse_cluster(x, C, iters, seed, role=0, init=None, workspace=None, stream=None,
+                 device_error=None):
+    """Lloyd k-means of each (b, h) row set of x [B,H,N,D].  Returns
+    (assign [B,H,N] int32, centroids [B,H,C,D] fp32, counts [B,H,C] int32).
+    `device_error` (optional int32 CUDA tensor of one element) receives the
+    device error word."""
+    lib = load_library()
+    _need_cuda(x, init, workspace, device_error)
     B, H, N, D = x.shape
     if init is not None and (init.dtype != torch.float32 or tuple(init.shape) != (B, H, C, D)):
         raise ValueError("init must be fp32 [B,H,C,D]")
@@ -239,26 +262,32 @@ def muse_cluster(x, C, iters, seed, role=0, init=None, workspace=None, stream=No
     counts = torch.empty(B, H, C, dtype=torch.int32, device=x.device)
     st = lib.muse_cluster(_ptr(x), _dtype_code(x), B, H, N, D, C, iters, int(seed) & (2 ** 64 - 1),
                           role, _ptr(init), _ptr(assign), _ptr(cent), _ptr(counts),
-                          _ptr(workspace), workspace.numel(), _stream(stream))
+                          _ptr(device_error), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(lib, st)
     return assign, cent, counts
 
 
-def muse_cluster_static(x, C, iters, seed, role=0, init=None, stream=None):
+def muse_cluster_static(x, C, iters, seed, role=0, init=None, stream=None, device_error=None):
     """muse_cluster for callers that cannot allocate a workspace: the scratch
     is the fixed array built into the library (see include/muse.h for its
     limit and its sharing rules).  Returns (assign, centroids, counts)."""
     lib = load_library()
-    _need_cuda(x, init)
+    _need_cuda(x, init, device_error)
     B, H, N, D = x.shape
     assign = torch.empty(B, H, N, dtype=torch.int32, device=x.device)
     cent = torch.empty(B, H, C, D, dtype=torch.float32, device=x.device)
     counts = torch.empty(B, H, C, dtype=torch.int32, device=x.device)
     st = lib.muse_cluster_static(_ptr(x), _dtype_code(x), B, H, N, D, C, iters,
                                  int(seed) & (2 ** 64 - 1), role, _ptr(init), _ptr(assign),
-                                 _ptr(cent), _ptr(counts), _stream(stream))
+                                 _ptr(cent), _ptr(counts), _ptr(device_error), _stream(stream))
     _check(lib, st)
     return assign, cent, counts
+
+
+def inject_barrier_fault(rank: int, spin_limit: int = 0) -> None:
+    """Failure-path testing: see muse_debug_inject_barrier_fault in
+    include/muse.h (rank < 0 switches it off)."""
+    load_library().muse_debug_inject_barrier_fault(int(rank), int(spin_limit))
 
 
 def muse_summarize(k, v, assign, C, with_dipole=True, stream=None):

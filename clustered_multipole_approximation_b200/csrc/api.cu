@@ -31,6 +31,10 @@ muse_status check_launch() {
   return MUSE_OK;
 }
 
+// A pointer argument that violates its alignment (NULL passes: the caller
+// checks required pointers separately).
+bool misaligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) != 0; }
+
 int ilog2_exact(int x) {  // -1 unless x is a power of two
   if (x <= 0 || (x & (x - 1))) return -1;
   int l = 0;
@@ -220,6 +224,14 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   muse_status s = validate(sh, pr, causal);
   if (s != MUSE_OK) return s;
   if (!Q || !K || !V || !O) return fail(MUSE_ERR_INVALID_ARG, "Q, K, V and O must not be NULL");
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16))
+    return fail(MUSE_ERR_INVALID_ARG, "Q, K, V and O must be 16-byte aligned");
+  if (misaligned(ws, 256)) return fail(MUSE_ERR_INVALID_ARG, "the workspace must be 256-byte aligned");
+  if (dbg && (misaligned(dbg->q_assign, 4) || misaligned(dbg->k_assign, 4) ||
+              misaligned(dbg->selected, 4) || misaligned(dbg->k_counts, 4) ||
+              misaligned(dbg->q_centroids, 4) || misaligned(dbg->k_centroids, 4) ||
+              misaligned(dbg->n_exact, 8) || misaligned(dbg->device_error, 4)))
+    return fail(MUSE_ERR_INVALID_ARG, "debug outputs must be aligned to their element size");
   const AttnLayout need = layout(sh, pr, causal, Q, K, nullptr);
   if (!ws || ws_bytes < need.bytes) return fail(MUSE_ERR_WORKSPACE, "workspace too small");
   AttnLayout L = layout(sh, pr, causal, Q, K, ws);
@@ -249,7 +261,11 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   if (a.n_exact && causal)
     cudaMemsetAsync(a.n_exact, 0, (size_t)sh->B * sh->Hq * sh->N * 8, st);
   cudaMemsetAsync(L.err, 0, 4, st);
-  if (L.nq > 0 && L.V16) run_bf16_to_half(V, L.V16, (size_t)sh->B * sh->Hkv * sh->N * sh->D, st);
+  // rows of small causal levels (C_eff < Cq) are never selected into: -1
+  if (dbg && dbg->selected && causal && pr->topk > 0)
+    cudaMemsetAsync(L.s1.sel, 0xFF, (size_t)L.nq * pr->Cq * pr->topk * 4, st);
+  if (L.nq > 0 && L.V16)
+    run_bf16_to_half(V, L.V16, (size_t)sh->B * sh->Hkv * sh->N * sh->D, L.err, st);
   if (L.nq > 0) {
     cudaMemsetAsync(L.ks.arrive, 0, (size_t)L.ks.nprob * 4, st);
     cudaMemsetAsync(L.qs.arrive, 0, (size_t)L.qs.nprob * 4, st);
@@ -279,12 +295,14 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
     if (dbg->device_error) cudaMemcpyAsync(dbg->device_error, L.err, 4, cudaMemcpyDeviceToDevice, st);
     if (dbg->q_assign) cudaMemcpyAsync(dbg->q_assign, L.qs.assign, (size_t)L.qs.ntok * 4, cudaMemcpyDeviceToDevice, st);
     if (dbg->k_assign) cudaMemcpyAsync(dbg->k_assign, L.ks.assign, (size_t)L.ks.ntok * 4, cudaMemcpyDeviceToDevice, st);
+    // acausal [B,Hq,Cq,topk]; causal [B,Hq,P,Cq,topk] (the same table: one
+    // row block per query problem, problems numbered (b, q-head, pair))
+    if (dbg->selected && pr->topk > 0)
+      cudaMemcpyAsync(dbg->selected, L.s1.sel, (size_t)L.nq * pr->Cq * pr->topk * 4, cudaMemcpyDeviceToDevice, st);
     if (!causal) {
       if (dbg->k_counts) cudaMemcpyAsync(dbg->k_counts, L.ks.counts, (size_t)L.ks.nprob * pr->Ck * 4, cudaMemcpyDeviceToDevice, st);
       if (dbg->q_centroids) cudaMemcpyAsync(dbg->q_centroids, L.qs.cent32, (size_t)L.qs.nprob * pr->Cq * D * 4, cudaMemcpyDeviceToDevice, st);
       if (dbg->k_centroids) cudaMemcpyAsync(dbg->k_centroids, L.ks.cent32, (size_t)L.ks.nprob * pr->Ck * D * 4, cudaMemcpyDeviceToDevice, st);
-      if (dbg->selected && pr->topk > 0)
-        cudaMemcpyAsync(dbg->selected, L.s1.sel, (size_t)L.nq * pr->Cq * pr->topk * 4, cudaMemcpyDeviceToDevice, st);
     }
   }
   (void)elt;
@@ -317,9 +335,13 @@ size_t muse_cluster_workspace_size(int B, int H, int N, int D, int C) {
 
 muse_status muse_cluster(const void* X, muse_dtype dtype, int B, int H, int N, int D, int C,
                          int iters, uint64_t seed, int role, const float* init, int32_t* assign,
-                         float* centroids, int32_t* counts, void* ws, size_t ws_bytes,
-                         cudaStream_t stream) {
+                         float* centroids, int32_t* counts, int32_t* device_error, void* ws,
+                         size_t ws_bytes, cudaStream_t stream) {
   if (!X || !assign || !centroids) return fail(MUSE_ERR_INVALID_ARG, "X, assign and centroids must not be NULL");
+  if (misaligned(X, 16) || misaligned(init, 16) || misaligned(assign, 4) ||
+      misaligned(centroids, 4) || misaligned(counts, 4) || misaligned(device_error, 4))
+    return fail(MUSE_ERR_INVALID_ARG, "X and init must be 16-byte aligned, the outputs 4-byte");
+  if (misaligned(ws, 256)) return fail(MUSE_ERR_INVALID_ARG, "the workspace must be 256-byte aligned");
   if (B < 1 || H < 1 || N < 1) return fail(MUSE_ERR_INVALID_ARG, "B, H and N must be >= 1");
   if (D != 64 && D != 128) return fail(MUSE_ERR_UNSUPPORTED, "D must be 64 or 128");
   if (dtype != MUSE_BF16 && dtype != MUSE_F32) return fail(MUSE_ERR_INVALID_ARG, "bad dtype");
@@ -349,6 +371,7 @@ muse_status muse_cluster(const void* X, muse_dtype dtype, int B, int H, int N, i
   cudaMemcpyAsync(assign, ks.assign, (size_t)ks.ntok * 4, cudaMemcpyDeviceToDevice, stream);
   cudaMemcpyAsync(centroids, ks.cent32, (size_t)ks.nprob * C * D * 4, cudaMemcpyDeviceToDevice, stream);
   if (counts) cudaMemcpyAsync(counts, ks.counts, (size_t)ks.nprob * C * 4, cudaMemcpyDeviceToDevice, stream);
+  if (device_error) cudaMemcpyAsync(device_error, err, 4, cudaMemcpyDeviceToDevice, stream);
   return check_launch();
 }
 
@@ -364,6 +387,9 @@ muse_status muse_summarize(const void* K, const void* V, muse_dtype dtype, int B
   if (dtype != MUSE_BF16 && dtype != MUSE_F32) return fail(MUSE_ERR_INVALID_ARG, "bad dtype");
   if (C < 1) return fail(MUSE_ERR_INVALID_ARG, "C must be >= 1");
   if (C > 65535) return fail(MUSE_ERR_UNSUPPORTED, "C must be < 65536");
+  if (misaligned(K, 16) || misaligned(V, 16) || misaligned(assign, 4) || misaligned(counts, 4) ||
+      misaligned(mu, 16) || misaligned(S, 16) || misaligned(M, 16))
+    return fail(MUSE_ERR_INVALID_ARG, "K, V, mu, S and M must be 16-byte aligned, assign and counts 4-byte");
   run_summarize(K, V, dtype == MUSE_BF16 ? 0 : 1, B * H, N, D, C, assign, counts, mu, S, M,
                 nullptr, nullptr, stream);
   return check_launch();
@@ -381,6 +407,28 @@ muse_status muse_attn_fwd_causal(const void* Q, const void* K, const void* V, vo
                                  cudaStream_t stream) {
   return attn(Q, K, V, O, shape, params, debug, ws, ws_bytes, stream, true);
 }
+
+muse_status muse_device_status(const int32_t* device_error, cudaStream_t stream) {
+  if (!device_error) return fail(MUSE_ERR_INVALID_ARG, "device_error must not be NULL");
+  if (misaligned(device_error, 4)) return fail(MUSE_ERR_INVALID_ARG, "device_error must be 4-byte aligned");
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, device_error, 4, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_last_error = std::string("reading the device error word failed: ") + cudaGetErrorString(e);
+    return MUSE_ERR_CUDA;
+  }
+  if (v == 0) return MUSE_OK;
+  std::string msg = "device error word " + std::to_string(v) + ":";
+  if (v & MUSE_DEVERR_MMA_WAIT) msg += " a tensor-core completion wait gave up;";
+  if (v & MUSE_DEVERR_TEAM_BARRIER) msg += " a k-means team barrier gave up (outputs invalid);";
+  if (v & MUSE_DEVERR_V_RANGE) msg += " V holds a finite value outside the fp16 range (output invalid);";
+  g_last_error = msg;
+  return MUSE_ERR_DEVICE_CHECK;
+}
+
+void muse_debug_inject_barrier_fault(int rank, int spin_limit) { set_barrier_fault(rank, spin_limit); }
 
 const char* muse_status_string(muse_status s) {
   switch (s) {

@@ -13,7 +13,9 @@
 // GPU that loads the library holds it until the process exits.  In host code
 // the symbol's name is only a host-side stand-in, so its device address is
 // looked up once per device with cudaGetSymbolAddress (on the first call made
-// on that device, with that device current) and passed to the kernels.
+// on that device, with that device current) and passed to the kernels; the
+// address is kept for the life of the process, so it is stale after a
+// cudaDeviceReset() of that device.
 // Every call shares the array and it keeps the last call's contents; the
 // parts that must start at zero (tile arrival counters, the error word) are
 // cleared on the stream by each call.  Calls whose work overlaps on the GPU
@@ -48,7 +50,7 @@ size_t muse_cluster_static_capacity(void) { return kStaticScratchBytes; }
 muse_status muse_cluster_static(const void* X, muse_dtype dtype, int B, int H, int N, int D,
                                 int C, int iters, uint64_t seed, int role, const float* init,
                                 int32_t* assign, float* centroids, int32_t* counts,
-                                cudaStream_t stream) {
+                                int32_t* device_error, cudaStream_t stream) {
   const size_t need = muse_cluster_workspace_size(B, H, N, D, C);
   if (need > kStaticScratchBytes) {
     // rejected before touching the device; argument errors are left to muse_cluster
@@ -84,7 +86,7 @@ muse_status muse_cluster_static(const void* X, muse_dtype dtype, int B, int H, i
     ws = g_scratch_addr[dev];
   }
   return muse_cluster(X, dtype, B, H, N, D, C, iters, seed, role, init, assign, centroids, counts,
-                      ws, kStaticScratchBytes, stream);
+                      device_error, ws, kStaticScratchBytes, stream);
 }
 
 }  // extern "C"

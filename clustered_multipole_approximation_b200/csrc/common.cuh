@@ -18,6 +18,11 @@ constexpr int kMaxLevels = 24;
 constexpr int kTile = 128;  // tokens per assignment tile
 constexpr int kMaxC = 1024;
 
+// Bits of the device error word (the public MUSE_DEVERR_* values).
+constexpr int kErrMmaWait = 1;      // a tensor-core completion wait gave up
+constexpr int kErrTeamBarrier = 2;  // a k-means team barrier gave up
+constexpr int kErrVRange = 4;       // a finite bf16 value of V overflowed fp16
+
 struct Levels {
   int nlev;                 // number of levels (acausal: 1)
   int causal;

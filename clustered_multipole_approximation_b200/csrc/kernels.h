@@ -71,6 +71,9 @@ void run_kmeans_init(const RoleGeo* gs, const KState* kss, int nsets, const floa
 bool launch_kmeans_fused(const RoleGeo* gs, const KState* kss, int nsets, int iters,
                          cudaStream_t st);
 
+// Failure-path testing of the persistent k-means' team barrier.
+void set_barrier_fault(int rank, int spin_limit);
+
 // Lloyd rounds one launch sequence at a time (any dtype / size).
 void run_kmeans_rounds(const RoleGeo& g, const KState& ks, int iters, cudaStream_t st);
 
@@ -80,8 +83,9 @@ void launch_assign_tc(const RoleGeo& g, const KState& ks, cudaStream_t st);
 // Stage 1 + selection + stage 2 for query problems [qp0, qp0 + nqp).
 void run_blocks(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 
-// fp16 copy of a bf16 tensor (n elements, n % 8 == 0).
-void run_bf16_to_half(const void* src, __half* dst, size_t n, cudaStream_t st);
+// fp16 copy of a bf16 tensor (n elements, n % 8 == 0); a finite value that
+// overflows fp16 sets kErrVRange in *err.
+void run_bf16_to_half(const void* src, __half* dst, size_t n, int* err, cudaStream_t st);
 
 // Stage 2 on mma.sync tensor-core tiles (bf16 inputs).
 void run_stage2_mma(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);

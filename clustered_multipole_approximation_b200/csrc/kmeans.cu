@@ -339,12 +339,9 @@ __global__ void __launch_bounds__(256) kmeans_reduce_kernel(RoleGeo g, KState ks
 // ----------------------------------------------------------------------------
 template <typename T, int D>
 static void launch_round(const RoleGeo& g, const KState& ks, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)assign_smem<D>());
-    attr = true;
-  }
+  // set on every launch: the attribute is per device, and the call is cheap
+  cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)assign_smem<D>());
   {
     ProfScope ps(st, "kmeans_assign");
     if (sizeof(T) == 2)

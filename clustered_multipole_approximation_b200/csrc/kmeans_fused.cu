@@ -46,6 +46,11 @@ constexpr int kFT = 256;           // threads of the fused kernel
 constexpr int kWarps = kFT / 32;
 constexpr int kMaxNCT = 32;        // CTAs per problem
 constexpr int kSpinLimit = 1 << 24;  // team barrier polls (64 ns apart) before giving up
+
+// Failure-path testing: a CTA rank that skips its first barrier arrival and
+// the poll bound of the barrier waits (muse_debug_inject_barrier_fault).
+int g_fault_rank = -1;
+int g_spin_limit = kSpinLimit;
 constexpr int kOT = kNCF + kMaxNCT;  // (owned cluster, rank) pairs per CTA, at most
 constexpr int kTilesPerCta = 16;     // cluster launches: target tiles per CTA
 constexpr size_t kSmemLimit = 218 * 1024;  // dynamic shared memory (static arrays come on top)
@@ -216,6 +221,8 @@ struct FusedSets {
   KState ks[2];
   int nblk0;
   int lvl;
+  int fault_rank;  // cooperative launches: this CTA rank skips its first arrival
+  int spin_limit;  // polls of a barrier wait before it gives up
 };
 
 // Exclusive scan of n <= 2 * blockDim.x ints in shared memory, called by
@@ -313,25 +320,26 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   // team barrier (COOP): arrival counter of this problem, monotonic over the launch
   int* bar_ctr = ks.arrive + pid;
   int nbar = 0;
+  // A wait that gives up (a CTA of the problem never arrived) records
+  // kErrTeamBarrier and sets bar_fail; the caller then leaves the round loop
+  // at once, so no CTA reads lists or centroids that were never published.
   auto team_sync = [&]() {
     if (COOP) {
       __syncthreads();
       if (tid == 0) {
         ++nbar;
         __threadfence();
-        atomicAdd(bar_ctr, 1);
-        if (!bar_fail) {
-          for (int it = 0;; ++it) {
-            int v;
-            asm volatile("ld.acquire.gpu.global.s32 %0, [%1];\n" : "=r"(v) : "l"(bar_ctr) : "memory");
-            if (v >= nbar * NCT) break;
-            if (it >= kSpinLimit) {  // a CTA of the problem never arrived: give up, flag
-              bar_fail = 1;
-              atomicExch(ks.err, 1);
-              break;
-            }
-            __nanosleep(64);
+        if (!(nbar == 1 && rank == fs.fault_rank)) atomicAdd(bar_ctr, 1);
+        for (int it = 0;; ++it) {
+          int v;
+          asm volatile("ld.acquire.gpu.global.s32 %0, [%1];\n" : "=r"(v) : "l"(bar_ctr) : "memory");
+          if (v >= nbar * NCT) break;
+          if (it >= fs.spin_limit) {
+            bar_fail = 1;
+            atomicOr(ks.err, kErrTeamBarrier);
+            break;
           }
+          __nanosleep(64);
         }
         __threadfence();
       }
@@ -465,7 +473,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       const bool done = mbar_wait(saddr(&mbar[buf]), phase[buf]);
       phase[buf] ^= 1u;
       const bool ok = __syncthreads_and(done);
-      if (!ok && tid == 0) atomicExch(ks.err, 1);
+      if (!ok && tid == 0) atomicOr(ks.err, kErrMmaWait);
       if (ring == 2 && k + 2 < ntl) {  // tile k's slot is free once its MMA is done
         load_tile(tl_ + 2, tile_buf(k + 2));
         cp_commit();
@@ -630,6 +638,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         for (int t = tid; t < ntok; t += kFT) ks.assign[p.slot0 + tok0 + t] = asg[t];
     }
     team_sync();
+    if (bar_fail) break;
     // ---- owners: counts, offsets, means over all CTAs' members ----------------
     if (last) {
       for (int c = tid; c < C; c += kFT) goff[c] = 0;
@@ -793,6 +802,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
       }
     }
     team_sync();
+    if (bar_fail) break;
   }
   fence_before();
   __syncthreads();
@@ -912,6 +922,8 @@ static void launch_plan(const RoleGeo* gs, const KState* kss, int nsets, int lvl
     np[k] = lvl < 0 ? kss[k].nprob : gs[k].BH * gs[k].lv.npairs[lvl];
   }
   fs.lvl = lvl;
+  fs.fault_rank = plan.coop ? g_fault_rank : -1;
+  fs.spin_limit = g_spin_limit;
   fs.nblk0 = np[0] * plan.NCT;
   const int nblk = (np[0] + np[1]) * plan.NCT;
   cudaLaunchConfig_t cfg = {};
@@ -971,6 +983,11 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
     if (!plan_fused<D>(gs, kss, nsets, l, NC, plans[l])) return false;
   for (int l = 0; l < nlev; ++l) launch_plan<D>(gs, kss, nsets, l, iters, NC, tcols, plans[l], st);
   return true;
+}
+
+void set_barrier_fault(int rank, int spin_limit) {
+  g_fault_rank = rank;
+  g_spin_limit = rank >= 0 && spin_limit > 0 ? spin_limit : kSpinLimit;
 }
 
 bool launch_kmeans_fused(const RoleGeo* gs, const KState* kss, int nsets, int iters,

@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(kTile) kmeans_assign_tc_kernel(RoleGeo g, KSta
     const bool done = mbar_wait(mb, phase);
     if (!__syncthreads_and(done)) {
       ok = false;  // CTA-uniform: skip the TMEM reads, re-decide every token in fp64
-      if (tid == 0) atomicExch(ks.err, 1);
+      if (tid == 0) atomicOr(ks.err, kErrMmaWait);
     }
     phase ^= 1u;
     fence_after();
@@ -258,12 +258,9 @@ static void launch(const RoleGeo& g, const KState& ks, cudaStream_t st) {
   int tcols = 32;
   while (tcols < NC) tcols <<= 1;
   const size_t smem = assign_tc_smem(D, NC);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(kmeans_assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)assign_tc_smem(D, kNCMax));
-    attr = true;
-  }
+  // set on every launch: the attribute is per device, and the call is cheap
+  cudaFuncSetAttribute(kmeans_assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)assign_tc_smem(D, kNCMax));
   kmeans_assign_tc_kernel<D><<<(unsigned)ks.ntiles, kTile, smem, st>>>(g, ks, NC, tcols);
 }
 

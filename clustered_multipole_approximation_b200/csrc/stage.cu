@@ -633,16 +633,13 @@ __global__ void __launch_bounds__(kQ * (D / 64)) local_merge_kernel(AttnArgs a, 
 // ----------------------------------------------------------------------------
 template <typename T, int D>
 static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(stage1_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)stage1_smem<D>());
-    cudaFuncSetAttribute(select_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kSelectSmemMax);
-    cudaFuncSetAttribute(select_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         8 * kMaxC * (int)sizeof(double));
-    attr = true;
-  }
+  // set on every launch: the attribute is per device, and the call is cheap
+  cudaFuncSetAttribute(stage1_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)stage1_smem<D>());
+  cudaFuncSetAttribute(select_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)kSelectSmemMax);
+  cudaFuncSetAttribute(select_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       8 * kMaxC * (int)sizeof(double));
   {
     ProfScope ps(st, "stage1_summaries");
     if (sizeof(T) == 2 && a.mode == 1)

@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
     __syncthreads();  // the next pass overwrites the operands and G
     fence_after();
   }
-  if (!ok && tid == 0) atomicExch(a.qs.err, 1);
+  if (!ok && tid == 0) atomicOr(a.qs.err, kErrMmaWait);
   fence_before();
   __syncthreads();
   if (warp == 0)
@@ -320,12 +320,9 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
 
 template <int D>
 static void launch_s1tc(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(stage1_dipole_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         S1Layout<D>::TOTAL);
-    attr = true;
-  }
+  // set on every launch: the attribute is per device, and the call is cheap
+  cudaFuncSetAttribute(stage1_dipole_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       S1Layout<D>::TOTAL);
   stage1_dipole_tc_kernel<D><<<dim3(nqp, a.Ck), kS1T, S1Layout<D>::TOTAL, st>>>(a, s1, qp0);
 }
 

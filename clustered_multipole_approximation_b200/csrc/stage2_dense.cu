@@ -294,12 +294,9 @@ __global__ void __launch_bounds__(kDThreads, D == 64 ? 2 : 1)
 template <int D>
 static void launch_dense(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, int smax,
                          cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(stage2_dense_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)sizeof(DenseSmem<D>));
-    attr = true;
-  }
+  // set on every launch: the attribute is per device, and the call is cheap
+  cudaFuncSetAttribute(stage2_dense_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)sizeof(DenseSmem<D>));
   const dim3 grid(nqp, smax / kDQ);
   stage2_dense_kernel<D><<<grid, kDThreads, sizeof(DenseSmem<D>), st>>>(a, s1, qp0);
 }

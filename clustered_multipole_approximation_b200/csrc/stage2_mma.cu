@@ -59,8 +59,11 @@ size_t stage2_mma_smem() {
   return sizeof(Smem2<D>);
 }
 
+// fp16 copy of bf16 V (the PV operand).  A finite value that overflows fp16
+// (|v| >= 65520) is flagged in the device error word.
 __global__ void bf16_to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
-                                    size_t n8) {
+                                    size_t n8, int* err) {
+  bool over = false;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
        i += (size_t)gridDim.x * blockDim.x) {
     const uint4 v = reinterpret_cast<const uint4*>(src)[i];
@@ -68,16 +71,24 @@ __global__ void bf16_to_half_kernel(const __nv_bfloat16* __restrict__ src, __hal
     uint4 o;
     __half2* h = reinterpret_cast<__half2*>(&o);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) h[u] = __float22half2_rn(__bfloat1622float2(b[u]));
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(b[u]);
+      h[u] = __float22half2_rn(f);
+      // finite and |v| >= 65520 (the fp16 overflow threshold)
+      over |= fabsf(f.x) >= 65520.f && fabsf(f.x) < INFINITY;
+      over |= fabsf(f.y) >= 65520.f && fabsf(f.y) < INFINITY;
+    }
     reinterpret_cast<uint4*>(dst)[i] = o;
   }
+  if (over) atomicOr(err, kErrVRange);
 }
 
-void run_bf16_to_half(const void* src, __half* dst, size_t n, cudaStream_t st) {
+void run_bf16_to_half(const void* src, __half* dst, size_t n, int* err, cudaStream_t st) {
   ProfScope ps(st, "v_to_half");
   const size_t n8 = n / 8;
   const int blocks = (int)((n8 + 255) / 256 < 148 * 8 ? (n8 + 255) / 256 : 148 * 8);
-  bf16_to_half_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), dst, n8);
+  bf16_to_half_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), dst, n8,
+                                              err);
 }
 
 template <typename TO, int D>
@@ -579,14 +590,11 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) local_mma_kernel(At
 
 template <int D>
 static void launch_local(const AttnArgs& a, int L, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(local_mma_kernel<float, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)sizeof(LocSmem<D>));
-    cudaFuncSetAttribute(local_mma_kernel<__nv_bfloat16, D>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(LocSmem<D>));
-    attr = true;
-  }
+  // set on every launch: the attribute is per device, and the call is cheap
+  cudaFuncSetAttribute(local_mma_kernel<float, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)sizeof(LocSmem<D>));
+  cudaFuncSetAttribute(local_mma_kernel<__nv_bfloat16, D>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(LocSmem<D>));
   dim3 grid(a.qg.BH, cdiv(a.qg.lv.N, kMQ));
   if (a.out_f32)
     local_mma_kernel<float, D><<<grid, kThreads, sizeof(LocSmem<D>), st>>>(a, L);
@@ -605,14 +613,11 @@ bool run_local_mma(const AttnArgs& a, int L, cudaStream_t st) {
 
 template <int D>
 static void launch_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(stage2_mma_kernel<float, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)stage2_mma_smem<D>());
-    cudaFuncSetAttribute(stage2_mma_kernel<__nv_bfloat16, D>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)stage2_mma_smem<D>());
-    attr = true;
-  }
+  // set on every launch: the attribute is per device, and the call is cheap
+  cudaFuncSetAttribute(stage2_mma_kernel<float, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)stage2_mma_smem<D>());
+  cudaFuncSetAttribute(stage2_mma_kernel<__nv_bfloat16, D>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)stage2_mma_smem<D>());
   dim3 grid(nqp, a.Cq);
   if (a.out_f32)
     stage2_mma_kernel<float, D><<<grid, kThreads, stage2_mma_smem<D>(), st>>>(a, s1, qp0);

@@ -25,6 +25,17 @@
  *     leaves every output untouched.  A launch error reported by the CUDA
  *     runtime returns MUSE_ERR_CUDA.  muse_last_error() then gives a message
  *     (per host thread).
+ *   - Alignment: every tensor pointer (Q, K, V, O, X, init, the summary
+ *     outputs) must be 16-byte aligned, the workspace 256-byte aligned, and
+ *     the optional int32 / int64 debug outputs aligned to their element
+ *     size; a misaligned pointer returns MUSE_ERR_INVALID_ARG before any
+ *     launch.
+ *   - Device-side status: a few conditions can only be seen on the GPU (a
+ *     bounded wait that gave up, a value the kernels cannot represent).  The
+ *     kernels then record a non-zero MUSE_DEVERR_* bit set in a device error
+ *     word instead of faulting; entry points that take a `device_error`
+ *     pointer copy that word there on the stream, and muse_device_status()
+ *     turns it into MUSE_OK or MUSE_ERR_DEVICE_CHECK.
  *   - Calls with distinct workspaces and outputs may run concurrently.
  */
 #ifndef MUSE_H_
@@ -47,6 +58,21 @@ typedef enum {
   MUSE_ERR_CUDA = 4,
   MUSE_ERR_DEVICE_CHECK = 5
 } muse_status;
+
+/* Bits of the device error word (0 = every kernel finished normally). */
+enum {
+  /* A wait for tensor-core (tcgen05) completion gave up after its bound.  The
+   * k-means re-decides the affected tokens on its fp64 path; other kernels'
+   * outputs are unreliable. */
+  MUSE_DEVERR_MMA_WAIT = 1,
+  /* A barrier between the CTAs of one k-means problem (cooperative launch)
+   * gave up after its bound, because a CTA never arrived; every CTA of the
+   * problem then stops, and the clustering outputs are invalid. */
+  MUSE_DEVERR_TEAM_BARRIER = 2,
+  /* A finite bf16 value of V lies outside the fp16 range (|v| >= 65520), so
+   * its fp16 tensor-core operand became infinite; the output is invalid. */
+  MUSE_DEVERR_V_RANGE = 4
+};
 
 typedef enum { MUSE_BF16 = 0, MUSE_F32 = 1 } muse_dtype;
 
@@ -81,15 +107,15 @@ typedef struct {
  *   selected [B,Hq,Cq,topk] (rank order, -1 padded), n_exact [B,Hq,N].
  * Causal layouts: q_assign [B,Hq,levels,N/2], k_assign [B,Hkv,levels,N/2]
  *   (entry (l, p*s + r) is token r of pair p's block at level l, s = L 2^l),
- *   n_exact [B,Hq,N]; the centroid, count and selection members are not
- *   written by the causal entry point. */
+ *   selected [B,Hq,P,Cq,topk] with P = N/L - 1 block problems per head,
+ *   numbered level by level (level l's pairs start at sum_{l'<l} N/(2 s_l')),
+ *   rows i >= min(Cq, s) are -1; n_exact [B,Hq,N]; the centroid and count
+ *   members are not written by the causal entry point. */
 typedef struct {
   int32_t *q_assign, *k_assign, *selected, *k_counts;
   float *q_centroids, *k_centroids;
   int64_t *n_exact;
-  int32_t *device_error; /* 0, or non-zero if a kernel's bounded wait on the
-                            tensor cores gave up (its tokens were then
-                            re-decided on the fp64 path) */
+  int32_t *device_error; /* the device error word: 0 or MUSE_DEVERR_* bits */
 } muse_debug;
 
 /* Workspace bytes muse_attn_fwd (causal == 0) or muse_attn_fwd_causal
@@ -97,6 +123,13 @@ typedef struct {
  * arguments are invalid. */
 size_t muse_workspace_size(const muse_shape *shape, const muse_params *params,
                            int causal);
+
+/* Waits for `stream`, reads a device error word written by an entry point
+ * (`device_error`, a device pointer to one int32) and returns MUSE_OK if it
+ * is 0, else MUSE_ERR_DEVICE_CHECK with a message naming the MUSE_DEVERR_*
+ * bits (MUSE_ERR_CUDA if the stream or the copy fails).  The one call of
+ * the library that synchronises. */
+muse_status muse_device_status(const int32_t *device_error, cudaStream_t stream);
 
 /* Workspace bytes of muse_cluster / muse_summarize for these sizes. */
 size_t muse_cluster_workspace_size(int B, int H, int N, int D, int C);
@@ -119,13 +152,14 @@ size_t muse_cluster_workspace_size(int B, int H, int N, int D, int C);
  *   assign       out [B,H,N] int32: cluster of each row after the last round.
  *   centroids    out [B,H,C,D] fp32: centroids after the last update.
  *   counts       out [B,H,C] int32 (may be NULL).
+ *   device_error out, one int32 (may be NULL): the device error word.
  * 1 <= C <= min(N, 1024); D in {64, 128}.
  */
 muse_status muse_cluster(const void *X, muse_dtype dtype, int B, int H, int N,
                          int D, int C, int iters, uint64_t seed, int role,
                          const float *init, int32_t *assign, float *centroids,
-                         int32_t *counts, void *ws, size_t ws_bytes,
-                         cudaStream_t stream);
+                         int32_t *counts, int32_t *device_error, void *ws,
+                         size_t ws_bytes, cudaStream_t stream);
 
 /*
  * Key-cluster summaries for a given assignment ([A1] Abstract: monopole and
@@ -189,17 +223,19 @@ muse_status muse_attn_fwd_causal(const void *Q, const void *K, const void *V,
  * muse_cluster_workspace_size() exceeds it return MUSE_ERR_WORKSPACE with a
  * message and launch nothing.  The first call on each device looks up the
  * array's device address (cudaGetSymbolAddress, with that device current):
- * make that first call before any stream capture.  All calls share the one
- * array and it keeps the last call's contents -- the parts that must start at
- * zero are cleared by each call -- so calls whose work overlaps on the GPU
- * (other streams, other host threads) race.  Arguments and outputs are those
- * of muse_cluster.
+ * make that first call before any stream capture.  The looked-up address is
+ * kept for the life of the process: after cudaDeviceReset() on a device the
+ * kept address is stale, so do not call this entry point on that device
+ * again in the same process.  All calls share the one array and it keeps the
+ * last call's contents -- the parts that must start at zero are cleared by
+ * each call -- so calls whose work overlaps on the GPU (other streams, other
+ * host threads) race.  Arguments and outputs are those of muse_cluster.
  */
 muse_status muse_cluster_static(const void *X, muse_dtype dtype, int B, int H,
                                 int N, int D, int C, int iters, uint64_t seed,
                                 int role, const float *init, int32_t *assign,
                                 float *centroids, int32_t *counts,
-                                cudaStream_t stream);
+                                int32_t *device_error, cudaStream_t stream);
 
 /* Bytes of the scratch array built into the library for muse_cluster_static. */
 size_t muse_cluster_static_capacity(void);
@@ -216,6 +252,14 @@ const char *muse_status_string(muse_status status);
 void muse_profile_enable(int on);
 int muse_profile_read(char *names, int name_stride, int *launches, double *ms,
                       int cap);
+
+/* Failure-path testing (no paper counterpart).  While rank >= 0, every
+ * cooperative launch of the persistent k-means in this process lets CTA
+ * `rank` of each problem skip its arrival at the first barrier, and every
+ * barrier wait gives up after `spin_limit` polls (about 64 ns apart): the
+ * kernel then records MUSE_DEVERR_TEAM_BARRIER and returns without touching
+ * its outputs.  rank < 0 restores normal operation.  Not thread-safe. */
+void muse_debug_inject_barrier_fault(int rank, int spin_limit);
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char *muse_last_error(void);

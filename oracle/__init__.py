@@ -62,9 +62,11 @@ def _bind(lib):
         _dp, _ip, _ip, _dp, _dp, _ip, _ip, _llp]
     lib.orc_muse_causal.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 8 + [
         ctypes.c_uint64, ctypes.c_int, ctypes.c_double, ctypes.c_int, _u8p, _ip, _ip,
-        _dp, _ip, _ip, _llp]
+        _dp, _ip, _ip, _ip, _llp]
     lib.orc_exact_attn.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 5 + [
         ctypes.c_double, ctypes.c_int, _u8p, _dp]
+    lib.orc_exact_attn_rows.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 5 + [
+        ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, _ip, _dp]
     lib.orc_stage1_debug.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 4 + [
         _ip, _ip, ctypes.c_int, ctypes.c_double, ctypes.c_int, _dp, _dp, _ip]
     lib.orc_num_threads.restype = ctypes.c_int
@@ -211,11 +213,18 @@ class Oracle:
         q_assign = np.zeros((B, Hq, lv, N // 2), dtype=np.int32)
         k_assign = np.zeros((B, Hkv, lv, N // 2), dtype=np.int32)
         n_exact = np.zeros((B, Hq, N), dtype=np.int64)
+        nprob = max(N // L - 1, 1)
+        selected = np.full((B, Hq, nprob, C, max(topk, 1)), -1, dtype=np.int32)
         self.lib.orc_muse_causal(
             qp, kp, vp, B, Hq, Hkv, N, D, L, C, iters, seed, topk, float(scale), MODES[mode],
             m_p, qa_p, ka_p, O.ctypes.data_as(_dp), q_assign.ctypes.data_as(_ip),
-            k_assign.ctypes.data_as(_ip), n_exact.ctypes.data_as(_llp))
-        return dict(O=O, q_assign=q_assign, k_assign=k_assign, n_exact=n_exact)
+            k_assign.ctypes.data_as(_ip),
+            selected.ctypes.data_as(_ip) if topk > 0 and N // L > 1 else None,
+            n_exact.ctypes.data_as(_llp))
+        out = dict(O=O, q_assign=q_assign, k_assign=k_assign, n_exact=n_exact)
+        if topk > 0 and N // L > 1:
+            out["selected"] = selected[..., :topk]
+        return out
 
     def exact_attention(self, Q, K, V, scale=1.0, causal=False, hq_mask=None):
         """Plain softmax attention in fp64 (GQA by kv-head = q-head / group)."""
@@ -227,6 +236,20 @@ class Oracle:
         E = np.zeros_like(Q)
         self.lib.orc_exact_attn(qp, kp, vp, B, Hq, K.shape[1], N, D, float(scale), int(causal), m_p,
                                E.ctypes.data_as(_dp))
+        return E
+
+    def exact_attention_rows(self, Q, K, V, b, hq, rows, scale=1.0, causal=False):
+        """Exact attention of the given query rows of (b, q-head hq) only:
+        [len(rows), D] (the same arithmetic as exact_attention, row by row)."""
+        Q, qp = _d(Q)
+        K, kp = _d(K)
+        V, vp = _d(V)
+        B, Hq, N, D = Q.shape
+        rows, rp = _i(rows)
+        E = np.zeros((len(rows), D))
+        self.lib.orc_exact_attn_rows(qp, kp, vp, B, Hq, K.shape[1], N, D, float(scale),
+                                     int(causal), b * Hq + hq, len(rows), rp,
+                                     E.ctypes.data_as(_dp))
         return E
 
     def stage1_debug(self, Qh, Kh, Vh, Cq, Ck, q_assign, k_assign, topk, scale=1.0, mode="dipole"):

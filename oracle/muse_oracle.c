@@ -517,6 +517,8 @@ void orc_muse_acausal(const double *Q, const double *K, const double *V, int B,
 /* levels tile [0, bL) exactly once.  All terms meet in one softmax.          */
 /* Debug layouts (optional): q_assign [B,Hq,Lv,N/2], k_assign [B,Hkv,Lv,N/2]  */
 /* where entry (l, p s + r) is token r of pair p's block at level l;          */
+/* selected [B,Hq,P,C,k1] with P = N/L - 1 block problems numbered level by   */
+/* level (rows i >= C_eff left as the caller filled them);                    */
 /* n_exact [B,Hq,N] counts exact keys per query including the local block.    */
 /* ------------------------------------------------------------------------ */
 void orc_muse_causal(const double *Q, const double *K, const double *V, int B,
@@ -524,7 +526,7 @@ void orc_muse_causal(const double *Q, const double *K, const double *V, int B,
                      uint64_t seed, int k1, double scale, int mode,
                      const unsigned char *hq_mask, const int *q_assign_in,
                      const int *k_assign_in, double *O, int *q_assign,
-                     int *k_assign, long long *n_exact) {
+                     int *k_assign, int *selected, long long *n_exact) {
   const int G = Hq / Hkv;
   const int nblk = N / L;
   int levels = 0;
@@ -544,6 +546,7 @@ void orc_muse_causal(const double *Q, const double *K, const double *V, int B,
     double *acc = (double *)calloc((size_t)G * N * D, sizeof(double));
     long long *ne = (long long *)calloc((size_t)G * N, sizeof(long long));
     for (size_t i = 0; i < (size_t)G * N; ++i) m[i] = -INFINITY;
+    int pbase = 0; /* block problems of the levels below lv */
     for (int lv = 0; lv < levels; ++lv) {
       int s = L << lv;
       int npairs = N / (2 * s);
@@ -570,11 +573,16 @@ void orc_muse_causal(const double *Q, const double *K, const double *V, int B,
           if (q_assign)
             memcpy(q_assign + (size_t)bq * levels * half + slot, qb.assign, sizeof(int) * (size_t)s);
           size_t o = (size_t)g * N + q0;
-          run_block(&qb, &kb, scale, mode, k1, m + o, l + o, acc + o * D, ne + o, NULL);
+          block_debug dbg = {selected ? selected + ((size_t)bq * (nblk - 1) + pbase + p) *
+                                                       (size_t)C * (k1 > 0 ? k1 : 1)
+                                      : NULL,
+                             NULL, NULL};
+          run_block(&qb, &kb, scale, mode, k1, m + o, l + o, acc + o * D, ne + o, &dbg);
           free_queries(&qb);
         }
         free_keys(&kb);
       }
+      pbase += npairs;
     }
     /* exact local block: keys t with floor(t/L) == floor(q/L) and t <= q */
     for (int g = 0; g < G; ++g) {
@@ -602,6 +610,24 @@ void orc_muse_causal(const double *Q, const double *K, const double *V, int B,
 /* Exact softmax attention (the quantity MuSe approximates; [G] "Problem      */
 /* Statement").  causal != 0 masks keys t > q.                                */
 /* ------------------------------------------------------------------------ */
+/* One query row: softmax over keys [0, tend) of Kh with values Vh. */
+static void exact_row(const double *q, const double *Kh, const double *Vh,
+                      int tend, int D, double scale, double *lg, double *e) {
+  double mx = -INFINITY;
+  for (int t = 0; t < tend; ++t) {
+    lg[t] = scale * dot(q, Kh + (size_t)t * D, D);
+    if (lg[t] > mx) mx = lg[t];
+  }
+  double z = 0.0;
+  for (int d = 0; d < D; ++d) e[d] = 0.0;
+  for (int t = 0; t < tend; ++t) {
+    double w = exp(lg[t] - mx);
+    z += w;
+    for (int d = 0; d < D; ++d) e[d] += w * Vh[(size_t)t * D + d];
+  }
+  for (int d = 0; d < D; ++d) e[d] /= z;
+}
+
 void orc_exact_attn(const double *Q, const double *K, const double *V, int B,
                     int Hq, int Hkv, int N, int D, double scale, int causal,
                     const unsigned char *hq_mask, double *E) {
@@ -613,22 +639,31 @@ void orc_exact_attn(const double *Q, const double *K, const double *V, int B,
     const double *Qh = Q + (size_t)bq * N * D;
     const double *Kh = K + (size_t)bk * N * D, *Vh = V + (size_t)bk * N * D;
     double *lg = (double *)malloc(sizeof(double) * (size_t)N);
-    for (int q = 0; q < N; ++q) {
-      int tend = causal ? q + 1 : N;
-      double mx = -INFINITY;
-      for (int t = 0; t < tend; ++t) {
-        lg[t] = scale * dot(Qh + (size_t)q * D, Kh + (size_t)t * D, D);
-        if (lg[t] > mx) mx = lg[t];
-      }
-      double z = 0.0;
-      double *e = E + ((size_t)bq * N + q) * D;
-      for (int d = 0; d < D; ++d) e[d] = 0.0;
-      for (int t = 0; t < tend; ++t) {
-        double w = exp(lg[t] - mx);
-        z += w;
-        for (int d = 0; d < D; ++d) e[d] += w * Vh[(size_t)t * D + d];
-      }
-      for (int d = 0; d < D; ++d) e[d] /= z;
+    for (int q = 0; q < N; ++q)
+      exact_row(Qh + (size_t)q * D, Kh, Vh, causal ? q + 1 : N, D, scale, lg,
+                E + ((size_t)bq * N + q) * D);
+    free(lg);
+  }
+}
+
+/* The same for selected query rows of one (b, q-head) bq: E [nrows][D]. */
+void orc_exact_attn_rows(const double *Q, const double *K, const double *V,
+                         int B, int Hq, int Hkv, int N, int D, double scale,
+                         int causal, int bq, int nrows, const int *rows,
+                         double *E) {
+  const int G = Hq / Hkv;
+  int b = bq / Hq, hq = bq % Hq, bk = b * Hkv + hq / G;
+  (void)B;
+  const double *Qh = Q + (size_t)bq * N * D;
+  const double *Kh = K + (size_t)bk * N * D, *Vh = V + (size_t)bk * N * D;
+#pragma omp parallel
+  {
+    double *lg = (double *)malloc(sizeof(double) * (size_t)N);
+#pragma omp for schedule(dynamic)
+    for (int i = 0; i < nrows; ++i) {
+      int q = rows[i];
+      exact_row(Qh + (size_t)q * D, Kh, Vh, causal ? q + 1 : N, D, scale, lg,
+                E + (size_t)i * D);
     }
     free(lg);
   }

@@ -77,10 +77,10 @@ def test_invalid_arguments_return_errors_without_launch(lib):
     st = lib.muse_attn_fwd_causal(fake, fake, fake, fake, ctypes.byref(sh),
                                   ctypes.byref(params(block=100)), None, fake, 1 << 30, None)
     assert st == 1
-    st = lib.muse_cluster(fake, 0, 1, 1, 100, 64, 200, 3, 0, 0, None, fake, fake, None, fake,
-                          1 << 30, None)
+    st = lib.muse_cluster(fake, 0, 1, 1, 100, 64, 200, 3, 0, 0, None, fake, fake, None, None,
+                          fake, 1 << 30, None)
     assert st == 1
-    st = lib.muse_cluster(fake, 0, 1, 1, 100, 64, 10, 3, 0, 2, None, fake, fake, None, fake,
+    st = lib.muse_cluster(fake, 0, 1, 1, 100, 64, 10, 3, 0, 2, None, fake, fake, None, None, fake,
                           1 << 30, None)
     assert st == 1
     st = lib.muse_summarize(fake, fake, 0, 1, 1, 100, 48, 10, fake, fake, fake, fake, None, None,
@@ -92,3 +92,33 @@ def test_invalid_arguments_return_errors_without_launch(lib):
 def test_product_path_fails_loudly_without_library(tmp_path):
     with pytest.raises(ImportError):
         muse.load_library(str(tmp_path / "missing.so"))
+
+
+def test_misaligned_pointers_are_rejected_without_launch(lib):
+    """Kernels load 16-byte vectors and carve the workspace in 256-byte
+    pieces: misaligned pointers must come back as MUSE_ERR_INVALID_ARG."""
+    ok = ctypes.c_void_p(0x10000)    # never dereferenced: validation fails first
+    odd = ctypes.c_void_p(0x10008)   # 8-byte aligned only
+    ws_odd = ctypes.c_void_p(0x10080)  # 128-byte aligned only
+    sh, pr = shape(), params()
+    for args in [(odd, ok, ok, ok, ok), (ok, odd, ok, ok, ok), (ok, ok, odd, ok, ok),
+                 (ok, ok, ok, odd, ok), (ok, ok, ok, ok, ws_odd)]:
+        q, k, v, o, ws = args
+        for f in (lib.muse_attn_fwd, lib.muse_attn_fwd_causal):
+            p = params(block=128) if f is lib.muse_attn_fwd_causal else pr
+            st = f(q, k, v, o, ctypes.byref(sh), ctypes.byref(p), None, ws, 1 << 40, None)
+            assert st == 1 and b"aligned" in lib.muse_last_error(), (args, st)
+    dbg = muse.muse_debug(None, None, None, None, None, None, ctypes.c_void_p(0x10004), None)
+    st = lib.muse_attn_fwd(ok, ok, ok, ok, ctypes.byref(sh), ctypes.byref(pr), ctypes.byref(dbg),
+                           ok, 1 << 40, None)
+    assert st == 1 and b"aligned" in lib.muse_last_error()
+    st = lib.muse_cluster(odd, 0, 1, 1, 100, 64, 10, 3, 0, 0, None, ok, ok, None, None, ok,
+                          1 << 30, None)
+    assert st == 1 and b"aligned" in lib.muse_last_error()
+    st = lib.muse_cluster(ok, 0, 1, 1, 100, 64, 10, 3, 0, 0, None, ok, ok, None, None, ws_odd,
+                          1 << 30, None)
+    assert st == 1 and b"aligned" in lib.muse_last_error()
+    st = lib.muse_summarize(odd, ok, 0, 1, 1, 100, 64, 10, ok, ok, ok, ok, None, None, 0, None)
+    assert st == 1 and b"aligned" in lib.muse_last_error()
+    st = lib.muse_device_status(None, None)
+    assert st == 1

@@ -6,6 +6,9 @@ outputs must match within 1e-5 (fp32 inputs) or 2e-3 (bf16 inputs) max-abs,
 and the relative squared error against exact attention within 1e-3 of the
 oracle's.
 """
+import concurrent.futures
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -84,10 +87,10 @@ def test_workload_acausal_f32_n1k():
 
 @pytest.mark.parametrize("mode", ["dipole", "monopole"])
 def test_workload_acausal_bf16_h8_n8k(mode):
+    """The 8-head 8k layer, every head against the oracle."""
     w = WORKLOADS["acausal-bf16-h8-n8k"]
     Q, K, V = make_inputs(w)
-    check_acausal(Q, K, V, w.dtype, w.C, w.iters, w.cluster_seed, w.topk, w.scale, mode,
-                  heads=[(0, 0), (0, 5)])
+    check_acausal(Q, K, V, w.dtype, w.C, w.iters, w.cluster_seed, w.topk, w.scale, mode)
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -179,20 +182,111 @@ def test_muse_cluster_one_round_from_given_centroids():
         np.testing.assert_allclose(c[0, h].cpu().numpy(), rc, rtol=2e-7, atol=1e-7)
 
 
-def test_muse_summarize():
-    K, _, V = clustered_qkv(1, 2, 2, 600, 64, 6, 0.3, 0.0, "f32", 42)
+@pytest.mark.parametrize("dtype,D", [("f32", 64), ("bf16", 64), ("bf16", 128)])
+def test_muse_summarize(dtype, D):
+    """Counts, centroids, monopole sums S and dipole moments M of a given
+    assignment against the oracle (bf16 inputs are exact in the oracle's
+    fp64; the GPU accumulates S and M in fp32)."""
+    K, _, V = clustered_qkv(1, 2, 2, 600, D, 6, 0.3, 0.0, dtype, 42 + D)
     rng = np.random.default_rng(3)
     assign = rng.integers(0, 7, (1, 2, 600)).astype(np.int32)
     assign[0, 1][assign[0, 1] == 3] = 4  # cluster 3 empty in head 1
-    cnt, mu, S, M = muse.muse_summarize(to_dev(K, "f32"), to_dev(V, "f32"),
+    cnt, mu, S, M = muse.muse_summarize(to_dev(K, dtype), to_dev(V, dtype),
                                         torch.from_numpy(assign).cuda(), 7)
+    torch.cuda.synchronize()
     for h in range(2):
-        rmu, rn = oracle.kmeans_update(K[0, h], assign[0, h], np.zeros((7, 64)))
+        rmu, rn = oracle.kmeans_update(K[0, h], assign[0, h], np.zeros((7, D)))
         rS, rM = oracle.summaries(K[0, h], V[0, h], 7, assign[0, h], rmu)
         assert (cnt[0, h].cpu().numpy() == rn).all()
         np.testing.assert_allclose(mu[0, h].cpu().numpy(), rmu, rtol=1e-6, atol=1e-6)
         np.testing.assert_allclose(S[0, h].cpu().numpy(), rS, rtol=1e-5, atol=1e-4)
         np.testing.assert_allclose(M[0, h].cpu().numpy(), rM, rtol=1e-4, atol=1e-4)
+    assert (cnt[0, 1, 3] == 0).item() and (mu[0, 1, 3] == 0).all().item()
+
+
+def _golden_init_cases():
+    path = os.path.join(os.path.dirname(__file__), "golden", "init_indices.txt")
+    cases = []
+    for ln in open(path):
+        if ln.startswith("#") or not ln.strip():
+            continue
+        head, idx = ln.split(":")
+        n, C, seed, sid, role = map(int, head.split())
+        cases.append((n, C, seed, sid, role, np.array(idx.split(), dtype=np.int64)))
+    return cases
+
+
+@pytest.mark.parametrize("case", range(7))
+def test_gpu_seeded_start_rows_match_golden(case):
+    """The GPU's seeded start rows are the stored ones: one Lloyd round from
+    them (assignment to those rows, then the means) is what muse_cluster
+    computes with iters = 1 for the stream (b = 0, h = sid) and role."""
+    n, C, seed, sid, role, idx = _golden_init_cases()[case]
+    X, _, _ = clustered_qkv(1, sid + 1, sid + 1, n, 64, 8, 0.3, 0.0, "bf16", 90 + case)
+    a, c, cnt = muse.muse_cluster(to_dev(X, "bf16"), C, 1, seed, role=role)
+    torch.cuda.synchronize()
+    Xh = X[0, sid].astype(np.float64)
+    start = Xh[idx]
+    ra, _ = oracle.kmeans_assign(Xh, start)
+    rc, rn = oracle.kmeans_update(Xh, ra, start)
+    assert_assign_match(a[0, sid].cpu().numpy(), ra, what="round-1 assignment")
+    assert (cnt[0, sid].cpu().numpy() == rn).all()
+    np.testing.assert_allclose(c[0, sid].cpu().numpy(), rc, rtol=2e-7, atol=1e-7)
+
+
+def test_v_outside_unit_range_large_and_tiny():
+    """V far from N(0, 1): large values (up to 3e4, still inside fp16) and tiny
+    ones (down to 1e-7, below fp16's normal range).  The output is linear in
+    V, so the bf16 tolerance scales with max |v|."""
+    Q, K, V = clustered_qkv(1, 2, 1, 1024, 64, 8, 0.3, 0.0, "bf16", 70)
+    rng = np.random.default_rng(5)
+    scale = np.where(rng.random(V.shape) < 0.5, 3e4 / 4, 1e-7).astype(np.float32)
+    V = (V * scale).astype(np.float32)
+    big = float(np.abs(V).max())
+    q, k, v = to_dev(Q, "bf16"), to_dev(K, "bf16"), to_dev(V, "bf16")
+    Vb = v.float().cpu().numpy()
+    O, dbg = muse.muse_attn_fwd(q, k, v, Cq=16, Ck=16, iters=4, seed=3, topk=2, debug=True,
+                                out_dtype=torch.float32)
+    muse.device_status(dbg["device_error"])
+    r = oracle.muse_acausal(Q, K, Vb, 16, 16, 4, 3, 2)
+    assert_close(O.cpu().numpy(), r["O"], TOL["bf16"] * big / 4.0, "O with large / tiny V")
+
+
+def test_v_beyond_fp16_is_reported():
+    """A finite bf16 value of V beyond fp16's range cannot enter the fp16
+    PV operand: the call still returns MUSE_OK (nothing is synchronised), and
+    the device error word reports MUSE_DEVERR_V_RANGE."""
+    Q, K, V = clustered_qkv(1, 1, 1, 512, 64, 8, 0.3, 0.0, "bf16", 71)
+    V[0, 0, 7, 3] = 1.0e5
+    q, k, v = to_dev(Q, "bf16"), to_dev(K, "bf16"), to_dev(V, "bf16")
+    _, dbg = muse.muse_attn_fwd(q, k, v, Cq=8, Ck=8, iters=2, seed=1, topk=1, debug=True)
+    with pytest.raises(muse.MuseError) as e:
+        muse.device_status(dbg["device_error"])
+    assert e.value.status == 5 and "fp16" in str(e.value)
+    assert int(dbg["device_error"].item()) == 4
+
+
+def test_team_barrier_that_runs_out_is_reported_and_context_survives():
+    """Failure path of the persistent k-means' cooperative barrier: one CTA
+    per problem skips its first arrival (test hook), every wait gives up after
+    a few thousand polls, the kernel records MUSE_DEVERR_TEAM_BARRIER and
+    returns; the next call, without the hook, is correct."""
+    X, _, _ = clustered_qkv(1, 4, 4, 4096, 64, 16, 0.3, 0.0, "bf16", 72)
+    x = to_dev(X, "bf16")
+    err = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    muse.inject_barrier_fault(1, 4096)
+    try:
+        muse.muse_cluster(x, 64, 3, 5, role=0, device_error=err)
+        with pytest.raises(muse.MuseError) as e:
+            muse.device_status(err)
+    finally:
+        muse.inject_barrier_fault(-1)
+    assert e.value.status == 5 and int(err.item()) & 2
+    a, c, n = muse.muse_cluster(x, 64, 3, 5, role=0, device_error=err)
+    muse.device_status(err)
+    ra, rc, rn, _ = oracle.kmeans(X[0, 2], 64, 3, 5, 2, 0)
+    assert_assign_match(a[0, 2].cpu().numpy(), ra)
+    np.testing.assert_allclose(c[0, 2].cpu().numpy(), rc, rtol=2e-7, atol=1e-7)
 
 
 # ---------------------------------------------------------------------------
@@ -211,8 +305,30 @@ def gpu_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale=1.0, mode="dipole"
     return O.cpu().numpy(), {n: t.cpu().numpy() for n, t in dbg.items()}
 
 
-def check_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale=1.0, mode="dipole", heads=None):
-    B, Hq = Q.shape[:2]
+def causal_problems(N, L):
+    """(problem index, level, pair, block size) of the hierarchical
+    decomposition, numbered level by level as the causal debug layouts are."""
+    out, k = [], 0
+    for lv in range(oracle.causal_levels(N, L)):
+        s = L << lv
+        for p in range(N // (2 * s)):
+            out.append((k, lv, p, s))
+            k += 1
+    return out
+
+
+def assert_causal_selected(g_sel, r_sel, q_assign, N, L, C, what):
+    """Retrieval sets of every block problem of one head, bit for bit, on the
+    rows of non-empty query clusters (the rows stage 2 uses)."""
+    for k, lv, p, s in causal_problems(N, L):
+        Ce = min(C, s)
+        live = np.bincount(q_assign[lv, p * s:(p + 1) * s], minlength=Ce) > 0
+        assert (g_sel[k, :Ce][live] == r_sel[k, :Ce][live]).all(), f"{what} R lv{lv} p{p}"
+
+
+def check_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale=1.0, mode="dipole", heads=None,
+                 rse_heads=None):
+    B, Hq, N = Q.shape[:3]
     G = Hq // K.shape[1]
     O, g = gpu_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale, mode)
     mask = None
@@ -225,10 +341,17 @@ def check_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale=1.0, mode="dipol
     for b, h in sel:
         assert_assign_match(g["k_assign"][b, h // G], r["k_assign"][b, h // G], what="k_assign")
         assert_assign_match(g["q_assign"][b, h], r["q_assign"][b, h], what="q_assign")
+        if "selected" in r:
+            assert_causal_selected(g["selected"][b, h], r["selected"][b, h], r["q_assign"][b, h],
+                                   N, L, C, f"b{b}h{h}")
         assert (g["n_exact"][b, h] == r["n_exact"][b, h]).all()
         assert_close(O[b, h], r["O"][b, h], TOL[dtype], f"O b{b}h{h}")
-    E = oracle.exact_attention(Q, K, V, scale, causal=True, hq_mask=mask)
-    idx = tuple(np.array(sel).T)
+    rh = sel if rse_heads is None else rse_heads
+    rmask = np.zeros((B, Hq), np.uint8)
+    for b, h in rh:
+        rmask[b, h] = 1
+    E = oracle.exact_attention(Q, K, V, scale, causal=True, hq_mask=rmask)
+    idx = tuple(np.array(rh).T)
     assert abs(rse(O[idx], E[idx]) - rse(r["O"][idx], E[idx])) < 1e-3
     return O, g, r
 
@@ -282,38 +405,79 @@ def test_causal_never_reads_the_future_on_gpu():
 
 
 def test_workload_causal_b2h8_n16k():
+    """The B=2, H=8 16k causal layer, every head against the oracle."""
     w = WORKLOADS["causal-bf16-b2h8-n16k"]
     Q, K, V = make_inputs(w)
     check_causal(Q, K, V, w.dtype, w.block, w.C, w.iters, w.cluster_seed, w.topk, w.scale,
-                 w.mode, heads=[(0, 0), (1, 7)])
+                 w.mode, rse_heads=[(0, 0), (1, 7)])
+
+
+# q-heads of the GQA layers checked against the oracle: the first kv-group
+# whole and the last q-head (kv-heads 0 and 7)
+GQA_HEADS = [0, 1, 2, 3, 31]
 
 
 @pytest.mark.parametrize("name", ["causal-gqa32x8-n64k-d64", "causal-gqa32x8-n32k-d128"])
-def test_workload_causal_gqa_full_size_sampled(name):
-    """Full-size GQA causal workloads: sampled k-means problems against the
-    oracle's k-means, then the oracle fed the GPU's clusterings
-    (teacher-forced) on one q-head, compared output by output."""
+def test_workload_causal_gqa_full_size(name):
+    """Full-size GQA causal workloads, on q-heads 0-3 and 31 and their
+    kv-heads 0 and 7:
+    - every (level, pair) k-means problem of both roles against the oracle's
+      own k-means (untethered), bit for bit;
+    - the oracle fed the GPU's clusterings (teacher-forced, which the line
+      above shows equal to the oracle's own) for the retrieval sets of every
+      block problem, the exact-key counts and the outputs;
+    - the relative squared error against exact causal attention on those
+      heads, GPU against oracle within 1e-3."""
     w = WORKLOADS[name]
     Q, K, V = make_inputs(w)
     O, g = gpu_causal(Q, K, V, w.dtype, w.block, w.C, w.iters, w.cluster_seed, w.topk, w.scale,
                       w.mode)
     assert np.isfinite(O).all()
-    N, L = w.N, w.block
+    N, L, C = w.N, w.block, w.C
+    G = w.Hq // w.Hkv
     levels = oracle.causal_levels(N, L)
     pmax = (N // L) // 2
-    for lv, p in [(0, 3), (2, 1), (levels - 1, 0)]:
-        s = L << lv
-        Ce = min(w.C, s)
-        slot = slice(lv * (N // 2) + p * s, lv * (N // 2) + (p + 1) * s)
-        ka, _, _, _ = oracle.kmeans(K[0, 0, 2 * p * s:(2 * p + 1) * s], Ce, w.iters,
-                                    w.cluster_seed, (0 * levels + lv) * pmax + p, 0)
-        assert_assign_match(g["k_assign"][0, 0].reshape(-1)[slot], ka, what=f"k lv{lv} p{p}")
-        qa, _, _, _ = oracle.kmeans(Q[0, 0, (2 * p + 1) * s:(2 * p + 2) * s], Ce, w.iters,
-                                    w.cluster_seed, (0 * levels + lv) * pmax + p, 1)
-        assert_assign_match(g["q_assign"][0, 0].reshape(-1)[slot], qa, what=f"q lv{lv} p{p}")
-    mask = np.zeros((1, w.Hq), np.uint8)
-    mask[0, 0] = 1
-    r = oracle.muse_causal(Q, K, V, L, w.C, w.iters, w.cluster_seed, w.topk, w.scale, w.mode,
-                           hq_mask=mask, q_assign_in=g["q_assign"], k_assign_in=g["k_assign"])
-    assert (g["n_exact"][0, 0] == r["n_exact"][0, 0]).all()
-    assert_close(O[0, 0], r["O"][0, 0], TOL[w.dtype], "O head 0")
+    kv_heads = sorted({h // G for h in GQA_HEADS})
+    jobs = []
+    for role, heads, X in ((0, kv_heads, K), (1, GQA_HEADS, Q)):
+        for h in heads:
+            for _, lv, p, s in causal_problems(N, L):
+                jobs.append((role, h, lv, p, s, X))
+
+    def run(job):
+        role, h, lv, p, s, X = job
+        blk = X[0, h, (2 * p + role) * s:(2 * p + role + 1) * s]
+        sid = (h * levels + lv) * pmax + p
+        return oracle.kmeans(blk, min(C, s), w.iters, w.cluster_seed, sid, role)[0]
+
+    # ctypes releases the GIL: the oracle's k-means problems run in parallel
+    with concurrent.futures.ThreadPoolExecutor(os.cpu_count() or 4) as ex:
+        results = list(ex.map(run, jobs))
+    for (role, h, lv, p, s, _), ra in zip(jobs, results):
+        ga = (g["k_assign"] if role == 0 else g["q_assign"])[0, h, lv, p * s:(p + 1) * s]
+        assert_assign_match(ga, ra, what=f"{'kq'[role]} h{h} lv{lv} p{p}")
+
+    def forced(h):
+        mask = np.zeros((1, w.Hq), np.uint8)
+        mask[0, h] = 1
+        return oracle.muse_causal(Q, K, V, L, C, w.iters, w.cluster_seed, w.topk, w.scale,
+                                  w.mode, hq_mask=mask, q_assign_in=g["q_assign"],
+                                  k_assign_in=g["k_assign"])
+
+    with concurrent.futures.ThreadPoolExecutor(len(GQA_HEADS)) as ex:
+        rs = list(ex.map(forced, GQA_HEADS))
+    for h, r in zip(GQA_HEADS, rs):
+        assert_causal_selected(g["selected"][0, h], r["selected"][0, h], g["q_assign"][0, h],
+                               N, L, C, f"h{h}")
+        assert (g["n_exact"][0, h] == r["n_exact"][0, h]).all(), f"n_exact h{h}"
+        assert_close(O[0, h], r["O"][0, h], TOL[w.dtype], f"O head {h}")
+    # exact causal attention is O(N^2) per head in fp64: the relative squared
+    # error is taken over 512 sampled query rows per head (the first and last
+    # rows, block edges and random rows), for the GPU and the oracle alike
+    rng = np.random.default_rng(11)
+    rows = np.unique(np.concatenate([[0, 1, L - 1, L, N - 1], rng.integers(0, N, 507)]))
+    E = np.stack([oracle.exact_attention_rows(Q, K, V, 0, h, rows, w.scale, causal=True)
+                  for h in GQA_HEADS])
+    r_gpu = rse(O[0, GQA_HEADS][:, rows], E)
+    r_orc = rse(np.stack([r["O"][0, h][rows] for h, r in zip(GQA_HEADS, rs)]), E)
+    assert abs(r_gpu - r_orc) < 1e-3, (r_gpu, r_orc)

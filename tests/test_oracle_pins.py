@@ -17,6 +17,7 @@ import pytest
 import torch
 
 from clustered_multipole_approximation_b200.inputs import clustered_qkv
+from oracle import causal_levels
 
 
 def small_qkv(B=1, Hq=1, Hkv=1, N=256, D=16, centres=8, noise=0.3, seed=7, lognormal=0.0):
@@ -420,3 +421,39 @@ def test_dipole_rse_sanity_bound(orc):
         O = orc.muse_acausal(Q, K, V, 16, 32, 6, 3, 2, mode=m)["O"]
         errs[m] = float(((O - E) ** 2).sum() / (E ** 2).sum())
     assert errs["dipole"] < 0.2, errs
+
+
+def test_exact_attention_rows_equal_the_full_computation(orc):
+    Q, K, V = clustered_qkv(1, 4, 2, 200, 64, 8, 0.3, 0.0, "f32", 14)
+    rows = np.array([0, 3, 64, 199, 120])
+    for causal in (False, True):
+        E = orc.exact_attention(Q, K, V, 0.7, causal=causal)
+        Er = orc.exact_attention_rows(Q, K, V, 0, 2, rows, 0.7, causal=causal)
+        assert (Er == E[0, 2, rows]).all()
+
+
+def test_causal_retrieval_sets_are_those_of_each_block_problem(orc):
+    """Every block problem of the causal decomposition is the acausal
+    operator on its (query block, key block) pair: with the same clusterings,
+    its reported retrieval sets equal stage 1 of that pair alone."""
+    N, L, C, k1 = 512, 64, 12, 3
+    Q, K, V = clustered_qkv(1, 2, 1, N, 64, 8, 0.3, 0.0, "f32", 15)
+    r = orc.muse_causal(Q, K, V, L, C, 3, 4, k1)
+    k = 0
+    for lv in range(causal_levels(N, L)):
+        s = L << lv
+        Ce = min(C, s)
+        for p in range(N // (2 * s)):
+            for h in range(2):
+                qa = r["q_assign"][0, h, lv, p * s:(p + 1) * s]
+                ka = r["k_assign"][0, 0, lv, p * s:(p + 1) * s]
+                _, _, R = orc.stage1_debug(Q[0, h, (2 * p + 1) * s:(2 * p + 2) * s],
+                                           K[0, 0, 2 * p * s:(2 * p + 1) * s],
+                                           V[0, 0, 2 * p * s:(2 * p + 1) * s], Ce, Ce, qa, ka, k1)
+                # rows of empty query clusters are unused (their centroid is
+                # the one kept by the k-means, not a mean of given members)
+                live = np.bincount(qa, minlength=Ce) > 0
+                assert (r["selected"][0, h, k, :Ce][live] == R[live]).all(), (lv, p, h)
+                assert (r["selected"][0, h, k, Ce:] == -1).all()
+            k += 1
+    assert k == N // L - 1

@@ -35,10 +35,12 @@ def test_static_scratch_matches_workspace_entry_point(dtype):
         a = torch.full_like(ref_a, -1)
         c = torch.full_like(ref_c, float("nan"))
         n = torch.full_like(ref_n, -1)
+        err = torch.full((1,), -1, dtype=torch.int32, device="cuda")
         st = lib.muse_cluster_static(_p(x), code, B, H, N, D, C, iters, seed, 1, None, _p(a),
-                                     _p(c), _p(n), stream)
+                                     _p(c), _p(n), _p(err), stream)
         assert st == 0, lib.muse_last_error()
         torch.cuda.synchronize()
+        assert int(err.item()) == 0
         assert torch.equal(a, ref_a)
         assert torch.equal(n, ref_n)
         np.testing.assert_allclose(c.cpu().numpy(), ref_c.cpu().numpy(), rtol=2e-7, atol=1e-7)
@@ -53,6 +55,6 @@ def test_static_scratch_rejects_sizes_beyond_its_capacity():
     x = torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16, device="cuda")  # never read
     out = torch.zeros(16, dtype=torch.int32, device="cuda")
     st = lib.muse_cluster_static(_p(x), 0, 1, 64, 32768, 128, 256, 3, 0, 0, None, _p(out),
-                                 _p(out), None, None)
+                                 _p(out), None, None, None)
     assert st == 3
     assert b"scratch" in lib.muse_last_error()
