@@ -108,6 +108,11 @@ void carve_kstate(Carver& cv, KState& ks, const RoleGeo& g) {
   ks.cbf_hi = cv.take<__nv_bfloat16>(np * C * D * 2);
   ks.cbf_lo = cv.take<__nv_bfloat16>(np * C * D * 2);
   ks.cn2 = cv.take<float>(np * C * 4);
+  ks.emin = cv.take<int>(np * 4);
+  ks.emax = cv.take<int>(np * 4);
+  ks.part_blocks = g.dtype == 0 ? resident_partial_blocks(g.lv, g.BH, g.D, g.C) : 0;
+  ks.part = cv.take<double>(ks.part_blocks * C * D * 8);
+  ks.pcnt = cv.take<int>(ks.part_blocks * C * 4);
 }
 
 RoleGeo make_geo(const void* X, int BH, int D, int C, int role, int dtype, uint64_t seed,
@@ -272,11 +277,13 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
     const RoleGeo gs[2] = {L.kg, L.qg};
     const KState kss[2] = {L.ks, L.qs};
     run_kmeans_init(gs, kss, 2, nullptr, st);
-    bool fused;
+#ifdef MUSE_PHASE_CLOCKS
     {
-      ProfScope ps(st, "kmeans_fused");
-      fused = launch_kmeans_fused(gs, kss, 2, pr->iters, st);
+      const cudaError_t e = cudaStreamSynchronize(st);
+      fprintf(stderr, "after v_to_half + kmeans_init: %s\n", cudaGetErrorString(e));
     }
+#endif
+    const bool fused = launch_kmeans_fused(gs, kss, 2, pr->iters, st);
     if (!fused) {
       run_kmeans_rounds(L.kg, L.ks, pr->iters, st);
       run_kmeans_rounds(L.qg, L.qs, pr->iters, st);
@@ -362,11 +369,7 @@ muse_status muse_cluster(const void* X, muse_dtype dtype, int B, int H, int N, i
   cudaMemsetAsync(err, 0, 4, stream);
   cudaMemsetAsync(ks.arrive, 0, (size_t)ks.nprob * 4, stream);
   run_kmeans_init(&g, &ks, 1, init, stream);
-  bool fused;
-  {
-    ProfScope ps(stream, "kmeans_fused");
-    fused = launch_kmeans_fused(&g, &ks, 1, iters, stream);
-  }
+  const bool fused = launch_kmeans_fused(&g, &ks, 1, iters, stream);
   if (!fused) run_kmeans_rounds(g, ks, iters, stream);
   cudaMemcpyAsync(assign, ks.assign, (size_t)ks.ntok * 4, cudaMemcpyDeviceToDevice, stream);
   cudaMemcpyAsync(centroids, ks.cent32, (size_t)ks.nprob * C * D * 4, cudaMemcpyDeviceToDevice, stream);

@@ -127,10 +127,29 @@ struct KState {
   __nv_bfloat16* cbf_hi;  // [nprob][C][D] bf16 rounding of cent32
   __nv_bfloat16* cbf_lo;  // [nprob][C][D] bf16 rounding of cent32 - cbf_hi
   float* cn2;       // [nprob][C]    ||c||^2 (fp64 sum rounded to fp32)
+  int* emin;        // [nprob]       smallest biased exponent of a nonzero value (bf16)
+  int* emax;        // [nprob]       largest biased exponent of a value (bf16)
+  double* part;     // [part_blocks][C][D] per-CTA partial centroid sums (resident k-means)
+  int* pcnt;        // [part_blocks][C]    per-CTA member counts (resident k-means)
+  size_t part_blocks;
   int* err;         // device error word (0 = ok)
   int nprob;
   long long ntiles;
   long long ntok;
 };
+
+// The centroid sums of a problem are exact in fp64 in any order -- and so
+// equal to a plain sequential fp64 sum bit for bit -- when every partial sum
+// is a representable multiple of the smallest value's ulp: with bf16 values
+// of biased exponents in [emin, emax] (ulp 2^(emin - 134) for emin >= 1, the
+// subnormals counted as emin = 1) and at most s members,
+// |partial| < s 2^(emax - 126) <= 2^53 ulp  <=  (emax - emin) + ceil(log2 s) <= 45.
+__device__ inline bool sums_exact(const KState& ks, int pid, int s) {
+  const int lo = ks.emin[pid], hi = ks.emax[pid];
+  if (hi < lo) return true;  // no nonzero value
+  int lg = 0;
+  while ((1 << lg) < s) ++lg;
+  return (hi - lo) + lg <= 45;
+}
 
 }  // namespace muse

@@ -74,6 +74,14 @@ bool launch_kmeans_fused(const RoleGeo* gs, const KState* kss, int nsets, int it
 // Failure-path testing of the persistent k-means' team barrier.
 void set_barrier_fault(int rank, int spin_limit);
 
+// The resident-tile k-means for the problems of one level (lvl < 0: the
+// acausal single level) whose centroid sums are certified exact; false when
+// these sizes are not covered (nothing launched).
+bool launch_kmeans_resident(const RoleGeo* gs, const KState* kss, int nsets, int lvl, int iters,
+                            cudaStream_t st);
+// Partial-sum blocks the resident k-means may need for one role's levels.
+size_t resident_partial_blocks(const Levels& lv, int BH, int D, int C);
+
 // Lloyd rounds one launch sequence at a time (any dtype / size).
 void run_kmeans_rounds(const RoleGeo& g, const KState& ks, int iters, cudaStream_t st);
 

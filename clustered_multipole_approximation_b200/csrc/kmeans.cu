@@ -101,6 +101,47 @@ __global__ void __launch_bounds__(256) kmeans_init_kernel(InitSets is, const flo
     }
     __syncthreads();
   }
+  if (sizeof(T) == 2) {
+    // exponent range of the problem's values: the exactness certificate of
+    // the order-free centroid sums (sums_exact); this CTA scans its share of
+    // the problem's rows, 8 bf16 values per 16-byte load
+    const int per = cdiv(p.s, is.nsplit);
+    const int t0 = part * per, t1 = imin(p.s, t0 + per);
+    int lo = 1 << 30, hi = -1;
+    if (t1 > t0) {
+      const uint4* xv = reinterpret_cast<const uint4*>(X + (p.row0 + t0) * D);
+      const int nv = (t1 - t0) * D / 8;
+      for (int i0 = threadIdx.x; i0 < nv; i0 += 4 * blockDim.x) {
+        uint4 v[4];  // four loads in flight; zero words count for nothing
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * (int)blockDim.x;
+          v[u] = i < nv ? xv[i] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t b = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+            if (b & 0x7FFFu) {
+              const int e = (int)((b >> 7) & 0xFFu);
+              lo = min(lo, e > 0 ? e : 1);
+              hi = max(hi, e);
+            }
+          }
+        }
+      }
+    }
+    for (int o = 16; o; o >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if ((threadIdx.x & 31) == 0 && hi >= 0) {
+      atomicMin(ks.emin + pid, lo);
+      atomicMax(ks.emax + pid, hi);
+    }
+  }
   // one warp per centroid row, four rows per step (loads issued together):
   // fp64/fp32 copies, the bf16 split for the tensor cores, and the norms
   const float* src = init ? init + (size_t)p.bh * g.C * D : nullptr;  // muse_cluster: one problem per bh
@@ -370,6 +411,11 @@ static void init_t(const RoleGeo* gs, const KState* kss, int nsets, const float*
     is.ks[k] = kss[k];
   }
   const int nprob = kss[0].nprob + (nsets > 1 ? kss[1].nprob : 0);
+  if (sizeof(T) == 2)
+    for (int k = 0; k < nsets; ++k) {  // empty ranges: emin = 0x7F7F7F7F > emax = 0x80808080
+      cudaMemsetAsync(kss[k].emin, 0x7F, (size_t)kss[k].nprob * 4, st);
+      cudaMemsetAsync(kss[k].emax, 0x80, (size_t)kss[k].nprob * 4, st);
+    }
   is.nsplit = nprob >= 148 ? 1 : 8;  // spread few problems over more SMs
   is.nblk0 = kss[0].nprob * is.nsplit;
   const int nblk = nprob * is.nsplit;

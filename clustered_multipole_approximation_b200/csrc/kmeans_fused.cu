@@ -30,6 +30,7 @@
 // owners write the counts, segment offsets and the cluster-sorted permutation
 // that the summaries and stage 2 read.
 #include <cooperative_groups.h>
+#include <stdio.h>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -51,6 +52,8 @@ constexpr int kSpinLimit = 1 << 24;  // team barrier polls (64 ns apart) before 
 // the poll bound of the barrier waits (muse_debug_inject_barrier_fault).
 int g_fault_rank = -1;
 int g_spin_limit = kSpinLimit;
+// Testing: route every problem through the sequential-order kernel.
+int g_no_resident = 0;
 constexpr int kOT = kNCF + kMaxNCT;  // (owned cluster, rank) pairs per CTA, at most
 constexpr int kTilesPerCta = 16;     // cluster launches: target tiles per CTA
 constexpr size_t kSmemLimit = 218 * 1024;  // dynamic shared memory (static arrays come on top)
@@ -223,6 +226,7 @@ struct FusedSets {
   int lvl;
   int fault_rank;  // cooperative launches: this CTA rank skips its first arrival
   int spin_limit;  // polls of a barrier wait before it gives up
+  int skip_certified;  // leave problems with certified-exact sums (the resident kernel's)
 };
 
 // Exclusive scan of n <= 2 * blockDim.x ints in shared memory, called by
@@ -303,6 +307,8 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     pid = (pid / np) * g.lv.pairs_per_bh + g.lv.pair_base[fs.lvl] + pid % np;
   }
   const Prob p = prob_of(g, pid);
+  // every CTA of the problem takes the same decision
+  if (fs.skip_certified && sums_exact(ks, pid, p.s)) return;
   const int C = p.C;
   const int ntp = cdiv(p.s, kTile);
   const int tpc = cdiv(ntp, NCT);
@@ -913,7 +919,8 @@ static bool plan_fused(const RoleGeo* gs, const KState* kss, int nsets, int lvl,
 
 template <int D>
 static void launch_plan(const RoleGeo* gs, const KState* kss, int nsets, int lvl, int iters,
-                        int NC, int tcols, const FusedPlan& plan, cudaStream_t st) {
+                        int NC, int tcols, const FusedPlan& plan, bool skip_certified,
+                        cudaStream_t st) {
   FusedSets fs{};
   int np[2] = {0, 0};
   for (int k = 0; k < nsets; ++k) {
@@ -924,6 +931,7 @@ static void launch_plan(const RoleGeo* gs, const KState* kss, int nsets, int lvl
   fs.lvl = lvl;
   fs.fault_rank = plan.coop ? g_fault_rank : -1;
   fs.spin_limit = g_spin_limit;
+  fs.skip_certified = skip_certified ? 1 : 0;
   fs.nblk0 = np[0] * plan.NCT;
   const int nblk = (np[0] + np[1]) * plan.NCT;
   cudaLaunchConfig_t cfg = {};
@@ -972,22 +980,48 @@ static bool launch_fused_t(const RoleGeo* gs, const KState* kss, int nsets, int 
   const int NC = (cmax + 31) & ~31;
   int tcols = 32;
   while (tcols < 2 * NC) tcols <<= 1;  // two accumulators (tiles in flight)
+  // per level: the resident-tile kernel where it covers the sizes, followed
+  // by this kernel for the problems whose sums it cannot certify exact
   const int nlev = gs[0].lv.nlev;
   FusedPlan plans[kMaxLevels];
+  auto level = [&](int l, const FusedPlan& plan) {
+    bool res;
+    {
+      ProfScope ps(st, "kmeans_resident");
+      res = !g_no_resident && launch_kmeans_resident(gs, kss, nsets, l, iters, st);
+    }
+#ifdef MUSE_PHASE_CLOCKS
+    {
+      const cudaError_t e = cudaStreamSynchronize(st);
+      fprintf(stderr, "after resident lvl %d (launched %d): %s\n", l, (int)res, cudaGetErrorString(e));
+    }
+#endif
+    ProfScope ps(st, "kmeans_ordered");
+    launch_plan<D>(gs, kss, nsets, l, iters, NC, tcols, plan, res, st);
+#ifdef MUSE_PHASE_CLOCKS
+    {
+      const cudaError_t e = cudaStreamSynchronize(st);
+      fprintf(stderr, "after ordered lvl %d (coop %d nct %d): %s\n", l, (int)plan.coop, plan.NCT,
+              cudaGetErrorString(e));
+    }
+#endif
+  };
   if (nlev == 1) {
     if (!plan_fused<D>(gs, kss, nsets, -1, NC, plans[0])) return false;
-    launch_plan<D>(gs, kss, nsets, -1, iters, NC, tcols, plans[0], st);
+    level(-1, plans[0]);
     return true;
   }
   for (int l = 0; l < nlev; ++l)
     if (!plan_fused<D>(gs, kss, nsets, l, NC, plans[l])) return false;
-  for (int l = 0; l < nlev; ++l) launch_plan<D>(gs, kss, nsets, l, iters, NC, tcols, plans[l], st);
+  for (int l = 0; l < nlev; ++l) level(l, plans[l]);
   return true;
 }
 
 void set_barrier_fault(int rank, int spin_limit) {
   g_fault_rank = rank;
   g_spin_limit = rank >= 0 && spin_limit > 0 ? spin_limit : kSpinLimit;
+  // the fault hook targets this kernel's cooperative barrier
+  g_no_resident = rank >= 0 ? 1 : 0;
 }
 
 bool launch_kmeans_fused(const RoleGeo* gs, const KState* kss, int nsets, int iters,

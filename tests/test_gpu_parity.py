@@ -169,6 +169,27 @@ def test_muse_cluster_bf16_cluster_counts(C, D, N):
         np.testing.assert_allclose(c[0, h].cpu().numpy(), rc, rtol=2e-7, atol=1e-7)
 
 
+@pytest.mark.parametrize("spread", ["wide", "narrow"])
+def test_muse_cluster_sums_outside_the_exactness_certificate(spread):
+    """Centroid sums are taken in any order only when the problem's exponent
+    range certifies them exact; a problem whose values span too many binades
+    (here tokens scaled by 2^40 next to tokens scaled by 2^-40) goes through
+    the sequential-order kernel.  Both must equal the oracle bit for bit."""
+    X, _, _ = clustered_qkv(1, 2, 2, 1500, 64, 12, 0.3, 0.0, "f32", 44)
+    if spread == "wide":
+        X[0, 0, ::7] *= 2.0 ** 40
+        X[0, 0, 3::7] *= 2.0 ** -40
+    Xb = to_dev(X, "bf16")
+    Xr = Xb.float().cpu().numpy()
+    a, c, n = muse.muse_cluster(Xb, 20, 4, 5, role=0)
+    torch.cuda.synchronize()
+    for h in range(2):
+        ra, rc, rn, _ = oracle.kmeans(Xr[0, h], 20, 4, 5, h, 0)
+        assert_assign_match(a[0, h].cpu().numpy(), ra, what=f"assign h{h}")
+        assert (n[0, h].cpu().numpy() == rn).all()
+        np.testing.assert_allclose(c[0, h].cpu().numpy(), rc, rtol=2e-7, atol=1e-30)
+
+
 def test_muse_cluster_one_round_from_given_centroids():
     X, _, _ = clustered_qkv(1, 2, 2, 1500, 128, 20, 0.3, 0.0, "bf16", 41)
     rng = np.random.default_rng(1)
