@@ -95,6 +95,10 @@ void run_blocks(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStrea
 // overflows fp16 sets kErrVRange in *err.
 void run_bf16_to_half(const void* src, __half* dst, size_t n, int* err, cudaStream_t st);
 
+// Top-k1 key clusters of every query cluster (certified fp32 screen, exact
+// fp64 scores for the candidates).
+void run_select(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
+
 // Stage 2 on mma.sync tensor-core tiles (bf16 inputs).
 void run_stage2_mma(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 // Stage 1 (DIPOLE) on tcgen05 tensor cores (bf16 inputs).

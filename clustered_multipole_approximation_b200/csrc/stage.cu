@@ -264,125 +264,6 @@ __global__ void __launch_bounds__(kS1T) stage1_kernel(AttnArgs a, Stage1 s1, int
 }
 
 // ----------------------------------------------------------------------------
-// selection: top-k key clusters per query cluster by s nu_i.mu_j + log W_ij,
-// ties to the lowest j, empty clusters never
-// ----------------------------------------------------------------------------
-// Query clusters handled by one CTA of the selection kernel (one per warp).
-constexpr int kSelQ = 8;
-
-// Key centroids per CTA staged in shared memory when they fit (row stride
-// D + 1 doubles keeps the lanes' rows on distinct banks).
-template <int D>
-constexpr size_t select_stage_bytes(int Ck) {
-  return (size_t)Ck * (D + 1) * sizeof(double);
-}
-constexpr size_t kSelectSmemMax = 200 * 1024;
-
-// One warp per query cluster: lanes over key clusters, four key clusters per
-// lane at a time (independent fp64 chains, each in dimension order with no
-// fused operations, as a plain sequential evaluation), then top-k1 by k1
-// rounds of warp argmax, ties to the lowest index.
-template <int D, bool STAGED>
-__global__ void __launch_bounds__(256) select_kernel(AttnArgs a, Stage1 s1, int qp0) {
-  extern __shared__ double sel_smem[];
-  const int lq = blockIdx.x, qpid = qp0 + lq;
-  const Prob pq = prob_of(a.qg, qpid);
-  const int kpid = kv_problem(a, qpid);
-  const Prob pk = prob_of(a.kg, kpid);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Cq = a.Cq, Ck = a.Ck, K1 = a.topk;
-  const int ck = pk.C;
-  const double* mug = a.ks.cent64 + (size_t)kpid * Ck * D;
-  double* mus = sel_smem;                                            // [ck][D + 1]
-  double* sc = sel_smem + (STAGED ? (size_t)Ck * (D + 1) : 0) + (size_t)warp * Ck;
-  if (STAGED) {
-    const int tot = ck * D;
-    for (int e0 = threadIdx.x; e0 < tot; e0 += 8 * blockDim.x) {  // 8 loads in flight
-      double v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = e0 + u * blockDim.x;
-        v[u] = e < tot ? mug[e] : 0.0;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = e0 + u * blockDim.x;
-        if (e < tot) {
-          const int j = e / D, d = e - j * D;
-          mus[j * (D + 1) + d] = v[u];
-        }
-      }
-    }
-    __syncthreads();
-  }
-  const double s = (double)a.scale;
-  const int* kc = a.ks.counts + (size_t)kpid * Ck;
-  const int i1 = imin(pq.C, (blockIdx.y + 1) * kSelQ);
-  for (int i = blockIdx.y * kSelQ + warp; i < i1; i += 8) {  // warp-uniform
-    const double* nu = a.qs.cent64 + ((size_t)qpid * Cq + i) * D;
-    for (int jb = 0; jb < ck; jb += 128) {
-      double dt[4] = {0.0, 0.0, 0.0, 0.0};
-      for (int d = 0; d < D; ++d) {
-        const double nv = nu[d];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = jb + lane + 32 * u;
-          if (j < ck) {
-            const double mv = STAGED ? mus[j * (D + 1) + d] : mug[(size_t)j * D + d];
-            dt[u] = __dadd_rn(dt[u], __dmul_rn(nv, mv));
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = jb + lane + 32 * u;
-        if (j < ck) {
-          double v = -INFINITY;
-          if (kc[j] > 0) {
-            const double lw = (a.mode == 2) ? (double)s1.logW[((size_t)lq * Cq + i) * Ck + j]
-                                            : log((double)kc[j]);
-            v = __dadd_rn(__dmul_rn(s, dt[u]), lw);
-          }
-          sc[j] = v;
-        }
-      }
-    }
-    __syncwarp();
-    int taken = 0;
-    int* out = s1.sel + ((size_t)qpid * Cq + i) * (K1 > 0 ? K1 : 1);
-    for (int r = 0; r < K1; ++r) {
-      double bv = -INFINITY;
-      int bj = -1;
-      for (int j = lane; j < ck; j += 32) {
-        const double v = sc[j];
-        if (v > -INFINITY && (bj < 0 || v > bv)) {
-          bv = v;
-          bj = j;
-        }
-      }
-      for (int o = 16; o; o >>= 1) {
-        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-        if (oj >= 0 && (bj < 0 || ov > bv || (ov == bv && oj < bj))) {
-          bv = ov;
-          bj = oj;
-        }
-      }
-      if (bj < 0) break;
-      if (lane == 0) out[r] = bj;
-      if (lane == (bj & 31)) sc[bj] = -INFINITY;  // remove from later rounds
-      __syncwarp();
-      ++taken;
-    }
-    if (lane == 0) {
-      for (int r = taken; r < K1; ++r) out[r] = -1;
-      s1.nsel[(size_t)qpid * Cq + i] = taken;
-    }
-    __syncwarp();
-  }
-}
-
-// ----------------------------------------------------------------------------
 // stage 2: far field + exact retrieval in one online softmax
 // ----------------------------------------------------------------------------
 constexpr int kQ = 64;     // queries per pass
@@ -636,10 +517,6 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
   // set on every launch: the attribute is per device, and the call is cheap
   cudaFuncSetAttribute(stage1_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)stage1_smem<D>());
-  cudaFuncSetAttribute(select_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)kSelectSmemMax);
-  cudaFuncSetAttribute(select_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       8 * kMaxC * (int)sizeof(double));
   {
     ProfScope ps(st, "stage1_summaries");
     if (sizeof(T) == 2 && a.mode == 1)
@@ -649,12 +526,7 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
   }
   if (a.topk > 0) {
     ProfScope ps(st, "stage1_select");
-    const size_t smem = (size_t)8 * a.Ck * sizeof(double);
-    const dim3 grid(nqp, cdiv(a.Cq, kSelQ));
-    if (smem + select_stage_bytes<D>(a.Ck) <= kSelectSmemMax)
-      select_kernel<D, true><<<grid, 256, smem + select_stage_bytes<D>(a.Ck), st>>>(a, s1, qp0);
-    else
-      select_kernel<D, false><<<grid, 256, smem, st>>>(a, s1, qp0);
+    run_select(a, s1, qp0, nqp, st);
   }
   if (sizeof(T) == 2) {
     {
