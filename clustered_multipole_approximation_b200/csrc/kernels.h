@@ -99,6 +99,10 @@ void run_bf16_to_half(const void* src, __half* dst, size_t n, int* err, cudaStre
 // fp64 scores for the candidates).
 void run_select(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 
+// Stage 2 with one warp per 16-query slice (bf16 inputs, topk <= 64); false
+// (nothing launched) when these arguments are not covered.
+bool run_stage2_warp(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
+
 // Stage 2 on mma.sync tensor-core tiles (bf16 inputs).
 void run_stage2_mma(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 // Stage 1 (DIPOLE) on tcgen05 tensor cores (bf16 inputs).
