@@ -43,7 +43,8 @@ class muse_shape(ctypes.Structure):
 class muse_params(ctypes.Structure):
     _fields_ = [("Cq", ctypes.c_int), ("Ck", ctypes.c_int), ("iters", ctypes.c_int),
                 ("seed", ctypes.c_uint64), ("topk", ctypes.c_int), ("block", ctypes.c_int),
-                ("scale", ctypes.c_float), ("mode", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("mode", ctypes.c_int),
+                ("key_stream0", ctypes.c_uint64), ("query_stream0", ctypes.c_uint64)]
 
 
 class muse_debug(ctypes.Structure):
@@ -140,9 +141,11 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
-def make_params(Cq, Ck, iters, seed, topk, block=0, scale=1.0, mode="dipole") -> muse_params:
+def make_params(Cq, Ck, iters, seed, topk, block=0, scale=1.0, mode="dipole", key_stream0=0,
+                query_stream0=0) -> muse_params:
     return muse_params(int(Cq), int(Ck), int(iters), int(seed) & (2 ** 64 - 1), int(topk),
-                       int(block), float(scale), MODES[mode] if isinstance(mode, str) else int(mode))
+                       int(block), float(scale), MODES[mode] if isinstance(mode, str) else int(mode),
+                       int(key_stream0) & (2 ** 64 - 1), int(query_stream0) & (2 ** 64 - 1))
 
 
 def make_shape(q, k, out_f32: bool = False) -> muse_shape:
@@ -216,19 +219,22 @@ def _attn(causal, q, k, v, params, out=None, workspace=None, debug=False, stream
 
 
 def muse_attn_fwd(q, k, v, *, Cq, Ck, iters, seed, topk, scale=1.0, mode="dipole", out=None,
-                  workspace=None, debug=False, stream=None, out_dtype=None):
+                  workspace=None, debug=False, stream=None, out_dtype=None, key_stream0=0,
+                  query_stream0=0):
     """Acausal MuSe forward.  q [B,Hq,N,D], k and v [B,Hkv,N,D] (bf16 or fp32,
     contiguous, CUDA).  Returns O (input dtype, or fp32 with out_dtype=float32)
-    and, with debug, a dict of inspection tensors."""
-    p = make_params(Cq, Ck, iters, seed, topk, 0, scale, mode)
+    and, with debug, a dict of inspection tensors.  key_stream0 /
+    query_stream0: see muse_params in include/muse.h (shards of a layer)."""
+    p = make_params(Cq, Ck, iters, seed, topk, 0, scale, mode, key_stream0, query_stream0)
     return _attn(False, q, k, v, p, out, workspace, debug, stream, out_dtype)
 
 
 def muse_attn_fwd_causal(q, k, v, *, C, block, iters, seed, topk, scale=1.0, mode="dipole",
-                         out=None, workspace=None, debug=False, stream=None, out_dtype=None):
+                         out=None, workspace=None, debug=False, stream=None, out_dtype=None,
+                         key_stream0=0, query_stream0=0):
     """Causal MuSe forward (hierarchical blocks of `block` tokens, C clusters
     per level and role)."""
-    p = make_params(C, C, iters, seed, topk, block, scale, mode)
+    p = make_params(C, C, iters, seed, topk, block, scale, mode, key_stream0, query_stream0)
     return _attn(True, q, k, v, p, out, workspace, debug, stream, out_dtype)
 
 

@@ -190,6 +190,8 @@ AttnLayout layout(const muse_shape* sh, const muse_params* pr, bool causal, cons
   const int dt = sh->dtype == MUSE_BF16 ? 0 : 1;
   L.kg = make_geo(K, sh->B * sh->Hkv, sh->D, pr->Ck, 0, dt, pr->seed, lv);
   L.qg = make_geo(Q, sh->B * sh->Hq, sh->D, pr->Cq, 1, dt, pr->seed, lv);
+  L.kg.sid0 = pr->key_stream0;
+  L.qg.sid0 = pr->query_stream0;
   Carver cv{static_cast<char*>(ws)};
   L.err = cv.take<int>(4);
   carve_kstate(cv, L.ks, L.kg);

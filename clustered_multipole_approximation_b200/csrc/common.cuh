@@ -49,6 +49,7 @@ struct RoleGeo {
   int dtype;   // 0 bf16, 1 f32
   const void* X;
   uint64_t seed;
+  uint64_t sid0;  // stream id of row set (b, h) = (0, 0): row set bh draws stream sid0 + bh
 };
 
 struct Prob {
@@ -78,8 +79,8 @@ __device__ inline Prob prob_of(const RoleGeo& g, int pid) {
   p.slot0 = (long long)p.bh * L.toks_per_bh + L.tok_base[l] + (long long)p.pair * p.s;
   p.tile0 = (long long)p.bh * L.tiles_per_bh + L.tile_base[l] +
             (long long)p.pair * L.tiles_per_pair[l];
-  p.sid = L.causal ? ((uint64_t)p.bh * L.nlev + l) * (uint64_t)L.pmax + p.pair
-                   : (uint64_t)p.bh;
+  p.sid = L.causal ? ((g.sid0 + (uint64_t)p.bh) * L.nlev + l) * (uint64_t)L.pmax + p.pair
+                   : g.sid0 + (uint64_t)p.bh;
   return p;
 }
 

@@ -99,6 +99,13 @@ typedef struct {
   int block;       /* causal local block L (ignored by muse_attn_fwd) */
   float scale;     /* softmax scale s: logits are s q.k */
   muse_mode mode;
+  /* Stream ids of the first key and query row sets, (b, h) = (0, 0): row set
+   * (b, h) of this call draws its seeded k-means start from stream
+   * stream0 + b H + h.  0 for a whole layer; a shard of a layer made of
+   * consecutive (b, kv-head) units u0 .. u1 (each unit one batch entry with
+   * Hkv = 1 and Hq = G) passes key_stream0 = u0 and query_stream0 = G u0 and
+   * gets bit for bit the whole layer's rows. */
+  uint64_t key_stream0, query_stream0;
 } muse_params;
 
 /* Optional device outputs for inspection; any member may be NULL.
@@ -253,12 +260,14 @@ void muse_profile_enable(int on);
 int muse_profile_read(char *names, int name_stride, int *launches, double *ms,
                       int cap);
 
-/* Failure-path testing (no paper counterpart).  While rank >= 0, every
- * cooperative launch of the persistent k-means in this process lets CTA
- * `rank` of each problem skip its arrival at the first barrier, and every
- * barrier wait gives up after `spin_limit` polls (about 64 ns apart): the
- * kernel then records MUSE_DEVERR_TEAM_BARRIER and returns without touching
- * its outputs.  rank < 0 restores normal operation.  Not thread-safe. */
+/* Failure-path testing (no paper counterpart).  While rank >= 0, the
+ * persistent k-means of this process runs every problem on its
+ * sequential-order kernel, and each of that kernel's cooperative launches
+ * lets CTA `rank` of each problem skip its arrival at the first barrier;
+ * every barrier wait gives up after `spin_limit` polls (about 64 ns apart):
+ * the kernel then records MUSE_DEVERR_TEAM_BARRIER and returns without
+ * touching its outputs.  rank < 0 restores normal operation.  Not
+ * thread-safe. */
 void muse_debug_inject_barrier_fault(int rank, int spin_limit);
 
 /* Message of the last failing call on this host thread ("" if none). */

@@ -58,11 +58,11 @@ def _bind(lib):
     lib.orc_summaries.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _ip,
                                   _dp, _dp, _dp]
     lib.orc_muse_acausal.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 8 + [
-        ctypes.c_uint64, ctypes.c_int, ctypes.c_double, ctypes.c_int, _u8p, _ip, _ip,
-        _dp, _ip, _ip, _dp, _dp, _ip, _ip, _llp]
+        ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int, ctypes.c_double,
+        ctypes.c_int, _u8p, _ip, _ip, _dp, _ip, _ip, _dp, _dp, _ip, _ip, _llp]
     lib.orc_muse_causal.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 8 + [
-        ctypes.c_uint64, ctypes.c_int, ctypes.c_double, ctypes.c_int, _u8p, _ip, _ip,
-        _dp, _ip, _ip, _ip, _llp]
+        ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int, ctypes.c_double,
+        ctypes.c_int, _u8p, _ip, _ip, _dp, _ip, _ip, _ip, _llp]
     lib.orc_exact_attn.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 5 + [
         ctypes.c_double, ctypes.c_int, _u8p, _dp]
     lib.orc_exact_attn_rows.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 5 + [
@@ -167,7 +167,8 @@ class Oracle:
         return S, M
 
     def muse_acausal(self, Q, K, V, Cq, Ck, iters, seed, topk, scale=1.0, mode="dipole",
-                     hq_mask=None, q_assign_in=None, k_assign_in=None):
+                     hq_mask=None, q_assign_in=None, k_assign_in=None, key_stream0=0,
+                     query_stream0=0):
         """Acausal MuSe in fp64.  Returns a dict with O, the clusterings, the
         selections R and the number of exactly-attended keys per query."""
         Q, qp = _d(Q)
@@ -187,7 +188,8 @@ class Oracle:
         selected = np.full((B, Hq, Cq, max(topk, 1)), -1, dtype=np.int32)
         n_exact = np.zeros((B, Hq, N), dtype=np.int64)
         self.lib.orc_muse_acausal(
-            qp, kp, vp, B, Hq, Hkv, N, D, Cq, Ck, iters, seed, topk, float(scale), MODES[mode],
+            qp, kp, vp, B, Hq, Hkv, N, D, Cq, Ck, iters, seed, key_stream0, query_stream0, topk,
+            float(scale), MODES[mode],
             m_p, qa_p, ka_p, O.ctypes.data_as(_dp), q_assign.ctypes.data_as(_ip),
             k_assign.ctypes.data_as(_ip), q_cent.ctypes.data_as(_dp), k_cent.ctypes.data_as(_dp),
             k_count.ctypes.data_as(_ip), selected.ctypes.data_as(_ip) if topk > 0 else None,
@@ -197,7 +199,7 @@ class Oracle:
 
 
     def muse_causal(self, Q, K, V, L, C, iters, seed, topk, scale=1.0, mode="dipole", hq_mask=None,
-                    q_assign_in=None, k_assign_in=None):
+                    q_assign_in=None, k_assign_in=None, key_stream0=0, query_stream0=0):
         """Causal MuSe (hierarchical blocks) in fp64.  Assignment layouts are
         [B,H,levels,N/2] (see the C file)."""
         Q, qp = _d(Q)
@@ -216,7 +218,8 @@ class Oracle:
         nprob = max(N // L - 1, 1)
         selected = np.full((B, Hq, nprob, C, max(topk, 1)), -1, dtype=np.int32)
         self.lib.orc_muse_causal(
-            qp, kp, vp, B, Hq, Hkv, N, D, L, C, iters, seed, topk, float(scale), MODES[mode],
+            qp, kp, vp, B, Hq, Hkv, N, D, L, C, iters, seed, key_stream0, query_stream0, topk,
+            float(scale), MODES[mode],
             m_p, qa_p, ka_p, O.ctypes.data_as(_dp), q_assign.ctypes.data_as(_ip),
             k_assign.ctypes.data_as(_ip),
             selected.ctypes.data_as(_ip) if topk > 0 and N // L > 1 else None,

@@ -459,14 +459,17 @@ static void finish(int nq, int D, const double *l, const double *acc, double *O)
 /* q_cent [B,Hq,Cq,D], k_cent [B,Hkv,Ck,D], k_count [B,Hkv,Ck],               */
 /* selected [B,Hq,Cq,k1], n_exact [B,Hq,N] (exact keys per query).            */
 /* q_assign_in / k_assign_in (optional) teacher-force the clusterings.        */
+/* ks0 / qs0: stream ids of the first key / query row set (0 for a whole     */
+/* layer): row set (b, h) draws the seeded start of stream ks0 + b Hkv + h.   */
 /* ------------------------------------------------------------------------ */
 void orc_muse_acausal(const double *Q, const double *K, const double *V, int B,
                       int Hq, int Hkv, int N, int D, int Cq, int Ck, int iters,
-                      uint64_t seed, int k1, double scale, int mode,
-                      const unsigned char *hq_mask, const int *q_assign_in,
-                      const int *k_assign_in, double *O, int *q_assign,
-                      int *k_assign, double *q_cent, double *k_cent,
-                      int *k_count, int *selected, long long *n_exact) {
+                      uint64_t seed, uint64_t ks0, uint64_t qs0, int k1,
+                      double scale, int mode, const unsigned char *hq_mask,
+                      const int *q_assign_in, const int *k_assign_in, double *O,
+                      int *q_assign, int *k_assign, double *q_cent,
+                      double *k_cent, int *k_count, int *selected,
+                      long long *n_exact) {
   const int G = Hq / Hkv;
 #pragma omp parallel for schedule(dynamic)
   for (int bk = 0; bk < B * Hkv; ++bk) {
@@ -478,7 +481,7 @@ void orc_muse_acausal(const double *Q, const double *K, const double *V, int B,
     size_t koff = (size_t)bk * N;
     key_block kb;
     make_keys(&kb, K + koff * D, V + koff * D, N, D, Ck, iters, seed,
-              (uint64_t)bk, k_assign_in ? k_assign_in + koff : NULL,
+              ks0 + (uint64_t)bk, k_assign_in ? k_assign_in + koff : NULL,
               mode == ORC_DIPOLE);
     if (k_assign) memcpy(k_assign + koff, kb.assign, sizeof(int) * (size_t)N);
     if (k_cent) memcpy(k_cent + (size_t)bk * Ck * D, kb.mu, sizeof(double) * (size_t)Ck * D);
@@ -488,7 +491,7 @@ void orc_muse_acausal(const double *Q, const double *K, const double *V, int B,
       if (hq_mask && !hq_mask[bq]) continue;
       size_t qoff = (size_t)bq * N;
       query_block qb;
-      make_queries(&qb, Q + qoff * D, N, D, Cq, iters, seed, (uint64_t)bq,
+      make_queries(&qb, Q + qoff * D, N, D, Cq, iters, seed, qs0 + (uint64_t)bq,
                    q_assign_in ? q_assign_in + qoff : NULL);
       double *m = (double *)malloc(sizeof(double) * (size_t)N);
       double *l = (double *)calloc((size_t)N, sizeof(double));
@@ -523,7 +526,8 @@ void orc_muse_acausal(const double *Q, const double *K, const double *V, int B,
 /* ------------------------------------------------------------------------ */
 void orc_muse_causal(const double *Q, const double *K, const double *V, int B,
                      int Hq, int Hkv, int N, int D, int L, int C, int iters,
-                     uint64_t seed, int k1, double scale, int mode,
+                     uint64_t seed, uint64_t ks0, uint64_t qs0, int k1,
+                     double scale, int mode,
                      const unsigned char *hq_mask, const int *q_assign_in,
                      const int *k_assign_in, double *O, int *q_assign,
                      int *k_assign, int *selected, long long *n_exact) {
@@ -554,7 +558,7 @@ void orc_muse_causal(const double *Q, const double *K, const double *V, int B,
       for (int p = 0; p < npairs; ++p) {
         int k0 = 2 * p * s, q0 = (2 * p + 1) * s;
         size_t slot = (size_t)lv * half + (size_t)p * s;
-        uint64_t ksid = ((uint64_t)bk * levels + lv) * pmax + p;
+        uint64_t ksid = ((ks0 + (uint64_t)bk) * levels + lv) * pmax + p;
         key_block kb;
         make_keys(&kb, Kh + (size_t)k0 * D, Vh + (size_t)k0 * D, s, D, Ce, iters,
                   seed, ksid,
@@ -566,7 +570,7 @@ void orc_muse_causal(const double *Q, const double *K, const double *V, int B,
           int hq = hk * G + g, bq = b * Hq + hq;
           if (hq_mask && !hq_mask[bq]) continue;
           const double *Qh = Q + (size_t)bq * N * D;
-          uint64_t qsid = ((uint64_t)bq * levels + lv) * pmax + p;
+          uint64_t qsid = ((qs0 + (uint64_t)bq) * levels + lv) * pmax + p;
           query_block qb;
           make_queries(&qb, Qh + (size_t)q0 * D, s, D, Ce, iters, seed, qsid,
                        q_assign_in ? q_assign_in + (size_t)bq * levels * half + slot : NULL);

@@ -502,3 +502,25 @@ def test_workload_causal_gqa_full_size(name):
     r_gpu = rse(O[0, GQA_HEADS][:, rows], E)
     r_orc = rse(np.stack([r["O"][0, h][rows] for h, r in zip(GQA_HEADS, rs)]), E)
     assert abs(r_gpu - r_orc) < 1e-3, (r_gpu, r_orc)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sharded_layer_equals_whole_layer_on_gpu(causal):
+    """The layer split into (batch, kv-head) units over 3 ranks, each shard run
+    by the CUDA operator with the whole layer's stream ids, reassembles to the
+    whole-layer output bit for bit.  The ranks run one after another on this
+    GPU (the path needs no exchange)."""
+    from clustered_multipole_approximation_b200 import sharding
+    Q, K, V = clustered_qkv(2, 8, 4, 1024, 64, 8, 0.3, 0.0, "bf16", 81)
+    q, k, v = to_dev(Q, "bf16"), to_dev(K, "bf16"), to_dev(V, "bf16")
+    kw = dict(iters=4, seed=9, topk=2, out_dtype=torch.float32)
+    kw.update(dict(C=12, block=128) if causal else dict(Cq=12, Ck=10))
+    fn = muse.muse_attn_fwd_causal if causal else muse.muse_attn_fwd
+    whole = fn(q, k, v, **kw)
+    world = 3
+    plan = sharding.partition(2, 4, world)
+    shards = [sharding.muse_attn_fwd_sharded(q, k, v, rank=r, world=world, causal=causal, **kw)[0]
+              for r in range(world)]
+    torch.cuda.synchronize()
+    O = sharding.assemble(shards, plan, 2, 8, 4)
+    assert torch.equal(O, whole)
