@@ -132,6 +132,9 @@ struct KState {
   int* emax;        // [nprob]       largest biased exponent of a value (bf16)
   double* part;     // [part_blocks][C][D] per-CTA partial centroid sums (resident k-means)
   int* pcnt;        // [part_blocks][C]    per-CTA member counts (resident k-means)
+  double* sum64;    // [nprob][C][D] resident k-means: exact running sums of the members
+  int* dirty;       // [nprob][C]    resident k-means: last round that changed the members
+  int* chg;         // [nprob][2]    resident k-means: tokens that changed cluster (round & 1)
   size_t part_blocks;
   int* err;         // device error word (0 = ok)
   int nprob;

@@ -21,15 +21,23 @@
 //   3. the queued tokens get the exact argmin among their candidates, each
 //      distance a plain sequential fp64 sum in dimension order (so ties
 //      resolve exactly as a sequential evaluation does);
-//   4. the CTA groups its tokens by cluster (stable counting sort) and sums
-//      each cluster's rows from shared memory in fp64, in any order: the
-//      exponent range of the problem's values, measured by the seeded-start
-//      kernel, certifies that every partial sum is exact (sums_exact), so
-//      the result equals a sequential fp64 sum bit for bit.  A problem that
-//      fails the certificate is left to the sequential-order kernel;
-//   5. the partial sums of the problem's CTAs meet in global memory (L2);
-//      after a cluster barrier the owner CTA of each centroid (c % NCT) adds
-//      them (exactly), divides by the count and writes the new centroid.
+//   4. first round: the CTA groups its tokens by cluster (stable counting
+//      sort) and sums each cluster's rows from shared memory in fp64, in any
+//      order: the exponent range of the problem's values, measured by the
+//      seeded-start kernel, certifies that every partial sum is exact
+//      (sums_exact), so the result equals a sequential fp64 sum bit for bit.
+//      A problem that fails the certificate is left to the sequential-order
+//      kernel.  The CTAs' partial sums meet in global memory (L2); after a
+//      team barrier the owner CTA of each centroid (c % NCT) adds them, keeps
+//      the exact total and the count as the problem's running state, and
+//      writes the new centroid;
+//   5. later rounds: only the tokens whose cluster changed move the running
+//      sums (fp64 atomic adds of +x and -x, exact in any order since every
+//      value passed through is the sum of a subset of the problem's tokens)
+//      and counts; after the barrier the owners recompute just the clusters
+//      whose members changed.  A round in which no token of the problem moved
+//      repeats the previous one exactly, and so would every later round: the
+//      problem ends there with the same result as running all rounds.
 // After the last round every CTA writes its tokens' assignments and its
 // members' places in the cluster-sorted permutation; the owners write the
 // counts and segment offsets.
@@ -206,17 +214,33 @@ __device__ inline void row_part(const unsigned char* tile, int r, int lane, floa
 }  // namespace
 
 // Phase clocks for tuning (compiled only with -DMUSE_PHASE_CLOCKS): thread 0
-// of every CTA adds the clock64 cycles of each phase to a per-CTA row.
+// of every CTA adds the clock64 cycles of each phase to a shared row, written
+// to a per-CTA global row when the CTA ends (slots 10..: event counts).
 #ifdef MUSE_PHASE_CLOCKS
-__device__ long long g_phase_clk[8192][12];
-#define PHASE_INIT long long ph_t = clock64()
+constexpr int kPhaseSlots = 16;
+__device__ long long g_phase_clk[8192][kPhaseSlots];
+#define PHASE_INIT                                            \
+  __shared__ long long ph_acc[kPhaseSlots];                   \
+  if (threadIdx.x < kPhaseSlots) ph_acc[threadIdx.x] = 0;     \
+  __syncthreads();                                            \
+  long long ph_t = clock64()
 #define PHASE(i)                                        \
   do {                                                  \
     if (threadIdx.x == 0) {                             \
       const long long t_ = clock64();                   \
-      g_phase_clk[blockIdx.x & 8191][i] += t_ - ph_t;   \
+      ph_acc[i] += t_ - ph_t;                           \
       ph_t = t_;                                        \
     }                                                   \
+  } while (0)
+#define PHASE_COUNT(i, v)                               \
+  do {                                                  \
+    if (threadIdx.x == 0) ph_acc[i] += (v);             \
+  } while (0)
+#define PHASE_FLUSH                                                          \
+  do {                                                                       \
+    __syncthreads();                                                         \
+    if (threadIdx.x < kPhaseSlots)                                           \
+      g_phase_clk[blockIdx.x & 8191][threadIdx.x] += ph_acc[threadIdx.x];    \
   } while (0)
 __device__ int g_bad[16];
 #define BADCHK(cond, code)                       \
@@ -230,6 +254,12 @@ __device__ int g_bad[16];
 #define PHASE_INIT
 #define PHASE(i) \
   do {           \
+  } while (0)
+#define PHASE_COUNT(i, v) \
+  do {                    \
+  } while (0)
+#define PHASE_FLUSH \
+  do {              \
   } while (0)
 #endif
 
@@ -302,7 +332,7 @@ __global__ void __launch_bounds__(kRT, 1) kmeans_resident_kernel(ResidentSets rs
   __shared__ uint32_t tmem_slot;
   __shared__ int scan_tmp[32];
   __shared__ float cmax_s;
-  __shared__ int qcount;
+  __shared__ int qcount, nchg_s;
   __shared__ int gtot[kNCFR], gbefore[kNCFR];
 
   if (warp == 0) {
@@ -459,8 +489,15 @@ __global__ void __launch_bounds__(kRT, 1) kmeans_resident_kernel(ResidentSets rs
       for (int k = wg; k < ntl; k += NACC) {
         const int kg = it * ntl + k, s = kg % NACC, use = kg / NACC;
         BADCHK(k < TPC && s < NACC, 8);
+#ifdef MUSE_PHASE_CLOCKS
+        const long long sw0 = clock64();
+#endif
         const bool ok = __all_sync(0xffffffffu, mbar_wait(sa(&mma_done[s]), (uint32_t)(use & 1)));
         tc_after();
+#ifdef MUSE_PHASE_CLOCKS
+        const long long sw1 = clock64();
+        PHASE_COUNT(14, sw1 - sw0);
+#endif
         const int u = k * kTile + row;  // CTA-local token of this thread's row
         const bool live = u < ntok;
         const uint32_t tm = tbase + (uint32_t)(s * NC) + ((uint32_t)(q4 * 32) << 16);
@@ -553,6 +590,9 @@ __global__ void __launch_bounds__(kRT, 1) kmeans_resident_kernel(ResidentSets rs
         tc_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(sa(&acc_free[s]));
+#ifdef MUSE_PHASE_CLOCKS
+        PHASE_COUNT(15, clock64() - sw1);
+#endif
       }
     }
     __syncthreads();
@@ -579,7 +619,7 @@ __global__ void __launch_bounds__(kRT, 1) kmeans_resident_kernel(ResidentSets rs
         const unsigned ncc = e < kCandCap ? ccnt[e] : kFull;
         const bool full = ncc == kFull;
 #ifdef MUSE_PHASE_CLOCKS
-        if (lane == 0) atomicAdd(reinterpret_cast<unsigned long long*>(&g_phase_clk[blockIdx.x & 8191][10]),
+        if (lane == 0) atomicAdd(reinterpret_cast<unsigned long long*>(&ph_acc[10]),
                                  full ? 1000ull : (unsigned long long)ncc);
 #endif
         const int nc = full ? C : (int)ncc;  // every cluster when the band was not recorded
@@ -627,12 +667,10 @@ __global__ void __launch_bounds__(kRT, 1) kmeans_resident_kernel(ResidentSets rs
     }
     __syncthreads();
     PHASE(3);
-#ifdef MUSE_PHASE_CLOCKS
-    if (tid == 0) g_phase_clk[blockIdx.x & 8191][11] += qcount;
-#endif
+    PHASE_COUNT(11, qcount);
 
-    // ---- 4. group this CTA's tokens by cluster (stable) ------------------------
-    {
+    // ---- 4. group this CTA's tokens by cluster (stable): lst, loff ------------
+    auto group = [&]() {
       const int per = cdiv(cdiv(ntok > 0 ? ntok : 1, kRW), 32) * 32;
       const int lo = imin(ntok, warp * per), hi = imin(ntok, lo + per);
       int* wh = whist + warp * NC;
@@ -674,14 +712,12 @@ __global__ void __launch_bounds__(kRT, 1) kmeans_resident_kernel(ResidentSets rs
         if (a >= 0 && __ffs(same) - 1 == lane) wh[a] += __popc(same);
         __syncwarp();
       }
-      if (last)
-        for (int t = tid; t < ntok; t += kRT) ks.assign[p.slot0 + tok0 + t] = asg[t];
       __syncthreads();
-    }
-    PHASE(4);
+    };
 
-    // ---- 5. cluster sums of this CTA's members, from the resident rows ---------
-    // (exact in any order: sums_exact holds for this problem)
+    // ---- 5. the problem's exact cluster sums ----------------------------------
+    // (exact in any order: sums_exact holds for this problem, and every value
+    // a sum passes through below is the sum of a subset of its tokens)
     auto write_centroid = [&](int c, int n, const double (&acc)[VPL]) {
       const double nn = (double)n;
       double q2 = 0.0;
@@ -718,96 +754,216 @@ __global__ void __launch_bounds__(kRT, 1) kmeans_resident_kernel(ResidentSets rs
         ks.cn2[cbase + c] = (float)q2;
       }
     };
-    // lane l holds dimensions l * VPL .. l * VPL + VPL - 1 of every sum
-    const size_t pslot = ((size_t)(blk / NCT) * NCT + rank) * g.C;  // this CTA's partial row block
-    for (int c = warp; c < C; c += kRW) {
-      const int m0 = loff[c], n = loff[c + 1] - m0;
-      double acc[VPL], acc2[VPL];
+    // The running state of the problem in global memory: sum64[c] = the exact
+    // sum of cluster c's members, counts[c] their number, dirty[c] = the last
+    // round whose membership changes touched c, chg[round & 1] the tokens
+    // that changed cluster in that round.
+    double* sumg = ks.sum64 + cbase * D;
+    int* cntg = ks.counts + cbase;
+    int* dirt = ks.dirty + cbase;
+    int* chgp = ks.chg + (size_t)pid * 2;
+    bool fin = last;
+    if (it == 0) {
+      // first round: every member summed, from the grouped rows
+      group();
+      PHASE(4);
+      // lane l holds dimensions l * VPL .. l * VPL + VPL - 1 of every sum
+      const size_t pslot = ((size_t)(blk / NCT) * NCT + rank) * g.C;  // this CTA's partial row block
+      for (int c = warp; c < C; c += kRW) {
+        const int m0 = loff[c], n = loff[c + 1] - m0;
+        double acc[VPL], acc2[VPL];
 #pragma unroll
-      for (int e = 0; e < VPL; ++e) acc[e] = acc2[e] = 0.0;
-      // four members per step, every row load issued before the first add
-      constexpr int MB = 4;
-      for (int j0 = 0; j0 < n; j0 += MB) {
-        float a[MB][VPL];
+        for (int e = 0; e < VPL; ++e) acc[e] = acc2[e] = 0.0;
+        // four members per step, every row load issued before the first add
+        constexpr int MB = 4;
+        for (int j0 = 0; j0 < n; j0 += MB) {
+          float a[MB][VPL];
 #pragma unroll
-        for (int m = 0; m < MB; ++m) {
-          if (j0 + m < n) {
-            const int u = lst[m0 + j0 + m];
-            row_part<D>(T + (u >> 7) * TILEB, u & (kTile - 1), lane, a[m]);
-          } else {
+          for (int m = 0; m < MB; ++m) {
+            if (j0 + m < n) {
+              const int u = lst[m0 + j0 + m];
+              row_part<D>(T + (u >> 7) * TILEB, u & (kTile - 1), lane, a[m]);
+            } else {
 #pragma unroll
-            for (int e = 0; e < VPL; ++e) a[m][e] = 0.f;
+              for (int e = 0; e < VPL; ++e) a[m][e] = 0.f;
+            }
           }
+#pragma unroll
+          for (int m = 0; m < MB; m += 2)
+#pragma unroll
+            for (int e = 0; e < VPL; ++e) {
+              acc[e] = __dadd_rn(acc[e], (double)a[m][e]);
+              acc2[e] = __dadd_rn(acc2[e], (double)a[m + 1][e]);
+            }
         }
 #pragma unroll
-        for (int m = 0; m < MB; m += 2)
-#pragma unroll
-          for (int e = 0; e < VPL; ++e) {
-            acc[e] = __dadd_rn(acc[e], (double)a[m][e]);
-            acc2[e] = __dadd_rn(acc2[e], (double)a[m + 1][e]);
-          }
-      }
-#pragma unroll
-      for (int e = 0; e < VPL; ++e) acc[e] = __dadd_rn(acc[e], acc2[e]);
-      if (NCT == 1) {
-        if (n > 0) write_centroid(c, n, acc);  // an empty cluster keeps its centroid
-      } else {
-        BADCHK(pslot / g.C < (size_t)ks.part_blocks, 5);
-        if (lane == 0) rs.pcnt[set][pslot + c] = n;
-        if (n > 0) {
-          double* pr = rs.part[set] + (pslot + c) * D + (size_t)lane * VPL;
+        for (int e = 0; e < VPL; ++e) acc[e] = __dadd_rn(acc[e], acc2[e]);
+        if (NCT == 1) {
+          double* sr = sumg + (size_t)c * D + (size_t)lane * VPL;
 #pragma unroll
           for (int e = 0; e < VPL / 2; ++e)
-            reinterpret_cast<double2*>(pr)[e] = make_double2(acc[2 * e], acc[2 * e + 1]);
-        }
-      }
-    }
-    __syncthreads();
-    PHASE(5);
-    if (NCT > 1) {
-      team_sync();
-      if (MODE == 2 && bar_fail) break;
-      PHASE(6);
-      // ---- owners: add the problem's partial sums (exact), write centroids ------
-      const size_t pbase = (size_t)(blk / NCT) * NCT * g.C;
-      for (int c = rank + NCT * warp; c < C; c += NCT * kRW) {
-        const int cnt = lane < NCT ? __ldcg(rs.pcnt[set] + pbase + (size_t)lane * g.C + c) : 0;
-        double acc[VPL];
-#pragma unroll
-        for (int e = 0; e < VPL; ++e) acc[e] = 0.0;
-        // eight ranks' rows in flight; a rank without members left no row
-        for (int r0 = 0; r0 < NCT; r0 += 8) {
-          double2 v[8][VPL / 2];
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const int rr = r0 + m < NCT ? r0 + m : NCT - 1;  // never past the problem's blocks
-            const double* pr = rs.part[set] + (pbase + (size_t)rr * g.C + c) * D + (size_t)lane * VPL;
+            reinterpret_cast<double2*>(sr)[e] = make_double2(acc[2 * e], acc[2 * e + 1]);
+          if (lane == 0) {
+            cntg[c] = n;
+            dirt[c] = 0;
+          }
+          if (n > 0) write_centroid(c, n, acc);  // an empty cluster keeps its centroid
+        } else {
+          BADCHK(pslot / g.C < (size_t)ks.part_blocks, 5);
+          if (lane == 0) rs.pcnt[set][pslot + c] = n;
+          if (n > 0) {
+            double* pr = rs.part[set] + (pslot + c) * D + (size_t)lane * VPL;
 #pragma unroll
             for (int e = 0; e < VPL / 2; ++e)
-              v[m][e] = r0 + m < NCT ? __ldcg(reinterpret_cast<const double2*>(pr) + e) : make_double2(0.0, 0.0);
+              reinterpret_cast<double2*>(pr)[e] = make_double2(acc[2 * e], acc[2 * e + 1]);
           }
+        }
+      }
+      __syncthreads();
+      PHASE(5);
+      if (NCT > 1) {
+        team_sync();
+        if (MODE == 2 && bar_fail) break;
+        PHASE(6);
+        // owners: add the problem's partial sums (exact), write centroids
+        const size_t pbase = (size_t)(blk / NCT) * NCT * g.C;
+        for (int c = rank + NCT * warp; c < C; c += NCT * kRW) {
+          const int cnt = lane < NCT ? __ldcg(rs.pcnt[set] + pbase + (size_t)lane * g.C + c) : 0;
+          double acc[VPL];
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const int cm = __shfl_sync(0xffffffffu, cnt, (r0 + m) & 31);
-            if (r0 + m < NCT && cm > 0) {
+          for (int e = 0; e < VPL; ++e) acc[e] = 0.0;
+          // eight ranks' rows in flight; a rank without members left no row
+          for (int r0 = 0; r0 < NCT; r0 += 8) {
+            double2 v[8][VPL / 2];
 #pragma unroll
-              for (int e = 0; e < VPL / 2; ++e) {
-                acc[2 * e] = __dadd_rn(acc[2 * e], v[m][e].x);
-                acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], v[m][e].y);
+            for (int m = 0; m < 8; ++m) {
+              const int rr = r0 + m < NCT ? r0 + m : NCT - 1;  // never past the problem's blocks
+              const double* pr = rs.part[set] + (pbase + (size_t)rr * g.C + c) * D + (size_t)lane * VPL;
+#pragma unroll
+              for (int e = 0; e < VPL / 2; ++e)
+                v[m][e] = r0 + m < NCT ? __ldcg(reinterpret_cast<const double2*>(pr) + e) : make_double2(0.0, 0.0);
+            }
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+              const int cm = __shfl_sync(0xffffffffu, cnt, (r0 + m) & 31);
+              if (r0 + m < NCT && cm > 0) {
+#pragma unroll
+                for (int e = 0; e < VPL / 2; ++e) {
+                  acc[2 * e] = __dadd_rn(acc[2 * e], v[m][e].x);
+                  acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], v[m][e].y);
+                }
               }
             }
           }
+          int n = cnt;
+          for (int o = 16; o; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+          double* sr = sumg + (size_t)c * D + (size_t)lane * VPL;
+#pragma unroll
+          for (int e = 0; e < VPL / 2; ++e)
+            reinterpret_cast<double2*>(sr)[e] = make_double2(acc[2 * e], acc[2 * e + 1]);
+          if (lane == 0) {
+            cntg[c] = n;
+            dirt[c] = 0;
+          }
+          if (n > 0) write_centroid(c, n, acc);
         }
-        int n = cnt;
-        for (int o = 16; o; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-        if (n == 0) continue;
-        write_centroid(c, n, acc);
+      }
+      // the change counter of the next round starts from zero (its slot was
+      // last read before the previous round's closing barrier)
+      if (rank == 0 && tid == 0) chgp[1] = 0;
+    } else {
+      // later rounds: only the tokens that changed cluster move the sums; a
+      // warp takes one such token, lane l dimensions l, l + 32, ...
+      if (tid == 0) nchg_s = 0;
+      __syncthreads();
+      for (int u0 = 0; u0 < ntok; u0 += kRT) {
+        const int u = u0 + tid;
+        const bool moved = u < ntok && asg[u] != lst[u];  // lst holds the previous round's clusters
+        const unsigned bal = __ballot_sync(0xffffffffu, moved);
+        int slot = 0;
+        if (lane == 0 && bal) slot = atomicAdd(&nchg_s, __popc(bal));
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+        if (moved) queue[slot + __popc(bal & ((1u << lane) - 1u))] = (unsigned short)u;
+      }
+      __syncthreads();
+      const int nmv = nchg_s;
+      for (int e = warp; e < nmv; e += kRW) {
+        const int u = queue[e];
+        const int a = asg[u], b = lst[u];
+        const unsigned char* tile = T + (u >> 7) * TILEB;
+        const int r = u & (kTile - 1);
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+          const int d = lane + 32 * j, kb = d >> 6, dd = d & 63;
+          const unsigned short h =
+              *reinterpret_cast<const unsigned short*>(tile + kb * kTile * 128 + swz(r, dd >> 3) + (dd & 7) * 2);
+          const double x = (double)__uint_as_float((uint32_t)h << 16);
+          atomicAdd(sumg + (size_t)a * D + d, x);
+          atomicAdd(sumg + (size_t)b * D + d, -x);
+        }
+        if (lane == 0) {
+          atomicAdd(cntg + a, 1);
+          atomicAdd(cntg + b, -1);
+          dirt[a] = it;
+          dirt[b] = it;
+        }
+      }
+      __syncthreads();
+      for (int e = tid; e < nmv; e += kRT) {
+        const int u = queue[e];
+        lst[u] = asg[u];
+      }
+      if (tid == 0 && nmv > 0) atomicAdd(chgp + (it & 1), nmv);
+      PHASE_COUNT(12, nmv);
+      PHASE(5);
+      if (MODE == 0) {
+        __threadfence();
+        __syncthreads();
+      } else {
+        team_sync();
+        if (MODE == 2 && bar_fail) break;
+      }
+      PHASE(6);
+      // every CTA of the problem reads the same total after the barrier: no
+      // token moved means the centroids are those of the previous round, and
+      // every later round would repeat this one exactly
+      const int moved_all = __ldcg(chgp + (it & 1));
+      fin = last || moved_all == 0;
+      if (rank == 0 && tid == 0) chgp[(it + 1) & 1] = 0;
+      if (moved_all > 0) {
+        // owners: new centroids of the clusters whose membership changed
+        for (int c = rank + NCT * warp; c < C; c += NCT * kRW) {
+          if (__ldcg(dirt + c) != it) continue;
+          const int n = __ldcg(cntg + c);
+          if (n == 0) continue;  // an empty cluster keeps its centroid
+          double acc[VPL];
+          const double* sr = sumg + (size_t)c * D + (size_t)lane * VPL;
+#pragma unroll
+          for (int e = 0; e < VPL / 2; ++e) {
+            const double2 v = __ldcg(reinterpret_cast<const double2*>(sr) + e);
+            acc[2 * e] = v.x;
+            acc[2 * e + 1] = v.y;
+          }
+          write_centroid(c, n, acc);
+        }
       }
     }
     __syncthreads();
     PHASE(7);
     // ---- last round: counts, offsets, the cluster-sorted permutation -----------
-    if (last) {
+    if (fin) {
+      PHASE_COUNT(13, it + 1);
+      if (it > 0) {
+        group();
+        if (NCT > 1) {
+          const size_t pslot = ((size_t)(blk / NCT) * NCT + rank) * g.C;
+          for (int c = tid; c < C; c += kRT) rs.pcnt[set][pslot + c] = loff[c + 1] - loff[c];
+          __syncthreads();
+          team_sync();
+          if (MODE == 2 && bar_fail) break;
+        }
+      }
+      for (int t = tid; t < ntok; t += kRT) ks.assign[p.slot0 + tok0 + t] = asg[t];
       // members of every cluster in the problem, and in the CTAs before this one
       const size_t pbase = (size_t)(blk / NCT) * NCT * g.C;
       for (int c = tid; c < C; c += kRT) {
@@ -842,6 +998,11 @@ __global__ void __launch_bounds__(kRT, 1) kmeans_resident_kernel(ResidentSets rs
         BADCHK(gtot[c] + gbefore[c] + n <= p.s, 4);
         for (int j = lane; j < n; j += 32) ks.perm[at + j] = tok0 + lst[m0 + j];
       }
+      PHASE(8);
+      break;
+    }
+    if (it == 0) {  // lst keeps each token's cluster of the previous round from here on
+      for (int t = tid; t < ntok; t += kRT) lst[t] = asg[t];
     }
     __syncthreads();
     PHASE(8);
@@ -849,6 +1010,7 @@ __global__ void __launch_bounds__(kRT, 1) kmeans_resident_kernel(ResidentSets rs
     if (MODE == 2 && bar_fail) break;
     PHASE(9);
   }
+  PHASE_FLUSH;
   // no MMA may still write the accumulators when they are freed: the MMA warp
   // waits (bounded) for the last commit of every slot of the last round
   if (warp == kEW && lane == 0 && issued > 0) {
@@ -889,6 +1051,12 @@ static int nct_cap(int ntp, int nprob, int tpc_max) {
   return cap < ntp ? cap : ntp;
 }
 
+bool resident_serves(const Levels& lv, int D, int C) {
+  for (int l = 0; l < lv.nlev; ++l)
+    if (resident_tpc_max(D, imin(C, lv.s[l])) >= 4) return true;
+  return false;
+}
+
 size_t resident_partial_blocks(const Levels& lv, int BH, int D, int C) {
   const int tmax = resident_tpc_max(D, C);
   if (tmax < 4) return 0;  // the resident kernel does not serve these sizes
@@ -918,7 +1086,7 @@ static bool resident_t(const RoleGeo* gs, const KState* kss, int nsets, int lvl,
                        cudaStream_t st) {
   int cmax = 0, ntp = 1, nprob = 0, np[2] = {0, 0};
   for (int k = 0; k < nsets; ++k) {
-    if (gs[k].dtype != 0 || gs[k].C > kNCFR || gs[k].D != D) return false;
+    if (gs[k].dtype != 0 || gs[k].C > kNCFR || gs[k].D != D || kss[k].sum64 == nullptr) return false;
     const int l0 = lvl < 0 ? 0 : lvl;
     const int ce = imin(gs[k].C, gs[k].lv.s[l0]);
     cmax = cmax > ce ? cmax : ce;
@@ -1091,11 +1259,11 @@ static bool launch_resident(const RoleGeo* gs, const KState* kss, int nsets, int
 
 #ifdef MUSE_PHASE_CLOCKS
 extern "C" void muse_phase_read(long long* out, int rows) {
-  cudaMemcpyFromSymbol(out, g_phase_clk, (size_t)rows * 12 * sizeof(long long));
+  cudaMemcpyFromSymbol(out, g_phase_clk, (size_t)rows * kPhaseSlots * sizeof(long long));
 }
 extern "C" void muse_bad_read(int* out) { cudaMemcpyFromSymbol(out, g_bad, sizeof(g_bad)); }
 extern "C" void muse_phase_clear(void) {
-  static long long zero[8192][12];
+  static long long zero[8192][kPhaseSlots];
   cudaMemcpyToSymbol(g_phase_clk, zero, sizeof(zero));
 }
 #endif
