@@ -113,7 +113,8 @@ void carve_kstate(Carver& cv, KState& ks, const RoleGeo& g) {
   ks.part_blocks = g.dtype == 0 ? resident_partial_blocks(g.lv, g.BH, g.D, g.C) : 0;
   ks.part = cv.take<double>(ks.part_blocks * C * D * 8);
   ks.pcnt = cv.take<int>(ks.part_blocks * C * 4);
-  const bool res = g.dtype == 0 && resident_serves(g.lv, g.D, g.C);
+  // running-sum tables of the persistent k-means kernels (bf16, C <= 256)
+  const bool res = g.dtype == 0 && g.C <= 256;
   ks.sum64 = res ? cv.take<double>(np * C * D * 8) : nullptr;
   ks.dirty = res ? cv.take<int>(np * C * 4) : nullptr;
   ks.chg = res ? cv.take<int>(np * 2 * 4) : nullptr;

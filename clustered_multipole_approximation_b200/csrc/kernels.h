@@ -81,9 +81,6 @@ bool launch_kmeans_resident(const RoleGeo* gs, const KState* kss, int nsets, int
                             cudaStream_t st);
 // Partial-sum blocks the resident k-means may need for one role's levels.
 size_t resident_partial_blocks(const Levels& lv, int BH, int D, int C);
-// Whether the resident k-means may serve some level of these sizes (its
-// running-sum tables are carved only then).
-bool resident_serves(const Levels& lv, int D, int C);
 
 // Lloyd rounds one launch sequence at a time (any dtype / size).
 void run_kmeans_rounds(const RoleGeo& g, const KState& ks, int iters, cudaStream_t st);

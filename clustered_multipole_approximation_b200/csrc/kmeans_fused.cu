@@ -56,6 +56,8 @@ int g_spin_limit = kSpinLimit;
 int g_no_resident = 0;
 constexpr int kOT = kNCF + kMaxNCT;  // (owned cluster, rank) pairs per CTA, at most
 constexpr int kTilesPerCta = 16;     // cluster launches: target tiles per CTA
+constexpr int kFCandCap = 128;       // queued tokens per round with a candidate list
+constexpr int kFMaxCand = 8;         // candidates kept per queued token
 constexpr size_t kSmemLimit = 218 * 1024;  // dynamic shared memory (static arrays come on top)
 
 __device__ inline uint32_t saddr(const void* p) {
@@ -114,7 +116,7 @@ __device__ inline void fence_async_smem() { asm volatile("fence.proxy.async.shar
 // keeps two token tiles in shared memory instead of three (large C and D).
 struct FusedLayout {
   int KB, NC, tpc, flags;  // K-blocks, centroid columns (multiple of 32), tiles per CTA
-  size_t a, bh, bl, cn2, xs, whist, loff, gtab, xn, asg, queue, cst, total;
+  size_t a, bh, bl, cn2, xs, whist, loff, gtab, xn, asg, queue, cand, ccnt, cst, total;
 };
 
 __host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc, int flags) {
@@ -139,6 +141,9 @@ __host__ __device__ inline FusedLayout fused_layout(int D, int NC, int tpc, int 
   L.xn = o;    o += (size_t)tpc * kTile * 4;          // token norms (screen bound)
   L.asg = o;   o += (size_t)tpc * kTile * 2;
   L.queue = o; o += (size_t)tpc * kTile * 2;
+  L.cand = o;  o += (size_t)kFCandCap * kFMaxCand * 2;  // candidate clusters of queued tokens
+  o = (o + 15) & ~(size_t)15;
+  L.ccnt = o;  o += (size_t)kFCandCap * 4;              // their counts (> kFMaxCand: every cluster)
   o = (o + 15) & ~(size_t)15;
   L.cst = o;                                          // fp64 centroids, row stride D + 1
   if (flags & 1) o += (size_t)NC * (D + 1) * 8;
@@ -286,6 +291,8 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
   float* xns = reinterpret_cast<float*>(base + Lo.xn);
   unsigned short* asg = reinterpret_cast<unsigned short*>(base + Lo.asg);
   unsigned short* queue = reinterpret_cast<unsigned short*>(base + Lo.queue);
+  unsigned short* cand = reinterpret_cast<unsigned short*>(base + Lo.cand);
+  int* ccnt = reinterpret_cast<int*>(base + Lo.ccnt);
   double* cst = reinterpret_cast<double*>(base + Lo.cst);
   __shared__ __align__(8) uint64_t mbar[2];
   __shared__ uint32_t tmem_slot;
@@ -404,9 +411,63 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
     mma_commit(saddr(&mbar[buf]));
   };
   auto tile_buf = [&](int k) { return A0 + (k % ring) * ATILE; };
+  // new centroid c = acc / n (lane l: dimensions l VPL ..): fp64, fp32, bf16
+  // hi / lo split and norms
+  auto write_centroid = [&](int c, int n, const double (&acc)[VPL]) {
+    const double nn = (double)n;
+    double q2 = 0.0;
+    float qf = 0.f;
+    double v64[VPL];
+    float v32[VPL];
+    uint32_t wh[VPL / 2], wl[VPL / 2];
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) {
+      v64[e] = __ddiv_rn(acc[e], nn);
+      v32[e] = (float)v64[e];
+      q2 += v64[e] * v64[e];
+      qf = fmaf(v32[e], v32[e], qf);
+    }
+#pragma unroll
+    for (int e = 0; e < VPL / 2; ++e) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(v32[2 * e]);
+      const __nv_bfloat16 h1 = __float2bfloat16_rn(v32[2 * e + 1]);
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(v32[2 * e] - __bfloat162float(h0));
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(v32[2 * e + 1] - __bfloat162float(h1));
+      wh[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+      wl[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+    }
+    const size_t i0 = (cbase + c) * D + (size_t)lane * VPL;
+#pragma unroll
+    for (int e = 0; e < VPL / 2; ++e) {
+      reinterpret_cast<double2*>(ks.cent64 + i0)[e] = make_double2(v64[2 * e], v64[2 * e + 1]);
+      reinterpret_cast<float2*>(ks.cent32 + i0)[e] = make_float2(v32[2 * e], v32[2 * e + 1]);
+      reinterpret_cast<uint32_t*>(ks.cbf_hi + i0)[e] = wh[e];
+      reinterpret_cast<uint32_t*>(ks.cbf_lo + i0)[e] = wl[e];
+    }
+    for (int o = 16; o; o >>= 1) {
+      qf += __shfl_xor_sync(0xffffffffu, qf, o);
+      q2 += __shfl_xor_sync(0xffffffffu, q2, o);
+    }
+    if (lane == 0) {
+      ks.cnorm[cbase + c] = sqrtf(qf) * 1.0001f;
+      ks.cn2[cbase + c] = (float)q2;
+    }
+  };
+  // Problems whose sums are certified exact in any order keep a running
+  // state after the first round (sum64 = exact member sums, counts, dirty =
+  // last round that changed the members, chg = tokens that moved): later
+  // rounds move only the changed tokens' rows, and a round without moves
+  // ends the problem (every later round would repeat it exactly).
+  const bool cert = ks.sum64 != nullptr && sums_exact(ks, pid, p.s);
+  double* sumg = cert ? ks.sum64 + cbase * D : nullptr;
+  int* cntg = ks.counts + cbase;
+  int* dirt = cert ? ks.dirty + cbase : nullptr;
+  int* chgp = cert ? ks.chg + (size_t)pid * 2 : nullptr;
+  __shared__ int nmv_s;
 
   for (int it = 0; it < iters; ++it) {
     const bool last = it + 1 == iters;
+    bool fin = last;  // the problem's final round
     // ---- centroids of this round (bf16 split, tensor-core operand) ----------
     for (int e = tid; e < ncp * KB * 8; e += kFT) {
       const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, cq = q & 7;
@@ -559,14 +620,56 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         const float xn = xns[u];
         const float E = 2.f * 3.0517578e-05f * xn * cm + 2.3841858e-07f * (cm * cm + 2.f * xn * cm);
         asg[u] = (unsigned short)bi;
-        if (!ok || (b2 - b1) <= 2.f * E) queue[atomicAdd(&qcount, 1)] = (unsigned short)u;
+        const bool queued = !ok || (b2 - b1) <= 2.f * E;
+        int qi = -1;
+        if (queued) {
+          qi = atomicAdd(&qcount, 1);
+          queue[qi] = (unsigned short)u;
+          if (qi < kFCandCap) ccnt[qi] = ok ? 0 : kFMaxCand + 1;  // unusable screen: every cluster
+        }
+        // the band of a queued row for the candidate scan below (the merged
+        // best and runner-up are read; hb2 / hbi now carry the band and slot)
+        hb2[row] = (queued && ok && qi < kFCandCap) ? b1 + 2.f * E : -INFINITY;
+        hbi[row] = qi;
+      } else if (half == 0) {
+        hb2[row] = -INFINITY;
+      }
+      __syncthreads();
+      // ---- candidates of the queued rows: every column inside the band, both
+      // column halves, while the tile's accumulator is still in TMEM (the next
+      // MMA into this buffer is issued after the next loop-top barrier) --------
+      {
+        const float lim = hb2[row];
+        const bool rec = lim > -INFINITY;
+        if (__any_sync(0xffffffffu, rec)) {
+          const int qi = hbi[row];
+          for (int c0 = half * hw; c0 < (half + 1) * hw; c0 += 16) {  // hw: a multiple of 16
+            uint32_t rv[16];
+            tmem_ld16_nw(tm + (uint32_t)c0, rv);
+            tmem_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c = c0 + e;
+              const float dd = fmaf(-2.f, __uint_as_float(rv[e]), cn2s[c]);
+              if (rec && dd <= lim) {
+                const int k = atomicAdd(&ccnt[qi], 1);
+                if (k < kFMaxCand) cand[qi * kFMaxCand + k] = (unsigned short)c;
+              }
+            }
+          }
+        }
       }
     }
     __syncthreads();
     // ---- exact fp64 decision of the queued tokens, one warp per token --------
     const int qn = qcount;
+    // tokens without a usable candidate list: an exact argmin over every cluster
+    bool any_full = qn > kFCandCap;
+    for (int e = tid; e < qn && e < kFCandCap; e += kFT)
+      if (ccnt[e] < 1 || ccnt[e] > kFMaxCand) any_full = true;
+    any_full = __syncthreads_or(any_full);
     if (qn > 0) {
-      if (stage & 1) {
+      if ((stage & 1) && any_full) {
         const int tot = C * D;
         for (int e0 = tid; e0 < tot; e0 += 16 * kFT) {  // 16 loads in flight per thread
           double v[16];
@@ -589,12 +692,104 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         const __nv_bfloat16* xr = X + (p.row0 + tok0 + uq) * D;
         for (int d = lane; d < D; d += 32) xw[d] = (double)__bfloat162float(xr[d]);
         __syncwarp();
-        const int bc = (stage & 1) ? exact_argmin<D, true>(xw, cst, c64g, C, lane)
-                             : exact_argmin<D, false>(xw, cst, c64g, C, lane);
+        const int nc = e < kFCandCap ? ccnt[e] : kFMaxCand + 1;
+        int bc;
+        if (nc >= 1 && nc <= kFMaxCand) {
+          // the exact winner lies in the band: one candidate per lane, each a
+          // plain sequential fp64 distance in dimension order
+          double bd = 0.0;
+          bc = -1;
+          if (lane < nc) {
+            const int c = cand[e * kFMaxCand + lane];
+            const double* cr = c64g + (size_t)c * D;
+            double sd = 0.0;
+#pragma unroll 16
+            for (int d = 0; d < D; ++d) {
+              const double t = __dsub_rn(xw[d], __ldcg(cr + d));
+              sd = __dadd_rn(sd, __dmul_rn(t, t));
+            }
+            bd = sd;
+            bc = c;
+          }
+          for (int o = 16; o; o >>= 1) {
+            const double od = __shfl_xor_sync(0xffffffffu, bd, o);
+            const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+            if (oc >= 0 && (bc < 0 || od < bd || (od == bd && oc < bc))) {
+              bd = od;
+              bc = oc;
+            }
+          }
+        } else {
+          bc = ((stage & 1) && any_full) ? exact_argmin<D, true>(xw, cst, c64g, C, lane)
+                                         : exact_argmin<D, false>(xw, cst, c64g, C, lane);
+        }
         if (lane == 0) asg[uq] = (unsigned short)bc;
         __syncwarp();
       }
       __syncthreads();
+    }
+    if (cert && it > 0) {
+      // ---- the tokens that changed cluster move the running sums ---------------
+      // (ks.assign holds every token's cluster of the previous round)
+      if (tid == 0) nmv_s = 0;
+      __syncthreads();
+      int* asg_g = ks.assign + p.slot0 + tok0;
+      for (int u0 = 0; u0 < ntok; u0 += kFT) {
+        const int u = u0 + tid;
+        const bool moved = u < ntok && (int)asg[u] != __ldcg(asg_g + u);
+        const unsigned bal = __ballot_sync(0xffffffffu, moved);
+        int slot = 0;
+        if (lane == 0 && bal) slot = atomicAdd(&nmv_s, __popc(bal));
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+        if (moved) queue[slot + __popc(bal & ((1u << lane) - 1u))] = (unsigned short)u;
+      }
+      __syncthreads();
+      const int nmv = nmv_s;
+      for (int e = warp; e < nmv; e += kWarps) {
+        const int u = queue[e];
+        const int a = asg[u], b = __ldcg(asg_g + u);
+        const __nv_bfloat16* xr = X + (p.row0 + tok0 + u) * D;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+          const int d = lane + 32 * j;
+          const double x = (double)__bfloat162float(xr[d]);
+          atomicAdd(sumg + (size_t)a * D + d, x);
+          atomicAdd(sumg + (size_t)b * D + d, -x);
+        }
+        if (lane == 0) {
+          atomicAdd(cntg + a, 1);
+          atomicAdd(cntg + b, -1);
+          dirt[a] = it;
+          dirt[b] = it;
+        }
+      }
+      __syncthreads();
+      for (int e = tid; e < nmv; e += kFT) {
+        const int u = queue[e];
+        asg_g[u] = asg[u];
+      }
+      if (tid == 0 && nmv > 0) atomicAdd(chgp + (it & 1), nmv);
+      team_sync();
+      if (bar_fail) break;
+      // every CTA of the problem reads the same total after the barrier
+      const int moved_all = __ldcg(chgp + (it & 1));
+      fin = last || moved_all == 0;
+      if (rank == 0 && tid == 0) chgp[(it + 1) & 1] = 0;
+      if (!fin) {
+        // owners: new centroids of the clusters whose members changed
+        for (int c = rank + NCT * warp; c < C; c += NCT * kWarps) {
+          const int n = __ldcg(dirt + c) == it ? __ldcg(cntg + c) : 0;
+          if (n == 0) continue;  // unchanged members, or an empty cluster: the centroid stays
+          double acc[VPL];
+          const double* sr = sumg + (size_t)c * D + (size_t)lane * VPL;
+#pragma unroll
+          for (int e = 0; e < VPL; ++e) acc[e] = __ldcg(sr + e);
+          write_centroid(c, n, acc);
+        }
+        team_sync();
+        if (bar_fail) break;
+        continue;
+      }
     }
     // ---- group this CTA's tokens by cluster (stable) and publish the list ----
     {
@@ -640,13 +835,13 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         if (a >= 0 && __ffs(same) - 1 == lane) wh[a] += __popc(same);
         __syncwarp();
       }
-      if (last)
+      if (fin || cert)
         for (int t = tid; t < ntok; t += kFT) ks.assign[p.slot0 + tok0 + t] = asg[t];
     }
     team_sync();
     if (bar_fail) break;
     // ---- owners: counts, offsets, means over all CTAs' members ----------------
-    if (last) {
+    if (fin) {
       for (int c = tid; c < C; c += kFT) goff[c] = 0;
       __syncthreads();
       for (int k = tid; k < C * nra; k += kFT) {  // (cluster, rank) pairs
@@ -724,7 +919,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
           while (gP[cur + 1] <= j) ++cur;
           return cur * tpc * kTile + (int)__ldcg(tl + gB[cur] + (j - gP[cur]));
         };
-        const size_t pbase = (size_t)p.slot0 + (last ? goff[c] : 0);
+        const size_t pbase = (size_t)p.slot0 + (fin ? goff[c] : 0);
         double acc[VPL];
 #pragma unroll
         for (int e = 0; e < VPL; ++e) acc[e] = 0.0;
@@ -746,7 +941,7 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
         for (int j0 = 0; j0 < n; j0 += kOB) {
           rows(ec, j0 + 2 * kOB, vc);
           const int ed = j0 + 3 * kOB < n ? entry(j0 + 3 * kOB + lane) : 0;
-          if (last && lane < kOB && j0 + lane < n) ks.perm[pbase + j0 + lane] = ea;
+          if (fin && lane < kOB && j0 + lane < n) ks.perm[pbase + j0 + lane] = ea;
 #pragma unroll
           for (int q = 0; q < kOB; ++q)
             if (j0 + q < n) add_row(acc, va[q]);
@@ -759,56 +954,29 @@ __global__ void __launch_bounds__(kFT, 1) kmeans_fused_kernel(FusedSets fs, int 
           eb = ec;
           ec = ed;
         }
-        if (last && lane == 0) {
+        if (fin && lane == 0) {
           ks.counts[cbase + c] = n;
           ks.off[(size_t)pid * (g.C + 1) + c] = goff[c];
           if (c == C - 1) ks.off[(size_t)pid * (g.C + 1) + C] = goff[C];
         }
-        if (n > 0) {  // an empty cluster keeps its centroid
-          const double nn = (double)n;
-          double q2 = 0.0;
-          float qf = 0.f;
-          double v64[VPL];
-          float v32[VPL];
-          uint32_t wh[VPL / 2], wl[VPL / 2];
+        if (cert) {  // the running state of the later rounds
+          double* sr = sumg + (size_t)c * D + (size_t)lane * VPL;
 #pragma unroll
-          for (int e = 0; e < VPL; ++e) {
-            v64[e] = __ddiv_rn(acc[e], nn);
-            v32[e] = (float)v64[e];
-            q2 += v64[e] * v64[e];
-            qf = fmaf(v32[e], v32[e], qf);
-          }
-#pragma unroll
-          for (int e = 0; e < VPL / 2; ++e) {
-            const __nv_bfloat16 h0 = __float2bfloat16_rn(v32[2 * e]);
-            const __nv_bfloat16 h1 = __float2bfloat16_rn(v32[2 * e + 1]);
-            const __nv_bfloat16 l0 = __float2bfloat16_rn(v32[2 * e] - __bfloat162float(h0));
-            const __nv_bfloat16 l1 = __float2bfloat16_rn(v32[2 * e + 1] - __bfloat162float(h1));
-            wh[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-            wl[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-          }
-          const size_t i0 = (cbase + c) * D + (size_t)lane * VPL;
-#pragma unroll
-          for (int e = 0; e < VPL / 2; ++e) {
-            reinterpret_cast<double2*>(ks.cent64 + i0)[e] = make_double2(v64[2 * e], v64[2 * e + 1]);
-            reinterpret_cast<float2*>(ks.cent32 + i0)[e] = make_float2(v32[2 * e], v32[2 * e + 1]);
-            reinterpret_cast<uint32_t*>(ks.cbf_hi + i0)[e] = wh[e];
-            reinterpret_cast<uint32_t*>(ks.cbf_lo + i0)[e] = wl[e];
-          }
-          for (int o = 16; o; o >>= 1) {
-            qf += __shfl_xor_sync(0xffffffffu, qf, o);
-            q2 += __shfl_xor_sync(0xffffffffu, q2, o);
-          }
+          for (int e = 0; e < VPL; ++e) sr[e] = acc[e];
           if (lane == 0) {
-            ks.cnorm[cbase + c] = sqrtf(qf) * 1.0001f;
-            ks.cn2[cbase + c] = (float)q2;
+            cntg[c] = n;
+            dirt[c] = 0;
           }
         }
+        if (n > 0) write_centroid(c, n, acc);  // an empty cluster keeps its centroid
         __syncwarp();  // the warp's tables are rewritten for its next cluster
       }
     }
+    // the change counter of round 1 starts from zero
+    if (cert && it == 0 && rank == 0 && tid == 0) chgp[1] = 0;
     team_sync();
     if (bar_fail) break;
+    if (fin) break;
   }
   fence_before();
   __syncthreads();

@@ -1051,12 +1051,6 @@ static int nct_cap(int ntp, int nprob, int tpc_max) {
   return cap < ntp ? cap : ntp;
 }
 
-bool resident_serves(const Levels& lv, int D, int C) {
-  for (int l = 0; l < lv.nlev; ++l)
-    if (resident_tpc_max(D, imin(C, lv.s[l])) >= 4) return true;
-  return false;
-}
-
 size_t resident_partial_blocks(const Levels& lv, int BH, int D, int C) {
   const int tmax = resident_tpc_max(D, C);
   if (tmax < 4) return 0;  // the resident kernel does not serve these sizes
