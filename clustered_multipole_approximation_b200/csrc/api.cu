@@ -148,6 +148,9 @@ struct AttnLayout {
   KState qs, ks;
   Stage1 s1;
   float* part;
+  void* kpad;  // sorted key copies of the tensor-core stage 2 (bf16 K, fp16 V)
+  void* vpad;
+  int* gofs;
   int nq;
   int wave;
   size_t bytes;
@@ -226,6 +229,16 @@ AttnLayout layout(const muse_shape* sh, const muse_params* pr, bool causal, cons
   L.s1.sel = cv.take<int>((size_t)L.nq * pr->Cq * k1 * 4);
   L.s1.nsel = cv.take<int>((size_t)L.nq * pr->Cq * 4);
   L.part = causal ? cv.take<float>((size_t)L.qs.ntok * (sh->D + 1) * 4) : nullptr;
+  if (dt == 0 && pr->Ck <= 256) {
+    // every key problem's tokens plus up to one padding group of 8 rows per cluster
+    const size_t rows = (size_t)L.ks.ntok + (size_t)8 * pr->Ck * L.ks.nprob;
+    L.kpad = cv.take<__nv_bfloat16>(rows * sh->D * 2);
+    L.vpad = cv.take<__half>(rows * sh->D * 2);
+    L.gofs = cv.take<int>((size_t)L.ks.nprob * (pr->Ck + 1) * 4);
+  } else {
+    L.kpad = L.vpad = nullptr;
+    L.gofs = nullptr;
+  }
   L.bytes = cv.used + 256;
   return L;
 }
@@ -269,6 +282,12 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   a.dense_lv = (causal && sh->dtype == MUSE_BF16 && pr->mode == MUSE_DIPOLE && L.V16)
                    ? dense_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck)
                    : 0;
+  a.tc_lv = (sh->dtype == MUSE_BF16 && L.V16 && L.kpad)
+                ? stage2_tc_levels(L.qg.lv, pr->Cq, pr->Ck, pr->topk, a.dense_lv)
+                : 0;
+  a.kpad = L.kpad;
+  a.vpad = L.vpad;
+  a.gofs = L.gofs;
   const size_t elt = sh->dtype == MUSE_BF16 ? 2 : 4;
   if (a.n_exact && causal)
     cudaMemsetAsync(a.n_exact, 0, (size_t)sh->B * sh->Hq * sh->N * 8, st);
@@ -295,6 +314,7 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
       run_kmeans_rounds(L.kg, L.ks, pr->iters, st);
       run_kmeans_rounds(L.qg, L.qs, pr->iters, st);
     }
+    run_permute_keys(a, st);
     for (int q0 = 0; q0 < L.nq; q0 += L.wave) {
       const int n = L.nq - q0 < L.wave ? L.nq - q0 : L.wave;
       run_blocks(a, L.s1, q0, n, st);

@@ -46,6 +46,10 @@ struct AttnArgs {
   float scale;
   int Cq, Ck;
   int dense_lv;       // causal levels (bit l) whose far field runs per key token
+  int tc_lv;          // levels (bit l) whose stage 2 runs on the tensor-core kernel
+  void* kpad;         // those levels' keys, cluster-sorted, group-padded, pre-swizzled (bf16)
+  void* vpad;         // the same for V (fp16)
+  int* gofs;          // [key problems][Ck + 1] first group of each cluster in kpad / vpad
 };
 
 // Key problem that a query problem attends: the same (b, level, pair) of the
@@ -102,6 +106,12 @@ void run_select(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStrea
 // Stage 2 with one warp per 16-query slice (bf16 inputs, topk <= 64); false
 // (nothing launched) when these arguments are not covered.
 bool run_stage2_warp(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
+// Tensor-core stage 2 (stage2_tc.cu): the levels it takes, the sorted key
+// copies it reads (once per call, after the k-means) and the launch for the
+// query problems [qp0, qp0 + nqp) at those levels.
+int stage2_tc_levels(const Levels& lv, int Cq, int Ck, int topk, int dense_lv);
+void run_permute_keys(const AttnArgs& a, cudaStream_t st);
+void run_stage2_tc(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 
 // Stage 2 on mma.sync tensor-core tiles (bf16 inputs).
 void run_stage2_mma(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);

@@ -531,6 +531,7 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
   if (sizeof(T) == 2) {
     {
       ProfScope ps(st, "stage2_attn");
+      run_stage2_tc(a, s1, qp0, nqp, st);
       if (!run_stage2_warp(a, s1, qp0, nqp, st)) run_stage2_mma(a, s1, qp0, nqp, st);
     }
     if (a.dense_lv) run_stage2_dense(a, s1, qp0, nqp, st);

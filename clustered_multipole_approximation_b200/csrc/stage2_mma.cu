@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) stage2_mma_kernel(A
   constexpr int CH = D / 8;    // 16-byte chunks per row
   const int lq = blockIdx.x, qpid = qp0 + lq, i = blockIdx.y;
   const Prob pq = prob_of(a.qg, qpid);
-  if (i >= pq.C || ((a.dense_lv >> pq.level) & 1)) return;
+  if (i >= pq.C || (((a.dense_lv | a.tc_lv) >> pq.level) & 1)) return;
   const int Cq = a.Cq, Ck = a.Ck;
   const int nqi = a.qs.counts[(size_t)qpid * Cq + i];
   if (nqi == 0) return;

@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(kWW * 32) stage2_warp_kernel(AttnArgs a, Stage
   const int lq = blockIdx.x, qpid = qp0 + lq;
   const Prob pq = prob_of(a.qg, qpid);
   if ((a.dense_lv >> pq.level) & 1) return;  // that level runs one key token at a time
+  if ((a.tc_lv >> pq.level) & 1) return;     // that level runs on the tensor-core kernel
   const int Cq = a.Cq, Ck = a.Ck, cq = pq.C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;
@@ -420,8 +421,8 @@ bool run_stage2_warp(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
   // slices of a query problem: at most one per 16 queries plus one per cluster
   int smax = 0;
   for (int l = 0; l < a.qg.lv.nlev; ++l)
-    if (!((a.dense_lv >> l) & 1)) smax = smax > a.qg.lv.s[l] ? smax : a.qg.lv.s[l];
-  if (smax == 0) return true;  // every level runs one key token at a time
+    if (!(((a.dense_lv | a.tc_lv) >> l) & 1)) smax = smax > a.qg.lv.s[l] ? smax : a.qg.lv.s[l];
+  if (smax == 0) return true;  // every level runs elsewhere
   const int nslice = cdiv(smax, 16) + imin(a.Cq, smax);
   if (a.qg.D == 64)
     launch_w<64>(a, s1, qp0, nqp, nslice, st);
