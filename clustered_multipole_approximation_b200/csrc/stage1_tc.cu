@@ -79,6 +79,28 @@ __device__ inline void tld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 __device__ inline void tld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+// The wait, tied to the 64 registers of four loads so that no use of them
+// moves above it.
+__device__ inline void tld_wait4(uint32_t (&r)[4][16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(r[0][0]), "+r"(r[0][1]), "+r"(r[0][2]), "+r"(r[0][3]), "+r"(r[0][4]), "+r"(r[0][5]),
+                 "+r"(r[0][6]), "+r"(r[0][7]), "+r"(r[0][8]), "+r"(r[0][9]), "+r"(r[0][10]),
+                 "+r"(r[0][11]), "+r"(r[0][12]), "+r"(r[0][13]), "+r"(r[0][14]), "+r"(r[0][15]),
+                 "+r"(r[1][0]), "+r"(r[1][1]), "+r"(r[1][2]), "+r"(r[1][3]), "+r"(r[1][4]), "+r"(r[1][5]),
+                 "+r"(r[1][6]), "+r"(r[1][7]), "+r"(r[1][8]), "+r"(r[1][9]), "+r"(r[1][10]),
+                 "+r"(r[1][11]), "+r"(r[1][12]), "+r"(r[1][13]), "+r"(r[1][14]), "+r"(r[1][15])
+               :
+               : "memory");
+  asm volatile(""
+               : "+r"(r[2][0]), "+r"(r[2][1]), "+r"(r[2][2]), "+r"(r[2][3]), "+r"(r[2][4]), "+r"(r[2][5]),
+                 "+r"(r[2][6]), "+r"(r[2][7]), "+r"(r[2][8]), "+r"(r[2][9]), "+r"(r[2][10]),
+                 "+r"(r[2][11]), "+r"(r[2][12]), "+r"(r[2][13]), "+r"(r[2][14]), "+r"(r[2][15]),
+                 "+r"(r[3][0]), "+r"(r[3][1]), "+r"(r[3][2]), "+r"(r[3][3]), "+r"(r[3][4]), "+r"(r[3][5]),
+                 "+r"(r[3][6]), "+r"(r[3][7]), "+r"(r[3][8]), "+r"(r[3][9]), "+r"(r[3][10]),
+                 "+r"(r[3][11]), "+r"(r[3][12]), "+r"(r[3][13]), "+r"(r[3][14]), "+r"(r[3][15])
+               :
+               : "memory");
+}
 __device__ inline void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ inline void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 __device__ inline void fence_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
@@ -188,26 +210,17 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
   uint32_t ph[2] = {0u, 0u};
   bool ok = true;
 
+  // members of this CTA's rows in the member-row loads below: thread t copies
+  // the 16-byte pieces t, t + 128, ... of the 128 x KB x 8 grid, rows
+  // (t + 128 m) / (KB 8)
+  constexpr int kPieces = kR * KB * 8 / kS1T;
   for (int i0 = 0; i0 < pq.C; i0 += kR) {
     const int ic = imin(kR, pq.C - i0);
-    {
-      float dt = 0.f;
-      if (tid < ic) {
-        const float4* nu = reinterpret_cast<const float4*>(a.qs.cent32 + ((size_t)qpid * Cq + i0 + tid) * D);
-#pragma unroll 4
-        for (int d4 = 0; d4 < D / 4; ++d4) {
-          const float4 v = nu[d4];
-          dt = fmaf(v.x, mu[4 * d4], dt);
-          dt = fmaf(v.y, mu[4 * d4 + 1], dt);
-          dt = fmaf(v.z, mu[4 * d4 + 2], dt);
-          dt = fmaf(v.w, mu[4 * d4 + 3], dt);
-        }
-      }
-      nm[tid] = dt;
-    }
     for (int t0 = 0; t0 < nj; t0 += kR) {
       const int nt = imin(kR, nj - t0);
-      // query centroids (bf16 split) of this pass; rows past ic are zero
+      // the copies first (query centroids as the bf16 split, rows past ic
+      // zero; member keys and values through the permutation, rows past nt
+      // zero); the dot products nu_i . mu_j run while they are in flight
       for (int e = tid; e < kR * KB * 8; e += kS1T) {
         const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, c = q & 7;
         const bool live = r < ic;
@@ -216,13 +229,39 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
         cp16(sb + Lt::NH + so, a.qs.cbf_hi + o, live ? 16 : 0);
         cp16(sb + Lt::NL + so, a.qs.cbf_lo + o, live ? 16 : 0);
       }
-      for (int e = tid; e < kR * KB * 8; e += kS1T) {
-        const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, c = q & 7;
-        const bool live = r < nt;
-        const long long row = pk.row0 + (live ? perm[off + t0 + r] : 0);
-        const uint32_t so = kb * kR * 128 + swz(r, c);
-        cp16(sb + Lt::KM + so, Kx + row * D + kb * 64 + c * 8, live ? 16 : 0);
-        cp16(sb + Lt::VM + so, a.V16 + row * D + kb * 64 + c * 8, live ? 16 : 0);
+      {
+        int rows[kPieces];  // every permutation entry read before the first copy
+#pragma unroll
+        for (int m = 0; m < kPieces; ++m) {
+          const int r = (tid + m * kS1T) / (KB * 8);
+          rows[m] = r < nt ? perm[off + t0 + r] : -1;
+        }
+#pragma unroll
+        for (int m = 0; m < kPieces; ++m) {
+          const int e = tid + m * kS1T;
+          const int r = e / (KB * 8), q = e - r * (KB * 8), kb = q >> 3, c = q & 7;
+          const long long row = pk.row0 + (rows[m] >= 0 ? rows[m] : 0);
+          const uint32_t so = kb * kR * 128 + swz(r, c);
+          cp16(sb + Lt::KM + so, Kx + row * D + kb * 64 + c * 8, rows[m] >= 0 ? 16 : 0);
+          cp16(sb + Lt::VM + so, a.V16 + row * D + kb * 64 + c * 8, rows[m] >= 0 ? 16 : 0);
+        }
+      }
+      if (t0 == 0) {  // nu_i . mu_j of this pass: every load in flight at once
+        float dt = 0.f;
+        if (tid < ic) {
+          const float4* nu = reinterpret_cast<const float4*>(a.qs.cent32 + ((size_t)qpid * Cq + i0 + tid) * D);
+          float4 v[D / 4];
+#pragma unroll
+          for (int d4 = 0; d4 < D / 4; ++d4) v[d4] = nu[d4];
+#pragma unroll
+          for (int d4 = 0; d4 < D / 4; ++d4) {
+            dt = fmaf(v[d4].x, mu[4 * d4], dt);
+            dt = fmaf(v[d4].y, mu[4 * d4 + 1], dt);
+            dt = fmaf(v[d4].z, mu[4 * d4 + 2], dt);
+            dt = fmaf(v[d4].w, mu[4 * d4 + 3], dt);
+          }
+        }
+        nm[tid] = dt;
       }
       cp_commit_wait();
       fence_async();
@@ -247,12 +286,17 @@ __global__ void __launch_bounds__(kS1T) stage1_dipole_tc_kernel(AttnArgs a, Stag
       fence_after();
       // W row of member t = tid over the 128 query clusters; members past nt
       // get 0 so they add nothing
+      // (the second half's TMEM loads run during the first half's arithmetic)
+      uint32_t gall[2][4][16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tld16(tl + 16 * q, gall[0][q]);
+      tld_wait4(gall[0]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tld16(tl + 64 + 16 * q, gall[1][q]);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {  // 64 query clusters per 128-byte row chunk
-        uint32_t g4[4][16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tld16(tl + 64 * h + 16 * q, g4[q]);
-        tld_wait();
+        if (h == 1) tld_wait4(gall[1]);
+        uint32_t (&g4)[4][16] = gall[h];
         unsigned char* wrow = sm + Lt::W + h * kR * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
