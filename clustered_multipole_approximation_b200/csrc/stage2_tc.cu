@@ -42,7 +42,8 @@ namespace {
 
 constexpr int kTQ = 128;      // query rows per CTA (TMEM lanes, one thread each)
 constexpr int kTK = 64;       // key rows per block
-constexpr int kTT = 192;      // threads: four warps of query rows, an MMA and a load warp
+constexpr int kTC = 256;      // softmax threads: two per query row, each half the columns
+constexpr int kTT = kTC + 64;  // threads: + an MMA warp and a load warp
 constexpr int kTMaxSel = 64;  // retrieved clusters per query cluster
 constexpr int kTStages = 3;   // key blocks in flight
 constexpr float kLazy = 8.f;  // headroom (base 2) of the reference maximum
@@ -127,8 +128,7 @@ __device__ inline void tld_wait(uint32_t (&r)[16]) {
                :
                : "memory");
 }
-// The same for four loads of 16 registers.
-__device__ inline void tld_wait4(uint32_t (&r)[4][16]) {
+__device__ inline void tld_wait2(uint32_t (&r)[2][16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;\n"
                : "+r"(r[0][0]), "+r"(r[0][1]), "+r"(r[0][2]), "+r"(r[0][3]), "+r"(r[0][4]), "+r"(r[0][5]),
                  "+r"(r[0][6]), "+r"(r[0][7]), "+r"(r[0][8]), "+r"(r[0][9]), "+r"(r[0][10]),
@@ -136,15 +136,6 @@ __device__ inline void tld_wait4(uint32_t (&r)[4][16]) {
                  "+r"(r[1][0]), "+r"(r[1][1]), "+r"(r[1][2]), "+r"(r[1][3]), "+r"(r[1][4]), "+r"(r[1][5]),
                  "+r"(r[1][6]), "+r"(r[1][7]), "+r"(r[1][8]), "+r"(r[1][9]), "+r"(r[1][10]),
                  "+r"(r[1][11]), "+r"(r[1][12]), "+r"(r[1][13]), "+r"(r[1][14]), "+r"(r[1][15])
-               :
-               : "memory");
-  asm volatile(""
-               : "+r"(r[2][0]), "+r"(r[2][1]), "+r"(r[2][2]), "+r"(r[2][3]), "+r"(r[2][4]), "+r"(r[2][5]),
-                 "+r"(r[2][6]), "+r"(r[2][7]), "+r"(r[2][8]), "+r"(r[2][9]), "+r"(r[2][10]),
-                 "+r"(r[2][11]), "+r"(r[2][12]), "+r"(r[2][13]), "+r"(r[2][14]), "+r"(r[2][15]),
-                 "+r"(r[3][0]), "+r"(r[3][1]), "+r"(r[3][2]), "+r"(r[3][3]), "+r"(r[3][4]), "+r"(r[3][5]),
-                 "+r"(r[3][6]), "+r"(r[3][7]), "+r"(r[3][8]), "+r"(r[3][9]), "+r"(r[3][10]),
-                 "+r"(r[3][11]), "+r"(r[3][12]), "+r"(r[3][13]), "+r"(r[3][14]), "+r"(r[3][15])
                :
                : "memory");
 }
@@ -297,7 +288,9 @@ __global__ void __launch_bounds__(256) permute_keys_kernel(AttnArgs a) {
 }
 
 template <typename TO, int D>
-__global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1, int qp0) {
+__global__ void __launch_bounds__(kTT, D == 64 ? 2 : 1) stage2_tc_kernel(AttnArgs a, Stage1 s1, int qp0) {
+  constexpr int HK = kTK / 2;  // columns of a block per softmax thread
+  constexpr int HD = D / 2;    // O columns per softmax thread
   using Lt = TcL<D>;
   constexpr int KB = Lt::KB;
   extern __shared__ __align__(1024) unsigned char tc_raw[];
@@ -312,13 +305,21 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
   __shared__ int jsel[kTMaxSel], jng[kTMaxSel], jgof[kTMaxSel], jn[kTMaxSel];
   __shared__ int gpre[kTMaxSel + 1];
   __shared__ float fbs[kTK];
+  // the two halves of a row exchange partial maxima (then sums) here, in a
+  // buffer that alternates between steps: a half writes step n + 2's value
+  // only after both passed step n + 1's barrier, so after the read of step n
+  __shared__ float xch[2][2][kTQ];
 
   const int lq = blockIdx.x, qpid = qp0 + lq;
   const Prob pq = prob_of(a.qg, qpid);
   if (!((a.tc_lv >> pq.level) & 1)) return;
   const int Cq = a.Cq, Ck = a.Ck, cq = pq.C;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool consumer = warp < kTQ / 32;  // warps 0-3: query rows; warp 4 issues
+  // warps 0-7 softmax: row (warp % 4) 32 + lane (its TMEM lane), column half
+  // warp / 4; warp 8 issues the MMAs, warp 9 the loads
+  const bool consumer = warp < kTC / 32;
+  const int row = tid & (kTQ - 1), hc = (warp >> 2) & 1;
+  const int kIssue = kTC;  // the MMA warp's lane 0
 
   // ---- this CTA's tile: cluster i, queries [r0, r0 + nq) of it ----------------
   const int* qcnt = a.qs.counts + (size_t)qpid * Cq;
@@ -362,16 +363,16 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;\n" ::"r"(s32(&tslot)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
   }
-  if (tid == kTQ) {
+  if (tid == kIssue) {
     for (int s = 0; s < kTStages; ++s) {
       mbar_init(s32(&mLd[s]), 1);
       mbar_init(s32(&mEmpty[s]), 1);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(s32(&mS[k]), 1);
-      mbar_init(s32(&mSfree[k]), kTQ / 32);
+      mbar_init(s32(&mSfree[k]), kTC / 32);
     }
-    mbar_init(s32(&mP), kTQ / 32);
+    mbar_init(s32(&mP), kTC / 32);
     mbar_init(s32(&mPV), 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n");
   }
@@ -428,6 +429,7 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
   int uS[2] = {0, 0}, uSf[2] = {0, 0}, uP = 0, uPV = 0, uLd[kTStages] = {0, 0, 0};
   bool o_init = false;  // some P V has written O
   float mref = kMaxFloor, lsum = 0.f;
+  int xstep = 0;  // exchanges made (the same count in both halves of a row)
 
   auto wait_on = [&](uint64_t& bar, int& use) {
     ok = mbar_wait(s32(&bar), (uint32_t)(use & 1)) && ok;
@@ -468,19 +470,20 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
   // logits with their bias first.
   auto softmax = [&](int k, auto biasf, unsigned long long emask, bool far, bool wait_pv, bool sfree) {
     const bool raw = !far && sl2 > 0.f;
-    float p[kTK];
+    float p[HK];
     float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    {  // the row's 64 scores: four loads in flight, one wait
-      uint32_t r[4][16];
+    {  // this thread's 32 scores of the row: two loads in flight, one wait
+      uint32_t r[2][16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tld16(tS[k] + lane_off + (uint32_t)(16 * q), r[q]);
-      tld_wait4(r);
+      for (int q = 0; q < 2; ++q) tld16(tS[k] + lane_off + (uint32_t)(HK * hc + 16 * q), r[q]);
+      tld_wait2(r);
       if (raw) {
 #pragma unroll
-        for (int c = 0; c < kTK; ++c) p[c] = __uint_as_float(r[c >> 4][c & 15]);
+        for (int c = 0; c < HK; ++c) p[c] = __uint_as_float(r[c >> 4][c & 15]);
+        const unsigned hm = (unsigned)(emask >> (HK * hc));
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const unsigned g = (unsigned)(emask >> (8 * q)) & 0xFFu;
+        for (int q = 0; q < HK / 8; ++q) {
+          const unsigned g = (hm >> (8 * q)) & 0xFFu;
           if (g != 0xFFu) {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -488,11 +491,11 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
           }
         }
 #pragma unroll
-        for (int c = 0; c < kTK; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], p[c]);
+        for (int c = 0; c < HK; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], p[c]);
       } else {
 #pragma unroll
-        for (int c = 0; c < kTK; ++c) {
-          const float lg = fmaf(sl2, __uint_as_float(r[c >> 4][c & 15]), biasf(c));
+        for (int c = 0; c < HK; ++c) {
+          const float lg = fmaf(sl2, __uint_as_float(r[c >> 4][c & 15]), biasf(HK * hc + c));
           p[c] = lg;
           mx4[c & 3] = fmaxf(mx4[c & 3], lg);
         }
@@ -503,7 +506,13 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(s32(&mSfree[k])) : "memory");
     }
+    // the row's maximum over both halves (the two threads of a row meet at a
+    // named barrier of their 64 threads)
     float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+    xch[xstep & 1][hc][row] = mx;
+    asm volatile("bar.sync %0, 64;\n" ::"r"(1 + (warp & 3)) : "memory");
+    mx = fmaxf(mx, xch[xstep & 1][hc ^ 1][row]);
+    ++xstep;
     if (raw) mx *= sl2;
     const bool move = mx > mref + kLazy;
     const float mnew = move ? mx : mref;
@@ -511,49 +520,49 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
     float rs4[4] = {0.f, 0.f, 0.f, 0.f};
     if (raw) {
 #pragma unroll
-      for (int c = 0; c < kTK; ++c) {
+      for (int c = 0; c < HK; ++c) {
         const float v = fast_exp2(fmaf(sl2, p[c], -mnew));
         p[c] = v;
         rs4[c & 3] += v;
       }
     } else {
 #pragma unroll
-      for (int c = 0; c < kTK; ++c) {
+      for (int c = 0; c < HK; ++c) {
         const float v = fast_exp2(p[c] - mnew);
         p[c] = v;
         rs4[c & 3] += v;
       }
     }
-    lsum = lsum * scale + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+    lsum = lsum * scale + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));  // this half's share
     mref = mnew;
     if (wait_pv) {  // P and O are free once the previous P V is done
       wait_on(mPV, uPV);
       fence_after();
     }
-    if (o_init && __any_sync(0xffffffffu, move)) {
+    if (o_init && __any_sync(0xffffffffu, move)) {  // each half rescales half of O's columns
 #pragma unroll
-      for (int d0 = 0; d0 < D; d0 += 16) {
+      for (int d0 = 0; d0 < HD; d0 += 16) {
         uint32_t r[16];
-        tld16(tO + lane_off + (uint32_t)d0, r);
+        tld16(tO + lane_off + (uint32_t)(HD * hc + d0), r);
         tld_wait(r);
 #pragma unroll
         for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * scale);
-        tst16(tO + lane_off + (uint32_t)d0, r);
+        tst16(tO + lane_off + (uint32_t)(HD * hc + d0), r);
       }
       tst_wait();
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < HK / 8; ++c) {  // 16-byte pieces 4 hc + c of the row
       uint32_t hv[4], lv[4];
       if (far) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) split_h2bits(p[8 * c + 2 * u], p[8 * c + 2 * u + 1], hv[u], lv[u]);
-        *reinterpret_cast<uint4*>(sm + Lt::PL + swz(tid, c)) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        *reinterpret_cast<uint4*>(sm + Lt::PL + swz(row, 4 * hc + c)) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
       } else {
 #pragma unroll
         for (int u = 0; u < 4; ++u) hv[u] = h2bits(p[8 * c + 2 * u], p[8 * c + 2 * u + 1]);
       }
-      *reinterpret_cast<uint4*>(sm + Lt::P + swz(tid, c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      *reinterpret_cast<uint4*>(sm + Lt::P + swz(row, 4 * hc + c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
     }
     fence_async();
     fence_before();
@@ -595,7 +604,7 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
     fence_before();
     __syncthreads();
     fence_after();
-    if (tid == kTQ) issue_S(0, st0K, st1K);
+    if (tid == kIssue) issue_S(0, st0K, st1K);
     if (consumer) {
       wait_on(mS[0], uS[0]);
       fence_after();
@@ -603,7 +612,7 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
     }
     __syncthreads();
     fence_after();
-    if (tid == kTQ) issue_PV(st0V, st1V, true);
+    if (tid == kIssue) issue_PV(st0V, st1V, true);
     o_init = true;
     wait_on(mPV, uPV);  // the stages and P are reloaded next
     fence_after();
@@ -637,7 +646,7 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
           gs += cnt;
         }
       };
-      if (warp == kTQ / 32 + 1) {
+      if (warp == kTC / 32 + 1) {
         // the load warp: a stage is refilled once the P V of its block is done
         int uE[kTStages] = {0, 0, 0};
         for (int b = 0; b < nblk; ++b) {
@@ -689,18 +698,21 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
   if (consumer) {
     int nexact = 0;
     for (int r = 0; r < nsel; ++r) nexact += jn[r];
-    const bool live = tid < nq;
-    const int tq = live ? qperm[qo + r0 + tid] : 0;
-    const long long row = pq.row0 + tq;
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    xch[xstep & 1][hc][row] = lsum;  // the row's sum over both halves
+    asm volatile("bar.sync %0, 64;\n" ::"r"(1 + (warp & 3)) : "memory");
+    const float ltot = lsum + xch[xstep & 1][hc ^ 1][row];
+    const bool live = row < nq;
+    const int tq = live ? qperm[qo + r0 + row] : 0;
+    const long long orow = pq.row0 + tq;
+    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
 #pragma unroll
-    for (int d0 = 0; d0 < D; d0 += 16) {
+    for (int d0 = 0; d0 < HD; d0 += 16) {
       uint32_t r[16];
-      tld16(tO + lane_off + (uint32_t)d0, r);
+      tld16(tO + lane_off + (uint32_t)(HD * hc + d0), r);
       tld_wait(r);
       if (!live) continue;
       if (a.O != nullptr) {
-        TO* O = static_cast<TO*>(a.O) + row * D + d0;
+        TO* O = static_cast<TO*>(a.O) + orow * D + HD * hc + d0;
         if (sizeof(TO) == 2) {
           uint32_t w[8];
 #pragma unroll
@@ -719,18 +731,18 @@ __global__ void __launch_bounds__(kTT, 2) stage2_tc_kernel(AttnArgs a, Stage1 s1
                             __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
         }
       } else {
-        float* pp = a.part + (size_t)(pq.slot0 + tq) * (D + 1) + d0;
+        float* pp = a.part + (size_t)(pq.slot0 + tq) * (D + 1) + HD * hc + d0;
 #pragma unroll
         for (int e = 0; e < 16; ++e) pp[e] = __uint_as_float(r[e]) * inv;
       }
     }
-    if (live && a.O == nullptr)
-      a.part[(size_t)(pq.slot0 + tq) * (D + 1) + D] = (mref + log2f(lsum)) * 0.6931471805599453f;
-    if (live && a.n_exact != nullptr) {
+    if (live && hc == 0 && a.O == nullptr)
+      a.part[(size_t)(pq.slot0 + tq) * (D + 1) + D] = (mref + log2f(ltot)) * 0.6931471805599453f;
+    if (live && hc == 0 && a.n_exact != nullptr) {
       if (a.O != nullptr)
-        a.n_exact[row] = nexact;
+        a.n_exact[orow] = nexact;
       else
-        atomicAdd(reinterpret_cast<unsigned long long*>(a.n_exact + row), (unsigned long long)nexact);
+        atomicAdd(reinterpret_cast<unsigned long long*>(a.n_exact + orow), (unsigned long long)nexact);
     }
   }
   if (!ok) atomicOr(a.qs.err, kErrMmaWait);
