@@ -25,7 +25,8 @@
  *     Fisher-Yates shuffle driven by Vigna's splitmix64;
  *   - the dipole uses the query-cluster centroid nu_i (first-order expansion
  *     of the kept cross term), the tilted mode expands about the tilted
- *     centroid k_hat_ij;
+ *     centroid k_hat_ij; the fine-query dipole (an accuracy variant) uses the
+ *     query itself: u_qj = (S_j + s M_j q) / n_j;
  *   - the causal scheme is the binary (Fenwick-style) block decomposition.
  *
  * Layouts: Q [B,Hq,N,D], K and V [B,Hkv,N,D], O [B,Hq,N,D], all row-major,
@@ -45,6 +46,7 @@
 #define ORC_MONOPOLE 0
 #define ORC_DIPOLE 1
 #define ORC_TILTED 2
+#define ORC_DIPOLE_Q 3
 
 /* ------------------------------------------------------------------------ */
 /* splitmix64 (Vigna): state advances by the golden-ratio increment, output  */
@@ -259,12 +261,13 @@ static void stage1(const query_block *qb, const key_block *kb, double scale,
         for (int d = 0; d < D; ++d) u[d] = kh[d] = 0.0;
         continue;
       }
-      if (mode == ORC_MONOPOLE || mode == ORC_DIPOLE) {
+      if (mode == ORC_MONOPOLE || mode == ORC_DIPOLE || mode == ORC_DIPOLE_Q) {
         logW[ij] = log((double)nj);
         for (int e = 0; e < D; ++e) {
           double x = S[e];
           if (mode == ORC_DIPOLE) {
-            /* first-order term of exp(s nu_i . k~): (s/n_j) M_j nu_i */
+            /* first-order term of exp(s nu_i . k~): (s/n_j) M_j nu_i
+             * (the fine-query dipole adds (s/n_j) M_j q per query in stage 2) */
             const double *Me = kb->M + ((size_t)j * D + e) * D;
             x += scale * dot(Me, nu, D);
           }
@@ -339,6 +342,7 @@ static void stage2(const query_block *qb, const key_block *kb, double scale,
                    long long *n_exact /* nullable, [nq] */) {
   const int D = kb->D, Ck = kb->C;
   char *inR = (char *)malloc((size_t)Ck);
+  double *uq = (double *)malloc(sizeof(double) * (size_t)D);
   for (int q = 0; q < qb->n; ++q) {
     const double *x = qb->Q + (size_t)q * D;
     int i = qb->assign[q];
@@ -358,7 +362,15 @@ static void stage2(const query_block *qb, const key_block *kb, double scale,
       } else {
         lam = scale * dot(x, kb->mu + (size_t)j * D, D) + logW[ij];
       }
-      acc_add(&m[q], &l[q], aq, D, lam, U + ij * D);
+      const double *val = U + ij * D;
+      if (mode == ORC_DIPOLE_Q) {
+        /* the first-order term of exp(s q . k~) with the query itself:
+         * u_qj = S_j / n_j + (s / n_j) M_j q */
+        for (int e = 0; e < D; ++e)
+          uq[e] = val[e] + scale * dot(kb->M + ((size_t)j * D + e) * D, x, D) / (double)kb->count[j];
+        val = uq;
+      }
+      acc_add(&m[q], &l[q], aq, D, lam, val);
     }
     long long ne = 0;
     for (int t = 0; t < kb->n; ++t) {
@@ -370,6 +382,7 @@ static void stage2(const query_block *qb, const key_block *kb, double scale,
     if (n_exact) n_exact[q] += ne;
   }
   free(inR);
+  free(uq);
 }
 
 /* Debug outputs of one block problem (all optional). */
@@ -482,7 +495,7 @@ void orc_muse_acausal(const double *Q, const double *K, const double *V, int B,
     key_block kb;
     make_keys(&kb, K + koff * D, V + koff * D, N, D, Ck, iters, seed,
               ks0 + (uint64_t)bk, k_assign_in ? k_assign_in + koff : NULL,
-              mode == ORC_DIPOLE);
+              mode == ORC_DIPOLE || mode == ORC_DIPOLE_Q);
     if (k_assign) memcpy(k_assign + koff, kb.assign, sizeof(int) * (size_t)N);
     if (k_cent) memcpy(k_cent + (size_t)bk * Ck * D, kb.mu, sizeof(double) * (size_t)Ck * D);
     if (k_count) memcpy(k_count + (size_t)bk * Ck, kb.count, sizeof(int) * (size_t)Ck);
@@ -563,7 +576,7 @@ void orc_muse_causal(const double *Q, const double *K, const double *V, int B,
         make_keys(&kb, Kh + (size_t)k0 * D, Vh + (size_t)k0 * D, s, D, Ce, iters,
                   seed, ksid,
                   k_assign_in ? k_assign_in + (size_t)bk * levels * half + slot : NULL,
-                  mode == ORC_DIPOLE);
+                  mode == ORC_DIPOLE || mode == ORC_DIPOLE_Q);
         if (k_assign)
           memcpy(k_assign + (size_t)bk * levels * half + slot, kb.assign, sizeof(int) * (size_t)s);
         for (int g = 0; g < G; ++g) {
@@ -681,7 +694,7 @@ void orc_stage1_debug(const double *Qh, const double *Kh, const double *Vh,
                       const int *k_assign, int k1, double scale, int mode,
                       double *logW, double *U, int *selected) {
   key_block kb;
-  make_keys(&kb, Kh, Vh, N, D, Ck, 1, 0, 0, k_assign, mode == ORC_DIPOLE);
+  make_keys(&kb, Kh, Vh, N, D, Ck, 1, 0, 0, k_assign, mode == ORC_DIPOLE || mode == ORC_DIPOLE_Q);
   query_block qb;
   make_queries(&qb, Qh, N, D, Cq, 1, 0, 0, q_assign);
   double *m = (double *)malloc(sizeof(double) * (size_t)N);

@@ -43,6 +43,11 @@ MUTANTS = {
     "local-block-reads-future": ("for (int t = t0; t <= q; ++t) {", "for (int t = t0; t < t0 + L; ++t) {"),
     "causal-level-skips-top": ("for (int lv = 0; lv < levels; ++lv) {",
                                "for (int lv = 0; lv + 1 < levels; ++lv) {"),
+    "fine-query-dipole-uses-centroid": (
+        "scale * dot(kb->M + ((size_t)j * D + e) * D, x, D) / (double)kb->count[j];",
+        "scale * dot(kb->M + ((size_t)j * D + e) * D, nu, D) / (double)kb->count[j];"),
+    "fine-query-dipole-sign": (
+        "uq[e] = val[e] + scale * dot(", "uq[e] = val[e] - scale * dot("),
 }
 
 

@@ -169,7 +169,7 @@ def test_exact_attention_matches_torch(orc, causal):
 # --------------------------------------------------------------------------
 # closed forms the approximation reduces to
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
 def test_singleton_key_clusters_are_exact(orc, mode):
     Q, K, V = small_qkv(B=1, Hq=2, Hkv=1, N=64, D=8, seed=4)
     E = orc.exact_attention(Q, K, V)
@@ -178,7 +178,7 @@ def test_singleton_key_clusters_are_exact(orc, mode):
         np.testing.assert_allclose(r["O"], E, rtol=1e-11, atol=1e-12)
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
 def test_retrieving_every_cluster_is_exact(orc, mode):
     Q, K, V = small_qkv(N=128, D=8, seed=6)
     E = orc.exact_attention(Q, K, V)
@@ -222,6 +222,25 @@ def test_dipole_single_cluster_is_cross_covariance_correction(orc):
     np.testing.assert_allclose(r["O"][0, 0], ref, rtol=1e-10, atol=1e-12)
 
 
+def test_fine_query_dipole_single_cluster_is_cross_covariance_at_the_query(orc):
+    """With one key cluster the fine-query dipole is v_bar + s C_vk q for every
+    query q itself (the query-centroid dipole uses nu instead)."""
+    Q, K, V = small_qkv(N=180, D=6, seed=14)
+    s = 1.3
+    r = orc.muse_acausal(Q, K, V, 4, 1, 3, 0, 0, scale=s, mode="dipole_q")
+    cvk = np.cov(np.concatenate([V[0, 0], K[0, 0]], 1).T, bias=True)[:6, 6:]
+    ref = V[0, 0].mean(0)[None, :] + s * Q[0, 0] @ cvk.T
+    np.testing.assert_allclose(r["O"][0, 0], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_fine_query_dipole_equals_dipole_with_singleton_query_clusters(orc):
+    """Each query its own cluster (nu_i = q): the two dipoles coincide."""
+    Q, K, V = small_qkv(N=64, D=8, seed=31)
+    a = orc.muse_acausal(Q, K, V, 64, 6, 3, 5, 1, scale=0.9, mode="dipole")["O"]
+    b = orc.muse_acausal(Q, K, V, 64, 6, 3, 5, 1, scale=0.9, mode="dipole_q")["O"]
+    np.testing.assert_allclose(b, a, rtol=1e-11, atol=1e-12)
+
+
 def test_modes_agree_when_cluster_keys_coincide(orc):
     rng = np.random.default_rng(2)
     N, D, Ck = 120, 8, 6
@@ -232,9 +251,10 @@ def test_modes_agree_when_cluster_keys_coincide(orc):
     Q = (base[rng.integers(0, Ck, N)] + 0.2 * rng.standard_normal((N, D)))[None, None]
     V = rng.standard_normal((1, 1, N, D))
     outs = [orc.muse_acausal(Q, K, V, 4, Ck, 3, 1, 1, mode=m, k_assign_in=z[None, None])["O"]
-            for m in ("monopole", "dipole", "tilted")]
+            for m in ("monopole", "dipole", "tilted", "dipole_q")]
     np.testing.assert_allclose(outs[1], outs[0], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(outs[2], outs[0], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(outs[3], outs[0], rtol=1e-11, atol=1e-12)
 
 
 def test_selection_ties_go_to_lowest_index(orc):
@@ -259,7 +279,7 @@ def test_selection_ties_go_to_lowest_index(orc):
 # --------------------------------------------------------------------------
 # invariants
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
 def test_weights_sum_to_one_and_monopole_tilted_nonnegative(orc, mode):
     # with V = identity each output row is the vector of per-token weights
     Q, K, _ = small_qkv(N=64, D=64, centres=6, seed=15)
@@ -267,7 +287,7 @@ def test_weights_sum_to_one_and_monopole_tilted_nonnegative(orc, mode):
     r = orc.muse_acausal(Q, K, V, 4, 8, 3, 2, 2, mode=mode)
     W = r["O"][0, 0]
     np.testing.assert_allclose(W.sum(1), 1.0, rtol=0, atol=1e-12)
-    if mode != "dipole":
+    if mode in ("monopole", "tilted"):  # the dipole factors take either sign
         assert W.min() >= -1e-15
     # a constant value vector comes back unchanged
     Vc = np.tile(np.arange(64.0), (64, 1))[None, None]
@@ -275,7 +295,7 @@ def test_weights_sum_to_one_and_monopole_tilted_nonnegative(orc, mode):
     np.testing.assert_allclose(r["O"][0, 0], Vc[0, 0], rtol=1e-12, atol=1e-10)
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
 def test_key_translation_invariance(orc, mode):
     Q, K, V = small_qkv(N=256, D=8, centres=6, noise=0.2, seed=16)
     shift = np.linspace(-0.5, 0.75, 8)
@@ -287,7 +307,7 @@ def test_key_translation_invariance(orc, mode):
     np.testing.assert_allclose(b["k_cent"], a["k_cent"] + shift, rtol=1e-12, atol=1e-12)
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
 def test_causal_never_reads_the_future(orc, mode):
     Q, K, V = small_qkv(B=1, Hq=2, Hkv=1, N=128, D=8, seed=17)
     base = orc.muse_causal(Q, K, V, 16, 4, 3, 5, 1, mode=mode)["O"]
@@ -299,7 +319,7 @@ def test_causal_never_reads_the_future(orc, mode):
         assert (o[:, :, : t0 + 1] == base[:, :, : t0 + 1]).all()
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
 def test_causal_with_singleton_clusters_is_exact_causal(orc, mode):
     # C >= block size at every level makes every summary exact, so the
     # decomposition must cover each earlier key exactly once.
@@ -354,12 +374,14 @@ def brute_block(Qb, Kb, Vb, qa, ka, Cq, Ck, k1, s, mode):
                     W[q, t] = math.exp(s * x @ mu[j])
                 elif mode == "dipole":
                     W[q, t] = math.exp(s * x @ mu[j]) * (1 + s * nu[i] @ (Kb[t] - mu[j]))
+                elif mode == "dipole_q":
+                    W[q, t] = math.exp(s * x @ mu[j]) * (1 + s * x @ (Kb[t] - mu[j]))
                 else:
                     W[q, t] = math.exp(s * (nu[i] @ Kb[t] + (x - nu[i]) @ khat[j]))
     return W
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
 def test_acausal_matches_per_token_bruteforce(orc, mode):
     Q, K, V = small_qkv(N=64, D=8, centres=5, seed=19)
     s, Cq, Ck, k1 = 1.1, 5, 9, 2
@@ -370,7 +392,7 @@ def test_acausal_matches_per_token_bruteforce(orc, mode):
     np.testing.assert_allclose(r["O"][0, 0], ref, rtol=1e-10, atol=1e-12)
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
 def test_causal_matches_per_token_bruteforce(orc, mode):
     Q, K, V = small_qkv(B=1, Hq=2, Hkv=1, N=64, D=8, centres=4, seed=20)
     N, L, C, k1, s = 64, 8, 3, 1, 0.8
