@@ -283,7 +283,7 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
                    ? dense_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck)
                    : 0;
   a.tc_lv = (sh->dtype == MUSE_BF16 && L.V16 && L.kpad)
-                ? stage2_tc_levels(L.qg.lv, pr->Cq, pr->Ck, pr->topk, a.dense_lv)
+                ? stage2_tc_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck, pr->topk, a.dense_lv)
                 : 0;
   a.kpad = L.kpad;
   a.vpad = L.vpad;

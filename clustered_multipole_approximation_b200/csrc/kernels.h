@@ -109,7 +109,7 @@ bool run_stage2_warp(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
 // Tensor-core stage 2 (stage2_tc.cu): the levels it takes, the sorted key
 // copies it reads (once per call, after the k-means) and the launch for the
 // query problems [qp0, qp0 + nqp) at those levels.
-int stage2_tc_levels(const Levels& lv, int Cq, int Ck, int topk, int dense_lv);
+int stage2_tc_levels(const Levels& lv, int D, int Cq, int Ck, int topk, int dense_lv);
 void run_permute_keys(const AttnArgs& a, cudaStream_t st);
 void run_stage2_tc(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 

@@ -754,14 +754,14 @@ __global__ void __launch_bounds__(kTT, D == 64 ? 2 : 1) stage2_tc_kernel(AttnArg
 
 // Levels whose query clusters average at least this many queries, and that
 // retrieve, take the tensor-core kernel (far-field-only tiles and small
-// clusters run better as 16-query warp slices).
-constexpr int kTcMinQueries = 64;
-
-int stage2_tc_levels(const Levels& lv, int Cq, int Ck, int topk, int dense_lv) {
+// clusters run better as 16-query warp slices; at D = 128 the warp slices are
+// register-bound, so smaller clusters already pay on the tensor cores).
+int stage2_tc_levels(const Levels& lv, int D, int Cq, int Ck, int topk, int dense_lv) {
   if (topk < 1 || topk > kTMaxSel || Cq > 256 || Ck > 256) return 0;
+  const int min_q = D == 128 ? 32 : 64;
   int m = 0;
   for (int l = 0; l < lv.nlev; ++l)
-    if (!((dense_lv >> l) & 1) && lv.s[l] >= kTcMinQueries * imin(Cq, lv.s[l]) && lv.s[l] >= kTQ)
+    if (!((dense_lv >> l) & 1) && lv.s[l] >= min_q * imin(Cq, lv.s[l]) && lv.s[l] >= kTQ)
       m |= 1 << l;
   return m;
 }
