@@ -2,7 +2,7 @@
 """Benchmark of the MuSe forward operator; rank 0 prints one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl muse|reference]
-                    [--workload NAME] [--mode dipole|monopole|tilted]
+                    [--workload NAME] [--mode dipole|monopole|tilted|dipole_q]
 
 A step is one full forward call of the operator (k-means of queries and keys,
 summaries, selection, far field + exact retrieval) over one layer of synthetic
@@ -52,7 +52,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="muse", choices=["muse", "reference"])
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
-    p.add_argument("--mode", default=None, choices=[None, "dipole", "monopole", "tilted"])
+    p.add_argument("--mode", default=None, choices=[None, "dipole", "monopole", "tilted", "dipole_q"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-side", action="store_true",
                    help="skip the other N >= 8k configurations of the default run")
@@ -144,18 +144,20 @@ TENSOR_KERNELS = ("kmeans", "stage1_summaries", "stage2_attn", "stage2_dense",
 KERNEL_GROUPS = {"kmeans_resident": "kmeans", "kmeans_ordered": "kmeans"}
 
 
-def level_table(w):
+def level_table(w, mode):
     """(block size s, pairs per head, effective clusters, per-key-token far field)
     of every level; the acausal operator is one level with one block problem.
     The per-key-token form runs where the library's dense-level rule admits it:
-    bf16 DIPOLE, C <= 256, s a multiple of 128, s <= 2048 and s <= 8 C_eff."""
+    bf16 DIPOLE, C <= 256, s a multiple of 128, s <= 2048 and s <= 8 C_eff; and
+    at every level in the fine-query mode (DIPOLE_Q)."""
+    fq = mode == "dipole_q"
     if not w.causal:
-        return [(w.N, 1, w.C, False)]
+        return [(w.N, 1, w.C, fq)]
     out, s = [], w.block
     while s < w.N:
         ce = min(w.C, s)
-        dense = (w.dtype == "bf16" and w.mode == "dipole" and w.C <= 256 and s % 128 == 0
-                 and s <= 2048 and s <= 8 * ce)
+        dense = fq or (w.dtype == "bf16" and mode == "dipole" and w.C <= 256 and s % 128 == 0
+                       and s <= 2048 and s <= 8 * ce)
         out.append((s, w.N // (2 * s), ce, dense))
         s *= 2
     return out
@@ -172,7 +174,7 @@ def retrieval_rows(w, mode, dbg):
     far = []
     exact = []
     pbase = 0
-    for lv, (s, npairs, ce, _dense) in enumerate(level_table(w)):
+    for lv, (s, npairs, ce, _dense) in enumerate(level_table(w, mode)):
         f_lv = e_lv = 0.0
         for b in range(w.B):
             for h in range(w.Hq):
@@ -209,20 +211,26 @@ def algorithmic_work(w, mode, dbg):
     (a multiply-add counts 2 FLOPs), and the operator's algorithmic bytes:
       k-means       T * 2 * tokens * C_eff * D per role (every level);
       stage 1       min(2 C_eff^2 D^2 + 2 s D^2, 4 s C_eff D) per query problem
-                    (the dipole contraction; 0 for MONOPOLE);
-      stage 2       4 D per far row and per exact retrieved key;
+                    (the dipole contraction; 0 for MONOPOLE and DIPOLE_Q);
+      stage 2       4 D per far row and per exact retrieved key; DIPOLE_Q
+                    (per key token: q.k_t, the factor's q.(k_t - mu) and
+                    the weighted v_t) 4 D per (query, key) pair of the block
+                    plus 2 D per (query, key cluster) for q.mu_j;
       local block   4 D per (query, key) pair of the causal local block;
       bytes         Q, K and V read once, O written once."""
     B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
     far, exact = retrieval_rows(w, mode, dbg)
     work = dict.fromkeys(TENSOR_KERNELS, 0.0)
-    for lv, (s, npairs, ce, dense) in enumerate(level_table(w)):
+    for lv, (s, npairs, ce, dense) in enumerate(level_table(w, mode)):
         toks = npairs * s
         work["kmeans"] += w.iters * 2.0 * toks * ce * D * B * (Hq + Hkv)
         if not dense and mode != "monopole":
             work["stage1_summaries"] += npairs * B * Hq * min(2.0 * ce * ce * D * D + 2.0 * s * D * D,
                                                               4.0 * s * ce * D)
-        work["stage2_dense" if dense else "stage2_attn"] += 4.0 * D * (far[lv] + exact[lv])
+        if mode == "dipole_q":
+            work["stage2_dense"] += B * Hq * toks * (4.0 * D * s + 2.0 * D * ce)
+        else:
+            work["stage2_dense" if dense else "stage2_attn"] += 4.0 * D * (far[lv] + exact[lv])
     if w.causal:
         L = w.block
         work["causal_local_merge"] = 4.0 * D * B * Hq * (w.N // L) * L * (L + 1) / 2

@@ -166,7 +166,7 @@ muse_status validate(const muse_shape* sh, const muse_params* pr, bool causal) {
     return fail(MUSE_ERR_INVALID_ARG, "dtype must be MUSE_BF16 or MUSE_F32");
   if (sh->out_f32 != 0 && sh->out_f32 != 1) return fail(MUSE_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
   if (pr->iters < 1) return fail(MUSE_ERR_INVALID_ARG, "iters must be >= 1");
-  if (pr->mode < MUSE_MONOPOLE || pr->mode > MUSE_TILTED)
+  if (pr->mode < MUSE_MONOPOLE || pr->mode > MUSE_DIPOLE_Q)
     return fail(MUSE_ERR_INVALID_ARG, "unknown mode");
   if (pr->Cq < 1 || pr->Ck < 1) return fail(MUSE_ERR_INVALID_ARG, "Cq and Ck must be >= 1");
   if (pr->Cq > kMaxC || pr->Ck > kMaxC)
@@ -278,10 +278,19 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   a.scale = pr->scale;
   a.Cq = pr->Cq;
   a.Ck = pr->Ck;
-  // bf16 DIPOLE causal levels with few tokens per cluster: per key token
-  a.dense_lv = (causal && sh->dtype == MUSE_BF16 && pr->mode == MUSE_DIPOLE && L.V16)
-                   ? dense_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck)
-                   : 0;
+  // bf16 DIPOLE causal levels with few tokens per cluster: per key token;
+  // the fine-query dipole: per key token at every level
+  if (pr->mode == MUSE_DIPOLE_Q) {
+    const int m = L.V16 ? fine_query_dense_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck) : -1;
+    if (m < 0)
+      return fail(MUSE_ERR_UNSUPPORTED,
+                  "DIPOLE_Q needs bf16, Cq and Ck <= 256 and block sizes that are multiples of 128");
+    a.dense_lv = m;
+  } else {
+    a.dense_lv = (causal && sh->dtype == MUSE_BF16 && pr->mode == MUSE_DIPOLE && L.V16)
+                     ? dense_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck)
+                     : 0;
+  }
   a.tc_lv = (sh->dtype == MUSE_BF16 && L.V16 && L.kpad)
                 ? stage2_tc_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck, pr->topk, a.dense_lv)
                 : 0;

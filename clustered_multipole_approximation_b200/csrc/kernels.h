@@ -123,6 +123,9 @@ void run_stage1_dipole_tc(const AttnArgs& a, const Stage1& s1, int qp0, int nqp,
 void run_stage2_dense(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 // Levels the dense form covers for these sizes (bit l set), 0 if none.
 int dense_levels(const Levels& lv, int D, int Cq, int Ck);
+// Levels of the fine-query dipole (every level, acausal included), or -1 when
+// the shape is outside the per-key-token kernel's limits.
+int fine_query_dense_levels(const Levels& lv, int D, int Cq, int Ck);
 
 // Causal: exact local block + merge of the level partials into O.
 void run_local_merge(const AttnArgs& a, int L, cudaStream_t st);

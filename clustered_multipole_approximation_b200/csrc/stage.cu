@@ -517,7 +517,10 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
   // set on every launch: the attribute is per device, and the call is cheap
   cudaFuncSetAttribute(stage1_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)stage1_smem<D>());
-  {
+  // the fine-query dipole needs no per-cluster-pair summaries: selection reads
+  // the centroids and counts, and stage 2 runs per key token at every level
+  const bool fq = a.mode == 3;
+  if (!fq) {
     ProfScope ps(st, "stage1_summaries");
     if (sizeof(T) == 2 && a.mode == 1)
       run_stage1_dipole_tc(a, s1, qp0, nqp, st);
@@ -529,7 +532,7 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
     run_select(a, s1, qp0, nqp, st);
   }
   if (sizeof(T) == 2) {
-    {
+    if (!fq) {
       ProfScope ps(st, "stage2_attn");
       run_stage2_tc(a, s1, qp0, nqp, st);
       if (!run_stage2_warp(a, s1, qp0, nqp, st)) run_stage2_mma(a, s1, qp0, nqp, st);

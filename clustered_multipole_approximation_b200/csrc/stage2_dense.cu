@@ -29,6 +29,14 @@
 // through sign-flipped nu fragments in the same accumulator, k-step by
 // k-step, so the cancellation of nu.k against nu.mu happens in fp32.  The
 // weights p f enter P V as an fp16 hi + lo pair, V in fp16.
+//
+// The fine-query dipole (mode DIPOLE_Q, an accuracy variant: u_qj = (S_j +
+// s M_j q) / n_j) is the same per-token sum with the query in place of its
+// cluster centroid: f = 1 + s q.(k_t - mu_a(t)) = 1 + s (S_ex - S_far), from
+// the two score tiles the kernel forms anyway.  It has no per-cluster form
+// short of q-dependent M_j products, so in that mode every level (and the
+// acausal layer, one block of N keys) runs here; the key clusters are then
+// read per block from global memory instead of a block table.
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -49,6 +57,7 @@ constexpr int kDTokPerCluster = 8;  // per key token where s <= 8 C
 
 template <int D>
 struct DenseBuf {
+  int kcl[kDK];                  // cluster of each key of the block
   __nv_bfloat16 k[kDK][D + 8];   // k_t
   __nv_bfloat16 mh[kDK][D + 8];  // hi part of mu_a(t)
   __nv_bfloat16 ml[kDK][D + 8];  // lo part of mu_a(t)
@@ -62,14 +71,13 @@ struct DenseSmem {
   __nv_bfloat16 nl[kDQ][D + 8];  // lo part of nu_i(q)
   DenseBuf<D> buf[2];
   unsigned rmask[kDMaxC][kDMaxC / 32];  // bit j of row i: key cluster j is in R_i
-  int kcl[kDMaxS];                      // cluster of every key of the key block
   int qcl[kDQ];                         // cluster of each query row
   int nex[kDMaxC];                      // keys of the retrieved clusters, per query cluster
 };
 
 }  // namespace
 
-template <int D>
+template <int D, bool FQ>
 __global__ void __launch_bounds__(kDThreads, D == 64 ? 2 : 1)
     stage2_dense_kernel(AttnArgs a, Stage1 s1, int qp0) {
   extern __shared__ __align__(16) unsigned char dn_raw[];
@@ -89,7 +97,6 @@ __global__ void __launch_bounds__(kDThreads, D == 64 ? 2 : 1)
   // ---- per-CTA tables ------------------------------------------------------
   const int* kas = a.ks.assign + pk.slot0;
   const int* qas = a.qs.assign + pq.slot0 + q0;
-  for (int t = tid; t < S; t += kDThreads) sm.kcl[t] = min(max(kas[t], 0), ck - 1);
   for (int r = tid; r < kDQ; r += kDThreads) sm.qcl[r] = min(max(qas[r], 0), cq - 1);
   for (int e = tid; e < cq * (kDMaxC / 32); e += kDThreads) (&sm.rmask[0][0])[e] = 0u;
   for (int i = tid; i < cq; i += kDThreads) sm.nex[i] = 0;
@@ -127,10 +134,11 @@ __global__ void __launch_bounds__(kDThreads, D == 64 ? 2 : 1)
   }
   auto issue = [&](int b, DenseBuf<D>& B) {
     const int t0 = b * kDK;
+    for (int r = tid; r < kDK; r += kDThreads) B.kcl[r] = min(max(kas[t0 + r], 0), ck - 1);
     for (int e = tid; e < kDK * CH; e += kDThreads) {
       const int r = e / CH, c = (e % CH) * 8, t = t0 + r;
       const size_t ko = (size_t)(pk.row0 + t) * D + c;
-      const size_t mo = (size_t)sm.kcl[t] * D + c;
+      const size_t mo = (size_t)min(max(kas[t], 0), ck - 1) * D + c;
       cp16(&B.k[r][c], K + ko, 16);
       cp16(&B.mh[r][c], muh + mo, 16);
       cp16(&B.ml[r][c], mul + mo, 16);
@@ -166,10 +174,12 @@ __global__ void __launch_bounds__(kDThreads, D == 64 ? 2 : 1)
 #pragma unroll
     for (int kk = 0; kk < KD; ++kk) {
       const int row = warp * 16 + (lane & 15), col = kk * 16 + (lane >> 4) * 8;
-      uint32_t qa[4], ha[4], la[4], hn[4], ln[4];
+      uint32_t qa[4], ha[4] = {0, 0, 0, 0}, la[4] = {0, 0, 0, 0}, hn[4], ln[4];
       ldsm_x4(smem_u32(&sm.q[row][col]), qa[0], qa[1], qa[2], qa[3]);
-      ldsm_x4(smem_u32(&sm.nh[row][col]), ha[0], ha[1], ha[2], ha[3]);
-      ldsm_x4(smem_u32(&sm.nl[row][col]), la[0], la[1], la[2], la[3]);
+      if (!FQ) {
+        ldsm_x4(smem_u32(&sm.nh[row][col]), ha[0], ha[1], ha[2], ha[3]);
+        ldsm_x4(smem_u32(&sm.nl[row][col]), la[0], la[1], la[2], la[3]);
+      }
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
         hn[x] = ha[x] ^ 0x80008000u;  // -nu_hi (sign bit of both bf16 halves)
@@ -183,23 +193,35 @@ __global__ void __launch_bounds__(kDThreads, D == 64 ? 2 : 1)
         ldsm_x4(smem_u32(&B.k[key][kc_]), b0, b1, b2, b3);
         mma_bf16(sx[2 * np], qa, b0, b1);
         mma_bf16(sx[2 * np + 1], qa, b2, b3);
-        mma_bf16(fd[2 * np], ha, b0, b1);
-        mma_bf16(fd[2 * np + 1], ha, b2, b3);
-        mma_bf16(fd[2 * np], la, b0, b1);
-        mma_bf16(fd[2 * np + 1], la, b2, b3);
+        if (!FQ) {
+          mma_bf16(fd[2 * np], ha, b0, b1);
+          mma_bf16(fd[2 * np + 1], ha, b2, b3);
+          mma_bf16(fd[2 * np], la, b0, b1);
+          mma_bf16(fd[2 * np + 1], la, b2, b3);
+        }
         ldsm_x4(smem_u32(&B.mh[key][kc_]), b0, b1, b2, b3);
         mma_bf16(sf[2 * np], qa, b0, b1);
         mma_bf16(sf[2 * np + 1], qa, b2, b3);
-        mma_bf16(fd[2 * np], hn, b0, b1);
-        mma_bf16(fd[2 * np + 1], hn, b2, b3);
-        mma_bf16(fd[2 * np], ln, b0, b1);
-        mma_bf16(fd[2 * np + 1], ln, b2, b3);
+        if (!FQ) {
+          mma_bf16(fd[2 * np], hn, b0, b1);
+          mma_bf16(fd[2 * np + 1], hn, b2, b3);
+          mma_bf16(fd[2 * np], ln, b0, b1);
+          mma_bf16(fd[2 * np + 1], ln, b2, b3);
+        }
         ldsm_x4(smem_u32(&B.ml[key][kc_]), b0, b1, b2, b3);
         mma_bf16(sf[2 * np], qa, b0, b1);
         mma_bf16(sf[2 * np + 1], qa, b2, b3);
-        mma_bf16(fd[2 * np], hn, b0, b1);
-        mma_bf16(fd[2 * np + 1], hn, b2, b3);
+        if (!FQ) {
+          mma_bf16(fd[2 * np], hn, b0, b1);
+          mma_bf16(fd[2 * np + 1], hn, b2, b3);
+        }
       }
+    }
+    if (FQ) {  // q.(k_t - mu_a(t)) from the exact and far scores
+#pragma unroll
+      for (int n = 0; n < kDK / 8; ++n)
+#pragma unroll
+        for (int h = 0; h < 4; ++h) fd[n][h] = sx[n][h] - sf[n][h];
     }
     // exact or far term per (row, key); running maximum of the chosen logits
     const int t0 = b * kDK;
@@ -208,7 +230,7 @@ __global__ void __launch_bounds__(kDThreads, D == 64 ? 2 : 1)
     for (int n = 0; n < kDK / 8; ++n) {
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        const int j = sm.kcl[t0 + n * 8 + 2 * t4 + (h & 1)];
+        const int j = B.kcl[n * 8 + 2 * t4 + (h & 1)];
         const bool ex = (mrow_bits[h >> 1][j >> 5] >> (j & 31)) & 1u;
         const float lg = sl2 * (ex ? sx[n][h] : sf[n][h]);
         fd[n][h] = ex ? 1.f : fmaf(s, fd[n][h], 1.f);
@@ -271,12 +293,28 @@ __global__ void __launch_bounds__(kDThreads, D == 64 ? 2 : 1)
     }
     __syncthreads();
   }
-  // ---- the level partial of each row: normalised output and log-sum-exp ------
+  // ---- each row: the normalised output (acausal), or the level partial:
+  // normalised output and log-sum-exp (causal) -------------------------------
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     const int tq = q0 + r0 + 8 * r;  // problem-local query index
-    float* pp = a.part + (size_t)(pq.slot0 + tq) * (D + 1);
     const float inv = 1.f / lrow[r];
+    if (FQ && a.O != nullptr) {  // only the fine-query dipole runs acausal layers here
+      const long long orow = pq.row0 + tq;
+#pragma unroll
+      for (int n = 0; n < ND; ++n) {
+        const float x0 = o[n][2 * r] * inv, x1 = o[n][2 * r + 1] * inv;
+        if (a.out_f32) {
+          *reinterpret_cast<float2*>(static_cast<float*>(a.O) + orow * D + n * 8 + 2 * t4) = make_float2(x0, x1);
+        } else {
+          *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.O) + orow * D + n * 8 + 2 * t4) =
+              __floats2bfloat162_rn(x0, x1);
+        }
+      }
+      if (t4 == 0 && a.n_exact != nullptr) a.n_exact[orow] = sm.nex[sm.qcl[r0 + 8 * r]];
+      continue;
+    }
+    float* pp = a.part + (size_t)(pq.slot0 + tq) * (D + 1);
 #pragma unroll
     for (int n = 0; n < ND; ++n) {
       pp[n * 8 + 2 * t4] = o[n][2 * r] * inv;
@@ -291,14 +329,14 @@ __global__ void __launch_bounds__(kDThreads, D == 64 ? 2 : 1)
   }
 }
 
-template <int D>
+template <int D, bool FQ>
 static void launch_dense(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, int smax,
                          cudaStream_t st) {
   // set on every launch: the attribute is per device, and the call is cheap
-  cudaFuncSetAttribute(stage2_dense_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaFuncSetAttribute(stage2_dense_kernel<D, FQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)sizeof(DenseSmem<D>));
   const dim3 grid(nqp, smax / kDQ);
-  stage2_dense_kernel<D><<<grid, kDThreads, sizeof(DenseSmem<D>), st>>>(a, s1, qp0);
+  stage2_dense_kernel<D, FQ><<<grid, kDThreads, sizeof(DenseSmem<D>), st>>>(a, s1, qp0);
 }
 
 int dense_levels(const Levels& lv, int D, int Cq, int Ck) {
@@ -311,16 +349,30 @@ int dense_levels(const Levels& lv, int D, int Cq, int Ck) {
   return m;
 }
 
+int fine_query_dense_levels(const Levels& lv, int D, int Cq, int Ck) {
+  if ((D != 64 && D != 128) || Cq > kDMaxC || Ck > kDMaxC) return -1;
+  int m = 0;
+  for (int l = 0; l < lv.nlev; ++l) {
+    if (lv.s[l] % kDQ != 0) return -1;
+    m |= 1 << l;
+  }
+  return m;
+}
+
 void run_stage2_dense(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st) {
   int smax = 0;
   for (int l = 0; l < a.qg.lv.nlev; ++l)
     if ((a.dense_lv >> l) & 1) smax = smax > a.qg.lv.s[l] ? smax : a.qg.lv.s[l];
   if (smax == 0) return;
   ProfScope ps(st, "stage2_dense");
-  if (a.qg.D == 64)
-    launch_dense<64>(a, s1, qp0, nqp, smax, st);
-  else
-    launch_dense<128>(a, s1, qp0, nqp, smax, st);
+  const bool fq = a.mode == 3;
+  if (a.qg.D == 64) {
+    if (fq) launch_dense<64, true>(a, s1, qp0, nqp, smax, st);
+    else launch_dense<64, false>(a, s1, qp0, nqp, smax, st);
+  } else {
+    if (fq) launch_dense<128, true>(a, s1, qp0, nqp, smax, st);
+    else launch_dense<128, false>(a, s1, qp0, nqp, smax, st);
+  }
 }
 
 }  // namespace muse

@@ -82,8 +82,20 @@ typedef enum { MUSE_BF16 = 0, MUSE_F32 = 1 } muse_dtype;
  *   DIPOLE    MONOPOLE plus the first-order correction (s/n_j) M_j nu_i with
  *             M_j = sum_{t in j} v_t (k_t - mu_j)^T ([A1] Abstract);
  *   TILTED    exponentially tilted summaries weighted by exp(s nu_i . k_t)
- *             ([G] Core Mechanisms, "Exponential Tilting"). */
-typedef enum { MUSE_MONOPOLE = 0, MUSE_DIPOLE = 1, MUSE_TILTED = 2 } muse_mode;
+ *             ([G] Core Mechanisms, "Exponential Tilting");
+ *   DIPOLE_Q  an accuracy variant of DIPOLE: the first-order correction is
+ *             taken at each query, (s/n_j) M_j q, instead of at its cluster
+ *             centroid nu_i ([A1] Abstract: the dipole expands exp(s q.k)
+ *             around the centroid of the keys, and q is the expansion's own
+ *             variable).  Selection is the same as DIPOLE's.  The far field
+ *             is evaluated as one softmax term per key token (weight
+ *             exp(s q.mu_a(t)), value factor 1 + s q.(k_t - mu_a(t))),
+ *             O(N^2 D) work like exact attention, so it serves as an
+ *             accuracy reference rather than a fast path.  Supported for
+ *             dtype MUSE_BF16 with Cq, Ck <= 256 and every block size (N for
+ *             muse_attn_fwd, L 2^l for muse_causal_fwd) a multiple of 128;
+ *             other shapes return MUSE_ERR_UNSUPPORTED. */
+typedef enum { MUSE_MONOPOLE = 0, MUSE_DIPOLE = 1, MUSE_TILTED = 2, MUSE_DIPOLE_Q = 3 } muse_mode;
 
 typedef struct {
   int B, Hq, Hkv, N, D; /* D in {64, 128}; Hq % Hkv == 0 */

@@ -46,8 +46,13 @@ def test_counted_retrieval_matches_exact_key_counts_acausal():
 
 def test_level_table_tiles_the_causal_decomposition():
     w = WORKLOADS["causal-gqa32x8-n64k-d64"]
-    lt = bench.level_table(w)
+    lt = bench.level_table(w, "dipole")
     assert [s for s, *_ in lt] == [1024 << l for l in range(6)]
     assert sum(npairs for _, npairs, _, _ in lt) == w.N // w.block - 1
     assert [d for *_, d in lt] == [True, True, False, False, False, False]
-    assert bench.level_table(WORKLOADS["acausal-bf16-h8-n8k"]) == [(8192, 1, 128, False)]
+    assert [d for *_, d in bench.level_table(w, "monopole")] == [False] * 6
+    # the fine-query dipole runs per key token at every level, acausal included
+    assert [d for *_, d in bench.level_table(w, "dipole_q")] == [True] * 6
+    a = WORKLOADS["acausal-bf16-h8-n8k"]
+    assert bench.level_table(a, "dipole") == [(8192, 1, 128, False)]
+    assert bench.level_table(a, "dipole_q") == [(8192, 1, 128, True)]

@@ -425,6 +425,85 @@ def test_causal_never_reads_the_future_on_gpu():
         assert (o[:, :, : t0 + 1] == base[:, :, : t0 + 1]).all(), t0
 
 
+# ---------------------------------------------------------------------------
+# fine-query dipole: the first-order term taken at each query (M_j q)
+def _stages_launched(fn):
+    muse.profile_read()
+    muse.profile_enable(True)
+    try:
+        out = fn()
+    finally:
+        muse.profile_enable(False)
+        launched = muse.profile_read()
+    return out, launched
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("topk", [0, 3])
+def test_small_acausal_fine_query_dipole(D, topk):
+    """GQA, Cq != Ck, every head against the oracle; the far field runs per
+    key token (the per-cluster-pair summaries are not formed)."""
+    Q, K, V = clustered_qkv(2, 4, 2, 1024, D, 12, 0.3, 0.5, "bf16", 90 + D + topk)
+    _, launched = _stages_launched(
+        lambda: check_acausal(Q, K, V, "bf16", 13, 5, 77, topk, 1.0, "dipole_q", Cq=11))
+    assert "stage2_dense" in launched, launched
+    assert "stage1_summaries" not in launched and "stage2_attn" not in launched, launched
+
+
+def test_fine_query_dipole_is_closer_to_exact_than_dipole():
+    """Taking the dipole at each query instead of at its cluster centroid
+    removes the (q - nu_i) part of the expansion error: on a spread-out
+    layer the GPU's fine-query output is nearer exact attention."""
+    Q, K, V = clustered_qkv(1, 2, 2, 2048, 64, 8, 0.6, 0.0, "bf16", 95)
+    Oq, _ = gpu_acausal(Q, K, V, "bf16", 32, 6, 5, 2, 1.0, "dipole_q")
+    Od, _ = gpu_acausal(Q, K, V, "bf16", 32, 6, 5, 2, 1.0, "dipole")
+    E = oracle.exact_attention(Q, K, V)
+    assert rse(Oq, E) < rse(Od, E), (rse(Oq, E), rse(Od, E))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_small_causal_fine_query_dipole(D):
+    """Every level (s = 128, 256, 512) per key token, every head."""
+    Q, K, V = clustered_qkv(1, 4, 2, 1024, D, 8, 0.3, 0.0, "bf16", 96 + D)
+    _, launched = _stages_launched(
+        lambda: check_causal(Q, K, V, "bf16", 128, 12, 4, 21, 2, 1.0, "dipole_q"))
+    assert "stage2_dense" in launched and "stage2_attn" not in launched, launched
+
+
+def test_workload_acausal_bf16_h8_n8k_fine_query_dipole():
+    """The 8-head 8k layer in the fine-query mode, heads 0 and 5 against the
+    oracle."""
+    w = WORKLOADS["acausal-bf16-h8-n8k"]
+    Q, K, V = make_inputs(w)
+    check_acausal(Q, K, V, w.dtype, w.C, w.iters, w.cluster_seed, w.topk, w.scale, "dipole_q",
+                  heads=[(0, 0), (0, 5)])
+
+
+def test_workload_causal_b2h8_n16k_fine_query_dipole():
+    """The 16k causal layer in the fine-query mode (levels s = 512 .. 8192
+    per key token), head (1, 3) against the oracle."""
+    w = WORKLOADS["causal-bf16-b2h8-n16k"]
+    Q, K, V = make_inputs(w)
+    check_causal(Q, K, V, w.dtype, w.block, w.C, w.iters, w.cluster_seed, w.topk, w.scale,
+                 "dipole_q", heads=[(1, 3)])
+
+
+@pytest.mark.parametrize("case", ["f32", "n_not_128", "block_not_128", "clusters_above_256"])
+def test_fine_query_dipole_unsupported_shapes_are_refused(case):
+    dtype = "f32" if case == "f32" else "bf16"
+    N = 1000 if case == "n_not_128" else 1024
+    Q, K, V = clustered_qkv(1, 1, 1, N, 64, 8, 0.3, 0.0, dtype, 97)
+    q, k, v = to_dev(Q, dtype), to_dev(K, dtype), to_dev(V, dtype)
+    with pytest.raises(muse.MuseError, match="DIPOLE_Q"):
+        if case == "block_not_128":
+            muse.muse_attn_fwd_causal(q, k, v, C=8, block=64, iters=2, seed=1, topk=1,
+                                      mode="dipole_q")
+        else:
+            C = 300 if case == "clusters_above_256" else 8
+            muse.muse_attn_fwd(q, k, v, Cq=C, Ck=C, iters=2, seed=1, topk=1, mode="dipole_q")
+    torch.cuda.synchronize()
+
+
 def test_workload_causal_b2h8_n16k():
     """The B=2, H=8 16k causal layer, every head against the oracle."""
     w = WORKLOADS["causal-bf16-b2h8-n16k"]
