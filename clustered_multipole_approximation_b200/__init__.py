@@ -57,7 +57,8 @@ class muse_debug(ctypes.Structure):
 EXPORTS = ["muse_workspace_size", "muse_cluster_workspace_size", "muse_cluster", "muse_summarize",
            "muse_attn_fwd", "muse_attn_fwd_causal", "muse_status_string", "muse_last_error",
            "muse_profile_enable", "muse_profile_read", "muse_cluster_static",
-           "muse_cluster_static_capacity", "muse_device_status", "muse_debug_inject_barrier_fault"]
+           "muse_cluster_static_capacity", "muse_device_status", "muse_debug_inject_barrier_fault",
+           "muse_attn_bwd_workspace_size", "muse_attn_bwd"]
 
 # Bits of the device error word (include/muse.h MUSE_DEVERR_*).
 DEVERR = {1: "MUSE_DEVERR_MMA_WAIT", 2: "MUSE_DEVERR_TEAM_BARRIER", 4: "MUSE_DEVERR_V_RANGE"}
@@ -90,6 +91,10 @@ def load_library(path: str = LIB_PATH):
     for f in ("muse_attn_fwd", "muse_attn_fwd_causal"):
         getattr(lib, f).restype = i32
         getattr(lib, f).argtypes = [vp, vp, vp, vp, sp, pp, dp, vp, sz, vp]
+    lib.muse_attn_bwd_workspace_size.restype = sz
+    lib.muse_attn_bwd_workspace_size.argtypes = [sp, pp]
+    lib.muse_attn_bwd.restype = i32
+    lib.muse_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, sp, pp, vp, sz, vp]
     lib.muse_status_string.restype = ctypes.c_char_p
     lib.muse_status_string.argtypes = [i32]
     lib.muse_last_error.restype = ctypes.c_char_p
@@ -236,6 +241,63 @@ def muse_attn_fwd_causal(q, k, v, *, C, block, iters, seed, topk, scale=1.0, mod
     per level and role)."""
     p = make_params(C, C, iters, seed, topk, block, scale, mode, key_stream0, query_stream0)
     return _attn(True, q, k, v, p, out, workspace, debug, stream, out_dtype)
+
+
+def backward_workspace_size(q, k, params: muse_params, out_f32: bool = False) -> int:
+    """Workspace bytes for a muse_attn_fwd call followed by muse_attn_bwd."""
+    lib = load_library()
+    sh = make_shape(q, k, out_f32)
+    n = lib.muse_attn_bwd_workspace_size(ctypes.byref(sh), ctypes.byref(params))
+    if n == 0:
+        raise MuseError(3, lib.muse_last_error().decode())
+    return int(n)
+
+
+def muse_attn_bwd(q, k, v, do, *, Cq, Ck, iters, seed, topk, scale=1.0, mode="dipole",
+                  workspace, stream=None, key_stream0=0, query_stream0=0):
+    """Gradients (dq, dk, dv) in fp32 of <do, O> for the acausal forward call
+    made with this `workspace` (sized by backward_workspace_size) and these
+    parameters; see muse_attn_bwd in include/muse.h."""
+    lib = load_library()
+    _need_cuda(q, k, v, do, workspace)
+    if do.shape != q.shape or do.dtype not in (q.dtype, torch.float32):
+        raise ValueError("do must be [B,Hq,N,D] in the input dtype or float32")
+    p = make_params(Cq, Ck, iters, seed, topk, 0, scale, mode, key_stream0, query_stream0)
+    sh = make_shape(q, k, do.dtype == torch.float32 and q.dtype != torch.float32)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    st = lib.muse_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                           ctypes.byref(sh), ctypes.byref(p), _ptr(workspace),
+                           workspace.numel(), _stream(stream))
+    _check(lib, st)
+    return dq, dk, dv
+
+
+class MuseAttention(torch.autograd.Function):
+    """Acausal MuSe as a differentiable op: forward and backward both run in
+    libmuse (the forward's workspace is kept for the backward)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, Cq, Ck, iters, seed, topk, scale, mode):
+        p = make_params(Cq, Ck, iters, seed, topk, 0, scale, mode)
+        ws = torch.empty(backward_workspace_size(q, k, p), dtype=torch.uint8, device=q.device)
+        o = _attn(False, q, k, v, p, None, ws, False, None, None)
+        ctx.save_for_backward(q, k, v, ws)
+        ctx.args = dict(Cq=Cq, Ck=Ck, iters=iters, seed=seed, topk=topk, scale=scale, mode=mode)
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, ws = ctx.saved_tensors
+        dq, dk, dv = muse_attn_bwd(q, k, v, do.contiguous().to(q.dtype), workspace=ws,
+                                   **ctx.args)
+        return (dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype)) + (None,) * 7
+
+
+def muse_attention(q, k, v, *, Cq, Ck, iters, seed, topk, scale=1.0, mode="dipole"):
+    """Differentiable acausal MuSe (see MuseAttention)."""
+    return MuseAttention.apply(q, k, v, Cq, Ck, iters, seed, topk, scale, mode)
 
 
 def device_status(device_error, stream=None) -> None:

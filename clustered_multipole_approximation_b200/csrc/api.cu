@@ -352,6 +352,37 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   return check_launch();
 }
 
+// The backward pass's scratch, carved after the forward's part of the
+// workspace (base == nullptr: sizes only).
+struct BwdLayout {
+  BwdArgs b;
+  size_t bytes;
+};
+
+BwdLayout bwd_layout(const muse_shape* sh, const muse_params* pr, const AttnLayout& L, void* ws) {
+  BwdLayout r{};
+  Carver cv{static_cast<char*>(ws)};
+  cv.used = L.bytes;
+  const size_t nk = L.ks.nprob, nq = L.qs.nprob, D = sh->D, Cq = pr->Cq, Ck = pr->Ck;
+  const bool dip = pr->mode == MUSE_DIPOLE;
+  r.b.Sst = cv.take<float>(nk * Ck * D * 4);
+  r.b.Mst = dip ? cv.take<float>(nk * Ck * D * D * 4) : nullptr;
+  r.b.U = dip ? cv.take<float>(nq * Cq * Ck * D * 4) : nullptr;
+  r.b.dU = cv.take<float>(nq * Cq * Ck * D * 4);
+  r.b.dmu = cv.take<float>(nk * Ck * D * 4);
+  r.b.dnu = cv.take<float>(nq * Cq * D * 4);
+  r.bytes = cv.used + 256;
+  return r;
+}
+
+muse_status validate_bwd(const muse_shape* sh, const muse_params* pr) {
+  muse_status s = validate(sh, pr, false);
+  if (s != MUSE_OK) return s;
+  if (!backward_supported(sh->D, pr->Ck, (int)pr->mode))
+    return fail(MUSE_ERR_UNSUPPORTED, "the backward pass needs mode MONOPOLE or DIPOLE and Ck * D <= 16384");
+  return MUSE_OK;
+}
+
 }  // namespace
 
 namespace muse {
@@ -363,6 +394,58 @@ extern "C" {
 size_t muse_workspace_size(const muse_shape* shape, const muse_params* params, int causal) {
   if (validate(shape, params, causal != 0) != MUSE_OK) return 0;
   return layout(shape, params, causal != 0, nullptr, nullptr, nullptr).bytes;
+}
+
+size_t muse_attn_bwd_workspace_size(const muse_shape* shape, const muse_params* params) {
+  if (validate_bwd(shape, params) != MUSE_OK) return 0;
+  const AttnLayout L = layout(shape, params, false, nullptr, nullptr, nullptr);
+  return bwd_layout(shape, params, L, nullptr).bytes;
+}
+
+muse_status muse_attn_bwd(const void* Q, const void* K, const void* V, const void* dO, float* dQ,
+                          float* dK, float* dV, const muse_shape* sh, const muse_params* pr,
+                          void* ws, size_t ws_bytes, cudaStream_t st) {
+  muse_status s = validate_bwd(sh, pr);
+  if (s != MUSE_OK) return s;
+  if (!Q || !K || !V || !dO || !dQ || !dK || !dV)
+    return fail(MUSE_ERR_INVALID_ARG, "Q, K, V, dO, dQ, dK and dV must not be NULL");
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(dO, 16) ||
+      misaligned(dQ, 16) || misaligned(dK, 16) || misaligned(dV, 16))
+    return fail(MUSE_ERR_INVALID_ARG, "all tensors must be 16-byte aligned");
+  if (misaligned(ws, 256)) return fail(MUSE_ERR_INVALID_ARG, "the workspace must be 256-byte aligned");
+  const AttnLayout need = layout(sh, pr, false, Q, K, nullptr);
+  if (!ws || ws_bytes < bwd_layout(sh, pr, need, nullptr).bytes)
+    return fail(MUSE_ERR_WORKSPACE, "workspace too small for the backward pass");
+  AttnLayout L = layout(sh, pr, false, Q, K, ws);
+  AttnArgs a{};
+  a.qg = L.qg;
+  a.kg = L.kg;
+  a.qs = L.qs;
+  a.ks = L.ks;
+  a.V = V;
+  a.B = sh->B;
+  a.G = sh->Hq / sh->Hkv;
+  a.mode = (int)pr->mode;
+  a.topk = pr->topk;
+  a.scale = pr->scale;
+  a.Cq = pr->Cq;
+  a.Ck = pr->Ck;
+  BwdLayout bl = bwd_layout(sh, pr, L, ws);
+  BwdArgs& b = bl.b;
+  b.dO = dO;
+  b.o_f32 = (sh->out_f32 || sh->dtype == MUSE_F32) ? 1 : 0;
+  b.dQ = dQ;
+  b.dK = dK;
+  b.dV = dV;
+  const size_t kv = (size_t)sh->B * sh->Hkv * sh->N * sh->D * 4;
+  cudaMemsetAsync(dK, 0, kv, st);
+  cudaMemsetAsync(dV, 0, kv, st);
+  const size_t nq = L.qs.nprob, nk = L.ks.nprob;
+  cudaMemsetAsync(b.dU, 0, nq * pr->Cq * pr->Ck * sh->D * 4, st);
+  cudaMemsetAsync(b.dmu, 0, nk * pr->Ck * sh->D * 4, st);
+  cudaMemsetAsync(b.dnu, 0, nq * pr->Cq * sh->D * 4, st);
+  run_attn_bwd(a, L.s1, b, st);
+  return check_launch();
 }
 
 size_t muse_cluster_workspace_size(int B, int H, int N, int D, int C) {

@@ -1,0 +1,688 @@
+// Gradients of the acausal operator with respect to Q, K and V.
+//
+// The pages train models with MuSe as the attention layer (gist.science page
+// "Multipole Semantic Attention: A Fast Approximation of Softmax Attention
+// for Pretraining", Experimental Results), so the layer has a backward pass.
+// The clusterings and the retrieval sets are piecewise constant in the inputs
+// and are held at the forward pass's values; everything else is
+// differentiated as the function of Q, K and V it is:
+//   mu_j = (1/n_j) sum_{a(t)=j} k_t,  S_j = sum v_t,  M_j = sum v_t (k_t - mu_j)^T,
+//   nu_i = (1/m_i) sum_{b(q)=i} q,
+//   u_ij = S_j / n_j (MONOPOLE)   or   (S_j + s M_j nu_i) / n_j (DIPOLE),
+// and the output of query q (cluster i) is one softmax over the far terms
+// (j outside R_i, n_j > 0: logit s q.mu_j + log n_j, value u_ij) and the
+// exact terms (keys of the clusters in R_i: logit s q.k_t, value v_t).
+//
+// With lse_q the log-sum-exp of the query's logits, per term p = exp(l -
+// lse_q) and g = dO_q . x (x the term's value), D_q = sum p g (= dO_q . O_q,
+// formed here from the same fp32 terms rather than read from the forward's
+// rounded output) and dl = p (g - D_q):
+//   exact t:  dq += s dl k_t,  dk_t += s dl q,  dv_t += p dO_q
+//   far j:    dq += s dl mu_j, dmu_j += s dl q, du_ij += p dO_q
+// and through the summaries (sums over the query clusters i of every q-head
+// that reads key set j):
+//   dS_j = sum_i du_ij / n_j
+//   dM_j = (s / n_j) sum_i du_ij nu_i^T,   dnu_i += (s / n_j) M_j^T du_ij
+//   dmu_j -= dM_j^T S_j                     (M_j's own dependence on mu_j)
+//   dv_t += dS_j + dM_j (k_t - mu_j),  dk_t += dmu_j / n_j + dM_j^T v_t
+//   dq   += dnu_i / m_i.
+//
+// Kernels (fp32 arithmetic throughout, gradients in fp32):
+//   bwd_key_stats   one CTA per (key set, cluster): S_j and M_j from the
+//                   cluster-sorted members;
+//   bwd_u_table     (DIPOLE) one CTA per (query set, key cluster): u_ij for
+//                   every query cluster i;
+//   bwd_query       one CTA per (query set, query cluster i), chunks of 32
+//                   member queries: log-sum-exp and D_q (the exact tiles'
+//                   terms online, the far terms' g kept per (query, cluster)),
+//                   the far terms (du_ij owned by the CTA, dmu_j by
+//                   atomics), then the exact tiles of R_i's clusters (dk, dv
+//                   by atomics);
+//   bwd_cluster     one CTA per (key set, cluster): dS_j, dM_j, dnu, and the
+//                   chain to the members' dk and dv;
+//   bwd_query_nu    dq += dnu_i / m_i.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace muse {
+
+namespace {
+
+constexpr int kBT = 256;  // threads per CTA
+constexpr int kBW = kBT / 32;
+constexpr int kQC = 32;   // queries per chunk
+constexpr int kKC = 32;   // keys per exact tile
+
+template <typename T>
+__device__ inline float ldg_(const T* p) {
+  return ld<T>(p);
+}
+
+// ---------------------------------------------------------------------------
+// S_j and M_j[e][d] = sum_t v_t[e] (k_t[d] - mu_j[d])
+// ---------------------------------------------------------------------------
+template <typename T, int D, bool DIP>
+__global__ void __launch_bounds__(kBT) bwd_key_stats_kernel(AttnArgs a, BwdArgs b) {
+  __shared__ float kt[kKC][D + 1];
+  __shared__ float vt[kKC][D + 1];
+  __shared__ float mu[D];
+  const int kpid = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+  const int Ck = a.Ck;
+  const Prob pk = prob_of(a.kg, kpid);
+  const size_t cj = (size_t)kpid * Ck + j;
+  const int n = j < pk.C ? a.ks.counts[cj] : 0;
+  const int off = n > 0 ? a.ks.off[(size_t)kpid * (Ck + 1) + j] : 0;
+  const int* perm = a.ks.perm + pk.slot0;
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  for (int d = tid; d < D; d += kBT) mu[d] = a.ks.cent32[cj * D + d];
+  constexpr int MR = DIP ? D * D / kBT : 0;
+  float m[MR > 0 ? MR : 1];
+#pragma unroll
+  for (int r = 0; r < (MR > 0 ? MR : 1); ++r) m[r] = 0.f;
+  float sacc = 0.f;
+  for (int c0 = 0; c0 < n; c0 += kKC) {
+    const int cnt = imin(kKC, n - c0);
+    __syncthreads();
+    for (int e = tid; e < cnt * D; e += kBT) {
+      const int r = e / D, d = e - r * D;
+      const long long row = pk.row0 + perm[off + c0 + r];
+      kt[r][d] = ldg_<T>(K + row * D + d) - mu[d];
+      vt[r][d] = ldg_<T>(V + row * D + d);
+    }
+    __syncthreads();
+    if (tid < D)
+      for (int t = 0; t < cnt; ++t) sacc += vt[t][tid];
+    if (DIP) {
+#pragma unroll
+      for (int r = 0; r < MR; ++r) {
+        const int idx = tid + kBT * r, e = idx / D, d = idx - e * D;
+        float x = m[r];
+        for (int t = 0; t < cnt; ++t) x = fmaf(vt[t][e], kt[t][d], x);
+        m[r] = x;
+      }
+    }
+  }
+  if (tid < D) b.Sst[cj * D + tid] = sacc;
+  if (DIP) {
+#pragma unroll
+    for (int r = 0; r < MR; ++r) b.Mst[cj * D * D + tid + kBT * r] = m[r];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// u_ij = (S_j + s M_j nu_i) / n_j for every query cluster i (DIPOLE)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kBT) bwd_u_table_kernel(AttnArgs a, BwdArgs b) {
+  extern __shared__ __align__(16) float ut_raw[];
+  float* M = ut_raw;                   // [D][D + 1]
+  float* nu = M + D * (D + 1);         // [kBT / D][D]
+  const int qpid = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+  const int Cq = a.Cq, Ck = a.Ck;
+  const int kpid = kv_problem(a, qpid);
+  const Prob pq = prob_of(a.qg, qpid);
+  const Prob pk = prob_of(a.kg, kpid);
+  const size_t cj = (size_t)kpid * Ck + j;
+  const int n = j < pk.C ? a.ks.counts[cj] : 0;
+  float* U = b.U + ((size_t)qpid * Cq * Ck + j) * D;  // row (i, j) at U + i * Ck * D
+  if (n == 0) {
+    for (int e = tid; e < pq.C * D; e += kBT) U[(size_t)(e / D) * Ck * D + e % D] = 0.f;
+    return;
+  }
+  for (int e = tid; e < D * D; e += kBT) M[(e / D) * (D + 1) + e % D] = b.Mst[cj * D * D + e];
+  constexpr int RI = kBT / D;  // query clusters per pass
+  const int e = tid % D, ri = tid / D;
+  const float s = a.scale, inv = 1.f / (float)n, Se = b.Sst[cj * D + e];
+  const float* cent = a.qs.cent32 + (size_t)qpid * Cq * D;
+  for (int i0 = 0; i0 < pq.C; i0 += RI) {
+    __syncthreads();
+    if (i0 + ri < pq.C) nu[ri * D + e] = cent[(size_t)(i0 + ri) * D + e];
+    __syncthreads();
+    if (i0 + ri < pq.C) {
+      float x = 0.f;
+#pragma unroll 8
+      for (int d = 0; d < D; ++d) x = fmaf(M[e * (D + 1) + d], nu[ri * D + d], x);
+      U[(size_t)(i0 + ri) * Ck * D + e] = fmaf(s, x, Se) * inv;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// per (query set, query cluster): the softmax's own gradient
+// ---------------------------------------------------------------------------
+template <int D>
+struct QuerySmem {
+  float q[kQC][D + 1];
+  float go[kQC][D + 1];  // dO
+  float kt[kKC][D + 1];
+  float vt[kKC][D + 1];
+  float pt[kQC][kKC];
+  float dst[kQC][kKC];
+  float lse[kQC];
+  float dq_[kQC];  // D_q
+  float dex[kQC];  // exact terms' sum of exp(l - m) g, at the running max m
+  float mq[kQC];   // running max
+  int row[kQC];
+  unsigned rmask[kMaxC / 32];
+};
+
+template <typename T, typename TO, int D, bool DIP>
+__global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, BwdArgs b) {
+  extern __shared__ __align__(16) unsigned char bq_raw[];
+  QuerySmem<D>& sm = *reinterpret_cast<QuerySmem<D>*>(bq_raw);
+  const int Cq = a.Cq, Ck = a.Ck;
+  float* mu_s = reinterpret_cast<float*>(bq_raw + sizeof(QuerySmem<D>));  // [Ck][D + 1]
+  float* lf = mu_s + (size_t)Ck * (D + 1);                               // [kQC][Ck]
+  float* gf = lf + (size_t)kQC * Ck;                                      // [kQC][Ck] dO.u
+  int* fl = reinterpret_cast<int*>(gf + (size_t)kQC * Ck);               // far clusters
+  int* xl = fl + Ck;                                                      // exact clusters
+  __shared__ int nfar, nex;
+  const int qpid = blockIdx.x, i = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const Prob pq = prob_of(a.qg, qpid);
+  if (i >= pq.C) return;
+  const int mi = a.qs.counts[(size_t)qpid * Cq + i];
+  if (mi == 0) return;
+  const int kpid = kv_problem(a, qpid);
+  const Prob pk = prob_of(a.kg, kpid);
+  const int ck = pk.C;
+  const int* kcnt = a.ks.counts + (size_t)kpid * Ck;
+  const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
+  const int* kperm = a.ks.perm + pk.slot0;
+  const int qoff = a.qs.off[(size_t)qpid * (Cq + 1) + i];
+  const int* qperm = a.qs.perm + pq.slot0;
+  const T* Q = static_cast<const T*>(a.qg.X);
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  const TO* GO = static_cast<const TO*>(b.dO);
+  const float s = a.scale;
+  constexpr int DL = D / 32;  // elements per lane
+
+  // retrieval set, far / exact cluster lists, centroid table
+  for (int w = tid; w < kMaxC / 32; w += kBT) sm.rmask[w] = 0u;
+  __syncthreads();
+  if (a.topk > 0) {
+    const int ns = s1.nsel[(size_t)qpid * Cq + i];
+    for (int r = tid; r < ns; r += kBT) {
+      const int j = s1.sel[((size_t)qpid * Cq + i) * a.topk + r];
+      if (j >= 0 && j < ck) atomicOr(&sm.rmask[j >> 5], 1u << (j & 31));
+    }
+  }
+  for (int e = tid; e < ck * D; e += kBT) {
+    const int j = e / D, d = e - j * D;
+    mu_s[j * (D + 1) + d] = a.ks.cent32[((size_t)kpid * Ck + j) * D + d];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int nf = 0, nx = 0;
+    for (int j = 0; j < ck; ++j) {
+      if (kcnt[j] == 0) continue;
+      if ((sm.rmask[j >> 5] >> (j & 31)) & 1u) xl[nx++] = j;
+      else fl[nf++] = j;
+    }
+    nfar = nf;
+    nex = nx;
+  }
+  __syncthreads();
+  const int nf = nfar, nx = nex;
+
+  for (int c0 = 0; c0 < mi; c0 += kQC) {
+    const int qc = imin(kQC, mi - c0);
+    // ---- chunk rows: q, dO, D_q ------------------------------------------
+    __syncthreads();
+    if (tid < qc) sm.row[tid] = (int)(pq.row0 + qperm[qoff + c0 + tid]);
+    __syncthreads();
+    for (int e = tid; e < qc * D; e += kBT) {
+      const int r = e / D, d = e - r * D;
+      const long long row = sm.row[r];
+      sm.q[r][d] = ldg_<T>(Q + row * D + d);
+      sm.go[r][d] = ldg_<TO>(GO + row * D + d);
+    }
+    __syncthreads();
+    // ---- far logits and the running max / sum per query -------------------
+    float mrun[kQC / kBW], lrun[kQC / kBW];
+#pragma unroll
+    for (int u = 0; u < kQC / kBW; ++u) {
+      mrun[u] = -INFINITY;
+      lrun[u] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kQC / kBW; ++u) {
+      const int r = warp + kBW * u;
+      if (r >= qc) continue;
+      float mx = -INFINITY;
+      for (int jj = lane; jj < nf; jj += 32) {
+        const int j = fl[jj];
+        float x = 0.f;
+#pragma unroll 8
+        for (int d = 0; d < D; ++d) x = fmaf(sm.q[r][d], mu_s[j * (D + 1) + d], x);
+        const float l = fmaf(s, x, __logf((float)kcnt[j]));
+        lf[r * Ck + jj] = l;
+        mx = fmaxf(mx, l);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float sum = 0.f;
+      for (int jj = lane; jj < nf; jj += 32) sum += __expf(lf[r * Ck + jj] - mx);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      mrun[u] = mx;
+      lrun[u] = nf > 0 ? sum : 0.f;
+    }
+    // ---- exact terms: finish the running max / sum, and their sum of p g --
+    float arun[kQC / kBW];
+#pragma unroll
+    for (int u = 0; u < kQC / kBW; ++u) arun[u] = 0.f;
+    for (int xi = 0; xi < nx; ++xi) {
+      const int j = xl[xi], nj = kcnt[j], o0 = koff[j];
+      for (int t0 = 0; t0 < nj; t0 += kKC) {
+        const int kc = imin(kKC, nj - t0);
+        __syncthreads();
+        for (int e = tid; e < kc * D; e += kBT) {
+          const int r = e / D, d = e - r * D;
+          const long long row = pk.row0 + kperm[o0 + t0 + r];
+          sm.kt[r][d] = ldg_<T>(K + row * D + d);
+          sm.vt[r][d] = ldg_<T>(V + row * D + d);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kQC / kBW; ++u) {
+          const int r = warp + kBW * u;
+          if (r >= qc) continue;
+          float l = -INFINITY, g = 0.f;
+          if (lane < kc) {
+            float x = 0.f;
+#pragma unroll 8
+            for (int d = 0; d < D; ++d) {
+              x = fmaf(sm.q[r][d], sm.kt[lane][d], x);
+              g = fmaf(sm.go[r][d], sm.vt[lane][d], g);
+            }
+            l = s * x;
+          }
+          float mx = l;
+#pragma unroll
+          for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float mn = fmaxf(mrun[u], mx);
+          float p = lane < kc ? __expf(l - mn) : 0.f;
+          float pg = p * g;
+#pragma unroll
+          for (int o = 16; o; o >>= 1) {
+            p += __shfl_xor_sync(0xffffffffu, p, o);
+            pg += __shfl_xor_sync(0xffffffffu, pg, o);
+          }
+          const float sc = __expf(mrun[u] - mn);
+          lrun[u] = lrun[u] * sc + p;
+          arun[u] = arun[u] * sc + pg;
+          mrun[u] = mn;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kQC / kBW; ++u) {
+      const int r = warp + kBW * u;
+      if (r < qc && lane == 0) {
+        sm.lse[r] = mrun[u] + __logf(lrun[u]);
+        sm.mq[r] = mrun[u];
+        sm.dex[r] = arun[u];
+      }
+    }
+    // ---- far terms' g = dO_q . u_ij: one warp per far cluster -------------
+    for (int jj = warp; jj < nf; jj += kBW) {
+      const int j = fl[jj];
+      float ux[DL];
+      const float invn = 1.f / (float)kcnt[j];
+#pragma unroll
+      for (int u = 0; u < DL; ++u) {
+        const int d = lane + 32 * u;
+        ux[u] = DIP ? b.U[(((size_t)qpid * Cq + i) * Ck + j) * D + d]
+                    : b.Sst[((size_t)kpid * Ck + j) * D + d] * invn;
+      }
+      for (int r = 0; r < qc; ++r) {
+        float g = 0.f;
+#pragma unroll
+        for (int u = 0; u < DL; ++u) g = fmaf(sm.go[r][lane + 32 * u], ux[u], g);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) g += __shfl_xor_sync(0xffffffffu, g, o);
+        if (lane == 0) gf[r * Ck + jj] = g;
+      }
+    }
+    __syncthreads();
+    // D_q = sum over the terms of p g
+#pragma unroll
+    for (int u = 0; u < kQC / kBW; ++u) {
+      const int r = warp + kBW * u;
+      if (r >= qc) continue;
+      const float m = sm.mq[r];
+      float a = 0.f;
+      for (int jj = lane; jj < nf; jj += 32) a = fmaf(__expf(lf[r * Ck + jj] - m), gf[r * Ck + jj], a);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0) sm.dq_[r] = (a + sm.dex[r]) * __expf(m - sm.lse[r]);
+    }
+    __syncthreads();
+
+    // ---- far terms: one warp per far cluster ------------------------------
+    for (int jj = warp; jj < nf; jj += kBW) {
+      const int j = fl[jj];
+      float gu[DL], gm[DL];
+#pragma unroll
+      for (int u = 0; u < DL; ++u) gu[u] = gm[u] = 0.f;
+      for (int r = 0; r < qc; ++r) {
+        const float p = __expf(lf[r * Ck + jj] - sm.lse[r]);
+        const float dl = p * (gf[r * Ck + jj] - sm.dq_[r]);
+#pragma unroll
+        for (int u = 0; u < DL; ++u) {
+          gu[u] = fmaf(p, sm.go[r][lane + 32 * u], gu[u]);
+          gm[u] = fmaf(s * dl, sm.q[r][lane + 32 * u], gm[u]);
+        }
+        __syncwarp();
+        if (lane == 0) lf[r * Ck + jj] = s * dl;  // now the coefficient of mu_j in dq
+      }
+      float* du = b.dU + (((size_t)qpid * Cq + i) * Ck + j) * D;
+      float* dm = b.dmu + ((size_t)kpid * Ck + j) * D;
+#pragma unroll
+      for (int u = 0; u < DL; ++u) {
+        const int d = lane + 32 * u;
+        du[d] += gu[u];  // this CTA owns the row (query set, i, j)
+        atomicAdd(dm + d, gm[u]);
+      }
+    }
+    __syncthreads();
+    // dq = sum_j (s dl_qj) mu_j
+    float dq[kQC / kBW][DL];
+#pragma unroll
+    for (int u = 0; u < kQC / kBW; ++u) {
+      const int r = warp + kBW * u;
+#pragma unroll
+      for (int v = 0; v < DL; ++v) dq[u][v] = 0.f;
+      if (r >= qc) continue;
+      for (int jj = 0; jj < nf; ++jj) {
+        const float c = lf[r * Ck + jj];
+        const float* m = mu_s + fl[jj] * (D + 1);
+#pragma unroll
+        for (int v = 0; v < DL; ++v) dq[u][v] = fmaf(c, m[lane + 32 * v], dq[u][v]);
+      }
+    }
+    // ---- exact tiles ------------------------------------------------------
+    float* dK = b.dK;
+    float* dV = b.dV;
+    for (int xi = 0; xi < nx; ++xi) {
+      const int j = xl[xi], nj = kcnt[j], o0 = koff[j];
+      for (int t0 = 0; t0 < nj; t0 += kKC) {
+        const int kc = imin(kKC, nj - t0);
+        __syncthreads();
+        for (int e = tid; e < kc * D; e += kBT) {
+          const int r = e / D, d = e - r * D;
+          const long long row = pk.row0 + kperm[o0 + t0 + r];
+          sm.kt[r][d] = ldg_<T>(K + row * D + d);
+          sm.vt[r][d] = ldg_<T>(V + row * D + d);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kQC / kBW; ++u) {
+          const int r = warp + kBW * u;
+          if (r >= qc) continue;
+          float p = 0.f, ds = 0.f;
+          if (lane < kc) {
+            float x = 0.f, g = 0.f;
+#pragma unroll 8
+            for (int d = 0; d < D; ++d) {
+              x = fmaf(sm.q[r][d], sm.kt[lane][d], x);
+              g = fmaf(sm.go[r][d], sm.vt[lane][d], g);
+            }
+            p = __expf(s * x - sm.lse[r]);
+            ds = p * (g - sm.dq_[r]);
+          }
+          sm.pt[r][lane] = p;
+          sm.dst[r][lane] = ds;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kQC / kBW; ++u) {
+          const int r = warp + kBW * u;
+          if (r >= qc) continue;
+          for (int t = 0; t < kc; ++t) {
+            const float c = s * sm.dst[r][t];
+#pragma unroll
+            for (int v = 0; v < DL; ++v) dq[u][v] = fmaf(c, sm.kt[t][lane + 32 * v], dq[u][v]);
+          }
+        }
+        for (int t = warp; t < kc; t += kBW) {
+          const long long row = pk.row0 + kperm[o0 + t0 + t];
+#pragma unroll
+          for (int v = 0; v < DL; ++v) {
+            const int d = lane + 32 * v;
+            float gk = 0.f, gv = 0.f;
+            for (int r = 0; r < qc; ++r) {
+              gk = fmaf(sm.dst[r][t], sm.q[r][d], gk);
+              gv = fmaf(sm.pt[r][t], sm.go[r][d], gv);
+            }
+            atomicAdd(dK + row * D + d, s * gk);
+            atomicAdd(dV + row * D + d, gv);
+          }
+        }
+      }
+    }
+    // ---- this chunk's dq (the centroid term is added later) ---------------
+#pragma unroll
+    for (int u = 0; u < kQC / kBW; ++u) {
+      const int r = warp + kBW * u;
+      if (r >= qc) continue;
+#pragma unroll
+      for (int v = 0; v < DL; ++v) b.dQ[(long long)sm.row[r] * D + lane + 32 * v] = dq[u][v];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// per (key set, cluster): the summaries' gradients and the chain to k and v
+// ---------------------------------------------------------------------------
+template <typename T, int D, bool DIP>
+__global__ void __launch_bounds__(kBT) bwd_cluster_kernel(AttnArgs a, BwdArgs b) {
+  extern __shared__ __align__(16) float bc_raw[];
+  float* M = bc_raw;                 // [D][D + 1]   M_j (DIPOLE)
+  float* dM = M + D * (D + 1);       // [D][D + 1]   dM_j (DIPOLE)
+  float* rows = dM + D * (D + 1);    // [32][D]      du rows, then k - mu rows
+  float* nus = rows + 32 * D;        // [32][D]      nu rows, then v rows
+  float* dS = nus + 32 * D;          // [D]
+  float* dmt = dS + D;               // [D]          dmu_j total / n_j
+  float* Sj = dmt + D;               // [D]
+  float* mu = Sj + D;                // [D]
+  const int kpid = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int Cq = a.Cq, Ck = a.Ck;
+  const Prob pk = prob_of(a.kg, kpid);
+  if (j >= pk.C) return;
+  const size_t cj = (size_t)kpid * Ck + j;
+  const int n = a.ks.counts[cj];
+  if (n == 0) return;
+  const float s = a.scale, invn = 1.f / (float)n;
+  for (int d = tid; d < D; d += kBT) {
+    Sj[d] = b.Sst[cj * D + d];
+    mu[d] = a.ks.cent32[cj * D + d];
+  }
+  if (DIP)
+    for (int e = tid; e < D * D; e += kBT) M[(e / D) * (D + 1) + e % D] = b.Mst[cj * D * D + e];
+  // query sets reading key set kpid: the G q-heads of its kv-head
+  const int ppb = a.kg.lv.pairs_per_bh;
+  const int bhk = kpid / ppb, pi = kpid - bhk * ppb;
+  const int Hq = a.qg.BH / a.B, Hkv = a.kg.BH / a.B;
+  const int bb = bhk / Hkv, hk = bhk - bb * Hkv;
+  constexpr int MR = DIP ? D * D / kBT : 1;
+  float dm[MR];
+#pragma unroll
+  for (int r = 0; r < MR; ++r) dm[r] = 0.f;
+  float dsacc = 0.f;
+  for (int g = 0; g < a.G; ++g) {
+    const int qpid = (bb * Hq + hk * a.G + g) * a.qg.lv.pairs_per_bh + pi;
+    const Prob pq = prob_of(a.qg, qpid);
+    for (int i0 = 0; i0 < pq.C; i0 += 32) {
+      const int ic = imin(32, pq.C - i0);
+      __syncthreads();
+      for (int e = tid; e < ic * D; e += kBT) {
+        const int r = e / D, d = e - r * D;
+        rows[r * D + d] = b.dU[(((size_t)qpid * Cq + i0 + r) * Ck + j) * D + d];
+        if (DIP) nus[r * D + d] = a.qs.cent32[((size_t)qpid * Cq + i0 + r) * D + d];
+      }
+      __syncthreads();
+      if (tid < D)
+        for (int r = 0; r < ic; ++r) dsacc += rows[r * D + tid];
+      if (DIP) {
+#pragma unroll
+        for (int r = 0; r < MR; ++r) {
+          const int idx = tid + kBT * r, e = idx / D, d = idx - e * D;
+          float x = dm[r];
+          for (int q = 0; q < ic; ++q) x = fmaf(rows[q * D + e], nus[q * D + d], x);
+          dm[r] = x;
+        }
+        // dnu_i += (s / n) M^T du_ij
+        for (int e = tid; e < ic * D; e += kBT) {
+          const int r = e / D, d = e - r * D;
+          float x = 0.f;
+#pragma unroll 8
+          for (int f = 0; f < D; ++f) x = fmaf(M[f * (D + 1) + d], rows[r * D + f], x);
+          atomicAdd(b.dnu + ((size_t)qpid * Cq + i0 + r) * D + d, s * invn * x);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < D) dS[tid] = dsacc * invn;
+  if (DIP) {
+#pragma unroll
+    for (int r = 0; r < MR; ++r) {
+      const int idx = tid + kBT * r, e = idx / D, d = idx - e * D;
+      dM[e * (D + 1) + d] = s * invn * dm[r];
+    }
+  }
+  __syncthreads();
+  // dmu_j total: the logits' part minus dM_j^T S_j, divided by n_j
+  for (int d = tid; d < D; d += kBT) {
+    float x = b.dmu[cj * D + d];
+    if (DIP)
+      for (int e = 0; e < D; ++e) x = fmaf(-dM[e * (D + 1) + d], Sj[e], x);
+    dmt[d] = x * invn;
+  }
+  __syncthreads();
+  // members: dv_t += dS + dM (k_t - mu), dk_t += dmu / n + dM^T v_t
+  const int off = a.ks.off[(size_t)kpid * (Ck + 1) + j];
+  const int* perm = a.ks.perm + pk.slot0;
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  constexpr int DL = D / 32;
+  for (int c0 = 0; c0 < n; c0 += 32) {
+    const int cnt = imin(32, n - c0);
+    __syncthreads();
+    for (int e = tid; e < cnt * D; e += kBT) {
+      const int r = e / D, d = e - r * D;
+      const long long row = pk.row0 + perm[off + c0 + r];
+      rows[r * D + d] = ldg_<T>(K + row * D + d) - mu[d];
+      nus[r * D + d] = ldg_<T>(V + row * D + d);
+    }
+    __syncthreads();
+    for (int r = warp; r < cnt; r += kBW) {
+      const long long row = pk.row0 + perm[off + c0 + r];
+#pragma unroll
+      for (int u = 0; u < DL; ++u) {
+        const int e = lane + 32 * u;
+        float gv = dS[e], gk = dmt[e];
+        if (DIP)
+          for (int f = 0; f < D; ++f) {
+            gv = fmaf(dM[e * (D + 1) + f], rows[r * D + f], gv);
+            gk = fmaf(dM[f * (D + 1) + e], nus[r * D + f], gk);
+          }
+        b.dV[row * D + e] += gv;  // the member's only writer in this launch
+        b.dK[row * D + e] += gk;
+      }
+    }
+  }
+}
+
+// dq += dnu_i / m_i for the members of every query cluster (DIPOLE)
+template <int D>
+__global__ void __launch_bounds__(kBT) bwd_query_nu_kernel(AttnArgs a, BwdArgs b) {
+  const int qpid = blockIdx.x, i = blockIdx.y, tid = threadIdx.x;
+  const int Cq = a.Cq;
+  const Prob pq = prob_of(a.qg, qpid);
+  if (i >= pq.C) return;
+  const int m = a.qs.counts[(size_t)qpid * Cq + i];
+  if (m == 0) return;
+  const int off = a.qs.off[(size_t)qpid * (Cq + 1) + i];
+  const int* perm = a.qs.perm + pq.slot0;
+  const float* dn = b.dnu + ((size_t)qpid * Cq + i) * D;
+  const float inv = 1.f / (float)m;
+  for (int e = tid; e < m * D; e += kBT) {
+    const int r = e / D, d = e - r * D;
+    const long long row = pq.row0 + perm[off + r];
+    b.dQ[row * D + d] += dn[d] * inv;
+  }
+}
+
+template <typename T, int D, bool DIP>
+size_t query_smem(int Ck) {
+  return sizeof(QuerySmem<D>) + (size_t)Ck * (D + 1) * 4 + (size_t)2 * kQC * Ck * 4 + (size_t)2 * Ck * 4;
+}
+
+template <typename T, typename TO, int D, bool DIP>
+void launch_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st) {
+  const int nk = a.ks.nprob, nq = a.qs.nprob;
+  {
+    ProfScope ps(st, "bwd_key_stats");
+    bwd_key_stats_kernel<T, D, DIP><<<dim3(nk, a.Ck), kBT, 0, st>>>(a, b);
+  }
+  if (DIP) {
+    ProfScope ps(st, "bwd_u_table");
+    const size_t sm = (size_t)(D * (D + 1) + kBT) * 4;
+    cudaFuncSetAttribute(bwd_u_table_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    bwd_u_table_kernel<D><<<dim3(nq, a.Ck), kBT, sm, st>>>(a, b);
+  }
+  {
+    ProfScope ps(st, "bwd_query");
+    const size_t sm = query_smem<T, D, DIP>(a.Ck);
+    cudaFuncSetAttribute(bwd_query_kernel<T, TO, D, DIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)sm);
+    bwd_query_kernel<T, TO, D, DIP><<<dim3(nq, a.Cq), kBT, sm, st>>>(a, s1, b);
+  }
+  {
+    ProfScope ps(st, "bwd_cluster");
+    const size_t sm = (size_t)(2 * D * (D + 1) + 64 * D + 4 * D) * 4;
+    cudaFuncSetAttribute(bwd_cluster_kernel<T, D, DIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)sm);
+    bwd_cluster_kernel<T, D, DIP><<<dim3(nk, a.Ck), kBT, sm, st>>>(a, b);
+  }
+  if (DIP) {
+    ProfScope ps(st, "bwd_query_nu");
+    bwd_query_nu_kernel<D><<<dim3(nq, a.Cq), kBT, 0, st>>>(a, b);
+  }
+}
+
+template <typename T, typename TO>
+void dispatch_d(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st) {
+  const bool dip = a.mode == 1;
+  if (a.qg.D == 64) {
+    if (dip) launch_bwd<T, TO, 64, true>(a, s1, b, st);
+    else launch_bwd<T, TO, 64, false>(a, s1, b, st);
+  } else {
+    if (dip) launch_bwd<T, TO, 128, true>(a, s1, b, st);
+    else launch_bwd<T, TO, 128, false>(a, s1, b, st);
+  }
+}
+
+}  // namespace
+
+bool backward_supported(int D, int Ck, int mode) {
+  return (mode == 0 || mode == 1) && (D == 64 || D == 128) && Ck * D <= 16384;
+}
+
+void run_attn_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  if (a.qg.dtype == 0) {
+    if (b.o_f32) dispatch_d<bf, float>(a, s1, b, st);
+    else dispatch_d<bf, bf>(a, s1, b, st);
+  } else {
+    dispatch_d<float, float>(a, s1, b, st);
+  }
+}
+
+}  // namespace muse

@@ -127,6 +127,23 @@ int dense_levels(const Levels& lv, int D, int Cq, int Ck);
 // the shape is outside the per-key-token kernel's limits.
 int fine_query_dense_levels(const Levels& lv, int D, int Cq, int Ck);
 
+// Backward pass of the acausal operator (backward.cu).
+struct BwdArgs {
+  const void* dO;  // gradient of the output [B,Hq,N,D]
+  int o_f32;       // dO is fp32 (else the input dtype)
+  float* dQ;       // [B,Hq,N,D]
+  float* dK;       // [B,Hkv,N,D], zeroed by the caller
+  float* dV;       // [B,Hkv,N,D], zeroed by the caller
+  float* Sst;      // [key sets][Ck][D]    S_j
+  float* Mst;      // [key sets][Ck][D][D] M_j (DIPOLE)
+  float* U;        // [query sets][Cq][Ck][D] u_ij (DIPOLE)
+  float* dU;       // [query sets][Cq][Ck][D], zeroed by the caller
+  float* dmu;      // [key sets][Ck][D], zeroed by the caller
+  float* dnu;      // [query sets][Cq][D], zeroed by the caller
+};
+bool backward_supported(int D, int Ck, int mode);
+void run_attn_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st);
+
 // Causal: exact local block + merge of the level partials into O.
 void run_local_merge(const AttnArgs& a, int L, cudaStream_t st);
 // The same on mma.sync tiles (bf16, L a multiple of 128); false if not covered.

@@ -234,6 +234,32 @@ muse_status muse_attn_fwd_causal(const void *Q, const void *K, const void *V,
                                  void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Gradients of the acausal operator: dQ, dK, dV of <dO, O> for the O of a
+ * muse_attn_fwd call ([G] Experimental Results: the layer is trained
+ * through).  The clusterings and the retrieval sets are held at the forward
+ * call's values (they are piecewise constant in the inputs); centroids, S_j,
+ * M_j and the query centroids are differentiated through the member means and
+ * sums they are.  Call order: size the workspace with
+ * muse_attn_bwd_workspace_size(), pass that workspace to muse_attn_fwd (with
+ * the same Q, K, V, shape and params), then to this function, unchanged in
+ * between: the backward reads the forward's clusterings and selections from
+ * it, and uses the space after the forward's part as scratch.  dO is
+ * [B,Hq,N,D] in the output dtype (fp32 if shape->out_f32); dQ [B,Hq,N,D],
+ * dK and dV [B,Hkv,N,D] are fp32, overwritten.  fp32 arithmetic; O itself is
+ * not read: sum_t p_t dO.x_t (= dO.O) is formed from the backward's own
+ * terms.  dK, dV and dQ are sums of fp32 atomic adds, so their last bits may
+ * differ from call to call.
+ * Supported: modes MONOPOLE and DIPOLE, Ck * D <= 16384; other modes and
+ * sizes return MUSE_ERR_UNSUPPORTED.  A workspace smaller than
+ * muse_attn_bwd_workspace_size() returns MUSE_ERR_WORKSPACE.
+ */
+size_t muse_attn_bwd_workspace_size(const muse_shape *shape, const muse_params *params);
+muse_status muse_attn_bwd(const void *Q, const void *K, const void *V, const void *dO,
+                          float *dQ, float *dK, float *dV, const muse_shape *shape,
+                          const muse_params *params, void *ws, size_t ws_bytes,
+                          cudaStream_t stream);
+
+/*
  * muse_cluster without a workspace argument, for callers that cannot
  * allocate device memory (no counterpart on the pages: this is a packaging
  * choice of this library).  The scratch comes from a fixed array compiled

@@ -122,3 +122,27 @@ def test_misaligned_pointers_are_rejected_without_launch(lib):
     assert st == 1 and b"aligned" in lib.muse_last_error()
     st = lib.muse_device_status(None, None)
     assert st == 1
+
+
+def test_backward_workspace_and_argument_checks(lib):
+    """The backward entry point sizes its workspace past the forward's part and
+    refuses unsupported modes and sizes, bad pointers and small workspaces
+    before launching anything."""
+    sh, pr = shape(), params()
+    fwd = lib.muse_workspace_size(ctypes.byref(sh), ctypes.byref(pr), 0)
+    bwd = lib.muse_attn_bwd_workspace_size(ctypes.byref(sh), ctypes.byref(pr))
+    assert bwd > fwd > 0
+    mono = lib.muse_attn_bwd_workspace_size(ctypes.byref(sh), ctypes.byref(params(mode=0)))
+    assert fwd < mono < bwd  # no M_j or u_ij tables for MONOPOLE
+    for bad in (params(mode=2), params(mode=3), params(Ck=512)):  # TILTED, DIPOLE_Q, Ck D > 16384
+        assert lib.muse_attn_bwd_workspace_size(ctypes.byref(sh), ctypes.byref(bad)) == 0
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+    args = [fake] * 7
+    st = lib.muse_attn_bwd(*([None] + args[1:]), ctypes.byref(sh), ctypes.byref(pr), fake,
+                           1 << 40, None)
+    assert st == 1 and b"NULL" in lib.muse_last_error()
+    st = lib.muse_attn_bwd(*args, ctypes.byref(sh), ctypes.byref(params(mode=2)), fake, 1 << 40,
+                           None)
+    assert st == 2
+    st = lib.muse_attn_bwd(*args, ctypes.byref(sh), ctypes.byref(pr), fake, fwd, None)
+    assert st == 3 and b"backward" in lib.muse_last_error()
