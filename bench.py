@@ -54,6 +54,8 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
     p.add_argument("--mode", default=None, choices=[None, "dipole", "monopole", "tilted", "dipole_q"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--backward", action="store_true",
+                   help="time only the backward pass of an acausal workload (one JSON line)")
     p.add_argument("--no-side", action="store_true",
                    help="skip the other N >= 8k configurations of the default run")
     return p.parse_args()
@@ -425,6 +427,90 @@ def run_muse(w, mode, steps, warmup, rank, world, device, e2e_leg=True):
 
 
 # ---------------------------------------------------------------------------
+# the backward pass (acausal): gradients of <dO, O> through the C ABI
+# ---------------------------------------------------------------------------
+BWD_KERNELS = ("bwd_key_stats", "bwd_u_table", "bwd_query", "bwd_cluster", "bwd_query_nu")
+
+
+def backward_work(w, mode, dbg):
+    """Algorithmic FLOPs of one backward call per kernel (multiply-add = 2):
+      bwd_key_stats  S_j: D per key; M_j (DIPOLE): 2 D^2 per key, per kv-head;
+      bwd_u_table    (DIPOLE) 2 C_k D^2 per query cluster, per q-head;
+      bwd_query      10 D per far row (logit, dO.u, dq, dmu, du) and per exact
+                     key (logit, dO.v, dq, dk, dv);
+      bwd_cluster    (DIPOLE) dM and dnu: 4 C_q D^2 per key cluster, per
+                     q-head; the members' chain: 4 D^2 per key, per kv-head;
+                     (MONOPOLE: 2 D per key)."""
+    far, exact = retrieval_rows(w, mode, dbg)
+    B, Hq, Hkv, D, N, C = w.B, w.Hq, w.Hkv, w.D, w.N, w.C
+    dip = mode == "dipole"
+    work = dict.fromkeys(BWD_KERNELS, 0.0)
+    work["bwd_key_stats"] = B * Hkv * N * (D + (2.0 * D * D if dip else 0.0))
+    if dip:
+        work["bwd_u_table"] = B * Hq * C * 2.0 * C * D * D
+        work["bwd_cluster"] = B * Hq * C * 4.0 * C * D * D + B * Hkv * N * 4.0 * D * D
+        work["bwd_query_nu"] = B * Hq * N * D
+    else:
+        work["bwd_cluster"] = B * Hkv * N * 2.0 * D
+    work["bwd_query"] = 10.0 * D * (sum(far) + sum(exact))
+    return work
+
+
+def run_backward(w, mode, steps, warmup, device):
+    """Times `steps` backward calls on workload `w` after one forward call that
+    fills the shared workspace (inputs and dO resident, L2 flushed between
+    calls); returns ms per call, per-kernel times and the algorithmic rate."""
+    import clustered_multipole_approximation_b200 as muse
+
+    Q, K, V = make_inputs(w)
+    cast = (lambda x: torch.from_numpy(x).to(torch.bfloat16)) if w.dtype == "bf16" else torch.from_numpy
+    q, k, v = cast(Q).to(device), cast(K).to(device), cast(V).to(device)
+    del Q, K, V
+    kw = dict(Cq=w.C, Ck=w.C, iters=w.iters, seed=w.cluster_seed, topk=w.topk, scale=w.scale,
+              mode=mode)
+    p = muse.make_params(w.C, w.C, w.iters, w.cluster_seed, w.topk, 0, w.scale, mode)
+    ws = torch.empty(muse.backward_workspace_size(q, k, p), dtype=torch.uint8, device=device)
+    o, dbg = muse.muse_attn_fwd(q, k, v, workspace=ws, debug=True, **kw)
+    dbg = {n: t.cpu().numpy() for n, t in dbg.items()}
+    do = torch.randn(o.shape, generator=torch.Generator(device=device).manual_seed(7),
+                     device=device).to(o.dtype)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        muse.muse_attn_bwd(q, k, v, do, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    muse.profile_read()
+    muse.profile_enable(True)
+    total = 0.0
+    for _ in range(steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        muse.muse_attn_bwd(q, k, v, do, workspace=ws, **kw)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1)
+    muse.profile_enable(False)
+    prof = muse.profile_read()
+    work = backward_work(w, mode, dbg)
+    ms = total / steps
+    kernels = {}
+    for n, (c, t) in sorted(prof.items(), key=lambda kv: -kv[1][1]):
+        e = {"launches": c, "ms_per_call": round(t / steps, 4)}
+        if work.get(n):
+            e["tflops"] = round(work[n] / (t / steps / 1e3) / 1e12, 3)
+        kernels[n] = e
+    del q, k, v, o, do, ws, flush
+    torch.cuda.empty_cache()
+    return {"config": config_of(w, mode), "ms_per_call": ms, "steps": steps, "warmup": warmup,
+            "algorithmic_gflop": sum(work.values()) / 1e9,
+            "achieved_tflops": sum(work.values()) / (ms / 1e3) / 1e12,
+            "arithmetic": "fp32 CUDA cores", "kernels": kernels}
+
+
+# ---------------------------------------------------------------------------
 # the oracle on the host cores (CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
 def oracle_sample(w, mode, heads):
@@ -509,6 +595,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     mode = args.mode or w.mode
+    if args.backward:
+        if rank == 0:
+            print(json.dumps(run_backward(w, mode, args.steps, args.warmup, device)), flush=True)
+        return
     r = run_muse(w, mode, args.steps, args.warmup, rank, world, device)
     line = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
@@ -529,6 +619,9 @@ def main():
             rr = run_muse(sw, sm, st, wu, rank, world, device, e2e_leg=False)
             side[f"{name}/{sm}"] = side_entry(rr, sw, st, wu)
         line["workloads"] = side
+    if world == 1 and not args.no_side and args.workload == DEFAULT_WORKLOAD and args.mode is None:
+        line["backward"] = {m: run_backward(w, m, args.steps, args.warmup, device)
+                            for m in ("dipole", "monopole")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads = min(w.B * w.Hq, 8)
         dt, tps, thr = oracle_sample(w, r["mode"], heads)
