@@ -54,11 +54,18 @@ class muse_debug(ctypes.Structure):
                 ("n_exact", ctypes.c_void_p), ("device_error", ctypes.c_void_p)]
 
 
+class muse_accum_debug(ctypes.Structure):
+    _fields_ = [("q_assign", ctypes.c_void_p), ("k_assign", ctypes.c_void_p),
+                ("sel1", ctypes.c_void_p), ("sel2", ctypes.c_void_p),
+                ("n_exact", ctypes.c_void_p), ("device_error", ctypes.c_void_p)]
+
+
 EXPORTS = ["muse_workspace_size", "muse_cluster_workspace_size", "muse_cluster", "muse_summarize",
            "muse_attn_fwd", "muse_attn_fwd_causal", "muse_status_string", "muse_last_error",
            "muse_profile_enable", "muse_profile_read", "muse_cluster_static",
            "muse_cluster_static_capacity", "muse_device_status", "muse_debug_inject_barrier_fault",
-           "muse_attn_bwd_workspace_size", "muse_attn_bwd"]
+           "muse_attn_bwd_workspace_size", "muse_attn_bwd", "muse_accum_workspace_size",
+           "muse_attn_fwd_causal_accum"]
 
 # Bits of the device error word (include/muse.h MUSE_DEVERR_*).
 DEVERR = {1: "MUSE_DEVERR_MMA_WAIT", 2: "MUSE_DEVERR_TEAM_BARRIER", 4: "MUSE_DEVERR_V_RANGE"}
@@ -91,6 +98,11 @@ def load_library(path: str = LIB_PATH):
     for f in ("muse_attn_fwd", "muse_attn_fwd_causal"):
         getattr(lib, f).restype = i32
         getattr(lib, f).argtypes = [vp, vp, vp, vp, sp, pp, dp, vp, sz, vp]
+    lib.muse_accum_workspace_size.restype = sz
+    lib.muse_accum_workspace_size.argtypes = [sp, pp, i32]
+    lib.muse_attn_fwd_causal_accum.restype = i32
+    lib.muse_attn_fwd_causal_accum.argtypes = [vp, vp, vp, vp, sp, pp, i32,
+                                               ctypes.POINTER(muse_accum_debug), vp, sz, vp]
     lib.muse_attn_bwd_workspace_size.restype = sz
     lib.muse_attn_bwd_workspace_size.argtypes = [sp, pp]
     lib.muse_attn_bwd.restype = i32
@@ -241,6 +253,59 @@ def muse_attn_fwd_causal(q, k, v, *, C, block, iters, seed, topk, scale=1.0, mod
     per level and role)."""
     p = make_params(C, C, iters, seed, topk, block, scale, mode, key_stream0, query_stream0)
     return _attn(True, q, k, v, p, out, workspace, debug, stream, out_dtype)
+
+
+def accum_workspace_size(q, k, params: muse_params, topk2: int) -> int:
+    """Workspace bytes of muse_attn_fwd_causal_accum."""
+    lib = load_library()
+    sh = make_shape(q, k)
+    n = lib.muse_accum_workspace_size(ctypes.byref(sh), ctypes.byref(params), int(topk2))
+    if n == 0:
+        raise MuseError(3, lib.muse_last_error().decode())
+    return int(n)
+
+
+def muse_attn_fwd_causal_accum(q, k, v, *, Cq, Ck, block, iters, seed, topk, topk2, scale=1.0,
+                               mode="dipole", out=None, workspace=None, debug=False, stream=None,
+                               out_dtype=None):
+    """Causal MuSe with block-summary accumulation and cluster/block retrieval
+    (see muse_attn_fwd_causal_accum in include/muse.h).  Returns O and, with
+    debug, a dict of inspection tensors (q_assign, k_assign, sel1, sel2,
+    n_exact, device_error)."""
+    lib = load_library()
+    _need_cuda(q, k, v, out, workspace)
+    if k.shape != v.shape or q.dtype != k.dtype or k.dtype != v.dtype:
+        raise ValueError("k and v must match in shape; q, k, v must share a dtype")
+    if out is not None:
+        out_dtype = out.dtype
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out_dtype not in (q.dtype, torch.float32):
+        raise ValueError("the output dtype must be the input dtype or float32")
+    p = make_params(Cq, Ck, iters, seed, topk, block, scale, mode)
+    sh = make_shape(q, k, out_dtype == torch.float32 and q.dtype != torch.float32)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(accum_workspace_size(q, k, p, topk2), dtype=torch.uint8,
+                                device=q.device)
+    bufs = dbg = None
+    if debug:
+        B, Hq, N, D = q.shape
+        NB = N // block
+        i32 = dict(dtype=torch.int32, device=q.device)
+        bufs = dict(q_assign=torch.empty(B, Hq, N, **i32),
+                    k_assign=torch.empty(B, k.shape[1], N, **i32),
+                    sel1=torch.full((B, Hq, NB, Cq, topk), -1, **i32),
+                    sel2=torch.full((B, Hq, NB, Cq, topk, topk2), -1, **i32),
+                    n_exact=torch.empty(B, Hq, N, dtype=torch.int64, device=q.device),
+                    device_error=torch.full((1,), -1, **i32))
+        dbg = muse_accum_debug(*[bufs[n].data_ptr() for n, _ in muse_accum_debug._fields_])
+    st = lib.muse_attn_fwd_causal_accum(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(sh),
+                                        ctypes.byref(p), int(topk2),
+                                        ctypes.byref(dbg) if dbg is not None else None,
+                                        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(lib, st)
+    return (out, bufs) if debug else out
 
 
 def backward_workspace_size(q, k, params: muse_params, out_f32: bool = False) -> int:

@@ -1,0 +1,541 @@
+// Causal operator with causal accumulation of block summaries and two-level
+// retrieval (gist.science page "Multipole Semantic Attention: A Fast
+// Approximation of Softmax Attention for Pretraining", Technical Summary,
+// Core Mechanisms: "Causal Accumulation" and "Retrieval-Augmented
+// Approximation").
+//
+// Both roles are clustered over the whole sequence of a (b, head) (the
+// acausal clustering).  The sequence is cut into blocks of L tokens.  Per
+// (key cluster j, block b): n_jb, the key sum (fp64) and the value sum, and for
+// DIPOLE, per query cluster i, A_ijb = sum_{t in (j, b)} v_t (k_t . nu_i)
+// (so that M nu_i = A - S (mu . nu_i) over any union of blocks).  The
+// summaries a query block b reads are the exclusive prefix over blocks
+// 0 .. b-1, accumulated in block order.  Per (query cluster i, block b):
+//   1. top-k1 key clusters by s nu_i . mu_j^{<b} + log n_j^{<b} (fp64, the
+//      dot product in dimension order, ties to the lowest j);
+//   2. per selected j, top-k2 blocks b' < b by s nu_i . mu_jb' + log n_jb';
+//   3. one online softmax over the keys of the retrieved (j, b') pairs
+//      (exact) and, per key cluster, the summary of its prefix members outside
+//      the retrieved blocks (far: logit s q.mu + log n, value S / n or
+//      (S + s M nu_i) / n); the result enters the local block's softmax as one
+//      term (normalised output, log-sum-exp), merged by the causal local
+//      kernels.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace muse {
+
+namespace {
+
+constexpr int kAT = 256;
+constexpr int kAW = kAT / 32;
+
+// ---------------------------------------------------------------------------
+// per (set, cluster): members per block (counts, first member of each block)
+// and, for keys, the block key sums (fp64, token order) and value sums
+// ---------------------------------------------------------------------------
+template <typename T, int D, bool KEYS>
+__global__ void __launch_bounds__(kAT) acc_block_stats_kernel(AttnArgs a, AccArgs c) {
+  const int pid = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+  const RoleGeo& g = KEYS ? a.kg : a.qg;
+  const KState& ks = KEYS ? a.ks : a.qs;
+  const int C = KEYS ? a.Ck : a.Cq, NB = c.NB, L = c.L;
+  const Prob p = prob_of(g, pid);
+  const size_t cj = (size_t)pid * C + j;
+  const int n = ks.counts[cj];
+  const int off = ks.off[(size_t)pid * (C + 1) + j];
+  const int* perm = ks.perm + p.slot0 + off;
+  int* boff = (KEYS ? c.kboff : c.qboff) + cj * (NB + 1);
+  // first member of each block: members are in token order within a cluster
+  for (int b = tid; b <= NB; b += kAT) {
+    int lo = 0, hi = n;
+    const int t = b * L;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (perm[mid] < t) lo = mid + 1;
+      else hi = mid;
+    }
+    boff[b] = lo;
+  }
+  if (!KEYS) return;
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  for (int d = tid; d < D; d += kAT) {
+    double sk = 0.0;
+    float sv = 0.f;
+    int cur = n > 0 ? perm[0] / L : 0, cnt = 0;
+    for (int m = 0; m < n; ++m) {
+      const int t = perm[m], b = t / L;
+      if (b != cur) {
+        const size_t o = ((size_t)pid * NB + cur) * C + j;
+        c.bk[o * D + d] = sk;
+        c.bs[o * D + d] = sv;
+        if (d == 0) c.bn[o] = cnt;
+        sk = 0.0;
+        sv = 0.f;
+        cnt = 0;
+        cur = b;
+      }
+      const long long row = p.row0 + t;
+      sk += (double)ld<T>(K + row * D + d);
+      sv += ld<T>(V + row * D + d);
+      ++cnt;
+    }
+    if (n > 0) {
+      const size_t o = ((size_t)pid * NB + cur) * C + j;
+      c.bk[o * D + d] = sk;
+      c.bs[o * D + d] = sv;
+      if (d == 0) c.bn[o] = cnt;
+    }
+  }
+}
+
+// exclusive prefix over blocks, in block order: one thread per (set, j, d)
+template <int D>
+__global__ void acc_prefix_kernel(AttnArgs a, AccArgs c) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int Ck = a.Ck, NB = c.NB;
+  const long long total = (long long)a.ks.nprob * Ck * D;
+  if (e >= total) return;
+  const int d = (int)(e % D);
+  const long long pj = e / D;  // pid * Ck + j
+  const int pid = (int)(pj / Ck), j = (int)(pj - (long long)pid * Ck);
+  double pk = 0.0;
+  float ps = 0.f;
+  int pn = 0;
+  for (int b = 0; b < NB; ++b) {
+    const size_t o = ((size_t)pid * NB + b) * Ck + j;
+    c.pk[o * D + d] = pk;
+    c.ps[o * D + d] = ps;
+    if (d == 0) c.pn[o] = pn;
+    pk += c.bk[o * D + d];
+    ps += c.bs[o * D + d];
+    pn += c.bn[o];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// DIPOLE: A_ijb = sum_{t in (j, b)} v_t (k_t . nu_i) for every query cluster i
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kAT) acc_block_a_kernel(AttnArgs a, AccArgs c) {
+  extern __shared__ __align__(16) float aa_raw[];
+  const int Cq = a.Cq, Ck = a.Ck, NB = c.NB, L = c.L;
+  float* nu = aa_raw;                     // [Cq][D + 1]
+  float* kt = nu + Cq * (D + 1);          // [32][D + 1]
+  float* vt = kt + 32 * (D + 1);          // [32][D]
+  float* gt = vt + 32 * D;                // [32][Cq]
+  int* tb = reinterpret_cast<int*>(gt + 32 * Cq);  // [32] block of each member
+  const int qpid = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+  const int kpid = kv_problem(a, qpid);
+  const Prob pk = prob_of(a.kg, kpid);
+  const size_t cj = (size_t)kpid * Ck + j;
+  const int n = a.ks.counts[cj];
+  const int off = a.ks.off[(size_t)kpid * (Ck + 1) + j];
+  const int* perm = a.ks.perm + pk.slot0 + off;
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  for (int e = tid; e < Cq * D; e += kAT) {
+    const int i = e / D, d = e - i * D;
+    nu[i * (D + 1) + d] = a.qs.cent32[((size_t)qpid * Cq + i) * D + d];
+  }
+  constexpr int R = 32;  // outputs (i, e) per thread: Cq * D <= kAT * R
+  float acc[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc[r] = 0.f;
+  const int nout = Cq * D;
+  int cur = -1;
+  auto flush = [&](int b) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int o = tid + kAT * r;
+      if (o < nout) {
+        const int i = o / D, e = o - i * D;
+        c.ba[((((size_t)qpid * NB + b) * Cq + i) * Ck + j) * D + e] = acc[r];
+      }
+      acc[r] = 0.f;
+    }
+  };
+  for (int m0 = 0; m0 < n; m0 += 32) {
+    const int cnt = imin(32, n - m0);
+    __syncthreads();
+    for (int e = tid; e < cnt * D; e += kAT) {
+      const int r = e / D, d = e - r * D;
+      const long long row = pk.row0 + perm[m0 + r];
+      kt[r * (D + 1) + d] = ld<T>(K + row * D + d);
+      vt[r * D + d] = ld<T>(V + row * D + d);
+    }
+    if (tid < cnt) tb[tid] = perm[m0 + tid] / L;
+    __syncthreads();
+    for (int e = tid; e < cnt * Cq; e += kAT) {
+      const int r = e / Cq, i = e - r * Cq;
+      float x = 0.f;
+#pragma unroll 8
+      for (int d = 0; d < D; ++d) x = fmaf(kt[r * (D + 1) + d], nu[i * (D + 1) + d], x);
+      gt[r * Cq + i] = x;
+    }
+    __syncthreads();
+    for (int r = 0; r < cnt; ++r) {
+      const int b = tb[r];
+      if (b != cur) {
+        if (cur >= 0) flush(cur);
+        cur = b;
+      }
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        const int o = tid + kAT * q;
+        if (o < nout) {
+          const int i = o / D, e = o - i * D;
+          acc[q] = fmaf(vt[r * D + e], gt[r * Cq + i], acc[q]);
+        }
+      }
+    }
+  }
+  if (cur >= 0) flush(cur);
+}
+
+// exclusive prefix of A over blocks: one thread per (q-set, i, j, e)
+template <int D>
+__global__ void acc_prefix_a_kernel(AttnArgs a, AccArgs c) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int Cq = a.Cq, Ck = a.Ck, NB = c.NB;
+  const long long per = (long long)Cq * Ck * D;  // one block of one q-set
+  const long long total = (long long)a.qs.nprob * per;
+  if (e >= total) return;
+  const long long qp = e / per, r = e - qp * per;
+  float s = 0.f;
+  for (int b = 0; b < NB; ++b) {
+    const size_t o = (size_t)(qp * NB + b) * per + r;
+    const float x = c.ba[o];
+    c.pa[o] = s;
+    s += x;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// selection: per (q-set, block b), warps over the query clusters present in b
+// ---------------------------------------------------------------------------
+__device__ inline double dot_ordered(const double* x, const double* y, double div, int D) {
+  double s = 0.0;
+  for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(x[d], __ddiv_rn(y[d], div)));
+  return s;
+}
+
+__global__ void __launch_bounds__(kAT) acc_select_kernel(AttnArgs a, AccArgs c) {
+  extern __shared__ __align__(16) double sel_raw[];
+  const int Cq = a.Cq, Ck = a.Ck, NB = c.NB, k1 = a.topk, k2 = c.k2, D = a.qg.D;
+  const int qpid = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int smax = Ck > NB ? Ck : NB;
+  double* sc = sel_raw + (size_t)warp * smax;
+  double* nu = sel_raw + (size_t)kAW * smax + (size_t)warp * D;
+  const int kpid = kv_problem(a, qpid);
+  const double s = (double)a.scale;
+  for (int i = warp; i < Cq; i += kAW) {
+    int* s1 = c.sel1 + (((size_t)qpid * NB + b) * Cq + i) * k1;
+    int* s2 = c.sel2 + ((((size_t)qpid * NB + b) * Cq + i) * k1) * k2;
+    for (int r = lane; r < k1; r += 32) s1[r] = -1;
+    for (int r = lane; r < k1 * k2; r += 32) s2[r] = -1;
+    const int* qb = c.qboff + ((size_t)qpid * Cq + i) * (NB + 1);
+    if (b == 0 || qb[b + 1] == qb[b]) continue;  // no query of cluster i in block b
+    for (int d = lane; d < D; d += 32) nu[d] = a.qs.cent64[((size_t)qpid * Cq + i) * D + d];
+    __syncwarp();
+    // 1. key clusters by their prefix summaries
+    for (int j = lane; j < Ck; j += 32) {
+      const size_t o = ((size_t)kpid * NB + b) * Ck + j;
+      const int n = c.pn[o];
+      sc[j] = n > 0 ? __dadd_rn(__dmul_rn(s, dot_ordered(nu, c.pk + o * D, (double)n, D)),
+                                log((double)n))
+                    : -INFINITY;
+    }
+    __syncwarp();
+    for (int r = 0; r < k1; ++r) {
+      double bv = -INFINITY;
+      int bj = -1;
+      for (int j = lane; j < Ck; j += 32)
+        if (sc[j] > bv) {  // the lowest j wins ties within a lane (ascending j)
+          bv = sc[j];
+          bj = j;
+        }
+      for (int o = 16; o; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+        if (oj >= 0 && (bj < 0 || ov > bv || (ov == bv && oj < bj))) {
+          bv = ov;
+          bj = oj;
+        }
+      }
+      if (bj < 0) break;
+      if (lane == 0) {
+        s1[r] = bj;
+        sc[bj] = -INFINITY;
+      }
+      __syncwarp();
+    }
+    __syncwarp();
+    // 2. blocks within each selected cluster, by their block summaries
+    for (int r = 0; r < k1; ++r) {
+      const int j = s1[r];
+      if (j < 0) break;
+      __syncwarp();
+      for (int bb = lane; bb < b; bb += 32) {
+        const size_t o = ((size_t)kpid * NB + bb) * Ck + j;
+        const int n = c.bn[o];
+        sc[bb] = n > 0 ? __dadd_rn(__dmul_rn(s, dot_ordered(nu, c.bk + o * D, (double)n, D)),
+                                   log((double)n))
+                       : -INFINITY;
+      }
+      __syncwarp();
+      for (int r2 = 0; r2 < k2; ++r2) {
+        double bv = -INFINITY;
+        int bj = -1;
+        for (int bb = lane; bb < b; bb += 32)
+          if (sc[bb] > bv) {
+            bv = sc[bb];
+            bj = bb;
+          }
+        for (int o = 16; o; o >>= 1) {
+          const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+          if (oj >= 0 && (bj < 0 || ov > bv || (ov == bv && oj < bj))) {
+            bv = ov;
+            bj = oj;
+          }
+        }
+        if (bj < 0) break;
+        if (lane == 0) {
+          s2[r * k2 + r2] = bj;
+          sc[bj] = -INFINITY;
+        }
+        __syncwarp();
+      }
+      __syncwarp();
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// far summaries + retrieved keys: one CTA per (q-set, block b, query cluster i)
+// ---------------------------------------------------------------------------
+template <typename T, int D, bool DIP>
+__global__ void __launch_bounds__(kAT) acc_stage2_kernel(AttnArgs a, AccArgs c) {
+  extern __shared__ __align__(16) float s2_raw[];
+  const int Cq = a.Cq, Ck = a.Ck, NB = c.NB, k1 = a.topk, k2 = c.k2, L = c.L;
+  float* mu_s = s2_raw;                  // [Ck][D]
+  float* u_s = mu_s + (size_t)Ck * D;    // [Ck][D]
+  float* ln_s = u_s + (size_t)Ck * D;    // [Ck]   log n of the far set, -inf if empty
+  float* nu = ln_s + Ck;                 // [D]
+  int* rsel = reinterpret_cast<int*>(nu + D);  // [Ck] rank of j among the selected clusters, or -1
+  __shared__ int nretr;
+  const int qpid = blockIdx.x, b = blockIdx.y, i = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (b == 0) return;
+  const int* qb = c.qboff + ((size_t)qpid * Cq + i) * (NB + 1);
+  const int m0 = qb[b], m1 = qb[b + 1];
+  if (m1 == m0) return;
+  const Prob pq = prob_of(a.qg, qpid);
+  const int kpid = kv_problem(a, qpid);
+  const Prob pk = prob_of(a.kg, kpid);
+  const float s = a.scale;
+  const int* s1 = c.sel1 + (((size_t)qpid * NB + b) * Cq + i) * k1;
+  const int* s2 = c.sel2 + ((((size_t)qpid * NB + b) * Cq + i) * k1) * k2;
+  for (int d = tid; d < D; d += kAT) nu[d] = a.qs.cent32[((size_t)qpid * Cq + i) * D + d];
+  for (int j = tid; j < Ck; j += kAT) rsel[j] = -1;  // index into s1, -1 if not selected
+  __syncthreads();
+  if (tid < k1 && s1[tid] >= 0) rsel[s1[tid]] = tid;
+  __syncthreads();
+  // far table: prefix minus the retrieved blocks, one warp per key cluster
+  for (int j = warp; j < Ck; j += kAW) {
+    const size_t o = ((size_t)kpid * NB + b) * Ck + j;
+    int n = c.pn[o];
+    const int r = rsel[j];
+    double ksum[D / 32];
+    float ss[D / 32], aa[D / 32];
+#pragma unroll
+    for (int u = 0; u < D / 32; ++u) {
+      const int d = lane + 32 * u;
+      ksum[u] = c.pk[o * D + d];
+      ss[u] = c.ps[o * D + d];
+      aa[u] = DIP ? c.pa[((((size_t)qpid * NB + b) * Cq + i) * Ck + j) * D + d] : 0.f;
+    }
+    if (r >= 0) {
+      for (int r2 = 0; r2 < k2; ++r2) {
+        const int bb = s2[r * k2 + r2];
+        if (bb < 0) break;
+        const size_t ob = ((size_t)kpid * NB + bb) * Ck + j;
+        n -= c.bn[ob];
+#pragma unroll
+        for (int u = 0; u < D / 32; ++u) {
+          const int d = lane + 32 * u;
+          ksum[u] -= c.bk[ob * D + d];
+          ss[u] -= c.bs[ob * D + d];
+          if (DIP) aa[u] -= c.ba[((((size_t)qpid * NB + bb) * Cq + i) * Ck + j) * D + d];
+        }
+      }
+    }
+    if (n <= 0) {
+      if (lane == 0) ln_s[j] = -INFINITY;
+      continue;
+    }
+    const float inv = 1.f / (float)n;
+    float mn = 0.f;
+#pragma unroll
+    for (int u = 0; u < D / 32; ++u) {
+      const int d = lane + 32 * u;
+      const float mu = (float)(ksum[u] / (double)n);
+      mu_s[j * D + d] = mu;
+      mn = fmaf(mu, nu[d], mn);
+    }
+#pragma unroll
+    for (int o2 = 16; o2; o2 >>= 1) mn += __shfl_xor_sync(0xffffffffu, mn, o2);
+#pragma unroll
+    for (int u = 0; u < D / 32; ++u) {
+      const int d = lane + 32 * u;
+      // M nu = A - S (mu . nu) over the far set
+      u_s[j * D + d] = DIP ? fmaf(s, fmaf(-ss[u], mn, aa[u]), ss[u]) * inv : ss[u] * inv;
+    }
+    if (lane == 0) ln_s[j] = logf((float)n);
+  }
+  if (tid == 0) {
+    int cnt = 0;
+    for (int r = 0; r < k1; ++r) {
+      const int j = s1[r];
+      if (j < 0) break;
+      for (int r2 = 0; r2 < k2; ++r2) {
+        const int bb = s2[r * k2 + r2];
+        if (bb < 0) break;
+        cnt += c.bn[((size_t)kpid * NB + bb) * Ck + j];
+      }
+    }
+    nretr = cnt;
+  }
+  __syncthreads();
+  // one warp per query of cluster i in block b
+  const T* Q = static_cast<const T*>(a.qg.X);
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  const int* qperm = a.qs.perm + pq.slot0 + a.qs.off[(size_t)qpid * (Cq + 1) + i];
+  const int* kperm = a.ks.perm + pk.slot0;
+  const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
+  constexpr int DL = D / 32;
+  for (int m = m0 + warp; m < m1; m += kAW) {
+    const int tq = qperm[m];
+    const long long qrow = pq.row0 + tq;
+    float q[DL], o[DL];
+#pragma unroll
+    for (int u = 0; u < DL; ++u) {
+      q[u] = ld<T>(Q + qrow * D + lane + 32 * u);
+      o[u] = 0.f;
+    }
+    float mx = -INFINITY, l = 0.f;
+    auto add = [&](float lg, const float* x, bool global_t, long long vrow) {
+      const float mn = fmaxf(mx, lg);
+      const float sc = __expf(mx - mn), w = __expf(lg - mn);
+      l = l * sc + w;
+#pragma unroll
+      for (int u = 0; u < DL; ++u) {
+        const float xv = global_t ? ld<T>(V + vrow * D + lane + 32 * u) : x[lane + 32 * u];
+        o[u] = fmaf(o[u], sc, w * xv);
+      }
+      mx = mn;
+    };
+    for (int j = 0; j < Ck; ++j) {
+      const float lnj = ln_s[j];
+      if (lnj == -INFINITY) continue;
+      float x = 0.f;
+#pragma unroll
+      for (int u = 0; u < DL; ++u) x = fmaf(q[u], mu_s[j * D + lane + 32 * u], x);
+#pragma unroll
+      for (int o2 = 16; o2; o2 >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o2);
+      add(fmaf(s, x, lnj), u_s + (size_t)j * D, false, 0);
+    }
+    for (int r = 0; r < k1; ++r) {
+      const int j = s1[r];
+      if (j < 0) break;
+      const int* kb = c.kboff + ((size_t)kpid * Ck + j) * (NB + 1);
+      for (int r2 = 0; r2 < k2; ++r2) {
+        const int bb = s2[r * k2 + r2];
+        if (bb < 0) break;
+        for (int mm = kb[bb]; mm < kb[bb + 1]; ++mm) {
+          const long long krow = pk.row0 + kperm[koff[j] + mm];
+          float x = 0.f;
+#pragma unroll
+          for (int u = 0; u < DL; ++u) x = fmaf(q[u], ld<T>(K + krow * D + lane + 32 * u), x);
+#pragma unroll
+          for (int o2 = 16; o2; o2 >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o2);
+          add(s * x, nullptr, true, krow);
+        }
+      }
+    }
+    float* pp = a.part + (size_t)qrow * (D + 1);
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int u = 0; u < DL; ++u) pp[lane + 32 * u] = o[u] * inv;
+    if (lane == 0) {
+      pp[D] = mx + logf(l);
+      if (a.n_exact != nullptr) a.n_exact[qrow] = nretr;
+    }
+  }
+}
+
+template <typename T, int D>
+void launch_accum(const AttnArgs& a, const AccArgs& c, cudaStream_t st) {
+  const int nk = a.ks.nprob, nq = a.qs.nprob;
+  const bool dip = a.mode == 1;
+  {
+    ProfScope ps(st, "accum_block_stats");
+    acc_block_stats_kernel<T, D, true><<<dim3(nk, a.Ck), kAT, 0, st>>>(a, c);
+    acc_block_stats_kernel<T, D, false><<<dim3(nq, a.Cq), kAT, 0, st>>>(a, c);
+    const long long tot = (long long)nk * a.Ck * D;
+    acc_prefix_kernel<D><<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(a, c);
+  }
+  if (dip) {
+    ProfScope ps(st, "accum_block_a");
+    const size_t sm = ((size_t)a.Cq * (D + 1) + 32 * (D + 1) + 32 * D + 32 * a.Cq) * 4 + 32 * 4;
+    cudaFuncSetAttribute(acc_block_a_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    acc_block_a_kernel<T, D><<<dim3(nq, a.Ck), kAT, sm, st>>>(a, c);
+    const long long tot = (long long)nq * a.Cq * a.Ck * D;
+    acc_prefix_a_kernel<D><<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(a, c);
+  }
+  if (a.topk > 0 && c.k2 > 0) {
+    ProfScope ps(st, "accum_select");
+    const int smax = a.Ck > c.NB ? a.Ck : c.NB;
+    const size_t sm = ((size_t)kAW * smax + (size_t)kAW * D) * 8;
+    cudaFuncSetAttribute(acc_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    acc_select_kernel<<<dim3(nq, c.NB), kAT, sm, st>>>(a, c);
+  }
+  {
+    ProfScope ps(st, "accum_stage2");
+    const size_t sm = ((size_t)2 * a.Ck * D + a.Ck + D) * 4 + (size_t)a.Ck * 4;
+    auto kern = dip ? acc_stage2_kernel<T, D, true> : acc_stage2_kernel<T, D, false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    kern<<<dim3(nq, c.NB, a.Cq), kAT, sm, st>>>(a, c);
+  }
+}
+
+}  // namespace
+
+bool accum_supported(int D, int Cq, int Ck, int NB, int k2, int mode) {
+  if (mode != 0 && mode != 1) return false;
+  if (D != 64 && D != 128) return false;
+  if (Cq > 256 || Ck > 256 || Ck * D > 16384) return false;
+  if (mode == 1 && Cq * D > kAT * 32) return false;  // acc_block_a: 32 outputs per thread
+  if (NB < 1 || NB > 1024 || k2 < 0 || k2 > NB) return false;
+  return true;
+}
+
+void run_accum(const AttnArgs& a, const AccArgs& c, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  if (a.qg.dtype == 0) {
+    if (a.qg.D == 64) launch_accum<bf, 64>(a, c, st);
+    else launch_accum<bf, 128>(a, c, st);
+  } else {
+    if (a.qg.D == 64) launch_accum<float, 64>(a, c, st);
+    else launch_accum<float, 128>(a, c, st);
+  }
+}
+
+}  // namespace muse

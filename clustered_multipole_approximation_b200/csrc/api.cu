@@ -375,6 +375,72 @@ BwdLayout bwd_layout(const muse_shape* sh, const muse_params* pr, const AttnLayo
   return r;
 }
 
+// Workspace of the block-accumulation causal operator: the acausal
+// clusterings' state, the fp16 copy of V, one partial per query, the block
+// tables and the selections.
+struct AccLayout {
+  int* err;
+  __half* V16;
+  RoleGeo qg, kg;
+  KState qs, ks;
+  float* part;
+  AccArgs c;
+  size_t bytes;
+};
+
+AccLayout accum_layout(const muse_shape* sh, const muse_params* pr, int k2, const void* Q,
+                       const void* K, void* ws) {
+  AccLayout L{};
+  const Levels lv = make_levels(sh->N, sh->N, false);
+  const int dt = sh->dtype == MUSE_BF16 ? 0 : 1;
+  L.kg = make_geo(K, sh->B * sh->Hkv, sh->D, pr->Ck, 0, dt, pr->seed, lv);
+  L.qg = make_geo(Q, sh->B * sh->Hq, sh->D, pr->Cq, 1, dt, pr->seed, lv);
+  L.kg.sid0 = pr->key_stream0;
+  L.qg.sid0 = pr->query_stream0;
+  Carver cv{static_cast<char*>(ws)};
+  L.err = cv.take<int>(4);
+  carve_kstate(cv, L.ks, L.kg);
+  carve_kstate(cv, L.qs, L.qg);
+  L.ks.err = L.qs.err = L.err;
+  const size_t BHq = (size_t)sh->B * sh->Hq, BHk = (size_t)sh->B * sh->Hkv, N = sh->N, D = sh->D;
+  L.V16 = dt == 0 ? cv.take<__half>(BHk * N * D * 2) : nullptr;
+  L.part = cv.take<float>(BHq * N * (D + 1) * 4);
+  AccArgs& c = L.c;
+  c.L = pr->block;
+  c.NB = pr->block > 0 ? (int)(N / pr->block) : 1;
+  c.k2 = k2;
+  const size_t nk = L.ks.nprob, nq = L.qs.nprob, NB = c.NB, Cq = pr->Cq, Ck = pr->Ck;
+  const size_t k1 = pr->topk > 0 ? pr->topk : 1, kk2 = k2 > 0 ? k2 : 1;
+  c.kboff = cv.take<int>(nk * Ck * (NB + 1) * 4);
+  c.qboff = cv.take<int>(nq * Cq * (NB + 1) * 4);
+  c.bn = cv.take<int>(nk * NB * Ck * 4);
+  c.pn = cv.take<int>(nk * NB * Ck * 4);
+  c.bk = cv.take<double>(nk * NB * Ck * D * 8);
+  c.pk = cv.take<double>(nk * NB * Ck * D * 8);
+  c.bs = cv.take<float>(nk * NB * Ck * D * 4);
+  c.ps = cv.take<float>(nk * NB * Ck * D * 4);
+  const bool dip = pr->mode == MUSE_DIPOLE;
+  c.ba = dip ? cv.take<float>(nq * NB * Cq * Ck * D * 4) : nullptr;
+  c.pa = dip ? cv.take<float>(nq * NB * Cq * Ck * D * 4) : nullptr;
+  c.sel1 = cv.take<int>(nq * NB * Cq * k1 * 4);
+  c.sel2 = cv.take<int>(nq * NB * Cq * k1 * kk2 * 4);
+  L.bytes = cv.used + 256;
+  return L;
+}
+
+muse_status validate_accum(const muse_shape* sh, const muse_params* pr, int k2) {
+  muse_status s = validate(sh, pr, false);
+  if (s != MUSE_OK) return s;
+  if (pr->block < 1 || sh->N % pr->block) return fail(MUSE_ERR_INVALID_ARG, "block must divide N");
+  if (k2 < 0 || k2 > sh->N / pr->block)
+    return fail(MUSE_ERR_INVALID_ARG, "topk2 must be in [0, N / block]");
+  if (!accum_supported(sh->D, pr->Cq, pr->Ck, sh->N / pr->block, k2, (int)pr->mode))
+    return fail(MUSE_ERR_UNSUPPORTED,
+                "block accumulation needs MONOPOLE or DIPOLE, Cq, Ck <= 256, Ck * D <= 16384, "
+                "N / block <= 1024 (DIPOLE: Cq * D <= 8192)");
+  return MUSE_OK;
+}
+
 muse_status validate_bwd(const muse_shape* sh, const muse_params* pr) {
   muse_status s = validate(sh, pr, false);
   if (s != MUSE_OK) return s;
@@ -445,6 +511,80 @@ muse_status muse_attn_bwd(const void* Q, const void* K, const void* V, const voi
   cudaMemsetAsync(b.dmu, 0, nk * pr->Ck * sh->D * 4, st);
   cudaMemsetAsync(b.dnu, 0, nq * pr->Cq * sh->D * 4, st);
   run_attn_bwd(a, L.s1, b, st);
+  return check_launch();
+}
+
+size_t muse_accum_workspace_size(const muse_shape* shape, const muse_params* params, int topk2) {
+  if (validate_accum(shape, params, topk2) != MUSE_OK) return 0;
+  return accum_layout(shape, params, topk2, nullptr, nullptr, nullptr).bytes;
+}
+
+muse_status muse_attn_fwd_causal_accum(const void* Q, const void* K, const void* V, void* O,
+                                       const muse_shape* sh, const muse_params* pr, int topk2,
+                                       muse_accum_debug* dbg, void* ws, size_t ws_bytes,
+                                       cudaStream_t st) {
+  muse_status s = validate_accum(sh, pr, topk2);
+  if (s != MUSE_OK) return s;
+  if (!Q || !K || !V || !O) return fail(MUSE_ERR_INVALID_ARG, "Q, K, V and O must not be NULL");
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16))
+    return fail(MUSE_ERR_INVALID_ARG, "Q, K, V and O must be 16-byte aligned");
+  if (misaligned(ws, 256)) return fail(MUSE_ERR_INVALID_ARG, "the workspace must be 256-byte aligned");
+  if (dbg && (misaligned(dbg->q_assign, 4) || misaligned(dbg->k_assign, 4) ||
+              misaligned(dbg->sel1, 4) || misaligned(dbg->sel2, 4) ||
+              misaligned(dbg->n_exact, 8) || misaligned(dbg->device_error, 4)))
+    return fail(MUSE_ERR_INVALID_ARG, "debug outputs must be aligned to their element size");
+  if (!ws || ws_bytes < accum_layout(sh, pr, topk2, Q, K, nullptr).bytes)
+    return fail(MUSE_ERR_WORKSPACE, "workspace too small");
+  AccLayout L = accum_layout(sh, pr, topk2, Q, K, ws);
+  AttnArgs a{};
+  a.qg = L.qg;
+  a.kg = L.kg;
+  a.qs = L.qs;
+  a.ks = L.ks;
+  a.V = V;
+  a.V16 = L.V16;
+  a.out_f32 = sh->out_f32 ? 1 : 0;
+  a.part = L.part;
+  a.n_exact = dbg ? reinterpret_cast<long long*>(dbg->n_exact) : nullptr;
+  a.B = sh->B;
+  a.G = sh->Hq / sh->Hkv;
+  a.mode = (int)pr->mode;
+  a.topk = topk2 > 0 ? pr->topk : 0;  // no block retrieved: no cluster retrieval either
+  a.scale = pr->scale;
+  a.Cq = pr->Cq;
+  a.Ck = pr->Ck;
+  a.accum = 1;
+  const AccArgs& c = L.c;
+  const size_t N = sh->N, D = sh->D, nk = L.ks.nprob, nq = L.qs.nprob, NB = c.NB;
+  cudaMemsetAsync(L.err, 0, 4, st);
+  if (a.n_exact) cudaMemsetAsync(a.n_exact, 0, (size_t)sh->B * sh->Hq * N * 8, st);
+  cudaMemsetAsync(c.bn, 0, nk * NB * pr->Ck * 4, st);
+  cudaMemsetAsync(c.bk, 0, nk * NB * pr->Ck * D * 8, st);
+  cudaMemsetAsync(c.bs, 0, nk * NB * pr->Ck * D * 4, st);
+  if (c.ba) cudaMemsetAsync(c.ba, 0, nq * NB * pr->Cq * pr->Ck * D * 4, st);
+  if (L.V16) run_bf16_to_half(V, L.V16, (size_t)sh->B * sh->Hkv * N * D, L.err, st);
+  cudaMemsetAsync(L.ks.arrive, 0, nk * 4, st);
+  cudaMemsetAsync(L.qs.arrive, 0, nq * 4, st);
+  const RoleGeo gs[2] = {L.kg, L.qg};
+  const KState kss[2] = {L.ks, L.qs};
+  run_kmeans_init(gs, kss, 2, nullptr, st);
+  if (!launch_kmeans_fused(gs, kss, 2, pr->iters, st)) {
+    run_kmeans_rounds(L.kg, L.ks, pr->iters, st);
+    run_kmeans_rounds(L.qg, L.qs, pr->iters, st);
+  }
+  run_accum(a, c, st);
+  a.O = O;
+  run_local_merge(a, pr->block, st);
+  if (dbg) {
+    if (dbg->device_error) cudaMemcpyAsync(dbg->device_error, L.err, 4, cudaMemcpyDeviceToDevice, st);
+    if (dbg->q_assign) cudaMemcpyAsync(dbg->q_assign, L.qs.assign, (size_t)L.qs.ntok * 4, cudaMemcpyDeviceToDevice, st);
+    if (dbg->k_assign) cudaMemcpyAsync(dbg->k_assign, L.ks.assign, (size_t)L.ks.ntok * 4, cudaMemcpyDeviceToDevice, st);
+    if (a.topk > 0) {
+      const size_t rows = nq * NB * pr->Cq * pr->topk;
+      if (dbg->sel1) cudaMemcpyAsync(dbg->sel1, c.sel1, rows * 4, cudaMemcpyDeviceToDevice, st);
+      if (dbg->sel2) cudaMemcpyAsync(dbg->sel2, c.sel2, rows * topk2 * 4, cudaMemcpyDeviceToDevice, st);
+    }
+  }
   return check_launch();
 }
 

@@ -50,6 +50,8 @@ struct AttnArgs {
   void* kpad;         // those levels' keys, cluster-sorted, group-padded, pre-swizzled (bf16)
   void* vpad;         // the same for V (fp16)
   int* gofs;          // [key problems][Ck + 1] first group of each cluster in kpad / vpad
+  int accum;          // causal local merge: one partial per query of blocks >= 1 at row
+                      // b H N + q (block-summary accumulation), else the level partials
 };
 
 // Key problem that a query problem attends: the same (b, level, pair) of the
@@ -143,6 +145,25 @@ struct BwdArgs {
 };
 bool backward_supported(int D, int Ck, int mode);
 void run_attn_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st);
+
+// Causal operator with block-summary accumulation (accum.cu).
+struct AccArgs {
+  int L, NB, k2;   // block size, blocks, blocks retrieved per selected cluster
+  int* kboff;      // [key sets][Ck][NB + 1] first member of each block in a cluster's list
+  int* qboff;      // [query sets][Cq][NB + 1]
+  int* bn;         // [key sets][NB][Ck] members of (block, cluster)
+  int* pn;         // [key sets][NB][Ck] exclusive prefix over blocks
+  double* bk;      // [key sets][NB][Ck][D] key sums (token order)
+  double* pk;      // prefix of bk (block order)
+  float* bs;       // [key sets][NB][Ck][D] value sums
+  float* ps;       // prefix of bs
+  float* ba;       // [query sets][NB][Cq][Ck][D] sum v (k . nu_i) (DIPOLE)
+  float* pa;       // prefix of ba
+  int* sel1;       // [query sets][NB][Cq][k1] selected key clusters, -1 padded
+  int* sel2;       // [query sets][NB][Cq][k1][k2] selected blocks, -1 padded
+};
+bool accum_supported(int D, int Cq, int Ck, int NB, int k2, int mode);
+void run_accum(const AttnArgs& a, const AccArgs& c, cudaStream_t st);
 
 // Causal: exact local block + merge of the level partials into O.
 void run_local_merge(const AttnArgs& a, int L, cudaStream_t st);

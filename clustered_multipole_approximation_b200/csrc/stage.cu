@@ -479,12 +479,13 @@ __global__ void __launch_bounds__(kQ * (D / 64)) local_merge_kernel(AttnArgs a, 
     }
   }
   if (!valid) return;
-  const int levels = a.qg.lv.nlev;
+  const int levels = a.accum ? (blk > 0 ? 1 : 0) : a.qg.lv.nlev;
   for (int lv = 0; lv < levels; ++lv) {
-    if (!((blk >> lv) & 1)) continue;
+    if (!a.accum && !((blk >> lv) & 1)) continue;
     const int sz = L << lv, p = blk >> (lv + 1);
-    const long long slot = (long long)bhq * a.qg.lv.toks_per_bh + a.qg.lv.tok_base[lv] +
-                           (long long)p * sz + (qpos - (2 * p + 1) * sz);
+    const long long slot = a.accum ? qrow
+                                   : (long long)bhq * a.qg.lv.toks_per_bh + a.qg.lv.tok_base[lv] +
+                                         (long long)p * sz + (qpos - (2 * p + 1) * sz);
     const float* pp = a.part + slot * (D + 1);
     const float lg = pp[D];
     if (lg > m) {

@@ -551,17 +551,18 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) local_mma_kernel(At
   }
   if (!wact) return;
   // ---- the level partials of each row, one softmax term each -----------------
-  const int levels = a.qg.lv.nlev;
+  const int levels = a.accum ? (blk > 0 ? 1 : 0) : a.qg.lv.nlev;
   const float* part = a.part;
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     const int qp = qpos[r];
     if (qp >= kend) continue;
     for (int lv = 0; lv < levels; ++lv) {
-      if (!((blk >> lv) & 1)) continue;
+      if (!a.accum && !((blk >> lv) & 1)) continue;
       const int sz = L << lv, pp_ = blk >> (lv + 1);
-      const long long slot = (long long)bhq * a.qg.lv.toks_per_bh + a.qg.lv.tok_base[lv] +
-                             (long long)pp_ * sz + (qp - (2 * pp_ + 1) * sz);
+      const long long slot = a.accum ? (long long)bhq * N + qp
+                                     : (long long)bhq * a.qg.lv.toks_per_bh + a.qg.lv.tok_base[lv] +
+                                           (long long)pp_ * sz + (qp - (2 * pp_ + 1) * sz);
       const float* pp = part + slot * (D + 1);
       const float lg = pp[D] * 1.4426950408889634f;  // natural log -> base 2
       const float mn = fmaxf(mrow[r], lg);

@@ -234,6 +234,41 @@ muse_status muse_attn_fwd_causal(const void *Q, const void *K, const void *V,
                                  void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Causal MuSe with causal accumulation of block summaries and two-level
+ * retrieval ([G] Technical Summary, Core Mechanisms: "Causal Accumulation"
+ * and "Retrieval-Augmented Approximation").  Keys and queries are clustered
+ * over the whole sequence (the clusterings of muse_attn_fwd).  With
+ * L = params->block (N % L == 0) and NB = N / L blocks, a query q in block b
+ * attends exactly to the keys [bL, q] of its own block and, for b >= 1:
+ *   - selects the top params->topk key clusters j by
+ *     s nu_i . mu_j^{<b} + log n_j^{<b}, the summary of j's members in blocks
+ *     0 .. b-1 accumulated block by block (fp64, ties to the lowest j);
+ *   - within each, the top topk2 blocks b' < b by s nu_i . mu_jb' + log n_jb'
+ *     (ties to the lowest block), and attends exactly to their keys;
+ *   - sees every key cluster's remaining prefix members (outside the
+ *     retrieved blocks) as one far term: logit s q.mu + log n, value S / n
+ *     (MONOPOLE) or (S + s M nu_i) / n (DIPOLE, M about that set's centroid).
+ * All terms meet in one softmax.  topk2 == 0 retrieves nothing.  Supported:
+ * MONOPOLE and DIPOLE, Cq, Ck <= 256, Ck * D <= 16384, N / L <= 1024, and
+ * for DIPOLE Cq * D <= 8192 (MUSE_ERR_UNSUPPORTED otherwise).
+ * Debug layouts: q_assign [B,Hq,N], k_assign [B,Hkv,N],
+ * sel1 [B,Hq,NB,Cq,topk], sel2 [B,Hq,NB,Cq,topk,topk2] (-1 padded; rows of
+ * block 0 and of clusters with no query in the block are -1),
+ * n_exact [B,Hq,N] (retrieved plus local keys).
+ */
+typedef struct {
+  int32_t *q_assign, *k_assign, *sel1, *sel2;
+  int64_t *n_exact;
+  int32_t *device_error;
+} muse_accum_debug;
+
+size_t muse_accum_workspace_size(const muse_shape *shape, const muse_params *params, int topk2);
+muse_status muse_attn_fwd_causal_accum(const void *Q, const void *K, const void *V, void *O,
+                                       const muse_shape *shape, const muse_params *params,
+                                       int topk2, muse_accum_debug *debug, void *ws,
+                                       size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Gradients of the acausal operator: dQ, dK, dV of <dO, O> for the O of a
  * muse_attn_fwd call ([G] Experimental Results: the layer is trained
  * through).  The clusterings and the retrieval sets are held at the forward

@@ -146,3 +146,25 @@ def test_backward_workspace_and_argument_checks(lib):
     assert st == 2
     st = lib.muse_attn_bwd(*args, ctypes.byref(sh), ctypes.byref(pr), fake, fwd, None)
     assert st == 3 and b"backward" in lib.muse_last_error()
+
+
+def test_accum_workspace_and_argument_checks(lib):
+    """The block-accumulation entry point sizes its workspace and refuses
+    unsupported modes, sizes and budgets before launching anything."""
+    sh = shape()
+    ok = lib.muse_accum_workspace_size(ctypes.byref(sh), ctypes.byref(params(block=128)), 2)
+    assert ok > 0
+    mono = lib.muse_accum_workspace_size(ctypes.byref(sh), ctypes.byref(params(block=128, mode=0)), 2)
+    assert 0 < mono < ok  # no A tables for MONOPOLE
+    bad = [(params(block=100), 2), (params(block=128), 9), (params(block=128, mode=2), 2),
+           (params(block=128, Ck=300), 2), (params(block=0), 0)]
+    for pr, k2 in bad:
+        assert lib.muse_accum_workspace_size(ctypes.byref(sh), ctypes.byref(pr), k2) == 0
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+    st = lib.muse_attn_fwd_causal_accum(None, fake, fake, fake, ctypes.byref(sh),
+                                        ctypes.byref(params(block=128)), 2, None, fake, 1 << 40,
+                                        None)
+    assert st == 1 and b"NULL" in lib.muse_last_error()
+    st = lib.muse_attn_fwd_causal_accum(fake, fake, fake, fake, ctypes.byref(sh),
+                                        ctypes.byref(params(block=128)), 2, None, fake, 16, None)
+    assert st == 3
