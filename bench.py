@@ -54,6 +54,8 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
     p.add_argument("--mode", default=None, choices=[None, "dipole", "monopole", "tilted", "dipole_q"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--accum", action="store_true",
+                   help="time only the block-accumulation causal form of a causal workload")
     p.add_argument("--backward", action="store_true",
                    help="time only the backward pass of an acausal workload (one JSON line)")
     p.add_argument("--no-side", action="store_true",
@@ -511,6 +513,74 @@ def run_backward(w, mode, steps, warmup, device):
 
 
 # ---------------------------------------------------------------------------
+# the causal operator with block-summary accumulation and cluster/block retrieval
+# ---------------------------------------------------------------------------
+ACCUM_K1, ACCUM_K2 = 4, 2  # no workload states k1 / k2 for this form: 4 clusters, 2 blocks each
+
+
+def run_accum_bench(w, mode, steps, warmup, device, k1=ACCUM_K1, k2=ACCUM_K2):
+    """Times `steps` calls of muse_attn_fwd_causal_accum on the causal
+    workload `w` (inputs resident, L2 flushed between calls); returns
+    tokens/s, ms per call, per-kernel times and the RSE against exact causal
+    attention."""
+    import clustered_multipole_approximation_b200 as muse
+
+    Q, K, V = make_inputs(w)
+    cast = (lambda x: torch.from_numpy(x).to(torch.bfloat16)) if w.dtype == "bf16" else torch.from_numpy
+    q, k, v = cast(Q).to(device), cast(K).to(device), cast(V).to(device)
+    del Q, K, V
+    kw = dict(Cq=w.C, Ck=w.C, block=w.block, iters=w.iters, seed=w.cluster_seed, topk=k1,
+              topk2=k2, scale=w.scale, mode=mode)
+    p = muse.make_params(w.C, w.C, w.iters, w.cluster_seed, k1, w.block, w.scale, mode)
+    ws = torch.empty(muse.accum_workspace_size(q, k, p, k2), dtype=torch.uint8, device=device)
+    out = torch.empty_like(q)
+    o = muse.muse_attn_fwd_causal_accum(q, k, v, workspace=ws, out_dtype=torch.float32, **kw)
+    G = w.Hq // w.Hkv
+    num = den = 0.0
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    for h0 in range(0, w.Hq, G):
+        qq = q[:, h0:h0 + G].float()
+        kk = k[:, h0 // G:h0 // G + 1].float().expand(-1, G, -1, -1)
+        vv = v[:, h0 // G:h0 // G + 1].float().expand(-1, G, -1, -1)
+        with sdpa_kernel([SDPBackend.EFFICIENT_ATTENTION]):
+            E = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, is_causal=True,
+                                                                 scale=w.scale)
+        num += float(((o[:, h0:h0 + G] - E) ** 2).sum())
+        den += float((E ** 2).sum())
+        del E, qq, kk, vv
+    del o
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        muse.muse_attn_fwd_causal_accum(q, k, v, out=out, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    muse.profile_read()
+    muse.profile_enable(True)
+    total = 0.0
+    for _ in range(steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        muse.muse_attn_fwd_causal_accum(q, k, v, out=out, workspace=ws, **kw)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1)
+    muse.profile_enable(False)
+    prof = muse.profile_read()
+    ms = total / steps
+    tot = sum(t for _, t in prof.values())
+    kernels = {n: {"launches": c, "ms_per_call": round(t / steps, 4), "share": round(t / tot, 4)}
+               for n, (c, t) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    del q, k, v, out, ws, flush
+    torch.cuda.empty_cache()
+    cfg = dict(config_of(w, mode), topk=k1, topk2=k2, form="block-summary accumulation")
+    return {"config": cfg, "value": w.B * w.N / (ms / 1e3), "unit": UNIT, "ms_per_call": ms,
+            "steps": steps, "warmup": warmup, "rse_vs_exact": num / den, "kernels": kernels}
+
+
+# ---------------------------------------------------------------------------
 # the oracle on the host cores (CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
 def oracle_sample(w, mode, heads):
@@ -595,6 +665,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     mode = args.mode or w.mode
+    if args.accum:
+        if rank == 0:
+            print(json.dumps(run_accum_bench(w, mode, args.steps, args.warmup, device)), flush=True)
+        return
     if args.backward:
         if rank == 0:
             print(json.dumps(run_backward(w, mode, args.steps, args.warmup, device)), flush=True)
@@ -622,6 +696,9 @@ def main():
     if world == 1 and not args.no_side and args.workload == DEFAULT_WORKLOAD and args.mode is None:
         line["backward"] = {m: run_backward(w, m, args.steps, args.warmup, device)
                             for m in ("dipole", "monopole")}
+        cw = WORKLOADS["causal-bf16-b2h8-n16k"]
+        line["accum"] = {m: run_accum_bench(cw, m, args.steps, args.warmup, device)
+                         for m in ("dipole", "monopole")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads = min(w.B * w.Hq, 8)
         dt, tps, thr = oracle_sample(w, r["mode"], heads)

@@ -107,12 +107,18 @@ __global__ void acc_prefix_kernel(AttnArgs a, AccArgs c) {
   int pn = 0;
   for (int b = 0; b < NB; ++b) {
     const size_t o = ((size_t)pid * NB + b) * Ck + j;
+    const int bn = c.bn[o];
+    const double bk = c.bk[o * D + d];
     c.pk[o * D + d] = pk;
     c.ps[o * D + d] = ps;
+    // centroids of the prefix and of the block, for the selection scores
+    const size_t ot = (((size_t)pid * NB + b) * D + d) * Ck + j;  // dimension-major
+    c.pmu[ot] = pn > 0 ? __ddiv_rn(pk, (double)pn) : 0.0;
+    c.bmu[ot] = bn > 0 ? __ddiv_rn(bk, (double)bn) : 0.0;
     if (d == 0) c.pn[o] = pn;
-    pk += c.bk[o * D + d];
+    pk += bk;
     ps += c.bs[o * D + d];
-    pn += c.bn[o];
+    pn += bn;
   }
 }
 
@@ -217,9 +223,10 @@ __global__ void acc_prefix_a_kernel(AttnArgs a, AccArgs c) {
 // ---------------------------------------------------------------------------
 // selection: per (q-set, block b), warps over the query clusters present in b
 // ---------------------------------------------------------------------------
-__device__ inline double dot_ordered(const double* x, const double* y, double div, int D) {
+// x . y in dimension order (no fused multiply-add); y strided by `ys`
+__device__ inline double dot_ordered(const double* x, const double* y, size_t ys, int D) {
   double s = 0.0;
-  for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(x[d], __ddiv_rn(y[d], div)));
+  for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(x[d], y[(size_t)d * ys]));
   return s;
 }
 
@@ -246,8 +253,8 @@ __global__ void __launch_bounds__(kAT) acc_select_kernel(AttnArgs a, AccArgs c) 
     for (int j = lane; j < Ck; j += 32) {
       const size_t o = ((size_t)kpid * NB + b) * Ck + j;
       const int n = c.pn[o];
-      sc[j] = n > 0 ? __dadd_rn(__dmul_rn(s, dot_ordered(nu, c.pk + o * D, (double)n, D)),
-                                log((double)n))
+      const double* mu = c.pmu + ((size_t)kpid * NB + b) * D * Ck + j;  // lanes: consecutive j
+      sc[j] = n > 0 ? __dadd_rn(__dmul_rn(s, dot_ordered(nu, mu, Ck, D)), log((double)n))
                     : -INFINITY;
     }
     __syncwarp();
@@ -283,8 +290,8 @@ __global__ void __launch_bounds__(kAT) acc_select_kernel(AttnArgs a, AccArgs c) 
       for (int bb = lane; bb < b; bb += 32) {
         const size_t o = ((size_t)kpid * NB + bb) * Ck + j;
         const int n = c.bn[o];
-        sc[bb] = n > 0 ? __dadd_rn(__dmul_rn(s, dot_ordered(nu, c.bk + o * D, (double)n, D)),
-                                   log((double)n))
+        const double* mu = c.bmu + ((size_t)kpid * NB + bb) * D * Ck + j;
+        sc[bb] = n > 0 ? __dadd_rn(__dmul_rn(s, dot_ordered(nu, mu, Ck, D)), log((double)n))
                        : -INFINITY;
       }
       __syncwarp();
@@ -318,165 +325,339 @@ __global__ void __launch_bounds__(kAT) acc_select_kernel(AttnArgs a, AccArgs c) 
 }
 
 // ---------------------------------------------------------------------------
-// far summaries + retrieved keys: one CTA per (q-set, block b, query cluster i)
+// far summaries + retrieved keys: one CTA per (q-set, block b, kCI query
+// clusters).  The prefix table of the block (centroids, log-counts and, for
+// MONOPOLE, the values) is built once per CTA; per query cluster i the CTA
+// adds the remainders of its selected clusters (prefix minus the retrieved
+// blocks) and, for DIPOLE, its values u_ij.  One warp per query; the far
+// terms one key cluster per lane.
 // ---------------------------------------------------------------------------
+constexpr int kCI = 16;   // query clusters per CTA
+constexpr int kST = 512;  // threads of the stage-2 CTA (one CTA per SM fits its tables)
+constexpr int kSW = kST / 32;
+constexpr int kXL = 1024; // retrieved keys listed in shared memory per pass
+
+template <int D>
+size_t stage2_smem(int Ck, int k1) {
+  return ((size_t)Ck * (D + 1) + (size_t)Ck * D + Ck + (size_t)k1 * (D + 1) + (size_t)k1 * D + k1 +
+          (size_t)kSW * D + D) * 4 + (size_t)Ck * 4 + 8 + (size_t)kXL * 8 + (size_t)kSW * 32 * 4 +
+         (size_t)kSW * 32 * 8;
+}
+
 template <typename T, int D, bool DIP>
-__global__ void __launch_bounds__(kAT) acc_stage2_kernel(AttnArgs a, AccArgs c) {
+__global__ void __launch_bounds__(kST) acc_stage2_kernel(AttnArgs a, AccArgs c) {
   extern __shared__ __align__(16) float s2_raw[];
-  const int Cq = a.Cq, Ck = a.Ck, NB = c.NB, k1 = a.topk, k2 = c.k2, L = c.L;
-  float* mu_s = s2_raw;                  // [Ck][D]
-  float* u_s = mu_s + (size_t)Ck * D;    // [Ck][D]
-  float* ln_s = u_s + (size_t)Ck * D;    // [Ck]   log n of the far set, -inf if empty
-  float* nu = ln_s + Ck;                 // [D]
-  int* rsel = reinterpret_cast<int*>(nu + D);  // [Ck] rank of j among the selected clusters, or -1
+  const int Cq = a.Cq, Ck = a.Ck, NB = c.NB, k1 = a.topk, k2 = c.k2;
+  float* mu_s = s2_raw;                         // [Ck][D + 1] prefix centroids
+  float* u_s = mu_s + (size_t)Ck * (D + 1);     // [Ck][D] values (DIPOLE: of cluster i)
+  float* ln_s = u_s + (size_t)Ck * D;           // [Ck] log n, -inf if empty
+  float* rm_s = ln_s + Ck;                      // [k1][D + 1] remainder centroids
+  float* ru_s = rm_s + (size_t)k1 * (D + 1);    // [k1][D] remainder values
+  float* rl_s = ru_s + (size_t)k1 * D;          // [k1] remainder log n
+  float* q_s = rl_s + k1;                       // [kSW][D] each warp's query
+  float* nu = q_s + kSW * D;                    // [D]
+  int* rsel = reinterpret_cast<int*>(nu + D);   // [Ck] rank among the selected, or -1
+  long long* xrow = reinterpret_cast<long long*>(  // [kXL] rows of the retrieved keys
+      reinterpret_cast<uintptr_t>(rsel + Ck + 1) & ~(uintptr_t)7);
+  float* pw_s = reinterpret_cast<float*>(xrow + kXL);             // [kSW][32] far weights
+  const float** uw_s = reinterpret_cast<const float**>(pw_s + kSW * 32);  // [kSW][32] their rows
   __shared__ int nretr;
-  const int qpid = blockIdx.x, b = blockIdx.y, i = blockIdx.z;
+  const int qpid = blockIdx.x, b = blockIdx.y, i0 = blockIdx.z * kCI;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (b == 0) return;
-  const int* qb = c.qboff + ((size_t)qpid * Cq + i) * (NB + 1);
-  const int m0 = qb[b], m1 = qb[b + 1];
-  if (m1 == m0) return;
   const Prob pq = prob_of(a.qg, qpid);
   const int kpid = kv_problem(a, qpid);
   const Prob pk = prob_of(a.kg, kpid);
   const float s = a.scale;
-  const int* s1 = c.sel1 + (((size_t)qpid * NB + b) * Cq + i) * k1;
-  const int* s2 = c.sel2 + ((((size_t)qpid * NB + b) * Cq + i) * k1) * k2;
-  for (int d = tid; d < D; d += kAT) nu[d] = a.qs.cent32[((size_t)qpid * Cq + i) * D + d];
-  for (int j = tid; j < Ck; j += kAT) rsel[j] = -1;  // index into s1, -1 if not selected
-  __syncthreads();
-  if (tid < k1 && s1[tid] >= 0) rsel[s1[tid]] = tid;
-  __syncthreads();
-  // far table: prefix minus the retrieved blocks, one warp per key cluster
-  for (int j = warp; j < Ck; j += kAW) {
+  constexpr int DL = D / 32;
+  // ---- the block's prefix table --------------------------------------------
+  for (int j = warp; j < Ck; j += kSW) {
     const size_t o = ((size_t)kpid * NB + b) * Ck + j;
-    int n = c.pn[o];
-    const int r = rsel[j];
-    double ksum[D / 32];
-    float ss[D / 32], aa[D / 32];
+    const int n = c.pn[o];
+    if (lane == 0) ln_s[j] = n > 0 ? logf((float)n) : -INFINITY;
+    if (n == 0) continue;
 #pragma unroll
-    for (int u = 0; u < D / 32; ++u) {
+    for (int u = 0; u < DL; ++u) {
       const int d = lane + 32 * u;
-      ksum[u] = c.pk[o * D + d];
-      ss[u] = c.ps[o * D + d];
-      aa[u] = DIP ? c.pa[((((size_t)qpid * NB + b) * Cq + i) * Ck + j) * D + d] : 0.f;
+      mu_s[j * (D + 1) + d] = (float)(c.pk[o * D + d] / (double)n);
+      if (!DIP) u_s[j * D + d] = c.ps[o * D + d] / (float)n;
     }
-    if (r >= 0) {
+  }
+  const T* Q = static_cast<const T*>(a.qg.X);
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  const int* kperm = a.ks.perm + pk.slot0;
+  const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
+  for (int i = i0; i < imin(i0 + kCI, Cq); ++i) {
+    const int* qb = c.qboff + ((size_t)qpid * Cq + i) * (NB + 1);
+    const int m0 = qb[b], m1 = qb[b + 1];
+    if (m1 == m0) continue;  // no query of cluster i in block b (CTA-uniform)
+    const int* s1 = c.sel1 + (((size_t)qpid * NB + b) * Cq + i) * k1;
+    const int* s2 = c.sel2 + ((((size_t)qpid * NB + b) * Cq + i) * k1) * k2;
+    __syncthreads();  // the previous cluster's readers are done
+    for (int d = tid; d < D; d += kST) nu[d] = a.qs.cent32[((size_t)qpid * Cq + i) * D + d];
+    for (int j = tid; j < Ck; j += kST) rsel[j] = -1;
+    __syncthreads();
+    if (tid < k1 && s1[tid] >= 0) rsel[s1[tid]] = tid;
+    if (tid == 0) {
+      int cnt = 0;
+      for (int r = 0; r < k1; ++r) {
+        const int j = s1[r];
+        if (j < 0) break;
+        for (int r2 = 0; r2 < k2; ++r2) {
+          const int bb = s2[r * k2 + r2];
+          if (bb < 0) break;
+          cnt += c.bn[((size_t)kpid * NB + bb) * Ck + j];
+        }
+      }
+      nretr = cnt;
+    }
+    __syncthreads();  // rsel and nretr complete
+    // the rows of the first kXL retrieved keys (the rest are read in place)
+    const int nx = imin(nretr, kXL);
+    if (warp == 0) {
+      int base = 0;
+      for (int r = 0; r < k1 && base < nx; ++r) {
+        const int j = s1[r];
+        if (j < 0) break;
+        const int* kb = c.kboff + ((size_t)kpid * Ck + j) * (NB + 1);
+        for (int r2 = 0; r2 < k2 && base < nx; ++r2) {
+          const int bb = s2[r * k2 + r2];
+          if (bb < 0) break;
+          const int cnt = kb[bb + 1] - kb[bb];
+          for (int mm = lane; mm < cnt && base + mm < nx; mm += 32)
+            xrow[base + mm] = pk.row0 + kperm[koff[j] + kb[bb] + mm];
+          base += cnt;
+        }
+      }
+    }
+    // remainders of the selected clusters: prefix minus the retrieved blocks
+    for (int r = warp; r < k1; r += kSW) {
+      const int j = s1[r];
+      if (j < 0) {
+        if (lane == 0) rl_s[r] = -INFINITY;
+        continue;
+      }
+      const size_t o = ((size_t)kpid * NB + b) * Ck + j;
+      int n = c.pn[o];
+      double ksum[DL];
+      float ss[DL], aa[DL];
+#pragma unroll
+      for (int u = 0; u < DL; ++u) {
+        const int d = lane + 32 * u;
+        ksum[u] = c.pk[o * D + d];
+        ss[u] = c.ps[o * D + d];
+        aa[u] = DIP ? c.pa[((((size_t)qpid * NB + b) * Cq + i) * Ck + j) * D + d] : 0.f;
+      }
       for (int r2 = 0; r2 < k2; ++r2) {
         const int bb = s2[r * k2 + r2];
         if (bb < 0) break;
         const size_t ob = ((size_t)kpid * NB + bb) * Ck + j;
         n -= c.bn[ob];
 #pragma unroll
-        for (int u = 0; u < D / 32; ++u) {
+        for (int u = 0; u < DL; ++u) {
           const int d = lane + 32 * u;
           ksum[u] -= c.bk[ob * D + d];
           ss[u] -= c.bs[ob * D + d];
           if (DIP) aa[u] -= c.ba[((((size_t)qpid * NB + bb) * Cq + i) * Ck + j) * D + d];
         }
       }
-    }
-    if (n <= 0) {
-      if (lane == 0) ln_s[j] = -INFINITY;
-      continue;
-    }
-    const float inv = 1.f / (float)n;
-    float mn = 0.f;
-#pragma unroll
-    for (int u = 0; u < D / 32; ++u) {
-      const int d = lane + 32 * u;
-      const float mu = (float)(ksum[u] / (double)n);
-      mu_s[j * D + d] = mu;
-      mn = fmaf(mu, nu[d], mn);
-    }
-#pragma unroll
-    for (int o2 = 16; o2; o2 >>= 1) mn += __shfl_xor_sync(0xffffffffu, mn, o2);
-#pragma unroll
-    for (int u = 0; u < D / 32; ++u) {
-      const int d = lane + 32 * u;
-      // M nu = A - S (mu . nu) over the far set
-      u_s[j * D + d] = DIP ? fmaf(s, fmaf(-ss[u], mn, aa[u]), ss[u]) * inv : ss[u] * inv;
-    }
-    if (lane == 0) ln_s[j] = logf((float)n);
-  }
-  if (tid == 0) {
-    int cnt = 0;
-    for (int r = 0; r < k1; ++r) {
-      const int j = s1[r];
-      if (j < 0) break;
-      for (int r2 = 0; r2 < k2; ++r2) {
-        const int bb = s2[r * k2 + r2];
-        if (bb < 0) break;
-        cnt += c.bn[((size_t)kpid * NB + bb) * Ck + j];
+      if (n <= 0) {
+        if (lane == 0) rl_s[r] = -INFINITY;
+        continue;
       }
-    }
-    nretr = cnt;
-  }
-  __syncthreads();
-  // one warp per query of cluster i in block b
-  const T* Q = static_cast<const T*>(a.qg.X);
-  const T* K = static_cast<const T*>(a.kg.X);
-  const T* V = static_cast<const T*>(a.V);
-  const int* qperm = a.qs.perm + pq.slot0 + a.qs.off[(size_t)qpid * (Cq + 1) + i];
-  const int* kperm = a.ks.perm + pk.slot0;
-  const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
-  constexpr int DL = D / 32;
-  for (int m = m0 + warp; m < m1; m += kAW) {
-    const int tq = qperm[m];
-    const long long qrow = pq.row0 + tq;
-    float q[DL], o[DL];
-#pragma unroll
-    for (int u = 0; u < DL; ++u) {
-      q[u] = ld<T>(Q + qrow * D + lane + 32 * u);
-      o[u] = 0.f;
-    }
-    float mx = -INFINITY, l = 0.f;
-    auto add = [&](float lg, const float* x, bool global_t, long long vrow) {
-      const float mn = fmaxf(mx, lg);
-      const float sc = __expf(mx - mn), w = __expf(lg - mn);
-      l = l * sc + w;
+      const float inv = 1.f / (float)n;
+      float mn = 0.f;
 #pragma unroll
       for (int u = 0; u < DL; ++u) {
-        const float xv = global_t ? ld<T>(V + vrow * D + lane + 32 * u) : x[lane + 32 * u];
-        o[u] = fmaf(o[u], sc, w * xv);
+        const int d = lane + 32 * u;
+        const float mu = (float)(ksum[u] / (double)n);
+        rm_s[r * (D + 1) + d] = mu;
+        mn = fmaf(mu, nu[d], mn);
       }
-      mx = mn;
-    };
-    for (int j = 0; j < Ck; ++j) {
-      const float lnj = ln_s[j];
-      if (lnj == -INFINITY) continue;
-      float x = 0.f;
 #pragma unroll
-      for (int u = 0; u < DL; ++u) x = fmaf(q[u], mu_s[j * D + lane + 32 * u], x);
+      for (int o2 = 16; o2; o2 >>= 1) mn += __shfl_xor_sync(0xffffffffu, mn, o2);
 #pragma unroll
-      for (int o2 = 16; o2; o2 >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o2);
-      add(fmaf(s, x, lnj), u_s + (size_t)j * D, false, 0);
+      for (int u = 0; u < DL; ++u) {
+        const int d = lane + 32 * u;
+        // M nu = A - S (mu . nu) over the remainder
+        ru_s[r * D + d] = DIP ? fmaf(s, fmaf(-ss[u], mn, aa[u]), ss[u]) * inv : ss[u] * inv;
+      }
+      if (lane == 0) rl_s[r] = logf((float)n);
     }
-    for (int r = 0; r < k1; ++r) {
-      const int j = s1[r];
-      if (j < 0) break;
-      const int* kb = c.kboff + ((size_t)kpid * Ck + j) * (NB + 1);
-      for (int r2 = 0; r2 < k2; ++r2) {
-        const int bb = s2[r * k2 + r2];
-        if (bb < 0) break;
-        for (int mm = kb[bb]; mm < kb[bb + 1]; ++mm) {
-          const long long krow = pk.row0 + kperm[koff[j] + mm];
-          float x = 0.f;
+    if (DIP) {  // u_ij of the unselected clusters: (S + s (A - S (mu . nu_i))) / n
+      for (int j = warp; j < Ck; j += kSW) {
+        const size_t o = ((size_t)kpid * NB + b) * Ck + j;
+        const int n = c.pn[o];
+        if (n == 0 || rsel[j] >= 0) continue;
+        float mn = 0.f;
 #pragma unroll
-          for (int u = 0; u < DL; ++u) x = fmaf(q[u], ld<T>(K + krow * D + lane + 32 * u), x);
+        for (int u = 0; u < DL; ++u) mn = fmaf(mu_s[j * (D + 1) + lane + 32 * u], nu[lane + 32 * u], mn);
 #pragma unroll
-          for (int o2 = 16; o2; o2 >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o2);
-          add(s * x, nullptr, true, krow);
+        for (int o2 = 16; o2; o2 >>= 1) mn += __shfl_xor_sync(0xffffffffu, mn, o2);
+        const float inv = 1.f / (float)n;
+#pragma unroll
+        for (int u = 0; u < DL; ++u) {
+          const int d = lane + 32 * u;
+          const float S = c.ps[o * D + d];
+          const float A = c.pa[((((size_t)qpid * NB + b) * Cq + i) * Ck + j) * D + d];
+          u_s[j * D + d] = fmaf(s, fmaf(-S, mn, A), S) * inv;
         }
       }
     }
-    float* pp = a.part + (size_t)qrow * (D + 1);
-    const float inv = 1.f / l;
+    __syncthreads();
+    // ---- one warp per query of cluster i in block b ----------------------
+    const int* qperm = a.qs.perm + pq.slot0 + a.qs.off[(size_t)qpid * (Cq + 1) + i];
+    float* qw = q_s + warp * D;
+    for (int m = m0 + warp; m < m1; m += kSW) {
+      const long long qrow = pq.row0 + qperm[m];
+      float o[DL];
 #pragma unroll
-    for (int u = 0; u < DL; ++u) pp[lane + 32 * u] = o[u] * inv;
-    if (lane == 0) {
-      pp[D] = mx + logf(l);
-      if (a.n_exact != nullptr) a.n_exact[qrow] = nretr;
+      for (int u = 0; u < DL; ++u) {
+        qw[lane + 32 * u] = ld<T>(Q + qrow * D + lane + 32 * u);
+        o[u] = 0.f;
+      }
+      __syncwarp();
+      float mx = -INFINITY, l = 0.f;
+      // far terms, 32 key clusters at a time (one per lane); the weights go
+      // through the warp's shared-memory row so the value loop has no shuffles
+      float* pw = pw_s + warp * 32;
+      const float** uw = uw_s + warp * 32;
+      for (int j0 = 0; j0 < Ck; j0 += 32) {
+        const int j = j0 + lane;
+        float lg = -INFINITY;
+        const float* urow = u_s;
+        if (j < Ck) {
+          const int r = rsel[j];
+          const float lnj = r >= 0 ? rl_s[r] : ln_s[j];
+          if (lnj != -INFINITY) {
+            const float* mrow = r >= 0 ? rm_s + r * (D + 1) : mu_s + j * (D + 1);
+            float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;  // four chains for latency
+#pragma unroll 4
+            for (int d = 0; d < D; d += 4) {
+              x0 = fmaf(qw[d], mrow[d], x0);
+              x1 = fmaf(qw[d + 1], mrow[d + 1], x1);
+              x2 = fmaf(qw[d + 2], mrow[d + 2], x2);
+              x3 = fmaf(qw[d + 3], mrow[d + 3], x3);
+            }
+            lg = fmaf(s, (x0 + x1) + (x2 + x3), lnj);
+            urow = r >= 0 ? ru_s + r * D : u_s + j * D;
+          }
+        }
+        float bm = lg;
+#pragma unroll
+        for (int o2 = 16; o2; o2 >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o2));
+        if (bm == -INFINITY) continue;
+        const float mn = fmaxf(mx, bm);
+        const float sc = __expf(mx - mn);
+        const float p = __expf(lg - mn);
+        pw[lane] = p;
+        uw[lane] = urow;
+        float ps = p;
+#pragma unroll
+        for (int o2 = 16; o2; o2 >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o2);
+        l = l * sc + ps;
+#pragma unroll
+        for (int u = 0; u < DL; ++u) o[u] *= sc;
+        mx = mn;
+        __syncwarp();
+#pragma unroll 8
+        for (int jj = 0; jj < 32; ++jj) {
+          const float pj = pw[jj];  // 0 for an empty or absent cluster (its row is unused)
+          const float* ur = uw[jj];
+#pragma unroll
+          for (int u = 0; u < DL; ++u) o[u] = fmaf(pj, ur[lane + 32 * u], o[u]);
+        }
+        __syncwarp();
+      }
+      // exact terms: the keys of the retrieved (cluster, block) pairs, 32 at
+      // a time (one per lane for the logits, then the warp over the values)
+      for (int x0 = 0; x0 < nx; x0 += 32) {
+        const int t = x0 + lane;
+        float lg = -INFINITY;
+        long long krow = 0;
+        if (t < nx) {
+          krow = xrow[t];
+          const uint4* kp = reinterpret_cast<const uint4*>(K + krow * D);
+          float x = 0.f;
+          if (sizeof(T) == 2) {
+#pragma unroll
+            for (int c8 = 0; c8 < D / 8; ++c8) {
+              const uint4 w = __ldg(kp + c8);
+              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h[e]);
+                x = fmaf(qw[c8 * 8 + 2 * e], f.x, x);
+                x = fmaf(qw[c8 * 8 + 2 * e + 1], f.y, x);
+              }
+            }
+          } else {
+#pragma unroll 16
+            for (int d = 0; d < D; ++d) x = fmaf(qw[d], ld<T>(K + krow * D + d), x);
+          }
+          lg = s * x;
+        }
+        float bm = lg;
+#pragma unroll
+        for (int o2 = 16; o2; o2 >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o2));
+        const float mn = fmaxf(mx, bm);
+        const float sc = __expf(mx - mn);
+        const float p = __expf(lg - mn);
+        float ps = p;
+#pragma unroll
+        for (int o2 = 16; o2; o2 >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o2);
+        l = l * sc + ps;
+#pragma unroll
+        for (int u = 0; u < DL; ++u) o[u] *= sc;
+        mx = mn;
+        const int nt = imin(32, nx - x0);
+        for (int jj = 0; jj < nt; ++jj) {
+          const float pj = __shfl_sync(0xffffffffu, p, jj);
+          const long long vr = xrow[x0 + jj];
+#pragma unroll
+          for (int u = 0; u < DL; ++u) o[u] = fmaf(pj, ld<T>(V + vr * D + lane + 32 * u), o[u]);
+        }
+      }
+      if (nretr > kXL) {  // retrieved keys past the list, one at a time
+        int idx = 0;
+        for (int r = 0; r < k1; ++r) {
+          const int j = s1[r];
+          if (j < 0) break;
+          const int* kb = c.kboff + ((size_t)kpid * Ck + j) * (NB + 1);
+          for (int r2 = 0; r2 < k2; ++r2) {
+            const int bb = s2[r * k2 + r2];
+            if (bb < 0) break;
+            for (int mm = kb[bb]; mm < kb[bb + 1]; ++mm, ++idx) {
+              if (idx < kXL) continue;
+              const long long krow = pk.row0 + kperm[koff[j] + mm];
+              float x = 0.f;
+#pragma unroll
+              for (int u = 0; u < DL; ++u)
+                x = fmaf(qw[lane + 32 * u], ld<T>(K + krow * D + lane + 32 * u), x);
+#pragma unroll
+              for (int o2 = 16; o2; o2 >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o2);
+              const float lg = s * x;
+              const float mn = fmaxf(mx, lg);
+              const float sc = __expf(mx - mn), w = __expf(lg - mn);
+              l = l * sc + w;
+#pragma unroll
+              for (int u = 0; u < DL; ++u)
+                o[u] = fmaf(o[u], sc, w * ld<T>(V + krow * D + lane + 32 * u));
+              mx = mn;
+            }
+          }
+        }
+      }
+      float* pp = a.part + (size_t)qrow * (D + 1);
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int u = 0; u < DL; ++u) pp[lane + 32 * u] = o[u] * inv;
+      if (lane == 0) {
+        pp[D] = mx + logf(l);
+        if (a.n_exact != nullptr) a.n_exact[qrow] = nretr;
+      }
+      __syncwarp();
     }
   }
 }
@@ -509,19 +690,20 @@ void launch_accum(const AttnArgs& a, const AccArgs& c, cudaStream_t st) {
   }
   {
     ProfScope ps(st, "accum_stage2");
-    const size_t sm = ((size_t)2 * a.Ck * D + a.Ck + D) * 4 + (size_t)a.Ck * 4;
+    const size_t sm = stage2_smem<D>(a.Ck, a.topk);
     auto kern = dip ? acc_stage2_kernel<T, D, true> : acc_stage2_kernel<T, D, false>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    kern<<<dim3(nq, c.NB, a.Cq), kAT, sm, st>>>(a, c);
+    kern<<<dim3(nq, c.NB, cdiv(a.Cq, kCI)), kST, sm, st>>>(a, c);
   }
 }
 
 }  // namespace
 
-bool accum_supported(int D, int Cq, int Ck, int NB, int k2, int mode) {
+bool accum_supported(int D, int Cq, int Ck, int NB, int k1, int k2, int mode) {
   if (mode != 0 && mode != 1) return false;
   if (D != 64 && D != 128) return false;
-  if (Cq > 256 || Ck > 256 || Ck * D > 16384) return false;
+  if (Cq > 256 || Ck > 256 || Ck * D > 16384 || k1 > 32) return false;
+  if ((D == 64 ? stage2_smem<64>(Ck, k1) : stage2_smem<128>(Ck, k1)) > 227 * 1024) return false;
   if (mode == 1 && Cq * D > kAT * 32) return false;  // acc_block_a: 32 outputs per thread
   if (NB < 1 || NB > 1024 || k2 < 0 || k2 > NB) return false;
   return true;

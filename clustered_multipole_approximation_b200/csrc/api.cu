@@ -417,6 +417,8 @@ AccLayout accum_layout(const muse_shape* sh, const muse_params* pr, int k2, cons
   c.pn = cv.take<int>(nk * NB * Ck * 4);
   c.bk = cv.take<double>(nk * NB * Ck * D * 8);
   c.pk = cv.take<double>(nk * NB * Ck * D * 8);
+  c.bmu = cv.take<double>(nk * NB * Ck * D * 8);
+  c.pmu = cv.take<double>(nk * NB * Ck * D * 8);
   c.bs = cv.take<float>(nk * NB * Ck * D * 4);
   c.ps = cv.take<float>(nk * NB * Ck * D * 4);
   const bool dip = pr->mode == MUSE_DIPOLE;
@@ -434,10 +436,10 @@ muse_status validate_accum(const muse_shape* sh, const muse_params* pr, int k2) 
   if (pr->block < 1 || sh->N % pr->block) return fail(MUSE_ERR_INVALID_ARG, "block must divide N");
   if (k2 < 0 || k2 > sh->N / pr->block)
     return fail(MUSE_ERR_INVALID_ARG, "topk2 must be in [0, N / block]");
-  if (!accum_supported(sh->D, pr->Cq, pr->Ck, sh->N / pr->block, k2, (int)pr->mode))
+  if (!accum_supported(sh->D, pr->Cq, pr->Ck, sh->N / pr->block, pr->topk, k2, (int)pr->mode))
     return fail(MUSE_ERR_UNSUPPORTED,
                 "block accumulation needs MONOPOLE or DIPOLE, Cq, Ck <= 256, Ck * D <= 16384, "
-                "N / block <= 1024 (DIPOLE: Cq * D <= 8192)");
+                "topk <= 32, N / block <= 1024 (DIPOLE: Cq * D <= 8192)");
   return MUSE_OK;
 }
 

@@ -155,6 +155,8 @@ struct AccArgs {
   int* pn;         // [key sets][NB][Ck] exclusive prefix over blocks
   double* bk;      // [key sets][NB][Ck][D] key sums (token order)
   double* pk;      // prefix of bk (block order)
+  double* bmu;     // [key sets][NB][D][Ck] bk / bn (fp64 division), dimension-major
+  double* pmu;     // [key sets][NB][D][Ck] pk / pn, dimension-major
   float* bs;       // [key sets][NB][Ck][D] value sums
   float* ps;       // prefix of bs
   float* ba;       // [query sets][NB][Cq][Ck][D] sum v (k . nu_i) (DIPOLE)
@@ -162,7 +164,7 @@ struct AccArgs {
   int* sel1;       // [query sets][NB][Cq][k1] selected key clusters, -1 padded
   int* sel2;       // [query sets][NB][Cq][k1][k2] selected blocks, -1 padded
 };
-bool accum_supported(int D, int Cq, int Ck, int NB, int k2, int mode);
+bool accum_supported(int D, int Cq, int Ck, int NB, int k1, int k2, int mode);
 void run_accum(const AttnArgs& a, const AccArgs& c, cudaStream_t st);
 
 // Causal: exact local block + merge of the level partials into O.

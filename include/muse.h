@@ -249,8 +249,9 @@ muse_status muse_attn_fwd_causal(const void *Q, const void *K, const void *V,
  *     retrieved blocks) as one far term: logit s q.mu + log n, value S / n
  *     (MONOPOLE) or (S + s M nu_i) / n (DIPOLE, M about that set's centroid).
  * All terms meet in one softmax.  topk2 == 0 retrieves nothing.  Supported:
- * MONOPOLE and DIPOLE, Cq, Ck <= 256, Ck * D <= 16384, N / L <= 1024, and
- * for DIPOLE Cq * D <= 8192 (MUSE_ERR_UNSUPPORTED otherwise).
+ * MONOPOLE and DIPOLE, Cq, Ck <= 256, Ck * D <= 16384, topk <= 32,
+ * N / L <= 1024, and for DIPOLE Cq * D <= 8192 (MUSE_ERR_UNSUPPORTED
+ * otherwise).
  * Debug layouts: q_assign [B,Hq,N], k_assign [B,Hkv,N],
  * sel1 [B,Hq,NB,Cq,topk], sel2 [B,Hq,NB,Cq,topk,topk2] (-1 padded; rows of
  * block 0 and of clusters with no query in the block are -1),

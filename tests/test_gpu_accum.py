@@ -97,6 +97,15 @@ def test_accum_retrieval_budgets(k1, k2):
     check_accum(Q, K, V, "bf16", 128, 16, 16, 4, 9, k1, k2, 1.0, "dipole")
 
 
+def test_accum_many_retrieved_keys():
+    # 4 clusters over blocks of 1024: each retrieved (cluster, block) pair
+    # holds ~256 keys, so a query cluster retrieves more keys than the
+    # stage-2 kernel lists in shared memory at once
+    Q, K, V = clustered_qkv(1, 1, 1, 4096, 64, 4, 0.3, 0.0, "bf16", 148)
+    _, g, _ = check_accum(Q, K, V, "bf16", 1024, 4, 4, 3, 7, 4, 2, 1.0, "dipole")
+    assert g["n_exact"].max() > 1024 + 1024
+
+
 def test_accum_never_reads_the_future_on_gpu():
     """Changing the values after position t0 changes no output up to t0 (the
     clusterings read only keys and queries, so they stay as they were)."""
