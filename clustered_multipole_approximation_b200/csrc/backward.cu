@@ -150,22 +150,56 @@ __global__ void __launch_bounds__(kBT) bwd_u_table_kernel(AttnArgs a, BwdArgs b)
 
 // ---------------------------------------------------------------------------
 // per (query set, query cluster): the softmax's own gradient
+//
+// The exact tiles (32 queries x 32 keys) are register-blocked: for S = Q K^T
+// and G = dO V^T every thread owns a 2 x 2 block (queries 2tq, 2tq+1; keys
+// tk, tk+16, so a quarter warp's 16-byte row reads hit distinct banks); for
+// dQ += dS K, dK = dS^T Q and dV = P^T dO every thread owns 2 rows x D/16
+// columns.
 // ---------------------------------------------------------------------------
 template <int D>
 struct QuerySmem {
-  float q[kQC][D + 1];
-  float go[kQC][D + 1];  // dO
-  float kt[kKC][D + 1];
-  float vt[kKC][D + 1];
-  float pt[kQC][kKC];
-  float dst[kQC][kKC];
+  float q[kQC][D + 4];
+  float go[kQC][D + 4];  // dO
+  float kt[kKC][D + 4];
+  float vt[kKC][D + 4];
+  float pt[kQC][kKC + 1];
+  float dst[kQC][kKC + 1];
   float lse[kQC];
   float dq_[kQC];  // D_q
-  float dex[kQC];  // exact terms' sum of exp(l - m) g, at the running max m
-  float mq[kQC];   // running max
+  float ml[kQC][2];  // running max and sum of the far terms, per query
+  float dex[kQC];  // exact terms' sum of exp(l - m) g at the running max m
+  float mq[kQC];   // running max after the exact terms
   int row[kQC];
   unsigned rmask[kMaxC / 32];
 };
+
+// s * q.k and dO.v for the thread's 2 x 2 block of the staged tile
+template <int D>
+__device__ inline void tile_sg(const QuerySmem<D>& sm, int tq, int tk, float sx[2][2], float gx[2][2]) {
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) sx[a][c] = gx[a][c] = 0.f;
+#pragma unroll 4
+  for (int d = 0; d < D; d += 4) {
+    float4 qv[2], gv[2], kv[2], vv[2];
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      qv[a] = *reinterpret_cast<const float4*>(&sm.q[2 * tq + a][d]);
+      gv[a] = *reinterpret_cast<const float4*>(&sm.go[2 * tq + a][d]);
+      kv[a] = *reinterpret_cast<const float4*>(&sm.kt[tk + 16 * a][d]);
+      vv[a] = *reinterpret_cast<const float4*>(&sm.vt[tk + 16 * a][d]);
+    }
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        sx[a][c] = fmaf(qv[a].x, kv[c].x, fmaf(qv[a].y, kv[c].y, fmaf(qv[a].z, kv[c].z, fmaf(qv[a].w, kv[c].w, sx[a][c]))));
+        gx[a][c] = fmaf(gv[a].x, vv[c].x, fmaf(gv[a].y, vv[c].y, fmaf(gv[a].z, vv[c].z, fmaf(gv[a].w, vv[c].w, gx[a][c]))));
+      }
+  }
+}
 
 template <typename T, typename TO, int D, bool DIP>
 __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, BwdArgs b) {
@@ -197,7 +231,8 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
   const T* V = static_cast<const T*>(a.V);
   const TO* GO = static_cast<const TO*>(b.dO);
   const float s = a.scale;
-  constexpr int DL = D / 32;  // elements per lane
+  constexpr int DV = D / 16;  // columns per thread in the dQ / dK / dV blocks
+  const int tq = tid >> 4, tk = tid & 15;  // 2 x 2 blocks of S and G; 2 rows x DV columns
 
   // retrieval set, far / exact cluster lists, centroid table
   for (int w = tid; w < kMaxC / 32; w += kBT) sm.rmask[w] = 0u;
@@ -227,30 +262,40 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
   __syncthreads();
   const int nf = nfar, nx = nex;
 
+  // stage one tile of retrieved keys (and values) into shared memory
+  auto load_tile = [&](int o0, int kc, bool with_v) {
+    for (int e = tid; e < kKC * D; e += kBT) {
+      const int r = e / D, d = e - r * D;
+      float kx = 0.f, vx = 0.f;
+      if (r < kc) {
+        const long long row = pk.row0 + kperm[o0 + r];
+        kx = ldg_<T>(K + row * D + d);
+        if (with_v) vx = ldg_<T>(V + row * D + d);
+      }
+      sm.kt[r][d] = kx;
+      sm.vt[r][d] = vx;
+    }
+  };
+
   for (int c0 = 0; c0 < mi; c0 += kQC) {
     const int qc = imin(kQC, mi - c0);
-    // ---- chunk rows: q, dO, D_q ------------------------------------------
+    // ---- chunk rows: q, dO (rows past qc are zero) --------------------------
     __syncthreads();
-    if (tid < qc) sm.row[tid] = (int)(pq.row0 + qperm[qoff + c0 + tid]);
+    if (tid < kQC) sm.row[tid] = tid < qc ? (int)(pq.row0 + qperm[qoff + c0 + tid]) : -1;
     __syncthreads();
-    for (int e = tid; e < qc * D; e += kBT) {
+    for (int e = tid; e < kQC * D; e += kBT) {
       const int r = e / D, d = e - r * D;
       const long long row = sm.row[r];
-      sm.q[r][d] = ldg_<T>(Q + row * D + d);
-      sm.go[r][d] = ldg_<TO>(GO + row * D + d);
+      sm.q[r][d] = row >= 0 ? ldg_<T>(Q + row * D + d) : 0.f;
+      sm.go[r][d] = row >= 0 ? ldg_<TO>(GO + row * D + d) : 0.f;
+    }
+    if (tid >= qc && tid < kQC) {  // rows past the chunk: no far terms
+      sm.ml[tid][0] = -INFINITY;
+      sm.ml[tid][1] = 0.f;
     }
     __syncthreads();
-    // ---- far logits and the running max / sum per query -------------------
-    float mrun[kQC / kBW], lrun[kQC / kBW];
-#pragma unroll
-    for (int u = 0; u < kQC / kBW; ++u) {
-      mrun[u] = -INFINITY;
-      lrun[u] = 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < kQC / kBW; ++u) {
-      const int r = warp + kBW * u;
-      if (r >= qc) continue;
+    // ---- far logits and their running max / sum (one warp per query) ------
+    for (int r = warp; r < qc; r += kBW) {
       float mx = -INFINITY;
       for (int jj = lane; jj < nf; jj += 32) {
         const int j = fl[jj];
@@ -267,73 +312,68 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
       for (int jj = lane; jj < nf; jj += 32) sum += __expf(lf[r * Ck + jj] - mx);
 #pragma unroll
       for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      mrun[u] = mx;
-      lrun[u] = nf > 0 ? sum : 0.f;
+      if (lane == 0) {
+        sm.ml[r][0] = mx;
+        sm.ml[r][1] = nf > 0 ? sum : 0.f;
+      }
     }
-    // ---- exact terms: finish the running max / sum, and their sum of p g --
-    float arun[kQC / kBW];
+    __syncthreads();
+    // ---- exact terms: finish the running max / sum, and their sum of p g ---
+    // (the 16 threads of a query pair hold identical running values)
+    float mrun[2], lrun[2], arun[2];
 #pragma unroll
-    for (int u = 0; u < kQC / kBW; ++u) arun[u] = 0.f;
+    for (int a2 = 0; a2 < 2; ++a2) {
+      mrun[a2] = sm.ml[2 * tq + a2][0];
+      lrun[a2] = sm.ml[2 * tq + a2][1];
+      arun[a2] = 0.f;
+    }
     for (int xi = 0; xi < nx; ++xi) {
       const int j = xl[xi], nj = kcnt[j], o0 = koff[j];
       for (int t0 = 0; t0 < nj; t0 += kKC) {
         const int kc = imin(kKC, nj - t0);
         __syncthreads();
-        for (int e = tid; e < kc * D; e += kBT) {
-          const int r = e / D, d = e - r * D;
-          const long long row = pk.row0 + kperm[o0 + t0 + r];
-          sm.kt[r][d] = ldg_<T>(K + row * D + d);
-          sm.vt[r][d] = ldg_<T>(V + row * D + d);
-        }
+        load_tile(o0 + t0, kc, true);
         __syncthreads();
+        float sx[2][2], gx[2][2];
+        tile_sg<D>(sm, tq, tk, sx, gx);
 #pragma unroll
-        for (int u = 0; u < kQC / kBW; ++u) {
-          const int r = warp + kBW * u;
-          if (r >= qc) continue;
-          float l = -INFINITY, g = 0.f;
-          if (lane < kc) {
-            float x = 0.f;
-#pragma unroll 8
-            for (int d = 0; d < D; ++d) {
-              x = fmaf(sm.q[r][d], sm.kt[lane][d], x);
-              g = fmaf(sm.go[r][d], sm.vt[lane][d], g);
-            }
-            l = s * x;
-          }
-          float mx = l;
+        for (int a2 = 0; a2 < 2; ++a2) {
+          float l0 = tk < kc ? s * sx[a2][0] : -INFINITY;
+          float l1 = tk + 16 < kc ? s * sx[a2][1] : -INFINITY;
+          float mx = fmaxf(l0, l1);
 #pragma unroll
-          for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          const float mn = fmaxf(mrun[u], mx);
-          float p = lane < kc ? __expf(l - mn) : 0.f;
-          float pg = p * g;
+          for (int o = 8; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float mn = fmaxf(mrun[a2], mx);
+          const float p0 = __expf(l0 - mn), p1 = __expf(l1 - mn);
+          float p = p0 + p1, pg = p0 * gx[a2][0] + p1 * gx[a2][1];
 #pragma unroll
-          for (int o = 16; o; o >>= 1) {
+          for (int o = 8; o; o >>= 1) {
             p += __shfl_xor_sync(0xffffffffu, p, o);
             pg += __shfl_xor_sync(0xffffffffu, pg, o);
           }
-          const float sc = __expf(mrun[u] - mn);
-          lrun[u] = lrun[u] * sc + p;
-          arun[u] = arun[u] * sc + pg;
-          mrun[u] = mn;
+          const float sc = __expf(mrun[a2] - mn);
+          lrun[a2] = lrun[a2] * sc + p;
+          arun[a2] = arun[a2] * sc + pg;
+          mrun[a2] = mn;
         }
       }
     }
+    if (tk == 0) {
 #pragma unroll
-    for (int u = 0; u < kQC / kBW; ++u) {
-      const int r = warp + kBW * u;
-      if (r < qc && lane == 0) {
-        sm.lse[r] = mrun[u] + __logf(lrun[u]);
-        sm.mq[r] = mrun[u];
-        sm.dex[r] = arun[u];
+      for (int a2 = 0; a2 < 2; ++a2) {
+        const int r = 2 * tq + a2;
+        sm.lse[r] = mrun[a2] + __logf(lrun[a2]);
+        sm.mq[r] = mrun[a2];
+        sm.dex[r] = arun[a2];
       }
     }
     // ---- far terms' g = dO_q . u_ij: one warp per far cluster -------------
     for (int jj = warp; jj < nf; jj += kBW) {
       const int j = fl[jj];
-      float ux[DL];
+      float ux[D / 32];
       const float invn = 1.f / (float)kcnt[j];
 #pragma unroll
-      for (int u = 0; u < DL; ++u) {
+      for (int u = 0; u < D / 32; ++u) {
         const int d = lane + 32 * u;
         ux[u] = DIP ? b.U[(((size_t)qpid * Cq + i) * Ck + j) * D + d]
                     : b.Sst[((size_t)kpid * Ck + j) * D + d] * invn;
@@ -341,7 +381,7 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
       for (int r = 0; r < qc; ++r) {
         float g = 0.f;
 #pragma unroll
-        for (int u = 0; u < DL; ++u) g = fmaf(sm.go[r][lane + 32 * u], ux[u], g);
+        for (int u = 0; u < D / 32; ++u) g = fmaf(sm.go[r][lane + 32 * u], ux[u], g);
 #pragma unroll
         for (int o = 16; o; o >>= 1) g += __shfl_xor_sync(0xffffffffu, g, o);
         if (lane == 0) gf[r * Ck + jj] = g;
@@ -349,30 +389,27 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
     }
     __syncthreads();
     // D_q = sum over the terms of p g
-#pragma unroll
-    for (int u = 0; u < kQC / kBW; ++u) {
-      const int r = warp + kBW * u;
-      if (r >= qc) continue;
+    for (int r = warp; r < qc; r += kBW) {
       const float m = sm.mq[r];
-      float a = 0.f;
-      for (int jj = lane; jj < nf; jj += 32) a = fmaf(__expf(lf[r * Ck + jj] - m), gf[r * Ck + jj], a);
+      float acc = 0.f;
+      for (int jj = lane; jj < nf; jj += 32) acc = fmaf(__expf(lf[r * Ck + jj] - m), gf[r * Ck + jj], acc);
 #pragma unroll
-      for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (lane == 0) sm.dq_[r] = (a + sm.dex[r]) * __expf(m - sm.lse[r]);
+      for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) sm.dq_[r] = (acc + sm.dex[r]) * __expf(m - sm.lse[r]);
     }
     __syncthreads();
 
     // ---- far terms: one warp per far cluster ------------------------------
     for (int jj = warp; jj < nf; jj += kBW) {
       const int j = fl[jj];
-      float gu[DL], gm[DL];
+      float gu[D / 32], gm[D / 32];
 #pragma unroll
-      for (int u = 0; u < DL; ++u) gu[u] = gm[u] = 0.f;
+      for (int u = 0; u < D / 32; ++u) gu[u] = gm[u] = 0.f;
       for (int r = 0; r < qc; ++r) {
         const float p = __expf(lf[r * Ck + jj] - sm.lse[r]);
         const float dl = p * (gf[r * Ck + jj] - sm.dq_[r]);
 #pragma unroll
-        for (int u = 0; u < DL; ++u) {
+        for (int u = 0; u < D / 32; ++u) {
           gu[u] = fmaf(p, sm.go[r][lane + 32 * u], gu[u]);
           gm[u] = fmaf(s * dl, sm.q[r][lane + 32 * u], gm[u]);
         }
@@ -382,95 +419,131 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
       float* du = b.dU + (((size_t)qpid * Cq + i) * Ck + j) * D;
       float* dm = b.dmu + ((size_t)kpid * Ck + j) * D;
 #pragma unroll
-      for (int u = 0; u < DL; ++u) {
+      for (int u = 0; u < D / 32; ++u) {
         const int d = lane + 32 * u;
         du[d] += gu[u];  // this CTA owns the row (query set, i, j)
         atomicAdd(dm + d, gm[u]);
       }
     }
     __syncthreads();
-    // dq = sum_j (s dl_qj) mu_j
-    float dq[kQC / kBW][DL];
+    // dq = sum_j (s dl_qj) mu_j: the thread's 2 rows x DV columns
+    float dq[2][DV];
 #pragma unroll
-    for (int u = 0; u < kQC / kBW; ++u) {
-      const int r = warp + kBW * u;
+    for (int a2 = 0; a2 < 2; ++a2)
 #pragma unroll
-      for (int v = 0; v < DL; ++v) dq[u][v] = 0.f;
-      if (r >= qc) continue;
+      for (int v = 0; v < DV; ++v) dq[a2][v] = 0.f;
+    {
+      const int r0 = 2 * tq;
       for (int jj = 0; jj < nf; ++jj) {
-        const float c = lf[r * Ck + jj];
-        const float* m = mu_s + fl[jj] * (D + 1);
+        const float c0_ = r0 < qc ? lf[r0 * Ck + jj] : 0.f;
+        const float c1_ = r0 + 1 < qc ? lf[(r0 + 1) * Ck + jj] : 0.f;
+        const float* m = mu_s + fl[jj] * (D + 1) + tk * DV;
 #pragma unroll
-        for (int v = 0; v < DL; ++v) dq[u][v] = fmaf(c, m[lane + 32 * v], dq[u][v]);
+        for (int v = 0; v < DV; ++v) {
+          dq[0][v] = fmaf(c0_, m[v], dq[0][v]);
+          dq[1][v] = fmaf(c1_, m[v], dq[1][v]);
+        }
       }
     }
-    // ---- exact tiles ------------------------------------------------------
-    float* dK = b.dK;
-    float* dV = b.dV;
+    // ---- exact tiles --------------------------------------------------------
     for (int xi = 0; xi < nx; ++xi) {
       const int j = xl[xi], nj = kcnt[j], o0 = koff[j];
       for (int t0 = 0; t0 < nj; t0 += kKC) {
         const int kc = imin(kKC, nj - t0);
         __syncthreads();
-        for (int e = tid; e < kc * D; e += kBT) {
-          const int r = e / D, d = e - r * D;
-          const long long row = pk.row0 + kperm[o0 + t0 + r];
-          sm.kt[r][d] = ldg_<T>(K + row * D + d);
-          sm.vt[r][d] = ldg_<T>(V + row * D + d);
-        }
+        load_tile(o0 + t0, kc, true);
         __syncthreads();
+        {
+          float sx[2][2], gx[2][2];
+          tile_sg<D>(sm, tq, tk, sx, gx);
 #pragma unroll
-        for (int u = 0; u < kQC / kBW; ++u) {
-          const int r = warp + kBW * u;
-          if (r >= qc) continue;
-          float p = 0.f, ds = 0.f;
-          if (lane < kc) {
-            float x = 0.f, g = 0.f;
-#pragma unroll 8
-            for (int d = 0; d < D; ++d) {
-              x = fmaf(sm.q[r][d], sm.kt[lane][d], x);
-              g = fmaf(sm.go[r][d], sm.vt[lane][d], g);
+          for (int a2 = 0; a2 < 2; ++a2) {
+            const int r = 2 * tq + a2;
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+              const int t = tk + 16 * c2;
+              float p = 0.f, ds = 0.f;
+              if (r < qc && t < kc) {
+                p = __expf(s * sx[a2][c2] - sm.lse[r]);
+                ds = p * (gx[a2][c2] - sm.dq_[r]);
+              }
+              sm.pt[r][t] = p;
+              sm.dst[r][t] = s * ds;
             }
-            p = __expf(s * x - sm.lse[r]);
-            ds = p * (g - sm.dq_[r]);
-          }
-          sm.pt[r][lane] = p;
-          sm.dst[r][lane] = ds;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int u = 0; u < kQC / kBW; ++u) {
-          const int r = warp + kBW * u;
-          if (r >= qc) continue;
-          for (int t = 0; t < kc; ++t) {
-            const float c = s * sm.dst[r][t];
-#pragma unroll
-            for (int v = 0; v < DL; ++v) dq[u][v] = fmaf(c, sm.kt[t][lane + 32 * v], dq[u][v]);
           }
         }
-        for (int t = warp; t < kc; t += kBW) {
-          const long long row = pk.row0 + kperm[o0 + t0 + t];
+        __syncthreads();
+        // dq += (s dS) K over the tile's keys
+#pragma unroll 4
+        for (int t = 0; t < kKC; ++t) {
+          const float c0_ = sm.dst[2 * tq][t], c1_ = sm.dst[2 * tq + 1][t];
 #pragma unroll
-          for (int v = 0; v < DL; ++v) {
-            const int d = lane + 32 * v;
-            float gk = 0.f, gv = 0.f;
-            for (int r = 0; r < qc; ++r) {
-              gk = fmaf(sm.dst[r][t], sm.q[r][d], gk);
-              gv = fmaf(sm.pt[r][t], sm.go[r][d], gv);
+          for (int v = 0; v < DV; v += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(&sm.kt[t][tk * DV + v]);
+            dq[0][v] = fmaf(c0_, k4.x, dq[0][v]);
+            dq[0][v + 1] = fmaf(c0_, k4.y, dq[0][v + 1]);
+            dq[0][v + 2] = fmaf(c0_, k4.z, dq[0][v + 2]);
+            dq[0][v + 3] = fmaf(c0_, k4.w, dq[0][v + 3]);
+            dq[1][v] = fmaf(c1_, k4.x, dq[1][v]);
+            dq[1][v + 1] = fmaf(c1_, k4.y, dq[1][v + 1]);
+            dq[1][v + 2] = fmaf(c1_, k4.z, dq[1][v + 2]);
+            dq[1][v + 3] = fmaf(c1_, k4.w, dq[1][v + 3]);
+          }
+        }
+        // dK = (s dS)^T Q and dV = P^T dO for the thread's 2 keys x DV columns
+        {
+          float gk[2][DV], gv[2][DV];
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+            for (int v = 0; v < DV; ++v) gk[c2][v] = gv[c2][v] = 0.f;
+#pragma unroll 4
+          for (int r = 0; r < kQC; ++r) {
+            const float d0 = sm.dst[r][2 * tq], d1 = sm.dst[r][2 * tq + 1];
+            const float p0 = sm.pt[r][2 * tq], p1 = sm.pt[r][2 * tq + 1];
+#pragma unroll
+            for (int v = 0; v < DV; v += 4) {
+              const float4 q4 = *reinterpret_cast<const float4*>(&sm.q[r][tk * DV + v]);
+              const float4 g4 = *reinterpret_cast<const float4*>(&sm.go[r][tk * DV + v]);
+              gk[0][v] = fmaf(d0, q4.x, gk[0][v]);
+              gk[0][v + 1] = fmaf(d0, q4.y, gk[0][v + 1]);
+              gk[0][v + 2] = fmaf(d0, q4.z, gk[0][v + 2]);
+              gk[0][v + 3] = fmaf(d0, q4.w, gk[0][v + 3]);
+              gk[1][v] = fmaf(d1, q4.x, gk[1][v]);
+              gk[1][v + 1] = fmaf(d1, q4.y, gk[1][v + 1]);
+              gk[1][v + 2] = fmaf(d1, q4.z, gk[1][v + 2]);
+              gk[1][v + 3] = fmaf(d1, q4.w, gk[1][v + 3]);
+              gv[0][v] = fmaf(p0, g4.x, gv[0][v]);
+              gv[0][v + 1] = fmaf(p0, g4.y, gv[0][v + 1]);
+              gv[0][v + 2] = fmaf(p0, g4.z, gv[0][v + 2]);
+              gv[0][v + 3] = fmaf(p0, g4.w, gv[0][v + 3]);
+              gv[1][v] = fmaf(p1, g4.x, gv[1][v]);
+              gv[1][v + 1] = fmaf(p1, g4.y, gv[1][v + 1]);
+              gv[1][v + 2] = fmaf(p1, g4.z, gv[1][v + 2]);
+              gv[1][v + 3] = fmaf(p1, g4.w, gv[1][v + 3]);
             }
-            atomicAdd(dK + row * D + d, s * gk);
-            atomicAdd(dV + row * D + d, gv);
+          }
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int t = 2 * tq + c2;
+            if (t >= kc) continue;
+            const long long row = pk.row0 + kperm[o0 + t0 + t];
+#pragma unroll
+            for (int v = 0; v < DV; ++v) {
+              atomicAdd(b.dK + row * D + tk * DV + v, gk[c2][v]);
+              atomicAdd(b.dV + row * D + tk * DV + v, gv[c2][v]);
+            }
           }
         }
       }
     }
     // ---- this chunk's dq (the centroid term is added later) ---------------
 #pragma unroll
-    for (int u = 0; u < kQC / kBW; ++u) {
-      const int r = warp + kBW * u;
+    for (int a2 = 0; a2 < 2; ++a2) {
+      const int r = 2 * tq + a2;
       if (r >= qc) continue;
 #pragma unroll
-      for (int v = 0; v < DL; ++v) b.dQ[(long long)sm.row[r] * D + lane + 32 * v] = dq[u][v];
+      for (int v = 0; v < DV; ++v) b.dQ[(long long)sm.row[r] * D + tk * DV + v] = dq[a2][v];
     }
   }
 }
