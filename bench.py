@@ -575,6 +575,8 @@ def run_accum_bench(w, mode, steps, warmup, device, k1=ACCUM_K1, k2=ACCUM_K2):
                for n, (c, t) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
     del q, k, v, out, ws, flush
     torch.cuda.empty_cache()
+    if not np.isfinite(num / den):
+        raise RuntimeError("non-finite output from the block-accumulation form")
     cfg = dict(config_of(w, mode), topk=k1, topk2=k2, form="block-summary accumulation")
     return {"config": cfg, "value": w.B * w.N / (ms / 1e3), "unit": UNIT, "ms_per_call": ms,
             "steps": steps, "warmup": warmup, "rse_vs_exact": num / den, "kernels": kernels}

@@ -375,7 +375,14 @@ __global__ void __launch_bounds__(kST) acc_stage2_kernel(AttnArgs a, AccArgs c) 
     const size_t o = ((size_t)kpid * NB + b) * Ck + j;
     const int n = c.pn[o];
     if (lane == 0) ln_s[j] = n > 0 ? logf((float)n) : -INFINITY;
-    if (n == 0) continue;
+    if (n == 0) {  // no prefix member: a zero row, never weighted
+#pragma unroll
+      for (int u = 0; u < DL; ++u) {
+        mu_s[j * (D + 1) + lane + 32 * u] = 0.f;
+        u_s[j * D + lane + 32 * u] = 0.f;
+      }
+      continue;
+    }
 #pragma unroll
     for (int u = 0; u < DL; ++u) {
       const int d = lane + 32 * u;
@@ -563,7 +570,8 @@ __global__ void __launch_bounds__(kST) acc_stage2_kernel(AttnArgs a, AccArgs c) 
         __syncwarp();
 #pragma unroll 8
         for (int jj = 0; jj < 32; ++jj) {
-          const float pj = pw[jj];  // 0 for an empty or absent cluster (its row is unused)
+          const float pj = pw[jj];
+          if (pj == 0.f) continue;  // an empty or absent cluster: its row is not read
           const float* ur = uw[jj];
 #pragma unroll
           for (int u = 0; u < DL; ++u) o[u] = fmaf(pj, ur[lane + 32 * u], o[u]);

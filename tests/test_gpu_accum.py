@@ -97,6 +97,15 @@ def test_accum_retrieval_budgets(k1, k2):
     check_accum(Q, K, V, "bf16", 128, 16, 16, 4, 9, k1, k2, 1.0, "dipole")
 
 
+@pytest.mark.parametrize("mode", ["monopole", "dipole"])
+def test_accum_clusters_with_empty_prefixes(mode):
+    # 64 key clusters and blocks of 64: the first blocks' prefixes leave most
+    # key clusters without a member
+    Q, K, V = clustered_qkv(1, 2, 1, 1024, 64, 16, 0.4, 0.0, "bf16", 149)
+    O, _, _ = check_accum(Q, K, V, "bf16", 64, 32, 64, 4, 11, 2, 1, 1.0, mode)
+    assert np.isfinite(O).all()
+
+
 def test_accum_many_retrieved_keys():
     # 4 clusters over blocks of 1024: each retrieved (cluster, block) pair
     # holds ~256 keys, so a query cluster retrieves more keys than the
