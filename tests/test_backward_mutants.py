@@ -23,6 +23,8 @@ MUTANTS = {
     "far-logit-drops-log-n": (" + torch.log(n.clamp(min=1.0))[None]", ""),
     "exact-values-are-keys": ("P[:, Ck:] @ v", "P[:, Ck:] @ k"),
     "selected-clusters-also-far": ("far_ok = (~R) & (n > 0)[None, :]", "far_ok = (n > 0)[None, :].expand(Cq, -1)"),
+    "causal-local-block-reads-ahead": ("torch.where(kl <= pos[:, None],", "torch.where(kl >= 0,"),
+    "causal-level-reads-the-query-block": ("k[k0:k0 + s], v[k0:k0 + s],", "k[q0:q0 + s], v[q0:q0 + s],"),
 }
 
 

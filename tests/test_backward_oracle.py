@@ -12,6 +12,9 @@ fixed, the same operator the C oracle evaluates.  It is pinned by:
     leaves O unchanged (so the key gradient sums to zero over the tokens of a
     key set), and translating every value by c moves O by c (so the value
     gradient sums to the sum of dO over the queries reading that key set);
+  * the same three for the causal operator (finite differences of the C
+    oracle's causal forward; singleton key clusters at every level against the
+    causal closed form; the translation invariants);
   * the mutants of test_backward_mutants.py, each caught by one of these.
 """
 import numpy as np
@@ -104,7 +107,78 @@ def pin_translation_invariants(mod, mode, seed=7, Cq=5, Ck=6, topk=2, scale=0.8)
         np.testing.assert_allclose(dV[0, hk].sum(0), want, rtol=0, atol=1e-10)
 
 
-PINS = (pin_finite_differences, pin_exact_special_cases, pin_translation_invariants)
+def causal_exact_grads(q, k, v, dO, scale):
+    """The closed form of exact_grads_closed_form with the causal mask."""
+    N = q.shape[0]
+    Sx = scale * q @ k.T
+    Sx[np.triu_indices(N, 1)] = -np.inf
+    P = np.exp(Sx - Sx.max(1, keepdims=True))
+    P /= P.sum(1, keepdims=True)
+    O = P @ v
+    dS = P * (dO @ v.T - (dO * O).sum(1, keepdims=True))
+    return O, scale * dS @ k, scale * dS.T @ q, P.T @ dO
+
+
+def pin_causal_finite_differences(mod, mode, seed=9, L=32, C=5, topk=2, scale=0.7, eps=1e-5):
+    Q, K, V, dO = small_case(seed, N=256)
+    r0 = oracle.muse_causal(Q, K, V, L, C, 4, 11, topk, scale, mode)
+    qa, ka, sel = r0["q_assign"], r0["k_assign"], r0.get("selected")
+    O, dQ, dK, dV = mod.muse_causal_grads(Q, K, V, dO, qa, ka, sel, L, C, scale, mode)
+    np.testing.assert_allclose(O, r0["O"], rtol=0, atol=1e-12)
+    rng = np.random.default_rng(seed + 100)
+    for which, g in (("Q", dQ), ("K", dK), ("V", dV)):
+        h = rng.standard_normal(g.shape)
+        X = {"Q": Q, "K": K, "V": V}
+
+        def f(sign):
+            Y = dict(X)
+            Y[which] = X[which] + sign * eps * h
+            r = oracle.muse_causal(Y["Q"], Y["K"], Y["V"], L, C, 4, 11, topk, scale, mode,
+                                   q_assign_in=qa, k_assign_in=ka)
+            if sel is not None:
+                assert (r["selected"] == sel).all(), "selection moved under the probe"
+            return float((r["O"] * dO).sum())
+
+        fd = (f(+1) - f(-1)) / (2 * eps)
+        an = float((g * h).sum())
+        assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (which, fd, an)
+
+
+def pin_causal_singletons_are_exact(mod, mode, L=16):
+    Q, K, V, dO = small_case(10, N=128, Hq=1)
+    N = 128
+    lv = oracle.causal_levels(N, L)
+    ka = np.zeros((1, 1, lv, N // 2), np.int32)
+    qa = np.zeros((1, 1, lv, N // 2), np.int32)
+    for l in range(lv):
+        s = L << l
+        ka[0, 0, l] = np.tile(np.arange(s), N // (2 * s))  # every key its own cluster
+    O, dQ, dK, dV = mod.muse_causal_grads(Q[:, :1], K, V, dO[:, :1], qa, ka, None, L, N, 0.9, mode)
+    Oe, dQe, dKe, dVe = causal_exact_grads(Q[0, 0], K[0, 0], V[0, 0], dO[0, 0], 0.9)
+    for a, b in ((O, Oe), (dQ, dQe), (dK, dKe), (dV, dVe)):
+        np.testing.assert_allclose(a[0, 0], b, rtol=0, atol=1e-10)
+
+
+def pin_causal_translation_invariants(mod, mode, L=32, C=6, topk=2, scale=0.8):
+    Q, K, V, dO = small_case(11, N=256, Hq=2, Hkv=2)
+    r = oracle.muse_causal(Q, K, V, L, C, 4, 11, topk, scale, mode)
+    _, _, dK, dV = mod.muse_causal_grads(Q, K, V, dO, r["q_assign"], r["k_assign"],
+                                         r.get("selected"), L, C, scale, mode)
+    for hk in range(2):
+        np.testing.assert_allclose(dK[0, hk].sum(0), 0.0, rtol=0, atol=1e-10)
+        np.testing.assert_allclose(dV[0, hk].sum(0), dO[0, hk].sum(0), rtol=0, atol=1e-10)
+
+
+PINS = (pin_finite_differences, pin_exact_special_cases, pin_translation_invariants,
+        pin_causal_finite_differences, pin_causal_singletons_are_exact,
+        pin_causal_translation_invariants)
+
+
+@pytest.mark.parametrize("mode", ["monopole", "dipole"])
+@pytest.mark.parametrize("pin", [pin_causal_finite_differences, pin_causal_singletons_are_exact,
+                                 pin_causal_translation_invariants], ids=lambda p: p.__name__)
+def test_causal_gradient_pin(pin, mode):
+    pin(mb, mode)
 
 
 @pytest.mark.parametrize("mode", ["monopole", "dipole"])
