@@ -65,7 +65,8 @@ EXPORTS = ["muse_workspace_size", "muse_cluster_workspace_size", "muse_cluster",
            "muse_profile_enable", "muse_profile_read", "muse_cluster_static",
            "muse_cluster_static_capacity", "muse_device_status", "muse_debug_inject_barrier_fault",
            "muse_attn_bwd_workspace_size", "muse_attn_bwd", "muse_accum_workspace_size",
-           "muse_attn_fwd_causal_accum"]
+           "muse_attn_fwd_causal_accum", "muse_attn_bwd_causal_workspace_size",
+           "muse_attn_bwd_causal"]
 
 # Bits of the device error word (include/muse.h MUSE_DEVERR_*).
 DEVERR = {1: "MUSE_DEVERR_MMA_WAIT", 2: "MUSE_DEVERR_TEAM_BARRIER", 4: "MUSE_DEVERR_V_RANGE"}
@@ -107,6 +108,10 @@ def load_library(path: str = LIB_PATH):
     lib.muse_attn_bwd_workspace_size.argtypes = [sp, pp]
     lib.muse_attn_bwd.restype = i32
     lib.muse_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, sp, pp, vp, sz, vp]
+    lib.muse_attn_bwd_causal_workspace_size.restype = sz
+    lib.muse_attn_bwd_causal_workspace_size.argtypes = [sp, pp]
+    lib.muse_attn_bwd_causal.restype = i32
+    lib.muse_attn_bwd_causal.argtypes = [vp, vp, vp, vp, vp, vp, vp, sp, pp, vp, sz, vp]
     lib.muse_status_string.restype = ctypes.c_char_p
     lib.muse_status_string.argtypes = [i32]
     lib.muse_last_error.restype = ctypes.c_char_p
@@ -308,11 +313,14 @@ def muse_attn_fwd_causal_accum(q, k, v, *, Cq, Ck, block, iters, seed, topk, top
     return (out, bufs) if debug else out
 
 
-def backward_workspace_size(q, k, params: muse_params, out_f32: bool = False) -> int:
-    """Workspace bytes for a muse_attn_fwd call followed by muse_attn_bwd."""
+def backward_workspace_size(q, k, params: muse_params, out_f32: bool = False,
+                            causal: bool = False) -> int:
+    """Workspace bytes for a forward call followed by its backward call
+    (muse_attn_fwd + muse_attn_bwd, or the causal pair)."""
     lib = load_library()
     sh = make_shape(q, k, out_f32)
-    n = lib.muse_attn_bwd_workspace_size(ctypes.byref(sh), ctypes.byref(params))
+    f = lib.muse_attn_bwd_causal_workspace_size if causal else lib.muse_attn_bwd_workspace_size
+    n = f(ctypes.byref(sh), ctypes.byref(params))
     if n == 0:
         raise MuseError(3, lib.muse_last_error().decode())
     return int(n)
@@ -335,6 +343,28 @@ def muse_attn_bwd(q, k, v, do, *, Cq, Ck, iters, seed, topk, scale=1.0, mode="di
     st = lib.muse_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
                            ctypes.byref(sh), ctypes.byref(p), _ptr(workspace),
                            workspace.numel(), _stream(stream))
+    _check(lib, st)
+    return dq, dk, dv
+
+
+def muse_attn_bwd_causal(q, k, v, do, *, C, block, iters, seed, topk, scale=1.0, mode="dipole",
+                         workspace, stream=None, key_stream0=0, query_stream0=0):
+    """Gradients (dq, dk, dv) in fp32 of <do, O> for the causal forward call
+    made with this `workspace` (sized by backward_workspace_size(...,
+    causal=True)) and these parameters; see muse_attn_bwd_causal in
+    include/muse.h."""
+    lib = load_library()
+    _need_cuda(q, k, v, do, workspace)
+    if do.shape != q.shape or do.dtype not in (q.dtype, torch.float32):
+        raise ValueError("do must be [B,Hq,N,D] in the input dtype or float32")
+    p = make_params(C, C, iters, seed, topk, block, scale, mode, key_stream0, query_stream0)
+    sh = make_shape(q, k, do.dtype == torch.float32 and q.dtype != torch.float32)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    st = lib.muse_attn_bwd_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), ctypes.byref(sh), ctypes.byref(p), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
     _check(lib, st)
     return dq, dk, dv
 

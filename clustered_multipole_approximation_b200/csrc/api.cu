@@ -359,7 +359,8 @@ struct BwdLayout {
   size_t bytes;
 };
 
-BwdLayout bwd_layout(const muse_shape* sh, const muse_params* pr, const AttnLayout& L, void* ws) {
+BwdLayout bwd_layout(const muse_shape* sh, const muse_params* pr, const AttnLayout& L, void* ws,
+                     bool causal = false) {
   BwdLayout r{};
   Carver cv{static_cast<char*>(ws)};
   cv.used = L.bytes;
@@ -371,6 +372,17 @@ BwdLayout bwd_layout(const muse_shape* sh, const muse_params* pr, const AttnLayo
   r.b.dU = cv.take<float>(nq * Cq * Ck * D * 4);
   r.b.dmu = cv.take<float>(nk * Ck * D * 4);
   r.b.dnu = cv.take<float>(nq * Cq * D * 4);
+  if (causal) {
+    const size_t toks = L.qs.ntok, rows = (size_t)sh->B * sh->Hq * sh->N;
+    r.b.pm = cv.take<float>(toks * 4);
+    r.b.pl = cv.take<float>(toks * 4);
+    r.b.pa = cv.take<float>(toks * 4);
+    r.b.lm = cv.take<float>(rows * 4);
+    r.b.ll = cv.take<float>(rows * 4);
+    r.b.la = cv.take<float>(rows * 4);
+    r.b.lse_all = cv.take<float>(rows * 4);
+    r.b.d_all = cv.take<float>(rows * 4);
+  }
   r.bytes = cv.used + 256;
   return r;
 }
@@ -443,9 +455,15 @@ muse_status validate_accum(const muse_shape* sh, const muse_params* pr, int k2) 
   return MUSE_OK;
 }
 
-muse_status validate_bwd(const muse_shape* sh, const muse_params* pr) {
-  muse_status s = validate(sh, pr, false);
+muse_status attn_bwd(const void* Q, const void* K, const void* V, const void* dO, float* dQ,
+                     float* dK, float* dV, const muse_shape* sh, const muse_params* pr, void* ws,
+                     size_t ws_bytes, cudaStream_t st, bool causal);
+
+muse_status validate_bwd(const muse_shape* sh, const muse_params* pr, bool causal = false) {
+  muse_status s = validate(sh, pr, causal);
   if (s != MUSE_OK) return s;
+  if (causal && pr->block % 32)
+    return fail(MUSE_ERR_UNSUPPORTED, "the causal backward pass needs block % 32 == 0");
   if (!backward_supported(sh->D, pr->Ck, (int)pr->mode))
     return fail(MUSE_ERR_UNSUPPORTED, "the backward pass needs mode MONOPOLE or DIPOLE and Ck * D <= 16384");
   return MUSE_OK;
@@ -470,10 +488,33 @@ size_t muse_attn_bwd_workspace_size(const muse_shape* shape, const muse_params* 
   return bwd_layout(shape, params, L, nullptr).bytes;
 }
 
+size_t muse_attn_bwd_causal_workspace_size(const muse_shape* shape, const muse_params* params) {
+  if (validate_bwd(shape, params, true) != MUSE_OK) return 0;
+  const AttnLayout L = layout(shape, params, true, nullptr, nullptr, nullptr);
+  return bwd_layout(shape, params, L, nullptr, true).bytes;
+}
+
 muse_status muse_attn_bwd(const void* Q, const void* K, const void* V, const void* dO, float* dQ,
                           float* dK, float* dV, const muse_shape* sh, const muse_params* pr,
                           void* ws, size_t ws_bytes, cudaStream_t st) {
-  muse_status s = validate_bwd(sh, pr);
+  return attn_bwd(Q, K, V, dO, dQ, dK, dV, sh, pr, ws, ws_bytes, st, false);
+}
+
+muse_status muse_attn_bwd_causal(const void* Q, const void* K, const void* V, const void* dO,
+                                 float* dQ, float* dK, float* dV, const muse_shape* sh,
+                                 const muse_params* pr, void* ws, size_t ws_bytes,
+                                 cudaStream_t st) {
+  return attn_bwd(Q, K, V, dO, dQ, dK, dV, sh, pr, ws, ws_bytes, st, true);
+}
+
+}  // extern "C"
+
+namespace {
+
+muse_status attn_bwd(const void* Q, const void* K, const void* V, const void* dO, float* dQ,
+                     float* dK, float* dV, const muse_shape* sh, const muse_params* pr, void* ws,
+                     size_t ws_bytes, cudaStream_t st, bool causal) {
+  muse_status s = validate_bwd(sh, pr, causal);
   if (s != MUSE_OK) return s;
   if (!Q || !K || !V || !dO || !dQ || !dK || !dV)
     return fail(MUSE_ERR_INVALID_ARG, "Q, K, V, dO, dQ, dK and dV must not be NULL");
@@ -481,10 +522,10 @@ muse_status muse_attn_bwd(const void* Q, const void* K, const void* V, const voi
       misaligned(dQ, 16) || misaligned(dK, 16) || misaligned(dV, 16))
     return fail(MUSE_ERR_INVALID_ARG, "all tensors must be 16-byte aligned");
   if (misaligned(ws, 256)) return fail(MUSE_ERR_INVALID_ARG, "the workspace must be 256-byte aligned");
-  const AttnLayout need = layout(sh, pr, false, Q, K, nullptr);
-  if (!ws || ws_bytes < bwd_layout(sh, pr, need, nullptr).bytes)
+  const AttnLayout need = layout(sh, pr, causal, Q, K, nullptr);
+  if (!ws || ws_bytes < bwd_layout(sh, pr, need, nullptr, causal).bytes)
     return fail(MUSE_ERR_WORKSPACE, "workspace too small for the backward pass");
-  AttnLayout L = layout(sh, pr, false, Q, K, ws);
+  AttnLayout L = layout(sh, pr, causal, Q, K, ws);
   AttnArgs a{};
   a.qg = L.qg;
   a.kg = L.kg;
@@ -498,7 +539,7 @@ muse_status muse_attn_bwd(const void* Q, const void* K, const void* V, const voi
   a.scale = pr->scale;
   a.Cq = pr->Cq;
   a.Ck = pr->Ck;
-  BwdLayout bl = bwd_layout(sh, pr, L, ws);
+  BwdLayout bl = bwd_layout(sh, pr, L, ws, causal);
   BwdArgs& b = bl.b;
   b.dO = dO;
   b.o_f32 = (sh->out_f32 || sh->dtype == MUSE_F32) ? 1 : 0;
@@ -512,9 +553,18 @@ muse_status muse_attn_bwd(const void* Q, const void* K, const void* V, const voi
   cudaMemsetAsync(b.dU, 0, nq * pr->Cq * pr->Ck * sh->D * 4, st);
   cudaMemsetAsync(b.dmu, 0, nk * pr->Ck * sh->D * 4, st);
   cudaMemsetAsync(b.dnu, 0, nq * pr->Cq * sh->D * 4, st);
-  run_attn_bwd(a, L.s1, b, st);
+  if (causal) {
+    cudaMemsetAsync(dQ, 0, (size_t)sh->B * sh->Hq * sh->N * sh->D * 4, st);  // sums over levels
+    run_attn_bwd_causal(a, L.s1, b, pr->block, st);
+  } else {
+    run_attn_bwd(a, L.s1, b, st);
+  }
   return check_launch();
 }
+
+}  // namespace
+
+extern "C" {
 
 size_t muse_accum_workspace_size(const muse_shape* shape, const muse_params* params, int topk2) {
   if (validate_accum(shape, params, topk2) != MUSE_OK) return 0;

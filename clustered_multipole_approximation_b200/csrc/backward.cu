@@ -170,6 +170,7 @@ struct QuerySmem {
   float ml[kQC][2];  // running max and sum of the far terms, per query
   float dex[kQC];  // exact terms' sum of exp(l - m) g at the running max m
   float mq[kQC];   // running max after the exact terms
+  float lsum[kQC]; // running sum after the exact terms
   int row[kQC];
   unsigned rmask[kMaxC / 32];
 };
@@ -201,7 +202,12 @@ __device__ inline void tile_sg(const QuerySmem<D>& sm, int tq, int tk, float sx[
   }
 }
 
-template <typename T, typename TO, int D, bool DIP>
+// MODE 0: one acausal problem per query (log-sum-exp and D_q formed here);
+// MODE 1: causal, write each query's (max, sum, sum of p g) over this level's
+//         terms and stop; MODE 2: causal gradients with the combined
+//         log-sum-exp and D_q of every query (dQ by atomics: a query sits in
+//         several level problems).
+template <typename T, typename TO, int D, bool DIP, int MODE>
 __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, BwdArgs b) {
   extern __shared__ __align__(16) unsigned char bq_raw[];
   QuerySmem<D>& sm = *reinterpret_cast<QuerySmem<D>*>(bq_raw);
@@ -321,13 +327,14 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
     // ---- exact terms: finish the running max / sum, and their sum of p g ---
     // (the 16 threads of a query pair hold identical running values)
     float mrun[2], lrun[2], arun[2];
+    const int nx1 = MODE == 2 ? 0 : nx;  // MODE 2 reads the combined values
 #pragma unroll
     for (int a2 = 0; a2 < 2; ++a2) {
       mrun[a2] = sm.ml[2 * tq + a2][0];
       lrun[a2] = sm.ml[2 * tq + a2][1];
       arun[a2] = 0.f;
     }
-    for (int xi = 0; xi < nx; ++xi) {
+    for (int xi = 0; xi < nx1; ++xi) {
       const int j = xl[xi], nj = kcnt[j], o0 = koff[j];
       for (int t0 = 0; t0 < nj; t0 += kKC) {
         const int kc = imin(kKC, nj - t0);
@@ -364,7 +371,12 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
         const int r = 2 * tq + a2;
         sm.lse[r] = mrun[a2] + __logf(lrun[a2]);
         sm.mq[r] = mrun[a2];
+        sm.lsum[r] = lrun[a2];
         sm.dex[r] = arun[a2];
+        if (MODE == 2 && r < qc) {  // the combined values of all the query's terms
+          sm.lse[r] = b.lse_all[sm.row[r]];
+          sm.dq_[r] = b.d_all[sm.row[r]];
+        }
       }
     }
     // ---- far terms' g = dO_q . u_ij: one warp per far cluster -------------
@@ -388,15 +400,27 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
       }
     }
     __syncthreads();
-    // D_q = sum over the terms of p g
-    for (int r = warp; r < qc; r += kBW) {
-      const float m = sm.mq[r];
-      float acc = 0.f;
-      for (int jj = lane; jj < nf; jj += 32) acc = fmaf(__expf(lf[r * Ck + jj] - m), gf[r * Ck + jj], acc);
+    // D_q = sum over the terms of p g (MODE 1: this level's share, unnormalised)
+    if (MODE != 2) {
+      for (int r = warp; r < qc; r += kBW) {
+        const float m = sm.mq[r];
+        float acc = 0.f;
+        for (int jj = lane; jj < nf; jj += 32) acc = fmaf(__expf(lf[r * Ck + jj] - m), gf[r * Ck + jj], acc);
 #pragma unroll
-      for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) sm.dq_[r] = (acc + sm.dex[r]) * __expf(m - sm.lse[r]);
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+          if (MODE == 1) {
+            const long long slot = pq.slot0 + (sm.row[r] - pq.row0);
+            b.pm[slot] = m;
+            b.pl[slot] = sm.lsum[r];
+            b.pa[slot] = acc + sm.dex[r];
+          } else {
+            sm.dq_[r] = (acc + sm.dex[r]) * __expf(m - sm.lse[r]);
+          }
+        }
+      }
     }
+    if (MODE == 1) continue;  // the partials are all this pass writes
     __syncthreads();
 
     // ---- far terms: one warp per far cluster ------------------------------
@@ -543,9 +567,219 @@ __global__ void __launch_bounds__(kBT) bwd_query_kernel(AttnArgs a, Stage1 s1, B
       const int r = 2 * tq + a2;
       if (r >= qc) continue;
 #pragma unroll
-      for (int v = 0; v < DV; ++v) b.dQ[(long long)sm.row[r] * D + tk * DV + v] = dq[a2][v];
+      for (int v = 0; v < DV; ++v) {
+        float* dst = b.dQ + (long long)sm.row[r] * D + tk * DV + v;
+        if (MODE == 2) atomicAdd(dst, dq[a2][v]);
+        else *dst = dq[a2][v];
+      }
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// causal: the local blocks (exact attention to the keys [bL, q] of the
+// query's own block), 32 queries per CTA, key tiles of 32 up to the chunk's
+// last query.  MODE 1: each query's (max, sum, sum of p g); MODE 2: the
+// gradients with the combined log-sum-exp and D_q.
+// ---------------------------------------------------------------------------
+template <typename T, typename TO, int D, int MODE>
+__global__ void __launch_bounds__(kBT) bwd_local_kernel(AttnArgs a, BwdArgs b, int L) {
+  extern __shared__ __align__(16) unsigned char bl_raw[];
+  QuerySmem<D>& sm = *reinterpret_cast<QuerySmem<D>*>(bl_raw);
+  const int bhq = blockIdx.x, c0 = blockIdx.y * kQC;
+  const int N = a.qg.lv.N, tid = threadIdx.x;
+  const int Hq = a.qg.BH / a.B, Hkv = a.kg.BH / a.B;
+  const int bb = bhq / Hq, hq = bhq - bb * Hq;
+  const long long qrow0 = (long long)bhq * N, krow0 = (long long)(bb * Hkv + hq / a.G) * N;
+  const T* Q = static_cast<const T*>(a.qg.X);
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  const TO* GO = static_cast<const TO*>(b.dO);
+  const float s = a.scale;
+  constexpr int DV = D / 16;
+  const int tq = tid >> 4, tk = tid & 15;
+  const int qc = imin(kQC, N - c0);
+  for (int e = tid; e < kQC * D; e += kBT) {
+    const int r = e / D, d = e - r * D;
+    sm.q[r][d] = r < qc ? ld<T>(Q + (qrow0 + c0 + r) * D + d) : 0.f;
+    sm.go[r][d] = r < qc ? ld<TO>(GO + (qrow0 + c0 + r) * D + d) : 0.f;
+  }
+  if (MODE == 2 && tid < kQC) {
+    sm.lse[tid] = tid < qc ? b.lse_all[qrow0 + c0 + tid] : 0.f;
+    sm.dq_[tid] = tid < qc ? b.d_all[qrow0 + c0 + tid] : 0.f;
+  }
+  float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f}, arun[2] = {0.f, 0.f};
+  float dq[2][DV];
+#pragma unroll
+  for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+    for (int v = 0; v < DV; ++v) dq[a2][v] = 0.f;
+  const int kbeg = (c0 / L) * L, kend = c0 + qc;  // keys [kbeg, kend)
+  for (int t0 = kbeg; t0 < kend; t0 += kKC) {
+    const int kc = imin(kKC, kend - t0);
+    __syncthreads();
+    for (int e = tid; e < kKC * D; e += kBT) {
+      const int r = e / D, d = e - r * D;
+      sm.kt[r][d] = r < kc ? ld<T>(K + (krow0 + t0 + r) * D + d) : 0.f;
+      sm.vt[r][d] = r < kc ? ld<T>(V + (krow0 + t0 + r) * D + d) : 0.f;
+    }
+    __syncthreads();
+    float sx[2][2], gx[2][2];
+    tile_sg<D>(sm, tq, tk, sx, gx);
+    if (MODE == 1) {
+#pragma unroll
+      for (int a2 = 0; a2 < 2; ++a2) {
+        const int qpos = c0 + 2 * tq + a2;
+        const int k0 = t0 + tk, k1 = t0 + tk + 16;
+        float l0 = (tk < kc && k0 <= qpos) ? s * sx[a2][0] : -INFINITY;
+        float l1 = (tk + 16 < kc && k1 <= qpos) ? s * sx[a2][1] : -INFINITY;
+        float mx = fmaxf(l0, l1);
+#pragma unroll
+        for (int o = 8; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const bool any = mx != -INFINITY;  // no key of this tile for these rows: no change
+        const float mn = any ? fmaxf(mrun[a2], mx) : mrun[a2];
+        const float p0 = any ? __expf(l0 - mn) : 0.f, p1 = any ? __expf(l1 - mn) : 0.f;
+        float p = p0 + p1, pg = p0 * gx[a2][0] + p1 * gx[a2][1];
+#pragma unroll
+        for (int o = 8; o; o >>= 1) {
+          p += __shfl_xor_sync(0xffffffffu, p, o);
+          pg += __shfl_xor_sync(0xffffffffu, pg, o);
+        }
+        const float sc = any ? __expf(mrun[a2] - mn) : 1.f;
+        lrun[a2] = lrun[a2] * sc + p;
+        arun[a2] = arun[a2] * sc + pg;
+        mrun[a2] = mn;
+      }
+      continue;
+    }
+    // MODE 2: P and s dS of the tile, then dq, dK, dV
+#pragma unroll
+    for (int a2 = 0; a2 < 2; ++a2) {
+      const int r = 2 * tq + a2;
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int t = tk + 16 * c2;
+        float p = 0.f, ds = 0.f;
+        if (r < qc && t < kc && t0 + t <= c0 + r) {
+          p = __expf(s * sx[a2][c2] - sm.lse[r]);
+          ds = p * (gx[a2][c2] - sm.dq_[r]);
+        }
+        sm.pt[r][t] = p;
+        sm.dst[r][t] = s * ds;
+      }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int t = 0; t < kKC; ++t) {
+      const float d0 = sm.dst[2 * tq][t], d1 = sm.dst[2 * tq + 1][t];
+#pragma unroll
+      for (int v = 0; v < DV; v += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(&sm.kt[t][tk * DV + v]);
+        dq[0][v] = fmaf(d0, k4.x, dq[0][v]);
+        dq[0][v + 1] = fmaf(d0, k4.y, dq[0][v + 1]);
+        dq[0][v + 2] = fmaf(d0, k4.z, dq[0][v + 2]);
+        dq[0][v + 3] = fmaf(d0, k4.w, dq[0][v + 3]);
+        dq[1][v] = fmaf(d1, k4.x, dq[1][v]);
+        dq[1][v + 1] = fmaf(d1, k4.y, dq[1][v + 1]);
+        dq[1][v + 2] = fmaf(d1, k4.z, dq[1][v + 2]);
+        dq[1][v + 3] = fmaf(d1, k4.w, dq[1][v + 3]);
+      }
+    }
+    float gk[2][DV], gv[2][DV];
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+      for (int v = 0; v < DV; ++v) gk[c2][v] = gv[c2][v] = 0.f;
+#pragma unroll 4
+    for (int r = 0; r < kQC; ++r) {
+      const float d0 = sm.dst[r][2 * tq], d1 = sm.dst[r][2 * tq + 1];
+      const float p0 = sm.pt[r][2 * tq], p1 = sm.pt[r][2 * tq + 1];
+#pragma unroll
+      for (int v = 0; v < DV; v += 4) {
+        const float4 q4 = *reinterpret_cast<const float4*>(&sm.q[r][tk * DV + v]);
+        const float4 g4 = *reinterpret_cast<const float4*>(&sm.go[r][tk * DV + v]);
+        gk[0][v] = fmaf(d0, q4.x, gk[0][v]);
+        gk[0][v + 1] = fmaf(d0, q4.y, gk[0][v + 1]);
+        gk[0][v + 2] = fmaf(d0, q4.z, gk[0][v + 2]);
+        gk[0][v + 3] = fmaf(d0, q4.w, gk[0][v + 3]);
+        gk[1][v] = fmaf(d1, q4.x, gk[1][v]);
+        gk[1][v + 1] = fmaf(d1, q4.y, gk[1][v + 1]);
+        gk[1][v + 2] = fmaf(d1, q4.z, gk[1][v + 2]);
+        gk[1][v + 3] = fmaf(d1, q4.w, gk[1][v + 3]);
+        gv[0][v] = fmaf(p0, g4.x, gv[0][v]);
+        gv[0][v + 1] = fmaf(p0, g4.y, gv[0][v + 1]);
+        gv[0][v + 2] = fmaf(p0, g4.z, gv[0][v + 2]);
+        gv[0][v + 3] = fmaf(p0, g4.w, gv[0][v + 3]);
+        gv[1][v] = fmaf(p1, g4.x, gv[1][v]);
+        gv[1][v + 1] = fmaf(p1, g4.y, gv[1][v + 1]);
+        gv[1][v + 2] = fmaf(p1, g4.z, gv[1][v + 2]);
+        gv[1][v + 3] = fmaf(p1, g4.w, gv[1][v + 3]);
+      }
+    }
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+      const int t = 2 * tq + c2;
+      if (t >= kc) continue;
+      const long long row = krow0 + t0 + t;
+#pragma unroll
+      for (int v = 0; v < DV; ++v) {
+        atomicAdd(b.dK + row * D + tk * DV + v, gk[c2][v]);
+        atomicAdd(b.dV + row * D + tk * DV + v, gv[c2][v]);
+      }
+    }
+  }
+  if (MODE == 1) {
+    if (tk == 0) {
+#pragma unroll
+      for (int a2 = 0; a2 < 2; ++a2) {
+        const int r = 2 * tq + a2;
+        if (r >= qc) continue;
+        b.lm[qrow0 + c0 + r] = mrun[a2];
+        b.ll[qrow0 + c0 + r] = lrun[a2];
+        b.la[qrow0 + c0 + r] = arun[a2];
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int a2 = 0; a2 < 2; ++a2) {
+    const int r = 2 * tq + a2;
+    if (r >= qc) continue;
+#pragma unroll
+    for (int v = 0; v < DV; ++v) atomicAdd(b.dQ + (qrow0 + c0 + r) * D + tk * DV + v, dq[a2][v]);
+  }
+}
+
+// causal: every query's log-sum-exp and D_q over its local block and the level
+// problems it is a query of (the forward's merge: level l when bit l of its
+// block index is set)
+__global__ void bwd_combine_kernel(AttnArgs a, BwdArgs b, int L) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int N = a.qg.lv.N;
+  if (e >= (long long)a.qg.BH * N) return;
+  const int bhq = (int)(e / N), qpos = (int)(e - (long long)bhq * N);
+  const Levels& lv = a.qg.lv;
+  const int blk = qpos / L;
+  float m = b.lm[e];
+  for (int l = 0; l < lv.nlev; ++l)
+    if ((blk >> l) & 1) {
+      const int sz = L << l, p = blk >> (l + 1);
+      const long long slot = (long long)bhq * lv.toks_per_bh + lv.tok_base[l] + (long long)p * sz +
+                             (qpos - (2 * p + 1) * sz);
+      m = fmaxf(m, b.pm[slot]);
+    }
+  float sum = b.ll[e] * __expf(b.lm[e] - m), acc = b.la[e] * __expf(b.lm[e] - m);
+  for (int l = 0; l < lv.nlev; ++l)
+    if ((blk >> l) & 1) {
+      const int sz = L << l, p = blk >> (l + 1);
+      const long long slot = (long long)bhq * lv.toks_per_bh + lv.tok_base[l] + (long long)p * sz +
+                             (qpos - (2 * p + 1) * sz);
+      const float w = __expf(b.pm[slot] - m);
+      sum = fmaf(b.pl[slot], w, sum);
+      acc = fmaf(b.pa[slot], w, acc);
+    }
+  b.lse_all[e] = m + __logf(sum);
+  b.d_all[e] = acc / sum;
 }
 
 // ---------------------------------------------------------------------------
@@ -665,8 +899,13 @@ __global__ void __launch_bounds__(kBT) bwd_cluster_kernel(AttnArgs a, BwdArgs b)
             gv = fmaf(dM[e * (D + 1) + f], rows[r * D + f], gv);
             gk = fmaf(dM[f * (D + 1) + e], nus[r * D + f], gk);
           }
-        b.dV[row * D + e] += gv;  // the member's only writer in this launch
-        b.dK[row * D + e] += gk;
+        if (a.qg.lv.causal) {  // a key sits in one key set per level
+          atomicAdd(b.dV + row * D + e, gv);
+          atomicAdd(b.dK + row * D + e, gk);
+        } else {  // the member's only writer in this launch
+          b.dV[row * D + e] += gv;
+          b.dK[row * D + e] += gk;
+        }
       }
     }
   }
@@ -688,7 +927,8 @@ __global__ void __launch_bounds__(kBT) bwd_query_nu_kernel(AttnArgs a, BwdArgs b
   for (int e = tid; e < m * D; e += kBT) {
     const int r = e / D, d = e - r * D;
     const long long row = pq.row0 + perm[off + r];
-    b.dQ[row * D + d] += dn[d] * inv;
+    if (a.qg.lv.causal) atomicAdd(b.dQ + row * D + d, dn[d] * inv);  // one query set per level
+    else b.dQ[row * D + d] += dn[d] * inv;
   }
 }
 
@@ -698,47 +938,72 @@ size_t query_smem(int Ck) {
 }
 
 template <typename T, typename TO, int D, bool DIP>
-void launch_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st) {
+void launch_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, int L, cudaStream_t st) {
   const int nk = a.ks.nprob, nq = a.qs.nprob;
-  {
+  if (nk > 0) {
     ProfScope ps(st, "bwd_key_stats");
     bwd_key_stats_kernel<T, D, DIP><<<dim3(nk, a.Ck), kBT, 0, st>>>(a, b);
   }
-  if (DIP) {
+  if (DIP && nq > 0) {
     ProfScope ps(st, "bwd_u_table");
     const size_t sm = (size_t)(D * (D + 1) + kBT) * 4;
     cudaFuncSetAttribute(bwd_u_table_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     bwd_u_table_kernel<D><<<dim3(nq, a.Ck), kBT, sm, st>>>(a, b);
   }
-  {
+  if (L == 0) {
     ProfScope ps(st, "bwd_query");
     const size_t sm = query_smem<T, D, DIP>(a.Ck);
-    cudaFuncSetAttribute(bwd_query_kernel<T, TO, D, DIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(bwd_query_kernel<T, TO, D, DIP, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)sm);
-    bwd_query_kernel<T, TO, D, DIP><<<dim3(nq, a.Cq), kBT, sm, st>>>(a, s1, b);
+    bwd_query_kernel<T, TO, D, DIP, 0><<<dim3(nq, a.Cq), kBT, sm, st>>>(a, s1, b);
+  } else {
+    const size_t sm = query_smem<T, D, DIP>(a.Ck);
+    const size_t sl = sizeof(QuerySmem<D>);
+    const long long rows = (long long)a.qg.BH * a.qg.lv.N;
+    const dim3 lgrid(a.qg.BH, cdiv(a.qg.lv.N, kQC));
+    cudaFuncSetAttribute(bwd_query_kernel<T, TO, D, DIP, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)sm);
+    cudaFuncSetAttribute(bwd_query_kernel<T, TO, D, DIP, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)sm);
+    cudaFuncSetAttribute(bwd_local_kernel<T, TO, D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sl);
+    cudaFuncSetAttribute(bwd_local_kernel<T, TO, D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sl);
+    {
+      ProfScope ps(st, "bwd_lse");
+      if (nq > 0) bwd_query_kernel<T, TO, D, DIP, 1><<<dim3(nq, a.Cq), kBT, sm, st>>>(a, s1, b);
+      bwd_local_kernel<T, TO, D, 1><<<lgrid, kBT, sl, st>>>(a, b, L);
+      bwd_combine_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(a, b, L);
+    }
+    {
+      ProfScope ps(st, "bwd_query");
+      if (nq > 0) bwd_query_kernel<T, TO, D, DIP, 2><<<dim3(nq, a.Cq), kBT, sm, st>>>(a, s1, b);
+    }
+    {
+      ProfScope ps(st, "bwd_local");
+      bwd_local_kernel<T, TO, D, 2><<<lgrid, kBT, sl, st>>>(a, b, L);
+    }
   }
-  {
+  if (nk > 0) {
     ProfScope ps(st, "bwd_cluster");
     const size_t sm = (size_t)(2 * D * (D + 1) + 64 * D + 4 * D) * 4;
     cudaFuncSetAttribute(bwd_cluster_kernel<T, D, DIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)sm);
     bwd_cluster_kernel<T, D, DIP><<<dim3(nk, a.Ck), kBT, sm, st>>>(a, b);
   }
-  if (DIP) {
+  if (DIP && nq > 0) {
     ProfScope ps(st, "bwd_query_nu");
     bwd_query_nu_kernel<D><<<dim3(nq, a.Cq), kBT, 0, st>>>(a, b);
   }
 }
 
 template <typename T, typename TO>
-void dispatch_d(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st) {
+void dispatch_d(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, int L, cudaStream_t st) {
   const bool dip = a.mode == 1;
   if (a.qg.D == 64) {
-    if (dip) launch_bwd<T, TO, 64, true>(a, s1, b, st);
-    else launch_bwd<T, TO, 64, false>(a, s1, b, st);
+    if (dip) launch_bwd<T, TO, 64, true>(a, s1, b, L, st);
+    else launch_bwd<T, TO, 64, false>(a, s1, b, L, st);
   } else {
-    if (dip) launch_bwd<T, TO, 128, true>(a, s1, b, st);
-    else launch_bwd<T, TO, 128, false>(a, s1, b, st);
+    if (dip) launch_bwd<T, TO, 128, true>(a, s1, b, L, st);
+    else launch_bwd<T, TO, 128, false>(a, s1, b, L, st);
   }
 }
 
@@ -748,14 +1013,23 @@ bool backward_supported(int D, int Ck, int mode) {
   return (mode == 0 || mode == 1) && (D == 64 || D == 128) && Ck * D <= 16384;
 }
 
-void run_attn_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st) {
+static void run_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, int L, cudaStream_t st) {
   using bf = __nv_bfloat16;
   if (a.qg.dtype == 0) {
-    if (b.o_f32) dispatch_d<bf, float>(a, s1, b, st);
-    else dispatch_d<bf, bf>(a, s1, b, st);
+    if (b.o_f32) dispatch_d<bf, float>(a, s1, b, L, st);
+    else dispatch_d<bf, bf>(a, s1, b, L, st);
   } else {
-    dispatch_d<float, float>(a, s1, b, st);
+    dispatch_d<float, float>(a, s1, b, L, st);
   }
+}
+
+void run_attn_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st) {
+  run_bwd(a, s1, b, 0, st);
+}
+
+void run_attn_bwd_causal(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, int L,
+                         cudaStream_t st) {
+  run_bwd(a, s1, b, L, st);
 }
 
 }  // namespace muse

@@ -142,8 +142,21 @@ struct BwdArgs {
   float* dU;       // [query sets][Cq][Ck][D], zeroed by the caller
   float* dmu;      // [key sets][Ck][D], zeroed by the caller
   float* dnu;      // [query sets][Cq][D], zeroed by the caller
+  // causal only: per level-problem slot and per query row, (max, sum, sum of
+  // p g) over that set of terms; then the combined log-sum-exp and D_q
+  float* pm;       // [query tokens of all levels]
+  float* pl;
+  float* pa;
+  float* lm;       // [B Hq N] the local block's
+  float* ll;
+  float* la;
+  float* lse_all;  // [B Hq N]
+  float* d_all;    // [B Hq N]
 };
 bool backward_supported(int D, int Ck, int mode);
+// Causal backward (the hierarchical levels plus the local blocks of L keys).
+void run_attn_bwd_causal(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, int L,
+                         cudaStream_t st);
 void run_attn_bwd(const AttnArgs& a, const Stage1& s1, const BwdArgs& b, cudaStream_t st);
 
 // Causal operator with block-summary accumulation (accum.cu).

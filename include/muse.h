@@ -286,7 +286,8 @@ muse_status muse_attn_fwd_causal_accum(const void *Q, const void *K, const void 
  * terms.  dK, dV and dQ are sums of fp32 atomic adds, so their last bits may
  * differ from call to call.
  * Supported: modes MONOPOLE and DIPOLE, Ck * D <= 16384; other modes and
- * sizes return MUSE_ERR_UNSUPPORTED.  A workspace smaller than
+ * sizes return MUSE_ERR_UNSUPPORTED.  (The causal operator's gradients:
+ * muse_attn_bwd_causal below.)  A workspace smaller than
  * muse_attn_bwd_workspace_size() returns MUSE_ERR_WORKSPACE.
  */
 size_t muse_attn_bwd_workspace_size(const muse_shape *shape, const muse_params *params);
@@ -294,6 +295,24 @@ muse_status muse_attn_bwd(const void *Q, const void *K, const void *V, const voi
                           float *dQ, float *dK, float *dV, const muse_shape *shape,
                           const muse_params *params, void *ws, size_t ws_bytes,
                           cudaStream_t stream);
+
+/*
+ * Gradients of the causal operator (muse_attn_fwd_causal), with the same
+ * contract as muse_attn_bwd: the workspace sized by
+ * muse_attn_bwd_causal_workspace_size() goes to muse_attn_fwd_causal first
+ * and then, unchanged, here.  Every query's terms -- its local block and the
+ * level problems it is a query of -- meet in one softmax, so the backward
+ * first forms each query's combined log-sum-exp and sum of p dO.x (per level
+ * problem and per local block, then combined), then the gradients of every
+ * term; a query's and a key's gradient is summed over its levels by fp32
+ * atomic adds.  Modes MONOPOLE and DIPOLE, Ck * D <= 16384, block % 32 == 0
+ * (MUSE_ERR_UNSUPPORTED otherwise).
+ */
+size_t muse_attn_bwd_causal_workspace_size(const muse_shape *shape, const muse_params *params);
+muse_status muse_attn_bwd_causal(const void *Q, const void *K, const void *V, const void *dO,
+                                 float *dQ, float *dK, float *dV, const muse_shape *shape,
+                                 const muse_params *params, void *ws, size_t ws_bytes,
+                                 cudaStream_t stream);
 
 /*
  * muse_cluster without a workspace argument, for callers that cannot

@@ -19,7 +19,7 @@ import oracle
 from clustered_multipole_approximation_b200 import build
 from clustered_multipole_approximation_b200.inputs import WORKLOADS, clustered_qkv, make_inputs
 from helpers import TOL, assert_close, to_dev
-from oracle.muse_backward import muse_acausal_grads
+from oracle.muse_backward import muse_acausal_grads, muse_causal_grads
 
 pytestmark = pytest.mark.gpu
 
@@ -171,3 +171,84 @@ def test_backward_unsupported_modes_are_refused(mode):
     with pytest.raises(muse.MuseError):
         muse.muse_attn_bwd(q, k, v, q, Cq=4, Ck=4, iters=2, seed=1, topk=1, mode=mode,
                            workspace=ws)
+
+
+# ---------------------------------------------------------------------------
+# causal
+def gpu_causal_fwd_bwd(Q, K, V, dO, dtype, L, C, iters, seed, topk, scale, mode):
+    q, k, v = to_dev(Q, dtype), to_dev(K, dtype), to_dev(V, dtype)
+    p = muse.make_params(C, C, iters, seed, topk, L, scale, mode)
+    ws = torch.empty(muse.backward_workspace_size(q, k, p, out_f32=True, causal=True),
+                     dtype=torch.uint8, device=q.device)
+    O, dbg = muse.muse_attn_fwd_causal(q, k, v, C=C, block=L, iters=iters, seed=seed, topk=topk,
+                                       scale=scale, mode=mode, debug=True,
+                                       out_dtype=torch.float32, workspace=ws)
+    do = torch.from_numpy(np.ascontiguousarray(dO, dtype=np.float32)).cuda()
+    dq, dk, dv = muse.muse_attn_bwd_causal(q, k, v, do, C=C, block=L, iters=iters, seed=seed,
+                                           topk=topk, scale=scale, mode=mode, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(dbg["device_error"].item()) == 0
+    g = {n: t.cpu().numpy() for n, t in dbg.items()}
+    return O.cpu().numpy(), g, dq.cpu().numpy(), dk.cpu().numpy(), dv.cpu().numpy()
+
+
+def check_causal_bwd(Q, K, V, dtype, L, C, iters, seed, topk, scale, mode, dseed=0):
+    B, Hq = Q.shape[:2]
+    dO = np.random.default_rng(dseed).standard_normal(Q.shape).astype(np.float32)
+    O, g, dq, dk, dv = gpu_causal_fwd_bwd(Q, K, V, dO, dtype, L, C, iters, seed, topk, scale, mode)
+    Or, dQr, dKr, dVr = muse_causal_grads(Q, K, V, dO, g["q_assign"], g["k_assign"],
+                                          g.get("selected"), L, C, scale, mode)
+    for b in range(B):
+        for h in range(Hq):
+            assert_close(O[b, h], Or[b, h], TOL[dtype], f"O b{b}h{h}")
+            grad_close(dq[b, h], dQr[b, h], f"dQ b{b}h{h}")
+        for hk in range(K.shape[1]):
+            grad_close(dk[b, hk], dKr[b, hk], f"dK b{b}h{hk}")
+            grad_close(dv[b, hk], dVr[b, hk], f"dV b{b}h{hk}")
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("dtype,D", [("f32", 64), ("bf16", 64), ("bf16", 128)])
+@pytest.mark.parametrize("mode", ["monopole", "dipole"])
+def test_small_causal_backward_gqa(dtype, D, mode):
+    Q, K, V = clustered_qkv(1, 4, 2, 512, D, 8, 0.3, 0.0, dtype, 151 + D)
+    check_causal_bwd(Q, K, V, dtype, 64, 12, 4, 21, 2, 0.9, mode, dseed=D)
+
+
+def test_causal_backward_low_levels_per_key_token():
+    # C = 32 with blocks of 128: the forward takes the lowest levels per key
+    # token (bf16 DIPOLE); the backward differentiates the same sums
+    Q, K, V = clustered_qkv(1, 2, 1, 512, 64, 12, 0.3, 0.0, "bf16", 152)
+    check_causal_bwd(Q, K, V, "bf16", 128, 32, 4, 61, 3, 1.0, "dipole")
+
+
+def test_causal_backward_singletons_is_exact_causal_attention_gradient():
+    Q, K, V = clustered_qkv(1, 2, 1, 256, 64, 8, 0.3, 0.0, "f32", 153)
+    dq, dk, dv = check_causal_bwd(Q, K, V, "f32", 32, 256, 2, 3, 0, 1.0, "dipole")
+    q, k, v = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (Q, K, V))
+    o = torch.nn.functional.scaled_dot_product_attention(q, k.expand(-1, 2, -1, -1),
+                                                         v.expand(-1, 2, -1, -1), is_causal=True,
+                                                         scale=1.0)
+    dO = np.random.default_rng(0).standard_normal(Q.shape)
+    gq, gk, gv = torch.autograd.grad((o * torch.tensor(dO)).sum(), (q, k, v))
+    for a, r, n in ((dq, gq, "dQ"), (dk, gk, "dK"), (dv, gv, "dV")):
+        grad_close(a, r.numpy(), n + " vs exact causal attention")
+
+
+def test_causal_backward_translation_invariants_full_size():
+    """The 16k causal layer (B=2, 8 heads, C=64, blocks of 512): every head's
+    key gradient sums to zero over its tokens and its value gradient to the
+    sum of dO."""
+    w = WORKLOADS["causal-bf16-b2h8-n16k"]
+    Q, K, V = make_inputs(w)
+    dO = np.random.default_rng(2).standard_normal(Q.shape).astype(np.float32)
+    _, _, _, dk, dv = gpu_causal_fwd_bwd(Q, K, V, dO, w.dtype, w.block, w.C, w.iters,
+                                         w.cluster_seed, w.topk, w.scale, "dipole")
+    assert np.isfinite(dk).all() and np.isfinite(dv).all()
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            scale = np.abs(dk[b, h]).max() * np.sqrt(w.N)
+            assert np.abs(dk[b, h].sum(0)).max() <= 1e-4 * scale, (b, h)
+            want = dO[b, h].astype(np.float64).sum(0)
+            got = dv[b, h].astype(np.float64).sum(0)
+            assert np.abs(got - want).max() <= 1e-4 * np.abs(want).max(), (b, h)
