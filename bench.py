@@ -431,7 +431,8 @@ def run_muse(w, mode, steps, warmup, rank, world, device, e2e_leg=True):
 # ---------------------------------------------------------------------------
 # the backward pass (acausal): gradients of <dO, O> through the C ABI
 # ---------------------------------------------------------------------------
-BWD_KERNELS = ("bwd_key_stats", "bwd_u_table", "bwd_query", "bwd_cluster", "bwd_query_nu")
+BWD_KERNELS = ("bwd_key_stats", "bwd_u_table", "bwd_lse", "bwd_query", "bwd_local", "bwd_cluster",
+               "bwd_query_nu")
 
 
 def backward_work(w, mode, dbg):
@@ -444,17 +445,21 @@ def backward_work(w, mode, dbg):
                      q-head; the members' chain: 4 D^2 per key, per kv-head;
                      (MONOPOLE: 2 D per key)."""
     far, exact = retrieval_rows(w, mode, dbg)
-    B, Hq, Hkv, D, N, C = w.B, w.Hq, w.Hkv, w.D, w.N, w.C
+    B, Hq, Hkv, D, N = w.B, w.Hq, w.Hkv, w.D, w.N
     dip = mode == "dipole"
     work = dict.fromkeys(BWD_KERNELS, 0.0)
-    work["bwd_key_stats"] = B * Hkv * N * (D + (2.0 * D * D if dip else 0.0))
-    if dip:
-        work["bwd_u_table"] = B * Hq * C * 2.0 * C * D * D
-        work["bwd_cluster"] = B * Hq * C * 4.0 * C * D * D + B * Hkv * N * 4.0 * D * D
-        work["bwd_query_nu"] = B * Hq * N * D
-    else:
-        work["bwd_cluster"] = B * Hkv * N * 2.0 * D
+    for s, npairs, ce, _dense in level_table(w, mode):
+        toks = npairs * s  # key tokens (and query tokens) of the level's problems, per head
+        work["bwd_key_stats"] += B * Hkv * toks * (D + (2.0 * D * D if dip else 0.0))
+        if dip:
+            work["bwd_u_table"] += B * Hq * npairs * ce * 2.0 * ce * D * D
+            work["bwd_cluster"] += B * Hq * npairs * ce * 4.0 * ce * D * D + B * Hkv * toks * 4.0 * D * D
+            work["bwd_query_nu"] += B * Hq * toks * D
+        else:
+            work["bwd_cluster"] += B * Hkv * toks * 2.0 * D
     work["bwd_query"] = 10.0 * D * (sum(far) + sum(exact))
+    if w.causal:  # the local blocks: 10 D per (query, key) pair, keys up to the query
+        work["bwd_local"] = 10.0 * D * B * Hq * (N // w.block) * w.block * (w.block + 1) / 2
     return work
 
 
@@ -468,11 +473,19 @@ def run_backward(w, mode, steps, warmup, device):
     cast = (lambda x: torch.from_numpy(x).to(torch.bfloat16)) if w.dtype == "bf16" else torch.from_numpy
     q, k, v = cast(Q).to(device), cast(K).to(device), cast(V).to(device)
     del Q, K, V
-    kw = dict(Cq=w.C, Ck=w.C, iters=w.iters, seed=w.cluster_seed, topk=w.topk, scale=w.scale,
-              mode=mode)
-    p = muse.make_params(w.C, w.C, w.iters, w.cluster_seed, w.topk, 0, w.scale, mode)
-    ws = torch.empty(muse.backward_workspace_size(q, k, p), dtype=torch.uint8, device=device)
-    o, dbg = muse.muse_attn_fwd(q, k, v, workspace=ws, debug=True, **kw)
+    if w.causal:
+        kw = dict(C=w.C, block=w.block, iters=w.iters, seed=w.cluster_seed, topk=w.topk,
+                  scale=w.scale, mode=mode)
+        p = muse.make_params(w.C, w.C, w.iters, w.cluster_seed, w.topk, w.block, w.scale, mode)
+        fwd, bwd = muse.muse_attn_fwd_causal, muse.muse_attn_bwd_causal
+    else:
+        kw = dict(Cq=w.C, Ck=w.C, iters=w.iters, seed=w.cluster_seed, topk=w.topk, scale=w.scale,
+                  mode=mode)
+        p = muse.make_params(w.C, w.C, w.iters, w.cluster_seed, w.topk, 0, w.scale, mode)
+        fwd, bwd = muse.muse_attn_fwd, muse.muse_attn_bwd
+    ws = torch.empty(muse.backward_workspace_size(q, k, p, causal=w.causal), dtype=torch.uint8,
+                     device=device)
+    o, dbg = fwd(q, k, v, workspace=ws, debug=True, **kw)
     dbg = {n: t.cpu().numpy() for n, t in dbg.items()}
     do = torch.randn(o.shape, generator=torch.Generator(device=device).manual_seed(7),
                      device=device).to(o.dtype)
@@ -480,7 +493,7 @@ def run_backward(w, mode, steps, warmup, device):
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         flush.zero_()
-        muse.muse_attn_bwd(q, k, v, do, workspace=ws, **kw)
+        bwd(q, k, v, do, workspace=ws, **kw)
     torch.cuda.synchronize()
     muse.profile_read()
     muse.profile_enable(True)
@@ -490,7 +503,7 @@ def run_backward(w, mode, steps, warmup, device):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        muse.muse_attn_bwd(q, k, v, do, workspace=ws, **kw)
+        bwd(q, k, v, do, workspace=ws, **kw)
         e1.record(stream)
         torch.cuda.synchronize()
         total += e0.elapsed_time(e1)
@@ -696,9 +709,11 @@ def main():
             side[f"{name}/{sm}"] = side_entry(rr, sw, st, wu)
         line["workloads"] = side
     if world == 1 and not args.no_side and args.workload == DEFAULT_WORKLOAD and args.mode is None:
+        cw = WORKLOADS["causal-bf16-b2h8-n16k"]
         line["backward"] = {m: run_backward(w, m, args.steps, args.warmup, device)
                             for m in ("dipole", "monopole")}
-        cw = WORKLOADS["causal-bf16-b2h8-n16k"]
+        line["backward"]["causal-16k/dipole"] = run_backward(cw, "dipole", args.steps, args.warmup,
+                                                             device)
         line["accum"] = {m: run_accum_bench(cw, m, args.steps, args.warmup, device)
                          for m in ("dipole", "monopole")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
