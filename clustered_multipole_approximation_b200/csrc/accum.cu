@@ -670,6 +670,286 @@ __global__ void __launch_bounds__(kST) acc_stage2_kernel(AttnArgs a, AccArgs c) 
   }
 }
 
+// ---------------------------------------------------------------------------
+// MONOPOLE: the same terms with every query of the CTA's clusters in flight at
+// once (the values of the unselected clusters are shared by all clusters, so
+// only the selected clusters' remainders are per cluster; kCM * k1 rows).
+// ---------------------------------------------------------------------------
+constexpr int kCM = 16;    // query clusters per CTA
+constexpr int kRM = 64;    // remainder rows per CTA: kCM clusters x k1, or fewer clusters for k1 > 4
+
+template <int D>
+size_t stage2_mono_smem(int Ck) {
+  return ((size_t)Ck * (D + 1) + (size_t)Ck * D + Ck + (size_t)kRM * (D + 1) + (size_t)kRM * D + kRM +
+          (size_t)kSW * D) * 4 + (size_t)kCM * Ck + (size_t)kSW * 32 * 4 + (size_t)kSW * 32 * 8 * 2 + 64;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArgs c, int nci) {
+  extern __shared__ __align__(16) float sm_raw[];
+  const int Cq = a.Cq, Ck = a.Ck, NB = c.NB, k1 = a.topk, k2 = c.k2;
+  float* mu_s = sm_raw;                         // [Ck][D + 1] prefix centroids
+  float* u_s = mu_s + (size_t)Ck * (D + 1);     // [Ck][D] prefix values S / n
+  float* ln_s = u_s + (size_t)Ck * D;           // [Ck]
+  float* rm_s = ln_s + Ck;                      // [kRM][D + 1] remainder centroids
+  float* ru_s = rm_s + (size_t)kRM * (D + 1);   // [kRM][D] remainder values
+  float* rl_s = ru_s + (size_t)kRM * D;         // [kRM]
+  float* q_s = rl_s + kRM;                      // [kSW][D]
+  float* pw_s = q_s + kSW * D;                  // [kSW][32]
+  const float** uw_s = reinterpret_cast<const float**>(  // [kSW][32]
+      (reinterpret_cast<uintptr_t>(pw_s + kSW * 32) + 7) & ~(uintptr_t)7);
+  long long* xb_s = reinterpret_cast<long long*>(uw_s + kSW * 32);   // [kSW][32] retrieved rows
+  signed char* rsel = reinterpret_cast<signed char*>(xb_s + kSW * 32);  // [nci][Ck]
+  __shared__ int qcum[kCM + 1];
+  __shared__ int nretr[kCM];
+  const int qpid = blockIdx.x, b = blockIdx.y, i0 = blockIdx.z * nci;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (b == 0) return;
+  const int ncl = imin(nci, Cq - i0);
+  const Prob pq = prob_of(a.qg, qpid);
+  const int kpid = kv_problem(a, qpid);
+  const Prob pk = prob_of(a.kg, kpid);
+  const float s = a.scale;
+  constexpr int DL = D / 32;
+  // ---- the block's prefix table --------------------------------------------
+  for (int j = warp; j < Ck; j += kSW) {
+    const size_t o = ((size_t)kpid * NB + b) * Ck + j;
+    const int n = c.pn[o];
+    if (lane == 0) ln_s[j] = n > 0 ? logf((float)n) : -INFINITY;
+#pragma unroll
+    for (int u = 0; u < DL; ++u) {
+      const int d = lane + 32 * u;
+      mu_s[j * (D + 1) + d] = n > 0 ? (float)(c.pk[o * D + d] / (double)n) : 0.f;
+      u_s[j * D + d] = n > 0 ? c.ps[o * D + d] / (float)n : 0.f;
+    }
+  }
+  // ---- per cluster: its query range, its selected clusters, their remainders
+  for (int e = tid; e < ncl * Ck; e += kST) rsel[e] = -1;
+  if (tid == 0) {
+    int acc = 0;
+    for (int cc = 0; cc < ncl; ++cc) {
+      const int* qb = c.qboff + ((size_t)qpid * Cq + i0 + cc) * (NB + 1);
+      qcum[cc] = acc;
+      acc += qb[b + 1] - qb[b];
+    }
+    qcum[ncl] = acc;
+  }
+  __syncthreads();
+  for (int e = tid; e < ncl * k1; e += kST) {
+    const int cc = e / k1, r = e - cc * k1;
+    const int j = c.sel1[(((size_t)qpid * NB + b) * Cq + i0 + cc) * k1 + r];
+    if (j >= 0) rsel[cc * Ck + j] = (signed char)r;
+  }
+  if (tid < ncl) {
+    const int* s1 = c.sel1 + (((size_t)qpid * NB + b) * Cq + i0 + tid) * k1;
+    const int* s2 = c.sel2 + ((((size_t)qpid * NB + b) * Cq + i0 + tid) * k1) * k2;
+    int cnt = 0;
+    for (int r = 0; r < k1; ++r) {
+      const int j = s1[r];
+      if (j < 0) break;
+      for (int r2 = 0; r2 < k2; ++r2) {
+        const int bb = s2[r * k2 + r2];
+        if (bb < 0) break;
+        cnt += c.bn[((size_t)kpid * NB + bb) * Ck + j];
+      }
+    }
+    nretr[tid] = cnt;
+  }
+  for (int e = warp; e < ncl * k1; e += kSW) {
+    const int cc = e / k1, r = e - cc * k1, row = cc * k1 + r;
+    const int* s1 = c.sel1 + (((size_t)qpid * NB + b) * Cq + i0 + cc) * k1;
+    const int* s2 = c.sel2 + ((((size_t)qpid * NB + b) * Cq + i0 + cc) * k1) * k2;
+    const int j = s1[r];
+    if (j < 0) {
+      if (lane == 0) rl_s[row] = -INFINITY;
+      continue;
+    }
+    const size_t o = ((size_t)kpid * NB + b) * Ck + j;
+    int n = c.pn[o];
+    double ksum[DL];
+    float ss[DL];
+#pragma unroll
+    for (int u = 0; u < DL; ++u) {
+      ksum[u] = c.pk[o * D + lane + 32 * u];
+      ss[u] = c.ps[o * D + lane + 32 * u];
+    }
+    for (int r2 = 0; r2 < k2; ++r2) {
+      const int bb = s2[r * k2 + r2];
+      if (bb < 0) break;
+      const size_t ob = ((size_t)kpid * NB + bb) * Ck + j;
+      n -= c.bn[ob];
+#pragma unroll
+      for (int u = 0; u < DL; ++u) {
+        ksum[u] -= c.bk[ob * D + lane + 32 * u];
+        ss[u] -= c.bs[ob * D + lane + 32 * u];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < DL; ++u) {
+      const int d = lane + 32 * u;
+      rm_s[row * (D + 1) + d] = n > 0 ? (float)(ksum[u] / (double)n) : 0.f;
+      ru_s[row * D + d] = n > 0 ? ss[u] / (float)n : 0.f;
+    }
+    if (lane == 0) rl_s[row] = n > 0 ? logf((float)n) : -INFINITY;
+  }
+  __syncthreads();
+  // ---- one warp per query, across all of the CTA's clusters ----------------
+  const T* Q = static_cast<const T*>(a.qg.X);
+  const T* K = static_cast<const T*>(a.kg.X);
+  const T* V = static_cast<const T*>(a.V);
+  const int* kperm = a.ks.perm + pk.slot0;
+  const int* koff = a.ks.off + (size_t)kpid * (Ck + 1);
+  float* qw = q_s + warp * D;
+  float* pw = pw_s + warp * 32;
+  const float** uw = uw_s + warp * 32;
+  for (int m = warp; m < qcum[ncl]; m += kSW) {
+    int cc = 0;
+    while (qcum[cc + 1] <= m) ++cc;
+    const int i = i0 + cc;
+    const int* qb = c.qboff + ((size_t)qpid * Cq + i) * (NB + 1);
+    const int* qperm = a.qs.perm + pq.slot0 + a.qs.off[(size_t)qpid * (Cq + 1) + i];
+    const long long qrow = pq.row0 + qperm[qb[b] + (m - qcum[cc])];
+    const signed char* rs = rsel + cc * Ck;
+    const int* s1 = c.sel1 + (((size_t)qpid * NB + b) * Cq + i) * k1;
+    const int* s2 = c.sel2 + ((((size_t)qpid * NB + b) * Cq + i) * k1) * k2;
+    float o[DL];
+#pragma unroll
+    for (int u = 0; u < DL; ++u) {
+      qw[lane + 32 * u] = ld<T>(Q + qrow * D + lane + 32 * u);
+      o[u] = 0.f;
+    }
+    __syncwarp();
+    float mx = -INFINITY, l = 0.f;
+    for (int j0 = 0; j0 < Ck; j0 += 32) {
+      const int j = j0 + lane;
+      float lg = -INFINITY;
+      const float* urow = u_s;
+      if (j < Ck) {
+        const int r = rs[j];
+        const int row = cc * k1 + r;
+        const float lnj = r >= 0 ? rl_s[row] : ln_s[j];
+        if (lnj != -INFINITY) {
+          const float* mrow = r >= 0 ? rm_s + row * (D + 1) : mu_s + j * (D + 1);
+          float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+#pragma unroll 4
+          for (int d = 0; d < D; d += 4) {
+            x0 = fmaf(qw[d], mrow[d], x0);
+            x1 = fmaf(qw[d + 1], mrow[d + 1], x1);
+            x2 = fmaf(qw[d + 2], mrow[d + 2], x2);
+            x3 = fmaf(qw[d + 3], mrow[d + 3], x3);
+          }
+          lg = fmaf(s, (x0 + x1) + (x2 + x3), lnj);
+          urow = r >= 0 ? ru_s + row * D : u_s + j * D;
+        }
+      }
+      float bm = lg;
+#pragma unroll
+      for (int o2 = 16; o2; o2 >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o2));
+      if (bm == -INFINITY) continue;
+      const float mn = fmaxf(mx, bm);
+      const float sc = __expf(mx - mn);
+      const float p = __expf(lg - mn);
+      pw[lane] = p;
+      uw[lane] = urow;
+      float ps = p;
+#pragma unroll
+      for (int o2 = 16; o2; o2 >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o2);
+      l = l * sc + ps;
+#pragma unroll
+      for (int u = 0; u < DL; ++u) o[u] *= sc;
+      mx = mn;
+      __syncwarp();
+#pragma unroll 8
+      for (int jj = 0; jj < 32; ++jj) {
+        const float pj = pw[jj];
+        if (pj == 0.f) continue;
+        const float* ur = uw[jj];
+#pragma unroll
+        for (int u = 0; u < DL; ++u) o[u] = fmaf(pj, ur[lane + 32 * u], o[u]);
+      }
+      __syncwarp();
+    }
+    // retrieved keys: their rows gathered 32 at a time into the warp's buffer,
+    // then one key per lane for the logits and the warp over the values
+    long long* xb = xb_s + warp * 32;
+    int nb = 0;
+    auto flush = [&]() {
+      float lg = -INFINITY;
+      if (lane < nb) {
+        const long long krow = xb[lane];
+        float x = 0.f;
+        if (sizeof(T) == 2) {
+          const uint4* kp = reinterpret_cast<const uint4*>(K + krow * D);
+#pragma unroll
+          for (int c8 = 0; c8 < D / 8; ++c8) {
+            const uint4 w = __ldg(kp + c8);
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h[e]);
+              x = fmaf(qw[c8 * 8 + 2 * e], f.x, x);
+              x = fmaf(qw[c8 * 8 + 2 * e + 1], f.y, x);
+            }
+          }
+        } else {
+#pragma unroll 16
+          for (int d = 0; d < D; ++d) x = fmaf(qw[d], ld<T>(K + krow * D + d), x);
+        }
+        lg = s * x;
+      }
+      float bm = lg;
+#pragma unroll
+      for (int o2 = 16; o2; o2 >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o2));
+      const float mn = fmaxf(mx, bm);
+      const float sc = __expf(mx - mn);
+      const float p = __expf(lg - mn);
+      float ps = p;
+#pragma unroll
+      for (int o2 = 16; o2; o2 >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o2);
+      l = l * sc + ps;
+#pragma unroll
+      for (int u = 0; u < DL; ++u) o[u] *= sc;
+      mx = mn;
+      for (int jj = 0; jj < nb; ++jj) {
+        const float pj = __shfl_sync(0xffffffffu, p, jj);
+        const long long vr = xb[jj];
+#pragma unroll
+        for (int u = 0; u < DL; ++u) o[u] = fmaf(pj, ld<T>(V + vr * D + lane + 32 * u), o[u]);
+      }
+      __syncwarp();
+      nb = 0;
+    };
+    for (int r = 0; r < k1; ++r) {
+      const int j = s1[r];
+      if (j < 0) break;
+      const int* kb = c.kboff + ((size_t)kpid * Ck + j) * (NB + 1);
+      for (int r2 = 0; r2 < k2; ++r2) {
+        const int bb = s2[r * k2 + r2];
+        if (bb < 0) break;
+        const int m0 = kb[bb], cnt = kb[bb + 1] - m0;
+        for (int x0 = 0; x0 < cnt;) {
+          const int take = imin(32 - nb, cnt - x0);
+          if (lane < take) xb[nb + lane] = pk.row0 + kperm[koff[j] + m0 + x0 + lane];
+          __syncwarp();
+          nb += take;
+          x0 += take;
+          if (nb == 32) flush();
+        }
+      }
+    }
+    if (nb > 0) flush();
+    float* pp = a.part + (size_t)qrow * (D + 1);
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int u = 0; u < DL; ++u) pp[lane + 32 * u] = o[u] * inv;
+    if (lane == 0) {
+      pp[D] = mx + logf(l);
+      if (a.n_exact != nullptr) a.n_exact[qrow] = nretr[cc];
+    }
+    __syncwarp();
+  }
+}
+
 template <typename T, int D>
 void launch_accum(const AttnArgs& a, const AccArgs& c, cudaStream_t st) {
   const int nk = a.ks.nprob, nq = a.qs.nprob;
@@ -698,10 +978,19 @@ void launch_accum(const AttnArgs& a, const AccArgs& c, cudaStream_t st) {
   }
   {
     ProfScope ps(st, "accum_stage2");
-    const size_t sm = stage2_smem<D>(a.Ck, a.topk);
-    auto kern = dip ? acc_stage2_kernel<T, D, true> : acc_stage2_kernel<T, D, false>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    kern<<<dim3(nq, c.NB, cdiv(a.Cq, kCI)), kST, sm, st>>>(a, c);
+    if (!dip) {
+      // query clusters per CTA: the remainder rows of all of them must fit
+      const int nci = a.topk > 0 ? imin(kCM, kRM / a.topk) : kCM;
+      const size_t sm = stage2_mono_smem<D>(a.Ck) + (size_t)nci * a.Ck;
+      cudaFuncSetAttribute(acc_stage2_mono_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sm);
+      acc_stage2_mono_kernel<T, D><<<dim3(nq, c.NB, cdiv(a.Cq, nci)), kST, sm, st>>>(a, c, nci);
+    } else {
+      const size_t sm = stage2_smem<D>(a.Ck, a.topk);
+      cudaFuncSetAttribute(acc_stage2_kernel<T, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sm);
+      acc_stage2_kernel<T, D, true><<<dim3(nq, c.NB, cdiv(a.Cq, kCI)), kST, sm, st>>>(a, c);
+    }
   }
 }
 
@@ -712,6 +1001,8 @@ bool accum_supported(int D, int Cq, int Ck, int NB, int k1, int k2, int mode) {
   if (D != 64 && D != 128) return false;
   if (Cq > 256 || Ck > 256 || Ck * D > 16384 || k1 > 32) return false;
   if ((D == 64 ? stage2_smem<64>(Ck, k1) : stage2_smem<128>(Ck, k1)) > 227 * 1024) return false;
+  if ((D == 64 ? stage2_mono_smem<64>(Ck) : stage2_mono_smem<128>(Ck)) + (size_t)kCM * Ck > 227 * 1024)
+    return false;
   if (mode == 1 && Cq * D > kAT * 32) return false;  // acc_block_a: 32 outputs per thread
   if (NB < 1 || NB > 1024 || k2 < 0 || k2 > NB) return false;
   return true;
