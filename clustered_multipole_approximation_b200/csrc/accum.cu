@@ -112,9 +112,10 @@ __global__ void acc_prefix_kernel(AttnArgs a, AccArgs c) {
     c.pk[o * D + d] = pk;
     c.ps[o * D + d] = ps;
     // centroids of the prefix and of the block, for the selection scores
-    const size_t ot = (((size_t)pid * NB + b) * D + d) * Ck + j;  // dimension-major
-    c.pmu[ot] = pn > 0 ? __ddiv_rn(pk, (double)pn) : 0.0;
-    c.bmu[ot] = bn > 0 ? __ddiv_rn(bk, (double)bn) : 0.0;
+    // prefix centroids [set][b][d][j] (a warp reads consecutive j), block
+    // centroids [set][j][d][b] (a warp reads consecutive b)
+    c.pmu[(((size_t)pid * NB + b) * D + d) * Ck + j] = pn > 0 ? __ddiv_rn(pk, (double)pn) : 0.0;
+    c.bmu[(((size_t)pid * Ck + j) * D + d) * NB + b] = bn > 0 ? __ddiv_rn(bk, (double)bn) : 0.0;
     if (d == 0) c.pn[o] = pn;
     pk += bk;
     ps += c.bs[o * D + d];
@@ -290,8 +291,8 @@ __global__ void __launch_bounds__(kAT) acc_select_kernel(AttnArgs a, AccArgs c) 
       for (int bb = lane; bb < b; bb += 32) {
         const size_t o = ((size_t)kpid * NB + bb) * Ck + j;
         const int n = c.bn[o];
-        const double* mu = c.bmu + ((size_t)kpid * NB + bb) * D * Ck + j;
-        sc[bb] = n > 0 ? __dadd_rn(__dmul_rn(s, dot_ordered(nu, mu, Ck, D)), log((double)n))
+        const double* mu = c.bmu + ((size_t)kpid * Ck + j) * D * NB + bb;  // lanes: consecutive bb
+        sc[bb] = n > 0 ? __dadd_rn(__dmul_rn(s, dot_ordered(nu, mu, NB, D)), log((double)n))
                        : -INFINITY;
       }
       __syncwarp();

@@ -168,7 +168,7 @@ struct AccArgs {
   int* pn;         // [key sets][NB][Ck] exclusive prefix over blocks
   double* bk;      // [key sets][NB][Ck][D] key sums (token order)
   double* pk;      // prefix of bk (block order)
-  double* bmu;     // [key sets][NB][D][Ck] bk / bn (fp64 division), dimension-major
+  double* bmu;     // [key sets][Ck][D][NB] bk / bn (fp64 division), block index fastest
   double* pmu;     // [key sets][NB][D][Ck] pk / pn, dimension-major
   float* bs;       // [key sets][NB][Ck][D] value sums
   float* ps;       // prefix of bs
