@@ -23,7 +23,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "muse_oracle.c")
 _SO = os.path.join(_HERE, "libmuse_oracle.so")
 
-MODES = {"monopole": 0, "dipole": 1, "tilted": 2, "dipole_q": 3}
+MODES = {"monopole": 0, "dipole": 1, "tilted": 2, "dipole_q": 3, "tilted_dipole": 4}
 
 
 def build(force: bool = False) -> str:

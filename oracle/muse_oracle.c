@@ -47,6 +47,7 @@
 #define ORC_DIPOLE 1
 #define ORC_TILTED 2
 #define ORC_DIPOLE_Q 3
+#define ORC_TILTED_DIPOLE 4
 
 /* ------------------------------------------------------------------------ */
 /* splitmix64 (Vigna): state advances by the golden-ratio increment, output  */
@@ -354,7 +355,7 @@ static void stage2(const query_block *qb, const key_block *kb, double scale,
       if (kb->count[j] == 0 || inR[j]) continue;
       size_t ij = (size_t)i * Ck + j;
       double lam;
-      if (mode == ORC_TILTED) {
+      if (mode == ORC_TILTED || mode == ORC_TILTED_DIPOLE) {
         const double *kh = Khat + ij * D, *mu = kb->mu + (size_t)j * D;
         double g = 0.0;
         for (int d = 0; d < D; ++d) g += (x[d] - nu[d]) * kh[d];
@@ -368,6 +369,28 @@ static void stage2(const query_block *qb, const key_block *kb, double scale,
          * u_qj = S_j / n_j + (s / n_j) M_j q */
         for (int e = 0; e < D; ++e)
           uq[e] = val[e] + scale * dot(kb->M + ((size_t)j * D + e) * D, x, D) / (double)kb->count[j];
+        val = uq;
+      }
+      if (mode == ORC_TILTED_DIPOLE) {
+        /* the tilted per-pair dipole: the tilt exp(s nu_i . k_t) is kept
+         * exactly and exp(s (q - nu_i) . k_t) is expanded to first order
+         * about the tilted centroid k^_ij, so the value gains
+         * s M^_ij (q - nu_i), M^_ij = sum_t w^_t v_t (k_t - k^_ij)^T with the
+         * tilted weights w^_t = exp(s nu_i . (k_t - mu_j) - log W_ij);
+         * summed here token by token */
+        const double *kh = Khat + ij * D, *mu = kb->mu + (size_t)j * D;
+        for (int e = 0; e < D; ++e) uq[e] = val[e];
+        for (int t = 0; t < kb->n; ++t) {
+          if (kb->assign[t] != j) continue;
+          const double *k = kb->K + (size_t)t * D;
+          double a = 0.0, g = 0.0;
+          for (int d = 0; d < D; ++d) {
+            a += nu[d] * (k[d] - mu[d]);
+            g += (x[d] - nu[d]) * (k[d] - kh[d]);
+          }
+          const double w = exp(scale * a - logW[ij]);
+          for (int e = 0; e < D; ++e) uq[e] += scale * w * g * kb->V[(size_t)t * D + e];
+        }
         val = uq;
       }
       acc_add(&m[q], &l[q], aq, D, lam, val);

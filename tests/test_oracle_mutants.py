@@ -48,6 +48,10 @@ MUTANTS = {
         "scale * dot(kb->M + ((size_t)j * D + e) * D, nu, D) / (double)kb->count[j];"),
     "fine-query-dipole-sign": (
         "uq[e] = val[e] + scale * dot(", "uq[e] = val[e] - scale * dot("),
+    "tilted-dipole-about-centroid": ("g += (x[d] - nu[d]) * (k[d] - kh[d]);",
+                                     "g += (x[d] - nu[d]) * (k[d] - mu[d]);"),
+    "tilted-dipole-uses-q": ("g += (x[d] - nu[d]) * (k[d] - kh[d]);", "g += x[d] * (k[d] - kh[d]);"),
+    "tilted-dipole-sign": ("uq[e] += scale * w * g * kb->V", "uq[e] -= scale * w * g * kb->V"),
 }
 
 

@@ -166,10 +166,13 @@ def test_exact_attention_matches_torch(orc, causal):
     np.testing.assert_allclose(E, ref, rtol=1e-12, atol=1e-12)
 
 
+ALL_MODES = ["monopole", "dipole", "tilted", "dipole_q", "tilted_dipole"]
+
+
 # --------------------------------------------------------------------------
 # closed forms the approximation reduces to
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_singleton_key_clusters_are_exact(orc, mode):
     Q, K, V = small_qkv(B=1, Hq=2, Hkv=1, N=64, D=8, seed=4)
     E = orc.exact_attention(Q, K, V)
@@ -178,7 +181,7 @@ def test_singleton_key_clusters_are_exact(orc, mode):
         np.testing.assert_allclose(r["O"], E, rtol=1e-11, atol=1e-12)
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_retrieving_every_cluster_is_exact(orc, mode):
     Q, K, V = small_qkv(N=128, D=8, seed=6)
     E = orc.exact_attention(Q, K, V)
@@ -241,6 +244,32 @@ def test_fine_query_dipole_equals_dipole_with_singleton_query_clusters(orc):
     np.testing.assert_allclose(b, a, rtol=1e-11, atol=1e-12)
 
 
+def test_tilted_dipole_equals_tilted_with_singleton_query_clusters(orc):
+    """Each query its own cluster (q = nu_i): the tilted per-pair dipole's
+    first-order term in q - nu_i vanishes."""
+    Q, K, V = small_qkv(N=64, D=8, seed=32)
+    a = orc.muse_acausal(Q, K, V, 64, 6, 3, 5, 1, scale=0.9, mode="tilted")["O"]
+    b = orc.muse_acausal(Q, K, V, 64, 6, 3, 5, 1, scale=0.9, mode="tilted_dipole")["O"]
+    np.testing.assert_allclose(b, a, rtol=1e-11, atol=1e-12)
+
+
+def test_tilted_dipole_single_clusters_is_tilted_cross_covariance_correction(orc):
+    """One query cluster and one key cluster: every query's output is the
+    tilted mean value plus s C^_vk (q - nu) with C^_vk the covariance of v and
+    k under the weights softmax(s k . nu)."""
+    Q, K, V = small_qkv(N=160, D=6, seed=33)
+    s = 0.8
+    r = orc.muse_acausal(Q, K, V, 1, 1, 2, 0, 0, scale=s, mode="tilted_dipole")
+    q, k, v = Q[0, 0], K[0, 0], V[0, 0]
+    nu = q.mean(0)
+    w = np.exp(s * k @ nu - (s * k @ nu).max())
+    w /= w.sum()
+    vbar, kbar = w @ v, w @ k
+    cvk = (w[:, None] * (v - vbar)).T @ (k - kbar)
+    ref = vbar[None, :] + s * (q - nu) @ cvk.T
+    np.testing.assert_allclose(r["O"][0, 0], ref, rtol=1e-10, atol=1e-12)
+
+
 def test_modes_agree_when_cluster_keys_coincide(orc):
     rng = np.random.default_rng(2)
     N, D, Ck = 120, 8, 6
@@ -251,10 +280,9 @@ def test_modes_agree_when_cluster_keys_coincide(orc):
     Q = (base[rng.integers(0, Ck, N)] + 0.2 * rng.standard_normal((N, D)))[None, None]
     V = rng.standard_normal((1, 1, N, D))
     outs = [orc.muse_acausal(Q, K, V, 4, Ck, 3, 1, 1, mode=m, k_assign_in=z[None, None])["O"]
-            for m in ("monopole", "dipole", "tilted", "dipole_q")]
-    np.testing.assert_allclose(outs[1], outs[0], rtol=1e-11, atol=1e-12)
-    np.testing.assert_allclose(outs[2], outs[0], rtol=1e-11, atol=1e-12)
-    np.testing.assert_allclose(outs[3], outs[0], rtol=1e-11, atol=1e-12)
+            for m in ALL_MODES]
+    for o in outs[1:]:
+        np.testing.assert_allclose(o, outs[0], rtol=1e-11, atol=1e-12)
 
 
 def test_selection_ties_go_to_lowest_index(orc):
@@ -279,7 +307,7 @@ def test_selection_ties_go_to_lowest_index(orc):
 # --------------------------------------------------------------------------
 # invariants
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_weights_sum_to_one_and_monopole_tilted_nonnegative(orc, mode):
     # with V = identity each output row is the vector of per-token weights
     Q, K, _ = small_qkv(N=64, D=64, centres=6, seed=15)
@@ -295,7 +323,7 @@ def test_weights_sum_to_one_and_monopole_tilted_nonnegative(orc, mode):
     np.testing.assert_allclose(r["O"][0, 0], Vc[0, 0], rtol=1e-12, atol=1e-10)
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_key_translation_invariance(orc, mode):
     Q, K, V = small_qkv(N=256, D=8, centres=6, noise=0.2, seed=16)
     shift = np.linspace(-0.5, 0.75, 8)
@@ -307,7 +335,7 @@ def test_key_translation_invariance(orc, mode):
     np.testing.assert_allclose(b["k_cent"], a["k_cent"] + shift, rtol=1e-12, atol=1e-12)
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_causal_never_reads_the_future(orc, mode):
     Q, K, V = small_qkv(B=1, Hq=2, Hkv=1, N=128, D=8, seed=17)
     base = orc.muse_causal(Q, K, V, 16, 4, 3, 5, 1, mode=mode)["O"]
@@ -319,7 +347,7 @@ def test_causal_never_reads_the_future(orc, mode):
         assert (o[:, :, : t0 + 1] == base[:, :, : t0 + 1]).all()
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_causal_with_singleton_clusters_is_exact_causal(orc, mode):
     # C >= block size at every level makes every summary exact, so the
     # decomposition must cover each earlier key exactly once.
@@ -357,7 +385,7 @@ def brute_block(Qb, Kb, Vb, qa, ka, Cq, Ck, k1, s, mode):
             if not cnt[j]:
                 continue
             kj = Kb[ka == j]
-            if mode == "tilted":
+            if mode in ("tilted", "tilted_dipole"):
                 e = np.exp(s * kj @ nu[i])
                 scores[j] = math.log(e.sum())
                 khat[j] = (e[:, None] * kj).sum(0) / e.sum()
@@ -376,12 +404,15 @@ def brute_block(Qb, Kb, Vb, qa, ka, Cq, Ck, k1, s, mode):
                     W[q, t] = math.exp(s * x @ mu[j]) * (1 + s * nu[i] @ (Kb[t] - mu[j]))
                 elif mode == "dipole_q":
                     W[q, t] = math.exp(s * x @ mu[j]) * (1 + s * x @ (Kb[t] - mu[j]))
-                else:
+                elif mode == "tilted":
                     W[q, t] = math.exp(s * (nu[i] @ Kb[t] + (x - nu[i]) @ khat[j]))
+                else:  # tilted per-pair dipole: first order in q - nu about k^
+                    W[q, t] = (math.exp(s * (nu[i] @ Kb[t] + (x - nu[i]) @ khat[j]))
+                               * (1 + s * (x - nu[i]) @ (Kb[t] - khat[j])))
     return W
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_acausal_matches_per_token_bruteforce(orc, mode):
     Q, K, V = small_qkv(N=64, D=8, centres=5, seed=19)
     s, Cq, Ck, k1 = 1.1, 5, 9, 2
@@ -392,7 +423,7 @@ def test_acausal_matches_per_token_bruteforce(orc, mode):
     np.testing.assert_allclose(r["O"][0, 0], ref, rtol=1e-10, atol=1e-12)
 
 
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "dipole_q"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_causal_matches_per_token_bruteforce(orc, mode):
     Q, K, V = small_qkv(B=1, Hq=2, Hkv=1, N=64, D=8, centres=4, seed=20)
     N, L, C, k1, s = 64, 8, 3, 1, 0.8
