@@ -52,7 +52,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="muse", choices=["muse", "reference"])
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
-    p.add_argument("--mode", default=None, choices=[None, "dipole", "monopole", "tilted", "dipole_q"])
+    p.add_argument("--mode", default=None, choices=[None, "dipole", "monopole", "tilted", "dipole_q",
+                                                       "tilted_dipole"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--accum", action="store_true",
                    help="time only the block-accumulation causal form of a causal workload")
@@ -140,7 +141,7 @@ NCU_TRAFFIC: dict = {
 }
 
 # The library's per-kernel profiling names -> what they compute.
-TENSOR_KERNELS = ("kmeans", "stage1_summaries", "stage2_attn", "stage2_dense",
+TENSOR_KERNELS = ("kmeans", "stage1_summaries", "stage2_attn", "stage2_dense", "stage2_tdip",
                   "causal_local_merge")
 # Launches that together do one algorithmic step: the persistent k-means runs
 # the problems whose centroid sums are certified exact with every token tile
@@ -216,7 +217,8 @@ def algorithmic_work(w, mode, dbg):
       k-means       T * 2 * tokens * C_eff * D per role (every level);
       stage 1       min(2 C_eff^2 D^2 + 2 s D^2, 4 s C_eff D) per query problem
                     (the dipole contraction; 0 for MONOPOLE and DIPOLE_Q);
-      stage 2       4 D per far row and per exact retrieved key; DIPOLE_Q
+      stage 2       4 D per far row and per exact retrieved key; DIPOLE_Q and
+                    TILTED_DIPOLE
                     (per key token: q.k_t, the factor's q.(k_t - mu) and
                     the weighted v_t) 4 D per (query, key) pair of the block
                     plus 2 D per (query, key cluster) for q.mu_j;
@@ -233,6 +235,8 @@ def algorithmic_work(w, mode, dbg):
                                                               4.0 * s * ce * D)
         if mode == "dipole_q":
             work["stage2_dense"] += B * Hq * toks * (4.0 * D * s + 2.0 * D * ce)
+        elif mode == "tilted_dipole":  # per key token: q.k_t, nu.k_t, the weighted v_t
+            work["stage2_tdip"] += B * Hq * toks * (4.0 * D * s + 2.0 * D * ce)
         else:
             work["stage2_dense" if dense else "stage2_attn"] += 4.0 * D * (far[lv] + exact[lv])
     if w.causal:

@@ -23,7 +23,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmuse.so")
 
-MODES = {"monopole": 0, "dipole": 1, "tilted": 2, "dipole_q": 3}
+MODES = {"monopole": 0, "dipole": 1, "tilted": 2, "dipole_q": 3, "tilted_dipole": 4}
 STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED",
           3: "MUSE_ERR_WORKSPACE", 4: "MUSE_ERR_CUDA", 5: "MUSE_ERR_DEVICE_CHECK"}
 

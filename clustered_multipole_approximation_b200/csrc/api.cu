@@ -166,7 +166,7 @@ muse_status validate(const muse_shape* sh, const muse_params* pr, bool causal) {
     return fail(MUSE_ERR_INVALID_ARG, "dtype must be MUSE_BF16 or MUSE_F32");
   if (sh->out_f32 != 0 && sh->out_f32 != 1) return fail(MUSE_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
   if (pr->iters < 1) return fail(MUSE_ERR_INVALID_ARG, "iters must be >= 1");
-  if (pr->mode < MUSE_MONOPOLE || pr->mode > MUSE_DIPOLE_Q)
+  if (pr->mode < MUSE_MONOPOLE || pr->mode > MUSE_TILTED_DIPOLE)
     return fail(MUSE_ERR_INVALID_ARG, "unknown mode");
   if (pr->Cq < 1 || pr->Ck < 1) return fail(MUSE_ERR_INVALID_ARG, "Cq and Ck must be >= 1");
   if (pr->Cq > kMaxC || pr->Ck > kMaxC)
@@ -207,14 +207,15 @@ AttnLayout layout(const muse_shape* sh, const muse_params* pr, bool causal, cons
   L.ks.err = L.qs.err = L.err;
   L.nq = L.qs.nprob;
   const size_t cc = (size_t)pr->Cq * pr->Ck;
-  const size_t per = cc * 4 * 2 + cc * sh->D * 4 * (pr->mode == MUSE_TILTED ? 2 : 1);  // upper bound
+  const bool tilt = pr->mode == MUSE_TILTED || pr->mode == MUSE_TILTED_DIPOLE;
+  const size_t per = cc * 4 * 2 + cc * sh->D * 4 * (tilt ? 2 : 1);  // upper bound
   size_t wave = L.nq;
   if (causal && per * wave > kStage1Budget) wave = kStage1Budget / per;
   if (wave < 1) wave = 1;
   L.wave = (int)wave;
   L.s1.logW = cv.take<float>(wave * cc * 4);
   L.s1.fbias = cv.take<float>(wave * cc * 4);
-  const bool tilted = pr->mode == MUSE_TILTED;
+  const bool tilted = tilt;  // the tilted centroids are carved for both tilted modes
   if (dt == 0) {
     L.s1.Uh = cv.take<__half>(wave * cc * sh->D * 2);
     L.s1.Ul = cv.take<__half>(wave * cc * sh->D * 2);
@@ -274,6 +275,10 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
   a.B = sh->B;
   a.G = sh->Hq / sh->Hkv;
   a.mode = (int)pr->mode;
+  if (pr->mode == MUSE_TILTED_DIPOLE) {  // stage 1 and selection are TILTED's
+    a.mode = MUSE_TILTED;
+    a.tdip = 1;
+  }
   a.topk = pr->topk;
   a.scale = pr->scale;
   a.Cq = pr->Cq;
@@ -291,7 +296,7 @@ muse_status attn(const void* Q, const void* K, const void* V, void* O, const mus
                      ? dense_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck)
                      : 0;
   }
-  a.tc_lv = (sh->dtype == MUSE_BF16 && L.V16 && L.kpad)
+  a.tc_lv = (sh->dtype == MUSE_BF16 && L.V16 && L.kpad && !a.tdip)
                 ? stage2_tc_levels(L.qg.lv, sh->D, pr->Cq, pr->Ck, pr->topk, a.dense_lv)
                 : 0;
   a.kpad = L.kpad;

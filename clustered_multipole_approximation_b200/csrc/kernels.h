@@ -50,6 +50,7 @@ struct AttnArgs {
   void* kpad;         // those levels' keys, cluster-sorted, group-padded, pre-swizzled (bf16)
   void* vpad;         // the same for V (fp16)
   int* gofs;          // [key problems][Ck + 1] first group of each cluster in kpad / vpad
+  int tdip;           // stage 2 of the tilted per-pair dipole (stage 1 and selection: TILTED)
   int accum;          // causal local merge: one partial per query of blocks >= 1 at row
                       // b H N + q (block-summary accumulation), else the level partials
 };
@@ -179,6 +180,9 @@ struct AccArgs {
 };
 bool accum_supported(int D, int Cq, int Ck, int NB, int k1, int k2, int mode);
 void run_accum(const AttnArgs& a, const AccArgs& c, cudaStream_t st);
+
+// Stage 2 of the tilted per-pair dipole (stage2_tdip.cu): per key token, SIMT.
+void run_stage2_tdip(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cudaStream_t st);
 
 // Causal: exact local block + merge of the level partials into O.
 void run_local_merge(const AttnArgs& a, int L, cudaStream_t st);

@@ -532,7 +532,9 @@ static void blocks_t(const AttnArgs& a, const Stage1& s1, int qp0, int nqp, cuda
     ProfScope ps(st, "stage1_select");
     run_select(a, s1, qp0, nqp, st);
   }
-  if (sizeof(T) == 2) {
+  if (a.tdip) {  // the tilted per-pair dipole: its own per-key-token stage 2
+    run_stage2_tdip(a, s1, qp0, nqp, st);
+  } else if (sizeof(T) == 2) {
     if (!fq) {
       ProfScope ps(st, "stage2_attn");
       run_stage2_tc(a, s1, qp0, nqp, st);

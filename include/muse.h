@@ -94,8 +94,23 @@ typedef enum { MUSE_BF16 = 0, MUSE_F32 = 1 } muse_dtype;
  *             accuracy reference rather than a fast path.  Supported for
  *             dtype MUSE_BF16 with Cq, Ck <= 256 and every block size (N for
  *             muse_attn_fwd, L 2^l for muse_causal_fwd) a multiple of 128;
- *             other shapes return MUSE_ERR_UNSUPPORTED. */
-typedef enum { MUSE_MONOPOLE = 0, MUSE_DIPOLE = 1, MUSE_TILTED = 2, MUSE_DIPOLE_Q = 3 } muse_mode;
+ *             other shapes return MUSE_ERR_UNSUPPORTED.
+ *   TILTED_DIPOLE  an accuracy variant of TILTED: the tilt exp(s nu_i . k_t)
+ *             is kept exactly and exp(s (q - nu_i) . k_t) is expanded to
+ *             first order about the tilted centroid k^_ij, so the value gains
+ *             s M^_ij (q - nu_i) (M^_ij: the tilted value-key moment about
+ *             k^_ij) and the weight is TILTED's.  Stage 1 and the selection
+ *             are TILTED's; the far field is evaluated per key token (fp32,
+ *             O(N^2 D) like exact attention), an accuracy reference.  Both
+ *             dtypes, acausal and causal.
+ */
+typedef enum {
+  MUSE_MONOPOLE = 0,
+  MUSE_DIPOLE = 1,
+  MUSE_TILTED = 2,
+  MUSE_DIPOLE_Q = 3,
+  MUSE_TILTED_DIPOLE = 4
+} muse_mode;
 
 typedef struct {
   int B, Hq, Hkv, N, D; /* D in {64, 128}; Hq % Hkv == 0 */

@@ -95,7 +95,7 @@ def test_workload_acausal_bf16_h8_n8k(mode):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "tilted_dipole"])
 def test_small_acausal_gqa_ragged(dtype, D, mode):
     Q, K, V = clustered_qkv(2, 4, 2, 1000, D, 12, 0.3, 0.0, dtype, 31 + D)
     check_acausal(Q, K, V, dtype, 13, 5, 77, 3, 1.0, mode, Cq=11)
@@ -378,7 +378,7 @@ def check_causal(Q, K, V, dtype, L, C, iters, seed, topk, scale=1.0, mode="dipol
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted"])
+@pytest.mark.parametrize("mode", ["monopole", "dipole", "tilted", "tilted_dipole"])
 def test_small_causal_gqa(dtype, mode):
     Q, K, V = clustered_qkv(1, 4, 2, 1024, 64, 8, 0.3, 0.0, dtype, 50)
     check_causal(Q, K, V, dtype, 64, 12, 4, 21, 2, 1.0, mode)
@@ -486,6 +486,28 @@ def test_workload_causal_b2h8_n16k_fine_query_dipole():
     Q, K, V = make_inputs(w)
     check_causal(Q, K, V, w.dtype, w.block, w.C, w.iters, w.cluster_seed, w.topk, w.scale,
                  "dipole_q", heads=[(1, 3)])
+
+
+def test_tilted_dipole_runs_per_key_token_and_beats_tilted():
+    """The tilted per-pair dipole takes its own stage 2 (no per-cluster-pair
+    stage-2 kernel runs) and lands nearer exact attention than TILTED."""
+    Q, K, V = clustered_qkv(1, 2, 2, 2048, 64, 8, 0.6, 0.0, "bf16", 95)
+    _, launched = _stages_launched(
+        lambda: gpu_acausal(Q, K, V, "bf16", 32, 6, 5, 2, 1.0, "tilted_dipole"))
+    assert "stage2_tdip" in launched and "stage2_attn" not in launched, launched
+    Ot, _ = gpu_acausal(Q, K, V, "bf16", 32, 6, 5, 2, 1.0, "tilted_dipole")
+    Oi, _ = gpu_acausal(Q, K, V, "bf16", 32, 6, 5, 2, 1.0, "tilted")
+    E = oracle.exact_attention(Q, K, V)
+    assert rse(Ot, E) < 0.5 * rse(Oi, E), (rse(Ot, E), rse(Oi, E))
+
+
+def test_workload_acausal_bf16_h8_n8k_tilted_dipole():
+    """The 8-head 8k layer in the tilted per-pair dipole mode, head 4 against
+    the oracle."""
+    w = WORKLOADS["acausal-bf16-h8-n8k"]
+    Q, K, V = make_inputs(w)
+    check_acausal(Q, K, V, w.dtype, w.C, w.iters, w.cluster_seed, w.topk, w.scale,
+                  "tilted_dipole", heads=[(0, 4)])
 
 
 @pytest.mark.parametrize("case", ["f32", "n_not_128", "block_not_128", "clusters_above_256"])
