@@ -1,4 +1,4 @@
-// Gradients of the acausal operator with respect to Q, K and V.
+// Gradients of the operator with respect to Q, K and V, acausal and causal.
 //
 // The pages train models with MuSe as the attention layer (gist.science page
 // "Multipole Semantic Attention: A Fast Approximation of Softmax Attention
@@ -41,6 +41,12 @@
 //   bwd_cluster     one CTA per (key set, cluster): dS_j, dM_j, dnu, and the
 //                   chain to the members' dk and dv;
 //   bwd_query_nu    dq += dnu_i / m_i.
+// Causal (the hierarchical levels and the local blocks of L keys, one softmax
+// per query): bwd_query first writes each level problem's (max, sum, sum of
+// p g) per query and bwd_local the local block's, bwd_combine merges them
+// into every query's log-sum-exp and D_q, then bwd_query and bwd_local take
+// the gradients of every term with those; a query's and a key's gradients
+// are summed over its levels by fp32 atomics.
 #include "common.cuh"
 #include "kernels.h"
 
