@@ -672,20 +672,24 @@ __global__ void __launch_bounds__(kST) acc_stage2_kernel(AttnArgs a, AccArgs c) 
 }
 
 // ---------------------------------------------------------------------------
-// MONOPOLE: the same terms with every query of the CTA's clusters in flight at
-// once (the values of the unselected clusters are shared by all clusters, so
-// only the selected clusters' remainders are per cluster; kCM * k1 rows).
+// The same terms with every query of the CTA's clusters in flight at once.
+// The unselected clusters' centroids and log-counts are shared by all query
+// clusters; so are their MONOPOLE values S / n.  A DIPOLE value adds
+// s (A_ij / n_j - (S_j / n_j)(mu_j . nu_i)), formed per query from the prefix
+// table A and the per-cluster dots mu_j . nu_i.  Only the selected clusters'
+// remainders are per query cluster (kCM * k1 rows).
 // ---------------------------------------------------------------------------
 constexpr int kCM = 16;    // query clusters per CTA
 constexpr int kRM = 64;    // remainder rows per CTA: kCM clusters x k1, or fewer clusters for k1 > 4
 
 template <int D>
-size_t stage2_mono_smem(int Ck) {
+size_t stage2_mono_smem(int Ck, bool dip) {
   return ((size_t)Ck * (D + 1) + (size_t)Ck * D + Ck + (size_t)kRM * (D + 1) + (size_t)kRM * D + kRM +
-          (size_t)kSW * D) * 4 + (size_t)kCM * Ck + (size_t)kSW * 32 * 4 + (size_t)kSW * 32 * 8 * 2 + 64;
+          (size_t)kSW * D) * 4 + (size_t)2 * kCM * Ck + (size_t)kSW * 32 * 4 + (size_t)kSW * 32 * 8 * 3 +
+         64 + (dip ? ((size_t)kCM * Ck + Ck + (size_t)kSW * 32 * 2 + (size_t)kCM * D) * 4 : 0);
 }
 
-template <typename T, int D>
+template <typename T, int D, bool DIP>
 __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArgs c, int nci) {
   extern __shared__ __align__(16) float sm_raw[];
   const int Cq = a.Cq, Ck = a.Ck, NB = c.NB, k1 = a.topk, k2 = c.k2;
@@ -700,7 +704,16 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
   const float** uw_s = reinterpret_cast<const float**>(  // [kSW][32]
       (reinterpret_cast<uintptr_t>(pw_s + kSW * 32) + 7) & ~(uintptr_t)7);
   long long* xb_s = reinterpret_cast<long long*>(uw_s + kSW * 32);   // [kSW][32] retrieved rows
-  signed char* rsel = reinterpret_cast<signed char*>(xb_s + kSW * 32);  // [nci][Ck]
+  const float** aw_s = reinterpret_cast<const float**>(xb_s + kSW * 32);  // [kSW][32] DIPOLE A rows
+  // DIPOLE only (the MONOPOLE allocation ends before them): mu_j . nu_i per
+  // (query cluster, key cluster), 1 / n_j, each warp's copies of both, nu_i
+  float* dip0 = reinterpret_cast<float*>(aw_s + kSW * 32);
+  float* mn_s = dip0;                                                  // [kCM][Ck]
+  float* inv_s = mn_s + (size_t)kCM * Ck;                              // [Ck]
+  float* cw_s = inv_s + Ck;                                            // [kSW][32]
+  float* iw_s = cw_s + kSW * 32;                                       // [kSW][32]
+  float* nu_s = iw_s + kSW * 32;                                       // [kCM][D]
+  signed char* rsel = reinterpret_cast<signed char*>(DIP ? nu_s + (size_t)kCM * D : dip0);  // [nci][Ck]
   __shared__ int qcum[kCM + 1];
   __shared__ int nretr[kCM];
   const int qpid = blockIdx.x, b = blockIdx.y, i0 = blockIdx.z * nci;
@@ -716,7 +729,10 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
   for (int j = warp; j < Ck; j += kSW) {
     const size_t o = ((size_t)kpid * NB + b) * Ck + j;
     const int n = c.pn[o];
-    if (lane == 0) ln_s[j] = n > 0 ? logf((float)n) : -INFINITY;
+    if (lane == 0) {
+      ln_s[j] = n > 0 ? logf((float)n) : -INFINITY;
+      if (DIP) inv_s[j] = n > 0 ? 1.f / (float)n : 0.f;
+    }
 #pragma unroll
     for (int u = 0; u < DL; ++u) {
       const int d = lane + 32 * u;
@@ -724,6 +740,11 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
       u_s[j * D + d] = n > 0 ? c.ps[o * D + d] / (float)n : 0.f;
     }
   }
+  if (DIP)
+    for (int e = tid; e < ncl * D; e += kST) {
+      const int cc = e / D, d = e - cc * D;
+      nu_s[cc * D + d] = a.qs.cent32[((size_t)qpid * Cq + i0 + cc) * D + d];
+    }
   // ---- per cluster: its query range, its selected clusters, their remainders
   for (int e = tid; e < ncl * Ck; e += kST) rsel[e] = -1;
   if (tid == 0) {
@@ -756,6 +777,16 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
     }
     nretr[tid] = cnt;
   }
+  if (DIP)  // mu_j . nu_i of every (query cluster, key cluster) of the CTA
+    for (int e = warp; e < ncl * Ck; e += kSW) {
+      const int cc = e / Ck, j = e - cc * Ck;
+      float x = 0.f;
+#pragma unroll
+      for (int u = 0; u < DL; ++u) x = fmaf(mu_s[j * (D + 1) + lane + 32 * u], nu_s[cc * D + lane + 32 * u], x);
+#pragma unroll
+      for (int o2 = 16; o2; o2 >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o2);
+      if (lane == 0) mn_s[cc * Ck + j] = x;
+    }
   for (int e = warp; e < ncl * k1; e += kSW) {
     const int cc = e / k1, r = e - cc * k1, row = cc * k1 + r;
     const int* s1 = c.sel1 + (((size_t)qpid * NB + b) * Cq + i0 + cc) * k1;
@@ -766,13 +797,15 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
       continue;
     }
     const size_t o = ((size_t)kpid * NB + b) * Ck + j;
+    const size_t oa = (((size_t)qpid * NB + b) * Cq + i0 + cc) * Ck + j;  // the A table row
     int n = c.pn[o];
     double ksum[DL];
-    float ss[DL];
+    float ss[DL], aa[DL];
 #pragma unroll
     for (int u = 0; u < DL; ++u) {
       ksum[u] = c.pk[o * D + lane + 32 * u];
       ss[u] = c.ps[o * D + lane + 32 * u];
+      aa[u] = DIP ? c.pa[oa * D + lane + 32 * u] : 0.f;
     }
     for (int r2 = 0; r2 < k2; ++r2) {
       const int bb = s2[r * k2 + r2];
@@ -783,13 +816,29 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
       for (int u = 0; u < DL; ++u) {
         ksum[u] -= c.bk[ob * D + lane + 32 * u];
         ss[u] -= c.bs[ob * D + lane + 32 * u];
+        if (DIP)
+          aa[u] -= c.ba[((((size_t)qpid * NB + bb) * Cq + i0 + cc) * Ck + j) * D + lane + 32 * u];
       }
+    }
+    float mn = 0.f;
+#pragma unroll
+    for (int u = 0; u < DL; ++u) {
+      const int d = lane + 32 * u;
+      const float mu = n > 0 ? (float)(ksum[u] / (double)n) : 0.f;
+      rm_s[row * (D + 1) + d] = mu;
+      if (DIP) mn = fmaf(mu, a.qs.cent32[((size_t)qpid * Cq + i0 + cc) * D + d], mn);
+    }
+    if (DIP) {
+#pragma unroll
+      for (int o2 = 16; o2; o2 >>= 1) mn += __shfl_xor_sync(0xffffffffu, mn, o2);
     }
 #pragma unroll
     for (int u = 0; u < DL; ++u) {
       const int d = lane + 32 * u;
-      rm_s[row * (D + 1) + d] = n > 0 ? (float)(ksum[u] / (double)n) : 0.f;
-      ru_s[row * D + d] = n > 0 ? ss[u] / (float)n : 0.f;
+      // M nu = A - S (mu . nu) over the remainder
+      ru_s[row * D + d] = n <= 0 ? 0.f
+                          : DIP ? fmaf(a.scale, fmaf(-ss[u], mn, aa[u]), ss[u]) / (float)n
+                                : ss[u] / (float)n;
     }
     if (lane == 0) rl_s[row] = n > 0 ? logf((float)n) : -INFINITY;
   }
@@ -803,6 +852,9 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
   float* qw = q_s + warp * D;
   float* pw = pw_s + warp * 32;
   const float** uw = uw_s + warp * 32;
+  const float** aw = aw_s + warp * 32;
+  float* cw = cw_s + warp * 32;
+  float* iw = iw_s + warp * 32;
   for (int m = warp; m < qcum[ncl]; m += kSW) {
     int cc = 0;
     while (qcum[cc + 1] <= m) ++cc;
@@ -821,10 +873,12 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
     }
     __syncwarp();
     float mx = -INFINITY, l = 0.f;
+    const float* arow0 = DIP ? c.pa + (((size_t)qpid * NB + b) * Cq + i) * Ck * D : nullptr;
     for (int j0 = 0; j0 < Ck; j0 += 32) {
       const int j = j0 + lane;
       float lg = -INFINITY;
       const float* urow = u_s;
+      const float* arow = nullptr;  // DIPOLE: the unselected cluster's A row (the value's dipole part)
       if (j < Ck) {
         const int r = rs[j];
         const int row = cc * k1 + r;
@@ -841,7 +895,13 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
           }
           lg = fmaf(s, (x0 + x1) + (x2 + x3), lnj);
           urow = r >= 0 ? ru_s + row * D : u_s + j * D;
+          if (DIP && r < 0) arow = arow0 + (size_t)j * D;
         }
+      }
+      if (DIP) {
+        aw[lane] = arow;
+        cw[lane] = j < Ck ? mn_s[cc * Ck + j] : 0.f;
+        iw[lane] = j < Ck ? inv_s[j] : 0.f;
       }
       float bm = lg;
 #pragma unroll
@@ -865,8 +925,18 @@ __global__ void __launch_bounds__(kST) acc_stage2_mono_kernel(AttnArgs a, AccArg
         const float pj = pw[jj];
         if (pj == 0.f) continue;
         const float* ur = uw[jj];
+        const float* ar = DIP ? aw[jj] : nullptr;
+        if (DIP && ar != nullptr) {  // u = S/n + s (A/n - (S/n)(mu . nu))
+          const float cj = cw[jj], ij = iw[jj];
 #pragma unroll
-        for (int u = 0; u < DL; ++u) o[u] = fmaf(pj, ur[lane + 32 * u], o[u]);
+          for (int u = 0; u < DL; ++u) {
+            const float u0 = ur[lane + 32 * u];
+            o[u] = fmaf(pj, fmaf(s, fmaf(ar[lane + 32 * u], ij, -u0 * cj), u0), o[u]);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < DL; ++u) o[u] = fmaf(pj, ur[lane + 32 * u], o[u]);
+        }
       }
       __syncwarp();
     }
@@ -979,13 +1049,14 @@ void launch_accum(const AttnArgs& a, const AccArgs& c, cudaStream_t st) {
   }
   {
     ProfScope ps(st, "accum_stage2");
-    if (!dip) {
+    const size_t smf = stage2_mono_smem<D>(a.Ck, dip);
+    if (!dip || smf <= 227 * 1024) {  // DIPOLE: where its per-query tables fit, else per cluster
       // query clusters per CTA: the remainder rows of all of them must fit
       const int nci = a.topk > 0 ? imin(kCM, kRM / a.topk) : kCM;
-      const size_t sm = stage2_mono_smem<D>(a.Ck) + (size_t)nci * a.Ck;
-      cudaFuncSetAttribute(acc_stage2_mono_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)sm);
-      acc_stage2_mono_kernel<T, D><<<dim3(nq, c.NB, cdiv(a.Cq, nci)), kST, sm, st>>>(a, c, nci);
+      const size_t sm = smf;
+      auto kern = dip ? acc_stage2_mono_kernel<T, D, true> : acc_stage2_mono_kernel<T, D, false>;
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      kern<<<dim3(nq, c.NB, cdiv(a.Cq, nci)), kST, sm, st>>>(a, c, nci);
     } else {
       const size_t sm = stage2_smem<D>(a.Ck, a.topk);
       cudaFuncSetAttribute(acc_stage2_kernel<T, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1002,7 +1073,8 @@ bool accum_supported(int D, int Cq, int Ck, int NB, int k1, int k2, int mode) {
   if (D != 64 && D != 128) return false;
   if (Cq > 256 || Ck > 256 || Ck * D > 16384 || k1 > 32) return false;
   if ((D == 64 ? stage2_smem<64>(Ck, k1) : stage2_smem<128>(Ck, k1)) > 227 * 1024) return false;
-  if ((D == 64 ? stage2_mono_smem<64>(Ck) : stage2_mono_smem<128>(Ck)) + (size_t)kCM * Ck > 227 * 1024)
+  if (mode == 0 && (D == 64 ? stage2_mono_smem<64>(Ck, false) : stage2_mono_smem<128>(Ck, false)) >
+                       227 * 1024)
     return false;
   if (mode == 1 && Cq * D > kAT * 32) return false;  // acc_block_a: 32 outputs per thread
   if (NB < 1 || NB > 1024 || k2 < 0 || k2 > NB) return false;
