@@ -168,3 +168,34 @@ def test_accum_workspace_and_argument_checks(lib):
     st = lib.muse_attn_fwd_causal_accum(fake, fake, fake, fake, ctypes.byref(sh),
                                         ctypes.byref(params(block=128)), 2, None, fake, 16, None)
     assert st == 3
+
+
+def test_causal_backward_workspace_and_argument_checks(lib):
+    """The causal backward sizes its workspace past the causal forward's part,
+    and refuses blocks that are not multiples of 32 and unsupported modes
+    before launching anything."""
+    sh = shape(N=1024)
+    pr = params(block=128)
+    fwd = lib.muse_workspace_size(ctypes.byref(sh), ctypes.byref(pr), 1)
+    bwd = lib.muse_attn_bwd_causal_workspace_size(ctypes.byref(sh), ctypes.byref(pr))
+    assert bwd > fwd > 0
+    for bad in (params(block=16 * 3), params(block=128, mode=2), params(block=128, mode=4)):
+        assert lib.muse_attn_bwd_causal_workspace_size(ctypes.byref(sh), ctypes.byref(bad)) == 0
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+    st = lib.muse_attn_bwd_causal(*([fake] * 7), ctypes.byref(sh), ctypes.byref(pr), fake, fwd,
+                                  None)
+    assert st == 3
+    st = lib.muse_attn_bwd_causal(*([fake] * 7), ctypes.byref(sh),
+                                  ctypes.byref(params(block=96)), fake, 1 << 40, None)
+    assert st == 1  # 96 does not divide N = 1024
+
+
+def test_accuracy_variant_modes_are_accepted_for_sizing(lib):
+    """DIPOLE_Q and TILTED_DIPOLE are valid modes (sized like DIPOLE and
+    TILTED); mode 5 is not."""
+    sh = shape()
+    for m in (3, 4):
+        assert lib.muse_workspace_size(ctypes.byref(sh), ctypes.byref(params(mode=m)), 0) > 0
+    assert lib.muse_workspace_size(ctypes.byref(sh), ctypes.byref(params(mode=5)), 0) == 0
+    tilted = lib.muse_workspace_size(ctypes.byref(sh), ctypes.byref(params(mode=2)), 0)
+    assert lib.muse_workspace_size(ctypes.byref(sh), ctypes.byref(params(mode=4)), 0) == tilted

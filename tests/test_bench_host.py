@@ -56,3 +56,30 @@ def test_level_table_tiles_the_causal_decomposition():
     a = WORKLOADS["acausal-bf16-h8-n8k"]
     assert bench.level_table(a, "dipole") == [(8192, 1, 128, False)]
     assert bench.level_table(a, "dipole_q") == [(8192, 1, 128, True)]
+
+
+def test_backward_and_variant_work_accounting():
+    """The backward's counted work has every kernel's share where it runs
+    (the causal form adds the local blocks), and the per-key-token variants
+    count their stage 2 against the kernel that runs it."""
+    a = WORKLOADS["acausal-bf16-h8-n8k"]
+    c = WORKLOADS["causal-bf16-b2h8-n16k"]
+
+    def fake_dbg(w):
+        rng = np.random.default_rng(0)
+        lv = len(bench.level_table(w, "dipole"))
+        if w.causal:
+            return {"q_assign": rng.integers(0, min(w.C, w.block), (w.B, w.Hq, lv, w.N // 2)),
+                    "k_assign": rng.integers(0, min(w.C, w.block), (w.B, w.Hkv, lv, w.N // 2))}
+        return {"q_assign": rng.integers(0, w.C, (w.B, w.Hq, w.N)),
+                "k_assign": rng.integers(0, w.C, (w.B, w.Hkv, w.N))}
+
+    wa = bench.backward_work(a, "dipole", fake_dbg(a))
+    assert wa["bwd_query"] > 0 and wa["bwd_u_table"] > 0 and wa["bwd_local"] == 0
+    wc = bench.backward_work(c, "dipole", fake_dbg(c))
+    assert wc["bwd_local"] > 0 and wc["bwd_query"] > 0
+    assert bench.backward_work(a, "monopole", fake_dbg(a))["bwd_u_table"] == 0
+    work, *_ = bench.algorithmic_work(a, "tilted_dipole", fake_dbg(a))
+    assert work["stage2_tdip"] > 0 and work["stage2_attn"] == 0
+    work, *_ = bench.algorithmic_work(a, "dipole_q", fake_dbg(a))
+    assert work["stage2_dense"] > 0 and work["stage2_attn"] == 0
